@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Benchmark of the TTT-layer forward pass on B200 (libttt.so through its C ABI).
+
+Default workload: TTT-Linear with f(k) = k + LN(k W), d = 64, mini-batch 16,
+B = 8, H = 12, T = 2048, bf16 Q/K/V, per-token eta (196,608 tokens per step).
+A step is one library call over one batch of seeded synthetic inputs that
+are already resident in HBM; between timed steps a 256 MiB buffer is written
+to flush the 126 MB L2. Steps are timed with CUDA events on the launching
+stream; with several GPUs (one process each, torchrun) every rank runs its
+own batch (different seed; weak scaling, no collective on the data path) and
+the slowest rank's time is reported.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from test_sequence_layers_layer_b200 import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "linear_ln_d64_b8h12_t2048"
+METRIC = "TTT-layer fwd tokens/sec at 1 B200; % of dense bf16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------- workload math
+
+def weight_bytes(wl) -> int:
+    return 4 * (2 * wl.d * wl.dh if wl.kind == "mlp" else wl.d * wl.d)
+
+
+def algo_bytes_per_token(wl) -> float:
+    """Interface bytes a token must move: Q, K, V in, eta in, Z (fp32) out, plus
+    the fast weight read once and written once per sequence, spread over T."""
+    e = 2 if wl.dtype == "bf16" else 4
+    return 3 * wl.d * e + 4 + 4 * wl.d + 2 * weight_bytes(wl) / wl.T
+
+
+def algo_flops_per_token(wl) -> float:
+    """Dense-contraction FLOPs per token of the method (dual form): for the
+    linear weight, K W, Q W and K^T G (2 d^2 each) plus the causal b x b terms;
+    for the MLP, seven 2 d dh products plus the causal terms; for large
+    chunks, Q W, K W and K^T G."""
+    d, b = wl.d, wl.b
+    if wl.kind == "linear":
+        return 6 * d * d + 2 * (b + 1) * d
+    if wl.kind == "mlp":
+        return 14 * d * wl.dh + 10 * (b + 1) * d
+    return 6 * d * d
+
+
+def bound_of(wl, peaks) -> str:
+    ai = algo_flops_per_token(wl) / algo_bytes_per_token(wl)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    return "tensor" if ai > ridge else "hbm"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# Kernel that dominates each workload's step, the source file it is built from,
+# and the arithmetic type it computes in.
+KERNELS = {
+    "linear": ("linear_simt_kernel", "ttt_simt.cu", "f32"),
+    "mlp": ("mlp_simt_kernel", "ttt_simt.cu", "f32"),
+    "chunk": ("chunk_simt_kernel", "ttt_simt.cu", "f32"),
+}
+
+
+def kernel_of(wl):
+    return KERNELS[wl.kind]
+
+
+def source_sha(fname: str) -> str:
+    path = os.path.join(ROOT, "test_sequence_layers_layer_b200", "csrc", fname)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str, sha: str):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/, valid
+    only while the kernel's source is unchanged (same sha)."""
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    pat = re.compile(r"traffic: kernel=(\S+) workload=(\S+) bytes_per_launch=([0-9.e+]+) "
+                     r"source_sha=(\S+)")
+    for fn in sorted(os.listdir(pdir)):
+        if not fn.endswith((".md", ".txt")):
+            continue
+        for line in open(os.path.join(pdir, fn)):
+            m = pat.search(line)
+            if m and m.group(1) == kernel and m.group(2) == workload and m.group(4) == sha:
+                return float(m.group(3))
+    return None
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running
+    (reads only; changes no setting)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_device):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nv = pynvml
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def start(self):
+        if self.ok:
+            self.th = threading.Thread(target=self._run, daemon=True)
+            self.th.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.th.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvml unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:  # region shorter than the sampling period: nearest samples
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+        reasons = sorted({name for _, _, rs in inside for bit, name in self.REASONS.items()
+                          if rs & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in inside) if inside else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def device_tensors(inp, dev):
+    import torch
+
+    def qkv(vals, bits):
+        if bits is not None:
+            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(vals).to(dev)
+
+    x = dict(Q=qkv(inp.Q, inp.Q_bits), K=qkv(inp.K, inp.K_bits), V=qkv(inp.V, inp.V_bits),
+             eta=torch.from_numpy(inp.eta).to(dev), W1=torch.from_numpy(inp.W1).to(dev),
+             gamma=torch.from_numpy(inp.gamma).to(dev), beta=torch.from_numpy(inp.beta).to(dev),
+             W2=torch.from_numpy(inp.W2).to(dev) if inp.W2 is not None else None)
+    return x
+
+
+def make_caller(wl, x, stream):
+    """Returns (call, outputs) where call() enqueues one library call on `stream`."""
+    import torch
+    import test_sequence_layers_layer_b200 as ttt
+    B, H, T, d = wl.B, wl.H, wl.T, wl.d
+    dev = x["Q"].device
+    dt = ttt.TTT_BF16 if wl.dtype == "bf16" else ttt.TTT_FP32
+    Z = torch.empty((B, H, T, d), dtype=torch.float32, device=dev)
+    sp = stream.cuda_stream
+    if wl.kind == "linear":
+        Wo = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+        flags = ttt.TTT_F_LN if wl.ln else 0
+
+        def call(x=x):
+            ttt.ttt_linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
+                               Z, Wo, B, H, T, d, wl.b, dt, flags, sp)
+        return call, (Z, Wo)
+    if wl.kind == "mlp":
+        W1o = torch.empty((B, H, d, wl.dh), dtype=torch.float32, device=dev)
+        W2o = torch.empty((B, H, wl.dh, d), dtype=torch.float32, device=dev)
+
+        def call(x=x):
+            ttt.ttt_mlp_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["W2"], x["gamma"],
+                            x["beta"], Z, W1o, W2o, B, H, T, d, wl.dh, wl.b, dt, ttt.TTT_F_LN, sp)
+        return call, (Z, W1o, W2o)
+    Wo = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+    need = ttt.ttt_chunk_workspace_bytes(B, H, T, d, wl.b)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+
+    def call(x=x):
+        ttt.ttt_chunk_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], Z, Wo, B, H, T, d, wl.b,
+                          dt, 0, ws, need, sp)
+    return call, (Z, Wo)
+
+
+def gpu_arm(args, wl, rank, world):
+    import torch
+    import torch.distributed as dist
+    import test_sequence_layers_layer_b200 as ttt
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    ttt.lib()
+    peaks, peaks_src = load_peaks()
+    inp = synth.make_inputs(wl.scaled(seed=wl.seed + rank))
+    x = device_tensors(inp, dev)
+    stream = torch.cuda.Stream(dev)
+    call, outs = make_caller(wl, x, stream)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[dev.index])
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            call()
+        stream.synchronize()
+        if ttt.ttt_device_status(stream.cuda_stream) != 0:
+            raise RuntimeError("device status error after warm-up")
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        n0 = ttt.ttt_launch_count()
+        t0 = time.perf_counter()
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record(stream)
+            call()
+            ends[k].record(stream)
+        torch.cuda.synchronize()
+        t1 = time.perf_counter()
+        launches = ttt.ttt_launch_count() - n0
+        barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+
+    # e2e through the C ABI with host buffers: pinned host -> device inputs,
+    # the call, device -> pinned host outputs, every step.
+    host_in = {k: v.cpu().pin_memory() for k, v in x.items() if v is not None}
+    dev_in = {k: torch.empty_like(v) for k, v in x.items() if v is not None}
+    call_e2e, outs_e2e = make_caller(wl, dev_in, stream)
+    host_out = [o.cpu().pin_memory() for o in outs_e2e if o is not None]
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(o.numel() * o.element_size() for o in host_out)
+    e2e_steps = max(3, min(args.steps, 10))
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            for k, v in host_in.items():
+                dev_in[k].copy_(v, non_blocking=True)
+            call_e2e()
+            for h, o in zip(host_out, [o for o in outs_e2e if o is not None]):
+                h.copy_(o, non_blocking=True)
+        e2e_step()
+        stream.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    sampler.stop()
+    if ttt.ttt_device_status(stream.cuda_stream) != 0:
+        raise RuntimeError("device status error in the timed region")
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+        lc = torch.tensor([launches], dtype=torch.float64, device=dev)
+        dist.all_reduce(lc)
+        launches = int(lc[0])
+
+    tokens = wl.tokens * world
+    ms_per_step = total_ms / args.steps
+    value = tokens * args.steps / (total_ms / 1e3)
+    kname, ksrc, kdtype = kernel_of(wl)
+    per_call = max(1, launches // (args.steps * world))
+    # The step is a single kernel launch, so the dominant kernel's average
+    # launch duration is the per-step event time.
+    kern_ms = ms_per_step if per_call == 1 else None
+    bound = bound_of(wl, peaks)
+    if bound == "hbm":
+        per_launch = algo_bytes_per_token(wl) * wl.tokens
+        achieved = per_launch / (kern_ms / 1e3) / 1e9 if kern_ms else None
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+    else:
+        per_launch = algo_flops_per_token(wl) * wl.tokens
+        achieved = per_launch / (kern_ms / 1e3) / 1e12 if kern_ms else None
+        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+    tflops = algo_flops_per_token(wl) * wl.tokens / (ms_per_step / 1e3) / 1e12
+    sha = source_sha(ksrc)
+    traffic = recorded_traffic(kname, wl.name, sha)
+    clocks = sampler.summary(t0, t1)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": kdtype,
+        "data": "synthetic (seeded SplitMix64 normals; bf16-rounded Q/K/V)",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "d": wl.d,
+                   "mini_batch": wl.b, "layer_norm": wl.ln, "qkv_dtype": wl.dtype,
+                   "tokens_per_step_per_gpu": wl.tokens, "l2": "flushed between steps (256 MiB write)",
+                   "parallelism": f"replicas x{world} (independent sequences)"},
+        "pct_of_bf16_tensor_peak": 100.0 * tflops / peaks["bf16_tflops"],
+        "algorithmic_tflops": tflops,
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                     "kernel": kname, "peak_source": peaks_src,
+                     "algorithmic_per_launch": per_launch},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "step_ms_min_median": [min(step_ms), statistics.median(step_ms)],
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------- CPU (oracle) arm
+
+def oracle_sample(wl, budget_s: float):
+    """Time the oracle on whole sequences of the workload, threaded over the
+    host cores, growing the sample until about budget_s of work or the whole
+    workload. Returns (tokens/s, cores, description)."""
+    import oracle
+
+    inp = synth.make_inputs(wl)
+    f64 = {k: (np.asarray(getattr(inp, k), dtype=np.float64) if getattr(inp, k) is not None else None)
+           for k in ("Q", "K", "V", "eta", "W1", "W2", "gamma", "beta")}
+    cores = oracle.num_threads()
+    nseq_total = wl.B * wl.H
+
+    def run(seqs):
+        t0 = time.perf_counter()
+        if wl.kind == "linear":
+            oracle.linear_primal(f64["Q"], f64["K"], f64["V"], f64["eta"], f64["W1"], f64["gamma"],
+                                 f64["beta"], b=wl.b, ln=wl.ln, seqs=seqs, with_w=True)
+        elif wl.kind == "mlp":
+            oracle.mlp_primal(f64["Q"], f64["K"], f64["V"], f64["eta"], f64["W1"], f64["W2"],
+                              f64["gamma"], f64["beta"], b=wl.b, seqs=seqs)
+        else:
+            oracle.chunk_primal(f64["Q"], f64["K"], f64["V"], f64["eta"], f64["W1"], chunk=wl.b,
+                                seqs=seqs)
+        return time.perf_counter() - t0
+
+    n = min(cores, nseq_total)
+    dt = run(list(range(n)))
+    while dt < budget_s / 4 and n < nseq_total:
+        n = min(nseq_total, max(n * 2, int(n * budget_s / max(dt, 1e-3) / 2)))
+        dt = run(list(range(n)))
+    tok = n * wl.T
+    desc = f"{n} of {nseq_total} sequences, full length T={wl.T} ({tok} tokens), {cores} threads"
+    return tok / dt, cores, desc
+
+
+def reference_arm(args, wl):
+    vals = []
+    cores, desc = None, None
+    per_step_budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    for k in range(args.warmup + args.steps):
+        v, cores, desc = oracle_sample(wl, per_step_budget)
+        if k >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.tokens / value * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded SplitMix64 normals; bf16-rounded Q/K/V)",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "d": wl.d,
+                   "mini_batch": wl.b},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ttt", choices=["ttt", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args, wl)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = gpu_arm(args, wl, rank, world)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            v, cores, desc = oracle_sample(wl, args.cpu_budget)
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
+                                    "kind": "oracle", "sample": desc}
+        elif rank == 0:
+            line["cpu_baseline"] = None
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,178 @@
+/*
+ * ttt.h -- C ABI of libttt.so: the forward pass of a Test-Time-Training (TTT)
+ * layer on one NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes. The hidden state of a TTT layer is a fast weight W
+ * per (batch, head) sequence: a linear map, or a small MLP. Tokens arrive as
+ * query/key/value rows q_t, k_t, v_t (the outer model's projections, computed
+ * elsewhere) with a per-token inner step size eta_t > 0. The fast weight is
+ * trained while the sequence streams, by gradient descent on the
+ * reconstruction loss l(W; t) = 1/2 || f(k_t; W) - v_t ||^2, and the layer
+ * emits z_t = f(q_t; W_t). Sources, on the TTT pages:
+ *   - "Test-Time Training: Linear Complexity Beyond Attention",
+ *     "The Dual-Loop Structure" (the inner loop is online gradient descent);
+ *     "Key Architectural Mechanics of TTT-Linear" part 1 (the loss), part 2
+ *     (gradient and update), part 3 (read-out with the updated weight, then
+ *     LayerNorm and a residual), part 4 "Mini-Batch Parallelism (Dual
+ *     Formulation)" (mini-batches of b tokens; gradients inside a mini-batch
+ *     at the weight it starts from; the change carried forward sequentially);
+ *   - "How to Master Test-Time Training for LLMs": the fast weight may be a
+ *     multi-layer perceptron;
+ *   - "Test-Time Training Done Right" (abstract): large-chunk TTT.
+ *
+ * Conventions common to every entry point.
+ *   - Row form: f(k; W) = k W with W[d_in][d_out] row-major (the pages write
+ *     the same map in column form, W k).
+ *   - Q, K, V, Z are [B][H][T][d], row-major and contiguous. eta is
+ *     [B][H][T] fp32. LayerNorm gain and bias are [H][d] fp32, fixed per head
+ *     (they belong to the outer model); LayerNorm uses eps = 1e-5 and the
+ *     population variance.
+ *   - A fast weight is shared by the batch ([H][...]) unless
+ *     TTT_F_W0_PER_SEQ is set, in which case it is [B][H][...] (this is how a
+ *     caller resumes a sequence: pass the previous call's W_out as W0).
+ *   - Z is written in fp32. W_out (fp32, [B][H][...]) may be NULL.
+ *   - Every pointer is a device pointer to memory the caller owns; the
+ *     library keeps no pointer after the call returns. Inputs are never
+ *     modified. W_out may alias W0 only when TTT_F_W0_PER_SEQ is set.
+ *     Q, K, V, Z, W0 and W_out must be 16-byte aligned.
+ *   - Calls enqueue work on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) and return without synchronising. Arguments are
+ *     checked on the host before anything is launched; a failed check
+ *     returns its error code and launches nothing.
+ *   - Kernels that wait on on-chip barriers bound every wait; if a wait runs
+ *     out they record it in a device-side status word and return early, so
+ *     the CUDA context stays usable. ttt_device_status() reports that word.
+ *   - There is no CPU fallback: a device that is not sm_100 returns
+ *     TTT_ERR_UNSUPPORTED_ARCH.
+ */
+#ifndef TTT_H
+#define TTT_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define TTT_API __attribute__((visibility("default")))
+#else
+#define TTT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TTT_OK = 0,
+    TTT_ERR_ARG = -1,            /* bad flag bits or an inconsistent argument   */
+    TTT_ERR_SHAPE = -2,          /* unsupported or inconsistent B,H,T,d,b       */
+    TTT_ERR_DTYPE = -3,          /* dtype not supported for this shape          */
+    TTT_ERR_ALIGN = -4,          /* a pointer is not 16-byte aligned            */
+    TTT_ERR_PTR = -5,            /* a required pointer is NULL or not device memory */
+    TTT_ERR_LAUNCH = -6,         /* the CUDA launch failed (see cudaGetLastError) */
+    TTT_ERR_DEVICE_TIMEOUT = -7, /* a bounded on-chip wait ran out (device status) */
+    TTT_ERR_UNSUPPORTED_ARCH = -8, /* current device is not sm_100              */
+    TTT_ERR_WORKSPACE = -9       /* workspace NULL, misaligned or too small     */
+} ttt_status;
+
+typedef enum { TTT_BF16 = 0, TTT_FP32 = 1 } ttt_dtype; /* element type of Q, K, V */
+
+typedef void *ttt_stream; /* a cudaStream_t */
+
+#define TTT_F_LN 1u         /* f(k) = k + LN(k W) instead of f(k) = k W        */
+#define TTT_F_W0_PER_SEQ 2u /* W0 is [B][H][...] instead of [H][...]           */
+
+#define TTT_ABI_VERSION 1
+
+/* ABI version of the loaded library (TTT_ABI_VERSION at build time). */
+TTT_API int ttt_abi_version(void);
+
+/* Static, human-readable text for a status code; never NULL. */
+TTT_API const char *ttt_status_string(int status);
+
+/*
+ * TTT-Linear forward, update-then-apply, mini-batch b.
+ *   For mini-batch m (tokens mb .. mb+b-1) starting from weight W_m:
+ *     G_s  = eta_s * dl/dx at x = k_s W_m        (one row per token s)
+ *     z_t  = f(q_t; W_m - sum_{s<=t} k_s^T G_s)   (the token's own step included)
+ *     W_{m+1} = W_m - K_m^T G
+ *   which is the mini-batch dual form Zpre = Q W_m - tril(Q K^T) G,
+ *   W_{m+1} = W_m - K^T G. Without TTT_F_LN, f(k) = k W and dl/dx = kW - v;
+ *   with it, f(k) = k + LN(k W) and dl/dx is the LayerNorm backward of
+ *   (f - v). ("Key Architectural Mechanics of TTT-Linear", parts 1-4.)
+ * Arguments:
+ *   Q, K, V   [B][H][T][d], dtype dt
+ *   eta       [B][H][T] fp32
+ *   W0        [H][d][d] (or [B][H][d][d] with TTT_F_W0_PER_SEQ) fp32
+ *   ln_gamma, ln_beta  [H][d] fp32; required with TTT_F_LN, ignored without
+ *   Z         [B][H][T][d] fp32 output
+ *   W_out     [B][H][d][d] fp32 output, the weight after the last token; may be NULL
+ * Supported: T % b == 0; d in {16, 32, 64} and 1 <= b <= 64 with b*d <= 4096
+ *   for TTT_FP32 and TTT_BF16; TTT_BF16 with d = 64, b = 16 runs the
+ *   tensor-core scan, every other case the fp32 CUDA-core kernel.
+ */
+TTT_API ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const float *eta,
+                          const float *W0, const float *ln_gamma, const float *ln_beta,
+                          float *Z, float *W_out, int B, int H, int T, int d, int b,
+                          ttt_dtype dt, unsigned flags, ttt_stream stream);
+
+/*
+ * TTT-MLP forward: f(k) = k + LN(GELU(k W1) W2) with W1 [d][dh], W2 [dh][d],
+ * GELU the exact erf form; same mini-batch rule as ttt_linear_fwd, with both
+ * layers updated ("How to Master Test-Time Training for LLMs": the hidden
+ * state may be an MLP). In dual form, with A = GELU(K W1),
+ * Gx_s = eta_s dl/dx_s and Gh = (Gx W2^T) * GELU'(K W1):
+ *   Zpre = GELU(Q W1 - tril(Q K^T) Gh) W2 - tril(Aq A^T) Gx, z = q + LN(Zpre),
+ *   W1 -= K^T Gh, W2 -= A^T Gx.
+ * Arguments as ttt_linear_fwd, plus:
+ *   W1_0  [H][d][dh] (or [B][H][d][dh]), W2_0 [H][dh][d] (or [B][H][dh][d]) fp32
+ *   W1_out [B][H][d][dh], W2_out [B][H][dh][d] fp32 outputs, each may be NULL
+ * flags must contain TTT_F_LN (the MLP form is defined with LayerNorm).
+ * Supported: d in {16, 32, 64}, dh = 4 d, 1 <= b <= 16, T % b == 0,
+ *   dtype TTT_BF16 or TTT_FP32.
+ */
+TTT_API ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float *eta,
+                       const float *W1_0, const float *W2_0, const float *ln_gamma,
+                       const float *ln_beta, float *Z, float *W1_out, float *W2_out, int B,
+                       int H, int T, int d, int dh, int b, ttt_dtype dt, unsigned flags,
+                       ttt_stream stream);
+
+/*
+ * Large-chunk TTT forward, apply-then-update ("Test-Time Training Done
+ * Right"): the tokens of chunk c all read out with W_c, the weight left by
+ * the chunks before it, then
+ *   W_{c+1} = W_c - sum_{s in c} eta_s k_s^T (k_s W_c - v_s).
+ * f(k) = k W (no LayerNorm). With eta_s = 1/chunk this is one step of
+ * gradient descent on the chunk's mean loss.
+ * Arguments as ttt_linear_fwd without LayerNorm; `chunk` is the chunk length.
+ * workspace: device scratch of at least ttt_chunk_workspace_bytes(...) bytes,
+ *   256-byte aligned, owned by the caller; its contents on entry do not
+ *   matter and are clobbered. Calls that share a workspace must not overlap.
+ * Supported: d = 128 and chunk % 128 == 0 with TTT_BF16; T % chunk == 0.
+ * flags: only TTT_F_W0_PER_SEQ.
+ */
+TTT_API size_t ttt_chunk_workspace_bytes(int B, int H, int T, int d, int chunk);
+
+TTT_API ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, const float *eta,
+                         const float *W0, float *Z, float *W_out, int B, int H, int T, int d,
+                         int chunk, ttt_dtype dt, unsigned flags, void *workspace,
+                         size_t workspace_bytes, ttt_stream stream);
+
+/*
+ * Synchronises `stream`, then returns TTT_OK, TTT_ERR_DEVICE_TIMEOUT if a
+ * kernel of this library ran out of a bounded wait since the last call
+ * (the word is then cleared), or TTT_ERR_LAUNCH if the stream reports a CUDA
+ * error.
+ */
+TTT_API ttt_status ttt_device_status(ttt_stream stream);
+
+/*
+ * Number of kernels this library has launched in this process so far (a
+ * host-side counter, incremented once per successful kernel launch). Lets a
+ * caller count the library's launches inside a timed region.
+ */
+TTT_API unsigned long long ttt_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_H */

@@ -1,0 +1,196 @@
+"""Python binding of libttt.so, the B200 library for the forward pass of a
+Test-Time-Training (TTT) layer.
+
+The functions named like the C ABI (ttt_linear_fwd, ttt_mlp_fwd,
+ttt_chunk_fwd, ...) take exactly the C arguments; a pointer argument may be a
+torch tensor (its data_ptr() is passed), an int address, or None. They only
+marshal arguments: every step of the computation runs in the library's CUDA
+kernels. linear_fwd / mlp_fwd / chunk_fwd are conveniences that read the
+shapes off torch tensors and allocate the outputs with torch.
+
+There is no fallback: if libttt.so is missing or fails to load, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libttt.so")
+HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "ttt.h")
+
+TTT_OK = 0
+TTT_BF16, TTT_FP32 = 0, 1
+TTT_F_LN = 1
+TTT_F_W0_PER_SEQ = 2
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_lib = None
+
+
+class TTTError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} returned {status}: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libttt.so (built in-tree by build.py). Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libttt.so not built at {LIB_PATH}; run build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        L.ttt_abi_version.restype = _I
+        L.ttt_abi_version.argtypes = []
+        L.ttt_status_string.restype = ctypes.c_char_p
+        L.ttt_status_string.argtypes = [_I]
+        L.ttt_linear_fwd.restype = _I
+        L.ttt_linear_fwd.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_uint, _P]
+        L.ttt_mlp_fwd.restype = _I
+        L.ttt_mlp_fwd.argtypes = [_P] * 11 + [_I] * 7 + [ctypes.c_uint, _P]
+        L.ttt_chunk_workspace_bytes.restype = ctypes.c_size_t
+        L.ttt_chunk_workspace_bytes.argtypes = [_I] * 5
+        L.ttt_chunk_fwd.restype = _I
+        L.ttt_chunk_fwd.argtypes = [_P] * 7 + [_I] * 6 + [ctypes.c_uint, _P, ctypes.c_size_t, _P]
+        L.ttt_device_status.restype = _I
+        L.ttt_device_status.argtypes = [_P]
+        L.ttt_launch_count.restype = ctypes.c_ulonglong
+        L.ttt_launch_count.argtypes = []
+        _lib = L
+    return _lib
+
+
+def header_symbols() -> list[str]:
+    """Names of the functions include/ttt.h declares."""
+    text = open(HEADER_PATH).read()
+    return re.findall(r"TTT_API\s+[\w\s\*]*?\b(ttt_\w+)\s*\(", text)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(fn, rc):
+    if rc != TTT_OK:
+        raise TTTError(fn, rc)
+    return rc
+
+
+def status_string(status: int) -> str:
+    return lib().ttt_status_string(int(status)).decode()
+
+
+def abi_version() -> int:
+    return lib().ttt_abi_version()
+
+
+# ----------------------------------------------------------------- C-ABI calls
+
+def ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b, dt, flags,
+                   stream=None, check=True):
+    rc = lib().ttt_linear_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(ln_gamma),
+                              _ptr(ln_beta), _ptr(Z), _ptr(W_out), B, H, T, d, b, dt, flags,
+                              _stream(stream))
+    return _check("ttt_linear_fwd", rc) if check else rc
+
+
+def ttt_mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out, B, H, T, d, dh,
+                b, dt, flags, stream=None, check=True):
+    rc = lib().ttt_mlp_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W1_0), _ptr(W2_0),
+                           _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z), _ptr(W1_out), _ptr(W2_out),
+                           B, H, T, d, dh, b, dt, flags, _stream(stream))
+    return _check("ttt_mlp_fwd", rc) if check else rc
+
+
+def ttt_chunk_workspace_bytes(B, H, T, d, chunk) -> int:
+    return int(lib().ttt_chunk_workspace_bytes(B, H, T, d, chunk))
+
+
+def ttt_chunk_fwd(Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, dt, flags, workspace,
+                  workspace_bytes, stream=None, check=True):
+    rc = lib().ttt_chunk_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(Z),
+                             _ptr(W_out), B, H, T, d, chunk, dt, flags, _ptr(workspace),
+                             workspace_bytes, _stream(stream))
+    return _check("ttt_chunk_fwd", rc) if check else rc
+
+
+def ttt_device_status(stream=None) -> int:
+    return lib().ttt_device_status(_stream(stream))
+
+
+def ttt_launch_count() -> int:
+    return int(lib().ttt_launch_count())
+
+
+# ----------------------------------------------------------------- conveniences
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return TTT_BF16
+    if t.dtype == torch.float32:
+        return TTT_FP32
+    raise TypeError(f"Q/K/V must be bf16 or fp32, got {t.dtype}")
+
+
+def linear_fwd(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, w0_per_seq=False,
+               stream=None, want_w=True):
+    """TTT-Linear forward. Q, K, V: [B,H,T,d] cuda tensors (bf16 or fp32).
+    Returns (Z fp32 [B,H,T,d], W_out fp32 [B,H,d,d] or None)."""
+    import torch
+    B, H, T, d = Q.shape
+    Z = torch.empty((B, H, T, d), dtype=torch.float32, device=Q.device)
+    W_out = torch.empty((B, H, d, d), dtype=torch.float32, device=Q.device) if want_w else None
+    flags = (TTT_F_LN if ln else 0) | (TTT_F_W0_PER_SEQ if w0_per_seq else 0)
+    ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
+                   _dtype_code(Q), flags, stream)
+    return Z, W_out
+
+
+def mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, *, b, w0_per_seq=False, stream=None,
+            want_w=True):
+    """TTT-MLP forward. Returns (Z, W1_out, W2_out)."""
+    import torch
+    B, H, T, d = Q.shape
+    dh = W1_0.shape[-1]
+    Z = torch.empty((B, H, T, d), dtype=torch.float32, device=Q.device)
+    W1o = torch.empty((B, H, d, dh), dtype=torch.float32, device=Q.device) if want_w else None
+    W2o = torch.empty((B, H, dh, d), dtype=torch.float32, device=Q.device) if want_w else None
+    flags = TTT_F_LN | (TTT_F_W0_PER_SEQ if w0_per_seq else 0)
+    ttt_mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1o, W2o, B, H, T, d, dh, b,
+                _dtype_code(Q), flags, stream)
+    return Z, W1o, W2o
+
+
+def chunk_fwd(Q, K, V, eta, W0, *, chunk, w0_per_seq=False, workspace=None, stream=None,
+              want_w=True):
+    """Large-chunk TTT forward (apply-then-update). Allocates the workspace
+    with torch unless one is given. Returns (Z, W_out)."""
+    import torch
+    B, H, T, d = Q.shape
+    Z = torch.empty((B, H, T, d), dtype=torch.float32, device=Q.device)
+    W_out = torch.empty((B, H, d, d), dtype=torch.float32, device=Q.device) if want_w else None
+    need = ttt_chunk_workspace_bytes(B, H, T, d, chunk)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    flags = TTT_F_W0_PER_SEQ if w0_per_seq else 0
+    ttt_chunk_fwd(Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, _dtype_code(Q), flags,
+                  workspace, need, stream)
+    return Z, W_out

@@ -1,0 +1,199 @@
+// ttt_api.cu -- the extern "C" entry points of libttt.so (declared in
+// include/ttt.h): host-side argument checks, then dispatch to a kernel
+// launcher on the caller's stream. No allocation, no synchronisation (except
+// in ttt_device_status).
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/ttt.h"
+#include "ttt_common.cuh"
+
+namespace ttt {
+
+__device__ int g_device_status;  // set by a kernel whose bounded wait ran out
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+int *device_status_word() {
+    int *p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_device_status) != cudaSuccess)
+        return nullptr;
+    return p;
+}
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A pointer the GPU can dereference: device or managed memory.
+bool is_device_ptr(const void *p) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the sticky-free error
+        return false;
+    }
+    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+// sm_100 check of the current device, cached per device ordinal.
+ttt_status check_arch() {
+    static int cached[64];  // 0 unknown, 1 ok, -1 not sm_100
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return TTT_ERR_UNSUPPORTED_ARCH;
+    }
+    if (dev < 0 || dev >= 64) return TTT_ERR_UNSUPPORTED_ARCH;
+    if (cached[dev] == 0) {
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        cached[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    return cached[dev] == 1 ? TTT_OK : TTT_ERR_UNSUPPORTED_ARCH;
+}
+
+bool supported_d(int d) { return d == 16 || d == 32 || d == 64; }
+
+ttt_status check_device_ptrs(const void *const *ptrs, int n) {
+    for (int i = 0; i < n; ++i)
+        if (ptrs[i] && !is_device_ptr(ptrs[i])) return TTT_ERR_PTR;
+    return TTT_OK;
+}
+
+ttt_status launched(cudaError_t e) { return e == cudaSuccess ? TTT_OK : TTT_ERR_LAUNCH; }
+
+}  // namespace
+}  // namespace ttt
+
+using namespace ttt;
+
+extern "C" {
+
+int ttt_abi_version(void) { return TTT_ABI_VERSION; }
+
+const char *ttt_status_string(int status) {
+    switch (status) {
+        case TTT_OK: return "ok";
+        case TTT_ERR_ARG: return "invalid argument or flag";
+        case TTT_ERR_SHAPE: return "unsupported or inconsistent shape";
+        case TTT_ERR_DTYPE: return "unsupported dtype";
+        case TTT_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case TTT_ERR_PTR: return "required pointer is NULL or not device memory";
+        case TTT_ERR_LAUNCH: return "CUDA launch failed";
+        case TTT_ERR_DEVICE_TIMEOUT: return "a bounded on-chip wait ran out on the device";
+        case TTT_ERR_UNSUPPORTED_ARCH: return "current device is not sm_100 (B200)";
+        case TTT_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        default: return "unknown status";
+    }
+}
+
+ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const float *eta,
+                          const float *W0, const float *ln_gamma, const float *ln_beta,
+                          float *Z, float *W_out, int B, int H, int T, int d, int b,
+                          ttt_dtype dt, unsigned flags, ttt_stream stream) {
+    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ)) return TTT_ERR_ARG;
+    const bool ln = flags & TTT_F_LN;
+    if (!Q || !K || !V || !eta || !W0 || !Z) return TTT_ERR_PTR;
+    if (ln && (!ln_gamma || !ln_beta)) return TTT_ERR_PTR;
+    if (B <= 0 || H <= 0 || T <= 0 || b <= 0 || b > 64 || T % b != 0) return TTT_ERR_SHAPE;
+    if (!supported_d(d) || b * d > 4096) return TTT_ERR_SHAPE;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return TTT_ERR_SHAPE;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Z) || !aligned16(W0) ||
+        (W_out && !aligned16(W_out)))
+        return TTT_ERR_ALIGN;
+    if (W_out && W_out == W0 && !(flags & TTT_F_W0_PER_SEQ)) return TTT_ERR_ARG;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out};
+    st = check_device_ptrs(ptrs, 9);
+    if (st != TTT_OK) return st;
+
+    LinearArgs a{Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
+                 dt == TTT_BF16, ln, (flags & TTT_F_W0_PER_SEQ) != 0};
+    return launched(launch_linear_simt(a, static_cast<cudaStream_t>(stream)));
+}
+
+ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float *eta,
+                       const float *W1_0, const float *W2_0, const float *ln_gamma,
+                       const float *ln_beta, float *Z, float *W1_out, float *W2_out, int B,
+                       int H, int T, int d, int dh, int b, ttt_dtype dt, unsigned flags,
+                       ttt_stream stream) {
+    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ)) return TTT_ERR_ARG;
+    if (!(flags & TTT_F_LN)) return TTT_ERR_ARG;
+    if (!Q || !K || !V || !eta || !W1_0 || !W2_0 || !ln_gamma || !ln_beta || !Z) return TTT_ERR_PTR;
+    if (B <= 0 || H <= 0 || T <= 0 || b <= 0 || b > 16 || T % b != 0) return TTT_ERR_SHAPE;
+    if (!supported_d(d) || dh != 4 * d) return TTT_ERR_SHAPE;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return TTT_ERR_SHAPE;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Z) || !aligned16(W1_0) ||
+        !aligned16(W2_0) || (W1_out && !aligned16(W1_out)) || (W2_out && !aligned16(W2_out)))
+        return TTT_ERR_ALIGN;
+    const bool per_seq = flags & TTT_F_W0_PER_SEQ;
+    if (!per_seq && ((W1_out && W1_out == W1_0) || (W2_out && W2_out == W2_0))) return TTT_ERR_ARG;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out};
+    st = check_device_ptrs(ptrs, 11);
+    if (st != TTT_OK) return st;
+
+    MlpArgs a{Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out,
+              B, H, T, d, dh, b, dt == TTT_BF16, per_seq};
+    return launched(launch_mlp_simt(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t ttt_chunk_workspace_bytes(int B, int H, int T, int d, int chunk) {
+    (void)B; (void)H; (void)T; (void)d; (void)chunk;
+    return 0;
+}
+
+ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, const float *eta,
+                         const float *W0, float *Z, float *W_out, int B, int H, int T, int d,
+                         int chunk, ttt_dtype dt, unsigned flags, void *workspace,
+                         size_t workspace_bytes, ttt_stream stream) {
+    if (flags & ~TTT_F_W0_PER_SEQ) return TTT_ERR_ARG;
+    if (!Q || !K || !V || !eta || !W0 || !Z) return TTT_ERR_PTR;
+    if (B <= 0 || H <= 0 || T <= 0 || chunk <= 0 || T % chunk != 0 || chunk % 128 != 0)
+        return TTT_ERR_SHAPE;
+    if (d != 64 && d != 128) return TTT_ERR_SHAPE;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return TTT_ERR_SHAPE;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Z) || !aligned16(W0) ||
+        (W_out && !aligned16(W_out)))
+        return TTT_ERR_ALIGN;
+    const size_t need = ttt_chunk_workspace_bytes(B, H, T, d, chunk);
+    if (need && (!workspace || workspace_bytes < need ||
+                 (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+        return TTT_ERR_WORKSPACE;
+    if (W_out && W_out == W0 && !(flags & TTT_F_W0_PER_SEQ)) return TTT_ERR_ARG;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {Q, K, V, eta, W0, Z, W_out, need ? workspace : nullptr};
+    st = check_device_ptrs(ptrs, 8);
+    if (st != TTT_OK) return st;
+
+    ChunkArgs a{Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, dt == TTT_BF16,
+                (flags & TTT_F_W0_PER_SEQ) != 0, workspace, workspace_bytes};
+    return launched(launch_chunk_simt(a, static_cast<cudaStream_t>(stream)));
+}
+
+ttt_status ttt_device_status(ttt_stream stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TTT_ERR_LAUNCH;
+    int *w = device_status_word();
+    if (!w) return TTT_ERR_LAUNCH;
+    int v = 0;
+    if (cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TTT_ERR_LAUNCH;
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        return TTT_ERR_DEVICE_TIMEOUT;
+    }
+    return TTT_OK;
+}
+
+unsigned long long ttt_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+// ttt_common.cuh -- internal declarations shared by the CUDA sources of libttt.
+// Not part of the public ABI (that is include/ttt.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ttt {
+
+constexpr float kLnEps = 1e-5f;  // torch nn.LayerNorm default, as in the pages' listing
+
+// Problem description handed from the ABI layer to a launcher. Pointers are
+// device pointers already validated by the ABI layer.
+struct LinearArgs {
+    const void *Q, *K, *V;
+    const float *eta, *W0, *gamma, *beta;
+    float *Z, *W_out;
+    int B, H, T, d, b;
+    bool bf16, ln, w0_per_seq;
+};
+
+struct MlpArgs {
+    const void *Q, *K, *V;
+    const float *eta, *W1_0, *W2_0, *gamma, *beta;
+    float *Z, *W1_out, *W2_out;
+    int B, H, T, d, dh, b;
+    bool bf16, w0_per_seq;
+};
+
+struct ChunkArgs {
+    const void *Q, *K, *V;
+    const float *eta, *W0;
+    float *Z, *W_out;
+    int B, H, T, d, chunk;
+    bool bf16, w0_per_seq;
+    void *workspace;
+    size_t workspace_bytes;
+};
+
+// Launchers return cudaSuccess or the launch error.
+cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s);
+cudaError_t launch_mlp_simt(const MlpArgs &a, cudaStream_t s);
+cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
+
+// Host-side count of kernel launches (ttt_launch_count); launchers call
+// count_launch() after each successful launch.
+void count_launch(int n = 1);
+
+// Device-side status word (bounded waits that ran out set it). Defined in
+// ttt_api.cu; kernels get its address as an argument.
+int *device_status_word();
+
+__device__ __forceinline__ float load_elem(const void *p, size_t i, bool bf16) {
+    if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+    return reinterpret_cast<const float *>(p)[i];
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+}  // namespace ttt

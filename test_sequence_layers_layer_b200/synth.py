@@ -22,6 +22,8 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -36,38 +38,60 @@ _BLOCK = 1 << 22  # elements generated per numpy block
 
 
 def _mix64(z: np.ndarray) -> np.ndarray:
-    """SplitMix64 output finaliser (wrapping uint64 arithmetic)."""
-    z = z ^ (z >> np.uint64(30))
-    z = z * _M1
-    z = z ^ (z >> np.uint64(27))
-    z = z * _M2
-    return z ^ (z >> np.uint64(31))
+    """SplitMix64 output finaliser (wrapping uint64 arithmetic), in place."""
+    with np.errstate(over="ignore"):
+        z ^= z >> np.uint64(30)
+        z *= _M1
+        z ^= z >> np.uint64(27)
+        z *= _M2
+        z ^= z >> np.uint64(31)
+    return z
 
 
 def stream_key(seed: int, tid: int) -> np.uint64:
     """Starting state of the stream for tensor `tid` under `seed`."""
     with np.errstate(over="ignore"):
         base = np.array([(int(seed) << 8) | int(tid)], dtype=np.uint64)
-        return _mix64(base + _GOLDEN)[0]
+        base += _GOLDEN
+        return _mix64(base)[0]
 
 
 def uniforms(seed: int, tid: int, start: int, count: int) -> np.ndarray:
     """Uniform doubles in (0, 1) for counters start .. start+count-1."""
     key = stream_key(seed, tid)
-    ctr = np.arange(start + 1, start + count + 1, dtype=np.uint64)
+    x = np.arange(start + 1, start + count + 1, dtype=np.uint64)
     with np.errstate(over="ignore"):
-        x = _mix64(key + ctr * _GOLDEN)
-    return ((x >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
+        x *= _GOLDEN
+        x += key
+    _mix64(x)
+    x >>= np.uint64(11)
+    u = x.astype(np.float64)
+    u += 0.5
+    u *= 2.0 ** -53
+    return u
 
 
 def normals(seed: int, tid: int, n: int) -> np.ndarray:
     """n standard normals (float64) of stream (seed, tid)."""
     out = np.empty(n, dtype=np.float64)
-    for lo in range(0, n, _BLOCK):
+
+    def block(lo):
         cnt = min(_BLOCK, n - lo)
         u = uniforms(seed, tid, 2 * lo, 2 * cnt)
-        u1, u2 = u[0::2], u[1::2]
-        out[lo:lo + cnt] = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * math.pi * u2)
+        r = np.log(u[0::2])
+        r *= -2.0
+        np.sqrt(r, out=r)
+        c = u[1::2] * (2.0 * math.pi)
+        np.cos(c, out=c)
+        np.multiply(r, c, out=out[lo:lo + cnt])
+
+    starts = range(0, n, _BLOCK)
+    if n > _BLOCK:
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(block, starts))
+    else:
+        for lo in starts:
+            block(lo)
     return out
 
 

@@ -1,0 +1,80 @@
+"""The C-ABI library without a GPU: it loads, exports every function
+include/ttt.h declares, and rejects bad arguments on the host before any
+launch."""
+import ctypes
+
+import pytest
+
+import test_sequence_layers_layer_b200 as ttt
+
+ALIGNED = 1 << 20  # a fake, 16-byte aligned "device" address; never dereferenced
+
+
+def test_library_loads_and_exports_header_symbols():
+    L = ttt.lib()
+    syms = ttt.header_symbols()
+    assert set(syms) >= {"ttt_linear_fwd", "ttt_mlp_fwd", "ttt_chunk_fwd",
+                         "ttt_chunk_workspace_bytes", "ttt_status_string",
+                         "ttt_abi_version", "ttt_device_status"}
+    for s in syms:
+        assert hasattr(L, s), s
+    assert ttt.abi_version() == 1
+
+
+def test_status_strings():
+    for code in range(-9, 1):
+        assert ttt.status_string(code) not in ("", "unknown status")
+    assert ttt.status_string(-1234) == "unknown status"
+
+
+def lin(**kw):
+    args = dict(Q=ALIGNED, K=ALIGNED, V=ALIGNED, eta=ALIGNED, W0=ALIGNED, ln_gamma=ALIGNED,
+                ln_beta=ALIGNED, Z=ALIGNED, W_out=None, B=1, H=1, T=64, d=64, b=16,
+                dt=ttt.TTT_BF16, flags=ttt.TTT_F_LN, stream=0)
+    args.update(kw)
+    return ttt.ttt_linear_fwd(**args, check=False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=60), -2),              # T % b != 0
+    (dict(d=48), -2),              # unsupported d
+    (dict(b=0), -2),
+    (dict(B=0), -2),
+    (dict(dt=7), -3),
+    (dict(flags=8), -1),           # unknown flag bit
+    (dict(Q=None), -5),
+    (dict(ln_gamma=None), -5),     # LN requires gamma/beta
+    (dict(Q=ALIGNED + 4), -4),     # misaligned
+    (dict(Z=ALIGNED + 8), -4),
+    (dict(W_out=ALIGNED, W0=ALIGNED), -1),  # aliasing W_out/W0 without per-seq W0
+])
+def test_linear_host_validation(kw, code):
+    assert lin(**kw) == code
+
+
+def test_linear_without_ln_does_not_need_gamma():
+    # validation passes; on a machine without a GPU the arch check then fails
+    rc = lin(ln_gamma=None, ln_beta=None, flags=0)
+    assert rc in (-8, -5)
+
+
+def test_mlp_and_chunk_host_validation():
+    m = dict(Q=ALIGNED, K=ALIGNED, V=ALIGNED, eta=ALIGNED, W1_0=ALIGNED, W2_0=ALIGNED,
+             ln_gamma=ALIGNED, ln_beta=ALIGNED, Z=ALIGNED, W1_out=None, W2_out=None,
+             B=1, H=1, T=32, d=64, dh=256, b=16, dt=ttt.TTT_BF16, flags=ttt.TTT_F_LN, stream=0)
+    assert ttt.ttt_mlp_fwd(**{**m, "dh": 128}, check=False) == -2
+    assert ttt.ttt_mlp_fwd(**{**m, "flags": 0}, check=False) == -1   # MLP needs LN
+    assert ttt.ttt_mlp_fwd(**{**m, "b": 32}, check=False) == -2
+    c = dict(Q=ALIGNED, K=ALIGNED, V=ALIGNED, eta=ALIGNED, W0=ALIGNED, Z=ALIGNED, W_out=None,
+             B=1, H=1, T=4096, d=128, chunk=2048, dt=ttt.TTT_BF16, flags=0,
+             workspace=None, workspace_bytes=0, stream=0)
+    assert ttt.ttt_chunk_fwd(**{**c, "chunk": 1000}, check=False) == -2
+    assert ttt.ttt_chunk_fwd(**{**c, "T": 3000}, check=False) == -2
+    assert ttt.ttt_chunk_fwd(**{**c, "flags": ttt.TTT_F_LN}, check=False) == -1
+
+
+def test_no_gpu_means_unsupported_not_fallback():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert lin() == -8

@@ -1,0 +1,141 @@
+"""Parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Small cases span several mini-batches/chunks, sequence counts that do not
+fill the machine evenly (150 > 148 SMs) and the degenerate shapes; the
+full-size workloads are checked on sampled sequences (each sequence is
+independent, so the oracle computes exactly those sequences)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import test_sequence_layers_layer_b200 as ttt
+from test_sequence_layers_layer_b200 import synth
+
+from gpu_helpers import check_parity, run_gpu, to_dev, TOL, max_rel_err, run_oracle
+
+pytestmark = pytest.mark.gpu
+W = synth.WORKLOADS
+
+SMALL = {
+    # fp32 CUDA-core path
+    "linear_fp32_d16_full": W["linear_fp32_d16"],
+    "linear_fp32_d64_noln": W["linear_fp32_d16"].scaled(B=2, H=3, T=128, d=64, b=16),
+    "linear_fp32_d32_ln_b8": W["linear_fp32_d16"].scaled(B=2, H=2, T=64, d=32, b=8, ln=True,
+                                                         eta="sigmoid_over_d"),
+    "linear_fp32_d16_b1": W["linear_fp32_d16"].scaled(T=32, b=1),
+    "linear_fp32_d64_ln_b64": W["linear_fp32_d16"].scaled(B=1, H=2, T=128, d=64, b=64, ln=True,
+                                                          eta="sigmoid_over_d"),
+    # bf16 linear + LN, d=64, b=16
+    "linear_ln_small": W["linear_ln_d64_b8h12_t2048"].scaled(B=2, H=3, T=64),
+    "linear_ln_T_eq_b": W["linear_ln_d64_b8h12_t2048"].scaled(B=1, H=5, T=16),
+    "linear_ln_150_seqs": W["linear_ln_d64_b8h12_t2048"].scaled(B=10, H=15, T=32),
+    "linear_ln_long": W["linear_ln_d64_b8h12_t2048"].scaled(B=1, H=2, T=1024),
+    "linear_noln_bf16": W["linear_ln_d64_b8h12_t2048"].scaled(B=2, H=2, T=128, ln=False),
+    # MLP
+    "mlp_small": W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=1, H=3, T=48),
+    "mlp_fp32_d16": W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=2, H=2, T=32, d=16, dh=64, b=4,
+                                                             dtype="fp32"),
+    # large chunk
+    "chunk_small": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=1, H=3, T=768, b=256,
+                                                            eta="const:0.00390625"),
+    "chunk_two_chunks": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=1, H=2, T=4096),
+    "chunk_d64": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=2, H=1, T=512, d=64, b=128,
+                                                          eta="const:0.0078125"),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_parity(name):
+    check_parity(synth.make_inputs(SMALL[name]))
+
+
+FULL = [
+    ("linear_fp32_d16", None),
+    ("linear_ln_d64_b8h12_t2048", None),
+    ("linear_ln_d64_b1h32_t32768", None),
+    ("mlp_ln_d64_dh256_b4h12_t8192", [0, 13, 26, 47]),
+    ("chunk_d128_c2048_b4h8_t32768", [0, 9, 18, 31]),
+]
+
+
+@pytest.mark.parametrize("name,seqs", FULL, ids=[f[0] for f in FULL])
+def test_full_size_parity(name, seqs):
+    inp = synth.make_inputs(W[name])
+    errs = check_parity(inp, seqs=seqs)
+    print(f"{name}: max rel err {errs}")
+
+
+# ------------------------------------------------------------------ edge cases
+
+def test_eta_zero_keeps_initial_weight():
+    wl = W["linear_ln_d64_b8h12_t2048"].scaled(B=1, H=2, T=64)
+    inp = synth.make_inputs(wl)
+    inp.eta[:] = 0
+    Z, Wo = run_gpu(inp)
+    np.testing.assert_array_equal(Wo[0], inp.W1.astype(np.float64))
+    check_parity(inp)
+
+
+@pytest.mark.parametrize("name", ["linear_ln_small", "linear_fp32_d64_noln"])
+def test_resume_split_equals_whole(name):
+    wl = SMALL[name]
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    Zw, Ww = ttt.linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
+                            b=wl.b, ln=wl.ln)
+    h = wl.T // 2
+    sl = lambda t: t[:, :, :h].contiguous()
+    sr = lambda t: t[:, :, h:].contiguous()
+    Z1, W1 = ttt.linear_fwd(sl(x["Q"]), sl(x["K"]), sl(x["V"]), sl(x["eta"]), x["W1"],
+                            x["gamma"], x["beta"], b=wl.b, ln=wl.ln)
+    Z2, W2 = ttt.linear_fwd(sr(x["Q"]), sr(x["K"]), sr(x["V"]), sr(x["eta"]), W1,
+                            x["gamma"], x["beta"], b=wl.b, ln=wl.ln, w0_per_seq=True)
+    torch.cuda.synchronize()
+    tol = TOL[wl.dtype]
+    assert max_rel_err(torch.cat([Z1, Z2], 2).cpu().numpy(), Zw.cpu().numpy(), wl) <= tol
+    assert max_rel_err(W2.cpu().numpy(), Ww.cpu().numpy(), wl) <= tol
+
+
+def test_w_out_null_and_alias():
+    wl = SMALL["linear_ln_small"]
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    Z0, W0o = ttt.linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
+                             b=16, ln=True)
+    Zn, none = ttt.linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
+                              b=16, ln=True, want_w=False)
+    assert none is None
+    torch.testing.assert_close(Zn, Z0, rtol=0, atol=0)
+    # in-place state update: W_out aliases a per-sequence W0
+    Wps = x["W1"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    Z = torch.empty_like(Z0)
+    ttt.ttt_linear_fwd(x["Q"], x["K"], x["V"], x["eta"], Wps, x["gamma"], x["beta"], Z, Wps,
+                       wl.B, wl.H, wl.T, 64, 16, ttt.TTT_BF16, ttt.TTT_F_LN | ttt.TTT_F_W0_PER_SEQ)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(Z, Z0, rtol=0, atol=0)
+    torch.testing.assert_close(Wps, W0o, rtol=0, atol=0)
+
+
+def test_deterministic():
+    inp = synth.make_inputs(SMALL["linear_ln_150_seqs"])
+    x = to_dev(inp)
+    a = run_gpu(inp, x)
+    b = run_gpu(inp, x)
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+
+
+def test_rejects_host_and_misaligned_pointers():
+    wl = SMALL["linear_ln_small"]
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    Z = torch.empty((wl.B, wl.H, wl.T, 64), device="cuda")
+    host_q = torch.from_numpy(inp.Q_bits.view(np.int16)).view(torch.bfloat16)
+    args = lambda Q, Zp: (Q, x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"], Zp, None,
+                          wl.B, wl.H, wl.T, 64, 16, ttt.TTT_BF16, ttt.TTT_F_LN)
+    assert ttt.ttt_linear_fwd(*args(host_q, Z), check=False) == -5
+    assert ttt.ttt_linear_fwd(*args(x["Q"].data_ptr() + 2, Z), check=False) == -4
+    assert ttt.ttt_linear_fwd(*args(x["Q"], Z), check=False) == 0
+    torch.cuda.synchronize()
