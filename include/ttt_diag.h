@@ -1,0 +1,38 @@
+/*
+ * ttt_diag.h -- diagnostics of libttt.so (not part of the TTT computation).
+ *
+ * ttt_selftest_umma checks the tensor-core plumbing the TTT kernels are built
+ * on (shared-memory operand layouts, matrix and instruction descriptors,
+ * tensor-memory accumulators) by computing one small product D = A * B on the
+ * current device and writing it out, so a caller can compare it with any
+ * reference matmul.
+ */
+#ifndef TTT_DIAG_H
+#define TTT_DIAG_H
+
+#include "ttt.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Operand layouts in shared memory. */
+#define TTT_DIAG_KMAJOR_SW128 0  /* rows of 64 K-elements, 128-byte swizzle */
+#define TTT_DIAG_MNMAJOR_SW128 1 /* rows of 64 M/N-elements, 128-byte swizzle */
+#define TTT_DIAG_KMAJOR_NONE 2   /* 8x8 core matrices, no swizzle */
+
+/*
+ * D[M][N] (fp32, row-major) = A[M][K] * B[K][N] (bf16, row-major), with A
+ * and B staged in the given layouts and one 1-CTA tcgen05 MMA chain over K.
+ * Supported: M in {64, 128}; N a multiple of 16 in [16, 256] (multiple of 8
+ * for M = 64); K a multiple of 16 in [16, 128]. Device pointers; enqueued on
+ * `stream`. Returns TTT_ERR_SHAPE / TTT_ERR_ARG for unsupported values.
+ */
+TTT_API ttt_status ttt_selftest_umma(int M, int N, int K, int a_layout, int b_layout,
+                                     const void *A, const void *B, float *D, ttt_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_DIAG_H */

@@ -60,14 +60,19 @@ def lib() -> ctypes.CDLL:
         L.ttt_device_status.argtypes = [_P]
         L.ttt_launch_count.restype = ctypes.c_ulonglong
         L.ttt_launch_count.argtypes = []
+        L.ttt_selftest_umma.restype = _I
+        L.ttt_selftest_umma.argtypes = [_I] * 5 + [_P, _P, _P, _P]
         _lib = L
     return _lib
 
 
 def header_symbols() -> list[str]:
-    """Names of the functions include/ttt.h declares."""
-    text = open(HEADER_PATH).read()
-    return re.findall(r"TTT_API\s+[\w\s\*]*?\b(ttt_\w+)\s*\(", text)
+    """Names of the functions the public headers (include/*.h) declare."""
+    import glob
+    names = []
+    for path in sorted(glob.glob(os.path.join(os.path.dirname(HEADER_PATH), "*.h"))):
+        names += re.findall(r"TTT_API\s+[\w\s\*]*?\b(ttt_\w+)\s*\(", open(path).read())
+    return names
 
 
 def _ptr(x):
@@ -137,6 +142,13 @@ def ttt_device_status(stream=None) -> int:
 
 def ttt_launch_count() -> int:
     return int(lib().ttt_launch_count())
+
+
+def ttt_selftest_umma(M, N, K, a_layout, b_layout, A, B, D, stream=None, check=True):
+    """Diagnostic (include/ttt_diag.h): D = A @ B through one tcgen05 MMA chain."""
+    rc = lib().ttt_selftest_umma(M, N, K, a_layout, b_layout, _ptr(A), _ptr(B), _ptr(D),
+                                 _stream(stream))
+    return _check("ttt_selftest_umma", rc) if check else rc
 
 
 # ----------------------------------------------------------------- conveniences

@@ -1,0 +1,225 @@
+// sm100.cuh -- thin inline-PTX layer for the Blackwell (sm_100a) features
+// used by the tensor-core kernels: shared-memory mbarriers with bounded waits,
+// tensor memory (TMEM) allocation / load, tcgen05.mma with shared-memory
+// matrix descriptors, and the canonical operand layouts those descriptors
+// describe. Written from the PTX ISA's description of tcgen05.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace ttt {
+namespace sm100 {
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ----------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+// Makes initialised mbarriers visible to the async proxy (tensor core, TMA).
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Upper bound of any single wait on an on-chip barrier. A correct kernel
+// waits microseconds; running out means a protocol bug, and the kernel then
+// records it and unwinds instead of hanging the GPU.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Waits for phase `parity` of the mbarrier to complete. On timeout sets
+// *abort (shared flag seen by the whole block), records `code` in the
+// device status word and returns false. Returns false at once if another
+// thread already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          int *status, int code) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(a, parity)) return true;
+        if ((i & 63u) == 0) {
+            if (*abort) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort = 1;
+                if (status) atomicExch(status, code);
+                return false;
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------- fences
+
+// Generic-proxy writes to shared memory -> visible to the async proxy (MMA).
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// ----------------------------------------------------------------- TMEM
+
+// Warp-collective: allocates `ncols` (power of two >= 32) TMEM columns and
+// writes the base address to *dst (shared memory).
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// TMEM address of (lane, column) relative to an allocation base.
+__device__ __forceinline__ uint32_t taddr(uint32_t base, uint32_t lane, uint32_t col) {
+    return base + (lane << 16) + col;
+}
+
+// Warp-collective 32-lane x 32-bit load, 16 consecutive columns: thread i
+// receives columns col..col+15 of lane (base lane + i). The warp may only
+// address the 32 lanes of its own subpartition (warp id % 4).
+__device__ __forceinline__ void tmem_ld16(uint32_t ta, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(ta));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ----------------------------------------------------------------- MMA
+
+// Shared-memory matrix descriptor (tcgen05 "matrix descriptor"):
+// start address, leading- and stride-dimension byte offsets (16-byte units),
+// descriptor version 1, swizzle mode.
+enum Swizzle : uint32_t { kSwNone = 0, kSw128 = 2, kSw64 = 4, kSw32 = 6 };
+
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo_bytes,
+                                               uint32_t sbo_bytes, Swizzle sw) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;  // version 1 (Blackwell)
+    d |= (uint64_t)sw << 61;
+    return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulator.
+// a_mn / b_mn: operand stored MN-major (transposed) instead of K-major.
+__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4)                      // D format f32
+           | (1u << 7)                    // A format bf16
+           | (1u << 10)                   // B format bf16
+           | ((a_mn ? 1u : 0u) << 15)     // A major
+           | ((b_mn ? 1u : 0u) << 16)     // B major
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]; issued by one thread.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// Arrive once on the mbarrier when every MMA issued so far by this thread has
+// completed.
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// ----------------------------------------------------------------- layouts
+// Byte offsets of element (row, col) of a bf16 operand tile in the canonical
+// shared-memory layouts the descriptors above describe. "K-major" tiles are
+// indexed (mn, k); "MN-major" tiles are indexed (k, mn), the contiguous index
+// last. Tile bases must be 1024-byte aligned for the 128-byte swizzle.
+
+// 128-byte swizzle, K-major: 8-row x 128-byte atoms (64 bf16 of K per row);
+// atoms stacked along MN every 1024 bytes; for K > 64 the next 64 columns
+// start after all MN rows (mn_rows * 128 bytes). SBO = 1024.
+__host__ __device__ __forceinline__ uint32_t off_kmajor_sw128(uint32_t mn, uint32_t k,
+                                                              uint32_t mn_rows) {
+    const uint32_t kb = k >> 6, kk = k & 63;
+    return kb * mn_rows * 128u + (mn >> 3) * 1024u + (mn & 7) * 128u +
+           ((((kk * 2) >> 4) ^ (mn & 7)) << 4) + (kk & 7) * 2;
+}
+
+// 128-byte swizzle, MN-major: 8-row (K) x 128-byte (64 MN elements) atoms;
+// 8-row groups along K every 1024 bytes (SBO); for MN > 64 the next 64 columns
+// start after all K rows (k_rows * 128 bytes = LBO).
+__host__ __device__ __forceinline__ uint32_t off_mnmajor_sw128(uint32_t k, uint32_t mn,
+                                                               uint32_t k_rows) {
+    const uint32_t mb = mn >> 6, mm = mn & 63;
+    return mb * k_rows * 128u + (k >> 3) * 1024u + (k & 7) * 128u +
+           ((((mm * 2) >> 4) ^ (k & 7)) << 4) + (mm & 7) * 2;
+}
+
+// No swizzle, K-major ("interleaved"): 8x8 core matrices of 16-byte rows;
+// the two 8-column halves of a 16-wide K step are LBO = 128 bytes apart and
+// 8-row groups are SBO = k_cols * 16 bytes apart.
+__host__ __device__ __forceinline__ uint32_t off_kmajor_none(uint32_t mn, uint32_t k,
+                                                             uint32_t k_cols) {
+    return (mn >> 3) * (k_cols * 16u) + (k >> 3) * 128u + (mn & 7) * 16u + (k & 7) * 2;
+}
+
+// Split an fp32 value into two bf16 whose sum carries ~16 significant bits:
+// hi = RN(x), lo = RN(x - hi).
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
+    hi = __float2bfloat16_rn(x);
+    lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
+}  // namespace sm100
+}  // namespace ttt

@@ -1,0 +1,131 @@
+// ttt_selftest.cu -- ttt_selftest_umma: one small tcgen05 product with
+// operands staged in a chosen canonical shared-memory layout, to check the
+// layouts and descriptors the TTT kernels use against a reference matmul.
+#include "../../include/ttt_diag.h"
+#include "sm100.cuh"
+#include "ttt_common.cuh"
+
+namespace ttt {
+namespace {
+
+using namespace sm100;
+
+struct SelftestArgs {
+    int M, N, K, a_layout, b_layout;
+    const __nv_bfloat16 *A, *B;
+    float *D;
+    int *status;
+};
+
+// Bytes a (mn_rows x k_rows) operand occupies in `layout`: the 128-byte
+// swizzle pads the contiguous dimension to whole 128-byte rows.
+__host__ __device__ uint32_t operand_bytes(int layout, uint32_t mn_rows, uint32_t k_rows) {
+    if (layout == TTT_DIAG_KMAJOR_SW128) return mn_rows * 128u * ((k_rows + 63) / 64);
+    if (layout == TTT_DIAG_MNMAJOR_SW128) return k_rows * 128u * ((mn_rows + 63) / 64);
+    return mn_rows * k_rows * 2u;
+}
+
+__device__ uint32_t operand_offset(int layout, uint32_t mn, uint32_t k, uint32_t mn_rows,
+                                   uint32_t k_rows) {
+    if (layout == TTT_DIAG_KMAJOR_SW128) return off_kmajor_sw128(mn, k, mn_rows);
+    if (layout == TTT_DIAG_MNMAJOR_SW128) return off_mnmajor_sw128(k, mn, k_rows);
+    return off_kmajor_none(mn, k, k_rows);
+}
+
+// Descriptor of K step s (16 elements) of an operand tile at `base`.
+__device__ uint64_t operand_desc(int layout, uint32_t base, int s, uint32_t mn_rows,
+                                 uint32_t k_rows) {
+    const uint32_t k0 = 16u * s;
+    if (layout == TTT_DIAG_KMAJOR_SW128)
+        return make_sdesc(base + (k0 >> 6) * mn_rows * 128u + (k0 & 63) * 2, 16, 1024, kSw128);
+    if (layout == TTT_DIAG_MNMAJOR_SW128)
+        return make_sdesc(base + (k0 >> 3) * 1024u, k_rows * 128u, 1024, kSw128);
+    return make_sdesc(base + (k0 >> 3) * 128u, 128, k_rows * 16u, kSwNone);
+}
+
+__global__ void __launch_bounds__(128) selftest_kernel(SelftestArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int M = a.M, N = a.N, K = a.K;
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + ((operand_bytes(a.a_layout, M, K) + 1023) & ~1023u);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t ncols = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(&tmem_base, ncols);
+    for (int e = threadIdx.x; e < M * K; e += blockDim.x) {
+        const int m = e / K, k = e % K;
+        *reinterpret_cast<__nv_bfloat16 *>(sA + operand_offset(a.a_layout, m, k, M, K)) = a.A[e];
+    }
+    for (int e = threadIdx.x; e < K * N; e += blockDim.x) {
+        const int k = e / N, n = e % N;
+        *reinterpret_cast<__nv_bfloat16 *>(sB + operand_offset(a.b_layout, n, k, N, K)) = a.B[e];
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_base;
+    if (threadIdx.x == 0) {
+        const uint32_t idesc = make_idesc_bf16(M, N, a.a_layout == TTT_DIAG_MNMAJOR_SW128,
+                                               a.b_layout == TTT_DIAG_MNMAJOR_SW128);
+        for (int s = 0; s < K / 16; ++s)
+            mma_bf16(tbase, operand_desc(a.a_layout, smem_u32(sA), s, M, K),
+                     operand_desc(a.b_layout, smem_u32(sB), s, N, K), idesc, s > 0);
+        mma_commit(&bar);
+    }
+    const bool ok = mbar_wait(&bar, 0, &abort_flag, a.status, 1);
+    tc_fence_after();
+    if (ok) {
+        // M = 128: row r lives in lane r. M = 64: row 16w + i lives in lane 32w + i.
+        const int row = (M == 128) ? 32 * warp + lane : 16 * warp + lane;
+        const bool valid = (M == 128) || lane < 16;
+        for (int c0 = 0; c0 < N; c0 += 16) {
+            float v[16];
+            tmem_ld16(taddr(tbase, 32 * warp, c0), v);
+            tmem_ld_wait();
+            if (valid)
+                for (int i = 0; i < 16; ++i) a.D[(size_t)row * N + c0 + i] = v[i];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, ncols);
+}
+
+}  // namespace
+}  // namespace ttt
+
+extern "C" ttt_status ttt_selftest_umma(int M, int N, int K, int a_layout, int b_layout,
+                                        const void *A, const void *B, float *D,
+                                        ttt_stream stream) {
+    using namespace ttt;
+    if (M != 64 && M != 128) return TTT_ERR_SHAPE;
+    if (N < 16 || N > 256 || N % (M == 64 ? 8 : 16) != 0 || N % 16 != 0) return TTT_ERR_SHAPE;
+    if (K < 16 || K > 128 || K % 16 != 0) return TTT_ERR_SHAPE;
+    if (a_layout < 0 || a_layout > 2 || b_layout < 0 || b_layout > 2) return TTT_ERR_ARG;
+    if ((a_layout == TTT_DIAG_MNMAJOR_SW128 && M % 64) || (b_layout == TTT_DIAG_MNMAJOR_SW128 && N % 64))
+        return TTT_ERR_SHAPE;
+    if (!A || !B || !D) return TTT_ERR_PTR;
+    SelftestArgs a{M, N, K, a_layout, b_layout, static_cast<const __nv_bfloat16 *>(A),
+                   static_cast<const __nv_bfloat16 *>(B), D, device_status_word()};
+    const size_t smem = 1024 + ((operand_bytes(a_layout, M, K) + 1023) & ~1023u) +
+                        operand_bytes(b_layout, N, K);
+    cudaError_t e = cudaFuncSetAttribute(selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return TTT_ERR_LAUNCH;
+    selftest_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return TTT_ERR_LAUNCH;
+    count_launch();
+    return TTT_OK;
+}
