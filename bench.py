@@ -65,12 +65,6 @@ def algo_flops_per_token(wl) -> float:
     return 6 * d * d
 
 
-def bound_of(wl, peaks) -> str:
-    ai = algo_flops_per_token(wl) / algo_bytes_per_token(wl)
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    return "tensor" if ai > ridge else "hbm"
-
-
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -81,17 +75,23 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-# Kernel that dominates each workload's step, the source file it is built from,
-# and the arithmetic type it computes in.
-KERNELS = {
-    "linear": ("linear_simt_kernel", "ttt_simt.cu", "f32"),
-    "mlp": ("mlp_simt_kernel", "ttt_simt.cu", "f32"),
-    "chunk": ("chunk_simt_kernel", "ttt_simt.cu", "f32"),
-}
-
-
-def kernel_of(wl):
-    return KERNELS[wl.kind]
+def kernel_plan(wl):
+    """Kernels one library call launches, in launch order:
+    (name, source file, arithmetic type, algorithmic bytes/token, FLOPs/token)."""
+    e = 2 if wl.dtype == "bf16" else 4
+    d = wl.d
+    if wl.kind == "chunk" and wl.dtype == "bf16" and d == 128 and wl.b % 128 == 0:
+        return [
+            # K, V and eta in; A_c | B_c = K^T [eta K | eta V]
+            ("chunk_gram_kernel", "ttt_chunk_tc.cu", "bf16", 2 * d * e + 4, 4 * d * d),
+            # W_{c+1} = W_c - A_c W_c + B_c: d^3 per chunk; W0 in, W_out out
+            ("chunk_scan_kernel", "ttt_chunk_tc.cu", "f32", 8 * d * d / wl.T, 2 * d ** 3 / wl.b),
+            # Q in, Z (fp32) out; Z = Q W_c
+            ("chunk_apply_kernel", "ttt_chunk_tc.cu", "bf16", d * e + 4 * d, 2 * d * d),
+        ]
+    name = {"linear": "linear_simt_kernel", "mlp": "mlp_simt_kernel",
+            "chunk": "chunk_simt_kernel"}[wl.kind]
+    return [(name, "ttt_simt.cu", "f32", algo_bytes_per_token(wl), algo_flops_per_token(wl))]
 
 
 def source_sha(fname: str) -> str:
@@ -246,6 +246,8 @@ def gpu_arm(args, wl, rank, world):
         if world > 1:
             dist.barrier(device_ids=[dev.index])
 
+    plan = kernel_plan(wl)
+    multi = len(plan) > 1
     sampler = ClockSampler(dev)
     sampler.start()
     with torch.cuda.stream(stream):
@@ -257,6 +259,10 @@ def gpu_arm(args, wl, rank, world):
             raise RuntimeError("device status error after warm-up")
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        kern_tot = [0.0] * len(plan)
+        if multi:
+            # the library records events between its own launches on `stream`
+            ttt.ttt_diag_kernel_timing(True)
         barrier()
         torch.cuda.synchronize()
         n0 = ttt.ttt_launch_count()
@@ -266,12 +272,19 @@ def gpu_arm(args, wl, rank, world):
             starts[k].record(stream)
             call()
             ends[k].record(stream)
+            if multi:
+                for i, ms in enumerate(ttt.ttt_diag_kernel_times(len(plan))):
+                    kern_tot[i] += ms
         torch.cuda.synchronize()
         t1 = time.perf_counter()
         launches = ttt.ttt_launch_count() - n0
+        if multi:
+            ttt.ttt_diag_kernel_timing(False)
         barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sum(step_ms)
+    if not multi:
+        kern_tot = [total_ms]
 
     # e2e through the C ABI with host buffers: pinned host -> device inputs,
     # the call, device -> pinned host outputs, every step.
@@ -314,24 +327,29 @@ def gpu_arm(args, wl, rank, world):
     tokens = wl.tokens * world
     ms_per_step = total_ms / args.steps
     value = tokens * args.steps / (total_ms / 1e3)
-    kname, ksrc, kdtype = kernel_of(wl)
-    per_call = max(1, launches // (args.steps * world))
-    # The step is a single kernel launch, so the dominant kernel's average
-    # launch duration is the per-step event time.
-    kern_ms = ms_per_step if per_call == 1 else None
-    bound = bound_of(wl, peaks)
+    # The dominant kernel: largest share of the timed device time. Its average
+    # launch duration comes from CUDA events on the launching stream (the
+    # step's own events when the call is one kernel).
+    dom = max(range(len(plan)), key=lambda i: kern_tot[i])
+    kname, ksrc, kdtype, kbytes, kflops = plan[dom]
+    kern_ms = kern_tot[dom] / args.steps
+    ai = kflops / kbytes
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    bound = "tensor" if ai > ridge else "hbm"
     if bound == "hbm":
-        per_launch = algo_bytes_per_token(wl) * wl.tokens
-        achieved = per_launch / (kern_ms / 1e3) / 1e9 if kern_ms else None
+        per_launch = kbytes * wl.tokens
+        achieved = per_launch / (kern_ms / 1e3) / 1e9
         peak, unit = peaks["hbm_gbs"], "GB/s"
     else:
-        per_launch = algo_flops_per_token(wl) * wl.tokens
-        achieved = per_launch / (kern_ms / 1e3) / 1e12 if kern_ms else None
+        per_launch = kflops * wl.tokens
+        achieved = per_launch / (kern_ms / 1e3) / 1e12
         peak, unit = peaks["bf16_tflops"], "TFLOP/s"
     tflops = algo_flops_per_token(wl) * wl.tokens / (ms_per_step / 1e3) / 1e12
     sha = source_sha(ksrc)
     traffic = recorded_traffic(kname, wl.name, sha)
     clocks = sampler.summary(t0, t1)
+    kernels = [{"name": p[0], "ms_per_launch": kern_tot[i] / args.steps,
+                "share": kern_tot[i] / max(sum(kern_tot), 1e-12)} for i, p in enumerate(plan)]
     line = {
         "metric": METRIC,
         "value": value,
@@ -354,7 +372,8 @@ def gpu_arm(args, wl, rank, world):
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                      "kernel": kname, "peak_source": peaks_src,
-                     "algorithmic_per_launch": per_launch},
+                     "algorithmic_per_launch": per_launch, "kernel_ms": kern_ms},
+        "kernels": kernels,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,

@@ -143,10 +143,15 @@ TTT_API ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, cons
  * f(k) = k W (no LayerNorm). With eta_s = 1/chunk this is one step of
  * gradient descent on the chunk's mean loss.
  * Arguments as ttt_linear_fwd without LayerNorm; `chunk` is the chunk length.
- * workspace: device scratch of at least ttt_chunk_workspace_bytes(...) bytes,
- *   256-byte aligned, owned by the caller; its contents on entry do not
- *   matter and are clobbered. Calls that share a workspace must not overlap.
- * Supported: d = 128 and chunk % 128 == 0 with TTT_BF16; T % chunk == 0.
+ * workspace: device scratch of at least ttt_chunk_workspace_bytes(...) bytes
+ *   (192 KiB per chunk of every sequence when d = 128; 0 for the shapes that
+ *   need none, when workspace may be NULL), 256-byte aligned, owned by the
+ *   caller; its contents on entry do not matter and are clobbered. Calls that
+ *   share a workspace must not overlap on the GPU.
+ * Supported: T % chunk == 0, chunk % 128 == 0; d = 128 with TTT_BF16 runs
+ *   on the tensor cores (three launches: per-chunk Gram products, the
+ *   sequential affine scan over chunks, and the read-out), d in {64, 128}
+ *   with TTT_FP32, and d = 64, run the fp32 CUDA-core kernel.
  * flags: only TTT_F_W0_PER_SEQ.
  */
 TTT_API size_t ttt_chunk_workspace_bytes(int B, int H, int T, int d, int chunk);

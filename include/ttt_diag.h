@@ -31,6 +31,19 @@ extern "C" {
 TTT_API ttt_status ttt_selftest_umma(int M, int N, int K, int a_layout, int b_layout,
                                      const void *A, const void *B, float *D, ttt_stream stream);
 
+/*
+ * Per-kernel timing of the library's own launches. While enabled, every
+ * entry point records a CUDA event on its stream before its first kernel and
+ * after each kernel it launches (events are created on first use on the
+ * current device; enabling costs nothing on the device beyond the event
+ * records). ttt_diag_kernel_times synchronises on the last event of the most
+ * recent call and writes the durations (ms) of that call's kernels, in launch
+ * order, to ms[0..max); it returns how many kernels the call launched, or a
+ * negative ttt_status. Not thread-safe; meant for benchmarks.
+ */
+TTT_API ttt_status ttt_diag_kernel_timing(int enable);
+TTT_API int ttt_diag_kernel_times(float *ms, int max);
+
 #ifdef __cplusplus
 }
 #endif

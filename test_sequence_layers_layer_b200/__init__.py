@@ -60,6 +60,10 @@ def lib() -> ctypes.CDLL:
         L.ttt_device_status.argtypes = [_P]
         L.ttt_launch_count.restype = ctypes.c_ulonglong
         L.ttt_launch_count.argtypes = []
+        L.ttt_diag_kernel_timing.restype = _I
+        L.ttt_diag_kernel_timing.argtypes = [_I]
+        L.ttt_diag_kernel_times.restype = _I
+        L.ttt_diag_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_float), _I]
         L.ttt_selftest_umma.restype = _I
         L.ttt_selftest_umma.argtypes = [_I] * 5 + [_P, _P, _P, _P]
         _lib = L
@@ -142,6 +146,19 @@ def ttt_device_status(stream=None) -> int:
 
 def ttt_launch_count() -> int:
     return int(lib().ttt_launch_count())
+
+
+def ttt_diag_kernel_timing(enable: bool) -> int:
+    return lib().ttt_diag_kernel_timing(int(bool(enable)))
+
+
+def ttt_diag_kernel_times(max_kernels: int = 8) -> list[float]:
+    """Durations (ms) of the kernels of the most recent call (diagnostic)."""
+    buf = (ctypes.c_float * max_kernels)()
+    n = lib().ttt_diag_kernel_times(buf, max_kernels)
+    if n < 0:
+        raise TTTError("ttt_diag_kernel_times", n)
+    return [buf[i] for i in range(min(n, max_kernels))]
 
 
 def ttt_selftest_umma(M, N, K, a_layout, b_layout, A, B, D, stream=None, check=True):

@@ -6,7 +6,10 @@
 
 #include <atomic>
 
+#include <cuda.h>
+
 #include "../../include/ttt.h"
+#include "../../include/ttt_diag.h"
 #include "ttt_common.cuh"
 
 namespace ttt {
@@ -16,11 +19,68 @@ __device__ int g_device_status;  // set by a kernel whose bounded wait ran out
 static std::atomic<unsigned long long> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
+// Optional per-kernel event timing (diagnostic, see ttt_diag.h).
+namespace {
+constexpr int kMaxMarks = 9;
+bool g_timing = false;
+int g_timing_dev = -1;
+cudaEvent_t g_marks[kMaxMarks];
+int g_nmarks = 0;
+
+void record_mark(cudaStream_t s) {
+    if (!g_timing || g_nmarks >= kMaxMarks) return;
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (dev != g_timing_dev) {
+        if (g_timing_dev >= 0) return;  // events belong to another device
+        for (int i = 0; i < kMaxMarks; ++i) cudaEventCreate(&g_marks[i]);
+        g_timing_dev = dev;
+    }
+    cudaEventRecord(g_marks[g_nmarks++], s);
+}
+}  // namespace
+
+void timing_begin(cudaStream_t s) {
+    g_nmarks = 0;
+    record_mark(s);
+}
+
+void count_launch(cudaStream_t s) {
+    count_launch(1);
+    record_mark(s);
+}
+
 int *device_status_word() {
     int *p = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_device_status) != cudaSuccess)
         return nullptr;
     return p;
+}
+
+bool encode_tmap_bf16_2d(void *map, const void *base, uint64_t cols, uint64_t rows,
+                         uint32_t box_cols, uint32_t box_rows) {
+    using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !p)
+            return false;
+        fn = reinterpret_cast<EncodeFn>(p);
+    }
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(static_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 namespace {
@@ -114,6 +174,7 @@ ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const flo
 
     LinearArgs a{Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                  dt == TTT_BF16, ln, (flags & TTT_F_W0_PER_SEQ) != 0};
+    timing_begin(static_cast<cudaStream_t>(stream));
     return launched(launch_linear_simt(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -142,12 +203,13 @@ ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float 
 
     MlpArgs a{Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out,
               B, H, T, d, dh, b, dt == TTT_BF16, per_seq};
+    timing_begin(static_cast<cudaStream_t>(stream));
     return launched(launch_mlp_simt(a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t ttt_chunk_workspace_bytes(int B, int H, int T, int d, int chunk) {
-    (void)B; (void)H; (void)T; (void)d; (void)chunk;
-    return 0;
+    if (B <= 0 || H <= 0 || T <= 0 || chunk <= 0 || T % chunk) return 0;
+    return chunk_tc_supported(d, chunk, true) ? chunk_tc_workspace_bytes(B, H, T, d, chunk) : 0;
 }
 
 ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, const float *eta,
@@ -164,7 +226,8 @@ ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, const floa
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Z) || !aligned16(W0) ||
         (W_out && !aligned16(W_out)))
         return TTT_ERR_ALIGN;
-    const size_t need = ttt_chunk_workspace_bytes(B, H, T, d, chunk);
+    const bool tc = chunk_tc_supported(d, chunk, dt == TTT_BF16);
+    const size_t need = tc ? ttt_chunk_workspace_bytes(B, H, T, d, chunk) : 0;
     if (need && (!workspace || workspace_bytes < need ||
                  (reinterpret_cast<uintptr_t>(workspace) & 255u)))
         return TTT_ERR_WORKSPACE;
@@ -177,7 +240,9 @@ ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, const floa
 
     ChunkArgs a{Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, dt == TTT_BF16,
                 (flags & TTT_F_W0_PER_SEQ) != 0, workspace, workspace_bytes};
-    return launched(launch_chunk_simt(a, static_cast<cudaStream_t>(stream)));
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    return launched(tc ? launch_chunk_tc(a, cs) : launch_chunk_simt(a, cs));
 }
 
 ttt_status ttt_device_status(ttt_stream stream) {
@@ -195,5 +260,21 @@ ttt_status ttt_device_status(ttt_stream stream) {
 }
 
 unsigned long long ttt_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+ttt_status ttt_diag_kernel_timing(int enable) {
+    g_timing = enable != 0;
+    g_nmarks = 0;
+    return TTT_OK;
+}
+
+int ttt_diag_kernel_times(float *ms, int max) {
+    if (!g_timing || g_nmarks < 1) return 0;
+    if (cudaEventSynchronize(g_marks[g_nmarks - 1]) != cudaSuccess) return TTT_ERR_LAUNCH;
+    const int n = g_nmarks - 1;
+    for (int i = 0; i < n && i < max; ++i)
+        if (cudaEventElapsedTime(&ms[i], g_marks[i], g_marks[i + 1]) != cudaSuccess)
+            return TTT_ERR_LAUNCH;
+    return n;
+}
 
 }  // extern "C"

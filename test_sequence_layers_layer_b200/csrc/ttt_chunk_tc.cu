@@ -1,0 +1,397 @@
+// ttt_chunk_tc.cu -- large-chunk TTT (apply-then-update) on the tensor cores.
+//
+// Method ("Test-Time Training Done Right", abstract: large chunks; the chunk
+// rule itself is the TTT update of "Test-Time Training: Linear Complexity
+// Beyond Attention", Key Architectural Mechanics part 2): every token of
+// chunk c reads out with W_c, then
+//   W_{c+1} = W_c - sum_{s in c} eta_s k_s^T (k_s W_c - v_s)
+//           = W_c - A_c W_c + B_c,   A_c = K_c^T diag(eta) K_c,  B_c = K_c^T diag(eta) V_c.
+// The update is affine in W, so the work splits into three launches:
+//   1. gram:  A_c | B_c for every chunk of every sequence at once (the only
+//             pass over K and V; tcgen05, M = d_in = 128, N = 256, K = tokens);
+//   2. scan:  W_{c+1} = W_c - A_c W_c + B_c, 16 steps per sequence in fp32;
+//   3. apply: Z_c = Q_c W_c for every chunk at once (the only pass over Q and
+//             the only write of Z; tcgen05, M = 128 tokens, N = d_out, K = d_in).
+// Q/K/V tiles arrive by TMA with the 128-byte swizzle; accumulators live in
+// tensor memory. W_c enters the apply products as two bf16 terms (hi + lo)
+// so the read-out keeps ~16 significant bits of the fp32 state.
+#include "sm100.cuh"
+#include "ttt_common.cuh"
+
+namespace ttt {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: math/epilogue
+
+// ---------------------------------------------------------------------------
+// 1. gram: A_c | B_c = K_c^T [diag(eta) K_c | diag(eta) V_c]
+constexpr int kGramRows = 64;                    // tokens per pipeline stage
+constexpr int kGramStages = 4;
+constexpr int kGramStageBytes = 3 * 16384;       // K raw | eta*K | V (scaled in place)
+constexpr size_t kGramSmem = 1024 + kGramStages * kGramStageBytes;
+
+struct GramArgs {
+    const float *eta;
+    float *AB;  // [chunks][128][256] fp32
+    int chunk;
+    int *status;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_gram_kernel(const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, GramArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[kGramStages], conv[kGramStages], empty[kGramStages], done, drain;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = blockIdx.x;
+    const long row0 = (long)g * a.chunk;  // first token row of this chunk in [B*H*T][d]
+    const int nst = a.chunk / kGramRows;
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < kGramStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&conv[s], 128);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&done, 1);
+        mbar_init(&drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&tmem_base, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_base;
+    int issued = 0;
+
+    if (warp == 0 && lane == 0) {
+        // TMA producer: K rows and V rows of each stage, two 64-column boxes each.
+        for (int r = 0; r < nst; ++r) {
+            const int s = r % kGramStages;
+            if (r >= kGramStages &&
+                !mbar_wait(&empty[s], ((r / kGramStages) - 1) & 1, &abort_flag, a.status, 11))
+                break;
+            uint8_t *st = smem + s * kGramStageBytes;
+            const int y = (int)(row0 + (long)r * kGramRows);
+            mbar_arrive_expect_tx(&full[s], 32768);
+            tma_load_2d(st, &tmK, 0, y, &full[s]);
+            tma_load_2d(st + 8192, &tmK, 64, y, &full[s]);
+            tma_load_2d(st + 32768, &tmV, 0, y, &full[s]);
+            tma_load_2d(st + 40960, &tmV, 64, y, &full[s]);
+            issued = r + 1;
+        }
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer: D[d_in][0:128) += K^T (eta K), D[d_in][128:256) += K^T (eta V).
+        const uint32_t idesc = make_idesc_bf16(128, 256, true, true);
+        for (int r = 0; r < nst; ++r) {
+            const int s = r % kGramStages;
+            if (!mbar_wait(&conv[s], (r / kGramStages) & 1, &abort_flag, a.status, 12)) break;
+            tc_fence_after();
+            const uint32_t ab = smem_u32(smem + s * kGramStageBytes);
+#pragma unroll
+            for (int k = 0; k < kGramRows / 16; ++k) {
+                const uint64_t ad = make_sdesc(ab + k * 2048, 8192, 1024, kSw128);
+                const uint64_t bd = make_sdesc(ab + 16384 + k * 2048, 8192, 1024, kSw128);
+                mma_bf16(tm, ad, bd, idesc, (r | k) != 0);
+            }
+            mma_commit(&empty[s]);
+        }
+        mma_commit(&done);
+    } else if (warp >= 2) {
+        // Scale rows by eta: eta*K into its own buffer (K raw stays the A
+        // operand), V in place. Swizzling permutes 16-byte chunks inside a
+        // 128-byte row only, so a chunk's row (token) is offset / 128.
+        const int c = threadIdx.x - 64;
+        for (int r = 0; r < nst; ++r) {
+            const int s = r % kGramStages;
+            if (!mbar_wait(&full[s], (r / kGramStages) & 1, &abort_flag, a.status, 13)) break;
+            uint8_t *st = smem + s * kGramStageBytes;
+            for (int q = c; q < 2048; q += 128) {
+                const int region = q >> 10;
+                const int o = (q & 1023) * 16;
+                const int row = (o & 8191) >> 7;
+                const float e = a.eta[row0 + (long)r * kGramRows + row];
+                const uint4 v = *reinterpret_cast<const uint4 *>(st + (region ? 32768 : 0) + o);
+                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+                uint4 out;
+                __nv_bfloat162 *ho = reinterpret_cast<__nv_bfloat162 *>(&out);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(h[i]);
+                    ho[i] = __floats2bfloat162_rn(f.x * e, f.y * e);
+                }
+                *reinterpret_cast<uint4 *>(st + (region ? 32768 : 16384) + o) = out;
+            }
+            fence_async_smem();
+            mbar_arrive(&conv[s]);
+        }
+        // Epilogue: lanes are d_in rows; write A_c | B_c rows (1 KB each).
+        // (__all_sync reconverges the warp for the warp-collective TMEM loads.)
+        if (__all_sync(0xffffffffu, mbar_wait(&done, 0, &abort_flag, a.status, 14))) {
+            tc_fence_after();
+            const int sp = warp & 3;
+            const int row = 32 * sp + lane;
+            float *dst = a.AB + ((size_t)g * kD + row) * 256;
+            for (int q = 0; q < 16; ++q) {
+                float v[16];
+                tmem_ld16(taddr(tm, 32 * sp, 16 * q), v);
+                tmem_ld_wait();
+                float4 *d4 = reinterpret_cast<float4 *>(dst + 16 * q);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+        }
+    }
+    // Teardown: after an abort, let this block's own copies and MMAs land
+    // before the shared memory and tensor memory are released.
+    if (abort_flag) {
+        if (warp == 0 && lane == 0)
+            for (int r = issued - kGramStages < 0 ? 0 : issued - kGramStages; r < issued; ++r)
+                mbar_drain(&full[r % kGramStages], (r / kGramStages) & 1);
+        if (warp == 1 && lane == 0) {
+            mma_commit(&drain);
+            mbar_drain(&drain, 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tm, 256);
+}
+
+// ---------------------------------------------------------------------------
+// 2. scan: W_{c+1} = W_c - A_c W_c + B_c, one block per (sequence, 16 columns).
+struct ScanArgs {
+    const float *AB, *W0;
+    float *Wc, *W_out;  // Wc: [chunks][128][128] = the weight each chunk reads out with
+    int H, chunks_per_seq;
+    bool w0_per_seq;
+};
+
+__global__ void __launch_bounds__(256) chunk_scan_kernel(ScanArgs a) {
+    __shared__ __align__(16) float sW[kD][16];
+    const int seq = blockIdx.x, j0 = 16 * blockIdx.y;
+    const int i = threadIdx.x >> 1, jh = 8 * (threadIdx.x & 1);
+    const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? seq : seq % a.H) * kD * kD;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sW[i][jh + j] = W0[i * kD + j0 + jh + j];
+    __syncthreads();
+    for (int c = 0; c < a.chunks_per_seq; ++c) {
+        const size_t g = (size_t)seq * a.chunks_per_seq + c;
+        float acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            acc[j] = sW[i][jh + j];
+            a.Wc[g * kD * kD + (size_t)i * kD + j0 + jh + j] = acc[j];
+        }
+        const float *Ar = a.AB + (g * kD + i) * 256;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] += Ar[128 + j0 + jh + j];
+        for (int k = 0; k < kD; k += 4) {
+            const float4 av = *reinterpret_cast<const float4 *>(Ar + k);
+            const float ak[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = fmaf(-ak[kk], sW[k + kk][jh + j], acc[j]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sW[i][jh + j] = acc[j];
+        __syncthreads();
+    }
+    if (a.W_out)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a.W_out[(size_t)seq * kD * kD + i * kD + j0 + jh + j] = sW[i][jh + j];
+}
+
+// ---------------------------------------------------------------------------
+// 3. apply: Z_c = Q_c (W_c,hi + W_c,lo), one block per chunk, 128-token tiles.
+constexpr int kApplyRows = 128;
+constexpr int kApplyStages = 3;
+constexpr size_t kApplySmem = 1024 + 65536 + kApplyStages * 32768;
+
+struct ApplyArgs {
+    const float *Wc;
+    float *Z;
+    int chunk;
+    int *status;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_apply_kernel(const __grid_constant__ CUtensorMap tmQ, ApplyArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sW = smem;               // hi [0, 32K), lo [32K, 64K): MN-major, d_in rows
+    uint8_t *sQ = smem + 65536;       // stages of 128 tokens x 128 d (two 64-column boxes)
+    __shared__ uint64_t full[kApplyStages], empty[kApplyStages], tfull[2], tempty[2], wready, drain;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = blockIdx.x;
+    const long row0 = (long)g * a.chunk;
+    const int ntile = a.chunk / kApplyRows;
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < kApplyStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 128);
+        }
+        mbar_init(&wready, 128);
+        mbar_init(&drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&tmem_base, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_base;
+    int issued = 0;
+
+    if (warp == 0 && lane == 0) {
+        for (int t = 0; t < ntile; ++t) {
+            const int s = t % kApplyStages;
+            if (t >= kApplyStages &&
+                !mbar_wait(&empty[s], ((t / kApplyStages) - 1) & 1, &abort_flag, a.status, 21))
+                break;
+            uint8_t *st = sQ + s * 32768;
+            const int y = (int)(row0 + (long)t * kApplyRows);
+            mbar_arrive_expect_tx(&full[s], 32768);
+            tma_load_2d(st, &tmQ, 0, y, &full[s]);
+            tma_load_2d(st + 16384, &tmQ, 64, y, &full[s]);
+            issued = t + 1;
+        }
+    } else if (warp == 1 && lane == 0) {
+        const uint32_t idesc = make_idesc_bf16(128, 128, false, true);
+        const uint32_t wb = smem_u32(sW);
+        if (mbar_wait(&wready, 0, &abort_flag, a.status, 22)) {
+            for (int t = 0; t < ntile; ++t) {
+                const int s = t % kApplyStages, acc = t & 1;
+                if (!mbar_wait(&full[s], (t / kApplyStages) & 1, &abort_flag, a.status, 23)) break;
+                if (t >= 2 && !mbar_wait(&tempty[acc], ((t >> 1) - 1) & 1, &abort_flag, a.status, 24))
+                    break;
+                tc_fence_after();
+                const uint32_t qb = smem_u32(sQ + s * 32768);
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k) {
+                    const int k0 = 16 * k;
+                    const uint64_t ad = make_sdesc(qb + (k0 >> 6) * 16384 + (k0 & 63) * 2, 16, 1024, kSw128);
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const uint64_t bd = make_sdesc(wb + p * 32768 + (k0 >> 3) * 1024, 16384, 1024, kSw128);
+                        mma_bf16(tm + acc * 128, ad, bd, idesc, (k | p) != 0);
+                    }
+                }
+                mma_commit(&empty[s]);
+                mma_commit(&tfull[acc]);
+            }
+        }
+    } else if (warp >= 2) {
+        // Stage W_c as bf16 hi/lo, MN-major (rows d_in, columns d_out contiguous).
+        const int c = threadIdx.x - 64;
+        const float *W = a.Wc + (size_t)g * kD * kD;
+        for (int e = c; e < kD * kD; e += 128) {
+            const int i = e >> 7, j = e & 127;
+            __nv_bfloat16 hi, lo;
+            split_bf16(W[e], hi, lo);
+            const uint32_t off = off_mnmajor_sw128(i, j, kD);
+            *reinterpret_cast<__nv_bfloat16 *>(sW + off) = hi;
+            *reinterpret_cast<__nv_bfloat16 *>(sW + 32768 + off) = lo;
+        }
+        fence_async_smem();
+        mbar_arrive(&wready);
+        // Epilogue: lane = token row of the tile; 128 fp32 columns per row.
+        const int sp = warp & 3;
+        for (int t = 0; t < ntile; ++t) {
+            const int acc = t & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (t >> 1) & 1, &abort_flag, a.status, 25)))
+                break;
+            tc_fence_after();
+            float *zrow = a.Z + ((size_t)(row0 + (long)t * kApplyRows) + 32 * sp + lane) * kD;
+#pragma unroll
+            for (int q = 0; q < kD / 16; ++q) {
+                float v[16];
+                tmem_ld16(taddr(tm, 32 * sp, acc * 128 + 16 * q), v);
+                tmem_ld_wait();
+                float4 *d4 = reinterpret_cast<float4 *>(zrow + 16 * q);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+        }
+    }
+    if (abort_flag) {
+        if (warp == 0 && lane == 0)
+            for (int t = issued - kApplyStages < 0 ? 0 : issued - kApplyStages; t < issued; ++t)
+                mbar_drain(&full[t % kApplyStages], (t / kApplyStages) & 1);
+        if (warp == 1 && lane == 0) {
+            mma_commit(&drain);
+            mbar_drain(&drain, 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tm, 256);
+}
+
+}  // namespace
+
+bool chunk_tc_supported(int d, int chunk, bool bf16) {
+    return bf16 && d == kD && chunk >= kApplyRows && chunk % kApplyRows == 0;
+}
+
+size_t chunk_tc_workspace_bytes(int B, int H, int T, int d, int chunk) {
+    if (d != kD || chunk <= 0 || T % chunk) return 0;
+    const size_t n = (size_t)B * H * (T / chunk);
+    return n * (kD * 256 + kD * kD) * sizeof(float);
+}
+
+cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
+    const int cps = a.T / a.chunk;
+    const int n = a.B * a.H * cps;
+    float *AB = static_cast<float *>(a.workspace);
+    float *Wc = AB + (size_t)n * kD * 256;
+    const uint64_t rows = (uint64_t)a.B * a.H * a.T;
+    alignas(64) CUtensorMap tmK, tmV, tmQ;
+    if (!encode_tmap_bf16_2d(&tmK, a.K, kD, rows, 64, kGramRows) ||
+        !encode_tmap_bf16_2d(&tmV, a.V, kD, rows, 64, kGramRows) ||
+        !encode_tmap_bf16_2d(&tmQ, a.Q, kD, rows, 64, kApplyRows))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(chunk_gram_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGramSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kApplySmem);
+    if (e != cudaSuccess) return e;
+    int *status = device_status_word();
+    chunk_gram_kernel<<<n, kThreads, kGramSmem, s>>>(tmK, tmV, GramArgs{a.eta, AB, a.chunk, status});
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launch(s);
+    chunk_scan_kernel<<<dim3(a.B * a.H, kD / 16), 256, 0, s>>>(
+        ScanArgs{AB, a.W0, Wc, a.W_out, a.H, cps, a.w0_per_seq});
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launch(s);
+    chunk_apply_kernel<<<n, kThreads, kApplySmem, s>>>(tmQ, ApplyArgs{Wc, a.Z, a.chunk, status});
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launch(s);
+    return cudaSuccess;
+}
+
+}  // namespace ttt

@@ -43,9 +43,24 @@ cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s);
 cudaError_t launch_mlp_simt(const MlpArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
 
+// Large-chunk tensor-core path (bf16, d = 128, chunk % 128 == 0).
+bool chunk_tc_supported(int d, int chunk, bool bf16);
+size_t chunk_tc_workspace_bytes(int B, int H, int T, int d, int chunk);
+cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
+
+// Encodes a 2-D bf16 TMA descriptor (CUtensorMap, 128 bytes) over a
+// row-major [rows][cols] tensor with a box of box_rows x box_cols elements and
+// the 128-byte swizzle. Returns false if the driver rejects it.
+bool encode_tmap_bf16_2d(void *map, const void *base, uint64_t cols, uint64_t rows,
+                         uint32_t box_cols, uint32_t box_rows);
+
 // Host-side count of kernel launches (ttt_launch_count); launchers call
-// count_launch() after each successful launch.
+// count_launch() after each successful launch. With per-kernel timing
+// enabled (ttt_diag_kernel_timing) it also records an event on `s` after the
+// launch; entry points call timing_begin(s) before their first launch.
 void count_launch(int n = 1);
+void count_launch(cudaStream_t s);
+void timing_begin(cudaStream_t s);
 
 // Device-side status word (bounded waits that ran out set it). Defined in
 // ttt_api.cu; kernels get its address as an argument.

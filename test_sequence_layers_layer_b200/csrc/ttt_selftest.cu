@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(128) selftest_kernel(SelftestArgs a) {
                      operand_desc(a.b_layout, smem_u32(sB), s, N, K), idesc, s > 0);
         mma_commit(&bar);
     }
-    const bool ok = mbar_wait(&bar, 0, &abort_flag, a.status, 1);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar, 0, &abort_flag, a.status, 1));
     tc_fence_after();
     if (ok) {
         // M = 128: row r lives in lane r. M = 64: row 16w + i lives in lane 32w + i.
@@ -126,6 +126,6 @@ extern "C" ttt_status ttt_selftest_umma(int M, int N, int K, int a_layout, int b
     selftest_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return TTT_ERR_LAUNCH;
-    count_launch();
+    count_launch(1);
     return TTT_OK;
 }

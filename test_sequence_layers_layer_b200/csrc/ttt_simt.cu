@@ -365,7 +365,7 @@ cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     linear_simt_kernel<<<a.B * a.H, kThreads, smem, s>>>(a);
     e = cudaGetLastError();
-    if (e == cudaSuccess) count_launch();
+    if (e == cudaSuccess) count_launch(s);
     return e;
 }
 
@@ -380,7 +380,7 @@ cudaError_t launch_mlp_simt(const MlpArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     mlp_simt_kernel<<<a.B * a.H, kThreads, smem, s>>>(a);
     e = cudaGetLastError();
-    if (e == cudaSuccess) count_launch();
+    if (e == cudaSuccess) count_launch(s);
     return e;
 }
 
@@ -390,7 +390,7 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     chunk_simt_kernel<<<a.B * a.H, kThreads, smem, s>>>(a);
     e = cudaGetLastError();
-    if (e == cudaSuccess) count_launch();
+    if (e == cudaSuccess) count_launch(s);
     return e;
 }
 

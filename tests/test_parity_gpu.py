@@ -43,6 +43,16 @@ SMALL = {
     "chunk_two_chunks": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=1, H=2, T=4096),
     "chunk_d64": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=2, H=1, T=512, d=64, b=128,
                                                           eta="const:0.0078125"),
+    "chunk_c128": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=2, H=2, T=512, b=128,
+                                                           eta="const:0.0078125"),
+    "chunk_single_chunk": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=1, H=5, T=256, b=256,
+                                                                   eta="const:0.00390625"),
+    "chunk_150_chunks": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=10, H=15, T=128, b=128,
+                                                                 eta="const:0.0078125"),
+    "chunk_eta_varied": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=1, H=2, T=1024, b=512,
+                                                                 eta="sigmoid_over_d"),
+    "chunk_fp32": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=1, H=2, T=512, b=256,
+                                                           dtype="fp32", eta="const:0.00390625"),
 }
 
 
@@ -138,4 +148,36 @@ def test_rejects_host_and_misaligned_pointers():
     assert ttt.ttt_linear_fwd(*args(host_q, Z), check=False) == -5
     assert ttt.ttt_linear_fwd(*args(x["Q"].data_ptr() + 2, Z), check=False) == -4
     assert ttt.ttt_linear_fwd(*args(x["Q"], Z), check=False) == 0
+    torch.cuda.synchronize()
+
+
+def test_chunk_resume_split_equals_whole():
+    wl = SMALL["chunk_c128"]
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    Zw, Ww = ttt.chunk_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], chunk=wl.b)
+    h = wl.T // 2
+    sl = lambda t: t[:, :, :h].contiguous()
+    sr = lambda t: t[:, :, h:].contiguous()
+    Z1, W1 = ttt.chunk_fwd(sl(x["Q"]), sl(x["K"]), sl(x["V"]), sl(x["eta"]), x["W1"], chunk=wl.b)
+    Z2, W2 = ttt.chunk_fwd(sr(x["Q"]), sr(x["K"]), sr(x["V"]), sr(x["eta"]), W1, chunk=wl.b,
+                           w0_per_seq=True)
+    torch.cuda.synchronize()
+    assert max_rel_err(torch.cat([Z1, Z2], 2).cpu().numpy(), Zw.cpu().numpy(), wl) <= 1e-6
+    assert max_rel_err(W2.cpu().numpy(), Ww.cpu().numpy(), wl) <= 1e-6
+
+
+def test_chunk_rejects_small_workspace():
+    wl = SMALL["chunk_c128"]
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    Z = torch.empty((wl.B, wl.H, wl.T, wl.d), device="cuda")
+    need = ttt.ttt_chunk_workspace_bytes(wl.B, wl.H, wl.T, wl.d, wl.b)
+    assert need == wl.B * wl.H * (wl.T // wl.b) * 192 * 1024
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    args = (x["Q"], x["K"], x["V"], x["eta"], x["W1"], Z, None, wl.B, wl.H, wl.T, wl.d, wl.b,
+            ttt.TTT_BF16, 0)
+    assert ttt.ttt_chunk_fwd(*args, ws, need - 256, check=False) == -9
+    assert ttt.ttt_chunk_fwd(*args, None, need, check=False) == -9
+    assert ttt.ttt_chunk_fwd(*args, ws, need, check=False) == 0
     torch.cuda.synchronize()
