@@ -174,8 +174,10 @@ ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const flo
 
     LinearArgs a{Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                  dt == TTT_BF16, ln, (flags & TTT_F_W0_PER_SEQ) != 0};
-    timing_begin(static_cast<cudaStream_t>(stream));
-    return launched(launch_linear_simt(a, static_cast<cudaStream_t>(stream)));
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    return launched(linear_tc_supported(d, b, dt == TTT_BF16) ? launch_linear_tc(a, cs)
+                                                                : launch_linear_simt(a, cs));
 }
 
 ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float *eta,

@@ -43,6 +43,10 @@ cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s);
 cudaError_t launch_mlp_simt(const MlpArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
 
+// TTT-Linear tensor-core scan (bf16, d = 64, b = 16).
+bool linear_tc_supported(int d, int b, bool bf16);
+cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s);
+
 // Large-chunk tensor-core path (bf16, d = 128, chunk % 128 == 0).
 bool chunk_tc_supported(int d, int chunk, bool bf16);
 size_t chunk_tc_workspace_bytes(int B, int H, int T, int d, int chunk);
