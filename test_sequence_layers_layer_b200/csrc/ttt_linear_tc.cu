@@ -28,6 +28,20 @@
 #include "sm100.cuh"
 #include "ttt_common.cuh"
 
+// Optional pipeline trace: compiled in only when TTT_TRACE is defined (a
+// profiling build); records SM clock stamps of block 0 at each hand-off.
+#ifdef TTT_TRACE
+__device__ long long g_ttt_trace[32 * 256];
+#define TRACE(ev, i)                                                                   \
+    do {                                                                               \
+        if (blockIdx.x == 0 && (i) < 256) g_ttt_trace[(ev) * 256 + (i)] = clock64(); \
+    } while (0)
+#else
+#define TRACE(ev, i) \
+    do {             \
+    } while (0)
+#endif
+
 namespace ttt {
 namespace {
 
@@ -221,6 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int j = 0; ok && j < NM; ++j) {
                 if (!mbar_wait(&gready[j & 3], (j >> 2) & 1, abrt, status, 34)) break;
+                TRACE(0, j);
                 tc_fence_after();
                 // W_{j+1} = W_j + K_j^T (-G_j)
                 const uint32_t krow = mb_row(sK, j);
@@ -230,9 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                              make_sdesc(gb + (j & 1) * 4096 + p * 2048, 2048, 1024, kSw128), I_UPD,
                              true);
                 mma_commit(&wdone);
+                TRACE(1, j);
                 if (j % kMbPerChunk == kMbPerChunk - 1) mma_commit(&tfree[(j / kMbPerChunk) % kSlots]);
                 if (j + 1 >= NM) break;
                 if (!mbar_wait(&wsm, (j + 1) & 1, abrt, status, 35)) break;
+                TRACE(2, j);
                 tc_fence_after();
                 if (j + 2 < NM) {
                     const int m = j + 2;
@@ -244,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     issue_pw(tm + TM_P + (m & 1) * 64, mb_row(sK, m));                    // P_{j+2}
                     issue_gram(tm + TM_C + (m & 1) * 16, mb_row(sK, m), mb_row(sK, m - 1));  // C_{j+2}
                     mma_commit(&pcdone);
+                    TRACE(3, j);
                 }
                 const int m = j + 1;
                 if (m >= 2 && !mbar_wait(&zfree[m & 1], ((m >> 1) - 1) & 1, abrt, status, 37)) break;
@@ -251,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 issue_pw(tm + TM_Z + (m & 1) * 64, mb_row(sQ, m));                     // Q_m W_m
                 issue_gram(tm + TM_S + (m & 1) * 16, mb_row(sQ, m), mb_row(sK, m));    // Q_m K_m^T
                 mma_commit(&zsdone[m & 1]);
+                TRACE(4, j);
             }
         }
     } else if (warp >= 4 && warp < 8) {
@@ -271,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait_warp(&tfull[c % kSlots], (c / kSlots) & 1, abrt, status, 41)) break;
             }
             if (!mbar_wait_warp(&pcready[j & 1], (j >> 1) & 1, abrt, status, 42)) break;
+            if (threadIdx.x == 128) TRACE(5, j);
             float x[8];
             {
                 const float4 *p4 = reinterpret_cast<const float4 *>(Pf + ((j & 1) * 16 + t) * 68 + 8 * g);
@@ -332,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4 *>(sG + (j & 1) * 4096 + 2048 + off) = lo;
             fence_async_smem();
             mbar_arrive(&gready[j & 3]);
+            if (threadIdx.x == 128) TRACE(6, j);
         }
     } else if (warp >= 8 && warp < 12) {
         // ------------------------------------------------------------ W re-emit
@@ -420,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int j = 0; ok && j < NM; ++j) {
             if (!mbar_wait_warp(&wdone, j & 1, abrt, status, 52)) break;
+            if (lane == 0) TRACE(7 + q, j);
             tc_fence_after();
             float w[64];
             load_w(w);
@@ -427,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 emit(w);
                 tc_fence_before();
                 mbar_arrive(&wsm);
+                if (lane == 0) TRACE(11 + q, j);
             } else if (a.W_out && live) {
                 float *dst = a.W_out + (size_t)seq * kD * kD + row * kD;
 #pragma unroll
@@ -435,8 +458,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (warp == 8 && j + 2 < NM) {
                 if (!mbar_wait_warp(&pcdone, (j + 1) & 1, abrt, status, 53)) break;
+                if (lane == 0) TRACE(15, j);
                 tc_fence_after();
                 copy_pc(j + 2, true);
+                if (lane == 0) TRACE(16, j);
             }
         }
     } else if (warp >= 12) {
@@ -482,7 +507,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (named_bar_or(1, 128, bad || *abrt != 0)) break;
+            if (threadIdx.x == 384) TRACE(17, m);
             bad = !mbar_wait_warp(&gready[m & 3], (m >> 2) & 1, abrt, status, 63);
+            if (threadIdx.x == 384) TRACE(18, m);
             if (!bad) {
                 float zp[8];
                 {
@@ -520,6 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (m % kMbPerChunk == kMbPerChunk - 1) mbar_arrive(&tfree[(m / kMbPerChunk) % kSlots]);
             }
             if (named_bar_or(1, 128, bad)) break;
+            if (threadIdx.x == 384) TRACE(19, m);
         }
     }
     // ---------------------------------------------------------------- teardown
@@ -560,3 +588,12 @@ cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s) {
 }
 
 }  // namespace ttt
+
+#ifdef TTT_TRACE
+extern "C" __attribute__((visibility("default"))) int ttt_trace_fetch(long long *host, int n) {
+    return cudaMemcpyFromSymbol(host, g_ttt_trace, sizeof(long long) * (n < 32 * 256 ? n : 32 * 256)) ==
+                   cudaSuccess
+               ? 0
+               : -1;
+}
+#endif
