@@ -70,7 +70,8 @@ typedef enum {
     TTT_ERR_LAUNCH = -6,         /* the CUDA launch failed (see cudaGetLastError) */
     TTT_ERR_DEVICE_TIMEOUT = -7, /* a bounded on-chip wait ran out (device status) */
     TTT_ERR_UNSUPPORTED_ARCH = -8, /* current device is not sm_100              */
-    TTT_ERR_WORKSPACE = -9       /* workspace NULL, misaligned or too small     */
+    TTT_ERR_WORKSPACE = -9,      /* workspace NULL, misaligned or too small     */
+    TTT_ERR_SCRATCH_LIMIT = -10  /* needs more scratch than the library's static buffer */
 } ttt_status;
 
 typedef enum { TTT_BF16 = 0, TTT_FP32 = 1 } ttt_dtype; /* element type of Q, K, V */
@@ -160,6 +161,36 @@ TTT_API ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, co
                          const float *W0, float *Z, float *W_out, int B, int H, int T, int d,
                          int chunk, ttt_dtype dt, unsigned flags, void *workspace,
                          size_t workspace_bytes, ttt_stream stream);
+
+/*
+ * Allocation-free ttt_chunk_fwd. The TTT pages have no counterpart to this
+ * call; it exists for callers that cannot allocate device memory themselves,
+ * for example a plugin running inside a host application whose own caching
+ * allocator owns the whole GPU, or a serving loop that must not trigger the
+ * implicit synchronisation of a device allocation. It computes exactly what
+ * ttt_chunk_fwd computes (same kernels), but its scratch is a buffer of
+ * TTT_CHUNK_NOALLOC_SCRATCH_BYTES that the library declares statically: every
+ * GPU that loads libttt.so holds that buffer until the process exits, and no
+ * call of this function allocates or frees anything.
+ *   - Limit: problems whose ttt_chunk_workspace_bytes(...) exceeds
+ *     TTT_CHUNK_NOALLOC_SCRATCH_BYTES (24 MiB: 128 chunks of d = 128) return
+ *     TTT_ERR_SCRATCH_LIMIT and launch nothing; use ttt_chunk_fwd with a
+ *     caller-allocated workspace for them.
+ *   - The first call on a device looks up the buffer's device address on
+ *     that device (once per device, with the device current); make that first
+ *     call before any stream capture on that device.
+ *   - All calls share the one buffer. Its contents persist between calls and
+ *     are fully overwritten before being read, so nothing needs clearing;
+ *     but calls whose GPU work overlaps (different streams, or different host
+ *     threads, on one device) race on it and must be serialised by the caller.
+ * Arguments, supported shapes and errors are those of ttt_chunk_fwd, without
+ * the workspace pair.
+ */
+#define TTT_CHUNK_NOALLOC_SCRATCH_BYTES (24u << 20)
+TTT_API ttt_status ttt_chunk_fwd_noalloc(const void *Q, const void *K, const void *V,
+                                         const float *eta, const float *W0, float *Z,
+                                         float *W_out, int B, int H, int T, int d, int chunk,
+                                         ttt_dtype dt, unsigned flags, ttt_stream stream);
 
 /*
  * Synchronises `stream`, then returns TTT_OK, TTT_ERR_DEVICE_TIMEOUT if a

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_chunk_workspace_bytes.argtypes = [_I] * 5
         L.ttt_chunk_fwd.restype = _I
         L.ttt_chunk_fwd.argtypes = [_P] * 7 + [_I] * 6 + [ctypes.c_uint, _P, ctypes.c_size_t, _P]
+        L.ttt_chunk_fwd_noalloc.restype = _I
+        L.ttt_chunk_fwd_noalloc.argtypes = [_P] * 7 + [_I] * 6 + [ctypes.c_uint, _P]
         L.ttt_device_status.restype = _I
         L.ttt_device_status.argtypes = [_P]
         L.ttt_launch_count.restype = ctypes.c_ulonglong
@@ -138,6 +140,15 @@ def ttt_chunk_fwd(Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, dt, flags, work
                              _ptr(W_out), B, H, T, d, chunk, dt, flags, _ptr(workspace),
                              workspace_bytes, _stream(stream))
     return _check("ttt_chunk_fwd", rc) if check else rc
+
+
+def ttt_chunk_fwd_noalloc(Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, dt, flags, stream=None,
+                          check=True):
+    """ttt_chunk_fwd with the library's static scratch instead of a workspace,
+    for callers that cannot allocate device memory (see include/ttt.h)."""
+    rc = lib().ttt_chunk_fwd_noalloc(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(Z),
+                                     _ptr(W_out), B, H, T, d, chunk, dt, flags, _stream(stream))
+    return _check("ttt_chunk_fwd_noalloc", rc) if check else rc
 
 
 def ttt_device_status(stream=None) -> int:

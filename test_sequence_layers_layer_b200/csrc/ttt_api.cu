@@ -146,6 +146,8 @@ const char *ttt_status_string(int status) {
         case TTT_ERR_DEVICE_TIMEOUT: return "a bounded on-chip wait ran out on the device";
         case TTT_ERR_UNSUPPORTED_ARCH: return "current device is not sm_100 (B200)";
         case TTT_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case TTT_ERR_SCRATCH_LIMIT:
+            return "problem needs more scratch than the library's static buffer holds";
         default: return "unknown status";
     }
 }

@@ -15,6 +15,9 @@
 // Q/K/V tiles arrive by TMA with the 128-byte swizzle; accumulators live in
 // tensor memory. W_c enters the apply products as two bf16 terms (hi + lo)
 // so the read-out keeps ~16 significant bits of the fp32 state.
+#include <mutex>
+
+#include "../../include/ttt.h"
 #include "sm100.cuh"
 #include "ttt_common.cuh"
 
@@ -395,3 +398,50 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
 }
 
 }  // namespace ttt
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point: the same three kernels, with their scratch in a
+// statically declared device buffer instead of a caller workspace.
+namespace {
+
+static __device__ __align__(256) unsigned char g_chunk_scratch[TTT_CHUNK_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_chunk_scratch on the current device, looked up once per
+// device with that device current. In host code the symbol is only a handle,
+// never an address a kernel may be given.
+void *chunk_scratch_on_current_device() {
+    static std::mutex mu;
+    static void *addr[64];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_chunk_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" ttt_status ttt_chunk_fwd_noalloc(const void *Q, const void *K, const void *V,
+                                            const float *eta, const float *W0, float *Z,
+                                            float *W_out, int B, int H, int T, int d, int chunk,
+                                            ttt_dtype dt, unsigned flags, ttt_stream stream) {
+    const size_t need = ttt_chunk_workspace_bytes(B, H, T, d, chunk);
+    if (need == 0)  // shapes that run without scratch
+        return ttt_chunk_fwd(Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, dt, flags, nullptr, 0,
+                             stream);
+    if (need > TTT_CHUNK_NOALLOC_SCRATCH_BYTES) return TTT_ERR_SCRATCH_LIMIT;
+    void *scratch = chunk_scratch_on_current_device();
+    if (!scratch) return TTT_ERR_LAUNCH;
+    return ttt_chunk_fwd(Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, dt, flags, scratch,
+                         TTT_CHUNK_NOALLOC_SCRATCH_BYTES, stream);
+}
