@@ -9,9 +9,11 @@
 // The update is affine in W, so the work splits into three launches:
 //   1. gram:  A_c | B_c for every chunk of every sequence at once (the only
 //             pass over K and V; tcgen05, M = d_in = 128, N = 256, K = tokens);
-//   2. scan:  W_{c+1} = W_c - A_c W_c + B_c, 16 steps per sequence in fp32;
+//   2. scan:  W_{c+1} = W_c - A_c W_c + B_c, 16 steps per sequence in fp32,
+//             writing each W_c as the ready-made bf16 hi/lo operand image;
 //   3. apply: Z_c = Q_c W_c for every chunk at once (the only pass over Q and
-//             the only write of Z; tcgen05, M = 128 tokens, N = d_out, K = d_in).
+//             the only write of Z; tcgen05, M = 128 tokens, N = d_out, K = d_in;
+//             W_c arrives by one bulk copy).
 // Q/K/V tiles arrive by TMA with the 128-byte swizzle; accumulators live in
 // tensor memory. W_c enters the apply products as two bf16 terms (hi + lo)
 // so the read-out keeps ~16 significant bits of the fp32 state.
@@ -31,10 +33,11 @@ constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: ma
 
 // ---------------------------------------------------------------------------
 // 1. gram: A_c | B_c = K_c^T [diag(eta) K_c | diag(eta) V_c]
-constexpr int kGramRows = 64;                    // tokens per pipeline stage
+constexpr int kGramRows = 32;                    // tokens per pipeline stage
 constexpr int kGramStages = 4;
-constexpr int kGramStageBytes = 3 * 16384;       // K raw | eta*K | V (scaled in place)
-constexpr size_t kGramSmem = 1024 + kGramStages * kGramStageBytes;
+constexpr int kGramBox = kGramRows * 128;        // one 64-column box of a stage (4 KB)
+constexpr int kGramStageBytes = 6 * kGramBox;    // K raw (2 boxes) | eta*K (2) | V scaled in place (2)
+constexpr size_t kGramSmem = 1024 + kGramStages * kGramStageBytes;  // 97 KB: two blocks per SM
 
 struct GramArgs {
     const float *eta;
@@ -43,7 +46,7 @@ struct GramArgs {
     int *status;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     chunk_gram_kernel(const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, GramArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -84,11 +87,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             uint8_t *st = smem + s * kGramStageBytes;
             const int y = (int)(row0 + (long)r * kGramRows);
-            mbar_arrive_expect_tx(&full[s], 32768);
+            mbar_arrive_expect_tx(&full[s], 4 * kGramBox);
             tma_load_2d(st, &tmK, 0, y, &full[s]);
-            tma_load_2d(st + 8192, &tmK, 64, y, &full[s]);
-            tma_load_2d(st + 32768, &tmV, 0, y, &full[s]);
-            tma_load_2d(st + 40960, &tmV, 64, y, &full[s]);
+            tma_load_2d(st + kGramBox, &tmK, 64, y, &full[s]);
+            tma_load_2d(st + 4 * kGramBox, &tmV, 0, y, &full[s]);
+            tma_load_2d(st + 5 * kGramBox, &tmV, 64, y, &full[s]);
             issued = r + 1;
         }
     } else if (warp == 1 && lane == 0) {
@@ -101,8 +104,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ab = smem_u32(smem + s * kGramStageBytes);
 #pragma unroll
             for (int k = 0; k < kGramRows / 16; ++k) {
-                const uint64_t ad = make_sdesc(ab + k * 2048, 8192, 1024, kSw128);
-                const uint64_t bd = make_sdesc(ab + 16384 + k * 2048, 8192, 1024, kSw128);
+                const uint64_t ad = make_sdesc(ab + k * 2048, kGramBox, 1024, kSw128);
+                const uint64_t bd = make_sdesc(ab + 2 * kGramBox + k * 2048, kGramBox, 1024, kSw128);
                 mma_bf16(tm, ad, bd, idesc, (r | k) != 0);
             }
             mma_commit(&empty[s]);
@@ -113,16 +116,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         // operand), V in place. Swizzling permutes 16-byte chunks inside a
         // 128-byte row only, so a chunk's row (token) is offset / 128.
         const int c = threadIdx.x - 64;
+        constexpr int kChunks = 4 * kGramBox / 16;  // 16-byte chunks of K and V per stage
         for (int r = 0; r < nst; ++r) {
             const int s = r % kGramStages;
+            // This thread's eta values for the stage, loaded before the wait.
+            float ev[kChunks / 128];
+#pragma unroll
+            for (int i = 0; i < kChunks / 128; ++i) {
+                const int q = c + 128 * i, o = (q % (kChunks / 2)) * 16;
+                ev[i] = a.eta[row0 + (long)r * kGramRows + ((o % kGramBox) >> 7)];
+            }
             if (!mbar_wait(&full[s], (r / kGramStages) & 1, &abort_flag, a.status, 13)) break;
             uint8_t *st = smem + s * kGramStageBytes;
-            for (int q = c; q < 2048; q += 128) {
-                const int region = q >> 10;
-                const int o = (q & 1023) * 16;
-                const int row = (o & 8191) >> 7;
-                const float e = a.eta[row0 + (long)r * kGramRows + row];
-                const uint4 v = *reinterpret_cast<const uint4 *>(st + (region ? 32768 : 0) + o);
+#pragma unroll
+            for (int i = 0; i < kChunks / 128; ++i) {
+                const int q = c + 128 * i;
+                const int region = q / (kChunks / 2);  // 0: K, 1: V
+                const int o = (q % (kChunks / 2)) * 16;
+                const float e = ev[i];
+                const uint4 v = *reinterpret_cast<const uint4 *>(st + (region ? 4 * kGramBox : 0) + o);
                 const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
                 uint4 out;
                 __nv_bfloat162 *ho = reinterpret_cast<__nv_bfloat162 *>(&out);
@@ -131,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float2 f = __bfloat1622float2(h[i]);
                     ho[i] = __floats2bfloat162_rn(f.x * e, f.y * e);
                 }
-                *reinterpret_cast<uint4 *>(st + (region ? 32768 : 16384) + o) = out;
+                *reinterpret_cast<uint4 *>(st + (region ? 4 * kGramBox : 2 * kGramBox) + o) = out;
             }
             fence_async_smem();
             mbar_arrive(&conv[s]);
@@ -171,71 +183,104 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------------------
 // 2. scan: W_{c+1} = W_c - A_c W_c + B_c, one block per (sequence, 16 columns).
+// A_c is staged in shared memory with coalesced loads each step; W_c is also
+// written out as the apply kernel's bf16 hi/lo operand image.
+constexpr int kScanPitch = kD + 4;  // padded A row (floats)
+constexpr size_t kScanSmem = (size_t)kD * kScanPitch * 4 + kD * 16 * 4;
+
 struct ScanArgs {
     const float *AB, *W0;
-    float *Wc, *W_out;  // Wc: [chunks][128][128] = the weight each chunk reads out with
+    uint8_t *Wimg;  // [chunks][hi 32 KB | lo 32 KB]: MN-major, 128-byte swizzle
+    float *W_out;
     int H, chunks_per_seq;
     bool w0_per_seq;
 };
 
-__global__ void __launch_bounds__(256) chunk_scan_kernel(ScanArgs a) {
-    __shared__ __align__(16) float sW[kD][16];
+__global__ void __launch_bounds__(256, 2) chunk_scan_kernel(ScanArgs a) {
+    extern __shared__ __align__(16) float scan_smem[];
+    float *sA = scan_smem;                 // [128][kScanPitch]
+    float *sW = scan_smem + kD * kScanPitch;  // [128][16]
     const int seq = blockIdx.x, j0 = 16 * blockIdx.y;
     const int i = threadIdx.x >> 1, jh = 8 * (threadIdx.x & 1);
     const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? seq : seq % a.H) * kD * kD;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) sW[i][jh + j] = W0[i * kD + j0 + jh + j];
-    __syncthreads();
+    for (int j = 0; j < 8; ++j) sW[i * 16 + jh + j] = W0[i * kD + j0 + jh + j];
     for (int c = 0; c < a.chunks_per_seq; ++c) {
         const size_t g = (size_t)seq * a.chunks_per_seq + c;
+        const float *AB = a.AB + g * kD * 256;
+        // stage A_c (columns 0..127 of the 256-wide rows), coalesced
+#pragma unroll 4
+        for (int e = threadIdx.x; e < kD * kD / 4; e += 256) {
+            const int r = e >> 5, c4 = e & 31;
+            *reinterpret_cast<float4 *>(sA + r * kScanPitch + 4 * c4) =
+                *reinterpret_cast<const float4 *>(AB + (size_t)r * 256 + 4 * c4);
+        }
+        const float4 b0 = *reinterpret_cast<const float4 *>(AB + (size_t)i * 256 + 128 + j0 + jh);
+        const float4 b1 = *reinterpret_cast<const float4 *>(AB + (size_t)i * 256 + 128 + j0 + jh + 4);
+        __syncthreads();
         float acc[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            acc[j] = sW[i][jh + j];
-            a.Wc[g * kD * kD + (size_t)i * kD + j0 + jh + j] = acc[j];
-        }
-        const float *Ar = a.AB + (g * kD + i) * 256;
+        for (int j = 0; j < 8; ++j) acc[j] = sW[i * 16 + jh + j];
+        {  // W_c as the bf16 hi/lo operand image of the apply kernel
+            uint4 hi, lo;
+            __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(&hi);
+            __nv_bfloat16 *l = reinterpret_cast<__nv_bfloat16 *>(&lo);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] += Ar[128 + j0 + jh + j];
+            for (int j = 0; j < 8; ++j) split_bf16(acc[j], h[j], l[j]);
+            uint8_t *img = a.Wimg + g * 65536;
+            const uint32_t off = off_mnmajor_sw128(i, j0 + jh, kD);
+            *reinterpret_cast<uint4 *>(img + off) = hi;
+            *reinterpret_cast<uint4 *>(img + 32768 + off) = lo;
+        }
+        acc[0] += b0.x; acc[1] += b0.y; acc[2] += b0.z; acc[3] += b0.w;
+        acc[4] += b1.x; acc[5] += b1.y; acc[6] += b1.z; acc[7] += b1.w;
+        const float *Ar = sA + i * kScanPitch;
+#pragma unroll 8
         for (int k = 0; k < kD; k += 4) {
             const float4 av = *reinterpret_cast<const float4 *>(Ar + k);
             const float ak[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[j] = fmaf(-ak[kk], sW[k + kk][jh + j], acc[j]);
+            for (int kk = 0; kk < 4; ++kk) {
+                const float4 w0 = *reinterpret_cast<const float4 *>(sW + (k + kk) * 16 + jh);
+                const float4 w1 = *reinterpret_cast<const float4 *>(sW + (k + kk) * 16 + jh + 4);
+                acc[0] = fmaf(-ak[kk], w0.x, acc[0]); acc[1] = fmaf(-ak[kk], w0.y, acc[1]);
+                acc[2] = fmaf(-ak[kk], w0.z, acc[2]); acc[3] = fmaf(-ak[kk], w0.w, acc[3]);
+                acc[4] = fmaf(-ak[kk], w1.x, acc[4]); acc[5] = fmaf(-ak[kk], w1.y, acc[5]);
+                acc[6] = fmaf(-ak[kk], w1.z, acc[6]); acc[7] = fmaf(-ak[kk], w1.w, acc[7]);
+            }
         }
         __syncthreads();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) sW[i][jh + j] = acc[j];
+        for (int j = 0; j < 8; ++j) sW[i * 16 + jh + j] = acc[j];
         __syncthreads();
     }
     if (a.W_out)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) a.W_out[(size_t)seq * kD * kD + i * kD + j0 + jh + j] = sW[i][jh + j];
+        for (int j = 0; j < 8; ++j) a.W_out[(size_t)seq * kD * kD + i * kD + j0 + jh + j] = sW[i * 16 + jh + j];
 }
 
 // ---------------------------------------------------------------------------
 // 3. apply: Z_c = Q_c (W_c,hi + W_c,lo), one block per chunk, 128-token tiles.
 constexpr int kApplyRows = 128;
 constexpr int kApplyStages = 3;
+constexpr int kApplyThreads = 320;  // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
 constexpr size_t kApplySmem = 1024 + 65536 + kApplyStages * 32768;
 
 struct ApplyArgs {
-    const float *Wc;
+    const uint8_t *Wimg;
     float *Z;
     int chunk;
     int *status;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kApplyThreads, 1)
     chunk_apply_kernel(const __grid_constant__ CUtensorMap tmQ, ApplyArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sW = smem;               // hi [0, 32K), lo [32K, 64K): MN-major, d_in rows
-    uint8_t *sQ = smem + 65536;       // stages of 128 tokens x 128 d (two 64-column boxes)
-    __shared__ uint64_t full[kApplyStages], empty[kApplyStages], tfull[2], tempty[2], wready, drain;
+    uint8_t *sW = smem;          // hi [0, 32K), lo [32K, 64K): MN-major, d_in rows
+    uint8_t *sQ = smem + 65536;  // stages of 128 tokens x 128 d (two 64-column boxes)
+    __shared__ uint64_t full[kApplyStages], empty[kApplyStages], tfull[2], tempty[2], wfull, drain;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -251,9 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 128);
+            mbar_init(&tempty[b], 256);
         }
-        mbar_init(&wready, 128);
+        mbar_init(&wfull, 1);
         mbar_init(&drain, 1);
         fence_mbar_init();
     }
@@ -263,8 +308,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tm = tmem_base;
     int issued = 0;
+    bool w_issued = false;
 
     if (warp == 0 && lane == 0) {
+        mbar_arrive_expect_tx(&wfull, 65536);
+        bulk_load(sW, a.Wimg + (size_t)g * 65536, 32768, &wfull);
+        bulk_load(sW + 32768, a.Wimg + (size_t)g * 65536 + 32768, 32768, &wfull);
+        w_issued = true;
         for (int t = 0; t < ntile; ++t) {
             const int s = t % kApplyStages;
             if (t >= kApplyStages &&
@@ -280,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1 && lane == 0) {
         const uint32_t idesc = make_idesc_bf16(128, 128, false, true);
         const uint32_t wb = smem_u32(sW);
-        if (mbar_wait(&wready, 0, &abort_flag, a.status, 22)) {
+        if (mbar_wait(&wfull, 0, &abort_flag, a.status, 22)) {
             for (int t = 0; t < ntile; ++t) {
                 const int s = t % kApplyStages, acc = t & 1;
                 if (!mbar_wait(&full[s], (t / kApplyStages) & 1, &abort_flag, a.status, 23)) break;
@@ -303,31 +353,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp >= 2) {
-        // Stage W_c as bf16 hi/lo, MN-major (rows d_in, columns d_out contiguous).
-        const int c = threadIdx.x - 64;
-        const float *W = a.Wc + (size_t)g * kD * kD;
-        for (int e = c; e < kD * kD; e += 128) {
-            const int i = e >> 7, j = e & 127;
-            __nv_bfloat16 hi, lo;
-            split_bf16(W[e], hi, lo);
-            const uint32_t off = off_mnmajor_sw128(i, j, kD);
-            *reinterpret_cast<__nv_bfloat16 *>(sW + off) = hi;
-            *reinterpret_cast<__nv_bfloat16 *>(sW + 32768 + off) = lo;
-        }
-        fence_async_smem();
-        mbar_arrive(&wready);
-        // Epilogue: lane = token row of the tile; 128 fp32 columns per row.
-        const int sp = warp & 3;
+        // Epilogue: lane = token row of the tile; each warp pair splits the
+        // 128 fp32 columns of its subpartition's 32 rows.
+        const int sp = warp & 3, half = (warp - 2) >> 2;
         for (int t = 0; t < ntile; ++t) {
             const int acc = t & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (t >> 1) & 1, &abort_flag, a.status, 25)))
                 break;
             tc_fence_after();
-            float *zrow = a.Z + ((size_t)(row0 + (long)t * kApplyRows) + 32 * sp + lane) * kD;
+            float *zrow = a.Z + ((size_t)(row0 + (long)t * kApplyRows) + 32 * sp + lane) * kD + 64 * half;
 #pragma unroll
-            for (int q = 0; q < kD / 16; ++q) {
+            for (int q = 0; q < 4; ++q) {
                 float v[16];
-                tmem_ld16(taddr(tm, 32 * sp, acc * 128 + 16 * q), v);
+                tmem_ld16(taddr(tm, 32 * sp, acc * 128 + 64 * half + 16 * q), v);
                 tmem_ld_wait();
                 float4 *d4 = reinterpret_cast<float4 *>(zrow + 16 * q);
 #pragma unroll
@@ -338,9 +376,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     if (abort_flag) {
-        if (warp == 0 && lane == 0)
+        if (warp == 0 && lane == 0) {
+            if (w_issued) mbar_drain(&wfull, 0);
             for (int t = issued - kApplyStages < 0 ? 0 : issued - kApplyStages; t < issued; ++t)
                 mbar_drain(&full[t % kApplyStages], (t / kApplyStages) & 1);
+        }
         if (warp == 1 && lane == 0) {
             mma_commit(&drain);
             mbar_drain(&drain, 0);
@@ -367,7 +407,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     const int cps = a.T / a.chunk;
     const int n = a.B * a.H * cps;
     float *AB = static_cast<float *>(a.workspace);
-    float *Wc = AB + (size_t)n * kD * 256;
+    uint8_t *Wimg = reinterpret_cast<uint8_t *>(AB + (size_t)n * kD * 256);
     const uint64_t rows = (uint64_t)a.B * a.H * a.T;
     alignas(64) CUtensorMap tmK, tmV, tmQ;
     if (!encode_tmap_bf16_2d(&tmK, a.K, kD, rows, 64, kGramRows) ||
@@ -385,12 +425,15 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
-    chunk_scan_kernel<<<dim3(a.B * a.H, kD / 16), 256, 0, s>>>(
-        ScanArgs{AB, a.W0, Wc, a.W_out, a.H, cps, a.w0_per_seq});
+    e = cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kScanSmem);
+    if (e != cudaSuccess) return e;
+    chunk_scan_kernel<<<dim3(a.B * a.H, kD / 16), 256, kScanSmem, s>>>(
+        ScanArgs{AB, a.W0, Wimg, a.W_out, a.H, cps, a.w0_per_seq});
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
-    chunk_apply_kernel<<<n, kThreads, kApplySmem, s>>>(tmQ, ApplyArgs{Wc, a.Z, a.chunk, status});
+    chunk_apply_kernel<<<n, kApplyThreads, kApplySmem, s>>>(tmQ, ApplyArgs{Wimg, a.Z, a.chunk, status});
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);

@@ -11,30 +11,43 @@
 //   Z_m     = epilogue( Q_m W_m - tril(Q_m K_m^T) G_m )
 // Only G_m -> G_{m+1} is sequential. Because
 //   X_{m+1} = K_{m+1} W_m - (K_{m+1} K_m^T) G_m = P_{m+1} - C_{m+1} G_m,
-// the tensor cores can form P_{m+1} = K_{m+1} W_m one mini-batch ahead; the
+// the tensor cores form P_{m+1} = K_{m+1} W_m one mini-batch ahead; the
 // critical chain per mini-batch is one 16x16 by 16x64 correction plus the
 // LayerNorm backward, done in fp32 on CUDA cores by the scan warps.
 //
-// Warp roles (16 warps):
-//   0      TMA producer: K, Q, V in chunks of 128 tokens (3-slot ring)
+// Per mini-batch the tensor core runs two MMA groups:
+//   update:  W^T += (-G_j)^T K_j                                   (M=64, N=64, K=16)
+//   product: [Q_{j+1}; K_{j+2}] x [W_{j+1}^T hi | W_{j+1}^T lo | K_{j+1}]^T  (M=128, N=144, K=64)
+// The product's rows give Q_{j+1} W_{j+1} (read-out), Q_{j+1} K_{j+1}^T (causal
+// term), K_{j+2} W_{j+1} (= P_{j+2}) and K_{j+2} K_{j+1}^T (= C_{j+2}) at once.
+// The fp32 state is kept as W^T so that re-emitting it as the bf16 hi/lo
+// operand writes whole 16-byte rows.
+//
+// Warp roles (20 warps):
+//   0      TMA producer: K, Q, V in chunks of 64 tokens (4-slot ring)
 //   1      MMA issuer (one thread) and tensor-memory owner
+//   2      stages the product's A tile [Q_{j+1}; K_{j+2}] from the TMA tiles
+//   3      copies the product (tensor-memory subpartition 3) out: P and C for
+//          the scan, Q W and Q K^T into a 4-slot ring for the output warps
 //   4-7    scan: X = P - C G_prev, LayerNorm backward, G (fp32 + bf16 hi/lo)
-//   8-11   W re-emit: fp32 W from tensor memory -> bf16 hi/lo operand in smem;
-//          warp 8 also copies P and C out of tensor memory for the scan
-//   12-15  output: Zpre = Q W - tril(S) G, LayerNorm + residual, store Z
+//   8-15   W re-emit: fp32 W^T from tensor memory -> bf16 hi/lo operand rows
+//   16-19  output: Zpre = Q W - tril(Q K^T) G, LayerNorm + residual, store Z
 // Precision: Q/K/V enter exactly (bf16); every other operand (W, G) enters
-// the tensor cores as two bf16 terms hi + lo, accumulation is fp32, and the
+// the tensor cores as two bf16 terms hi + lo with fp32 accumulation, and the
 // chain's corrections and all LayerNorm math are fp32.
 #include "sm100.cuh"
 #include "ttt_common.cuh"
 
 // Optional pipeline trace: compiled in only when TTT_TRACE is defined (a
-// profiling build); records SM clock stamps of block 0 at each hand-off.
+// profiling build). Block 0 records 32-bit SM clock stamps at each hand-off
+// into shared memory (so tracing adds no global-memory traffic inside the
+// pipeline) and copies them out when it exits.
+constexpr int kTraceEvents = 32, kTraceSteps = 128;
 #ifdef TTT_TRACE
-__device__ long long g_ttt_trace[32 * 256];
-#define TRACE(ev, i)                                                                   \
-    do {                                                                               \
-        if (blockIdx.x == 0 && (i) < 256) g_ttt_trace[(ev) * 256 + (i)] = clock64(); \
+__device__ unsigned g_ttt_trace[kTraceEvents * kTraceSteps];
+#define TRACE(ev, i)                                                                  \
+    do {                                                                              \
+        if ((i) >= 0 && (i) < kTraceSteps) trace_smem[(ev) * kTraceSteps + (i)] = (unsigned)clock(); \
     } while (0)
 #else
 #define TRACE(ev, i) \
@@ -48,28 +61,41 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 64, kMB = 16;
-constexpr int kChunkTok = 128, kMbPerChunk = kChunkTok / kMB, kSlots = 3;
-constexpr int kTile = kChunkTok * kD * 2;  // 16 KB per tensor per chunk
-constexpr int kThreads = 512;
+constexpr int kChunkTok = 64, kMbPerChunk = kChunkTok / kMB, kSlots = 4;
+constexpr int kTile = kChunkTok * kD * 2;  // 8 KB per tensor per chunk
+constexpr int kThreads = 640;
+constexpr int kBRows = 144;                // W^T hi (64) | W^T lo (64) | K_{j+1} (16)
 
 // Shared memory map (offsets from a 1024-aligned base).
-constexpr int OFF_K = 0;                               // K ring + 48 rows of slack
-constexpr int OFF_Q = OFF_K + kSlots * kTile + 6144;   // Q ring + slack
-constexpr int OFF_V = OFF_Q + kSlots * kTile + 6144;   // V ring
-constexpr int OFF_W = OFF_V + kSlots * kTile;          // W hi | lo (MN-major, 8 KB each)
-constexpr int OFF_G = OFF_W + 16384;                   // -G hi | lo, 2 buffers (2 KB each)
-constexpr int OFF_PF = OFF_G + 8192;                   // P fp32 [2][16][68]
-constexpr int OFF_CF = OFF_PF + 2 * 16 * 68 * 4;       // C fp32 [2][16][17]
-constexpr int OFF_GF = OFF_CF + 2 * 16 * 17 * 4;       // G fp32 [4][16][64]
-constexpr int OFF_ZQ = OFF_GF + 4 * 16 * 64 * 4;       // Q W fp32 [16][68]
-constexpr int OFF_SF = OFF_ZQ + 16 * 68 * 4;           // Q K^T fp32 [16][17]
-constexpr int kSmemBytes = OFF_SF + 16 * 17 * 4 + 1024;
-static_assert(OFF_Q % 1024 == 0 && OFF_V % 1024 == 0 && OFF_W % 1024 == 0 && OFF_G % 1024 == 0,
+constexpr int OFF_K = 0;
+constexpr int OFF_Q = OFF_K + kSlots * kTile;
+constexpr int OFF_V = OFF_Q + kSlots * kTile;
+constexpr int OFF_A = OFF_V + kSlots * kTile + 12288;  // 4 slots of 32 rows; the MMA window starts 96 rows earlier
+constexpr int OFF_B = OFF_A + 4 * 4096;
+constexpr int OFF_G = OFF_B + kBRows * 128;           // -G hi | lo (MN-major, 2 KB each), 2 buffers
+constexpr int OFF_PF = OFF_G + 8192;                  // P fp32 [2][16][64], float4-swizzled
+constexpr int kCStride = 20;                          // C rows padded to 16-byte multiples
+constexpr int OFF_CF = OFF_PF + 2 * 16 * 64 * 4;      // C fp32 [2][16][kCStride]
+constexpr int OFF_GF = OFF_CF + 2 * 16 * kCStride * 4;  // G fp32 [4][16][64]
+constexpr int OFF_ZQ = OFF_GF + 4 * 16 * 64 * 4;      // Q W fp32 [4][16][64], float4-swizzled
+constexpr int OFF_SF = OFF_ZQ + 4 * 16 * 64 * 4;      // Q K^T fp32 [4][16][kCStride]
+constexpr int OFF_ETA = OFF_SF + 4 * 16 * kCStride * 4;  // eta fp32 [kSlots][64], one row per chunk
+constexpr int OFF_TRACE = OFF_ETA + kSlots * kChunkTok * 4;
+#ifdef TTT_TRACE
+constexpr int kTraceBytes = kTraceEvents * kTraceSteps * 4;
+#else
+constexpr int kTraceBytes = 0;
+#endif
+constexpr int kSmemBytes = OFF_TRACE + kTraceBytes + 1024;
+static_assert(OFF_Q % 1024 == 0 && OFF_V % 1024 == 0 && OFF_A % 1024 == 0 && OFF_B % 1024 == 0 &&
+                  OFF_G % 1024 == 0,
               "operand tiles need 1024-byte alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// Tensor-memory columns (512 allocated; M = 64 accumulators use lanes 16w..).
-constexpr uint32_t TM_W = 0, TM_P = 64, TM_Z = 192, TM_C = 320, TM_S = 352;
+// Tensor-memory columns (512 allocated). The M = 64 W^T accumulator keeps row
+// r in lane 32 (r / 16) + r % 16; the M = 128 product keeps row r in lane r.
+constexpr uint32_t TM_WT = 0, TM_B = 64;  // W^T (64 cols); product, 2 buffers of 144 cols
+// Product rows 96-111 = Q_{j+1}, 112-127 = K_{j+2}: lanes 96-127 (subpartition 3).
 
 struct Args {
     const float *eta, *W0, *gamma, *beta;
@@ -79,16 +105,9 @@ struct Args {
     int *status;
 };
 
-__device__ __forceinline__ float sum8(float v) {
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    return v;
-}
-
 // Mean and 1/sigma of a 64-value row spread over 8 lanes (8 values each):
 // local mean and sum of squared deviations, merged pairwise across lanes
-// (equal-count merge of Chan et al.), LayerNorm eps inside the root.
+// (the equal-count case of Chan et al.'s update), LayerNorm eps inside the root.
 __device__ __forceinline__ void row_stats(const float (&x)[8], float &mu, float &rstd) {
     float m = 0.f;
 #pragma unroll
@@ -112,17 +131,54 @@ __device__ __forceinline__ void row_stats(const float (&x)[8], float &mu, float 
     rstd = rsqrtf(M2 * (1.f / kD) + kLnEps);
 }
 
-// 8 consecutive bf16 (columns 8g..8g+7) of row `row` of a 128-byte-swizzled
-// [rows][64] tile, widened to fp32.
-__device__ __forceinline__ void load_row8(const uint8_t *tile, int row, int g, float (&v)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4 *>(tile + row * 128 + ((g ^ (row & 7)) << 4));
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+// A thread (t, g) of the scan and output groups owns columns 4g..4g+3 and
+// 32+4g..32+4g+3 of token row t ("two quads"), so eight threads of a row
+// touch 128 contiguous bytes per access.
+
+// The thread's 8 bf16 of row `row` of a 128-byte-swizzled [rows][64] tile.
+__device__ __forceinline__ void load_quads_bf16(const uint8_t *tile, int row, int g,
+                                                float (&v)[8]) {
+    const uint8_t *r = tile + row * 128;
+    const int sw = row & 7;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(h[i]);
-        v[2 * i] = f.x;
-        v[2 * i + 1] = f.y;
+    for (int h = 0; h < 2; ++h) {
+        const int chunk = 4 * h + (g >> 1);
+        const uint2 u = *reinterpret_cast<const uint2 *>(r + ((chunk ^ sw) << 4) + (g & 1) * 8);
+        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+        v[4 * h] = f0.x;
+        v[4 * h + 1] = f0.y;
+        v[4 * h + 2] = f1.x;
+        v[4 * h + 3] = f1.y;
     }
+}
+
+// fp32 [16][64] staging rows written by tensor-memory readers (one row per
+// lane) and read by (t, g) threads: float4 q of row t sits at q ^ (t & 7).
+__device__ __forceinline__ int swz4(int row, int q) { return row * 16 + (q ^ (row & 7)); }
+
+__device__ __forceinline__ void load_quads_f32_swz(const float *base, int row, int g,
+                                                   float (&v)[8]) {
+    const float4 *b = reinterpret_cast<const float4 *>(base);
+    const float4 u0 = b[swz4(row, g)], u1 = b[swz4(row, 8 + g)];
+    v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+    v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+}
+
+// Two-term bf16 split of a pair: hi = x with the low 16 bits cleared (exact
+// bf16, |x - hi| < 2^-7 |x|), lo = RN_bf16(x - hi); hi + lo carries ~16
+// significant bits. Returns the packed hi pair and lo pair.
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const uint32_t ua = __float_as_uint(a) & 0xFFFF0000u, ub = __float_as_uint(b) & 0xFFFF0000u;
+    hi = __byte_perm(ua, ub, 0x7632);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - __uint_as_float(ua), b - __uint_as_float(ub));
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// Packs 4 floats to 4 bf16 hi terms and 4 bf16 lo terms (hi + lo ~ x).
+__device__ __forceinline__ void split4(float a, float b, float c, float d, uint2 &hi, uint2 &lo) {
+    split2(a, b, hi.x, lo.x);
+    split2(c, d, hi.y, lo.y);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -133,15 +189,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sK = smem + OFF_K, *sQ = smem + OFF_Q, *sV = smem + OFF_V;
-    uint8_t *sW = smem + OFF_W, *sG = smem + OFF_G;
+    uint8_t *sA = smem + OFF_A, *sB = smem + OFF_B, *sG = smem + OFF_G;
     float *Pf = reinterpret_cast<float *>(smem + OFF_PF);
     float *Cf = reinterpret_cast<float *>(smem + OFF_CF);
     float *Gf = reinterpret_cast<float *>(smem + OFF_GF);
     float *Zqf = reinterpret_cast<float *>(smem + OFF_ZQ);
     float *Sf = reinterpret_cast<float *>(smem + OFF_SF);
+    float *etas = reinterpret_cast<float *>(smem + OFF_ETA);
+#ifdef TTT_TRACE
+    volatile unsigned *trace_smem = reinterpret_cast<volatile unsigned *>(smem + OFF_TRACE);
+    for (int e = threadIdx.x; e < kTraceEvents * kTraceSteps; e += blockDim.x) trace_smem[e] = 0;
+#endif
 
-    __shared__ uint64_t tfull[kSlots], tfree[kSlots], gready[4], efree[4], pcready[2], zsdone[2],
-        zfree[2], wdone, wsm, pcdone, drain;
+    __shared__ uint64_t tfull[kSlots], tfree[kSlots], gready[4], efree[4], aready[4], afree[4],
+        zready[4], zfree[4], pzdone[2], pcready[2], wdone, wsm, drain;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -160,15 +221,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) {
             mbar_init(&gready[i], 128);
             mbar_init(&efree[i], 128);
+            mbar_init(&aready[i], 32);
+            mbar_init(&afree[i], 1);
+            mbar_init(&zready[i], 32);
+            mbar_init(&zfree[i], 128);
         }
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&pzdone[i], 1);
             mbar_init(&pcready[i], 32);
-            mbar_init(&zsdone[i], 1);
-            mbar_init(&zfree[i], 32);
         }
         mbar_init(&wdone, 1);
-        mbar_init(&wsm, 128);
-        mbar_init(&pcdone, 1);
+        mbar_init(&wsm, 256);
         mbar_init(&drain, 1);
         fence_mbar_init();
     }
@@ -179,9 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm = tmem_base;
     volatile int *abrt = &abort_flag;
 
-    // Address of mini-batch m's first row in a K or Q ring (16 rows = 2 KB).
-    auto mb_row = [&](uint8_t *ring, int m) -> uint32_t {
-        return smem_u32(ring) + ((m / kMbPerChunk) % kSlots) * kTile + (m % kMbPerChunk) * 2048;
+    // Row r of mini-batch m in a K/Q/V ring (generic pointer to its 128 bytes).
+    auto ring_row = [&](uint8_t *ring, int m, int r) -> uint8_t * {
+        return ring + ((m / kMbPerChunk) % kSlots) * kTile + ((m % kMbPerChunk) * kMB + r) * 128;
+    };
+    auto chunk_wait = [&](int m, int code) -> bool {  // warp-uniform wait for m's chunk
+        const int c = m / kMbPerChunk;
+        return mbar_wait_warp(&tfull[c % kSlots], (c / kSlots) & 1, abrt, status, code);
     };
 
     if (warp == 0) {
@@ -202,75 +269,123 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t I_UPD = make_idesc_bf16(64, 64, true, true);
-            const uint32_t I_PW = make_idesc_bf16(64, 64, false, true);
-            const uint32_t I_GRAM = make_idesc_bf16(64, 16, false, false);
-            const uint32_t wb = smem_u32(sW), gb = smem_u32(sG);
-            // D = A_window(64 rows from `arow`) * W   (W as hi + lo)
-            auto issue_pw = [&](uint32_t d, uint32_t arow) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-#pragma unroll
-                    for (int p = 0; p < 2; ++p)
-                        mma_bf16(d, make_sdesc(arow + 32 * k, 16, 1024, kSw128),
-                                 make_sdesc(wb + p * 8192 + 2048 * k, 8192, 1024, kSw128), I_PW,
-                                 (k | p) != 0);
-            };
-            // D = A_window(64 rows from `arow`) * (16 rows from `brow`)^T
-            auto issue_gram = [&](uint32_t d, uint32_t arow, uint32_t brow) {
+            const uint32_t I_PROD = make_idesc_bf16(128, kBRows, false, false);
+            const uint32_t bb = smem_u32(sB), gb = smem_u32(sG);
+            // Product i (i = -2 .. NM-2): A slot (i+2)%4, accumulator (i+2)%2.
+            auto product = [&](int i) {
+                const uint32_t arow = smem_u32(sA) + ((i + 2) & 3) * 4096 - 12288;  // 96 rows earlier
+                const uint32_t d = tm + TM_B + ((i + 2) & 1) * kBRows;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_bf16(d, make_sdesc(arow + 32 * k, 16, 1024, kSw128),
-                             make_sdesc(brow + 32 * k, 16, 1024, kSw128), I_GRAM, k != 0);
+                             make_sdesc(bb + 32 * k, 16, 1024, kSw128), I_PROD, k != 0);
+                mma_commit(&pzdone[(i + 2) & 1]);
+                mma_commit(&afree[(i + 2) & 3]);
             };
-            bool ok = mbar_wait(&tfull[0], 0, abrt, status, 32) && mbar_wait(&wsm, 0, abrt, status, 33);
+            bool ok = mbar_wait(&wsm, 0, abrt, status, 32) &&
+                      mbar_wait(&aready[0], 0, abrt, status, 33) &&
+                      mbar_wait(&aready[1], 0, abrt, status, 33);
             if (ok) {
                 tc_fence_after();
-                issue_pw(tm + TM_P, mb_row(sK, 0));                       // P_0 = K_0 W_0
-                issue_pw(tm + TM_P + 64, mb_row(sK, 1));                  // P_1 = K_1 W_0
-                issue_gram(tm + TM_C + 16, mb_row(sK, 1), mb_row(sK, 0));  // C_1 = K_1 K_0^T
-                mma_commit(&pcdone);
-                issue_pw(tm + TM_Z, mb_row(sQ, 0));                       // Q_0 W_0
-                issue_gram(tm + TM_S, mb_row(sQ, 0), mb_row(sK, 0));      // Q_0 K_0^T
-                mma_commit(&zsdone[0]);
+                product(-2);  // P_0 = K_0 W_0
+                product(-1);  // P_1, C_1, Q_0 W_0, Q_0 K_0^T
             }
             for (int j = 0; ok && j < NM; ++j) {
                 if (!mbar_wait(&gready[j & 3], (j >> 2) & 1, abrt, status, 34)) break;
                 TRACE(0, j);
                 tc_fence_after();
-                // W_{j+1} = W_j + K_j^T (-G_j)
-                const uint32_t krow = mb_row(sK, j);
+                // W_{j+1}^T = W_j^T + (-G_j)^T K_j
+                const uint32_t krow = smem_u32(ring_row(sK, j, 0));
 #pragma unroll
                 for (int p = 0; p < 2; ++p)
-                    mma_bf16(tm + TM_W, make_sdesc(krow, 8192, 1024, kSw128),
-                             make_sdesc(gb + (j & 1) * 4096 + p * 2048, 2048, 1024, kSw128), I_UPD,
-                             true);
+                    mma_bf16(tm + TM_WT, make_sdesc(gb + (j & 1) * 4096 + p * 2048, 8192, 1024, kSw128),
+                             make_sdesc(krow, 8192, 1024, kSw128), I_UPD, true);
                 mma_commit(&wdone);
                 TRACE(1, j);
                 if (j % kMbPerChunk == kMbPerChunk - 1) mma_commit(&tfree[(j / kMbPerChunk) % kSlots]);
                 if (j + 1 >= NM) break;
+                const int i = j;
                 if (!mbar_wait(&wsm, (j + 1) & 1, abrt, status, 35)) break;
                 TRACE(2, j);
+                if (!mbar_wait(&aready[(i + 2) & 3], ((i + 2) >> 2) & 1, abrt, status, 36)) break;
+                TRACE(18, j);
                 tc_fence_after();
-                if (j + 2 < NM) {
-                    const int m = j + 2;
-                    if (m % kMbPerChunk == 0) {
-                        const int c = m / kMbPerChunk;
-                        if (!mbar_wait(&tfull[c % kSlots], (c / kSlots) & 1, abrt, status, 36)) break;
-                        tc_fence_after();
-                    }
-                    issue_pw(tm + TM_P + (m & 1) * 64, mb_row(sK, m));                    // P_{j+2}
-                    issue_gram(tm + TM_C + (m & 1) * 16, mb_row(sK, m), mb_row(sK, m - 1));  // C_{j+2}
-                    mma_commit(&pcdone);
-                    TRACE(3, j);
-                }
-                const int m = j + 1;
-                if (m >= 2 && !mbar_wait(&zfree[m & 1], ((m >> 1) - 1) & 1, abrt, status, 37)) break;
-                tc_fence_after();
-                issue_pw(tm + TM_Z + (m & 1) * 64, mb_row(sQ, m));                     // Q_m W_m
-                issue_gram(tm + TM_S + (m & 1) * 16, mb_row(sQ, m), mb_row(sK, m));    // Q_m K_m^T
-                mma_commit(&zsdone[m & 1]);
-                TRACE(4, j);
+                product(i);
+                TRACE(3, j);
             }
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ A stager
+        // A_i rows 0-15 = Q_{i+1}, rows 16-31 = K_{i+2} (copies of the TMA rows;
+        // source and destination rows agree mod 8, so the swizzle carries over).
+        for (int i = -2; i <= NM - 2; ++i) {
+            const int s = (i + 2) & 3;
+            if (i + 2 >= 4 && !mbar_wait_warp(&afree[s], (((i + 2) >> 2) - 1) & 1, abrt, status, 71)) break;
+            if (i + 2 < NM && (i + 2) % kMbPerChunk == 0) {
+                // First use of a new chunk: wait for it, and stage its eta row.
+                if (!chunk_wait(i + 2, 72)) break;
+                const int c = (i + 2) / kMbPerChunk;
+                for (int e = lane; e < kChunkTok; e += 32) {
+                    const long tok = (long)c * kChunkTok + e;
+                    etas[(c % kSlots) * kChunkTok + e] = tok < T ? a.eta[tok0 + tok] : 0.f;
+                }
+            }
+            uint8_t *dst = sA + s * 4096;
+#pragma unroll
+            for (int e = lane; e < 256; e += 32) {
+                const int r = e >> 3, c = e & 7;
+                const int m = r < 16 ? i + 1 : i + 2;
+                if (m >= 0 && m < NM) {
+                    const uint8_t *src = ring_row(r < 16 ? sQ : sK, m, r & 15);
+                    *reinterpret_cast<uint4 *>(dst + r * 128 + c * 16) =
+                        *reinterpret_cast<const uint4 *>(src + c * 16);
+                }
+            }
+            fence_async_smem();
+            mbar_arrive(&aready[s]);
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ product copy-out
+        // Product i (rows 96-127 = lanes 96-127): lanes 0-15 hold Q_{i+1} rows
+        // (Q W, Q K^T -> output ring slot (i+1)%4), lanes 16-31 hold K_{i+2} rows
+        // (P, C -> scan buffer (i+2)%2).
+        const bool qrow = lane < 16;
+        const int row = lane & 15;
+        for (int i = -2; i <= NM - 2; ++i) {
+            const int mz = i + 1, mp = i + 2;
+            if (!mbar_wait_warp(&pzdone[(i + 2) & 1], ((i + 2) >> 1) & 1, abrt, status, 81)) break;
+            if (mz >= 4 && !mbar_wait_warp(&zfree[mz & 3], ((mz >> 2) - 1) & 1, abrt, status, 82)) break;
+            tc_fence_after();
+            const uint32_t col = TM_B + ((i + 2) & 1) * kBRows;
+            float *dst = qrow ? Zqf + (mz & 3) * 1024 : Pf + (mp & 1) * 1024;
+            const bool live = qrow ? mz >= 0 : mp < NM;
+            float v0[16], v1[16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {  // hi + lo, 16 columns at a time
+                tmem_ld16(taddr(tm, 96, col + 16 * c), v0);
+                tmem_ld16(taddr(tm, 96, col + 64 + 16 * c), v1);
+                tmem_ld_wait();
+                if (live) {
+                    float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        d4[swz4(row, 4 * c + q)] =
+                            make_float4(v0[4 * q] + v1[4 * q], v0[4 * q + 1] + v1[4 * q + 1],
+                                        v0[4 * q + 2] + v1[4 * q + 2], v0[4 * q + 3] + v1[4 * q + 3]);
+                }
+            }
+            tmem_ld16(taddr(tm, 96, col + 128), v0);
+            tmem_ld_wait();
+            if (live) {
+                float *g16 = qrow ? Sf + ((mz & 3) * 16 + row) * kCStride : Cf + ((mp & 1) * 16 + row) * kCStride;
+                float4 *c4 = reinterpret_cast<float4 *>(g16);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) c4[q] = make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
+            }
+            tc_fence_before();
+            if (mp < NM) mbar_arrive(&pcready[mp & 1]);
+            if (mz >= 0) mbar_arrive(&zready[mz & 3]);
+            if (lane == 0) TRACE(4, mp);
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ scan
@@ -278,46 +393,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         float gam[8], bet[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            gam[i] = a.ln ? a.gamma[head * kD + 8 * g + i] : 1.f;
-            bet[i] = a.ln ? a.beta[head * kD + 8 * g + i] : 0.f;
+            const int col = (i < 4 ? 4 * g : 28 + 4 * g) + i;
+            gam[i] = a.ln ? a.gamma[head * kD + col] : 1.f;
+            bet[i] = a.ln ? a.beta[head * kD + col] : 0.f;
         }
-        float eta_next = a.eta[tok0 + t];
         for (int j = 0; j < NM; ++j) {
-            const float eta = eta_next;
-            if (j + 1 < NM) eta_next = a.eta[tok0 + (long)(j + 1) * kMB + t];
-            if (j % kMbPerChunk == 0) {
-                const int c = j / kMbPerChunk;
-                if (!mbar_wait_warp(&tfull[c % kSlots], (c / kSlots) & 1, abrt, status, 41)) break;
-            }
+            if (j % kMbPerChunk == 0 && !chunk_wait(j, 41)) break;
             if (!mbar_wait_warp(&pcready[j & 1], (j >> 1) & 1, abrt, status, 42)) break;
             if (threadIdx.x == 128) TRACE(5, j);
             float x[8];
-            {
-                const float4 *p4 = reinterpret_cast<const float4 *>(Pf + ((j & 1) * 16 + t) * 68 + 8 * g);
-                const float4 u0 = p4[0], u1 = p4[1];
-                x[0] = u0.x; x[1] = u0.y; x[2] = u0.z; x[3] = u0.w;
-                x[4] = u1.x; x[5] = u1.y; x[6] = u1.z; x[7] = u1.w;
-            }
-            if (j > 0) {  // X_j = P_j - C_j G_{j-1}
-                const float *crow = Cf + ((j & 1) * 16 + t) * 17;
-                const float *gprev = Gf + ((j - 1) & 3) * 1024 + 8 * g;
+            load_quads_f32_swz(Pf + (j & 1) * 1024, t, g, x);
+            if (j > 0) {  // X_j = P_j - C_j G_{j-1}: coefficients in registers, two chains
+                const float4 *c4 = reinterpret_cast<const float4 *>(Cf + ((j & 1) * 16 + t) * kCStride);
+                float c[16];
 #pragma unroll
-                for (int s = 0; s < kMB; ++s) {
-                    const float c = crow[s];
-                    const float4 *g4 = reinterpret_cast<const float4 *>(gprev + s * kD);
-                    const float4 u0 = g4[0], u1 = g4[1];
-                    x[0] = fmaf(-c, u0.x, x[0]); x[1] = fmaf(-c, u0.y, x[1]);
-                    x[2] = fmaf(-c, u0.z, x[2]); x[3] = fmaf(-c, u0.w, x[3]);
-                    x[4] = fmaf(-c, u1.x, x[4]); x[5] = fmaf(-c, u1.y, x[5]);
-                    x[6] = fmaf(-c, u1.z, x[6]); x[7] = fmaf(-c, u1.w, x[7]);
+                for (int q = 0; q < 4; ++q) {
+                    const float4 u = c4[q];
+                    c[4 * q] = u.x; c[4 * q + 1] = u.y; c[4 * q + 2] = u.z; c[4 * q + 3] = u.w;
                 }
+                const float *gprev = Gf + ((j - 1) & 3) * 1024;
+                float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int s = 0; s < kMB; s += 2) {
+                    const float4 u0 = *reinterpret_cast<const float4 *>(gprev + s * kD + 4 * g);
+                    const float4 u1 = *reinterpret_cast<const float4 *>(gprev + s * kD + 32 + 4 * g);
+                    const float4 w0 = *reinterpret_cast<const float4 *>(gprev + (s + 1) * kD + 4 * g);
+                    const float4 w1 = *reinterpret_cast<const float4 *>(gprev + (s + 1) * kD + 32 + 4 * g);
+                    x[0] = fmaf(-c[s], u0.x, x[0]); x[1] = fmaf(-c[s], u0.y, x[1]);
+                    x[2] = fmaf(-c[s], u0.z, x[2]); x[3] = fmaf(-c[s], u0.w, x[3]);
+                    x[4] = fmaf(-c[s], u1.x, x[4]); x[5] = fmaf(-c[s], u1.y, x[5]);
+                    x[6] = fmaf(-c[s], u1.z, x[6]); x[7] = fmaf(-c[s], u1.w, x[7]);
+                    y[0] = fmaf(-c[s + 1], w0.x, y[0]); y[1] = fmaf(-c[s + 1], w0.y, y[1]);
+                    y[2] = fmaf(-c[s + 1], w0.z, y[2]); y[3] = fmaf(-c[s + 1], w0.w, y[3]);
+                    y[4] = fmaf(-c[s + 1], w1.x, y[4]); y[5] = fmaf(-c[s + 1], w1.y, y[5]);
+                    y[6] = fmaf(-c[s + 1], w1.z, y[6]); y[7] = fmaf(-c[s + 1], w1.w, y[7]);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] += y[i];
             }
-            const int row = (j % kMbPerChunk) * kMB + t;
-            const int slot = (j / kMbPerChunk) % kSlots;
-            float kv[8], vv[8], G[8];
-            load_row8(sV + slot * kTile, row, g, vv);
+            if (threadIdx.x == 128) TRACE(6, j);
+            // eta was staged (with the chunk) before the product that made P_j
+            const float eta = etas[((j / kMbPerChunk) % kSlots) * kChunkTok + (j % kMbPerChunk) * kMB + t];
+            float vv[8], G[8];
+            load_quads_bf16(ring_row(sV, j, 0), t, g, vv);
             if (a.ln) {
-                load_row8(sK + slot * kTile, row, g, kv);
+                float kv[8];
+                load_quads_bf16(ring_row(sK, j, 0), t, g, kv);
                 float mu, rstd;
                 row_stats(x, mu, rstd);
                 float xh[8], gh[8], s1 = 0.f, s2 = 0.f;
@@ -328,8 +449,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     s1 += gh[i];
                     s2 = fmaf(gh[i], xh[i], s2);
                 }
-                s1 = sum8(s1) * (1.f / kD);
-                s2 = sum8(s2) * (1.f / kD);
+#pragma unroll
+                for (int o = 1; o < 8; o <<= 1) {
+                    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+                    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+                }
+                s1 *= 1.f / kD;
+                s2 *= 1.f / kD;
                 const float sc = eta * rstd;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) G[i] = sc * (gh[i] - s1 - xh[i] * s2);
@@ -337,89 +463,65 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) G[i] = eta * (x[i] - vv[i]);
             }
+            if (threadIdx.x == 128) TRACE(7, j);
             if (j >= 4 && !mbar_wait_warp(&efree[j & 3], ((j >> 2) - 1) & 1, abrt, status, 43)) break;
-            float4 *gf4 = reinterpret_cast<float4 *>(Gf + (j & 3) * 1024 + t * kD + 8 * g);
-            gf4[0] = make_float4(G[0], G[1], G[2], G[3]);
-            gf4[1] = make_float4(G[4], G[5], G[6], G[7]);
-            // -G as bf16 hi + lo, MN-major rows = tokens: one 16-byte chunk each.
-            uint4 hi, lo;
-            __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(&hi);
-            __nv_bfloat16 *l = reinterpret_cast<__nv_bfloat16 *>(&lo);
+            float *gf = Gf + (j & 3) * 1024 + t * kD;
+            *reinterpret_cast<float4 *>(gf + 4 * g) = make_float4(G[0], G[1], G[2], G[3]);
+            *reinterpret_cast<float4 *>(gf + 32 + 4 * g) = make_float4(G[4], G[5], G[6], G[7]);
+            // -G as bf16 hi + lo, MN-major (rows = tokens, 128-byte swizzle)
+            uint8_t *gb = sG + (j & 1) * 4096;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) split_bf16(-G[i], h[i], l[i]);
-            const uint32_t off = off_mnmajor_sw128(t, 8 * g, kMB);
-            *reinterpret_cast<uint4 *>(sG + (j & 1) * 4096 + off) = hi;
-            *reinterpret_cast<uint4 *>(sG + (j & 1) * 4096 + 2048 + off) = lo;
+            for (int h = 0; h < 2; ++h) {
+                uint2 hi, lo;
+                split4(-G[4 * h], -G[4 * h + 1], -G[4 * h + 2], -G[4 * h + 3], hi, lo);
+                const uint32_t off = off_mnmajor_sw128(t, 32 * h + 4 * g, kMB);
+                *reinterpret_cast<uint2 *>(gb + off) = hi;
+                *reinterpret_cast<uint2 *>(gb + 2048 + off) = lo;
+            }
             fence_async_smem();
             mbar_arrive(&gready[j & 3]);
-            if (threadIdx.x == 128) TRACE(6, j);
+            if (threadIdx.x == 128) TRACE(8, j);
         }
-    } else if (warp >= 8 && warp < 12) {
+    } else if (warp >= 8 && warp < 16) {
         // ------------------------------------------------------------ W re-emit
-        const int q = warp & 3;  // subpartition: W rows 16q..16q+15 in lanes 32q..32q+15
-        const int row = 16 * q + (lane & 15);
+        const int q = warp & 3;              // subpartition: W^T rows 16q..16q+15
+        const int half = (warp - 8) >> 2;    // d_in columns 32*half .. +31
+        const int n = 16 * q + (lane & 15);  // W^T row = d_out index
         const bool live = lane < 16;
-        const uint32_t wl = taddr(tm, 32 * q, TM_W);
-        auto emit = [&](const float (&w)[64]) {
+        const int rt = threadIdx.x - 256;    // 0..255
+        const uint32_t wl = taddr(tm, 32 * q, TM_WT + 32 * half);
+        // Writes W^T row n, this half's columns, as hi (row n) and lo (row 64+n).
+        auto emit = [&](const float (&w)[32]) {
             if (live) {
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    uint4 hi, lo;
-                    __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(&hi);
-                    __nv_bfloat16 *l = reinterpret_cast<__nv_bfloat16 *>(&lo);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) split_bf16(w[8 * c8 + i], h[i], l[i]);
-                    const uint32_t off = off_mnmajor_sw128(row, 8 * c8, kD);
-                    *reinterpret_cast<uint4 *>(sW + off) = hi;
-                    *reinterpret_cast<uint4 *>(sW + 8192 + off) = lo;
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    uint2 h0, l0, h1, l1;
+                    split4(w[8 * c8], w[8 * c8 + 1], w[8 * c8 + 2], w[8 * c8 + 3], h0, l0);
+                    split4(w[8 * c8 + 4], w[8 * c8 + 5], w[8 * c8 + 6], w[8 * c8 + 7], h1, l1);
+                    const int chunk = 4 * half + c8;
+                    *reinterpret_cast<uint4 *>(sB + n * 128 + ((chunk ^ (n & 7)) << 4)) =
+                        make_uint4(h0.x, h0.y, h1.x, h1.y);
+                    *reinterpret_cast<uint4 *>(sB + (64 + n) * 128 + ((chunk ^ (n & 7)) << 4)) =
+                        make_uint4(l0.x, l0.y, l1.x, l1.y);
                 }
             }
-            fence_async_smem();
         };
-        auto load_w = [&](float (&w)[64]) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float v[16];
-                tmem_ld16(wl + 16 * c, v);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) w[16 * c + i] = v[i];
+        // Rows 128-143 of the B tile: K_m (same swizzle phase: 128 = 0 mod 8).
+        auto copy_k = [&](int m) {
+            if (rt < 128 && m < NM) {
+                const int r = rt >> 3, c = rt & 7;
+                *reinterpret_cast<uint4 *>(sB + (128 + r) * 128 + c * 16) =
+                    *reinterpret_cast<const uint4 *>(ring_row(sK, m, r) + c * 16);
             }
-            tmem_ld_wait();
         };
-        // P_m and C_m (rows 0-15 of their accumulators, lanes 0-15) -> smem.
-        auto copy_pc = [&](int m, bool with_c) {
-            float v[16];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                tmem_ld16(taddr(tm, 0, TM_P + (m & 1) * 64 + 16 * c), v);
-                tmem_ld_wait();
-                if (lane < 16) {
-                    float4 *d4 = reinterpret_cast<float4 *>(Pf + ((m & 1) * 16 + lane) * 68 + 16 * c);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                }
-            }
-            if (with_c) {
-                tmem_ld16(taddr(tm, 0, TM_C + (m & 1) * 16), v);
-                tmem_ld_wait();
-                if (lane < 16)
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) Cf[((m & 1) * 16 + lane) * 17 + i] = v[i];
-            }
-            tc_fence_before();
-            mbar_arrive(&pcready[m & 1]);
-        };
-        {  // initial weight -> tensor memory (fp32) and the bf16 operand
+        bool ok = chunk_wait(0, 51);
+        if (ok) {  // initial weight -> tensor memory (fp32, transposed) and the operand
             const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? seq : head) * kD * kD;
-            float w[64];
+            float w[32];
 #pragma unroll
-            for (int c = 0; c < 64; c += 4) {
-                const float4 u = live ? *reinterpret_cast<const float4 *>(W0 + row * kD + c)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-                w[c] = u.x; w[c + 1] = u.y; w[c + 2] = u.z; w[c + 3] = u.w;
-            }
+            for (int k = 0; k < 32; ++k) w[k] = live ? W0[(32 * half + k) * kD + n] : 0.f;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 float v[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) v[i] = w[16 * c + i];
@@ -427,127 +529,88 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_st_wait();
             emit(w);
+            copy_k(0);
+            fence_async_smem();
             tc_fence_before();
             mbar_arrive(&wsm);
         }
-        bool ok = true;
-        if (warp == 8) {
-            ok = mbar_wait_warp(&pcdone, 0, abrt, status, 51);
-            if (ok) {
-                tc_fence_after();
-                copy_pc(0, false);
-                copy_pc(1, true);
-            }
-        }
         for (int j = 0; ok && j < NM; ++j) {
             if (!mbar_wait_warp(&wdone, j & 1, abrt, status, 52)) break;
-            if (lane == 0) TRACE(7 + q, j);
+            if (lane == 0 && half == 0) TRACE(9 + q, j);
             tc_fence_after();
-            float w[64];
-            load_w(w);
+            float w[32];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                float v[16];
+                tmem_ld16(wl + 16 * c, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) w[16 * c + i] = v[i];
+            }
+            tmem_ld_wait();
+            if (lane == 0 && half == 0 && q == 0) TRACE(19, j);
             if (j + 1 < NM) {
+                if ((j + 1) % kMbPerChunk == 0 && !chunk_wait(j + 1, 53)) break;
                 emit(w);
+                copy_k(j + 1);
+                if (lane == 0 && half == 0 && q == 0) TRACE(20, j);
+                fence_async_smem();
                 tc_fence_before();
                 mbar_arrive(&wsm);
-                if (lane == 0) TRACE(11 + q, j);
+                if (lane == 0 && half == 0) TRACE(13 + q, j);
             } else if (a.W_out && live) {
-                float *dst = a.W_out + (size_t)seq * kD * kD + row * kD;
+                float *dst = a.W_out + (size_t)seq * kD * kD + n;
 #pragma unroll
-                for (int c = 0; c < 64; c += 4)
-                    *reinterpret_cast<float4 *>(dst + c) = make_float4(w[c], w[c + 1], w[c + 2], w[c + 3]);
-            }
-            if (warp == 8 && j + 2 < NM) {
-                if (!mbar_wait_warp(&pcdone, (j + 1) & 1, abrt, status, 53)) break;
-                if (lane == 0) TRACE(15, j);
-                tc_fence_after();
-                copy_pc(j + 2, true);
-                if (lane == 0) TRACE(16, j);
+                for (int k = 0; k < 32; ++k) dst[(32 * half + k) * kD] = w[k];
             }
         }
-    } else if (warp >= 12) {
+    } else {
         // ------------------------------------------------------------ output
-        const int r = threadIdx.x - 384, t = r >> 3, g = r & 7;
+        const int r = threadIdx.x - 512, t = r >> 3, g = r & 7;
         float gam[8], bet[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            gam[i] = a.ln ? a.gamma[head * kD + 8 * g + i] : 1.f;
-            bet[i] = a.ln ? a.beta[head * kD + 8 * g + i] : 0.f;
+            const int col = (i < 4 ? 4 * g : 28 + 4 * g) + i;
+            gam[i] = a.ln ? a.gamma[head * kD + col] : 1.f;
+            bet[i] = a.ln ? a.beta[head * kD + col] : 0.f;
         }
         for (int m = 0; m < NM; ++m) {
-            // Every wait below is warp-uniform, and the group of four output
-            // warps leaves the loop together (named_bar_or), so an abort can
-            // never strand part of the group at a barrier.
-            bool bad = false;
-            if (m % kMbPerChunk == 0) {
-                const int c = m / kMbPerChunk;
-                bad = !mbar_wait_warp(&tfull[c % kSlots], (c / kSlots) & 1, abrt, status, 61);
+            if (m % kMbPerChunk == 0 && !chunk_wait(m, 61)) break;
+            if (!mbar_wait_warp(&zready[m & 3], (m >> 2) & 1, abrt, status, 62)) break;
+            if (!mbar_wait_warp(&gready[m & 3], (m >> 2) & 1, abrt, status, 63)) break;
+            float zp[8];
+            load_quads_f32_swz(Zqf + (m & 3) * 1024, t, g, zp);
+            const float *gm = Gf + (m & 3) * 1024;
+            const float *srow = Sf + ((m & 3) * 16 + t) * kCStride;
+            for (int s = 0; s <= t; ++s) {  // - tril(Q K^T) G, diagonal included
+                const float c = srow[s];
+                const float4 u0 = *reinterpret_cast<const float4 *>(gm + s * kD + 4 * g);
+                const float4 u1 = *reinterpret_cast<const float4 *>(gm + s * kD + 32 + 4 * g);
+                zp[0] = fmaf(-c, u0.x, zp[0]); zp[1] = fmaf(-c, u0.y, zp[1]);
+                zp[2] = fmaf(-c, u0.z, zp[2]); zp[3] = fmaf(-c, u0.w, zp[3]);
+                zp[4] = fmaf(-c, u1.x, zp[4]); zp[5] = fmaf(-c, u1.y, zp[5]);
+                zp[6] = fmaf(-c, u1.z, zp[6]); zp[7] = fmaf(-c, u1.w, zp[7]);
             }
-            if (warp == 12 && !bad) {  // Q_m W_m and Q_m K_m^T out of tensor memory (lanes 0-15)
-                bad = !mbar_wait_warp(&zsdone[m & 1], (m >> 1) & 1, abrt, status, 62);
-                if (!bad) {
-                    tc_fence_after();
-                    float v[16];
+            float qv[8];
+            if (a.ln) load_quads_bf16(ring_row(sQ, m, 0), t, g, qv);
+            // G_m, Q W, Q K^T and the Q rows are read: release them before the
+            // global stores, so the arrivals do not wait for the stores.
+            mbar_arrive(&efree[m & 3]);
+            mbar_arrive(&zfree[m & 3]);
+            if (m % kMbPerChunk == kMbPerChunk - 1) mbar_arrive(&tfree[(m / kMbPerChunk) % kSlots]);
+            float out[8];
+            if (a.ln) {
+                float mu, rstd;
+                row_stats(zp, mu, rstd);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        tmem_ld16(taddr(tm, 0, TM_Z + (m & 1) * 64 + 16 * c), v);
-                        tmem_ld_wait();
-                        if (lane < 16) {
-                            float4 *d4 = reinterpret_cast<float4 *>(Zqf + lane * 68 + 16 * c);
+                for (int i = 0; i < 8; ++i) out[i] = qv[i] + gam[i] * ((zp[i] - mu) * rstd) + bet[i];
+            } else {
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                        }
-                    }
-                    tmem_ld16(taddr(tm, 0, TM_S + (m & 1) * 16), v);
-                    tmem_ld_wait();
-                    if (lane < 16)
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) Sf[lane * 17 + i] = v[i];
-                    tc_fence_before();
-                    mbar_arrive(&zfree[m & 1]);
-                }
+                for (int i = 0; i < 8; ++i) out[i] = zp[i];
             }
-            if (named_bar_or(1, 128, bad || *abrt != 0)) break;
-            if (threadIdx.x == 384) TRACE(17, m);
-            bad = !mbar_wait_warp(&gready[m & 3], (m >> 2) & 1, abrt, status, 63);
-            if (threadIdx.x == 384) TRACE(18, m);
-            if (!bad) {
-                float zp[8];
-                {
-                    const float4 *z4 = reinterpret_cast<const float4 *>(Zqf + t * 68 + 8 * g);
-                    const float4 u0 = z4[0], u1 = z4[1];
-                    zp[0] = u0.x; zp[1] = u0.y; zp[2] = u0.z; zp[3] = u0.w;
-                    zp[4] = u1.x; zp[5] = u1.y; zp[6] = u1.z; zp[7] = u1.w;
-                }
-                const float *gm = Gf + (m & 3) * 1024 + 8 * g;
-                for (int s = 0; s <= t; ++s) {  // - tril(Q K^T) G, diagonal included
-                    const float c = Sf[t * 17 + s];
-                    const float4 *g4 = reinterpret_cast<const float4 *>(gm + s * kD);
-                    const float4 u0 = g4[0], u1 = g4[1];
-                    zp[0] = fmaf(-c, u0.x, zp[0]); zp[1] = fmaf(-c, u0.y, zp[1]);
-                    zp[2] = fmaf(-c, u0.z, zp[2]); zp[3] = fmaf(-c, u0.w, zp[3]);
-                    zp[4] = fmaf(-c, u1.x, zp[4]); zp[5] = fmaf(-c, u1.y, zp[5]);
-                    zp[6] = fmaf(-c, u1.z, zp[6]); zp[7] = fmaf(-c, u1.w, zp[7]);
-                }
-                float out[8];
-                if (a.ln) {
-                    float qv[8];
-                    load_row8(sQ + ((m / kMbPerChunk) % kSlots) * kTile, (m % kMbPerChunk) * kMB + t, g, qv);
-                    float mu, rstd;
-                    row_stats(zp, mu, rstd);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) out[i] = qv[i] + gam[i] * ((zp[i] - mu) * rstd) + bet[i];
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) out[i] = zp[i];
-                }
-                float4 *zo = reinterpret_cast<float4 *>(a.Z + (tok0 + (long)m * kMB + t) * kD + 8 * g);
-                zo[0] = make_float4(out[0], out[1], out[2], out[3]);
-                zo[1] = make_float4(out[4], out[5], out[6], out[7]);
-                mbar_arrive(&efree[m & 3]);
-                if (m % kMbPerChunk == kMbPerChunk - 1) mbar_arrive(&tfree[(m / kMbPerChunk) % kSlots]);
-            }
-            if (named_bar_or(1, 128, bad)) break;
-            if (threadIdx.x == 384) TRACE(19, m);
+            float *zo = a.Z + (tok0 + (long)m * kMB + t) * kD;
+            *reinterpret_cast<float4 *>(zo + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
+            *reinterpret_cast<float4 *>(zo + 32 + 4 * g) = make_float4(out[4], out[5], out[6], out[7]);
+            if (threadIdx.x == 512) TRACE(17, m);
         }
     }
     // ---------------------------------------------------------------- teardown
@@ -563,6 +626,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tm, 512);
+#ifdef TTT_TRACE
+    if (blockIdx.x == 0)
+        for (int e = threadIdx.x; e < kTraceEvents * kTraceSteps; e += blockDim.x)
+            g_ttt_trace[e] = trace_smem[e];
+#endif
 }
 
 }  // namespace
@@ -590,8 +658,9 @@ cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s) {
 }  // namespace ttt
 
 #ifdef TTT_TRACE
-extern "C" __attribute__((visibility("default"))) int ttt_trace_fetch(long long *host, int n) {
-    return cudaMemcpyFromSymbol(host, g_ttt_trace, sizeof(long long) * (n < 32 * 256 ? n : 32 * 256)) ==
+extern "C" __attribute__((visibility("default"))) int ttt_trace_fetch(unsigned *host, int n) {
+    const int cap = kTraceEvents * kTraceSteps;
+    return cudaMemcpyFromSymbol(host, g_ttt_trace, sizeof(unsigned) * (n < cap ? n : cap)) ==
                    cudaSuccess
                ? 0
                : -1;
