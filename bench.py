@@ -459,10 +459,14 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--B", type=int, default=None,
+                    help="override the workload's batch size (smaller profiling cases)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = synth.WORKLOADS[args.workload]
+    if args.B:
+        wl = wl.scaled(B=args.B, name=f"{wl.name}_B{args.B}")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
 
