@@ -92,6 +92,9 @@ def kernel_plan(wl):
     if wl.kind == "linear" and wl.dtype == "bf16" and d == 64 and wl.b == 16:
         return [("linear_ln_scan_kernel", "ttt_linear_tc.cu", "bf16", algo_bytes_per_token(wl),
                  algo_flops_per_token(wl))]
+    if wl.kind == "mlp" and wl.dtype == "bf16" and d == 64 and wl.dh == 256 and wl.b == 16:
+        return [("mlp_ln_scan_kernel", "ttt_mlp_tc.cu", "bf16", algo_bytes_per_token(wl),
+                 algo_flops_per_token(wl))]
     name = {"linear": "linear_simt_kernel", "mlp": "mlp_simt_kernel",
             "chunk": "chunk_simt_kernel"}[wl.kind]
     return [(name, "ttt_simt.cu", "f32", algo_bytes_per_token(wl), algo_flops_per_token(wl))]

@@ -303,9 +303,156 @@ __host__ __device__ __forceinline__ uint32_t off_kmajor_none(uint32_t mn, uint32
 
 // Split an fp32 value into two bf16 whose sum carries ~16 significant bits:
 // hi = RN(x), lo = RN(x - hi).
+// Two-term bf16 split of a pair: hi = x with the low 16 bits cleared (exact
+// bf16, |x - hi| < 2^-7 |x|), lo = RN_bf16(x - hi); hi + lo carries ~16
+// significant bits. Returns the packed hi pair and lo pair.
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const uint32_t ua = __float_as_uint(a) & 0xFFFF0000u, ub = __float_as_uint(b) & 0xFFFF0000u;
+    hi = __byte_perm(ua, ub, 0x7632);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - __uint_as_float(ua), b - __uint_as_float(ub));
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
 __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
     hi = __float2bfloat16_rn(x);
     lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
+}  // namespace sm100
+}  // namespace ttt
+
+// ----------------------------------------------------------------- warp-level MMA
+// m16n8k16 bf16 MMA with fp32 accumulation, issued by one warp, operands in
+// registers. Fragment ownership (g = lane / 4, q = lane % 4; a register holds
+// two bf16, the lower column in the low half):
+//   A (16x16, row-major): a0 = A[g][2q..2q+1], a1 = A[g+8][2q..], a2 = A[g][2q+8..], a3 = A[g+8][2q+8..]
+//   B (16x8):             b0 = B[2q..2q+1][g], b1 = B[2q+8..2q+9][g]
+//   D (16x8):             d0 = D[g][2q], d1 = D[g][2q+1], d2 = D[g+8][2q], d3 = D[g+8][2q+1]
+// Two side-by-side D tiles of a 16x16 matrix, packed pairwise, are that
+// matrix's A fragment; movmatrix transposes an 8x8 block between the
+// row-pair layouts of A/D and the column-pair layout of B.
+namespace ttt {
+namespace sm100 {
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Transpose of an 8x8 b16 block held one row-pair per lane.
+__device__ __forceinline__ uint32_t movt(uint32_t x) {
+    uint32_t y;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// ldmatrix: lanes 8i..8i+7 give the shared addresses of the eight 16-byte
+// rows of 8x8 b16 matrix i; each lane receives its row-pair of every matrix
+// (.trans: of every matrix's transpose).
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+}  // namespace sm100
+}  // namespace ttt
+
+// ----------------------------------------------------------------- clusters
+// Distributed shared memory of a thread-block cluster: addresses of another
+// CTA's shared memory come from mapa; mbarriers there are arrived on with
+// release at cluster scope and waited on (locally) with acquire at cluster
+// scope.
+namespace ttt {
+namespace sm100 {
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address, in the cluster's shared window, of the variable at this CTA's
+// shared address `a` in CTA `rank`.
+__device__ __forceinline__ uint32_t mapa(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float2 ld_cluster_f2(uint32_t a) {
+    float2 v;
+    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_cluster_f2(uint32_t a, float x, float y) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(x), "f"(y) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t a, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+
+// Arrive (release, cluster scope) on an mbarrier given by its cluster address.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kTryWaitSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+
+// mbar_wait for a barrier that other CTAs of the cluster arrive on; every
+// lane of the warp waits and the warp agrees on the outcome.
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t parity,
+                                                       volatile int *abort, int *status, int code) {
+    const uint32_t a = smem_u32(bar);
+    bool ok = mbar_try_wait_cluster(a, parity);
+    if (!ok) {
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t i = 1;; ++i) {
+            if (mbar_try_wait_cluster(a, parity)) {
+                ok = true;
+                break;
+            }
+            if ((i & 3u) == 0) {
+                if (*abort) break;
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    *abort = 1;
+                    if (status) atomicExch(status, code);
+                    break;
+                }
+            }
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Whole-cluster barrier (every thread of every CTA), release/acquire.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
 }  // namespace sm100

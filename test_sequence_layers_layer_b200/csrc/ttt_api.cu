@@ -207,8 +207,11 @@ ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float 
 
     MlpArgs a{Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out,
               B, H, T, d, dh, b, dt == TTT_BF16, per_seq};
-    timing_begin(static_cast<cudaStream_t>(stream));
-    return launched(launch_mlp_simt(a, static_cast<cudaStream_t>(stream)));
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    return launched(mlp_tc_supported(d, dh, b, dt == TTT_BF16, (long long)B * H * T)
+                        ? launch_mlp_tc(a, cs)
+                        : launch_mlp_simt(a, cs));
 }
 
 size_t ttt_chunk_workspace_bytes(int B, int H, int T, int d, int chunk) {

@@ -47,6 +47,10 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
 bool linear_tc_supported(int d, int b, bool bf16);
 cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s);
 
+// TTT-MLP warp-MMA scan (bf16, d = 64, hidden 256, b = 16; rows = B*H*T).
+bool mlp_tc_supported(int d, int dh, int b, bool bf16, long long rows);
+cudaError_t launch_mlp_tc(const MlpArgs &a, cudaStream_t s);
+
 // Large-chunk tensor-core path (bf16, d = 128, chunk % 128 == 0).
 bool chunk_tc_supported(int d, int chunk, bool bf16);
 size_t chunk_tc_workspace_bytes(int B, int H, int T, int d, int chunk);

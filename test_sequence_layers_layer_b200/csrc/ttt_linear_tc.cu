@@ -165,16 +165,6 @@ __device__ __forceinline__ void load_quads_f32_swz(const float *base, int row, i
     v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
 }
 
-// Two-term bf16 split of a pair: hi = x with the low 16 bits cleared (exact
-// bf16, |x - hi| < 2^-7 |x|), lo = RN_bf16(x - hi); hi + lo carries ~16
-// significant bits. Returns the packed hi pair and lo pair.
-__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
-    const uint32_t ua = __float_as_uint(a) & 0xFFFF0000u, ub = __float_as_uint(b) & 0xFFFF0000u;
-    hi = __byte_perm(ua, ub, 0x7632);
-    const __nv_bfloat162 l = __floats2bfloat162_rn(a - __uint_as_float(ua), b - __uint_as_float(ub));
-    lo = *reinterpret_cast<const uint32_t *>(&l);
-}
-
 // Packs 4 floats to 4 bf16 hi terms and 4 bf16 lo terms (hi + lo ~ x).
 __device__ __forceinline__ void split4(float a, float b, float c, float d, uint2 &hi, uint2 &lo) {
     split2(a, b, hi.x, lo.x);

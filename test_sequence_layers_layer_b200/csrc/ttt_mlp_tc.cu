@@ -1,0 +1,626 @@
+// ttt_mlp_tc.cu -- TTT-MLP (d = 64, hidden 256, mini-batch b = 16, bf16 Q/K/V)
+// on the tensor cores with warp-level MMA: each (batch, head) sequence is
+// scanned by one thread-block cluster whose CTAs keep both fast-weight layers
+// resident in registers (fp32) for all mini-batches.
+//
+// Method ("Test-Time Training: Linear Complexity Beyond Attention", TTT-MLP;
+// the dual form of "Key Architectural Mechanics of TTT-Linear" applied to
+// each layer). With f(x) = x + LN(GELU(x W1) W2) and the mini-batch's
+// starting weights W1, W2:
+//   H  = K W1,  A = GELU(H),  X = A W2
+//   Gx = diag(eta) dl/dX        (LayerNorm backward of f(K) - V)
+//   Gh = (Gx W2^T) * GELU'(H)
+//   Hq = Q W1 - tril(Q K^T) Gh,  Aq = GELU(Hq)
+//   Z  = Q + LN( Aq W2 - tril(Aq A^T) Gx )
+//   W1 <- W1 - K^T Gh,  W2 <- W2 - A^T Gx
+// tril keeps the diagonal.
+//
+// Why warp-level MMA: every product here is 16 tokens tall and the scan is
+// sequential over the mini-batches, so a product is a handful of 16 x 8 x 16
+// tiles. Issued by 16 warps at once they stay in registers end to end; a
+// single-thread tcgen05 issuer would serialise ~2600 tile products per
+// mini-batch behind one thread.
+//
+// Work split: the 16 warps of a cluster (kCL CTAs of 16/kCL warps) each own
+// 16 hidden units j: rows j of W1^T and of W2 as fp32 MMA accumulator
+// fragments (64 registers a thread). Products whose contraction runs over
+// the hidden units (X = A W2, Aq W2, Aq A^T) are summed across the 16 warps
+// through the cluster's distributed shared memory; products over d or over
+// tokens stay inside the warp. Each warp also owns one token of the
+// mini-batch for the LayerNorm work.
+//
+// Per mini-batch (three split-phase cluster barriers, A, B, C, each counting
+// the 16 warps):
+//   all warps:  H^T = W1^T K^T, A = GELU(H), GELU'(H); partial X; arrive A
+//   token warp: X = sum of the 16 partials, LayerNorm backward -> Gx (fp32
+//               and bf16 hi/lo) into every CTA; arrive B
+//   all warps:  Gh^T = W2 Gx^T * GELU'(H);  Hq0^T = W1^T Q^T, S1 = tril(Q K^T)
+//               Hq^T = Hq0^T - Gh^T S1^T;  Aq = GELU(Hq)
+//               partial Aq A^T and Aq W2; arrive C
+//               W1^T -= Gh^T K,  W2 -= A^T Gx (own rows, no wait)
+//   token warp: Zpre = sum of partials - tril(S2) Gx, LayerNorm, + Q -> Z
+// Precision: Q/K/V enter exactly (bf16); every other operand enters as two
+// bf16 terms hi + lo (hi*hi + hi*lo + lo*hi, fp32 accumulation); sums
+// across warps, the causal correction of Zpre and all LayerNorm math are fp32.
+// Small increments (the weight updates, the causal correction of Hq) are
+// accumulated from zero and then added to the large value in fp32: the tensor
+// core aligns each product to the accumulator's exponent and truncates, so
+// accumulating them into the weight directly would drop most of the lo
+// terms, always toward zero.
+#include "sm100.cuh"
+#include "ttt_common.cuh"
+
+namespace ttt {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 64, kDH = 256, kMB = 16;
+constexpr int kWarpsTotal = kDH / 16;                // 16 hidden units per warp
+constexpr int kSlots = 4, kTileBytes = kMB * kD * 2;  // 2 KB: one [16][64] bf16 tile
+constexpr int kSlotBytes = 3 * kTileBytes;           // K | Q | V
+constexpr int kS2Pitch = 24;                         // padded row of a 16x16 partial
+constexpr int kPart = kMB * kD;                      // floats in one [16][64] partial
+constexpr int kS2Part = kMB * kS2Pitch;              // floats in one 16x16 partial
+
+// Shared memory map of one CTA of a kCL-CTA cluster (offsets from a
+// 1024-aligned base). Tiles of bf16 [16][64] use the 128-byte swizzle:
+// 16-byte chunk c of row t sits at chunk c ^ (t & 7).
+template <int kCL>
+struct Layout {
+    static constexpr int kWarps = kWarpsTotal / kCL, kThreads = kWarps * 32;
+    static constexpr int TILES = 0;                             // [slot][K | Q | V]
+    static constexpr int GXB = TILES + kSlots * kSlotBytes;     // Gx hi | Gx lo tiles
+    static constexpr int GXF = GXB + 2 * kTileBytes;            // Gx fp32 [16][64]
+    static constexpr int XP = GXF + kPart * 4;                  // X partials [warp][16][64]
+    static constexpr int ZP = XP + kWarps * kPart * 4;          // Zpre partials
+    static constexpr int S2P = ZP + kWarps * kPart * 4;         // Aq A^T partials [warp][16][24]
+    static constexpr int BAR = S2P + kWarps * kS2Part * 4;
+    static constexpr int kSmemBytes = BAR + 128 + 1024;         // barriers + alignment slack
+};
+
+constexpr float kRsqrt2 = 0.70710678118654752f, kInvSqrt2Pi = 0.39894228040143268f;
+
+struct Args {
+    const float *eta, *W1_0, *W2_0, *gamma, *beta;
+    float *Z, *W1_out, *W2_out;
+    int H, T;
+    bool w0_per_seq;
+    int *status;
+};
+
+// Byte offset, inside a swizzled [16][64] tile, of the row this lane feeds
+// to ldmatrix.x4 for k-step ks: matrices (tokens 0-7 | 8-15) x (columns
+// 16ks..+7 | 16ks+8..+15), in the order b0, b1 of token tile 0 then of token
+// tile 1 (equally: a0, a2, a1, a3 of the tile as a 16x16 A operand).
+__device__ __forceinline__ uint32_t frag_off(int ks, int lane) {
+    const int mi = lane >> 3, r = lane & 7;
+    const int t = 8 * (mi >> 1) + r, chunk = 2 * ks + (mi & 1);
+    return t * 128 + ((chunk ^ r) << 4);
+}
+
+// Same tile read transposed (ldmatrix .trans) as the B operand [token][col]
+// of two column tiles 2np, 2np+1: matrices (tokens 0-7, tile 2np),
+// (8-15, 2np), (0-7, 2np+1), (8-15, 2np+1).
+__device__ __forceinline__ uint32_t frag_off_t(int np, int lane) {
+    const int mi = lane >> 3, r = lane & 7;
+    const int t = r + 8 * (mi & 1), chunk = 2 * np + (mi >> 1);
+    return t * 128 + ((chunk ^ r) << 4);
+}
+
+// Byte offset of the bf16 pair (columns 2*lane, 2*lane+1) of row t.
+__device__ __forceinline__ uint32_t pair_off(int t, int lane) {
+    return t * 128 + (((lane >> 2) ^ (t & 7)) << 4) + (lane & 3) * 4;
+}
+
+// fp32 [16][64] partial: element (t, i) at word t*64 + ((i/8 ^ (t&7)) * 8) + i%8.
+__device__ __forceinline__ int part_idx(int t, int i) {
+    return t * 64 + ((((i >> 3) ^ (t & 7))) << 3) + (i & 7);
+}
+
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u));
+}
+
+__device__ __forceinline__ float gelu_and_prime(float h, float &prime) {
+    const float Phi = 0.5f * (1.f + erff(h * kRsqrt2));
+    prime = Phi + h * kInvSqrt2Pi * expf(-0.5f * h * h);
+    return h * Phi;
+}
+
+__device__ __forceinline__ float gelu(float h) {
+    return h * 0.5f * (1.f + erff(h * kRsqrt2));
+}
+
+// Packs a warp's 16x16 block held as two D tiles (rows = this warp's hidden
+// units, columns = tokens) into its A fragment, split into hi and lo.
+__device__ __forceinline__ void pack_split(const float (&x)[2][4], uint32_t (&hi)[4],
+                                           uint32_t (&lo)[4]) {
+    split2(x[0][0], x[0][1], hi[0], lo[0]);
+    split2(x[0][2], x[0][3], hi[1], lo[1]);
+    split2(x[1][0], x[1][1], hi[2], lo[2]);
+    split2(x[1][2], x[1][3], hi[3], lo[3]);
+}
+
+// A fragment of the transpose of a 16x16 block given as an A fragment.
+__device__ __forceinline__ void transpose_a(const uint32_t (&a)[4], uint32_t (&t)[4]) {
+    t[0] = movt(a[0]);
+    t[1] = movt(a[2]);
+    t[2] = movt(a[1]);
+    t[3] = movt(a[3]);
+}
+
+// A fragment (hi, lo) of k-step ks of a state block held as 8 D tiles
+// (16 rows x 64 columns).
+__device__ __forceinline__ void state_a(const float (&w)[8][4], int ks, uint32_t (&hi)[4],
+                                        uint32_t (&lo)[4]) {
+    split2(w[2 * ks][0], w[2 * ks][1], hi[0], lo[0]);
+    split2(w[2 * ks][2], w[2 * ks][3], hi[1], lo[1]);
+    split2(w[2 * ks + 1][0], w[2 * ks + 1][1], hi[2], lo[2]);
+    split2(w[2 * ks + 1][2], w[2 * ks + 1][3], hi[3], lo[3]);
+}
+
+// Partial [16 tokens][64] = Act[t][j] W2[j][i] over this warp's 16 hidden
+// units (act = A fragment of Act, hi/lo), written to the swizzled partial.
+__device__ __forceinline__ void partial_times_w2(const uint32_t (&ah)[4], const uint32_t (&al)[4],
+                                                 const float (&w2)[8][4], float *part, int g,
+                                                 int q) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        float acc[4][4];
+#pragma unroll
+        for (int n4 = 0; n4 < 4; ++n4) {
+            const int ni = 4 * half + n4;
+            acc[n4][0] = acc[n4][1] = acc[n4][2] = acc[n4][3] = 0.f;
+            uint32_t bh0, bl0, bh1, bl1;
+            split2(w2[ni][0], w2[ni][1], bh0, bl0);
+            split2(w2[ni][2], w2[ni][3], bh1, bl1);
+            bh0 = movt(bh0);
+            bl0 = movt(bl0);
+            bh1 = movt(bh1);
+            bl1 = movt(bl1);
+            mma16816(acc[n4], ah, bh0, bh1);
+            mma16816(acc[n4], ah, bl0, bl1);
+            mma16816(acc[n4], al, bh0, bh1);
+        }
+#pragma unroll
+        for (int n4 = 0; n4 < 4; ++n4) {
+            const int ni = 4 * half + n4;
+            *reinterpret_cast<float2 *>(part + part_idx(g, 8 * ni + 2 * q)) =
+                make_float2(acc[n4][0], acc[n4][1]);
+            *reinterpret_cast<float2 *>(part + part_idx(g + 8, 8 * ni + 2 * q)) =
+                make_float2(acc[n4][2], acc[n4][3]);
+        }
+    }
+}
+
+template <int kCL>
+__global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
+    mlp_ln_scan_kernel(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmV, Args a) {
+    using L = Layout<kCL>;
+    constexpr int kWarps = L::kWarps;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int rank = kCL > 1 ? (int)cluster_rank() : 0;
+    const int seq = blockIdx.x / kCL, h = seq % a.H, T = a.T, NM = T / kMB;
+    const size_t row0 = (size_t)seq * T;
+    const int gw = rank * kWarps + warp;  // warp index within the cluster
+
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::BAR);
+    uint64_t *barA = full + kSlots, *barB = barA + 1, *barC = barA + 2;
+    volatile int *abrt = reinterpret_cast<volatile int *>(barA + 3);
+    int *status = a.status;
+    float *Xp = reinterpret_cast<float *>(smem + L::XP) + warp * kPart;
+    float *Zp = reinterpret_cast<float *>(smem + L::ZP) + warp * kPart;
+    float *S2p = reinterpret_cast<float *>(smem + L::S2P) + warp * kS2Part;
+    const float *Gxf = reinterpret_cast<const float *>(smem + L::GXF);
+    const uint32_t sGxh = smem_u32(smem + L::GXB), sGxl = sGxh + kTileBytes;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kSlots; ++s) mbar_init(&full[s], 1);
+        mbar_init(barA, kWarpsTotal);
+        mbar_init(barB, kWarpsTotal);
+        mbar_init(barC, kWarpsTotal);
+        *abrt = 0;
+        fence_mbar_init();
+    }
+    if (kCL > 1) cluster_sync(); else __syncthreads();
+
+    // Cluster addresses of the shared buffers of CTA c.
+    auto cl = [&](int off, int c) { return kCL > 1 ? mapa(smem_u32(smem + off), c) : smem_u32(smem + off); };
+    // Arrive on barrier `bar` of every CTA of the cluster (lane 0, after the
+    // warp's writes).
+    auto arrive_all = [&](uint64_t *bar) {
+        __syncwarp();
+        if (lane == 0) {
+            if (kCL > 1) {
+#pragma unroll
+                for (int c = 0; c < kCL; ++c) mbar_arrive_cluster(mapa(smem_u32(bar), c));
+            } else {
+                mbar_arrive(bar);
+            }
+        }
+    };
+
+    // TMA producer (thread 0 of each CTA): mini-batch m into slot m % kSlots,
+    // two ahead. Slot (m + 2) % 4 last held mini-batch m - 2, whose readers in
+    // this CTA all finished before arriving at barrier A of m - 1; thread 0
+    // issues after it passed barrier C of m - 1.
+    int issued = 0;
+    auto issue = [&](int m) {
+        const int s = m % kSlots;
+        uint8_t *dst = smem + L::TILES + s * kSlotBytes;
+        const int y = (int)(row0 + (size_t)m * kMB);
+        mbar_arrive_expect_tx(&full[s], kSlotBytes);
+        tma_load_2d(dst, &tmK, 0, y, &full[s]);
+        tma_load_2d(dst + kTileBytes, &tmQ, 0, y, &full[s]);
+        tma_load_2d(dst + 2 * kTileBytes, &tmV, 0, y, &full[s]);
+    };
+    if (threadIdx.x == 0)
+        for (; issued < 2 && issued < NM; ++issued) issue(issued);
+
+    // State: hidden rows j0 = 16*gw + g and j0 + 8 of W1^T and W2, as 8 D
+    // tiles over the 64 columns (tile n: columns 8n + 2q, 8n + 2q + 1).
+    const int widx = a.w0_per_seq ? seq : h;
+    const float *W1g = a.W1_0 + (size_t)widx * kD * kDH;
+    const float *W2g = a.W2_0 + (size_t)widx * kDH * kD;
+    const int j0 = 16 * gw + g;
+    float w1[8][4], w2[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+        const int i = 8 * n + 2 * q;
+        w1[n][0] = W1g[(size_t)i * kDH + j0];
+        w1[n][1] = W1g[(size_t)(i + 1) * kDH + j0];
+        w1[n][2] = W1g[(size_t)i * kDH + j0 + 8];
+        w1[n][3] = W1g[(size_t)(i + 1) * kDH + j0 + 8];
+        const float2 u = *reinterpret_cast<const float2 *>(W2g + (size_t)j0 * kD + i);
+        const float2 v = *reinterpret_cast<const float2 *>(W2g + (size_t)(j0 + 8) * kD + i);
+        w2[n][0] = u.x;
+        w2[n][1] = u.y;
+        w2[n][2] = v.x;
+        w2[n][3] = v.y;
+    }
+    // Token-warp work: token t_own, columns 2*lane and 2*lane + 1.
+    const int t_own = gw;
+    const float2 gam = make_float2(a.gamma[(size_t)h * kD + 2 * lane], a.gamma[(size_t)h * kD + 2 * lane + 1]);
+    const float2 bet = make_float2(a.beta[(size_t)h * kD + 2 * lane], a.beta[(size_t)h * kD + 2 * lane + 1]);
+    const uint32_t pcol4 = 4u * part_idx(t_own, 2 * lane);
+    const uint32_t po = pair_off(t_own, lane);
+
+    int m = 0;
+    for (; m < NM; ++m) {
+        const int slot = m % kSlots;
+        const uint32_t par = m & 1;
+        if (threadIdx.x == 0 && issued < NM && issued <= m + 2) issue(issued++);
+        const float eta_t = a.eta[row0 + (size_t)m * kMB + t_own];
+        if (!mbar_wait_warp(&full[slot], (m / kSlots) & 1, abrt, status, 61)) break;
+        const uint8_t *tile = smem + L::TILES + slot * kSlotBytes;
+        const uint32_t sK = smem_u32(tile), sQ = sK + kTileBytes;
+
+        // ---- H^T = W1^T K^T  (rows: hidden units, columns: tokens)
+        float hk[2][4] = {};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t ah[4], al[4], kb[4];
+            state_a(w1, ks, ah, al);
+            ldsm_x4(kb, sK + frag_off(ks, lane));
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                mma16816(hk[nt], ah, kb[2 * nt], kb[2 * nt + 1]);
+                mma16816(hk[nt], al, kb[2 * nt], kb[2 * nt + 1]);
+            }
+        }
+        // A = GELU(H), GELU'(H); A^T as an A fragment (hi/lo)
+        float gp[2][4];
+        uint32_t akT_h[4], akT_l[4];
+        {
+            float ak[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ak[nt][e] = gelu_and_prime(hk[nt][e], gp[nt][e]);
+            pack_split(ak, akT_h, akT_l);
+        }
+        // ---- partial X = A W2 over this warp's hidden units
+        {
+            uint32_t ah[4], al[4];
+            transpose_a(akT_h, ah);
+            transpose_a(akT_l, al);
+            partial_times_w2(ah, al, w2, Xp, g, q);
+        }
+        arrive_all(barA);
+
+        // ---- token warp: X row = sum of the 16 partials, LayerNorm backward -> Gx
+        if (!mbar_wait_cluster_warp(barA, par, abrt, status, 62)) break;
+        {
+            float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+            for (int c = 0; c < kCL; ++c) {
+                const uint32_t base = cl(L::XP, c) + pcol4;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) {
+                    const float2 u = ld_cluster_f2(base + w * kPart * 4);
+                    x0 += u.x;
+                    x1 += u.y;
+                }
+            }
+            const float2 kv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(tile + po));
+            const float2 vv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(tile + 2 * kTileBytes + po));
+            const float mu = warp_sum(x0 + x1) * (1.f / kD);
+            const float d0 = x0 - mu, d1 = x1 - mu;
+            const float rstd = rsqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.f / kD) + kLnEps);
+            const float xh0 = d0 * rstd, xh1 = d1 * rstd;
+            const float gh0 = gam.x * (kv.x + gam.x * xh0 + bet.x - vv.x);
+            const float gh1 = gam.y * (kv.y + gam.y * xh1 + bet.y - vv.y);
+            const float m1 = warp_sum(gh0 + gh1) * (1.f / kD);
+            const float m2 = warp_sum(gh0 * xh0 + gh1 * xh1) * (1.f / kD);
+            const float sc = eta_t * rstd;
+            const float G0 = sc * (gh0 - m1 - xh0 * m2), G1 = sc * (gh1 - m1 - xh1 * m2);
+            uint32_t hi, lo;
+            split2(G0, G1, hi, lo);
+#pragma unroll
+            for (int c = 0; c < kCL; ++c) {
+                st_cluster_f2(cl(L::GXF, c) + 4u * (t_own * kD + 2 * lane), G0, G1);
+                st_cluster_u32(cl(L::GXB, c) + po, hi);
+                st_cluster_u32(cl(L::GXB + kTileBytes, c) + po, lo);
+            }
+        }
+        arrive_all(barB);
+        if (!mbar_wait_cluster_warp(barB, par, abrt, status, 63)) break;
+
+        // ---- Gh^T = (W2 Gx^T) * GELU'(H), negated
+        float gh[2][4] = {};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t ah[4], al[4], bh[4], bl[4];
+            state_a(w2, ks, ah, al);
+            ldsm_x4(bh, sGxh + frag_off(ks, lane));
+            ldsm_x4(bl, sGxl + frag_off(ks, lane));
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                mma16816(gh[nt], ah, bh[2 * nt], bh[2 * nt + 1]);
+                mma16816(gh[nt], ah, bl[2 * nt], bl[2 * nt + 1]);
+                mma16816(gh[nt], al, bh[2 * nt], bh[2 * nt + 1]);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) gh[nt][e] = -gh[nt][e] * gp[nt][e];
+        uint32_t ngh_h[4], ngh_l[4];  // -Gh^T (rows: hidden units, columns: tokens)
+        pack_split(gh, ngh_h, ngh_l);
+
+        // ---- Hq0^T = W1^T Q^T and S1 = tril(Q K^T)
+        float hq[2][4] = {}, s1[2][4] = {};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t ah[4], al[4], kb[4], qb[4];
+            state_a(w1, ks, ah, al);
+            ldsm_x4(kb, sK + frag_off(ks, lane));
+            ldsm_x4(qb, sQ + frag_off(ks, lane));
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                mma16816(hq[nt], ah, qb[2 * nt], qb[2 * nt + 1]);
+                mma16816(hq[nt], al, qb[2 * nt], qb[2 * nt + 1]);
+            }
+            const uint32_t qa[4] = {qb[0], qb[2], qb[1], qb[3]};
+#pragma unroll
+            for (int ns = 0; ns < 2; ++ns) mma16816(s1[ns], qa, kb[2 * ns], kb[2 * ns + 1]);
+        }
+#pragma unroll
+        for (int ns = 0; ns < 2; ++ns)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (8 * ns + 2 * q + (e & 1) > g + 8 * (e >> 1)) s1[ns][e] = 0.f;
+
+        // ---- Hq^T = Hq0^T - Gh^T S1^T;  Aq = GELU(Hq)
+        {
+            uint32_t sbh[2][2], sbl[2][2];  // B[s][t] = S1[t][s], token tiles 0 and 1
+            split2(s1[0][0], s1[0][1], sbh[0][0], sbl[0][0]);
+            split2(s1[1][0], s1[1][1], sbh[0][1], sbl[0][1]);
+            split2(s1[0][2], s1[0][3], sbh[1][0], sbl[1][0]);
+            split2(s1[1][2], s1[1][3], sbh[1][1], sbl[1][1]);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                float c[4] = {};
+                mma16816(c, ngh_h, sbh[nt][0], sbh[nt][1]);
+                mma16816(c, ngh_h, sbl[nt][0], sbl[nt][1]);
+                mma16816(c, ngh_l, sbh[nt][0], sbh[nt][1]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) hq[nt][e] += c[e];
+            }
+        }
+        uint32_t aqA_h[4], aqA_l[4];  // Aq[t][j] as an A fragment
+        {
+            float aq[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) aq[nt][e] = gelu(hq[nt][e]);
+            uint32_t th[4], tl[4];
+            pack_split(aq, th, tl);
+            transpose_a(th, aqA_h);
+            transpose_a(tl, aqA_l);
+        }
+        // ---- partial S2 = Aq A^T over this warp's hidden units
+        {
+            uint32_t bh[4], bl[4];  // A[t][j] as an A fragment; B of A^T by token tiles
+            transpose_a(akT_h, bh);
+            transpose_a(akT_l, bl);
+            float s2[2][4] = {};
+#pragma unroll
+            for (int ns = 0; ns < 2; ++ns) {
+                mma16816(s2[ns], aqA_h, bh[ns], bh[ns + 2]);
+                mma16816(s2[ns], aqA_h, bl[ns], bl[ns + 2]);
+                mma16816(s2[ns], aqA_l, bh[ns], bh[ns + 2]);
+            }
+#pragma unroll
+            for (int ns = 0; ns < 2; ++ns) {
+                *reinterpret_cast<float2 *>(S2p + g * kS2Pitch + 8 * ns + 2 * q) =
+                    make_float2(s2[ns][0], s2[ns][1]);
+                *reinterpret_cast<float2 *>(S2p + (g + 8) * kS2Pitch + 8 * ns + 2 * q) =
+                    make_float2(s2[ns][2], s2[ns][3]);
+            }
+        }
+        // ---- partial Zpre = Aq W2 over this warp's hidden units
+        partial_times_w2(aqA_h, aqA_l, w2, Zp, g, q);
+        arrive_all(barC);
+
+        // ---- own state rows: W1^T -= Gh^T K,  W2 -= A^T Gx
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+            uint32_t kb[4];
+            ldsm_x4_t(kb, sK + frag_off_t(np, lane));
+            float u[2][4] = {};
+            mma16816(u[0], ngh_h, kb[0], kb[1]);
+            mma16816(u[0], ngh_l, kb[0], kb[1]);
+            mma16816(u[1], ngh_h, kb[2], kb[3]);
+            mma16816(u[1], ngh_l, kb[2], kb[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                w1[2 * np][e] += u[0][e];
+                w1[2 * np + 1][e] += u[1][e];
+            }
+        }
+        {
+            uint32_t nah[4], nal[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                nah[r] = akT_h[r] ^ 0x80008000u;
+                nal[r] = akT_l[r] ^ 0x80008000u;
+            }
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bh[4], bl[4];
+                ldsm_x4_t(bh, sGxh + frag_off_t(np, lane));
+                ldsm_x4_t(bl, sGxl + frag_off_t(np, lane));
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    float c[4] = {};
+                    mma16816(c, nah, bh[2 * u], bh[2 * u + 1]);
+                    mma16816(c, nah, bl[2 * u], bl[2 * u + 1]);
+                    mma16816(c, nal, bh[2 * u], bh[2 * u + 1]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) w2[2 * np + u][e] += c[e];
+                }
+            }
+        }
+
+        // ---- token warp: Zpre row, causal correction, LayerNorm, residual
+        if (!mbar_wait_cluster_warp(barC, par, abrt, status, 64)) break;
+        {
+            float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+            for (int c = 0; c < kCL; ++c) {
+                const uint32_t base = cl(L::ZP, c) + pcol4;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) {
+                    const float2 u = ld_cluster_f2(base + w * kPart * 4);
+                    z0 += u.x;
+                    z1 += u.y;
+                }
+            }
+            // S2[t][s], s = lane & 15: lanes 0-15 sum cluster warps 0-7,
+            // lanes 16-31 warps 8-15.
+            float sv = 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int w = (lane >> 4) * 8 + k;
+                sv += ld_cluster_f32(cl(L::S2P, w / kWarps) +
+                                     4u * ((w % kWarps) * kS2Part + t_own * kS2Pitch + (lane & 15)));
+            }
+            sv += __shfl_down_sync(0xffffffffu, sv, 16);
+            for (int s = 0; s <= t_own; ++s) {
+                const float c = __shfl_sync(0xffffffffu, sv, s);
+                const float2 gx = *reinterpret_cast<const float2 *>(Gxf + s * kD + 2 * lane);
+                z0 = fmaf(-c, gx.x, z0);
+                z1 = fmaf(-c, gx.y, z1);
+            }
+            const float mu = warp_sum(z0 + z1) * (1.f / kD);
+            const float d0 = z0 - mu, d1 = z1 - mu;
+            const float rstd = rsqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.f / kD) + kLnEps);
+            const float2 qv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(tile + kTileBytes + po));
+            *reinterpret_cast<float2 *>(a.Z + (row0 + (size_t)m * kMB + t_own) * kD + 2 * lane) =
+                make_float2(qv.x + gam.x * d0 * rstd + bet.x, qv.y + gam.y * d1 * rstd + bet.y);
+        }
+    }
+
+    const bool done = m == NM;
+    if (!done && threadIdx.x == 0)
+        // Aborted: let this CTA's in-flight tile loads land before exiting.
+        for (int i = m; i < issued; ++i) mbar_drain(&full[i % kSlots], (i / kSlots) & 1);
+    __syncwarp();
+    if (done && a.W1_out) {
+        float *o = a.W1_out + (size_t)seq * kD * kDH;
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            const int i = 8 * n + 2 * q;
+            o[(size_t)i * kDH + j0] = w1[n][0];
+            o[(size_t)(i + 1) * kDH + j0] = w1[n][1];
+            o[(size_t)i * kDH + j0 + 8] = w1[n][2];
+            o[(size_t)(i + 1) * kDH + j0 + 8] = w1[n][3];
+        }
+    }
+    if (done && a.W2_out) {
+        float *o = a.W2_out + (size_t)seq * kDH * kD;
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            const int i = 8 * n + 2 * q;
+            *reinterpret_cast<float2 *>(o + (size_t)j0 * kD + i) = make_float2(w2[n][0], w2[n][1]);
+            *reinterpret_cast<float2 *>(o + (size_t)(j0 + 8) * kD + i) =
+                make_float2(w2[n][2], w2[n][3]);
+        }
+    }
+    // No CTA leaves while another may still read its partials or write its
+    // Gx buffers and barriers. Every wait above is bounded, so every thread
+    // of the cluster gets here.
+    if (kCL > 1) cluster_sync();
+}
+
+}  // namespace
+
+bool mlp_tc_supported(int d, int dh, int b, bool bf16, long long rows) {
+    return bf16 && d == kD && dh == kDH && b == kMB && rows < (1LL << 31);
+}
+
+// Cluster size: 2 CTAs of 8 warps per sequence (255 registers a thread for
+// the 64-register state plus the working set, two SMs per sequence).
+constexpr int kCluster = 2;
+
+cudaError_t launch_mlp_tc(const MlpArgs &a, cudaStream_t s) {
+    using L = Layout<kCluster>;
+    const uint64_t rows = (uint64_t)a.B * a.H * a.T;
+    alignas(64) CUtensorMap tmK, tmQ, tmV;
+    if (!encode_tmap_bf16_2d(&tmK, a.K, kD, rows, kD, kMB) ||
+        !encode_tmap_bf16_2d(&tmQ, a.Q, kD, rows, kD, kMB) ||
+        !encode_tmap_bf16_2d(&tmV, a.V, kD, rows, kD, kMB))
+        return cudaErrorInvalidValue;
+    auto kernel = mlp_ln_scan_kernel<kCluster>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    Args args{a.eta, a.W1_0, a.W2_0, a.gamma, a.beta, a.Z, a.W1_out, a.W2_out, a.H, a.T,
+              a.w0_per_seq, device_status_word()};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.B * a.H * kCluster));
+    cfg.blockDim = dim3(L::kThreads);
+    cfg.dynamicSmemBytes = L::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, tmK, tmQ, tmV, args);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e == cudaSuccess) count_launch(s);
+    return e;
+}
+
+}  // namespace ttt

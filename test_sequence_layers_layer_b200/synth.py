@@ -15,7 +15,8 @@ with and without LayerNorm, a long-context run, TTT-MLP, and large-chunk
 apply-then-update); their value distributions are:
 Q, K, V ~ N(0, 1)/sqrt(d); fast weights ~ N(0, 0.02^2); LayerNorm gain
 1 + N(0, 0.02^2) and bias N(0, 0.02^2); per-token inner step size
-eta_t = sigmoid(u_t)/d with u_t ~ N(0, 1), or a constant.
+eta_t = base * sigmoid(u_t)/d with u_t ~ N(0, 1) (base 1, or 0.1 for the MLP),
+or a constant.
 bf16 tensors are the round-to-nearest-even bf16 values of the fp32 draws.
 """
 from __future__ import annotations
@@ -121,7 +122,7 @@ class Workload:
     b: int              # mini-batch (linear, mlp) or chunk (chunk) size
     ln: bool            # f(k) = k + LN(...) when True
     dtype: str          # "fp32" | "bf16" (dtype of Q, K, V)
-    eta: str            # "const:<value>" | "sigmoid_over_d"
+    eta: str            # "const:<value>" | "sigmoid_over_d" | "sigmoid_over_d:<base>"
     dh: int = 0         # MLP hidden width
     seed: int = 0
 
@@ -187,9 +188,10 @@ def make_inputs(wl: Workload) -> Inputs:
     V, Vb = _qkv(wl, TID_V)
     if wl.eta.startswith("const:"):
         eta = np.full((wl.B, wl.H, wl.T), float(wl.eta[6:]), dtype=np.float32)
-    elif wl.eta == "sigmoid_over_d":
+    elif wl.eta == "sigmoid_over_d" or wl.eta.startswith("sigmoid_over_d:"):
+        base = float(wl.eta.split(":")[1]) if ":" in wl.eta else 1.0
         u = normals(wl.seed, TID_U, wl.B * wl.H * wl.T)
-        eta = ((1.0 / (1.0 + np.exp(-u))) / wl.d).astype(np.float32)
+        eta = (base * (1.0 / (1.0 + np.exp(-u))) / wl.d).astype(np.float32)
         eta = eta.reshape(wl.B, wl.H, wl.T)
     else:
         raise ValueError(f"unknown eta recipe {wl.eta!r}")

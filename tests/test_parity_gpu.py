@@ -13,6 +13,7 @@ import torch
 import test_sequence_layers_layer_b200 as ttt
 from test_sequence_layers_layer_b200 import synth
 
+from conditioning import conditioned_horizon
 from gpu_helpers import check_parity, run_gpu, to_dev, TOL, max_rel_err, run_oracle
 
 pytestmark = pytest.mark.gpu
@@ -37,6 +38,10 @@ SMALL = {
     "mlp_small": W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=1, H=3, T=48),
     "mlp_fp32_d16": W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=2, H=2, T=32, d=16, dh=64, b=4,
                                                              dtype="fp32"),
+    "mlp_T_eq_b": W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=1, H=2, T=16),
+    "mlp_150_seqs": W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=10, H=15, T=32),
+    "mlp_long": W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=1, H=2, T=1024),
+    "mlp_eta_varied": W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=2, H=2, T=256, eta="sigmoid_over_d"),
     # large chunk
     "chunk_small": W["chunk_d128_c2048_b4h8_t32768"].scaled(B=1, H=3, T=768, b=256,
                                                             eta="const:0.00390625"),
@@ -65,7 +70,6 @@ FULL = [
     ("linear_fp32_d16", None),
     ("linear_ln_d64_b8h12_t2048", None),
     ("linear_ln_d64_b1h32_t32768", None),
-    ("mlp_ln_d64_dh256_b4h12_t8192", [0, 13, 26, 47]),
     ("chunk_d128_c2048_b4h8_t32768", [0, 9, 18, 31]),
 ]
 
@@ -75,6 +79,45 @@ def test_full_size_parity(name, seqs):
     inp = synth.make_inputs(W[name])
     errs = check_parity(inp, seqs=seqs)
     print(f"{name}: max rel err {errs}")
+
+
+def test_mlp_full_size_parity_conditioned():
+    """Every sequence of the full MLP workload. The recurrence with this step
+    size is chaotic on some sequences (see test_conditioning): there even the
+    exact result moves by O(1) under rounding-size input changes after a few
+    thousand tokens, so no finite-precision path can follow it. A sequence
+    counts as conditioned when the oracle, fed inputs changed by 3e-5 relative
+    (2^-15, the precision of a two-term bf16 operand), stays within half the
+    tolerance over all tokens; those are compared over all tokens and their
+    final weights. The others are compared over their first 2048 tokens, which
+    the same probe shows the exact recurrence still tracks."""
+    wl = W["mlp_ln_d64_dh256_b4h12_t8192"]
+    tol = TOL[wl.dtype]
+    inp = synth.make_inputs(wl)
+    horizon, ref = conditioned_horizon(inp, noise=3e-5, rel=tol / 2)
+    Z, W1o, W2o = run_gpu(inp)
+    n = wl.B * wl.H
+    Zg, Zr = Z.reshape(n, wl.T, wl.d), ref[0].reshape(n, wl.T, wl.d)
+    scale = np.abs(Zr).max()
+    full = horizon == wl.T
+    prefix = np.where(full, wl.T, 2048)
+    errs = np.array([np.abs(Zg[s, :p] - Zr[s, :p]).max() / scale for s, p in enumerate(prefix)])
+    cond = np.where(full)[0]
+    e1 = max_rel_err(W1o, ref[1], wl, cond)
+    e2 = max_rel_err(W2o, ref[2], wl, cond)
+    print(f"{len(cond)}/{n} sequences conditioned over all T (shortest horizon {horizon.min()}); "
+          f"Z err conditioned {errs[full].max():.2e}, chaotic prefixes {errs[~full].max():.2e}; "
+          f"W1 {e1:.2e} W2 {e2:.2e}")
+    assert len(cond) >= 32 and horizon.min() >= 2560
+    assert errs.max() <= tol and max(e1, e2) <= tol
+
+
+def test_mlp_full_size_parity_small_step():
+    """The full MLP workload with a 10x smaller inner step, which is well
+    conditioned on every sequence: all sequences, all tokens, final weights."""
+    inp = synth.make_inputs(W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(eta="sigmoid_over_d:0.1"))
+    errs = check_parity(inp)
+    print(f"mlp small step: max rel err {errs}")
 
 
 # ------------------------------------------------------------------ edge cases
@@ -149,6 +192,41 @@ def test_rejects_host_and_misaligned_pointers():
     assert ttt.ttt_linear_fwd(*args(x["Q"].data_ptr() + 2, Z), check=False) == -4
     assert ttt.ttt_linear_fwd(*args(x["Q"], Z), check=False) == 0
     torch.cuda.synchronize()
+
+
+def test_mlp_resume_split_equals_whole():
+    wl = SMALL["mlp_long"].scaled(T=256)
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    args = (x["gamma"], x["beta"])
+    Zw, W1w, W2w = ttt.mlp_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["W2"], *args, b=wl.b)
+    h = wl.T // 2
+    sl = lambda t: t[:, :, :h].contiguous()
+    sr = lambda t: t[:, :, h:].contiguous()
+    Z1, W1a, W2a = ttt.mlp_fwd(sl(x["Q"]), sl(x["K"]), sl(x["V"]), sl(x["eta"]), x["W1"], x["W2"],
+                               *args, b=wl.b)
+    Z2, W1b, W2b = ttt.mlp_fwd(sr(x["Q"]), sr(x["K"]), sr(x["V"]), sr(x["eta"]), W1a, W2a, *args,
+                               b=wl.b, w0_per_seq=True)
+    torch.cuda.synchronize()
+    # The same kernel on the same values: the split run reproduces the whole run exactly.
+    torch.testing.assert_close(torch.cat([Z1, Z2], 2), Zw, rtol=0, atol=0)
+    torch.testing.assert_close(W1b, W1w, rtol=0, atol=0)
+    torch.testing.assert_close(W2b, W2w, rtol=0, atol=0)
+
+
+def test_mlp_deterministic_and_w_out_null():
+    wl = SMALL["mlp_150_seqs"]
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    a = run_gpu(inp, x)
+    b = run_gpu(inp, x)
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
+    Zn, n1, n2 = ttt.mlp_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["W2"], x["gamma"],
+                             x["beta"], b=wl.b, want_w=False)
+    torch.cuda.synchronize()
+    assert n1 is None and n2 is None
+    np.testing.assert_array_equal(Zn.cpu().numpy().astype(np.float64), a[0])
 
 
 def test_chunk_resume_split_equals_whole():
