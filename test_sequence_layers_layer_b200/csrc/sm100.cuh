@@ -457,3 +457,24 @@ __device__ __forceinline__ void cluster_sync() {
 
 }  // namespace sm100
 }  // namespace ttt
+
+// ----------------------------------------------------------------- cluster bulk copies
+namespace ttt {
+namespace sm100 {
+
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
+// this CTA's shared memory to shared memory of a CTA of the cluster; the
+// bytes count as completed transactions on the mbarrier `cluster_bar` (in
+// the destination CTA). The writers of the source fence it for the async
+// proxy first (fence_async_smem).
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t cluster_dst, uint32_t src,
+                                                     uint32_t bytes, uint32_t cluster_bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            cluster_dst),
+        "r"(src), "r"(bytes), "r"(cluster_bar)
+        : "memory");
+}
+
+}  // namespace sm100
+}  // namespace ttt

@@ -29,16 +29,21 @@
 // tokens stay inside the warp. Each warp also owns one token of the
 // mini-batch for the LayerNorm work.
 //
-// Per mini-batch (three split-phase cluster barriers, A, B, C, each counting
-// the 16 warps):
-//   all warps:  H^T = W1^T K^T, A = GELU(H), GELU'(H); partial X; arrive A
-//   token warp: X = sum of the 16 partials, LayerNorm backward -> Gx (fp32
-//               and bf16 hi/lo) into every CTA; arrive B
-//   all warps:  Gh^T = W2 Gx^T * GELU'(H);  Hq0^T = W1^T Q^T, S1 = tril(Q K^T)
-//               Hq^T = Hq0^T - Gh^T S1^T;  Aq = GELU(Hq)
-//               partial Aq A^T and Aq W2; arrive C
-//               W1^T -= Gh^T K,  W2 -= A^T Gx (own rows, no wait)
-//   token warp: Zpre = sum of partials - tril(S2) Gx, LayerNorm, + Q -> Z
+// Per mini-batch m, one exchange between the CTAs (distributed shared memory
+// round trips cost ~1000 cycles here, so the scan makes one per mini-batch):
+//   wait A(m)   (cluster: every CTA's X sums of m and Zpre / S2 sums of m - 1)
+//   LayerNorm backward of all 16 tokens, in every CTA (identical results):
+//               X = sum of the CTAs' sums -> Gx (fp32 and bf16 hi/lo); arrive B
+//   LayerNorm forward of m - 1 for the warp's own token (overlaps B):
+//               Zpre = sums - tril(S2) Gx,  Z = Q + LN(Zpre)
+//   wait B(m)   (CTA: Gx of m)
+//   Gh^T = W2 Gx^T * GELU'(H);  Hq0^T = W1^T Q^T, S1 = tril(Q K^T)
+//   Hq^T = Hq0^T - Gh^T S1^T;  Aq = GELU(Hq);  partials of Aq A^T and Aq W2
+//   W1^T -= Gh^T K,  W2 -= A^T Gx (own rows)
+//   H^T = W1^T K^T of m + 1, A = GELU(H), GELU'(H), partial X = A W2
+//   wait L      (CTA: all partials written)
+//   sums of this CTA's partials per token, pushed to the CTAs that need
+//               them; arrive A(m + 1) in every CTA
 // Precision: Q/K/V enter exactly (bf16); every other operand enters as two
 // bf16 terms hi + lo (hi*hi + hi*lo + lo*hi, fp32 accumulation); sums
 // across warps, the causal correction of Zpre and all LayerNorm math are fp32.
@@ -49,6 +54,24 @@
 // terms, always toward zero.
 #include "sm100.cuh"
 #include "ttt_common.cuh"
+
+// Optional phase trace, compiled in only when TTT_TRACE is defined (a
+// profiling build): lane 0 of warps 0 and 7 of block 0 store the SM clock at
+// each phase boundary of the first kMlpTraceSteps mini-batches.
+#ifdef TTT_TRACE
+constexpr int kMlpTraceEvents = 24, kMlpTraceSteps = 128;
+__device__ unsigned g_ttt_mlp_trace[2 * kMlpTraceEvents * kMlpTraceSteps];
+#define MTRACE(ev)                                                                              \
+    do {                                                                                        \
+        if (blockIdx.x == 0 && lane == 0 && (warp == 0 || warp == 7) && m < kMlpTraceSteps)    \
+            g_ttt_mlp_trace[((warp == 7) * kMlpTraceEvents + (ev)) * kMlpTraceSteps + m] =     \
+                (unsigned)clock();                                                              \
+    } while (0)
+#else
+#define MTRACE(ev) \
+    do {           \
+    } while (0)
+#endif
 
 namespace ttt {
 namespace {
@@ -71,11 +94,18 @@ struct Layout {
     static constexpr int kWarps = kWarpsTotal / kCL, kThreads = kWarps * 32;
     static constexpr int TILES = 0;                             // [slot][K | Q | V]
     static constexpr int GXB = TILES + kSlots * kSlotBytes;     // Gx hi | Gx lo tiles
-    static constexpr int GXF = GXB + 2 * kTileBytes;            // Gx fp32 [16][64]
-    static constexpr int XP = GXF + kPart * 4;                  // X partials [warp][16][64]
-    static constexpr int ZP = XP + kWarps * kPart * 4;          // Zpre partials
-    static constexpr int S2P = ZP + kWarps * kPart * 4;         // Aq A^T partials [warp][16][24]
-    static constexpr int BAR = S2P + kWarps * kS2Part * 4;
+    static constexpr int GXF = GXB + 2 * kTileBytes;            // Gx fp32 [2][16][64]
+    // This CTA's warps' partials (swizzled [16][64] / padded [16][24])
+    static constexpr int XP = GXF + 2 * kPart * 4;              // X   [warp][16][64]
+    static constexpr int ZP = XP + kWarps * kPart * 4;          // Zpre [warp][16][64]
+    static constexpr int S2P = ZP + kWarps * kPart * 4;         // S2  [warp][16][24]
+    // Per-CTA sums of those partials (index: mini-batch parity, source CTA),
+    // at the same offsets in every CTA: the source CTA writes its own slot
+    // and copies it into the others.
+    static constexpr int XS = S2P + kWarps * kS2Part * 4;       // X    [2][kCL][warp][kCL][64]
+    static constexpr int ZS = XS + 2 * kCL * kPart * 4;         // Zpre [2][kCL][16][64]
+    static constexpr int SS = ZS + 2 * kCL * kPart * 4;         // S2   [2][kCL][16][16]
+    static constexpr int BAR = SS + 2 * kCL * kMB * kMB * 4;
     static constexpr int kSmemBytes = BAR + 128 + 1024;         // barriers + alignment slack
 };
 
@@ -130,6 +160,69 @@ __device__ __forceinline__ float gelu_and_prime(float h, float &prime) {
 
 __device__ __forceinline__ float gelu(float h) {
     return h * 0.5f * (1.f + erff(h * kRsqrt2));
+}
+
+// Mean and 1/sigma of N 64-value rows held two values per lane: each lane's
+// mean and sum of squared deviations, merged pairwise across the warp
+// (equal-count case of Chan, Golub and LeVeque's update; the N rows'
+// butterflies interleaved), LayerNorm eps inside the root. Every lane ends
+// with the same bits.
+template <int N>
+__device__ __forceinline__ void row_stats64(const float (&x0)[N], const float (&x1)[N],
+                                            float (&mu)[N], float (&rstd)[N]) {
+    float m[N], M2[N];
+#pragma unroll
+    for (int r = 0; r < N; ++r) {
+        m[r] = 0.5f * (x0[r] + x1[r]);
+        M2[r] = (x0[r] - m[r]) * (x0[r] - m[r]) + (x1[r] - m[r]) * (x1[r] - m[r]);
+    }
+#pragma unroll
+    for (int o = 1, n = 2; o < 32; o <<= 1, n <<= 1) {
+        float mo[N], M2o[N];
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+            mo[r] = __shfl_xor_sync(0xffffffffu, m[r], o);
+            M2o[r] = __shfl_xor_sync(0xffffffffu, M2[r], o);
+        }
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+            const float dl = mo[r] - m[r];
+            m[r] = 0.5f * (m[r] + mo[r]);
+            M2[r] = (M2[r] + M2o[r]) + dl * dl * (0.5f * n);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < N; ++r) {
+        mu[r] = m[r];
+        rstd[r] = rsqrtf(M2[r] * (1.f / kD) + kLnEps);
+    }
+}
+
+__device__ __forceinline__ void row_stats64(float x0, float x1, float &mu, float &rstd) {
+    const float a0[1] = {x0}, a1[1] = {x1};
+    float m[1], r[1];
+    row_stats64<1>(a0, a1, m, r);
+    mu = m[0];
+    rstd = r[0];
+}
+
+// Warp sums of 2N values at once (interleaved butterflies).
+template <int N>
+__device__ __forceinline__ void warp_sum2(float (&a)[N], float (&b)[N]) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        float ao[N], bo[N];
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+            ao[r] = __shfl_xor_sync(0xffffffffu, a[r], o);
+            bo[r] = __shfl_xor_sync(0xffffffffu, b[r], o);
+        }
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+            a[r] += ao[r];
+            b[r] += bo[r];
+        }
+    }
 }
 
 // Packs a warp's 16x16 block held as two D tiles (rows = this warp's hidden
@@ -211,50 +304,46 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
     const int gw = rank * kWarps + warp;  // warp index within the cluster
 
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::BAR);
-    uint64_t *barA = full + kSlots, *barB = barA + 1, *barC = barA + 2;
-    volatile int *abrt = reinterpret_cast<volatile int *>(barA + 3);
+    // Barrier A (one per mini-batch parity) completes when this CTA's warps
+    // have arrived and the other CTAs' sums have landed (as transaction
+    // bytes of their bulk copies). Alternating objects keep a copy for
+    // mini-batch m + 1 out of the phase of m: a CTA sends for m + 2 only
+    // after its own barrier of m + 1 completed, i.e. after every CTA's
+    // copies for m + 1, which each sent after its barrier of m completed.
+    uint64_t *barA = full + kSlots, *barB = barA + 2, *barL = barA + 3;
+    volatile int *abrt = reinterpret_cast<volatile int *>(barA + 4);
     int *status = a.status;
-    float *Xp = reinterpret_cast<float *>(smem + L::XP) + warp * kPart;
-    float *Zp = reinterpret_cast<float *>(smem + L::ZP) + warp * kPart;
-    float *S2p = reinterpret_cast<float *>(smem + L::S2P) + warp * kS2Part;
-    const float *Gxf = reinterpret_cast<const float *>(smem + L::GXF);
     const uint32_t sGxh = smem_u32(smem + L::GXB), sGxl = sGxh + kTileBytes;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSlots; ++s) mbar_init(&full[s], 1);
-        mbar_init(barA, kWarpsTotal);
-        mbar_init(barB, kWarpsTotal);
-        mbar_init(barC, kWarpsTotal);
+        mbar_init(&barA[0], kWarps);  // this CTA's warps (+ the other CTAs' bytes)
+        mbar_init(&barA[1], kWarps);
+        mbar_init(barB, kWarps);       // this CTA's warps
+        mbar_init(barL, kWarps);
         *abrt = 0;
         fence_mbar_init();
     }
     if (kCL > 1) cluster_sync(); else __syncthreads();
 
-    // Cluster addresses of the shared buffers of CTA c.
+    // Cluster address of this CTA's shared offset `off` in CTA c.
     auto cl = [&](int off, int c) { return kCL > 1 ? mapa(smem_u32(smem + off), c) : smem_u32(smem + off); };
-    // Arrive on barrier `bar` of every CTA of the cluster (lane 0, after the
-    // warp's writes).
-    auto arrive_all = [&](uint64_t *bar) {
+    auto arrive_local = [&](uint64_t *bar) {
         __syncwarp();
-        if (lane == 0) {
-            if (kCL > 1) {
-#pragma unroll
-                for (int c = 0; c < kCL; ++c) mbar_arrive_cluster(mapa(smem_u32(bar), c));
-            } else {
-                mbar_arrive(bar);
-            }
-        }
+        if (lane == 0) mbar_arrive(bar);
     };
-
-    // TMA producer (thread 0 of each CTA): mini-batch m into slot m % kSlots,
-    // two ahead. Slot (m + 2) % 4 last held mini-batch m - 2, whose readers in
-    // this CTA all finished before arriving at barrier A of m - 1; thread 0
-    // issues after it passed barrier C of m - 1.
-    int issued = 0;
-    auto issue = [&](int m) {
-        const int s = m % kSlots;
+    auto wait_a = [&](int i) {
+        return mbar_wait_warp(&barA[i & 1], (i >> 1) & 1, abrt, status, 62);
+    };
+    // TMA producer (thread 0 of each CTA): mini-batch i into slot i % kSlots.
+    // Tiles 0 and 1 before the scan; tile m + 2 after barrier B of m, when the
+    // slot's previous tile (m - 2) has had its last reader (the LayerNorm
+    // forward of m - 2, done before every warp's arrival at B of m).
+    int issued = 0, waited = -1;  // tiles issued / last tile waited for (thread 0)
+    auto issue = [&](int i) {
+        const int s = i % kSlots;
         uint8_t *dst = smem + L::TILES + s * kSlotBytes;
-        const int y = (int)(row0 + (size_t)m * kMB);
+        const int y = (int)(row0 + (size_t)i * kMB);
         mbar_arrive_expect_tx(&full[s], kSlotBytes);
         tma_load_2d(dst, &tmK, 0, y, &full[s]);
         tma_load_2d(dst + kTileBytes, &tmQ, 0, y, &full[s]);
@@ -284,24 +373,21 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
         w2[n][2] = v.x;
         w2[n][3] = v.y;
     }
-    // Token-warp work: token t_own, columns 2*lane and 2*lane + 1.
+    // Token work of this warp: tokens warp + kWarps*c (c < kCL) for the
+    // partial sums and the LayerNorm backward (every CTA computes Gx for all
+    // 16 tokens, identically); token t_own = warp + kWarps*rank for the output.
     const int t_own = gw;
     const float2 gam = make_float2(a.gamma[(size_t)h * kD + 2 * lane], a.gamma[(size_t)h * kD + 2 * lane + 1]);
     const float2 bet = make_float2(a.beta[(size_t)h * kD + 2 * lane], a.beta[(size_t)h * kD + 2 * lane + 1]);
-    const uint32_t pcol4 = 4u * part_idx(t_own, 2 * lane);
-    const uint32_t po = pair_off(t_own, lane);
 
-    int m = 0;
-    for (; m < NM; ++m) {
-        const int slot = m % kSlots;
-        const uint32_t par = m & 1;
-        if (threadIdx.x == 0 && issued < NM && issued <= m + 2) issue(issued++);
-        const float eta_t = a.eta[row0 + (size_t)m * kMB + t_own];
-        if (!mbar_wait_warp(&full[slot], (m / kSlots) & 1, abrt, status, 61)) break;
-        const uint8_t *tile = smem + L::TILES + slot * kSlotBytes;
-        const uint32_t sK = smem_u32(tile), sQ = sK + kTileBytes;
-
-        // ---- H^T = W1^T K^T  (rows: hidden units, columns: tokens)
+    // Front half of mini-batch i (all warps): H^T = W1^T K^T, A = GELU(H),
+    // GELU'(H), partial X = A W2 over this warp's hidden units.
+    float gp[2][4];
+    uint32_t akT_h[4], akT_l[4];
+    auto front = [&](int i) -> bool {
+        if (!mbar_wait_warp(&full[i % kSlots], (i / kSlots) & 1, abrt, status, 61)) return false;
+        waited = i;
+        const uint32_t sK = smem_u32(smem + L::TILES + (i % kSlots) * kSlotBytes);
         float hk[2][4] = {};
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
@@ -314,63 +400,206 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
                 mma16816(hk[nt], al, kb[2 * nt], kb[2 * nt + 1]);
             }
         }
-        // A = GELU(H), GELU'(H); A^T as an A fragment (hi/lo)
-        float gp[2][4];
-        uint32_t akT_h[4], akT_l[4];
-        {
-            float ak[2][4];
+        float ak[2][4];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) ak[nt][e] = gelu_and_prime(hk[nt][e], gp[nt][e]);
-            pack_split(ak, akT_h, akT_l);
-        }
-        // ---- partial X = A W2 over this warp's hidden units
-        {
-            uint32_t ah[4], al[4];
-            transpose_a(akT_h, ah);
-            transpose_a(akT_l, al);
-            partial_times_w2(ah, al, w2, Xp, g, q);
-        }
-        arrive_all(barA);
+            for (int e = 0; e < 4; ++e) ak[nt][e] = gelu_and_prime(hk[nt][e], gp[nt][e]);
+        pack_split(ak, akT_h, akT_l);
+        uint32_t ah[4], al[4];
+        transpose_a(akT_h, ah);
+        transpose_a(akT_l, al);
+        partial_times_w2(ah, al, w2, reinterpret_cast<float *>(smem + L::XP) + warp * kPart, g, q);
+        return true;
+    };
 
-        // ---- token warp: X row = sum of the 16 partials, LayerNorm backward -> Gx
-        if (!mbar_wait_cluster_warp(barA, par, abrt, status, 62)) break;
-        {
-            float x0 = 0.f, x1 = 0.f;
+    // This CTA's sums over its warps' partials for this warp's tokens t_c:
+    // X rows of mini-batch `ix` (ix < 0: none) for every CTA, Zpre and S2 rows
+    // of mini-batch `iz` (iz < 0: none) for the CTA owning token t_c. Written
+    // to this CTA's slot, copied to the other CTAs' same slot with bulk copies
+    // that complete on their barrier A of mini-batch `ia`; then this warp
+    // arrives on its own barrier A, expecting its twin warps' copies.
+    auto reduce_push = [&](int ix, int iz, int ia) {
 #pragma unroll
-            for (int c = 0; c < kCL; ++c) {
-                const uint32_t base = cl(L::XP, c) + pcol4;
+        for (int c = 0; c < kCL; ++c) {
+            const int t = warp + kWarps * c;
+            const int off = 4 * part_idx(t, 2 * lane);
+            if (ix >= 0) {
+                float2 r = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int w = 0; w < kWarps; ++w) {
-                    const float2 u = ld_cluster_f2(base + w * kPart * 4);
-                    x0 += u.x;
-                    x1 += u.y;
+                    const float2 u = *reinterpret_cast<const float2 *>(smem + L::XP + w * kPart * 4 + off);
+                    r.x += u.x;
+                    r.y += u.y;
+                }
+                *reinterpret_cast<float2 *>(
+                    smem + L::XS + ((((ix & 1) * kCL + rank) * kWarps + warp) * kCL + c) * kD * 4 + 8 * lane) = r;
+            }
+            if (iz >= 0) {
+                float2 r = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) {
+                    const float2 u = *reinterpret_cast<const float2 *>(smem + L::ZP + w * kPart * 4 + off);
+                    r.x += u.x;
+                    r.y += u.y;
+                }
+                *reinterpret_cast<float2 *>(smem + L::ZS + (((iz & 1) * kCL + rank) * kMB + t) * kD * 4 + 8 * lane) = r;
+                if ((lane >> 4) == c) {
+                    float sv = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kWarps; ++w)
+                        sv += *reinterpret_cast<const float *>(
+                            smem + L::S2P + 4 * (w * kS2Part + t * kS2Pitch + (lane & 15)));
+                    *reinterpret_cast<float *>(
+                        smem + L::SS + 4 * ((((iz & 1) * kCL + rank) * kMB + t) * kMB + (lane & 15))) = sv;
                 }
             }
-            const float2 kv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(tile + po));
-            const float2 vv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(tile + 2 * kTileBytes + po));
-            const float mu = warp_sum(x0 + x1) * (1.f / kD);
-            const float d0 = x0 - mu, d1 = x1 - mu;
-            const float rstd = rsqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.f / kD) + kLnEps);
-            const float xh0 = d0 * rstd, xh1 = d1 * rstd;
-            const float gh0 = gam.x * (kv.x + gam.x * xh0 + bet.x - vv.x);
-            const float gh1 = gam.y * (kv.y + gam.y * xh1 + bet.y - vv.y);
-            const float m1 = warp_sum(gh0 + gh1) * (1.f / kD);
-            const float m2 = warp_sum(gh0 * xh0 + gh1 * xh1) * (1.f / kD);
-            const float sc = eta_t * rstd;
-            const float G0 = sc * (gh0 - m1 - xh0 * m2), G1 = sc * (gh1 - m1 - xh1 * m2);
-            uint32_t hi, lo;
-            split2(G0, G1, hi, lo);
+        }
+        uint32_t bytes = 0;  // from each other CTA's twin warp
+        if (kCL > 1) {
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const int xs = L::XS + (((ix & 1) * kCL + rank) * kWarps + warp) * kCL * kD * 4;
+#pragma unroll
+                for (int k = 1; k < kCL; ++k) {
+                    const int c = (rank + k) % kCL, t = warp + kWarps * c;
+                    const uint32_t bar = mapa(smem_u32(&barA[ia & 1]), c);
+                    if (ix >= 0) bulk_copy_to_cluster(cl(xs, c), smem_u32(smem + xs), kCL * kD * 4, bar);
+                    if (iz >= 0) {
+                        const int zs = L::ZS + (((iz & 1) * kCL + rank) * kMB + t) * kD * 4;
+                        const int ss = L::SS + (((iz & 1) * kCL + rank) * kMB + t) * kMB * 4;
+                        bulk_copy_to_cluster(cl(zs, c), smem_u32(smem + zs), kD * 4, bar);
+                        bulk_copy_to_cluster(cl(ss, c), smem_u32(smem + ss), kMB * 4, bar);
+                    }
+                }
+            }
+            bytes = (kCL - 1) * ((ix >= 0 ? kCL * kD * 4 : 0) + (iz >= 0 ? (kD + kMB) * 4 : 0));
+        }
+        __syncwarp();
+        if (lane == 0) {
+            if (bytes) mbar_arrive_expect_tx(&barA[ia & 1], bytes);
+            else mbar_arrive(&barA[ia & 1]);
+        }
+    };
+
+    // LayerNorm forward of mini-batch i for token t_own: Zpre = sum of the
+    // Aq W2 partials - tril(S2) Gx with S2 = sum of the Aq A^T partials;
+    // Z = Q + LN(Zpre).
+    auto ln_forward = [&](int i) {
+        const float *Gxf = reinterpret_cast<const float *>(smem + L::GXF) + (i & 1) * kPart;
+        float z0 = 0.f, z1 = 0.f, sv = 0.f;
+#pragma unroll
+        for (int c = 0; c < kCL; ++c) {
+            const int row = ((i & 1) * kCL + c) * kMB + t_own;
+            const float2 u = *reinterpret_cast<const float2 *>(smem + L::ZS + row * kD * 4 + 8 * lane);
+            z0 += u.x;
+            z1 += u.y;
+            sv += *reinterpret_cast<const float *>(smem + L::SS + 4 * (row * kMB + (lane & 15)));
+        }
+        float cs[kMB];
+#pragma unroll
+        for (int s = 0; s < kMB; ++s) cs[s] = __shfl_sync(0xffffffffu, sv, s);
+        float y0 = 0.f, y1 = 0.f;  // second chain: odd s
+#pragma unroll
+        for (int s = 0; s < kMB; s += 2) {
+            const float c0 = s <= t_own ? cs[s] : 0.f, c1 = s + 1 <= t_own ? cs[s + 1] : 0.f;
+            const float2 g0 = *reinterpret_cast<const float2 *>(Gxf + s * kD + 2 * lane);
+            const float2 g1 = *reinterpret_cast<const float2 *>(Gxf + (s + 1) * kD + 2 * lane);
+            z0 = fmaf(-c0, g0.x, z0);
+            z1 = fmaf(-c0, g0.y, z1);
+            y0 = fmaf(-c1, g1.x, y0);
+            y1 = fmaf(-c1, g1.y, y1);
+        }
+        z0 += y0;
+        z1 += y1;
+        float mu, rstd;
+        row_stats64(z0, z1, mu, rstd);
+        const uint8_t *tile = smem + L::TILES + (i % kSlots) * kSlotBytes;
+        const float2 qv =
+            bf2_to_f2(*reinterpret_cast<const uint32_t *>(tile + kTileBytes + pair_off(t_own, lane)));
+        *reinterpret_cast<float2 *>(a.Z + (row0 + (size_t)i * kMB + t_own) * kD + 2 * lane) =
+            make_float2(qv.x + gam.x * (z0 - mu) * rstd + bet.x, qv.y + gam.y * (z1 - mu) * rstd + bet.y);
+    };
+
+    int m = 0;
+    bool ok = front(0);
+    arrive_local(barL);
+    ok = ok && mbar_wait_warp(barL, 0, abrt, status, 65);
+    if (ok) reduce_push(0, -1, 0);
+    float eta_c[kCL];  // eta of this warp's tokens in mini-batch m
+#pragma unroll
+    for (int c = 0; c < kCL; ++c) eta_c[c] = a.eta[row0 + warp + kWarps * c];
+
+    // Scan. Barrier A of m (cluster): the X sums of m and the Zpre / S2 sums
+    // of m - 1 are in place in every CTA; barrier B of m (CTA): Gx of m is in
+    // place; barrier L (CTA): this CTA's partials are in place.
+    for (; ok && m < NM; ++m) {
+        const uint32_t par = m & 1;
+        float eta_n[kCL];
+#pragma unroll
+        for (int c = 0; c < kCL; ++c)
+            eta_n[c] = m + 1 < NM ? a.eta[row0 + (size_t)(m + 1) * kMB + warp + kWarps * c] : 0.f;
+        MTRACE(3);
+        if (!wait_a(m)) break;
+        MTRACE(4);
+        const uint8_t *tile = smem + L::TILES + (m % kSlots) * kSlotBytes;
+        const uint32_t sK = smem_u32(tile), sQ = sK + kTileBytes;
+
+        // ---- LayerNorm backward of this warp's tokens -> Gx (fp32 and hi/lo),
+        // the kCL tokens' reductions interleaved
+        {
+            float x0[kCL], x1[kCL], mu[kCL], rstd[kCL];
 #pragma unroll
             for (int c = 0; c < kCL; ++c) {
-                st_cluster_f2(cl(L::GXF, c) + 4u * (t_own * kD + 2 * lane), G0, G1);
-                st_cluster_u32(cl(L::GXB, c) + po, hi);
-                st_cluster_u32(cl(L::GXB + kTileBytes, c) + po, lo);
+                x0[c] = x1[c] = 0.f;
+#pragma unroll
+                for (int src = 0; src < kCL; ++src) {
+                    const float2 u = *reinterpret_cast<const float2 *>(
+                        smem + L::XS + (((par * kCL + src) * kWarps + warp) * kCL + c) * kD * 4 + 8 * lane);
+                    x0[c] += u.x;
+                    x1[c] += u.y;
+                }
+            }
+            row_stats64<kCL>(x0, x1, mu, rstd);
+            float xh0[kCL], xh1[kCL], gh0[kCL], gh1[kCL], m1[kCL], m2[kCL];
+#pragma unroll
+            for (int c = 0; c < kCL; ++c) {
+                const uint32_t po = pair_off(warp + kWarps * c, lane);
+                const float2 kv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(tile + po));
+                const float2 vv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(tile + 2 * kTileBytes + po));
+                xh0[c] = (x0[c] - mu[c]) * rstd[c];
+                xh1[c] = (x1[c] - mu[c]) * rstd[c];
+                gh0[c] = gam.x * (kv.x + gam.x * xh0[c] + bet.x - vv.x);
+                gh1[c] = gam.y * (kv.y + gam.y * xh1[c] + bet.y - vv.y);
+                m1[c] = gh0[c] + gh1[c];
+                m2[c] = gh0[c] * xh0[c] + gh1[c] * xh1[c];
+            }
+            warp_sum2<kCL>(m1, m2);
+#pragma unroll
+            for (int c = 0; c < kCL; ++c) {
+                const int t = warp + kWarps * c;
+                const float sc = eta_c[c] * rstd[c], a1 = m1[c] * (1.f / kD), a2 = m2[c] * (1.f / kD);
+                const float G0 = sc * (gh0[c] - a1 - xh0[c] * a2), G1 = sc * (gh1[c] - a1 - xh1[c] * a2);
+                *reinterpret_cast<float2 *>(smem + L::GXF + (par * kPart + t * kD + 2 * lane) * 4) =
+                    make_float2(G0, G1);
+                uint32_t hi, lo;
+                split2(G0, G1, hi, lo);
+                const uint32_t po = pair_off(t, lane);
+                *reinterpret_cast<uint32_t *>(smem + L::GXB + po) = hi;
+                *reinterpret_cast<uint32_t *>(smem + L::GXB + kTileBytes + po) = lo;
             }
         }
-        arrive_all(barB);
-        if (!mbar_wait_cluster_warp(barB, par, abrt, status, 63)) break;
+        arrive_local(barB);
+        MTRACE(5);
+#pragma unroll
+        for (int c = 0; c < kCL; ++c) eta_c[c] = eta_n[c];
+        // ---- output of the previous mini-batch (overlaps the wait)
+        if (m > 0) ln_forward(m - 1);
+        MTRACE(14);
+        if (!mbar_wait_warp(barB, par, abrt, status, 63)) break;
+        MTRACE(6);
+        if (threadIdx.x == 0 && issued < NM) issue(issued++);
 
         // ---- Gh^T = (W2 Gx^T) * GELU'(H), negated
         float gh[2][4] = {};
@@ -393,6 +622,7 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
             for (int e = 0; e < 4; ++e) gh[nt][e] = -gh[nt][e] * gp[nt][e];
         uint32_t ngh_h[4], ngh_l[4];  // -Gh^T (rows: hidden units, columns: tokens)
         pack_split(gh, ngh_h, ngh_l);
+        MTRACE(7);
 
         // ---- Hq0^T = W1^T Q^T and S1 = tril(Q K^T)
         float hq[2][4] = {}, s1[2][4] = {};
@@ -416,6 +646,7 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 if (8 * ns + 2 * q + (e & 1) > g + 8 * (e >> 1)) s1[ns][e] = 0.f;
+        MTRACE(8);
 
         // ---- Hq^T = Hq0^T - Gh^T S1^T;  Aq = GELU(Hq)
         {
@@ -446,6 +677,7 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
             transpose_a(th, aqA_h);
             transpose_a(tl, aqA_l);
         }
+        MTRACE(9);
         // ---- partial S2 = Aq A^T over this warp's hidden units
         {
             uint32_t bh[4], bl[4];  // A[t][j] as an A fragment; B of A^T by token tiles
@@ -458,6 +690,7 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
                 mma16816(s2[ns], aqA_h, bl[ns], bl[ns + 2]);
                 mma16816(s2[ns], aqA_l, bh[ns], bh[ns + 2]);
             }
+            float *S2p = reinterpret_cast<float *>(smem + L::S2P) + warp * kS2Part;
 #pragma unroll
             for (int ns = 0; ns < 2; ++ns) {
                 *reinterpret_cast<float2 *>(S2p + g * kS2Pitch + 8 * ns + 2 * q) =
@@ -466,9 +699,10 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
                     make_float2(s2[ns][2], s2[ns][3]);
             }
         }
+        MTRACE(10);
         // ---- partial Zpre = Aq W2 over this warp's hidden units
-        partial_times_w2(aqA_h, aqA_l, w2, Zp, g, q);
-        arrive_all(barC);
+        partial_times_w2(aqA_h, aqA_l, w2, reinterpret_cast<float *>(smem + L::ZP) + warp * kPart, g, q);
+        MTRACE(11);
 
         // ---- own state rows: W1^T -= Gh^T K,  W2 -= A^T Gx
 #pragma unroll
@@ -509,50 +743,27 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
                 }
             }
         }
-
-        // ---- token warp: Zpre row, causal correction, LayerNorm, residual
-        if (!mbar_wait_cluster_warp(barC, par, abrt, status, 64)) break;
-        {
-            float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-            for (int c = 0; c < kCL; ++c) {
-                const uint32_t base = cl(L::ZP, c) + pcol4;
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) {
-                    const float2 u = ld_cluster_f2(base + w * kPart * 4);
-                    z0 += u.x;
-                    z1 += u.y;
-                }
-            }
-            // S2[t][s], s = lane & 15: lanes 0-15 sum cluster warps 0-7,
-            // lanes 16-31 warps 8-15.
-            float sv = 0.f;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int w = (lane >> 4) * 8 + k;
-                sv += ld_cluster_f32(cl(L::S2P, w / kWarps) +
-                                     4u * ((w % kWarps) * kS2Part + t_own * kS2Pitch + (lane & 15)));
-            }
-            sv += __shfl_down_sync(0xffffffffu, sv, 16);
-            for (int s = 0; s <= t_own; ++s) {
-                const float c = __shfl_sync(0xffffffffu, sv, s);
-                const float2 gx = *reinterpret_cast<const float2 *>(Gxf + s * kD + 2 * lane);
-                z0 = fmaf(-c, gx.x, z0);
-                z1 = fmaf(-c, gx.y, z1);
-            }
-            const float mu = warp_sum(z0 + z1) * (1.f / kD);
-            const float d0 = z0 - mu, d1 = z1 - mu;
-            const float rstd = rsqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.f / kD) + kLnEps);
-            const float2 qv = bf2_to_f2(*reinterpret_cast<const uint32_t *>(tile + kTileBytes + po));
-            *reinterpret_cast<float2 *>(a.Z + (row0 + (size_t)m * kMB + t_own) * kD + 2 * lane) =
-                make_float2(qv.x + gam.x * d0 * rstd + bet.x, qv.y + gam.y * d1 * rstd + bet.y);
-        }
+        MTRACE(12);
+        // ---- front half of the next mini-batch; sums of this CTA's partials
+        const bool more = m + 1 < NM;
+        if (more && !front(m + 1)) break;
+        MTRACE(0);
+        arrive_local(barL);
+        if (!mbar_wait_warp(barL, (m + 1) & 1, abrt, status, 65)) break;
+        MTRACE(15);
+        reduce_push(more ? m + 1 : -1, m, m + 1);
+        MTRACE(16);
     }
 
-    const bool done = m == NM;
+    bool done = m == NM;
+    if (done) {
+        // Output of the last mini-batch once its sums are in place.
+        if (wait_a(NM)) ln_forward(NM - 1);
+        else done = false;
+    }
     if (!done && threadIdx.x == 0)
         // Aborted: let this CTA's in-flight tile loads land before exiting.
-        for (int i = m; i < issued; ++i) mbar_drain(&full[i % kSlots], (i / kSlots) & 1);
+        for (int i = waited + 1; i < issued; ++i) mbar_drain(&full[i % kSlots], (i / kSlots) & 1);
     __syncwarp();
     if (done && a.W1_out) {
         float *o = a.W1_out + (size_t)seq * kD * kDH;
@@ -575,9 +786,11 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
                 make_float2(w2[n][2], w2[n][3]);
         }
     }
-    // No CTA leaves while another may still read its partials or write its
-    // Gx buffers and barriers. Every wait above is bounded, so every thread
-    // of the cluster gets here.
+    // No CTA leaves while another may still copy into its shared memory: a
+    // CTA's copies are waited for by their receiver before it gets here, and
+    // on an aborted scan every sender waited out its own bounded wait after
+    // its last copy. Every wait above is bounded, so every thread of the
+    // cluster gets here.
     if (kCL > 1) cluster_sync();
 }
 
@@ -624,3 +837,13 @@ cudaError_t launch_mlp_tc(const MlpArgs &a, cudaStream_t s) {
 }
 
 }  // namespace ttt
+
+#ifdef TTT_TRACE
+extern "C" __attribute__((visibility("default"))) int ttt_mlp_trace_fetch(unsigned *host, int n) {
+    const int cap = 2 * kMlpTraceEvents * kMlpTraceSteps;
+    return cudaMemcpyFromSymbol(host, g_ttt_mlp_trace, sizeof(unsigned) * (n < cap ? n : cap)) ==
+                   cudaSuccess
+               ? 0
+               : -1;
+}
+#endif
