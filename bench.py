@@ -233,6 +233,33 @@ def make_caller(wl, x, stream):
     return call, (Z, Wo)
 
 
+def rank_workload(wl, rank):
+    """Weak scaling: every rank runs the whole workload on its own seeded
+    inputs (its own independent sequences); no data moves between ranks."""
+    return wl.scaled(seed=wl.seed + rank)
+
+
+def reduce_across_ranks(total_ms, e2e_ms, launches, world, device):
+    """Job-level figures from per-rank ones: the slowest rank's device time
+    (MAX) and the launches of all ranks (SUM). Every rank takes both
+    collectives in the same order."""
+    if world <= 1:
+        return total_ms, e2e_ms, launches
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    lc = torch.tensor([launches], dtype=torch.float64, device=device)
+    dist.all_reduce(lc)
+    return float(t[0]), float(t[1]), int(lc[0])
+
+
+def aggregate(wl, world, steps, total_ms):
+    """(tokens per step over all ranks, ms per step, whole-job tokens/s)."""
+    tokens = wl.tokens * world
+    return tokens, total_ms / steps, tokens * steps / (total_ms / 1e3)
+
+
 def gpu_arm(args, wl, rank, world):
     import torch
     import torch.distributed as dist
@@ -242,7 +269,7 @@ def gpu_arm(args, wl, rank, world):
     torch.cuda.set_device(dev)
     ttt.lib()
     peaks, peaks_src = load_peaks()
-    inp = synth.make_inputs(wl.scaled(seed=wl.seed + rank))
+    inp = synth.make_inputs(rank_workload(wl, rank))
     x = device_tensors(inp, dev)
     stream = torch.cuda.Stream(dev)
     call, outs = make_caller(wl, x, stream)
@@ -322,17 +349,8 @@ def gpu_arm(args, wl, rank, world):
     if ttt.ttt_device_status(stream.cuda_stream) != 0:
         raise RuntimeError("device status error in the timed region")
 
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
-        lc = torch.tensor([launches], dtype=torch.float64, device=dev)
-        dist.all_reduce(lc)
-        launches = int(lc[0])
-
-    tokens = wl.tokens * world
-    ms_per_step = total_ms / args.steps
-    value = tokens * args.steps / (total_ms / 1e3)
+    total_ms, e2e_ms, launches = reduce_across_ranks(total_ms, e2e_ms, launches, world, dev)
+    tokens, ms_per_step, value = aggregate(wl, world, args.steps, total_ms)
     # The dominant kernel: largest share of the timed device time. Its average
     # launch duration comes from CUDA events on the launching stream (the
     # step's own events when the call is one kernel).

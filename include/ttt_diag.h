@@ -5,7 +5,7 @@
  * on (shared-memory operand layouts, matrix and instruction descriptors,
  * tensor-memory accumulators) by computing one small product D = A * B on the
  * current device and writing it out, so a caller can compare it with any
- * reference matmul.
+ * reference matmul. ttt_diag_gelu exposes the MLP kernel's activation.
  */
 #ifndef TTT_DIAG_H
 #define TTT_DIAG_H
@@ -30,6 +30,27 @@ extern "C" {
  */
 TTT_API ttt_status ttt_selftest_umma(int M, int N, int K, int a_layout, int b_layout,
                                      const void *A, const void *B, float *D, ttt_stream stream);
+
+/*
+ * GELU(h) and GELU'(h) as the TTT-MLP tensor-core kernel evaluates them
+ * (exact-erf GELU; erf from Abramowitz & Stegun 7.1.26, |error| <= 1.5e-7),
+ * for n fp32 values h -> gelu, gelu_prime (device pointers, n >= 0, either
+ * output may be NULL). Enqueued on `stream`. Lets a caller check the
+ * kernel's activation against any reference.
+ */
+TTT_API ttt_status ttt_diag_gelu(const float *h, float *gelu, float *gelu_prime, int n,
+                                 ttt_stream stream);
+
+/*
+ * Failure-path check: launches one small kernel whose on-chip wait (an
+ * mbarrier that nothing ever arrives on) runs out after limit_us
+ * microseconds (1 <= limit_us <= 1000000), the same bounded wait the TTT
+ * kernels use. The kernel then records the timeout in the device status word
+ * and exits normally, so the context stays usable; ttt_device_status() then
+ * returns TTT_ERR_DEVICE_TIMEOUT once (and clears the word). Returns
+ * TTT_ERR_ARG for a limit out of range.
+ */
+TTT_API ttt_status ttt_diag_wait_timeout(unsigned limit_us, ttt_stream stream);
 
 /*
  * Per-kernel timing of the library's own launches. While enabled, every

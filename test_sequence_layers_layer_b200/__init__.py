@@ -68,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L.ttt_diag_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_float), _I]
         L.ttt_selftest_umma.restype = _I
         L.ttt_selftest_umma.argtypes = [_I] * 5 + [_P, _P, _P, _P]
+        L.ttt_diag_gelu.restype = _I
+        L.ttt_diag_gelu.argtypes = [_P, _P, _P, _I, _P]
+        L.ttt_diag_wait_timeout.restype = _I
+        L.ttt_diag_wait_timeout.argtypes = [ctypes.c_uint, _P]
         _lib = L
     return _lib
 
@@ -177,6 +181,18 @@ def ttt_selftest_umma(M, N, K, a_layout, b_layout, A, B, D, stream=None, check=T
     rc = lib().ttt_selftest_umma(M, N, K, a_layout, b_layout, _ptr(A), _ptr(B), _ptr(D),
                                  _stream(stream))
     return _check("ttt_selftest_umma", rc) if check else rc
+
+
+def ttt_diag_wait_timeout(limit_us, stream=None, check=True):
+    """Diagnostic (include/ttt_diag.h): a bounded on-chip wait that runs out."""
+    rc = lib().ttt_diag_wait_timeout(limit_us, _stream(stream))
+    return _check("ttt_diag_wait_timeout", rc) if check else rc
+
+
+def ttt_diag_gelu(h, gelu, gelu_prime, n, stream=None, check=True):
+    """Diagnostic (include/ttt_diag.h): the MLP kernel's GELU and GELU'."""
+    rc = lib().ttt_diag_gelu(_ptr(h), _ptr(gelu), _ptr(gelu_prime), n, _stream(stream))
+    return _check("ttt_diag_gelu", rc) if check else rc
 
 
 # ----------------------------------------------------------------- conveniences

@@ -65,7 +65,8 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 // device status word and returns false. Returns false at once if another
 // thread already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int *status, int code) {
+                                          int *status, int code,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
@@ -73,7 +74,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (mbar_try_wait(a, parity)) return true;
         if ((i & 3u) == 0) {
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 *abort = 1;
                 if (status) atomicExch(status, code);
                 return false;

@@ -54,6 +54,7 @@
 // terms, always toward zero.
 #include "sm100.cuh"
 #include "ttt_common.cuh"
+#include "ttt_gelu.cuh"
 
 // Optional phase trace, compiled in only when TTT_TRACE is defined (a
 // profiling build): lane 0 of warps 0 and 7 of block 0 store the SM clock at
@@ -109,8 +110,6 @@ struct Layout {
     static constexpr int kSmemBytes = BAR + 128 + 1024;         // barriers + alignment slack
 };
 
-constexpr float kRsqrt2 = 0.70710678118654752f, kInvSqrt2Pi = 0.39894228040143268f;
-
 struct Args {
     const float *eta, *W1_0, *W2_0, *gamma, *beta;
     float *Z, *W1_out, *W2_out;
@@ -150,16 +149,6 @@ __device__ __forceinline__ int part_idx(int t, int i) {
 
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
     return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u));
-}
-
-__device__ __forceinline__ float gelu_and_prime(float h, float &prime) {
-    const float Phi = 0.5f * (1.f + erff(h * kRsqrt2));
-    prime = Phi + h * kInvSqrt2Pi * expf(-0.5f * h * h);
-    return h * Phi;
-}
-
-__device__ __forceinline__ float gelu(float h) {
-    return h * 0.5f * (1.f + erff(h * kRsqrt2));
 }
 
 // Mean and 1/sigma of N 64-value rows held two values per lane: each lane's
@@ -312,6 +301,7 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
     // copies for m + 1, which each sent after its barrier of m completed.
     uint64_t *barA = full + kSlots, *barB = barA + 2, *barL = barA + 3;
     volatile int *abrt = reinterpret_cast<volatile int *>(barA + 4);
+    volatile int *issued_s = abrt + 1;  // tiles issued so far (for the abort drain)
     int *status = a.status;
     const uint32_t sGxh = smem_u32(smem + L::GXB), sGxl = sGxh + kTileBytes;
 
@@ -322,6 +312,7 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
         mbar_init(barB, kWarps);       // this CTA's warps
         mbar_init(barL, kWarps);
         *abrt = 0;
+        *issued_s = 0;
         fence_mbar_init();
     }
     if (kCL > 1) cluster_sync(); else __syncthreads();
@@ -335,11 +326,12 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
     auto wait_a = [&](int i) {
         return mbar_wait_warp(&barA[i & 1], (i >> 1) & 1, abrt, status, 62);
     };
-    // TMA producer (thread 0 of each CTA): mini-batch i into slot i % kSlots.
-    // Tiles 0 and 1 before the scan; tile m + 2 after barrier B of m, when the
-    // slot's previous tile (m - 2) has had its last reader (the LayerNorm
-    // forward of m - 2, done before every warp's arrival at B of m).
-    int issued = 0, waited = -1;  // tiles issued / last tile waited for (thread 0)
+    // TMA producer: mini-batch i into slot i % kSlots, issued by lane 0 of one
+    // warp (warps take turns, so no warp carries it every mini-batch). Tiles 0
+    // and 1 before the scan; tile m + 2 after barrier B of m, when the slot's
+    // previous tile (m - 2) has had its last reader (the LayerNorm forward of
+    // m - 2, done before every warp's arrival at B of m).
+    int waited = -1;  // last tile this thread waited for
     auto issue = [&](int i) {
         const int s = i % kSlots;
         uint8_t *dst = smem + L::TILES + s * kSlotBytes;
@@ -348,9 +340,10 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
         tma_load_2d(dst, &tmK, 0, y, &full[s]);
         tma_load_2d(dst + kTileBytes, &tmQ, 0, y, &full[s]);
         tma_load_2d(dst + 2 * kTileBytes, &tmV, 0, y, &full[s]);
+        *issued_s = i + 1;
     };
     if (threadIdx.x == 0)
-        for (; issued < 2 && issued < NM; ++issued) issue(issued);
+        for (int i = 0; i < 2 && i < NM; ++i) issue(i);
 
     // State: hidden rows j0 = 16*gw + g and j0 + 8 of W1^T and W2, as 8 D
     // tiles over the 64 columns (tile n: columns 8n + 2q, 8n + 2q + 1).
@@ -599,7 +592,7 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
         MTRACE(14);
         if (!mbar_wait_warp(barB, par, abrt, status, 63)) break;
         MTRACE(6);
-        if (threadIdx.x == 0 && issued < NM) issue(issued++);
+        if (lane == 0 && warp == m % kWarps && m + 2 < NM) issue(m + 2);
 
         // ---- Gh^T = (W2 Gx^T) * GELU'(H), negated
         float gh[2][4] = {};
@@ -761,9 +754,15 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
         if (wait_a(NM)) ln_forward(NM - 1);
         else done = false;
     }
-    if (!done && threadIdx.x == 0)
-        // Aborted: let this CTA's in-flight tile loads land before exiting.
-        for (int i = waited + 1; i < issued; ++i) mbar_drain(&full[i % kSlots], (i / kSlots) & 1);
+    if (!done) {
+        // Aborted: let this CTA's in-flight tile loads land before exiting
+        // (every warp takes part in issuing, so every warp's lane 0 checks).
+        __syncwarp();
+        if (lane == 0) {
+            const int n = *issued_s;
+            for (int i = waited + 1; i < n; ++i) mbar_drain(&full[i % kSlots], (i / kSlots) & 1);
+        }
+    }
     __syncwarp();
     if (done && a.W1_out) {
         float *o = a.W1_out + (size_t)seq * kD * kDH;

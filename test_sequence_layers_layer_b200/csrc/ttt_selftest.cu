@@ -4,6 +4,7 @@
 #include "../../include/ttt_diag.h"
 #include "sm100.cuh"
 #include "ttt_common.cuh"
+#include "ttt_gelu.cuh"
 
 namespace ttt {
 namespace {
@@ -102,8 +103,54 @@ __global__ void __launch_bounds__(128) selftest_kernel(SelftestArgs a) {
     if (warp == 0) tmem_dealloc(tbase, ncols);
 }
 
+__global__ void gelu_kernel(const float *h, float *g, float *gp, int n) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        float prime;
+        const float v = gelu_and_prime(h[i], prime);
+        if (g) g[i] = v;
+        if (gp) gp[i] = prime;
+    }
+}
+
+// One warp waits on an mbarrier nobody arrives on, with a short limit.
+__global__ void wait_timeout_kernel(uint64_t limit_ns, int *status) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(&bar, 1);
+        abort_flag = 0;
+        sm100::fence_mbar_init();
+    }
+    __syncwarp();
+    sm100::mbar_wait(&bar, 0, &abort_flag, status, 90, limit_ns);
+}
+
 }  // namespace
 }  // namespace ttt
+
+extern "C" ttt_status ttt_diag_wait_timeout(unsigned limit_us, ttt_stream stream) {
+    using namespace ttt;
+    if (limit_us < 1 || limit_us > 1000000) return TTT_ERR_ARG;
+    int *status = device_status_word();
+    if (!status) return TTT_ERR_LAUNCH;
+    wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(1000ull * limit_us, status);
+    if (cudaGetLastError() != cudaSuccess) return TTT_ERR_LAUNCH;
+    count_launch(1);
+    return TTT_OK;
+}
+
+extern "C" ttt_status ttt_diag_gelu(const float *h, float *gelu, float *gelu_prime, int n,
+                                    ttt_stream stream) {
+    using namespace ttt;
+    if (n < 0) return TTT_ERR_SHAPE;
+    if (n == 0) return TTT_OK;
+    if (!h) return TTT_ERR_PTR;
+    const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
+    gelu_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(h, gelu, gelu_prime, n);
+    if (cudaGetLastError() != cudaSuccess) return TTT_ERR_LAUNCH;
+    count_launch(1);
+    return TTT_OK;
+}
 
 extern "C" ttt_status ttt_selftest_umma(int M, int N, int K, int a_layout, int b_layout,
                                         const void *A, const void *B, float *D,

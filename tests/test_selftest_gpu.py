@@ -31,3 +31,46 @@ def test_umma_layouts(M, N, K, al, bl):
     ref = A.double() @ B.double()
     err = (D.double() - ref).abs().max().item() / ref.abs().max().item()
     assert err < 1e-5, f"layout case {(M, N, K, al, bl)}: rel err {err}"
+
+
+def test_mlp_gelu_against_exact():
+    """The MLP kernel's GELU / GELU' (erf from Abramowitz & Stegun 7.1.26,
+    |erf error| <= 1.5e-7) against the oracle's double-precision exact-erf
+    GELU, on a dense grid over the range the scan sees and far tails."""
+    import numpy as np
+    import oracle
+    h = np.concatenate([np.linspace(-12, 12, 200001), [0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0]])
+    h = h.astype(np.float32)
+    x = torch.from_numpy(h).cuda()
+    g = torch.empty_like(x)
+    gp = torch.empty_like(x)
+    ttt.ttt_diag_gelu(x, g, gp, x.numel())
+    torch.cuda.synchronize()
+    hd = h.astype(np.float64)
+    ref_g = np.array([oracle.gelu(v) for v in hd[::7]])
+    ref_gp = np.array([oracle.gelu_prime(v) for v in hd[::7]])
+    g = g.double().cpu().numpy()[::7]
+    gp = gp.double().cpu().numpy()[::7]
+    # The formula in fp32 (evaluated off line on this grid) stays within 1.8e-7 * max(|h|, 1)
+    # for GELU and 2.9e-7 for GELU'; the bounds leave room for the fast exp / reciprocal.
+    assert np.all(np.abs(g - ref_g) <= 4e-7 * np.maximum(np.abs(hd[::7]), 1.0))
+    assert np.all(np.abs(gp - ref_gp) <= 6e-7)
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A device-side wait on a barrier nothing arrives on runs out after its
+    limit, the kernel reports it through the status word and exits; the
+    context stays usable (a TTT call afterwards is still correct)."""
+    import time
+    from test_sequence_layers_layer_b200 import synth
+    from gpu_helpers import check_parity
+    assert ttt.ttt_device_status() == 0
+    assert ttt.ttt_diag_wait_timeout(0, check=False) == -1
+    t0 = time.perf_counter()
+    ttt.ttt_diag_wait_timeout(20000)  # 20 ms
+    assert ttt.ttt_device_status() == -7  # TTT_ERR_DEVICE_TIMEOUT, read once and cleared
+    elapsed = time.perf_counter() - t0
+    assert 0.015 <= elapsed < 5.0
+    assert ttt.ttt_device_status() == 0
+    wl = synth.WORKLOADS["linear_ln_d64_b8h12_t2048"].scaled(B=1, H=2, T=64)
+    check_parity(synth.make_inputs(wl))
