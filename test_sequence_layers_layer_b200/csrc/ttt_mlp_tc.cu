@@ -37,10 +37,11 @@
 //   LayerNorm forward of m - 1 for the warp's own token (overlaps B):
 //               Zpre = sums - tril(S2) Gx,  Z = Q + LN(Zpre)
 //   wait B(m)   (CTA: Gx of m)
-//   Gh^T = W2 Gx^T * GELU'(H);  Hq0^T = W1^T Q^T, S1 = tril(Q K^T)
+//   Gh^T = W2 Gx^T * GELU'(H);  S1 = tril(Q K^T)
 //   Hq^T = Hq0^T - Gh^T S1^T;  Aq = GELU(Hq);  partials of Aq A^T and Aq W2
 //   W1^T -= Gh^T K,  W2 -= A^T Gx (own rows)
-//   H^T = W1^T K^T of m + 1, A = GELU(H), GELU'(H), partial X = A W2
+//   H^T = W1^T K^T and Hq0^T = W1^T Q^T of m + 1, A = GELU(H), GELU'(H),
+//               partial X = A W2
 //   wait L      (CTA: all partials written)
 //   sums of this CTA's partials per token, pushed to the CTAs that need
 //               them; arrive A(m + 1) in every CTA
@@ -62,17 +63,19 @@
 #ifdef TTT_TRACE
 constexpr int kMlpTraceEvents = 24, kMlpTraceSteps = 128;
 __device__ unsigned g_ttt_mlp_trace[2 * kMlpTraceEvents * kMlpTraceSteps];
-#define MTRACE(ev)                                                                              \
+#define MTRACE_AT(ev, i)                                                                        \
     do {                                                                                        \
-        if (blockIdx.x == 0 && lane == 0 && (warp == 0 || warp == 7) && m < kMlpTraceSteps)    \
-            g_ttt_mlp_trace[((warp == 7) * kMlpTraceEvents + (ev)) * kMlpTraceSteps + m] =     \
+        if (blockIdx.x == 0 && lane == 0 && (warp == 0 || warp == 7) && (i) >= 0 &&             \
+            (i) < kMlpTraceSteps)                                                               \
+            g_ttt_mlp_trace[((warp == 7) * kMlpTraceEvents + (ev)) * kMlpTraceSteps + (i)] =   \
                 (unsigned)clock();                                                              \
     } while (0)
 #else
-#define MTRACE(ev) \
-    do {           \
+#define MTRACE_AT(ev, i) \
+    do {                 \
     } while (0)
 #endif
+#define MTRACE(ev) MTRACE_AT(ev, m)
 
 namespace ttt {
 namespace {
@@ -373,24 +376,33 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
     const float2 gam = make_float2(a.gamma[(size_t)h * kD + 2 * lane], a.gamma[(size_t)h * kD + 2 * lane + 1]);
     const float2 bet = make_float2(a.beta[(size_t)h * kD + 2 * lane], a.beta[(size_t)h * kD + 2 * lane + 1]);
 
-    // Front half of mini-batch i (all warps): H^T = W1^T K^T, A = GELU(H),
-    // GELU'(H), partial X = A W2 over this warp's hidden units.
-    float gp[2][4];
+    // Front half of mini-batch i (all warps): H^T = W1^T K^T and
+    // Hq0^T = W1^T Q^T (one split of W1), A = GELU(H), GELU'(H), partial
+    // X = A W2 over this warp's hidden units.
+    float gp[2][4], hq[2][4];
     uint32_t akT_h[4], akT_l[4];
     auto front = [&](int i) -> bool {
         if (!mbar_wait_warp(&full[i % kSlots], (i / kSlots) & 1, abrt, status, 61)) return false;
         waited = i;
         const uint32_t sK = smem_u32(smem + L::TILES + (i % kSlots) * kSlotBytes);
+        const uint32_t sQ = sK + kTileBytes;
         float hk[2][4] = {};
 #pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) hq[nt][e] = 0.f;
+#pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            uint32_t ah[4], al[4], kb[4];
+            uint32_t ah[4], al[4], kb[4], qb[4];
             state_a(w1, ks, ah, al);
             ldsm_x4(kb, sK + frag_off(ks, lane));
+            ldsm_x4(qb, sQ + frag_off(ks, lane));
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 mma16816(hk[nt], ah, kb[2 * nt], kb[2 * nt + 1]);
+                mma16816(hq[nt], ah, qb[2 * nt], qb[2 * nt + 1]);
                 mma16816(hk[nt], al, kb[2 * nt], kb[2 * nt + 1]);
+                mma16816(hq[nt], al, qb[2 * nt], qb[2 * nt + 1]);
             }
         }
         float ak[2][4];
@@ -449,9 +461,11 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
             }
         }
         uint32_t bytes = 0;  // from each other CTA's twin warp
+        MTRACE_AT(17, ia - 1);
         if (kCL > 1) {
             fence_async_smem();
             __syncwarp();
+            MTRACE_AT(18, ia - 1);
             if (lane == 0) {
                 const int xs = L::XS + (((ix & 1) * kCL + rank) * kWarps + warp) * kCL * kD * 4;
 #pragma unroll
@@ -468,6 +482,7 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
                 }
             }
             bytes = (kCL - 1) * ((ix >= 0 ? kCL * kD * 4 : 0) + (iz >= 0 ? (kD + kMB) * 4 : 0));
+            MTRACE_AT(19, ia - 1);
         }
         __syncwarp();
         if (lane == 0) {
@@ -520,19 +535,24 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
     arrive_local(barL);
     ok = ok && mbar_wait_warp(barL, 0, abrt, status, 65);
     if (ok) reduce_push(0, -1, 0);
-    float eta_c[kCL];  // eta of this warp's tokens in mini-batch m
+    // eta of this warp's tokens in mini-batches m and m + 1 (loaded two
+    // mini-batches ahead, so its latency never stalls the scan)
+    float eta_c[kCL], eta_n[kCL];
 #pragma unroll
-    for (int c = 0; c < kCL; ++c) eta_c[c] = a.eta[row0 + warp + kWarps * c];
+    for (int c = 0; c < kCL; ++c) {
+        eta_c[c] = a.eta[row0 + warp + kWarps * c];
+        eta_n[c] = NM > 1 ? a.eta[row0 + kMB + warp + kWarps * c] : 0.f;
+    }
 
     // Scan. Barrier A of m (cluster): the X sums of m and the Zpre / S2 sums
     // of m - 1 are in place in every CTA; barrier B of m (CTA): Gx of m is in
     // place; barrier L (CTA): this CTA's partials are in place.
     for (; ok && m < NM; ++m) {
         const uint32_t par = m & 1;
-        float eta_n[kCL];
+        float eta_nn[kCL];
 #pragma unroll
         for (int c = 0; c < kCL; ++c)
-            eta_n[c] = m + 1 < NM ? a.eta[row0 + (size_t)(m + 1) * kMB + warp + kWarps * c] : 0.f;
+            eta_nn[c] = m + 2 < NM ? a.eta[row0 + (size_t)(m + 2) * kMB + warp + kWarps * c] : 0.f;
         MTRACE(3);
         if (!wait_a(m)) break;
         MTRACE(4);
@@ -586,7 +606,10 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
         arrive_local(barB);
         MTRACE(5);
 #pragma unroll
-        for (int c = 0; c < kCL; ++c) eta_c[c] = eta_n[c];
+        for (int c = 0; c < kCL; ++c) {
+            eta_c[c] = eta_n[c];
+            eta_n[c] = eta_nn[c];
+        }
         // ---- output of the previous mini-batch (overlaps the wait)
         if (m > 0) ln_forward(m - 1);
         MTRACE(14);
@@ -617,19 +640,13 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
         pack_split(gh, ngh_h, ngh_l);
         MTRACE(7);
 
-        // ---- Hq0^T = W1^T Q^T and S1 = tril(Q K^T)
-        float hq[2][4] = {}, s1[2][4] = {};
+        // ---- S1 = tril(Q K^T)  (Hq0^T = W1^T Q^T came with the front half)
+        float s1[2][4] = {};
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            uint32_t ah[4], al[4], kb[4], qb[4];
-            state_a(w1, ks, ah, al);
+            uint32_t kb[4], qb[4];
             ldsm_x4(kb, sK + frag_off(ks, lane));
             ldsm_x4(qb, sQ + frag_off(ks, lane));
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                mma16816(hq[nt], ah, qb[2 * nt], qb[2 * nt + 1]);
-                mma16816(hq[nt], al, qb[2 * nt], qb[2 * nt + 1]);
-            }
             const uint32_t qa[4] = {qb[0], qb[2], qb[1], qb[3]};
 #pragma unroll
             for (int ns = 0; ns < 2; ++ns) mma16816(s1[ns], qa, kb[2 * ns], kb[2 * ns + 1]);
