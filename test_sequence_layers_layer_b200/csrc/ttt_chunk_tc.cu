@@ -32,11 +32,11 @@ constexpr int kD = 128;
 constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: math/epilogue
 
 // ---------------------------------------------------------------------------
-// 1. gram: A_c | B_c = K_c^T [diag(eta) K_c | diag(eta) V_c]
+// 1. gram: A_c | B_c = (diag(eta) K_c)^T [K_c | V_c]
 constexpr int kGramRows = 32;                    // tokens per pipeline stage
 constexpr int kGramStages = 4;
 constexpr int kGramBox = kGramRows * 128;        // one 64-column box of a stage (4 KB)
-constexpr int kGramStageBytes = 6 * kGramBox;    // K raw (2 boxes) | eta*K (2) | V scaled in place (2)
+constexpr int kGramStageBytes = 6 * kGramBox;    // K (2 boxes) | V (2) | eta*K (2)
 constexpr size_t kGramSmem = 1024 + kGramStages * kGramStageBytes;  // 97 KB: two blocks per SM
 
 struct GramArgs {
@@ -90,12 +90,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_arrive_expect_tx(&full[s], 4 * kGramBox);
             tma_load_2d(st, &tmK, 0, y, &full[s]);
             tma_load_2d(st + kGramBox, &tmK, 64, y, &full[s]);
-            tma_load_2d(st + 4 * kGramBox, &tmV, 0, y, &full[s]);
-            tma_load_2d(st + 5 * kGramBox, &tmV, 64, y, &full[s]);
+            tma_load_2d(st + 2 * kGramBox, &tmV, 0, y, &full[s]);
+            tma_load_2d(st + 3 * kGramBox, &tmV, 64, y, &full[s]);
             issued = r + 1;
         }
     } else if (warp == 1 && lane == 0) {
-        // MMA issuer: D[d_in][0:128) += K^T (eta K), D[d_in][128:256) += K^T (eta V).
+        // MMA issuer: D[d_in][0:128) += (eta K)^T K, D[d_in][128:256) += (eta K)^T V.
         const uint32_t idesc = make_idesc_bf16(128, 256, true, true);
         for (int r = 0; r < nst; ++r) {
             const int s = r % kGramStages;
@@ -104,37 +104,35 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint32_t ab = smem_u32(smem + s * kGramStageBytes);
 #pragma unroll
             for (int k = 0; k < kGramRows / 16; ++k) {
-                const uint64_t ad = make_sdesc(ab + k * 2048, kGramBox, 1024, kSw128);
-                const uint64_t bd = make_sdesc(ab + 2 * kGramBox + k * 2048, kGramBox, 1024, kSw128);
+                const uint64_t ad = make_sdesc(ab + 4 * kGramBox + k * 2048, kGramBox, 1024, kSw128);
+                const uint64_t bd = make_sdesc(ab + k * 2048, kGramBox, 1024, kSw128);
                 mma_bf16(tm, ad, bd, idesc, (r | k) != 0);
             }
             mma_commit(&empty[s]);
         }
         mma_commit(&done);
     } else if (warp >= 2) {
-        // Scale rows by eta: eta*K into its own buffer (K raw stays the A
-        // operand), V in place. Swizzling permutes 16-byte chunks inside a
+        // Scale K's rows by eta into the A operand's buffer (K and V stay raw
+        // as the B operand). Swizzling permutes 16-byte chunks inside a
         // 128-byte row only, so a chunk's row (token) is offset / 128.
         const int c = threadIdx.x - 64;
-        constexpr int kChunks = 4 * kGramBox / 16;  // 16-byte chunks of K and V per stage
+        constexpr int kChunks = 2 * kGramBox / 16;  // 16-byte chunks of K per stage
         for (int r = 0; r < nst; ++r) {
             const int s = r % kGramStages;
             // This thread's eta values for the stage, loaded before the wait.
             float ev[kChunks / 128];
 #pragma unroll
             for (int i = 0; i < kChunks / 128; ++i) {
-                const int q = c + 128 * i, o = (q % (kChunks / 2)) * 16;
+                const int o = (c + 128 * i) * 16;
                 ev[i] = a.eta[row0 + (long)r * kGramRows + ((o % kGramBox) >> 7)];
             }
             if (!mbar_wait(&full[s], (r / kGramStages) & 1, &abort_flag, a.status, 13)) break;
             uint8_t *st = smem + s * kGramStageBytes;
 #pragma unroll
             for (int i = 0; i < kChunks / 128; ++i) {
-                const int q = c + 128 * i;
-                const int region = q / (kChunks / 2);  // 0: K, 1: V
-                const int o = (q % (kChunks / 2)) * 16;
+                const int o = (c + 128 * i) * 16;
                 const float e = ev[i];
-                const uint4 v = *reinterpret_cast<const uint4 *>(st + (region ? 4 * kGramBox : 0) + o);
+                const uint4 v = *reinterpret_cast<const uint4 *>(st + o);
                 const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
                 uint4 out;
                 __nv_bfloat162 *ho = reinterpret_cast<__nv_bfloat162 *>(&out);
@@ -143,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const float2 f = __bfloat1622float2(h[i]);
                     ho[i] = __floats2bfloat162_rn(f.x * e, f.y * e);
                 }
-                *reinterpret_cast<uint4 *>(st + (region ? 4 * kGramBox : 2 * kGramBox) + o) = out;
+                *reinterpret_cast<uint4 *>(st + 4 * kGramBox + o) = out;
             }
             fence_async_smem();
             mbar_arrive(&conv[s]);
@@ -264,7 +262,8 @@ __global__ void __launch_bounds__(256, 2) chunk_scan_kernel(ScanArgs a) {
 constexpr int kApplyRows = 128;
 constexpr int kApplyStages = 3;
 constexpr int kApplyThreads = 320;  // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
-constexpr size_t kApplySmem = 1024 + 65536 + kApplyStages * 32768;
+constexpr int kApplyStageOff = 65536 + kApplyStages * 32768;  // epilogue staging, 8 KB per warp
+constexpr size_t kApplySmem = 1024 + kApplyStageOff + 8 * 8192;
 
 struct ApplyArgs {
     const uint8_t *Wimg;
@@ -354,25 +353,38 @@ __global__ void __launch_bounds__(kApplyThreads, 1)
         }
     } else if (warp >= 2) {
         // Epilogue: lane = token row of the tile; each warp pair splits the
-        // 128 fp32 columns of its subpartition's 32 rows.
+        // 128 fp32 columns of its subpartition's 32 rows. The warp's 32 x 64
+        // block goes through shared memory (16-byte chunk c of row r at chunk
+        // c ^ (r & 7): conflict-free both ways) so that every global store
+        // writes two whole 256-byte half-rows of Z.
         const int sp = warp & 3, half = (warp - 2) >> 2;
+        float *stage = reinterpret_cast<float *>(smem + kApplyStageOff) + (warp - 2) * 2048;
         for (int t = 0; t < ntile; ++t) {
             const int acc = t & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (t >> 1) & 1, &abort_flag, a.status, 25)))
                 break;
             tc_fence_after();
-            float *zrow = a.Z + ((size_t)(row0 + (long)t * kApplyRows) + 32 * sp + lane) * kD + 64 * half;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 float v[16];
                 tmem_ld16(taddr(tm, 32 * sp, acc * 128 + 64 * half + 16 * q), v);
                 tmem_ld_wait();
-                float4 *d4 = reinterpret_cast<float4 *>(zrow + 16 * q);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                for (int i = 0; i < 4; ++i)
+                    *reinterpret_cast<float4 *>(stage + lane * 64 + (((4 * q + i) ^ (lane & 7)) << 2)) =
+                        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             }
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);
+            mbar_arrive(&tempty[acc]);  // the accumulator is read; the MMA may reuse it
+            __syncwarp();
+            float *zbase = a.Z + ((size_t)(row0 + (long)t * kApplyRows) + 32 * sp) * kD + 64 * half;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int r = 2 * i + (lane >> 4), c = lane & 15;
+                *reinterpret_cast<float4 *>(zbase + (size_t)r * kD + 4 * c) =
+                    *reinterpret_cast<const float4 *>(stage + r * 64 + ((c ^ (r & 7)) << 2));
+            }
+            __syncwarp();
         }
     }
     if (abort_flag) {

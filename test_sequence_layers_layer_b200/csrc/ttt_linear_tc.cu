@@ -394,6 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             float x[8];
             load_quads_f32_swz(Pf + (j & 1) * 1024, t, g, x);
             if (j > 0) {  // X_j = P_j - C_j G_{j-1}: coefficients in registers, two chains
+                // G_{j-1} comes from all four scan warps: wait for all of it.
+                if (!mbar_wait_warp(&gready[(j - 1) & 3], ((j - 1) >> 2) & 1, abrt, status, 44)) break;
                 const float4 *c4 = reinterpret_cast<const float4 *>(Cf + ((j & 1) * 16 + t) * kCStride);
                 float c[16];
 #pragma unroll
