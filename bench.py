@@ -470,6 +470,70 @@ def reference_arm(args, wl):
 
 # ----------------------------------------------------------------------------- main
 
+def decode_arm(args, wl):
+    """Single-token decode (b = 1 streaming): `--decode N` runs N one-token
+    calls per sequence with the state updated in place, as a CUDA graph when
+    capture works (else plain launches), and reports the time per step."""
+    import torch
+    import test_sequence_layers_layer_b200 as ttt
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    n = args.decode
+    dwl = wl.scaled(T=n, b=1)
+    inp = synth.make_inputs(dwl)
+    x = device_tensors(inp, dev)
+    dt = ttt.TTT_BF16 if dwl.dtype == "bf16" else ttt.TTT_FP32
+    flags = (ttt.TTT_F_LN if dwl.ln else 0) | ttt.TTT_F_W0_PER_SEQ
+    toks = [{k: x[k][:, :, i:i + 1].contiguous() for k in ("Q", "K", "V", "eta")} for i in range(n)]
+    state = x["W1"].unsqueeze(0).expand(dwl.B, -1, -1, -1).contiguous()
+    W0 = state.clone()
+    z = torch.empty((dwl.B, dwl.H, 1, dwl.d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    def steps():
+        for t in toks:
+            ttt.ttt_linear_fwd(t["Q"], t["K"], t["V"], t["eta"], state, x["gamma"], x["beta"], z,
+                               state, dwl.B, dwl.H, 1, dwl.d, 1, dt, flags, stream.cuda_stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            steps()
+        stream.synchronize()
+        graph = None
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                steps()
+            graph = g
+        except Exception:
+            graph = None
+        state.copy_(W0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(1, args.steps)
+        e0.record(stream)
+        for _ in range(reps):
+            if graph is not None:
+                graph.replay()
+            else:
+                steps()
+        e1.record(stream)
+        stream.synchronize()
+    if ttt.ttt_device_status(stream.cuda_stream) != 0:
+        raise RuntimeError("device status error in the decode loop")
+    us = e0.elapsed_time(e1) * 1e3 / (reps * n)
+    return {
+        "metric": "TTT-Linear single-token decode step (b = 1, state updated in place)",
+        "value": us, "unit": "us/step", "higher_is_better": False,
+        "tokens_per_s": dwl.B * dwl.H / (us * 1e-6),
+        "n_gpus": 1, "steps": reps * n, "warmup": args.warmup, "dtype": dwl.dtype,
+        "data": "synthetic (seeded SplitMix64 normals; bf16-rounded Q/K/V)",
+        "config": {"workload": wl.name + "_decode", "B": dwl.B, "H": dwl.H, "d": dwl.d,
+                   "layer_norm": dwl.ln, "tokens_per_step": dwl.B * dwl.H,
+                   "cuda_graph": graph is not None},
+    }
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -480,6 +544,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", type=int, default=0,
+                    help="time N single-token decode steps (linear workloads) instead")
     ap.add_argument("--B", type=int, default=None,
                     help="override the workload's batch size (smaller profiling cases)")
     args = ap.parse_args()
@@ -490,6 +556,13 @@ def main():
         wl = wl.scaled(B=args.B, name=f"{wl.name}_B{args.B}")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+
+    if args.decode:
+        if wl.kind != "linear":
+            ap.error("--decode times the linear workloads")
+        if rank == 0:
+            print(json.dumps(decode_arm(args, wl)), flush=True)
+        return
 
     if args.impl == "reference":
         if rank == 0:

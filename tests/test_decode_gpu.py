@@ -1,0 +1,69 @@
+"""Single-token decode (b = 1 streaming): one call per token, the state passed
+in and updated in place (TTT_F_W0_PER_SEQ with W_out aliasing W0). The loop
+must reproduce the whole-sequence call with b = 1 exactly, and the oracle's
+token-by-token online update within the dtype's tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import test_sequence_layers_layer_b200 as ttt
+from test_sequence_layers_layer_b200 import synth
+
+from gpu_helpers import TOL, max_rel_err, run_oracle, to_dev
+
+pytestmark = pytest.mark.gpu
+W = synth.WORKLOADS
+
+
+def _tok(t, i):
+    return t[:, :, i:i + 1].contiguous()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_linear_decode_loop(dtype):
+    wl = W["linear_ln_d64_b8h12_t2048"].scaled(B=2, H=3, T=24, b=1, dtype=dtype)
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    Zw, Ww = ttt.linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
+                            b=1, ln=True)
+    state = x["W1"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    Z = torch.empty_like(Zw)
+    for i in range(wl.T):
+        z = torch.empty((wl.B, wl.H, 1, wl.d), dtype=torch.float32, device="cuda")
+        ttt.ttt_linear_fwd(_tok(x["Q"], i), _tok(x["K"], i), _tok(x["V"], i), _tok(x["eta"], i),
+                           state, x["gamma"], x["beta"], z, state, wl.B, wl.H, 1, wl.d, 1,
+                           ttt.TTT_BF16 if dtype == "bf16" else ttt.TTT_FP32,
+                           ttt.TTT_F_LN | ttt.TTT_F_W0_PER_SEQ)
+        Z[:, :, i:i + 1] = z
+    torch.cuda.synchronize()
+    assert ttt.ttt_device_status() == 0
+    torch.testing.assert_close(Z, Zw, rtol=0, atol=0)
+    torch.testing.assert_close(state, Ww, rtol=0, atol=0)
+    Zr, Wr = run_oracle(inp)
+    assert max_rel_err(Z.double().cpu().numpy(), Zr, wl) <= TOL[dtype]
+    assert max_rel_err(state.double().cpu().numpy(), Wr, wl) <= TOL[dtype]
+
+
+def test_mlp_decode_loop():
+    wl = W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=1, H=2, T=12, b=1)
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    Zw, W1w, W2w = ttt.mlp_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["W2"], x["gamma"],
+                               x["beta"], b=1)
+    s1 = x["W1"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    s2 = x["W2"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    Z = torch.empty_like(Zw)
+    for i in range(wl.T):
+        z = torch.empty((wl.B, wl.H, 1, wl.d), dtype=torch.float32, device="cuda")
+        ttt.ttt_mlp_fwd(_tok(x["Q"], i), _tok(x["K"], i), _tok(x["V"], i), _tok(x["eta"], i),
+                        s1, s2, x["gamma"], x["beta"], z, s1, s2, wl.B, wl.H, 1, wl.d, wl.dh, 1,
+                        ttt.TTT_BF16, ttt.TTT_F_LN | ttt.TTT_F_W0_PER_SEQ)
+        Z[:, :, i:i + 1] = z
+    torch.cuda.synchronize()
+    assert ttt.ttt_device_status() == 0
+    torch.testing.assert_close(Z, Zw, rtol=0, atol=0)
+    torch.testing.assert_close(s1, W1w, rtol=0, atol=0)
+    torch.testing.assert_close(s2, W2w, rtol=0, atol=0)
+    Zr, W1r, W2r = run_oracle(inp)
+    assert max_rel_err(Z.double().cpu().numpy(), Zr, wl) <= TOL["bf16"]
+    assert max_rel_err(s2.double().cpu().numpy(), W2r, wl) <= TOL["bf16"]
