@@ -9,8 +9,9 @@
 // The update is affine in W, so the work splits into three launches:
 //   1. gram:  A_c | B_c for every chunk of every sequence at once (the only
 //             pass over K and V; tcgen05, M = d_in = 128, N = 256, K = tokens);
-//   2. scan:  W_{c+1} = W_c - A_c W_c + B_c, 16 steps per sequence in fp32,
-//             writing each W_c as the ready-made bf16 hi/lo operand image;
+//   2. scan:  W_{c+1} = W_c - A_c W_c + B_c, 16 steps per sequence (tcgen05,
+//             M = N = K = 128, hi/lo operands; the state and the update in
+//             fp32), writing each W_c as the ready-made bf16 hi/lo operand image;
 //   3. apply: Z_c = Q_c W_c for every chunk at once (the only pass over Q and
 //             the only write of Z; tcgen05, M = 128 tokens, N = d_out, K = d_in;
 //             W_c arrives by one bulk copy).
@@ -31,6 +32,12 @@ using namespace sm100;
 constexpr int kD = 128;
 constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: math/epilogue
 
+// Workspace per chunk: A_c as a bf16 hi | lo operand image (K-major, 32 KB
+// each) and B_c as fp32 [128][128] (64 KB); after all chunks, each W_c as the
+// apply kernel's bf16 hi | lo image (MN-major, 64 KB).
+constexpr int kImgBytes = kD * kD * 2;            // one bf16 128 x 128 image
+constexpr int kChunkWs = 2 * kImgBytes + kD * kD * 4;
+
 // ---------------------------------------------------------------------------
 // 1. gram: A_c | B_c = (diag(eta) K_c)^T [K_c | V_c]
 constexpr int kGramRows = 32;                    // tokens per pipeline stage
@@ -41,7 +48,7 @@ constexpr size_t kGramSmem = 1024 + kGramStages * kGramStageBytes;  // 97 KB: tw
 
 struct GramArgs {
     const float *eta;
-    float *AB;  // [chunks][128][256] fp32
+    float *AB;  // [chunks][kChunkWs bytes]: A_c hi | A_c lo | B_c
     int chunk;
     int *status;
 };
@@ -146,20 +153,38 @@ __global__ void __launch_bounds__(kThreads, 2)
             fence_async_smem();
             mbar_arrive(&conv[s]);
         }
-        // Epilogue: lanes are d_in rows; write A_c | B_c rows (1 KB each).
-        // (__all_sync reconverges the warp for the warp-collective TMEM loads.)
+        // Epilogue: lanes are d_in rows i. A_c goes out as the scan's bf16
+        // hi/lo operand image (K-major, 128-byte swizzle: row i = 128 bytes
+        // per 64 columns j), B_c as fp32 rows. (__all_sync reconverges the
+        // warp for the warp-collective TMEM loads.)
         if (__all_sync(0xffffffffu, mbar_wait(&done, 0, &abort_flag, a.status, 14))) {
             tc_fence_after();
             const int sp = warp & 3;
             const int row = 32 * sp + lane;
-            float *dst = a.AB + ((size_t)g * kD + row) * 256;
+            uint8_t *blk = reinterpret_cast<uint8_t *>(a.AB) + (size_t)g * kChunkWs;
+            float *bdst = reinterpret_cast<float *>(blk + 2 * kImgBytes) + (size_t)row * kD;
             for (int q = 0; q < 16; ++q) {
                 float v[16];
                 tmem_ld16(taddr(tm, 32 * sp, 16 * q), v);
                 tmem_ld_wait();
-                float4 *d4 = reinterpret_cast<float4 *>(dst + 16 * q);
+                if (q < 8) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    for (int h = 0; h < 2; ++h) {
+                        uint4 hi, lo;
+                        __nv_bfloat16 *hb = reinterpret_cast<__nv_bfloat16 *>(&hi);
+                        __nv_bfloat16 *lb = reinterpret_cast<__nv_bfloat16 *>(&lo);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) split_bf16(v[8 * h + e], hb[e], lb[e]);
+                        const uint32_t off = off_kmajor_sw128(row, 16 * q + 8 * h, kD);
+                        *reinterpret_cast<uint4 *>(blk + off) = hi;
+                        *reinterpret_cast<uint4 *>(blk + kImgBytes + off) = lo;
+                    }
+                } else {
+                    float4 *d4 = reinterpret_cast<float4 *>(bdst + 16 * (q - 8));
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                }
             }
         }
     }
@@ -180,81 +205,198 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ---------------------------------------------------------------------------
-// 2. scan: W_{c+1} = W_c - A_c W_c + B_c, one block per (sequence, 16 columns).
-// A_c is staged in shared memory with coalesced loads each step; W_c is also
-// written out as the apply kernel's bf16 hi/lo operand image.
-constexpr int kScanPitch = kD + 4;  // padded A row (floats)
-constexpr size_t kScanSmem = (size_t)kD * kScanPitch * 4 + kD * 16 * 4;
+// 2. scan: W_{c+1} = W_c - A_c W_c + B_c, one block per sequence, on the
+// tensor cores. The fp32 state W lives in the registers of 8 epilogue warps
+// (row i = TMEM lane, 64 columns each); per chunk the MMA thread forms
+// D = A_c W_c from the bf16 hi/lo images of A_c (written by the gram kernel,
+// brought in by bulk copy, double-buffered) and of W_c (in shared memory):
+// A_hi W_hi + A_hi W_lo + A_lo W_hi, M = N = 128, K = 128, fp32 in TMEM. The
+// epilogue adds W_c + B_c - D in fp32 (B_c read from global ahead of time),
+// rewrites the W image for the next chunk and bulk-stores it to global as the
+// apply kernel's operand for that chunk.
+constexpr int kScanThreads = 320;  // warp 0: A loads, warp 1: MMA + TMEM, warps 2-9: epilogue
+constexpr size_t kScanSmem = 1024 + 2 * (size_t)kImgBytes /* W */ + 4 * (size_t)kImgBytes /* A x2 */;
 
 struct ScanArgs {
-    const float *AB, *W0;
-    uint8_t *Wimg;  // [chunks][hi 32 KB | lo 32 KB]: MN-major, 128-byte swizzle
+    const uint8_t *AB;  // per chunk: A_c hi | lo image, B_c fp32
+    const float *W0;
+    uint8_t *Wimg;      // [chunks][hi 32 KB | lo 32 KB]: MN-major, 128-byte swizzle
     float *W_out;
     int H, chunks_per_seq;
     bool w0_per_seq;
+    int *status;
 };
 
-__global__ void __launch_bounds__(256, 2) chunk_scan_kernel(ScanArgs a) {
-    extern __shared__ __align__(16) float scan_smem[];
-    float *sA = scan_smem;                 // [128][kScanPitch]
-    float *sW = scan_smem + kD * kScanPitch;  // [128][16]
-    const int seq = blockIdx.x, j0 = 16 * blockIdx.y;
-    const int i = threadIdx.x >> 1, jh = 8 * (threadIdx.x & 1);
-    const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? seq : seq % a.H) * kD * kD;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) sW[i * 16 + jh + j] = W0[i * kD + j0 + jh + j];
-    for (int c = 0; c < a.chunks_per_seq; ++c) {
-        const size_t g = (size_t)seq * a.chunks_per_seq + c;
-        const float *AB = a.AB + g * kD * 256;
-        // stage A_c (columns 0..127 of the 256-wide rows), coalesced
-#pragma unroll 4
-        for (int e = threadIdx.x; e < kD * kD / 4; e += 256) {
-            const int r = e >> 5, c4 = e & 31;
-            *reinterpret_cast<float4 *>(sA + r * kScanPitch + 4 * c4) =
-                *reinterpret_cast<const float4 *>(AB + (size_t)r * 256 + 4 * c4);
+__device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+                 "r"(smem_u32(ssrc)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(ScanArgs a) {
+    extern __shared__ uint8_t scan_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(scan_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sW = smem;                  // W image: hi | lo (MN-major)
+    uint8_t *sA = smem + 2 * kImgBytes;  // A images: [2 buffers][hi | lo] (K-major)
+    __shared__ uint64_t aready[2], afree[2], dfull, wready, drain;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int seq = blockIdx.x, cps = a.chunks_per_seq;
+    const size_t g0 = (size_t)seq * cps;
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&aready[b], 1);
+            mbar_init(&afree[b], 1);
         }
-        const float4 b0 = *reinterpret_cast<const float4 *>(AB + (size_t)i * 256 + 128 + j0 + jh);
-        const float4 b1 = *reinterpret_cast<const float4 *>(AB + (size_t)i * 256 + 128 + j0 + jh + 4);
-        __syncthreads();
-        float acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = sW[i * 16 + jh + j];
-        {  // W_c as the bf16 hi/lo operand image of the apply kernel
-            uint4 hi, lo;
-            __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(&hi);
-            __nv_bfloat16 *l = reinterpret_cast<__nv_bfloat16 *>(&lo);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) split_bf16(acc[j], h[j], l[j]);
-            uint8_t *img = a.Wimg + g * 65536;
-            const uint32_t off = off_mnmajor_sw128(i, j0 + jh, kD);
-            *reinterpret_cast<uint4 *>(img + off) = hi;
-            *reinterpret_cast<uint4 *>(img + 32768 + off) = lo;
-        }
-        acc[0] += b0.x; acc[1] += b0.y; acc[2] += b0.z; acc[3] += b0.w;
-        acc[4] += b1.x; acc[5] += b1.y; acc[6] += b1.z; acc[7] += b1.w;
-        const float *Ar = sA + i * kScanPitch;
-#pragma unroll 8
-        for (int k = 0; k < kD; k += 4) {
-            const float4 av = *reinterpret_cast<const float4 *>(Ar + k);
-            const float ak[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const float4 w0 = *reinterpret_cast<const float4 *>(sW + (k + kk) * 16 + jh);
-                const float4 w1 = *reinterpret_cast<const float4 *>(sW + (k + kk) * 16 + jh + 4);
-                acc[0] = fmaf(-ak[kk], w0.x, acc[0]); acc[1] = fmaf(-ak[kk], w0.y, acc[1]);
-                acc[2] = fmaf(-ak[kk], w0.z, acc[2]); acc[3] = fmaf(-ak[kk], w0.w, acc[3]);
-                acc[4] = fmaf(-ak[kk], w1.x, acc[4]); acc[5] = fmaf(-ak[kk], w1.y, acc[5]);
-                acc[6] = fmaf(-ak[kk], w1.z, acc[6]); acc[7] = fmaf(-ak[kk], w1.w, acc[7]);
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) sW[i * 16 + jh + j] = acc[j];
-        __syncthreads();
+        mbar_init(&dfull, 1);
+        mbar_init(&wready, 1);
+        mbar_init(&drain, 1);
+        fence_mbar_init();
     }
-    if (a.W_out)
+    if (warp == 1) tmem_alloc(&tmem_base, 128);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_base;
+    int issued = 0;
+
+    if (warp == 0 && lane == 0) {
+        // A_c images, two chunks ahead of nothing: buffer c & 1 is reused once
+        // the MMAs of chunk c - 2 have completed.
+        for (int c = 0; c < cps; ++c) {
+            const int b = c & 1;
+            if (c >= 2 && !mbar_wait(&afree[b], ((c >> 1) - 1) & 1, &abort_flag, a.status, 16)) break;
+            mbar_arrive_expect_tx(&aready[b], 2 * kImgBytes);
+            bulk_load(sA + b * 2 * kImgBytes, a.AB + (g0 + c) * kChunkWs, 2 * kImgBytes, &aready[b]);
+            issued = c + 1;
+        }
+    } else if (warp == 1 && lane == 0) {
+        const uint32_t idesc = make_idesc_bf16(128, 128, false, true);
+        const uint32_t wb = smem_u32(sW);
+        for (int c = 0; c < cps; ++c) {
+            const int b = c & 1;
+            if (!mbar_wait(&aready[b], (c >> 1) & 1, &abort_flag, a.status, 17)) break;
+            if (!mbar_wait(&wready, c & 1, &abort_flag, a.status, 18)) break;
+            tc_fence_after();
+            const uint32_t ab = smem_u32(sA + b * 2 * kImgBytes);
+            // (A, W) term pairs: hi hi, hi lo, lo hi
+            const uint32_t aoff[3] = {0, 0, (uint32_t)kImgBytes}, woff[3] = {0, (uint32_t)kImgBytes, 0};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) a.W_out[(size_t)seq * kD * kD + i * kD + j0 + jh + j] = sW[i * 16 + jh + j];
+            for (int p = 0; p < 3; ++p)
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k) {
+                    const int k0 = 16 * k;
+                    const uint64_t ad = make_sdesc(ab + aoff[p] + (k0 >> 6) * 16384 + (k0 & 63) * 2, 16, 1024, kSw128);
+                    const uint64_t bd = make_sdesc(wb + woff[p] + (k0 >> 3) * 1024, 16384, 1024, kSw128);
+                    mma_bf16(tm, ad, bd, idesc, (p | k) != 0);
+                }
+            mma_commit(&afree[b]);
+            mma_commit(&dfull);
+        }
+    } else if (warp >= 2) {
+        // Epilogue: row i = 32 (warp & 3) + lane, columns 64 half .. +63.
+        const int sp = warp & 3, half = (warp - 2) >> 2;
+        const int row = 32 * sp + lane, col0 = 64 * half;
+        const bool leader = warp == 2 && lane == 0;
+        const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? seq : seq % a.H) * kD * kD;
+        float w[64];
+#pragma unroll
+        for (int j4 = 0; j4 < 16; ++j4) {
+            const float4 u = *reinterpret_cast<const float4 *>(W0 + (size_t)row * kD + col0 + 4 * j4);
+            w[4 * j4] = u.x;
+            w[4 * j4 + 1] = u.y;
+            w[4 * j4 + 2] = u.z;
+            w[4 * j4 + 3] = u.w;
+        }
+        // Write this thread's 64 values of W as its row of the MN-major image
+        // (k = row, 64-column atom = half): 8 chunks of 8 bf16, hi and lo.
+        auto emit = [&]() {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint4 hi, lo;
+                __nv_bfloat16 *hb = reinterpret_cast<__nv_bfloat16 *>(&hi);
+                __nv_bfloat16 *lb = reinterpret_cast<__nv_bfloat16 *>(&lo);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) split_bf16(w[8 * ch + e], hb[e], lb[e]);
+                const uint32_t off = off_mnmajor_sw128(row, col0 + 8 * ch, kD);
+                *reinterpret_cast<uint4 *>(sW + off) = hi;
+                *reinterpret_cast<uint4 *>(sW + kImgBytes + off) = lo;
+            }
+            fence_async_smem();
+        };
+        // image of W_c -> global (apply's operand for chunk c); W ready for the MMA
+        auto publish = [&](int c) {
+            if (leader) {
+                bulk_store(a.Wimg + (g0 + c) * 65536, sW, 2 * kImgBytes);
+                bulk_commit();
+                mbar_arrive(&wready);
+            }
+        };
+        emit();
+        bool ok = !named_bar_or(1, 256, false);
+        if (ok) publish(0);
+        for (int c = 0; ok && c < cps; ++c) {
+            // B_c row of this thread, read ahead of the product
+            const float *Bc = reinterpret_cast<const float *>(a.AB + (g0 + c) * kChunkWs + 2 * kImgBytes) +
+                              (size_t)row * kD + col0;
+            float bv[64];
+#pragma unroll
+            for (int j4 = 0; j4 < 16; ++j4) {
+                const float4 u = *reinterpret_cast<const float4 *>(Bc + 4 * j4);
+                bv[4 * j4] = u.x;
+                bv[4 * j4 + 1] = u.y;
+                bv[4 * j4 + 2] = u.z;
+                bv[4 * j4 + 3] = u.w;
+            }
+            bool got = mbar_wait(&dfull, c & 1, &abort_flag, a.status, 19);
+            if (leader) bulk_wait_read();  // the image's last store has read it
+            // every epilogue warp agrees before anyone moves on
+            if (named_bar_or(1, 256, !__all_sync(0xffffffffu, got))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float v[16];
+                tmem_ld16(taddr(tm, 32 * sp, col0 + 16 * q), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) w[16 * q + e] = (w[16 * q + e] + bv[16 * q + e]) - v[e];
+            }
+            tc_fence_before();
+            if (c + 1 < cps) emit();
+            if (named_bar_or(1, 256, false)) break;
+            if (c + 1 < cps) publish(c + 1);
+        }
+        if (leader) bulk_wait_all();
+        if (ok && !abort_flag && a.W_out) {
+            float *o = a.W_out + (size_t)seq * kD * kD + (size_t)row * kD + col0;
+#pragma unroll
+            for (int j4 = 0; j4 < 16; ++j4)
+                *reinterpret_cast<float4 *>(o + 4 * j4) =
+                    make_float4(w[4 * j4], w[4 * j4 + 1], w[4 * j4 + 2], w[4 * j4 + 3]);
+        }
+    }
+    // Teardown: after an abort, let this block's own copies and MMAs land
+    // before the shared memory and tensor memory are released.
+    if (abort_flag) {
+        if (warp == 0 && lane == 0)
+            for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
+                mbar_drain(&aready[c & 1], (c >> 1) & 1);
+        if (warp == 1 && lane == 0) {
+            mma_commit(&drain);
+            mbar_drain(&drain, 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tm, 128);
 }
 
 // ---------------------------------------------------------------------------
@@ -440,8 +582,8 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     e = cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kScanSmem);
     if (e != cudaSuccess) return e;
-    chunk_scan_kernel<<<dim3(a.B * a.H, kD / 16), 256, kScanSmem, s>>>(
-        ScanArgs{AB, a.W0, Wimg, a.W_out, a.H, cps, a.w0_per_seq});
+    chunk_scan_kernel<<<a.B * a.H, kScanThreads, kScanSmem, s>>>(
+        ScanArgs{reinterpret_cast<const uint8_t *>(AB), a.W0, Wimg, a.W_out, a.H, cps, a.w0_per_seq, status});
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
