@@ -370,10 +370,8 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
 }  // namespace ttt
 
 // ----------------------------------------------------------------- clusters
-// Distributed shared memory of a thread-block cluster: addresses of another
-// CTA's shared memory come from mapa; mbarriers there are arrived on with
-// release at cluster scope and waited on (locally) with acquire at cluster
-// scope.
+// Thread-block clusters: the CTA's rank, addresses of another CTA's shared
+// memory (mapa), and the whole-cluster barrier.
 namespace ttt {
 namespace sm100 {
 
@@ -389,66 +387,6 @@ __device__ __forceinline__ uint32_t mapa(uint32_t a, uint32_t rank) {
     uint32_t r;
     asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
     return r;
-}
-
-__device__ __forceinline__ float2 ld_cluster_f2(uint32_t a) {
-    float2 v;
-    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a) : "memory");
-    return v;
-}
-__device__ __forceinline__ float ld_cluster_f32(uint32_t a) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_cluster_f2(uint32_t a, float x, float y) {
-    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(x), "f"(y) : "memory");
-}
-__device__ __forceinline__ void st_cluster_u32(uint32_t a, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-
-// Arrive (release, cluster scope) on an mbarrier given by its cluster address.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kTryWaitSuspendNs)
-        : "memory");
-    return ok != 0;
-}
-
-// mbar_wait for a barrier that other CTAs of the cluster arrive on; every
-// lane of the warp waits and the warp agrees on the outcome.
-__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t parity,
-                                                       volatile int *abort, int *status, int code) {
-    const uint32_t a = smem_u32(bar);
-    bool ok = mbar_try_wait_cluster(a, parity);
-    if (!ok) {
-        const uint64_t t0 = globaltimer_ns();
-        for (uint32_t i = 1;; ++i) {
-            if (mbar_try_wait_cluster(a, parity)) {
-                ok = true;
-                break;
-            }
-            if ((i & 3u) == 0) {
-                if (*abort) break;
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                    *abort = 1;
-                    if (status) atomicExch(status, code);
-                    break;
-                }
-            }
-        }
-    }
-    return __all_sync(0xffffffffu, ok);
 }
 
 // Whole-cluster barrier (every thread of every CTA), release/acquire.
