@@ -33,7 +33,7 @@ constexpr int kD = 128;
 constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: math/epilogue
 
 // Workspace per chunk: A_c as a bf16 hi | lo operand image (K-major, 32 KB
-// each) and B_c as fp32 [128][128] (64 KB); after all chunks, each W_c as the
+// each) and B_c in fp32 (64 KB; column quad q of row i at float4 q * 128 + i); after all chunks, each W_c as the
 // apply kernel's bf16 hi | lo image (MN-major, 64 KB).
 constexpr int kImgBytes = kD * kD * 2;            // one bf16 128 x 128 image
 constexpr int kChunkWs = 2 * kImgBytes + kD * kD * 4;
@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int sp = warp & 3;
             const int row = 32 * sp + lane;
             uint8_t *blk = reinterpret_cast<uint8_t *>(a.AB) + (size_t)g * kChunkWs;
-            float *bdst = reinterpret_cast<float *>(blk + 2 * kImgBytes) + (size_t)row * kD;
+            float4 *bdst = reinterpret_cast<float4 *>(blk + 2 * kImgBytes);
             for (int q = 0; q < 16; ++q) {
                 float v[16];
                 tmem_ld16(taddr(tm, 32 * sp, 16 * q), v);
@@ -179,11 +179,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                         *reinterpret_cast<uint4 *>(blk + off) = hi;
                         *reinterpret_cast<uint4 *>(blk + kImgBytes + off) = lo;
                     }
-                } else {
-                    float4 *d4 = reinterpret_cast<float4 *>(bdst + 16 * (q - 8));
+                } else {  // B_c: column quad q4 of row i at float4 q4 * 128 + i
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        bdst[(4 * (q - 8) + i) * kD + row] =
+                            make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                 }
             }
         }
@@ -345,12 +345,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(ScanArgs a)
         if (ok) publish(0);
         for (int c = 0; ok && c < cps; ++c) {
             // B_c row of this thread, read ahead of the product
-            const float *Bc = reinterpret_cast<const float *>(a.AB + (g0 + c) * kChunkWs + 2 * kImgBytes) +
-                              (size_t)row * kD + col0;
+            // (column quad q4 of row i at float4 q4 * 128 + i: a warp reads 512
+            // contiguous bytes per load)
+            const float4 *Bc = reinterpret_cast<const float4 *>(a.AB + (g0 + c) * kChunkWs + 2 * kImgBytes);
             float bv[64];
 #pragma unroll
             for (int j4 = 0; j4 < 16; ++j4) {
-                const float4 u = *reinterpret_cast<const float4 *>(Bc + 4 * j4);
+                const float4 u = Bc[(col0 / 4 + j4) * kD + row];
                 bv[4 * j4] = u.x;
                 bv[4 * j4 + 1] = u.y;
                 bv[4 * j4 + 2] = u.z;
