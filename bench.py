@@ -293,6 +293,8 @@ def gpu_arm(args, wl, rank, world):
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         kern_tot = [0.0] * len(plan)
+        if multi and (args.steps > 512 or args.steps * (len(plan) + 1) > 2048):
+            raise SystemExit("--steps: at most 512 calls / 2048 kernel events are timed per run")
         if multi:
             # the library records events between its own launches on `stream`
             ttt.ttt_diag_kernel_timing(True)
@@ -305,14 +307,16 @@ def gpu_arm(args, wl, rank, world):
             starts[k].record(stream)
             call()
             ends[k].record(stream)
-            if multi:
-                for i, ms in enumerate(ttt.ttt_diag_kernel_times(len(plan))):
-                    kern_tot[i] += ms
         torch.cuda.synchronize()
         t1 = time.perf_counter()
         launches = ttt.ttt_launch_count() - n0
         if multi:
+            # summed over the timed calls; read once, after the loop, so the
+            # host never waits on the device inside it
+            kern_tot = ttt.ttt_diag_kernel_times(len(plan))
             ttt.ttt_diag_kernel_timing(False)
+            if len(kern_tot) != len(plan):
+                raise RuntimeError(f"expected {len(plan)} kernels per call, got {len(kern_tot)}")
         barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sum(step_ms)

@@ -57,10 +57,15 @@ TTT_API ttt_status ttt_diag_wait_timeout(unsigned limit_us, ttt_stream stream);
  * entry point records a CUDA event on its stream before its first kernel and
  * after each kernel it launches (events are created on first use on the
  * current device; enabling costs nothing on the device beyond the event
- * records). ttt_diag_kernel_times synchronises on the last event of the most
- * recent call and writes the durations (ms) of that call's kernels, in launch
- * order, to ms[0..max); it returns how many kernels the call launched, or a
- * negative ttt_status. Not thread-safe; meant for benchmarks.
+ * records, and nothing synchronises). Up to 512 calls and 2048 events are kept;
+ * ttt_diag_kernel_timing(enable) clears them. ttt_diag_kernel_times
+ * synchronises on the last event and writes, for each kernel position in
+ * launch order, the sum over the recorded calls of that kernel's duration (ms)
+ * to ms[0..max); it returns how many kernels a call launched (0 when nothing
+ * was recorded), TTT_ERR_ARG when the calls launched different numbers of
+ * kernels, the record overflowed or the calls ran on another device, or
+ * TTT_ERR_LAUNCH when an event query failed. Not thread-safe; meant for
+ * benchmarks.
  */
 TTT_API ttt_status ttt_diag_kernel_timing(int enable);
 TTT_API int ttt_diag_kernel_times(float *ms, int max);

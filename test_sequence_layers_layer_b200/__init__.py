@@ -168,7 +168,8 @@ def ttt_diag_kernel_timing(enable: bool) -> int:
 
 
 def ttt_diag_kernel_times(max_kernels: int = 8) -> list[float]:
-    """Durations (ms) of the kernels of the most recent call (diagnostic)."""
+    """Per kernel position, the summed duration (ms) over the calls recorded since
+    timing was enabled (diagnostic)."""
     buf = (ctypes.c_float * max_kernels)()
     n = lib().ttt_diag_kernel_times(buf, max_kernels)
     if n < 0:

@@ -19,30 +19,56 @@ __device__ int g_device_status;  // set by a kernel whose bounded wait ran out
 static std::atomic<unsigned long long> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
-// Optional per-kernel event timing (diagnostic, see ttt_diag.h).
+// Optional per-kernel event timing (diagnostic, see ttt_diag.h). Marks of
+// every call since timing was enabled are kept, so nothing synchronises until
+// the durations are read.
 namespace {
-constexpr int kMaxMarks = 9;
+constexpr int kMaxMarks = 2048;
+constexpr int kMaxCalls = 512;
 bool g_timing = false;
+bool g_timing_overflow = false;
 int g_timing_dev = -1;
 cudaEvent_t g_marks[kMaxMarks];
+int g_nevents = 0;  // events created so far on g_timing_dev
 int g_nmarks = 0;
+int g_call_start[kMaxCalls];
+int g_ncalls = 0;
 
-void record_mark(cudaStream_t s) {
-    if (!g_timing || g_nmarks >= kMaxMarks) return;
+bool record_mark(cudaStream_t s) {
+    if (!g_timing) return false;
+    if (g_nmarks >= kMaxMarks) {
+        g_timing_overflow = true;
+        return false;
+    }
     int dev = -1;
     cudaGetDevice(&dev);
     if (dev != g_timing_dev) {
-        if (g_timing_dev >= 0) return;  // events belong to another device
-        for (int i = 0; i < kMaxMarks; ++i) cudaEventCreate(&g_marks[i]);
+        if (g_timing_dev >= 0) {  // events belong to another device
+            g_timing_overflow = true;
+            return false;
+        }
         g_timing_dev = dev;
     }
+    if (g_nmarks == g_nevents) {
+        if (cudaEventCreate(&g_marks[g_nevents]) != cudaSuccess) {
+            g_timing_overflow = true;
+            return false;
+        }
+        ++g_nevents;
+    }
     cudaEventRecord(g_marks[g_nmarks++], s);
+    return true;
 }
 }  // namespace
 
 void timing_begin(cudaStream_t s) {
-    g_nmarks = 0;
-    record_mark(s);
+    if (!g_timing) return;
+    if (g_ncalls >= kMaxCalls || g_nmarks >= kMaxMarks) {
+        g_timing_overflow = true;
+        return;
+    }
+    g_call_start[g_ncalls] = g_nmarks;
+    if (record_mark(s)) ++g_ncalls;
 }
 
 void count_launch(cudaStream_t s) {
@@ -270,17 +296,31 @@ unsigned long long ttt_launch_count(void) { return g_launches.load(std::memory_o
 
 ttt_status ttt_diag_kernel_timing(int enable) {
     g_timing = enable != 0;
+    g_timing_overflow = false;
     g_nmarks = 0;
+    g_ncalls = 0;
     return TTT_OK;
 }
 
 int ttt_diag_kernel_times(float *ms, int max) {
-    if (!g_timing || g_nmarks < 1) return 0;
+    if (!g_timing || g_ncalls < 1) return 0;
+    if (g_timing_overflow || !ms || max < 0) return TTT_ERR_ARG;
     if (cudaEventSynchronize(g_marks[g_nmarks - 1]) != cudaSuccess) return TTT_ERR_LAUNCH;
-    const int n = g_nmarks - 1;
-    for (int i = 0; i < n && i < max; ++i)
-        if (cudaEventElapsedTime(&ms[i], g_marks[i], g_marks[i + 1]) != cudaSuccess)
-            return TTT_ERR_LAUNCH;
+    // every call must have launched the same number of kernels
+    const int n = (g_ncalls > 1 ? g_call_start[1] : g_nmarks) - 1;
+    for (int c = 0; c < g_ncalls; ++c) {
+        const int end = c + 1 < g_ncalls ? g_call_start[c + 1] : g_nmarks;
+        if (end - g_call_start[c] - 1 != n) return TTT_ERR_ARG;
+    }
+    for (int i = 0; i < n && i < max; ++i) ms[i] = 0.f;
+    for (int c = 0; c < g_ncalls; ++c)
+        for (int i = 0; i < n && i < max; ++i) {
+            float t = 0.f;
+            const int m = g_call_start[c] + i;
+            if (cudaEventElapsedTime(&t, g_marks[m], g_marks[m + 1]) != cudaSuccess)
+                return TTT_ERR_LAUNCH;
+            ms[i] += t;
+        }
     return n;
 }
 
