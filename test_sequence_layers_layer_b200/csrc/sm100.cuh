@@ -175,6 +175,24 @@ __device__ __forceinline__ void tmem_ld16(uint32_t ta, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Warp-collective load of the first 16 lanes of the subpartition, twice:
+// thread i < 16 receives columns col..col+15 of lane (base lane + i), thread
+// 16 + i the columns col+kSplit..col+kSplit+15 of the same lane. For an
+// M = 64 accumulator (16 lanes per subpartition) this keeps all 32 threads busy.
+template <int kSplit>
+__device__ __forceinline__ void tmem_ld16_x2(uint32_t ta, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(ta), "n"(kSplit));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // Warp-collective 32-lane x 32-bit store of 16 consecutive columns (the
 // mirror of tmem_ld16).
 __device__ __forceinline__ void tmem_st16(uint32_t ta, const float (&v)[16]) {

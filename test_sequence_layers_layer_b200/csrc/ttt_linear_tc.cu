@@ -23,15 +23,15 @@
 // The fp32 state is kept as W^T so that re-emitting it as the bf16 hi/lo
 // operand writes whole 16-byte rows.
 //
-// Warp roles (20 warps):
+// Warp roles (16 warps):
 //   0      TMA producer: K, Q, V in chunks of 64 tokens (4-slot ring)
 //   1      MMA issuer (one thread) and tensor-memory owner
 //   2      stages the product's A tile [Q_{j+1}; K_{j+2}] from the TMA tiles
 //   3      copies the product (tensor-memory subpartition 3) out: P and C for
 //          the scan, Q W and Q K^T into a 4-slot ring for the output warps
 //   4-7    scan: X = P - C G_prev, LayerNorm backward, G (fp32 + bf16 hi/lo)
-//   8-15   W re-emit: fp32 W^T from tensor memory -> bf16 hi/lo operand rows
-//   16-19  output: Zpre = Q W - tril(Q K^T) G, LayerNorm + residual, store Z
+//   8-11   W re-emit: fp32 W^T from tensor memory -> bf16 hi/lo operand rows
+//   12-15  output: Zpre = Q W - tril(Q K^T) G, LayerNorm + residual, store Z
 // Precision: Q/K/V enter exactly (bf16); every other operand (W, G) enters
 // the tensor cores as two bf16 terms hi + lo with fp32 accumulation, and the
 // chain's corrections and all LayerNorm math are fp32.
@@ -63,7 +63,7 @@ using namespace sm100;
 constexpr int kD = 64, kMB = 16;
 constexpr int kChunkTok = 64, kMbPerChunk = kChunkTok / kMB, kSlots = 4;
 constexpr int kTile = kChunkTok * kD * 2;  // 8 KB per tensor per chunk
-constexpr int kThreads = 640;
+constexpr int kThreads = 512;
 constexpr int kBRows = 144;                // W^T hi (64) | W^T lo (64) | K_{j+1} (16)
 
 // Shared memory map (offsets from a 1024-aligned base).
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&pcready[i], 32);
         }
         mbar_init(&wdone, 1);
-        mbar_init(&wsm, 256);
+        mbar_init(&wsm, 128);
         mbar_init(&drain, 1);
         fence_mbar_init();
     }
@@ -474,33 +474,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&gready[j & 3]);
             if (threadIdx.x == 128) TRACE(8, j);
         }
-    } else if (warp >= 8 && warp < 16) {
+    } else if (warp >= 8 && warp < 12) {
         // ------------------------------------------------------------ W re-emit
-        const int q = warp & 3;              // subpartition: W^T rows 16q..16q+15
-        const int half = (warp - 8) >> 2;    // d_in columns 32*half .. +31
+        // Warp 8+q owns W^T rows 16q..16q+15 (tensor-memory subpartition q,
+        // lanes 0-15): thread i < 16 handles d_in columns 0-31 of row 16q+i,
+        // thread 16+i columns 32-63 of the same row.
+        const int q = warp & 3;
+        const int half = lane >> 4;          // d_in columns 32*half .. +31
         const int n = 16 * q + (lane & 15);  // W^T row = d_out index
-        const bool live = lane < 16;
-        const int rt = threadIdx.x - 256;    // 0..255
-        const uint32_t wl = taddr(tm, 32 * q, TM_WT + 32 * half);
+        const int rt = threadIdx.x - 256;    // 0..127
+        const uint32_t wl = taddr(tm, 32 * q, TM_WT);
         // Writes W^T row n, this half's columns, as hi (row n) and lo (row 64+n).
         auto emit = [&](const float (&w)[32]) {
-            if (live) {
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    uint2 h0, l0, h1, l1;
-                    split4(w[8 * c8], w[8 * c8 + 1], w[8 * c8 + 2], w[8 * c8 + 3], h0, l0);
-                    split4(w[8 * c8 + 4], w[8 * c8 + 5], w[8 * c8 + 6], w[8 * c8 + 7], h1, l1);
-                    const int chunk = 4 * half + c8;
-                    *reinterpret_cast<uint4 *>(sB + n * 128 + ((chunk ^ (n & 7)) << 4)) =
-                        make_uint4(h0.x, h0.y, h1.x, h1.y);
-                    *reinterpret_cast<uint4 *>(sB + (64 + n) * 128 + ((chunk ^ (n & 7)) << 4)) =
-                        make_uint4(l0.x, l0.y, l1.x, l1.y);
-                }
+            for (int c8 = 0; c8 < 4; ++c8) {
+                uint2 h0, l0, h1, l1;
+                split4(w[8 * c8], w[8 * c8 + 1], w[8 * c8 + 2], w[8 * c8 + 3], h0, l0);
+                split4(w[8 * c8 + 4], w[8 * c8 + 5], w[8 * c8 + 6], w[8 * c8 + 7], h1, l1);
+                const int chunk = 4 * half + c8;
+                *reinterpret_cast<uint4 *>(sB + n * 128 + ((chunk ^ (n & 7)) << 4)) =
+                    make_uint4(h0.x, h0.y, h1.x, h1.y);
+                *reinterpret_cast<uint4 *>(sB + (64 + n) * 128 + ((chunk ^ (n & 7)) << 4)) =
+                    make_uint4(l0.x, l0.y, l1.x, l1.y);
             }
         };
         // Rows 128-143 of the B tile: K_m (same swizzle phase: 128 = 0 mod 8).
         auto copy_k = [&](int m) {
-            if (rt < 128 && m < NM) {
+            if (m < NM) {
                 const int r = rt >> 3, c = rt & 7;
                 *reinterpret_cast<uint4 *>(sB + (128 + r) * 128 + c * 16) =
                     *reinterpret_cast<const uint4 *>(ring_row(sK, m, r) + c * 16);
@@ -511,12 +511,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? seq : head) * kD * kD;
             float w[32];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) w[k] = live ? W0[(32 * half + k) * kD + n] : 0.f;
+            for (int k = 0; k < 32; ++k) w[k] = W0[(32 * half + k) * kD + n];
+            // 32-lane stores: thread i < 16 writes all 64 columns of lane i
+            // (columns 32-63 from thread 16+i); lanes 16-31 are not used by
+            // the M = 64 accumulator and receive don't-care values.
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 float v[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = w[16 * c + i];
+                for (int i = 0; i < 16; ++i) {
+                    const float mine = w[16 * (c & 1) + i];
+                    const float up = __shfl_down_sync(0xffffffffu, mine, 16);
+                    v[i] = c < 2 ? mine : up;
+                }
                 tmem_st16(wl + 16 * c, v);
             }
             tmem_st_wait();
@@ -528,28 +535,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int j = 0; ok && j < NM; ++j) {
             if (!mbar_wait_warp(&wdone, j & 1, abrt, status, 52)) break;
-            if (lane == 0 && half == 0) TRACE(9 + q, j);
+            if (lane == 0) TRACE(9 + q, j);
             tc_fence_after();
             float w[32];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 float v[16];
-                tmem_ld16(wl + 16 * c, v);
+                tmem_ld16_x2<32>(wl + 16 * c, v);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) w[16 * c + i] = v[i];
             }
             tmem_ld_wait();
-            if (lane == 0 && half == 0 && q == 0) TRACE(19, j);
+            if (lane == 0 && q == 0) TRACE(19, j);
             if (j + 1 < NM) {
                 if ((j + 1) % kMbPerChunk == 0 && !chunk_wait(j + 1, 53)) break;
                 emit(w);
                 copy_k(j + 1);
-                if (lane == 0 && half == 0 && q == 0) TRACE(20, j);
+                if (lane == 0 && q == 0) TRACE(20, j);
                 fence_async_smem();
                 tc_fence_before();
                 mbar_arrive(&wsm);
-                if (lane == 0 && half == 0) TRACE(13 + q, j);
-            } else if (a.W_out && live) {
+                if (lane == 0) TRACE(13 + q, j);
+            } else if (a.W_out) {
                 float *dst = a.W_out + (size_t)seq * kD * kD + n;
 #pragma unroll
                 for (int k = 0; k < 32; ++k) dst[(32 * half + k) * kD] = w[k];
@@ -557,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ output
-        const int r = threadIdx.x - 512, t = r >> 3, g = r & 7;
+        const int r = threadIdx.x - 384, t = r >> 3, g = r & 7;
         float gam[8], bet[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -602,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float *zo = a.Z + (tok0 + (long)m * kMB + t) * kD;
             *reinterpret_cast<float4 *>(zo + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
             *reinterpret_cast<float4 *>(zo + 32 + 4 * g) = make_float4(out[4], out[5], out[6], out[7]);
-            if (threadIdx.x == 512) TRACE(17, m);
+            if (threadIdx.x == 384) TRACE(17, m);
         }
     }
     // ---------------------------------------------------------------- teardown
