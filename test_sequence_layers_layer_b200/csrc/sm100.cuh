@@ -60,15 +60,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // records it and unwinds instead of hanging the GPU.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-// Waits for phase `parity` of the mbarrier to complete. On timeout sets
-// *abort (shared flag seen by the whole block), records `code` in the
-// device status word and returns false. Returns false at once if another
-// thread already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int *status, int code,
-                                          uint64_t limit_ns = kWaitLimitNs) {
-    const uint32_t a = smem_u32(bar);
-    if (mbar_try_wait(a, parity)) return true;
+// Retry loop of mbar_wait, kept out of line: the first try_wait (which parks
+// the warp until the phase completes) nearly always succeeds, and inlining
+// the loop at every wait site would multiply the kernels' code size.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity,
+                                                   volatile int *abort, int *status, int code,
+                                                   uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(a, parity)) return true;
@@ -81,6 +78,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
             }
         }
     }
+}
+
+// Waits for phase `parity` of the mbarrier to complete. On timeout sets
+// *abort (shared flag seen by the whole block), records `code` in the
+// device status word and returns false. Returns false at once if another
+// thread already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          int *status, int code,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    return mbar_wait_slow(a, parity, abort, status, code, limit_ns);
 }
 
 // Arrive and add `bytes` to the transaction count the phase waits for.
