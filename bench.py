@@ -17,6 +17,7 @@ Prints one JSON line (rank 0).
 from __future__ import annotations
 
 import argparse
+import glob
 import hashlib
 import json
 import os
@@ -101,9 +102,14 @@ def kernel_plan(wl):
 
 
 def source_sha(fname: str) -> str:
-    path = os.path.join(ROOT, "test_sequence_layers_layer_b200", "csrc", fname)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of a kernel's source file together with the device headers (.cuh)
+    beside it, so that a recorded ncu figure goes stale when either changes."""
+    csrc = os.path.join(ROOT, "test_sequence_layers_layer_b200", "csrc")
+    h = hashlib.sha256()
+    for path in [os.path.join(csrc, fname)] + sorted(glob.glob(os.path.join(csrc, "*.cuh"))):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str, sha: str):
