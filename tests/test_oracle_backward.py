@@ -1,0 +1,109 @@
+"""Pins of the backward oracle (oracle/backward.py) to things other than itself:
+its forward against the C oracle's token-by-token forward, its outer gradients
+against central finite differences (torch.autograd.gradcheck), and special
+cases the method fixes (eta = 0 freezes the weight, so Z cannot depend on K
+or V)."""
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import oracle  # noqa: E402
+from oracle import backward as ob  # noqa: E402
+
+
+def _inputs(seed, B, H, T, d, *, w0_per_seq=False, eta_scale=0.1):
+    r = np.random.default_rng(seed)
+    Q, K, V = (r.standard_normal((B, H, T, d)) for _ in range(3))
+    eta = eta_scale * r.uniform(0.2, 1.0, (B, H, T))
+    W0 = r.standard_normal((B, H, d, d) if w0_per_seq else (H, d, d)) / np.sqrt(d)
+    gamma = 1.0 + 0.2 * r.standard_normal((H, d))
+    beta = 0.2 * r.standard_normal((H, d))
+    return Q, K, V, eta, W0, gamma, beta
+
+
+@pytest.mark.parametrize("ln,b,w0_per_seq", [(True, 4, False), (False, 4, False), (True, 1, True),
+                                             (True, 8, False)])
+def test_forward_matches_c_oracle(ln, b, w0_per_seq):
+    Q, K, V, eta, W0, gamma, beta = _inputs(1, 2, 2, 16, 8, w0_per_seq=w0_per_seq)
+    Z, Wo = ob.linear_forward_np(Q, K, V, eta, W0, gamma, beta, b=b, ln=ln)
+    Zc, Woc = oracle.linear_primal(Q, K, V, eta, W0, gamma if ln else None, beta if ln else None,
+                                   b=b, ln=ln, w0_per_seq=w0_per_seq)
+    assert np.abs(Z - Zc).max() <= 1e-12 * max(1.0, np.abs(Zc).max())
+    assert np.abs(Wo - Woc).max() <= 1e-12 * max(1.0, np.abs(Woc).max())
+
+
+@pytest.mark.parametrize("ln", [True, False])
+def test_inner_gradient_matches_c_closed_form(ln):
+    """The autograd inner gradient used by the oracle's forward equals the C
+    oracle's closed-form k^T dl/dx."""
+    r = np.random.default_rng(5)
+    d = 6
+    k, v = r.standard_normal(d), r.standard_normal(d)
+    W = r.standard_normal((d, d)) / np.sqrt(d)
+    gamma, beta = 1.0 + 0.3 * r.standard_normal(d), 0.3 * r.standard_normal(d)
+    Wt = torch.tensor(W, requires_grad=True)
+    kt, vt = torch.tensor(k), torch.tensor(v)
+    x = kt @ Wt
+    f = kt + torch.nn.functional.layer_norm(x, (d,), eps=ob.LN_EPS) * torch.tensor(gamma) \
+        + torch.tensor(beta) if ln else x
+    g = torch.autograd.grad(0.5 * ((f - vt) ** 2).sum(), Wt)[0].numpy()
+    Gc = oracle.grad_linear(k, v, W, gamma if ln else None, beta if ln else None, ln=ln)
+    assert np.abs(g - Gc).max() <= 1e-12 * np.abs(Gc).max()
+
+
+@pytest.mark.parametrize("ln", [True, False])
+def test_gradients_match_finite_differences(ln):
+    """gradcheck: autograd through the unrolled inner loop (a gradient of a
+    gradient) against central differences, for every input at once."""
+    Q, K, V, eta, W0, gamma, beta = _inputs(2, 1, 1, 6, 3, eta_scale=0.5)
+    ts = [torch.tensor(a, requires_grad=True) for a in (Q, K, V, eta, W0, gamma, beta)]
+    r = np.random.default_rng(3)
+    dZ = torch.tensor(r.standard_normal(Q.shape))
+    dW = torch.tensor(r.standard_normal((1, 1, 3, 3)))
+
+    def fn(*a):
+        Z, Wo = ob.linear_forward(*a, b=2, ln=ln)
+        return (Z * dZ).sum() + (Wo * dW).sum()
+
+    inputs = tuple(ts if ln else ts[:5])
+    if not ln:
+        g0, b0 = ts[5].detach(), ts[6].detach()
+        fn_noln = lambda *a: fn(*a, g0, b0)  # noqa: E731
+        assert torch.autograd.gradcheck(fn_noln, inputs, eps=1e-6, atol=1e-7, rtol=1e-6)
+    else:
+        assert torch.autograd.gradcheck(fn, inputs, eps=1e-6, atol=1e-7, rtol=1e-6)
+
+
+def test_linear_grads_equal_gradcheck_function():
+    """linear_grads (the entry the GPU tests use) returns what autograd of the
+    same scalar gives, key by key, and a zero dW_out equals no dW_out."""
+    Q, K, V, eta, W0, gamma, beta = _inputs(4, 1, 2, 8, 4)
+    r = np.random.default_rng(6)
+    dZ = r.standard_normal(Q.shape)
+    g1 = ob.linear_grads(Q, K, V, eta, W0, gamma, beta, dZ, None, b=4, ln=True)
+    g2 = ob.linear_grads(Q, K, V, eta, W0, gamma, beta, dZ, np.zeros((1, 2, 4, 4)), b=4, ln=True)
+    for n in g1:
+        assert np.array_equal(g1[n], g2[n])
+    assert set(g1) == {"Q", "K", "V", "eta", "W0", "gamma", "beta"}
+
+
+def test_eta_zero_freezes_weight_so_k_and_v_get_no_gradient():
+    """With eta = 0 the weight never moves, so Z depends on Q, W0, gamma and beta
+    only: dK = dV = 0 exactly, dW_out flows straight to dW0, and deta is the
+    first-order effect of each token's step (nonzero)."""
+    Q, K, V, eta, W0, gamma, beta = _inputs(7, 1, 1, 8, 4, eta_scale=0.0)
+    r = np.random.default_rng(8)
+    dZ = r.standard_normal(Q.shape)
+    dW = r.standard_normal((1, 1, 4, 4))
+    g = ob.linear_grads(Q, K, V, eta, W0, gamma, beta, dZ * 0.0, dW, b=4, ln=True)
+    assert np.abs(g["K"]).max() == 0.0 and np.abs(g["V"]).max() == 0.0
+    assert np.allclose(g["W0"][0], dW[0, 0], rtol=0, atol=1e-15)
+    g = ob.linear_grads(Q, K, V, eta, W0, gamma, beta, dZ, None, b=4, ln=True)
+    assert np.abs(g["K"]).max() == 0.0 and np.abs(g["V"]).max() == 0.0
+    assert np.abs(g["eta"]).max() > 0.0
