@@ -116,6 +116,37 @@ TTT_API ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, c
                           ttt_dtype dt, unsigned flags, ttt_stream stream);
 
 /*
+ * TTT-Linear backward: the outer gradients of the forward above ("Key
+ * Architectural Mechanics of TTT-Linear", parts 1-4; the inner loop is
+ * differentiated through, weight updates included). Given dZ = dL/dZ and,
+ * optionally, dW_out = dL/dW_out, writes dL/d of every input:
+ *   dQ, dK, dV  [B][H][T][d] fp32
+ *   deta        [B][H][T] fp32
+ *   dW0         [H][d][d] fp32, summed over the batch (or [B][H][d][d] with
+ *               TTT_F_W0_PER_SEQ)
+ *   dgamma, dbeta  [H][d] fp32, summed over the batch; required with
+ *               TTT_F_LN, ignored (may be NULL) without
+ * Inputs as ttt_linear_fwd, plus dZ [B][H][T][d] fp32 (required) and dW_out
+ * [B][H][d][d] fp32 or NULL (taken as zero). The kernel first re-runs the
+ * forward to checkpoint each mini-batch's starting weight, then walks the
+ * mini-batches in reverse; the workspace (device memory, 256-byte aligned, at
+ * least ttt_linear_bwd_workspace_bytes() bytes, owned by the caller and free
+ * to reuse after the stream has passed the call) holds those checkpoints.
+ * Outputs are overwritten, never accumulated into. fp32 CUDA cores for both
+ * TTT_FP32 and TTT_BF16 inputs; deterministic (fixed summation order).
+ * Supported: T % b == 0, 1 <= d <= 64, 1 <= b with b*d <= 1024. Errors as
+ * ttt_linear_fwd, plus TTT_ERR_WORKSPACE.
+ */
+TTT_API size_t ttt_linear_bwd_workspace_bytes(int B, int H, int T, int d, int b);
+TTT_API ttt_status ttt_linear_bwd(const void *Q, const void *K, const void *V, const float *eta,
+                                  const float *W0, const float *ln_gamma, const float *ln_beta,
+                                  const float *dZ, const float *dW_out, float *dQ, float *dK,
+                                  float *dV, float *deta, float *dW0, float *dgamma,
+                                  float *dbeta, int B, int H, int T, int d, int b, ttt_dtype dt,
+                                  unsigned flags, void *workspace, size_t workspace_bytes,
+                                  ttt_stream stream);
+
+/*
  * TTT-MLP forward: f(k) = k + LN(GELU(k W1) W2) with W1 [d][dh], W2 [dh][d],
  * GELU the exact erf form; same mini-batch rule as ttt_linear_fwd, with both
  * layers updated ("How to Master Test-Time Training for LLMs": the hidden

@@ -1,5 +1,5 @@
-"""Python binding of libttt.so, the B200 library for the forward pass of a
-Test-Time-Training (TTT) layer.
+"""Python binding of libttt.so, the B200 library for a Test-Time-Training (TTT)
+layer: its forward pass, and the backward pass of TTT-Linear.
 
 The functions named like the C ABI (ttt_linear_fwd, ttt_mlp_fwd,
 ttt_chunk_fwd, ...) take exactly the C arguments; a pointer argument may be a
@@ -50,6 +50,10 @@ def lib() -> ctypes.CDLL:
         L.ttt_status_string.argtypes = [_I]
         L.ttt_linear_fwd.restype = _I
         L.ttt_linear_fwd.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_uint, _P]
+        L.ttt_linear_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.ttt_linear_bwd_workspace_bytes.argtypes = [_I] * 5
+        L.ttt_linear_bwd.restype = _I
+        L.ttt_linear_bwd.argtypes = [_P] * 16 + [_I] * 6 + [ctypes.c_uint, _P, ctypes.c_size_t, _P]
         L.ttt_mlp_fwd.restype = _I
         L.ttt_mlp_fwd.argtypes = [_P] * 11 + [_I] * 7 + [ctypes.c_uint, _P]
         L.ttt_chunk_workspace_bytes.restype = ctypes.c_size_t
@@ -124,6 +128,20 @@ def ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                               _ptr(ln_beta), _ptr(Z), _ptr(W_out), B, H, T, d, b, dt, flags,
                               _stream(stream))
     return _check("ttt_linear_fwd", rc) if check else rc
+
+
+def ttt_linear_bwd_workspace_bytes(B, H, T, d, b) -> int:
+    return int(lib().ttt_linear_bwd_workspace_bytes(B, H, T, d, b))
+
+
+def ttt_linear_bwd(Q, K, V, eta, W0, ln_gamma, ln_beta, dZ, dW_out, dQ, dK, dV, deta, dW0, dgamma,
+                   dbeta, B, H, T, d, b, dt, flags, workspace, workspace_bytes, stream=None,
+                   check=True):
+    rc = lib().ttt_linear_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(ln_gamma),
+                              _ptr(ln_beta), _ptr(dZ), _ptr(dW_out), _ptr(dQ), _ptr(dK), _ptr(dV),
+                              _ptr(deta), _ptr(dW0), _ptr(dgamma), _ptr(dbeta), B, H, T, d, b, dt,
+                              flags, _ptr(workspace), workspace_bytes, _stream(stream))
+    return _check("ttt_linear_bwd", rc) if check else rc
 
 
 def ttt_mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out, B, H, T, d, dh,
@@ -219,6 +237,31 @@ def linear_fwd(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, w0_per_s
     ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                    _dtype_code(Q), flags, stream)
     return Z, W_out
+
+
+def linear_bwd(Q, K, V, eta, W0, ln_gamma, ln_beta, dZ, dW_out=None, *, b, ln, w0_per_seq=False,
+               workspace=None, stream=None):
+    """TTT-Linear backward. Returns a dict of fp32 cuda tensors: Q, K, V, eta,
+    W0 and (with ln) gamma, beta -- the gradients of sum(Z * dZ) +
+    sum(W_out * dW_out). Allocates the workspace with torch unless one is given."""
+    import torch
+    B, H, T, d = Q.shape
+    dev = Q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    need = ttt_linear_bwd_workspace_bytes(B, H, T, d, b)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    g = dict(Q=torch.empty((B, H, T, d), **f32), K=torch.empty((B, H, T, d), **f32),
+             V=torch.empty((B, H, T, d), **f32), eta=torch.empty((B, H, T), **f32),
+             W0=torch.empty(tuple(W0.shape), **f32))
+    if ln:
+        g["gamma"] = torch.empty((H, d), **f32)
+        g["beta"] = torch.empty((H, d), **f32)
+    flags = (TTT_F_LN if ln else 0) | (TTT_F_W0_PER_SEQ if w0_per_seq else 0)
+    ttt_linear_bwd(Q, K, V, eta, W0, ln_gamma, ln_beta, dZ, dW_out, g["Q"], g["K"], g["V"],
+                   g["eta"], g["W0"], g.get("gamma"), g.get("beta"), B, H, T, d, b, _dtype_code(Q),
+                   flags, workspace, workspace.numel() * workspace.element_size(), stream)
+    return g
 
 
 def mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, *, b, w0_per_seq=False, stream=None,

@@ -208,6 +208,43 @@ ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const flo
                                                                 : launch_linear_simt(a, cs));
 }
 
+size_t ttt_linear_bwd_workspace_bytes(int B, int H, int T, int d, int b) {
+    return linear_bwd_workspace_bytes(B, H, T, d, b);
+}
+
+ttt_status ttt_linear_bwd(const void *Q, const void *K, const void *V, const float *eta,
+                          const float *W0, const float *ln_gamma, const float *ln_beta,
+                          const float *dZ, const float *dW_out, float *dQ, float *dK, float *dV,
+                          float *deta, float *dW0, float *dgamma, float *dbeta, int B, int H,
+                          int T, int d, int b, ttt_dtype dt, unsigned flags, void *workspace,
+                          size_t workspace_bytes, ttt_stream stream) {
+    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ)) return TTT_ERR_ARG;
+    const bool ln = flags & TTT_F_LN;
+    if (!Q || !K || !V || !eta || !W0 || !dZ || !dQ || !dK || !dV || !deta || !dW0)
+        return TTT_ERR_PTR;
+    if (ln && (!ln_gamma || !ln_beta || !dgamma || !dbeta)) return TTT_ERR_PTR;
+    if (B <= 0 || H <= 0 || T <= 0 || b <= 0 || T % b != 0 || !linear_bwd_supported(d, b))
+        return TTT_ERR_SHAPE;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return TTT_ERR_SHAPE;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
+    const size_t need = linear_bwd_workspace_bytes(B, H, T, d, b);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return TTT_ERR_WORKSPACE;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {Q, K, V, eta, W0, ln ? ln_gamma : nullptr, ln ? ln_beta : nullptr, dZ,
+                          dW_out, dQ, dK, dV, deta, dW0, ln ? dgamma : nullptr,
+                          ln ? dbeta : nullptr, workspace};
+    st = check_device_ptrs(ptrs, 17);
+    if (st != TTT_OK) return st;
+    LinearBwdArgs a{Q, K, V, eta, W0, ln_gamma, ln_beta, dZ, dW_out, dQ, dK, dV, deta, dW0,
+                    dgamma, dbeta, B, H, T, d, b, dt == TTT_BF16, ln,
+                    (flags & TTT_F_W0_PER_SEQ) != 0, workspace};
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    return launched(launch_linear_bwd(a, cs));
+}
+
 ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float *eta,
                        const float *W1_0, const float *W2_0, const float *ln_gamma,
                        const float *ln_beta, float *Z, float *W1_out, float *W2_out, int B,

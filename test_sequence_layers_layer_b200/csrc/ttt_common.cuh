@@ -38,6 +38,19 @@ struct ChunkArgs {
     size_t workspace_bytes;
 };
 
+// TTT-Linear backward (outer gradients), fp32 CUDA cores.
+struct LinearBwdArgs {
+    const void *Q, *K, *V;
+    const float *eta, *W0, *gamma, *beta, *dZ, *dW_out;
+    float *dQ, *dK, *dV, *deta, *dW0, *dgamma, *dbeta;
+    int B, H, T, d, b;
+    bool bf16, ln, w0_per_seq;
+    void *workspace;
+};
+bool linear_bwd_supported(int d, int b);
+size_t linear_bwd_workspace_bytes(int B, int H, int T, int d, int b);
+cudaError_t launch_linear_bwd(const LinearBwdArgs &a, cudaStream_t s);
+
 // Launchers return cudaSuccess or the launch error.
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s);
 cudaError_t launch_mlp_simt(const MlpArgs &a, cudaStream_t s);
