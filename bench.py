@@ -544,6 +544,124 @@ def decode_arm(args, wl):
     }
 
 
+# fp32 FMA lanes of a B200 (148 SMs x 128 lanes, 2 FLOP per FMA) at the SM clock:
+# the peak of a kernel bound by plain fp32 arithmetic on CUDA cores.
+FP32_LANES = 148 * 128
+
+
+def bwd_flops_per_token(d: int) -> float:
+    """Algorithmic FLOPs of the TTT-Linear backward per token: the forward
+    re-run (k W, and the K^T G update: 4 d^2) and the reverse step (k W and q W,
+    dzpre W^T, G Om^T, k Om, dx W^T, and the two weight-gradient outer products:
+    16 d^2); the O(b d) causal terms are left out."""
+    return 20.0 * d * d
+
+
+def bwd_bytes_per_token(wl) -> float:
+    """Algorithmic HBM bytes per token: Q, K, V in once, dZ and eta in, dQ, dK,
+    dV and deta out (the W_m checkpoints are the kernel's choice, not counted)."""
+    e = 2 if wl.dtype == "bf16" else 4
+    return 3 * wl.d * e + 4 * wl.d + 4 + 3 * 4 * wl.d + 4
+
+
+def backward_arm(args, wl):
+    """TTT-Linear backward (`--backward`): ttt_linear_bwd on the workload's
+    inputs with a seeded dZ, all resident in HBM, L2 flushed between steps."""
+    import torch
+    import test_sequence_layers_layer_b200 as ttt
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    ttt.lib()
+    inp = synth.make_inputs(wl)
+    x = device_tensors(inp, dev)
+    rng = np.random.default_rng(wl.seed + 101)
+    dZ = torch.from_numpy(rng.standard_normal((wl.B, wl.H, wl.T, wl.d)).astype(np.float32)).to(dev)
+    need = ttt.ttt_linear_bwd_workspace_bytes(wl.B, wl.H, wl.T, wl.d, wl.b)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = [torch.empty((wl.B, wl.H, wl.T, wl.d), **f32) for _ in range(3)]
+    geta = torch.empty((wl.B, wl.H, wl.T), **f32)
+    gW0 = torch.empty(tuple(x["W1"].shape), **f32)
+    gg, gb = torch.empty((wl.H, wl.d), **f32), torch.empty((wl.H, wl.d), **f32)
+    dt = ttt.TTT_BF16 if wl.dtype == "bf16" else ttt.TTT_FP32
+    flags = ttt.TTT_F_LN if wl.ln else 0
+    stream = torch.cuda.Stream(dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def call():
+        ttt.ttt_linear_bwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"], dZ,
+                           None, *g, geta, gW0, gg, gb, wl.B, wl.H, wl.T, wl.d, wl.b, dt, flags, ws,
+                           need, stream.cuda_stream)
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            call()
+        stream.synchronize()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ttt.ttt_diag_kernel_timing(True)
+        n0 = ttt.ttt_launch_count()
+        t0 = time.perf_counter()
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record(stream)
+            call()
+            ends[k].record(stream)
+        torch.cuda.synchronize()
+        t1 = time.perf_counter()
+        launches = ttt.ttt_launch_count() - n0
+        kern = ttt.ttt_diag_kernel_times(8)
+        ttt.ttt_diag_kernel_timing(False)
+    sampler.stop()
+    if ttt.ttt_device_status(stream.cuda_stream) != 0:
+        raise RuntimeError("device status error in the timed region")
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    ms = sum(step_ms) / args.steps
+    kern_ms = kern[0] / args.steps
+    clocks = sampler.summary(t0, t1)
+    mhz = clocks.get("sm_mhz") or 1965
+    peak = FP32_LANES * 2 * mhz * 1e6 / 1e12
+    flop = bwd_flops_per_token(wl.d) * wl.tokens
+    achieved = flop / (kern_ms / 1e3) / 1e12
+    line = {
+        "metric": "TTT-Linear backward tokens/sec at 1 B200 (outer gradients of every input)",
+        "value": wl.tokens / (ms / 1e3), "unit": "tokens/s", "higher_is_better": True,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "dtype": "f32", "data": "synthetic (seeded SplitMix64 normals; bf16-rounded Q/K/V; normal dZ)",
+        "config": {"workload": wl.name + "_backward", "B": wl.B, "H": wl.H, "T": wl.T, "d": wl.d,
+                   "mini_batch": wl.b, "layer_norm": wl.ln, "qkv_dtype": wl.dtype,
+                   "l2": "flushed between steps (256 MiB write)"},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "linear_bwd_kernel",
+                     "peak_source": f"derived: {FP32_LANES} fp32 lanes x 2 FLOP x {mhz} MHz",
+                     "algorithmic_per_launch": flop, "kernel_ms": kern_ms,
+                     "hbm_bytes_per_token": bwd_bytes_per_token(wl)},
+        "kernels": [{"name": n, "ms_per_launch": t / args.steps} for n, t in
+                    zip(["linear_bwd_kernel", "sum_over_batch_kernel (dW0)",
+                         "sum_over_batch_kernel (dgamma)", "sum_over_batch_kernel (dbeta)"], kern)],
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "step_ms_min_median": [min(step_ms), statistics.median(step_ms)],
+    }
+    if not args.no_cpu_baseline:
+        from oracle import backward as ob
+        sub = wl.scaled(B=1, H=1, T=min(wl.T, 512))
+        si = synth.make_inputs(sub)
+        dz = rng.standard_normal((1, 1, sub.T, sub.d))
+        t0 = time.perf_counter()
+        ob.linear_grads(si.Q, si.K, si.V, si.eta, si.W1, si.gamma, si.beta, dz, None, b=sub.b,
+                        ln=sub.ln)
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": sub.T / el, "unit": "tokens/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"1 sequence, T={sub.T}: float64 autograd backward"}
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -554,6 +672,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the TTT-Linear backward (linear workloads) instead")
     ap.add_argument("--decode", type=int, default=0,
                     help="time N single-token decode steps (linear workloads) instead")
     ap.add_argument("--B", type=int, default=None,
@@ -566,6 +686,13 @@ def main():
         wl = wl.scaled(B=args.B, name=f"{wl.name}_B{args.B}")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+
+    if args.backward:
+        if wl.kind != "linear":
+            ap.error("--backward times the linear workloads")
+        if rank == 0:
+            print(json.dumps(backward_arm(args, wl)), flush=True)
+        return
 
     if args.decode:
         if wl.kind != "linear":
