@@ -134,7 +134,7 @@ TTT_API ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, c
  * to reuse after the stream has passed the call) holds those checkpoints.
  * Outputs are overwritten, never accumulated into. fp32 CUDA cores for both
  * TTT_FP32 and TTT_BF16 inputs; deterministic (fixed summation order).
- * Supported: T % b == 0, 1 <= d <= 64, 1 <= b with b*d <= 1024. Errors as
+ * Supported: T % b == 0, d in {16, 32, 64}, 1 <= b with b*d <= 1024. Errors as
  * ttt_linear_fwd, plus TTT_ERR_WORKSPACE.
  */
 TTT_API size_t ttt_linear_bwd_workspace_bytes(int B, int H, int T, int d, int b);

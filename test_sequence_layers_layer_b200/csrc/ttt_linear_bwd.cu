@@ -170,13 +170,94 @@ __device__ __forceinline__ void inner_token(const Smem &S, int s, int d, bool ln
     if (lane == 0) S.sig[s] = sig;
 }
 
-template <typename TIn>
+// Register-blocked products of the block (D = d, compile time). In a b x D
+// product, thread (row group rg = tid / D, column c = tid % D) owns rows
+// rg + RG k (k < 4) of column c and reads the row operand as float4
+// broadcasts; in a D x D weight update it owns rows a0 .. a0 + WR - 1 of
+// column c. Matrices W and Om have row stride D + 1.
+template <int D>
+struct Blk {
+    static constexpr int RG = kBwdThreads / D;  // row groups: 16, 8, 4
+    static constexpr int WR = D / RG;           // weight rows per thread: 1, 4, 16
+    static constexpr int P = D + 1;
+    int c, rg, b;
+
+    __device__ __forceinline__ int row(int k) const { return rg + RG * k; }
+
+    // acc[k] = sum_i A[r_k][i] B[i][c]          (B row stride D + 1)
+    __device__ __forceinline__ void ab(const float *A, const float *B, float (&acc)[4]) const {
+        for (int i = 0; i < D; i += 4) {
+            const float b0 = B[i * P + c], b1 = B[(i + 1) * P + c], b2 = B[(i + 2) * P + c],
+                        b3 = B[(i + 3) * P + c];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (row(k) < b) {
+                    const float4 x = *reinterpret_cast<const float4 *>(A + row(k) * D + i);
+                    acc[k] = fmaf(x.x, b0, fmaf(x.y, b1, fmaf(x.z, b2, fmaf(x.w, b3, acc[k]))));
+                }
+        }
+    }
+    // acc[k] = sum_j A[r_k][j] B[c][j]          (B row stride D + 1)
+    __device__ __forceinline__ void abt(const float *A, const float *B, float (&acc)[4]) const {
+        for (int j = 0; j < D; j += 4) {
+            const float b0 = B[c * P + j], b1 = B[c * P + j + 1], b2 = B[c * P + j + 2],
+                        b3 = B[c * P + j + 3];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (row(k) < b) {
+                    const float4 x = *reinterpret_cast<const float4 *>(A + row(k) * D + j);
+                    acc[k] = fmaf(x.x, b0, fmaf(x.y, b1, fmaf(x.z, b2, fmaf(x.w, b3, acc[k]))));
+                }
+        }
+    }
+    // M[a][c] += sum_s X[s][a] Y[s][c] (+ X2[s][a] Y2[s][c]) for a in a0 .. a0 + WR - 1
+    __device__ __forceinline__ void outer(float *M, const float *X, const float *Y, const float *X2,
+                                          const float *Y2) const {
+        const int a0 = rg * WR;
+        float acc[WR];
+#pragma unroll
+        for (int k = 0; k < WR; ++k) acc[k] = M[(a0 + k) * P + c];
+        for (int s = 0; s < b; ++s) {
+            const float y = Y[s * D + c], y2 = X2 ? Y2[s * D + c] : 0.f;
+            if constexpr (WR >= 4) {
+#pragma unroll
+                for (int k = 0; k < WR; k += 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(X + s * D + a0 + k);
+                    acc[k] = fmaf(x.x, y, acc[k]);
+                    acc[k + 1] = fmaf(x.y, y, acc[k + 1]);
+                    acc[k + 2] = fmaf(x.z, y, acc[k + 2]);
+                    acc[k + 3] = fmaf(x.w, y, acc[k + 3]);
+                    if (X2) {
+                        const float4 z = *reinterpret_cast<const float4 *>(X2 + s * D + a0 + k);
+                        acc[k] = fmaf(z.x, y2, acc[k]);
+                        acc[k + 1] = fmaf(z.y, y2, acc[k + 1]);
+                        acc[k + 2] = fmaf(z.z, y2, acc[k + 2]);
+                        acc[k + 3] = fmaf(z.w, y2, acc[k + 3]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < WR; ++k) {
+                    acc[k] = fmaf(X[s * D + a0 + k], y, acc[k]);
+                    if (X2) acc[k] = fmaf(X2[s * D + a0 + k], y2, acc[k]);
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < WR; ++k) M[(a0 + k) * P + c] = acc[k];
+    }
+};
+
+template <typename TIn, int D>
 __global__ void __launch_bounds__(kBwdThreads) linear_bwd_kernel(BwdArgs a) {
     extern __shared__ float smem_f[];
-    const int d = a.d, b = a.b, bd = b * d, dp1 = d + 1;
+    constexpr int dp1 = D + 1, d = D;
+    const int b = a.b, bd = b * d;
     const Smem S = carve(smem_f, d, b);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int seq = blockIdx.x, head = seq % a.H, M = a.T / b;
+    const Blk<D> bk{tid % D, tid / D, b};
+    const int c = bk.c;
     const size_t tok0 = (size_t)seq * a.T;
     const TIn *Qg = static_cast<const TIn *>(a.Q), *Kg = static_cast<const TIn *>(a.K),
               *Vg = static_cast<const TIn *>(a.V);
@@ -202,21 +283,20 @@ __global__ void __launch_bounds__(kBwdThreads) linear_bwd_kernel(BwdArgs a) {
         }
         for (int s = tid; s < b; s += kBwdThreads) S.eta[s] = a.eta[r0 + s];
         __syncthreads();
-        for (int e = tid; e < bd; e += kBwdThreads) {  // x = K W
-            const int s = e / d, j = e % d;
-            float acc = 0.f;
-            for (int i = 0; i < d; ++i) acc = fmaf(S.K[s * d + i], S.W[i * dp1 + j], acc);
-            S.Xh[e] = acc;
+        {  // x = K W
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            bk.ab(S.K, S.W, acc);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (bk.row(k) < b) S.Xh[bk.row(k) * d + c] = acc[k];
         }
         __syncthreads();
         for (int s = warp; s < b; s += kWarps) inner_token(S, s, d, a.ln, lane);
         __syncthreads();
-        for (int e = tid; e < d * d; e += kBwdThreads) {  // W -= K^T G
-            const int i = e / d, j = e % d;
-            float acc = 0.f;
-            for (int s = 0; s < b; ++s) acc = fmaf(S.K[s * d + i], S.G[s * d + j], acc);
-            S.W[i * dp1 + j] -= acc;
-        }
+        // W -= K^T G  (as W += K^T (-G): negate G in place first)
+        for (int e = tid; e < bd; e += kBwdThreads) S.G[e] = -S.G[e];
+        __syncthreads();
+        bk.outer(S.W, S.K, S.G, nullptr, nullptr);
         __syncthreads();
     }
 
@@ -234,23 +314,27 @@ __global__ void __launch_bounds__(kBwdThreads) linear_bwd_kernel(BwdArgs a) {
         }
         for (int s = tid; s < b; s += kBwdThreads) S.eta[s] = a.eta[r0 + s];
         __syncthreads();
-        // x = K W and q W; A_ts = q_t . k_s (s <= t)
-        for (int e = tid; e < bd; e += kBwdThreads) {
-            const int s = e / d, j = e % d;
-            float x = 0.f, y = 0.f;
-            for (int i = 0; i < d; ++i) {
-                const float w = S.W[i * dp1 + j];
-                x = fmaf(S.K[s * d + i], w, x);
-                y = fmaf(S.Q[s * d + i], w, y);
-            }
-            S.Xh[e] = x;
-            S.Y[e] = y;
+        {  // x = K W and q W
+            float x[4] = {0.f, 0.f, 0.f, 0.f}, y[4] = {0.f, 0.f, 0.f, 0.f};
+            bk.ab(S.K, S.W, x);
+            bk.ab(S.Q, S.W, y);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (bk.row(k) < b) {
+                    S.Xh[bk.row(k) * d + c] = x[k];
+                    S.Y[bk.row(k) * d + c] = y[k];
+                }
         }
+        // A_ts = q_t . k_s (s <= t)
         for (int e = tid; e < b * b; e += kBwdThreads) {
             const int t = e / b, s = e % b;
             float acc = 0.f;
             if (s <= t)
-                for (int i = 0; i < d; ++i) acc = fmaf(S.Q[t * d + i], S.K[s * d + i], acc);
+                for (int i = 0; i < d; i += 4) {
+                    const float4 u = *reinterpret_cast<const float4 *>(S.Q + t * d + i);
+                    const float4 v = *reinterpret_cast<const float4 *>(S.K + s * d + i);
+                    acc = fmaf(u.x, v.x, fmaf(u.y, v.y, fmaf(u.z, v.z, fmaf(u.w, v.w, acc))));
+                }
             S.A[e] = acc;
         }
         __syncthreads();
@@ -316,7 +400,11 @@ __global__ void __launch_bounds__(kBwdThreads) linear_bwd_kernel(BwdArgs a) {
             const int t = e / b, s = e % b;
             float acc = 0.f;
             if (s <= t)
-                for (int j = 0; j < d; ++j) acc = fmaf(S.DZP[t * d + j], S.G[s * d + j], acc);
+                for (int j = 0; j < d; j += 4) {
+                    const float4 u = *reinterpret_cast<const float4 *>(S.DZP + t * d + j);
+                    const float4 v = *reinterpret_cast<const float4 *>(S.G + s * d + j);
+                    acc = fmaf(u.x, v.x, fmaf(u.y, v.y, fmaf(u.z, v.z, fmaf(u.w, v.w, acc))));
+                }
             S.Bm[e] = acc;
         }
         if (a.ln)
@@ -330,23 +418,27 @@ __global__ void __launch_bounds__(kBwdThreads) linear_bwd_kernel(BwdArgs a) {
                 S.dgam[j] += gg;
             }
         __syncthreads();
-        // read-out and update terms of dq, dk, dG
-        for (int e = tid; e < bd; e += kBwdThreads) {
-            const int r = e / d, i = e % d;
-            float dq = S.DQ[e], dk = 0.f, dg = 0.f;
-            for (int j = 0; j < d; ++j) {
-                dq = fmaf(S.DZP[r * d + j], S.W[i * dp1 + j], dq);  // dzpre W^T
-                dk = fmaf(-S.Om[i * dp1 + j], S.G[r * d + j], dk);  // -G_r Om^T
-                dg = fmaf(-S.K[r * d + j], S.Om[j * dp1 + i], dg);  // -k_r Om
+        {  // read-out and update terms: dq += dzpre W^T; dk = -G Om^T; dG = -k Om; causal sums
+            float dq[4], dk[4] = {0.f, 0.f, 0.f, 0.f}, dg[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dq[k] = bk.row(k) < b ? S.DQ[bk.row(k) * d + c] : 0.f;
+            bk.abt(S.DZP, S.W, dq);
+            bk.abt(S.G, S.Om, dk);
+            bk.ab(S.K, S.Om, dg);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int r = bk.row(k);
+                if (r >= b) continue;
+                float q = dq[k], kk = -dk[k], g = -dg[k];
+                for (int s = 0; s <= r; ++s) q = fmaf(-S.Bm[r * b + s], S.K[s * d + c], q);
+                for (int t = r; t < b; ++t) {
+                    kk = fmaf(-S.Bm[t * b + r], S.Q[t * d + c], kk);
+                    g = fmaf(-S.A[t * b + r], S.DZP[t * d + c], g);
+                }
+                S.DQ[r * d + c] = q;
+                S.DK[r * d + c] = kk;
+                S.DG[r * d + c] = g;
             }
-            for (int s = 0; s <= r; ++s) dq = fmaf(-S.Bm[r * b + s], S.K[s * d + i], dq);
-            for (int t = r; t < b; ++t) {
-                dk = fmaf(-S.Bm[t * b + r], S.Q[t * d + i], dk);
-                dg = fmaf(-S.A[t * b + r], S.DZP[t * d + i], dg);
-            }
-            S.DQ[e] = dq;
-            S.DK[e] = dk;
-            S.DG[e] = dg;
         }
         __syncthreads();
         // step size and the inner loss gradient's own backward (per token)
@@ -388,14 +480,14 @@ __global__ void __launch_bounds__(kBwdThreads) linear_bwd_kernel(BwdArgs a) {
             }
             const float inv_d = 1.f / d;
             const float mdp = warp_sum(s1) * inv_d, e_ = warp_sum(s2) * inv_d,
-                        c = warp_sum(s3) * inv_d, dsig = -warp_sum(s4) / sig;
+                        cc = warp_sum(s3) * inv_d, dsig = -warp_sum(s4) / sig;
             float dgh[2], dxh[2], t1 = 0.f, t2 = 0.f;
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int j = lane + 32 * r;
                 const float g = j < d ? S.gam[j] : 0.f;
                 dgh[r] = j < d ? (dpsi[r] - mdp - xh[r] * e_) / sig : 0.f;
-                dxh[r] = j < d ? (-c * dpsi[r] - gh[r] * e_) / sig + g * g * dgh[r] : 0.f;
+                dxh[r] = j < d ? (-cc * dpsi[r] - gh[r] * e_) / sig + g * g * dgh[r] : 0.f;
                 t1 += dxh[r];
                 t2 += dxh[r] * xh[r];
             }
@@ -413,15 +505,21 @@ __global__ void __launch_bounds__(kBwdThreads) linear_bwd_kernel(BwdArgs a) {
             }
         }
         __syncthreads();
-        // key map: dk_s += dx_s W^T; store dq, dk; inner-LN parameter gradients
-        for (int e = tid; e < bd; e += kBwdThreads) {
-            const int s = e / d, i = e % d;
-            float dk = S.DK[e];
-            for (int c = 0; c < d; ++c) dk = fmaf(S.DX[s * d + c], S.W[i * dp1 + c], dk);
-            a.dK[r0 * d + e] = dk;
-            a.dQ[r0 * d + e] = S.DQ[e];
+        {  // key map: dk_s += dx_s W^T; store dq, dk
+            float dk[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dk[k] = bk.row(k) < b ? S.DK[bk.row(k) * d + c] : 0.f;
+            bk.abt(S.DX, S.W, dk);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int r = bk.row(k);
+                if (r < b) {
+                    a.dK[(r0 + r) * d + c] = dk[k];
+                    a.dQ[(r0 + r) * d + c] = S.DQ[r * d + c];
+                }
+            }
         }
-        if (a.ln)
+        if (a.ln)  // inner-LN parameter gradients
             for (int j = tid; j < d; j += kBwdThreads) {
                 const float g = S.gam[j], be = S.bet[j];
                 float gb = 0.f, gg = 0.f;
@@ -435,15 +533,7 @@ __global__ void __launch_bounds__(kBwdThreads) linear_bwd_kernel(BwdArgs a) {
             }
         __syncthreads();
         // dW_m = Om + sum_t q_t^T dzpre_t + sum_s k_s^T dx_s
-        for (int e = tid; e < d * d; e += kBwdThreads) {
-            const int i = e / d, j = e % d;
-            float acc = S.Om[i * dp1 + j];
-            for (int t = 0; t < b; ++t) {
-                acc = fmaf(S.Q[t * d + i], S.DZP[t * d + j], acc);
-                acc = fmaf(S.K[t * d + i], S.DX[t * d + j], acc);
-            }
-            S.Om[i * dp1 + j] = acc;
-        }
+        bk.outer(S.Om, S.Q, S.DZP, S.K, S.DX);
         __syncthreads();
     }
     for (int e = tid; e < d * d; e += kBwdThreads) a.dW0s[(size_t)seq * d * d + e] = S.Om[(e / d) * dp1 + e % d];
@@ -468,7 +558,7 @@ __global__ void sum_over_batch_kernel(const float *in, float *out, int B, int H,
 }  // namespace
 
 bool linear_bwd_supported(int d, int b) {
-    return d >= 1 && d <= 64 && b >= 1 && b * d <= 1024;
+    return (d == 16 || d == 32 || d == 64) && b >= 1 && b * d <= 1024;
 }
 
 size_t linear_bwd_workspace_bytes(int B, int H, int T, int d, int b) {
@@ -487,17 +577,19 @@ cudaError_t launch_linear_bwd(const LinearBwdArgs &a, cudaStream_t s) {
               a.H, a.T, a.d, a.b, a.ln, a.w0_per_seq};
     const size_t smem = bwd_smem_floats(a.d, a.b) * sizeof(float);
     cudaError_t e;
-    if (a.bf16) {
-        e = cudaFuncSetAttribute(linear_bwd_kernel<__nv_bfloat16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        linear_bwd_kernel<__nv_bfloat16><<<(unsigned)S, kBwdThreads, smem, s>>>(k);
-    } else {
-        e = cudaFuncSetAttribute(linear_bwd_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e != cudaSuccess) return e;
-        linear_bwd_kernel<float><<<(unsigned)S, kBwdThreads, smem, s>>>(k);
-    }
+    auto go = [&](auto kernel) -> cudaError_t {
+        cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (r != cudaSuccess) return r;
+        kernel<<<(unsigned)S, kBwdThreads, smem, s>>>(k);
+        return cudaSuccess;
+    };
+    if (a.bf16)
+        e = a.d == 16 ? go(linear_bwd_kernel<__nv_bfloat16, 16>)
+          : a.d == 32 ? go(linear_bwd_kernel<__nv_bfloat16, 32>) : go(linear_bwd_kernel<__nv_bfloat16, 64>);
+    else
+        e = a.d == 16 ? go(linear_bwd_kernel<float, 16>)
+          : a.d == 32 ? go(linear_bwd_kernel<float, 32>) : go(linear_bwd_kernel<float, 64>);
+    if (e != cudaSuccess) return e;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
