@@ -294,7 +294,8 @@ static void linear_primal_seq(const problem_t *p, int seq) {
     memcpy(W, w1_init(p, seq), dd * sizeof(double));
     for (int m0 = 0; m0 < T; m0 += b) {
         memcpy(Wm, W, dd * sizeof(double)); /* W_m; W now holds the running W^(t) */
-        for (int t = m0; t < m0 + b; ++t) {
+        const int m1 = m0 + b < T ? m0 + b : T; /* a last mini-batch may be partial */
+        for (int t = m0; t < m1; ++t) {
             linear_grad_into(K + (size_t)t * d, V + (size_t)t * d, Wm, gamma, beta, d, p->ln,
                              p->eps, &s, Gam);
             for (size_t e = 0; e < dd; ++e) W[e] -= eta[t] * Gam[e];
@@ -328,13 +329,14 @@ static void linear_dual_seq(const problem_t *p, int seq) {
     scratch_init(&s, d, 0);
     memcpy(W, w1_init(p, seq), dd * sizeof(double));
     for (int m0 = 0; m0 < T; m0 += b) {
-        for (int r = 0; r < b; ++r) {
+        const int nb = T - m0 < b ? T - m0 : b; /* a last mini-batch may be partial */
+        for (int r = 0; r < nb; ++r) {
             const int t = m0 + r;
             linear_dloss_dx(K + (size_t)t * d, V + (size_t)t * d, W, gamma, beta, d, p->ln, p->eps,
                             &s, G + (size_t)r * d);
             for (int j = 0; j < d; ++j) G[(size_t)r * d + j] *= eta[t];
         }
-        for (int r = 0; r < b; ++r) {
+        for (int r = 0; r < nb; ++r) {
             const double *q = Q + (size_t)(m0 + r) * d;
             vec_mat(q, W, d, d, zp);
             for (int sr = 0; sr <= r; ++sr) {
@@ -349,7 +351,7 @@ static void linear_dual_seq(const problem_t *p, int seq) {
                 for (int j = 0; j < d; ++j) z[j] = zp[j];
             }
         }
-        for (int r = 0; r < b; ++r) {
+        for (int r = 0; r < nb; ++r) {
             const double *k = K + (size_t)(m0 + r) * d;
             for (int i = 0; i < d; ++i)
                 for (int j = 0; j < d; ++j) W[(size_t)i * d + j] -= k[i] * G[(size_t)r * d + j];
@@ -526,8 +528,13 @@ int orc_num_threads(void) {
     return n > 0 ? (int)n : 1;
 }
 
+static void linear_primal_seq(const problem_t *p, int seq);
+static void linear_dual_seq(const problem_t *p, int seq);
+
 static int run(const problem_t *p, seq_fn fn, const int *seqs, int nseqs, int nthreads) {
-    if (p->T % p->b != 0 || p->b <= 0 || p->d <= 0) return -2;
+    if (p->b <= 0 || p->d <= 0) return -2;
+    /* Only the linear forms define a partial last mini-batch (fewer tokens). */
+    if (p->T % p->b != 0 && fn != linear_primal_seq && fn != linear_dual_seq) return -2;
     const int total = p->B * p->H;
     if (!seqs) nseqs = total;
     for (int i = 0; seqs && i < nseqs; ++i)

@@ -478,7 +478,50 @@ def test_sequence_subset_and_threads_agree():
         np.testing.assert_array_equal(Ws[bi, h], Wall[bi, h])
 
 
-def test_rejects_ragged_minibatch():
+def test_rejects_ragged_minibatch_where_undefined():
+    """Only TTT-Linear defines a partial last mini-batch; the MLP and the
+    large-chunk forms still require T to be a multiple of b."""
+    Q, K, V, eta, W1, W2, gamma, beta = rand_problem(1, 1, 10, 4, dh=16)
+    with pytest.raises(ValueError):
+        oracle.mlp_primal(Q, K, V, eta, W1, W2, gamma, beta, b=4)
     Q, K, V, eta, W0, *_ = rand_problem(1, 1, 10, 4)
     with pytest.raises(ValueError):
-        oracle.linear_primal(Q, K, V, eta, W0, b=4, ln=False)
+        oracle.chunk_primal(Q, K, V, eta, W0, chunk=4)
+
+
+@pytest.mark.parametrize("ln", [True, False])
+def test_partial_last_minibatch_primal_equals_dual(ln):
+    """T = 10 with b = 4: two full mini-batches and a partial one of 2 tokens;
+    the token-by-token and the dual forms agree."""
+    Q, K, V, eta, W0, _, gamma, beta = rand_problem(2, 2, 10, 6, seed=3)
+    g, be = (gamma, beta) if ln else (None, None)
+    Zp, Wp = oracle.linear_primal(Q, K, V, eta, W0, g, be, b=4, ln=ln)
+    Zd, Wd = oracle.linear_dual(Q, K, V, eta, W0, g, be, b=4, ln=ln)
+    np.testing.assert_allclose(Zd, Zp, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Wd, Wp, rtol=0, atol=1e-12)
+
+
+def test_partial_single_minibatch_is_one_batch_of_all_tokens():
+    """T = 10 < b = 16: the only mini-batch holds all 10 tokens, the same
+    computation as b = 10."""
+    Q, K, V, eta, W0, _, gamma, beta = rand_problem(1, 2, 10, 6, seed=4)
+    Z16, W16 = oracle.linear_primal(Q, K, V, eta, W0, gamma, beta, b=16, ln=True)
+    Z10, W10 = oracle.linear_primal(Q, K, V, eta, W0, gamma, beta, b=10, ln=True)
+    np.testing.assert_array_equal(Z16, Z10)
+    np.testing.assert_array_equal(W16, W10)
+
+
+@pytest.mark.parametrize("ln", [True, False])
+def test_partial_minibatch_equals_zero_step_padding(ln):
+    """A partial last mini-batch equals padding the sequence to a multiple of
+    b with tokens of step size 0 (any q, k, v) under the full-batch rule: those
+    tokens change no weight, and the real tokens' outputs are the same."""
+    Q, K, V, eta, W0, _, gamma, beta = rand_problem(1, 2, 12, 6, seed=5)
+    eta = eta.copy()
+    eta[..., 10:] = 0.0
+    g, be = (gamma, beta) if ln else (None, None)
+    Zpad, Wpad = oracle.linear_primal(Q, K, V, eta, W0, g, be, b=4, ln=ln)
+    Zr, Wr = oracle.linear_primal(Q[:, :, :10].copy(), K[:, :, :10].copy(), V[:, :, :10].copy(),
+                                  eta[:, :, :10].copy(), W0, g, be, b=4, ln=ln)
+    np.testing.assert_allclose(Zr, Zpad[:, :, :10], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(Wr, Wpad, rtol=0, atol=1e-13)
