@@ -106,7 +106,9 @@ TTT_API const char *ttt_status_string(int status);
  *   ln_gamma, ln_beta  [H][d] fp32; required with TTT_F_LN, ignored without
  *   Z         [B][H][T][d] fp32 output
  *   W_out     [B][H][d][d] fp32 output, the weight after the last token; may be NULL
- * Supported: T % b == 0; d in {16, 32, 64} and 1 <= b <= 64 with b*d <= 4096
+ * Supported: any T >= 1 (when T is not a multiple of b, the last mini-batch
+ *   holds the remaining T mod b tokens, every gradient again taken at its
+ *   starting weight); d in {16, 32, 64} and 1 <= b <= 64 with b*d <= 4096
  *   for TTT_FP32 and TTT_BF16; TTT_BF16 with d = 64, b = 16 runs the
  *   tensor-core scan, every other case the fp32 CUDA-core kernel.
  */

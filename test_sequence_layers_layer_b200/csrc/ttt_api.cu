@@ -186,7 +186,7 @@ ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const flo
     const bool ln = flags & TTT_F_LN;
     if (!Q || !K || !V || !eta || !W0 || !Z) return TTT_ERR_PTR;
     if (ln && (!ln_gamma || !ln_beta)) return TTT_ERR_PTR;
-    if (B <= 0 || H <= 0 || T <= 0 || b <= 0 || b > 64 || T % b != 0) return TTT_ERR_SHAPE;
+    if (B <= 0 || H <= 0 || T <= 0 || b <= 0 || b > 64) return TTT_ERR_SHAPE;
     if (!supported_d(d) || b * d > 4096) return TTT_ERR_SHAPE;
     if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return TTT_ERR_SHAPE;
     if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;

@@ -198,7 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int seq = blockIdx.x, head = seq % a.H;
-    const int T = a.T, NM = T / kMB, NC = (T + kChunkTok - 1) / kChunkTok;
+    // NM counts a partial last mini-batch: its rows past T get step size 0 (the
+    // eta staging below), so their G rows are zero, and their Z is not stored.
+    const int T = a.T, NM = (T + kMB - 1) / kMB, NC = (T + kChunkTok - 1) / kChunkTok;
     const long tok0 = (long)seq * T;  // first row of this sequence in [B*H*T][64]
     int *status = a.status;
 
@@ -606,9 +608,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) out[i] = zp[i];
             }
-            float *zo = a.Z + (tok0 + (long)m * kMB + t) * kD;
-            *reinterpret_cast<float4 *>(zo + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
-            *reinterpret_cast<float4 *>(zo + 32 + 4 * g) = make_float4(out[4], out[5], out[6], out[7]);
+            if (m * kMB + t < T) {
+                float *zo = a.Z + (tok0 + (long)m * kMB + t) * kD;
+                *reinterpret_cast<float4 *>(zo + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
+                *reinterpret_cast<float4 *>(zo + 32 + 4 * g) = make_float4(out[4], out[5], out[6], out[7]);
+            }
             if (threadIdx.x == 384) TRACE(17, m);
         }
     }

@@ -101,10 +101,14 @@ __global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a) {
     for (int e = threadIdx.x; e < d * d; e += blockDim.x) W[e] = W0[e];
     for (int m0 = 0; m0 < T; m0 += b) {
         const size_t base = ((size_t)seq * T + m0) * d;
-        load_tile(Qs, a.Q, base, b * d, a.bf16);
-        load_tile(Ks, a.K, base, b * d, a.bf16);
-        load_tile(Vs, a.V, base, b * d, a.bf16);
-        for (int e = threadIdx.x; e < b; e += blockDim.x) es[e] = a.eta[(size_t)seq * T + m0 + e];
+        // A partial last mini-batch holds nb < b tokens: the other rows are
+        // zero with step size 0, so they change no weight and are not stored.
+        const int nb = T - m0 < b ? T - m0 : b;
+        load_tile(Qs, a.Q, base, nb * d, a.bf16);
+        load_tile(Ks, a.K, base, nb * d, a.bf16);
+        load_tile(Vs, a.V, base, nb * d, a.bf16);
+        for (int e = nb * d + threadIdx.x; e < b * d; e += blockDim.x) Qs[e] = Ks[e] = Vs[e] = 0.f;
+        for (int e = threadIdx.x; e < b; e += blockDim.x) es[e] = e < nb ? a.eta[(size_t)seq * T + m0 + e] : 0.f;
         __syncthreads();
         // X = K W_m and Q W_m
         for (int e = threadIdx.x; e < b * d; e += blockDim.x) {
@@ -153,7 +157,7 @@ __global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a) {
         }
         __syncthreads();
         // output epilogue
-        for (int t = warp; t < b; t += kWarps) {
+        for (int t = warp; t < nb; t += kWarps) {
             float *out = a.Z + base + (size_t)t * d;
             if (a.ln) {
                 ln_residual_store(Zs + t * d, Qs + t * d, gamma, beta, out, d);

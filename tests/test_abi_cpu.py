@@ -36,7 +36,7 @@ def lin(**kw):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(T=60), -2),              # T % b != 0
+    (dict(T=0), -2),
     (dict(d=48), -2),              # unsupported d
     (dict(b=0), -2),
     (dict(B=0), -2),
@@ -52,6 +52,13 @@ def test_linear_host_validation(kw, code):
     assert lin(**kw) == code
 
 
+def test_linear_accepts_a_partial_last_minibatch():
+    # T = 60 with b = 16: three full mini-batches and one of 12 tokens pass the
+    # host checks; without a GPU the arch check then fails
+    assert lin(T=60) in (-8, -5)
+    assert lin(T=7) in (-8, -5)
+
+
 def test_linear_without_ln_does_not_need_gamma():
     # validation passes; on a machine without a GPU the arch check then fails
     rc = lin(ln_gamma=None, ln_beta=None, flags=0)
@@ -65,6 +72,7 @@ def test_mlp_and_chunk_host_validation():
     assert ttt.ttt_mlp_fwd(**{**m, "dh": 128}, check=False) == -2
     assert ttt.ttt_mlp_fwd(**{**m, "flags": 0}, check=False) == -1   # MLP needs LN
     assert ttt.ttt_mlp_fwd(**{**m, "b": 32}, check=False) == -2
+    assert ttt.ttt_mlp_fwd(**{**m, "T": 40}, check=False) == -2   # MLP: T % b == 0
     c = dict(Q=ALIGNED, K=ALIGNED, V=ALIGNED, eta=ALIGNED, W0=ALIGNED, Z=ALIGNED, W_out=None,
              B=1, H=1, T=4096, d=128, chunk=2048, dt=ttt.TTT_BF16, flags=0,
              workspace=None, workspace_bytes=0, stream=0)

@@ -34,6 +34,16 @@ SMALL = {
     "linear_ln_150_seqs": W["linear_ln_d64_b8h12_t2048"].scaled(B=10, H=15, T=32),
     "linear_ln_long": W["linear_ln_d64_b8h12_t2048"].scaled(B=1, H=2, T=1024),
     "linear_noln_bf16": W["linear_ln_d64_b8h12_t2048"].scaled(B=2, H=2, T=128, ln=False),
+    # partial last mini-batch (T not a multiple of b): tensor-core path with 3
+    # full mini-batches + 2 tokens, a lone partial one, and one past a 64-token
+    # TMA chunk; the fp32 path; and bf16 with b = 32 (fp32 kernel)
+    "linear_ln_partial_T50": W["linear_ln_d64_b8h12_t2048"].scaled(B=2, H=3, T=50),
+    "linear_ln_partial_T7": W["linear_ln_d64_b8h12_t2048"].scaled(B=1, H=2, T=7),
+    "linear_ln_partial_T130": W["linear_ln_d64_b8h12_t2048"].scaled(B=1, H=3, T=130),
+    "linear_noln_partial_T41": W["linear_ln_d64_b8h12_t2048"].scaled(B=2, H=1, T=41, ln=False),
+    "linear_fp32_partial_T37": W["linear_fp32_d16"].scaled(B=2, H=2, T=37, d=32, b=8, ln=True,
+                                                          eta="sigmoid_over_d"),
+    "linear_bf16_b32_partial_T70": W["linear_ln_d64_b8h12_t2048"].scaled(B=1, H=2, T=70, b=32),
     # MLP
     "mlp_small": W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=1, H=3, T=48),
     "mlp_fp32_d16": W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=2, H=2, T=32, d=16, dh=64, b=4,
