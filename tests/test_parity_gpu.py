@@ -91,6 +91,14 @@ def test_full_size_parity(name, seqs):
     print(f"{name}: max rel err {errs}")
 
 
+def test_full_size_partial_last_minibatch():
+    """The bench workload's shape with T = 2047 (127 full mini-batches and one
+    of 15 tokens) in one launch, every sequence against the oracle."""
+    inp = synth.make_inputs(W["linear_ln_d64_b8h12_t2048"].scaled(T=2047))
+    errs = check_parity(inp)
+    print(f"linear T=2047: max rel err {errs}")
+
+
 def test_mlp_full_size_parity_conditioned():
     """Every sequence of the full MLP workload. The recurrence with this step
     size is chaotic on some sequences (see test_conditioning): there even the
