@@ -46,11 +46,12 @@ def weight_bytes(wl) -> int:
     return 4 * (2 * wl.d * wl.dh if wl.kind == "mlp" else wl.d * wl.d)
 
 
-def algo_bytes_per_token(wl) -> float:
-    """Interface bytes a token must move: Q, K, V in, eta in, Z (fp32) out, plus
-    the fast weight read once and written once per sequence, spread over T."""
+def algo_bytes_per_token(wl, zb: int = 4) -> float:
+    """Interface bytes a token must move: Q, K, V in, eta in, Z out (zb bytes an
+    element: 4 for fp32, 2 for bf16), plus the fast weight read once and
+    written once per sequence, spread over T."""
     e = 2 if wl.dtype == "bf16" else 4
-    return 3 * wl.d * e + 4 + 4 * wl.d + 2 * weight_bytes(wl) / wl.T
+    return 3 * wl.d * e + 4 + zb * wl.d + 2 * weight_bytes(wl) / wl.T
 
 
 def algo_flops_per_token(wl) -> float:
@@ -76,7 +77,7 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_plan(wl):
+def kernel_plan(wl, zb: int = 4):
     """Kernels one library call launches, in launch order:
     (name, source file, arithmetic type, algorithmic bytes/token, FLOPs/token)."""
     e = 2 if wl.dtype == "bf16" else 4
@@ -88,17 +89,17 @@ def kernel_plan(wl):
             # W_{c+1} = W_c - A_c W_c + B_c: d^3 per chunk; W0 in, W_out out
             ("chunk_scan_kernel", "ttt_chunk_tc.cu", "f32", 8 * d * d / wl.T, 2 * d ** 3 / wl.b),
             # Q in, Z (fp32) out; Z = Q W_c
-            ("chunk_apply_kernel", "ttt_chunk_tc.cu", "bf16", d * e + 4 * d, 2 * d * d),
+            ("chunk_apply_kernel", "ttt_chunk_tc.cu", "bf16", d * e + zb * d, 2 * d * d),
         ]
     if wl.kind == "linear" and wl.dtype == "bf16" and d == 64 and wl.b == 16:
-        return [("linear_ln_scan_kernel", "ttt_linear_tc.cu", "bf16", algo_bytes_per_token(wl),
+        return [("linear_ln_scan_kernel", "ttt_linear_tc.cu", "bf16", algo_bytes_per_token(wl, zb),
                  algo_flops_per_token(wl))]
     if wl.kind == "mlp" and wl.dtype == "bf16" and d == 64 and wl.dh == 256 and wl.b == 16:
-        return [("mlp_ln_scan_kernel", "ttt_mlp_tc.cu", "bf16", algo_bytes_per_token(wl),
+        return [("mlp_ln_scan_kernel", "ttt_mlp_tc.cu", "bf16", algo_bytes_per_token(wl, zb),
                  algo_flops_per_token(wl))]
     name = {"linear": "linear_simt_kernel", "mlp": "mlp_simt_kernel",
             "chunk": "chunk_simt_kernel"}[wl.kind]
-    return [(name, "ttt_simt.cu", "f32", algo_bytes_per_token(wl), algo_flops_per_token(wl))]
+    return [(name, "ttt_simt.cu", "f32", algo_bytes_per_token(wl, zb), algo_flops_per_token(wl))]
 
 
 def source_sha(fname: str) -> str:
@@ -204,18 +205,19 @@ def device_tensors(inp, dev):
     return x
 
 
-def make_caller(wl, x, stream):
+def make_caller(wl, x, stream, z_bf16=False):
     """Returns (call, outputs) where call() enqueues one library call on `stream`."""
     import torch
     import test_sequence_layers_layer_b200 as ttt
     B, H, T, d = wl.B, wl.H, wl.T, wl.d
     dev = x["Q"].device
     dt = ttt.TTT_BF16 if wl.dtype == "bf16" else ttt.TTT_FP32
-    Z = torch.empty((B, H, T, d), dtype=torch.float32, device=dev)
+    Z = torch.empty((B, H, T, d), dtype=torch.bfloat16 if z_bf16 else torch.float32, device=dev)
+    zf = ttt.TTT_F_Z_BF16 if z_bf16 else 0
     sp = stream.cuda_stream
     if wl.kind == "linear":
         Wo = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
-        flags = ttt.TTT_F_LN if wl.ln else 0
+        flags = (ttt.TTT_F_LN if wl.ln else 0) | zf
 
         def call(x=x):
             ttt.ttt_linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
@@ -227,7 +229,7 @@ def make_caller(wl, x, stream):
 
         def call(x=x):
             ttt.ttt_mlp_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["W2"], x["gamma"],
-                            x["beta"], Z, W1o, W2o, B, H, T, d, wl.dh, wl.b, dt, ttt.TTT_F_LN, sp)
+                            x["beta"], Z, W1o, W2o, B, H, T, d, wl.dh, wl.b, dt, ttt.TTT_F_LN | zf, sp)
         return call, (Z, W1o, W2o)
     Wo = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
     need = ttt.ttt_chunk_workspace_bytes(B, H, T, d, wl.b)
@@ -235,7 +237,7 @@ def make_caller(wl, x, stream):
 
     def call(x=x):
         ttt.ttt_chunk_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], Z, Wo, B, H, T, d, wl.b,
-                          dt, 0, ws, need, sp)
+                          dt, zf, ws, need, sp)
     return call, (Z, Wo)
 
 
@@ -278,14 +280,15 @@ def gpu_arm(args, wl, rank, world):
     inp = synth.make_inputs(rank_workload(wl, rank))
     x = device_tensors(inp, dev)
     stream = torch.cuda.Stream(dev)
-    call, outs = make_caller(wl, x, stream)
+    zb = 2 if args.z_bf16 else 4
+    call, outs = make_caller(wl, x, stream, args.z_bf16)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[dev.index])
 
-    plan = kernel_plan(wl)
+    plan = kernel_plan(wl, zb)
     multi = len(plan) > 1
     sampler = ClockSampler(dev)
     sampler.start()
@@ -333,7 +336,7 @@ def gpu_arm(args, wl, rank, world):
     # the call, device -> pinned host outputs, every step.
     host_in = {k: v.cpu().pin_memory() for k, v in x.items() if v is not None}
     dev_in = {k: torch.empty_like(v) for k, v in x.items() if v is not None}
-    call_e2e, outs_e2e = make_caller(wl, dev_in, stream)
+    call_e2e, outs_e2e = make_caller(wl, dev_in, stream, args.z_bf16)
     host_out = [o.cpu().pin_memory() for o in outs_e2e if o is not None]
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = sum(o.numel() * o.element_size() for o in host_out)
@@ -380,7 +383,8 @@ def gpu_arm(args, wl, rank, world):
         peak, unit = peaks["bf16_tflops"], "TFLOP/s"
     tflops = algo_flops_per_token(wl) * wl.tokens / (ms_per_step / 1e3) / 1e12
     sha = source_sha(ksrc)
-    traffic = recorded_traffic(kname, wl.name, sha)
+    wname = wl.name + ("_zbf16" if args.z_bf16 else "")
+    traffic = recorded_traffic(kname, wname, sha)
     clocks = sampler.summary(t0, t1)
     kernels = [{"name": p[0], "ms_per_launch": kern_tot[i] / args.steps,
                 "share": kern_tot[i] / max(sum(kern_tot), 1e-12)} for i, p in enumerate(plan)]
@@ -397,8 +401,9 @@ def gpu_arm(args, wl, rank, world):
         "vs_baseline": None,
         "dtype": kdtype,
         "data": "synthetic (seeded SplitMix64 normals; bf16-rounded Q/K/V)",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "d": wl.d,
+        "config": {"workload": wname, "B": wl.B, "H": wl.H, "T": wl.T, "d": wl.d,
                    "mini_batch": wl.b, "layer_norm": wl.ln, "qkv_dtype": wl.dtype,
+                   "z_dtype": "bf16" if args.z_bf16 else "fp32",
                    "tokens_per_step_per_gpu": wl.tokens, "l2": "flushed between steps (256 MiB write)",
                    "parallelism": f"replicas x{world} (independent sequences)"},
         "pct_of_bf16_tensor_peak": 100.0 * tflops / peaks["bf16_tflops"],
@@ -672,6 +677,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--z-bf16", action="store_true",
+                    help="store Z as bf16 (TTT_F_Z_BF16) instead of fp32")
     ap.add_argument("--backward", action="store_true",
                     help="time the TTT-Linear backward (linear workloads) instead")
     ap.add_argument("--decode", type=int, default=0,

@@ -80,6 +80,8 @@ typedef void *ttt_stream; /* a cudaStream_t */
 
 #define TTT_F_LN 1u         /* f(k) = k + LN(k W) instead of f(k) = k W        */
 #define TTT_F_W0_PER_SEQ 2u /* W0 is [B][H][...] instead of [H][...]           */
+#define TTT_F_Z_BF16 4u     /* forward entry points: Z is stored as bf16,
+                               rounded to nearest even, instead of fp32     */
 
 #define TTT_ABI_VERSION 1
 
@@ -104,7 +106,7 @@ TTT_API const char *ttt_status_string(int status);
  *   eta       [B][H][T] fp32
  *   W0        [H][d][d] (or [B][H][d][d] with TTT_F_W0_PER_SEQ) fp32
  *   ln_gamma, ln_beta  [H][d] fp32; required with TTT_F_LN, ignored without
- *   Z         [B][H][T][d] fp32 output
+ *   Z         [B][H][T][d] output: fp32, or bf16 with TTT_F_Z_BF16
  *   W_out     [B][H][d][d] fp32 output, the weight after the last token; may be NULL
  * Supported: any T >= 1 (when T is not a multiple of b, the last mini-batch
  *   holds the remaining T mod b tokens, every gradient again taken at its
@@ -114,7 +116,7 @@ TTT_API const char *ttt_status_string(int status);
  */
 TTT_API ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const float *eta,
                           const float *W0, const float *ln_gamma, const float *ln_beta,
-                          float *Z, float *W_out, int B, int H, int T, int d, int b,
+                          void *Z, float *W_out, int B, int H, int T, int d, int b,
                           ttt_dtype dt, unsigned flags, ttt_stream stream);
 
 /*
@@ -165,7 +167,7 @@ TTT_API ttt_status ttt_linear_bwd(const void *Q, const void *K, const void *V, c
  */
 TTT_API ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float *eta,
                        const float *W1_0, const float *W2_0, const float *ln_gamma,
-                       const float *ln_beta, float *Z, float *W1_out, float *W2_out, int B,
+                       const float *ln_beta, void *Z, float *W1_out, float *W2_out, int B,
                        int H, int T, int d, int dh, int b, ttt_dtype dt, unsigned flags,
                        ttt_stream stream);
 
@@ -186,12 +188,12 @@ TTT_API ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, cons
  *   on the tensor cores (three launches: per-chunk Gram products, the
  *   sequential affine scan over chunks, and the read-out), d in {64, 128}
  *   with TTT_FP32, and d = 64, run the fp32 CUDA-core kernel.
- * flags: only TTT_F_W0_PER_SEQ.
+ * flags: TTT_F_W0_PER_SEQ, TTT_F_Z_BF16.
  */
 TTT_API size_t ttt_chunk_workspace_bytes(int B, int H, int T, int d, int chunk);
 
 TTT_API ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, const float *eta,
-                         const float *W0, float *Z, float *W_out, int B, int H, int T, int d,
+                         const float *W0, void *Z, float *W_out, int B, int H, int T, int d,
                          int chunk, ttt_dtype dt, unsigned flags, void *workspace,
                          size_t workspace_bytes, ttt_stream stream);
 
@@ -221,7 +223,7 @@ TTT_API ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, co
  */
 #define TTT_CHUNK_NOALLOC_SCRATCH_BYTES (24u << 20)
 TTT_API ttt_status ttt_chunk_fwd_noalloc(const void *Q, const void *K, const void *V,
-                                         const float *eta, const float *W0, float *Z,
+                                         const float *eta, const float *W0, void *Z,
                                          float *W_out, int B, int H, int T, int d, int chunk,
                                          ttt_dtype dt, unsigned flags, ttt_stream stream);
 

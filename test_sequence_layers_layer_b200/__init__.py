@@ -25,6 +25,7 @@ TTT_OK = 0
 TTT_BF16, TTT_FP32 = 0, 1
 TTT_F_LN = 1
 TTT_F_W0_PER_SEQ = 2
+TTT_F_Z_BF16 = 4
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -226,14 +227,15 @@ def _dtype_code(t):
 
 
 def linear_fwd(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, w0_per_seq=False,
-               stream=None, want_w=True):
+               stream=None, want_w=True, z_bf16=False):
     """TTT-Linear forward. Q, K, V: [B,H,T,d] cuda tensors (bf16 or fp32).
     Returns (Z fp32 [B,H,T,d], W_out fp32 [B,H,d,d] or None)."""
     import torch
     B, H, T, d = Q.shape
-    Z = torch.empty((B, H, T, d), dtype=torch.float32, device=Q.device)
+    Z = torch.empty((B, H, T, d), dtype=torch.bfloat16 if z_bf16 else torch.float32, device=Q.device)
     W_out = torch.empty((B, H, d, d), dtype=torch.float32, device=Q.device) if want_w else None
-    flags = (TTT_F_LN if ln else 0) | (TTT_F_W0_PER_SEQ if w0_per_seq else 0)
+    flags = (TTT_F_LN if ln else 0) | (TTT_F_W0_PER_SEQ if w0_per_seq else 0) | \
+        (TTT_F_Z_BF16 if z_bf16 else 0)
     ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                    _dtype_code(Q), flags, stream)
     return Z, W_out
@@ -265,32 +267,32 @@ def linear_bwd(Q, K, V, eta, W0, ln_gamma, ln_beta, dZ, dW_out=None, *, b, ln, w
 
 
 def mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, *, b, w0_per_seq=False, stream=None,
-            want_w=True):
+            want_w=True, z_bf16=False):
     """TTT-MLP forward. Returns (Z, W1_out, W2_out)."""
     import torch
     B, H, T, d = Q.shape
     dh = W1_0.shape[-1]
-    Z = torch.empty((B, H, T, d), dtype=torch.float32, device=Q.device)
+    Z = torch.empty((B, H, T, d), dtype=torch.bfloat16 if z_bf16 else torch.float32, device=Q.device)
     W1o = torch.empty((B, H, d, dh), dtype=torch.float32, device=Q.device) if want_w else None
     W2o = torch.empty((B, H, dh, d), dtype=torch.float32, device=Q.device) if want_w else None
-    flags = TTT_F_LN | (TTT_F_W0_PER_SEQ if w0_per_seq else 0)
+    flags = TTT_F_LN | (TTT_F_W0_PER_SEQ if w0_per_seq else 0) | (TTT_F_Z_BF16 if z_bf16 else 0)
     ttt_mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1o, W2o, B, H, T, d, dh, b,
                 _dtype_code(Q), flags, stream)
     return Z, W1o, W2o
 
 
 def chunk_fwd(Q, K, V, eta, W0, *, chunk, w0_per_seq=False, workspace=None, stream=None,
-              want_w=True):
+              want_w=True, z_bf16=False):
     """Large-chunk TTT forward (apply-then-update). Allocates the workspace
     with torch unless one is given. Returns (Z, W_out)."""
     import torch
     B, H, T, d = Q.shape
-    Z = torch.empty((B, H, T, d), dtype=torch.float32, device=Q.device)
+    Z = torch.empty((B, H, T, d), dtype=torch.bfloat16 if z_bf16 else torch.float32, device=Q.device)
     W_out = torch.empty((B, H, d, d), dtype=torch.float32, device=Q.device) if want_w else None
     need = ttt_chunk_workspace_bytes(B, H, T, d, chunk)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
-    flags = TTT_F_W0_PER_SEQ if w0_per_seq else 0
+    flags = (TTT_F_W0_PER_SEQ if w0_per_seq else 0) | (TTT_F_Z_BF16 if z_bf16 else 0)
     ttt_chunk_fwd(Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, _dtype_code(Q), flags,
                   workspace, need, stream)
     return Z, W_out

@@ -180,9 +180,9 @@ const char *ttt_status_string(int status) {
 
 ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const float *eta,
                           const float *W0, const float *ln_gamma, const float *ln_beta,
-                          float *Z, float *W_out, int B, int H, int T, int d, int b,
+                          void *Z, float *W_out, int B, int H, int T, int d, int b,
                           ttt_dtype dt, unsigned flags, ttt_stream stream) {
-    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ)) return TTT_ERR_ARG;
+    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ | TTT_F_Z_BF16)) return TTT_ERR_ARG;
     const bool ln = flags & TTT_F_LN;
     if (!Q || !K || !V || !eta || !W0 || !Z) return TTT_ERR_PTR;
     if (ln && (!ln_gamma || !ln_beta)) return TTT_ERR_PTR;
@@ -200,8 +200,8 @@ ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const flo
     st = check_device_ptrs(ptrs, 9);
     if (st != TTT_OK) return st;
 
-    LinearArgs a{Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
-                 dt == TTT_BF16, ln, (flags & TTT_F_W0_PER_SEQ) != 0};
+    LinearArgs a{Q, K, V, eta, W0, ln_gamma, ln_beta, static_cast<float *>(Z), W_out, B, H, T, d, b,
+                 dt == TTT_BF16, ln, (flags & TTT_F_W0_PER_SEQ) != 0, (flags & TTT_F_Z_BF16) != 0};
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
     return launched(linear_tc_supported(d, b, dt == TTT_BF16) ? launch_linear_tc(a, cs)
@@ -247,10 +247,10 @@ ttt_status ttt_linear_bwd(const void *Q, const void *K, const void *V, const flo
 
 ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float *eta,
                        const float *W1_0, const float *W2_0, const float *ln_gamma,
-                       const float *ln_beta, float *Z, float *W1_out, float *W2_out, int B,
+                       const float *ln_beta, void *Z, float *W1_out, float *W2_out, int B,
                        int H, int T, int d, int dh, int b, ttt_dtype dt, unsigned flags,
                        ttt_stream stream) {
-    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ)) return TTT_ERR_ARG;
+    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ | TTT_F_Z_BF16)) return TTT_ERR_ARG;
     if (!(flags & TTT_F_LN)) return TTT_ERR_ARG;
     if (!Q || !K || !V || !eta || !W1_0 || !W2_0 || !ln_gamma || !ln_beta || !Z) return TTT_ERR_PTR;
     if (B <= 0 || H <= 0 || T <= 0 || b <= 0 || b > 16 || T % b != 0) return TTT_ERR_SHAPE;
@@ -268,8 +268,8 @@ ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float 
     st = check_device_ptrs(ptrs, 11);
     if (st != TTT_OK) return st;
 
-    MlpArgs a{Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out,
-              B, H, T, d, dh, b, dt == TTT_BF16, per_seq};
+    MlpArgs a{Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, static_cast<float *>(Z), W1_out, W2_out,
+              B, H, T, d, dh, b, dt == TTT_BF16, per_seq, (flags & TTT_F_Z_BF16) != 0};
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
     return launched(mlp_tc_supported(d, dh, b, dt == TTT_BF16, (long long)B * H * T)
@@ -283,10 +283,10 @@ size_t ttt_chunk_workspace_bytes(int B, int H, int T, int d, int chunk) {
 }
 
 ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, const float *eta,
-                         const float *W0, float *Z, float *W_out, int B, int H, int T, int d,
+                         const float *W0, void *Z, float *W_out, int B, int H, int T, int d,
                          int chunk, ttt_dtype dt, unsigned flags, void *workspace,
                          size_t workspace_bytes, ttt_stream stream) {
-    if (flags & ~TTT_F_W0_PER_SEQ) return TTT_ERR_ARG;
+    if (flags & ~(TTT_F_W0_PER_SEQ | TTT_F_Z_BF16)) return TTT_ERR_ARG;
     if (!Q || !K || !V || !eta || !W0 || !Z) return TTT_ERR_PTR;
     if (B <= 0 || H <= 0 || T <= 0 || chunk <= 0 || T % chunk != 0 || chunk % 128 != 0)
         return TTT_ERR_SHAPE;
@@ -308,8 +308,8 @@ ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, const floa
     st = check_device_ptrs(ptrs, 8);
     if (st != TTT_OK) return st;
 
-    ChunkArgs a{Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, dt == TTT_BF16,
-                (flags & TTT_F_W0_PER_SEQ) != 0, workspace, workspace_bytes};
+    ChunkArgs a{Q, K, V, eta, W0, static_cast<float *>(Z), W_out, B, H, T, d, chunk, dt == TTT_BF16,
+                (flags & TTT_F_W0_PER_SEQ) != 0, (flags & TTT_F_Z_BF16) != 0, workspace, workspace_bytes};
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
     return launched(tc ? launch_chunk_tc(a, cs) : launch_chunk_simt(a, cs));

@@ -410,8 +410,9 @@ constexpr size_t kApplySmem = 1024 + kApplyStageOff + 8 * 8192;
 
 struct ApplyArgs {
     const uint8_t *Wimg;
-    float *Z;
+    float *Z;  // bf16 instead when z_bf16
     int chunk;
+    bool z_bf16;
     int *status;
 };
 
@@ -520,12 +521,12 @@ __global__ void __launch_bounds__(kApplyThreads, 1)
             tc_fence_before();
             mbar_arrive(&tempty[acc]);  // the accumulator is read; the MMA may reuse it
             __syncwarp();
-            float *zbase = a.Z + ((size_t)(row0 + (long)t * kApplyRows) + 32 * sp) * kD + 64 * half;
+            const size_t zbase = ((size_t)(row0 + (long)t * kApplyRows) + 32 * sp) * kD + 64 * half;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int r = 2 * i + (lane >> 4), c = lane & 15;
-                *reinterpret_cast<float4 *>(zbase + (size_t)r * kD + 4 * c) =
-                    *reinterpret_cast<const float4 *>(stage + r * 64 + ((c ^ (r & 7)) << 2));
+                const float4 f = *reinterpret_cast<const float4 *>(stage + r * 64 + ((c ^ (r & 7)) << 2));
+                store_z4(a.Z, a.z_bf16, zbase + (size_t)r * kD + 4 * c, f.x, f.y, f.z, f.w);
             }
             __syncwarp();
         }
@@ -588,7 +589,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
-    chunk_apply_kernel<<<n, kApplyThreads, kApplySmem, s>>>(tmQ, ApplyArgs{Wimg, a.Z, a.chunk, status});
+    chunk_apply_kernel<<<n, kApplyThreads, kApplySmem, s>>>(tmQ, ApplyArgs{Wimg, a.Z, a.chunk, a.z_bf16, status});
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
@@ -630,7 +631,7 @@ void *chunk_scratch_on_current_device() {
 }  // namespace
 
 extern "C" ttt_status ttt_chunk_fwd_noalloc(const void *Q, const void *K, const void *V,
-                                            const float *eta, const float *W0, float *Z,
+                                            const float *eta, const float *W0, void *Z,
                                             float *W_out, int B, int H, int T, int d, int chunk,
                                             ttt_dtype dt, unsigned flags, ttt_stream stream) {
     const size_t need = ttt_chunk_workspace_bytes(B, H, T, d, chunk);

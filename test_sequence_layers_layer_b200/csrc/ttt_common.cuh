@@ -15,25 +15,25 @@ constexpr float kLnEps = 1e-5f;  // torch nn.LayerNorm default, as in the pages'
 struct LinearArgs {
     const void *Q, *K, *V;
     const float *eta, *W0, *gamma, *beta;
-    float *Z, *W_out;
+    float *Z, *W_out;  // Z is bf16 [..][d] instead when z_bf16
     int B, H, T, d, b;
-    bool bf16, ln, w0_per_seq;
+    bool bf16, ln, w0_per_seq, z_bf16;
 };
 
 struct MlpArgs {
     const void *Q, *K, *V;
     const float *eta, *W1_0, *W2_0, *gamma, *beta;
-    float *Z, *W1_out, *W2_out;
+    float *Z, *W1_out, *W2_out;  // Z is bf16 instead when z_bf16
     int B, H, T, d, dh, b;
-    bool bf16, w0_per_seq;
+    bool bf16, w0_per_seq, z_bf16;
 };
 
 struct ChunkArgs {
     const void *Q, *K, *V;
     const float *eta, *W0;
-    float *Z, *W_out;
+    float *Z, *W_out;  // Z is bf16 instead when z_bf16
     int B, H, T, d, chunk;
-    bool bf16, w0_per_seq;
+    bool bf16, w0_per_seq, z_bf16;
     void *workspace;
     size_t workspace_bytes;
 };
@@ -50,6 +50,31 @@ struct LinearBwdArgs {
 bool linear_bwd_supported(int d, int b);
 size_t linear_bwd_workspace_bytes(int B, int H, int T, int d, int b);
 cudaError_t launch_linear_bwd(const LinearBwdArgs &a, cudaStream_t s);
+
+// Output stores: Z as fp32, or rounded to nearest-even bf16 (TTT_F_Z_BF16).
+// off is the element offset of the first value; vector forms need off a
+// multiple of their width.
+__device__ __forceinline__ void store_z1(float *Z, bool bf16, size_t off, float v) {
+    if (bf16) reinterpret_cast<__nv_bfloat16 *>(Z)[off] = __float2bfloat16_rn(v);
+    else Z[off] = v;
+}
+__device__ __forceinline__ void store_z2(float *Z, bool bf16, size_t off, float a, float b) {
+    if (bf16) reinterpret_cast<__nv_bfloat162 *>(reinterpret_cast<__nv_bfloat16 *>(Z) + off)[0] =
+        __floats2bfloat162_rn(a, b);
+    else *reinterpret_cast<float2 *>(Z + off) = make_float2(a, b);
+}
+__device__ __forceinline__ void store_z4(float *Z, bool bf16, size_t off, float a, float b, float c,
+                                         float d) {
+    if (bf16) {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+        uint2 u;
+        u.x = *reinterpret_cast<const uint32_t *>(&lo);
+        u.y = *reinterpret_cast<const uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(Z) + off) = u;
+    } else {
+        *reinterpret_cast<float4 *>(Z + off) = make_float4(a, b, c, d);
+    }
+}
 
 // Launchers return cudaSuccess or the launch error.
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s);

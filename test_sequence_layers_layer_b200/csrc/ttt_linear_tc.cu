@@ -101,7 +101,7 @@ struct Args {
     const float *eta, *W0, *gamma, *beta;
     float *Z, *W_out;
     int H, T;
-    bool ln, w0_per_seq;
+    bool ln, w0_per_seq, z_bf16;
     int *status;
 };
 
@@ -609,9 +609,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < 8; ++i) out[i] = zp[i];
             }
             if (m * kMB + t < T) {
-                float *zo = a.Z + (tok0 + (long)m * kMB + t) * kD;
-                *reinterpret_cast<float4 *>(zo + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
-                *reinterpret_cast<float4 *>(zo + 32 + 4 * g) = make_float4(out[4], out[5], out[6], out[7]);
+                const size_t zo = (size_t)(tok0 + (long)m * kMB + t) * kD;
+                store_z4(a.Z, a.z_bf16, zo + 4 * g, out[0], out[1], out[2], out[3]);
+                store_z4(a.Z, a.z_bf16, zo + 32 + 4 * g, out[4], out[5], out[6], out[7]);
             }
             if (threadIdx.x == 384) TRACE(17, m);
         }
@@ -651,7 +651,7 @@ cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     Args args{a.eta, a.W0, a.gamma, a.beta, a.Z, a.W_out, a.H, a.T, a.ln, a.w0_per_seq,
-              device_status_word()};
+              a.z_bf16, device_status_word()};
     linear_ln_scan_kernel<<<a.B * a.H, kThreads, kSmemBytes, s>>>(tmK, tmQ, tmV, args);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch(s);

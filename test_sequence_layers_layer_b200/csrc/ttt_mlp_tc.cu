@@ -117,7 +117,7 @@ struct Args {
     const float *eta, *W1_0, *W2_0, *gamma, *beta;
     float *Z, *W1_out, *W2_out;
     int H, T;
-    bool w0_per_seq;
+    bool w0_per_seq, z_bf16;
     int *status;
 };
 
@@ -526,8 +526,8 @@ __global__ void __launch_bounds__(Layout<kCL>::kThreads, 1)
         const uint8_t *tile = smem + L::TILES + (i % kSlots) * kSlotBytes;
         const float2 qv =
             bf2_to_f2(*reinterpret_cast<const uint32_t *>(tile + kTileBytes + pair_off(t_own, lane)));
-        *reinterpret_cast<float2 *>(a.Z + (row0 + (size_t)i * kMB + t_own) * kD + 2 * lane) =
-            make_float2(qv.x + gam.x * (z0 - mu) * rstd + bet.x, qv.y + gam.y * (z1 - mu) * rstd + bet.y);
+        store_z2(a.Z, a.z_bf16, (row0 + (size_t)i * kMB + t_own) * kD + 2 * lane,
+                 qv.x + gam.x * (z0 - mu) * rstd + bet.x, qv.y + gam.y * (z1 - mu) * rstd + bet.y);
     };
 
     int m = 0;
@@ -833,7 +833,7 @@ cudaError_t launch_mlp_tc(const MlpArgs &a, cudaStream_t s) {
                                          L::kSmemBytes);
     if (e != cudaSuccess) return e;
     Args args{a.eta, a.W1_0, a.W2_0, a.gamma, a.beta, a.Z, a.W1_out, a.W2_out, a.H, a.T,
-              a.w0_per_seq, device_status_word()};
+              a.w0_per_seq, a.z_bf16, device_status_word()};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.B * a.H * kCluster));
     cfg.blockDim = dim3(L::kThreads);

@@ -62,13 +62,13 @@ __device__ __forceinline__ void ln_grad_row(float *x, const float *k, const floa
     }
 }
 
-// out[j] = q[j] + gamma[j] * LN(x)[j] + beta[j]
+// Z[off + j] = q[j] + gamma[j] * LN(x)[j] + beta[j]   (fp32, or bf16 when zb)
 __device__ __forceinline__ void ln_residual_store(const float *x, const float *q,
                                                   const float *gamma, const float *beta,
-                                                  float *out, int n) {
+                                                  float *Z, bool zb, size_t off, int n) {
     const float2 st = row_stats(x, n);
     for (int j = threadIdx.x & 31; j < n; j += 32)
-        out[j] = q[j] + gamma[j] * ((x[j] - st.x) * st.y) + beta[j];
+        store_z1(Z, zb, off + j, q[j] + gamma[j] * ((x[j] - st.x) * st.y) + beta[j]);
 }
 
 __device__ __forceinline__ float gelu(float h) {
@@ -158,11 +158,11 @@ __global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a) {
         __syncthreads();
         // output epilogue
         for (int t = warp; t < nb; t += kWarps) {
-            float *out = a.Z + base + (size_t)t * d;
+            const size_t out = base + (size_t)t * d;
             if (a.ln) {
-                ln_residual_store(Zs + t * d, Qs + t * d, gamma, beta, out, d);
+                ln_residual_store(Zs + t * d, Qs + t * d, gamma, beta, a.Z, a.z_bf16, out, d);
             } else {
-                for (int j = threadIdx.x & 31; j < d; j += 32) out[j] = Zs[t * d + j];
+                for (int j = threadIdx.x & 31; j < d; j += 32) store_z1(a.Z, a.z_bf16, out + j, Zs[t * d + j]);
             }
         }
         __syncthreads();
@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kThreads) mlp_simt_kernel(MlpArgs a) {
             }
         }
         for (int t = warp; t < b; t += kWarps)
-            ln_residual_store(Zs + t * d, Qs + t * d, gamma, beta, a.Z + base + (size_t)t * d, d);
+            ln_residual_store(Zs + t * d, Qs + t * d, gamma, beta, a.Z, a.z_bf16, base + (size_t)t * d, d);
         __syncthreads();
     }
     if (a.W1_out)
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
                     az = fmaf(Qs[t * d + i], w, az);
                     ax = fmaf(Ks[t * d + i], w, ax);
                 }
-                a.Z[base + e] = az;
+                store_z1(a.Z, a.z_bf16, base + e, az);
                 Gs[e] = es[t] * (ax - Vs[e]);
             }
             __syncthreads();
