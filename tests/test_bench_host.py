@@ -32,3 +32,23 @@ def test_recorded_traffic_goes_stale_with_kernel_or_header(tmp_path, monkeypatch
     assert current() == 1234.0
     (csrc / "k.cu").write_text("kernel v2")  # the kernel itself changed
     assert current() is None
+
+
+def test_workload_accounting():
+    """Bytes and FLOPs per token that the roofline divides by, from the
+    shapes: Z costs 4 bytes an element, 2 with a bf16 Z; the large-chunk
+    read-out moves Q in and Z out; the backward does 20 d^2 FLOPs a token."""
+    from test_sequence_layers_layer_b200 import synth
+    lin = synth.WORKLOADS["linear_ln_d64_b8h12_t2048"]
+    d = lin.d
+    fp32_z = bench.algo_bytes_per_token(lin)
+    assert fp32_z == 3 * d * 2 + 4 + 4 * d + 2 * 4 * d * d / lin.T
+    assert bench.algo_bytes_per_token(lin, 2) == fp32_z - 2 * d
+    ch = synth.WORKLOADS["chunk_d128_c2048_b4h8_t32768"]
+    plan = {p[0]: p for p in bench.kernel_plan(ch)}
+    plan16 = {p[0]: p for p in bench.kernel_plan(ch, 2)}
+    assert plan["chunk_apply_kernel"][3] == ch.d * 2 + 4 * ch.d
+    assert plan16["chunk_apply_kernel"][3] == ch.d * 2 + 2 * ch.d
+    assert plan["chunk_gram_kernel"][3] == plan16["chunk_gram_kernel"][3]
+    assert bench.bwd_flops_per_token(64) == 20 * 64 * 64
+    assert bench.bwd_bytes_per_token(lin) == 3 * d * 2 + 4 * d + 4 + 3 * 4 * d + 4
