@@ -1,4 +1,5 @@
-"""Outer gradients of the TTT-Linear layer (its backward pass), for the tests.
+"""Outer gradients of the TTT-Linear layer and of large-chunk TTT (their
+backward passes), for the tests.
 
 TEST INFRASTRUCTURE ONLY: imported by the test suite, never by the library.
 It shares nothing with the CUDA library and does not import it.
@@ -21,6 +22,9 @@ gradients of  sum(Z * dZ) + sum(W_out * dW_out)  then come from autograd
 through the whole unrolled loop. Conventions as in ttt_oracle.c: row form
 x = k W with W[d_in][d_out], Q/K/V/Z [B][H][T][d], eta [B][H][T], W0 [H][d][d]
 (or [B][H][d][d]), gamma/beta [H][d], LayerNorm eps 1e-5 with biased variance.
+The large-chunk form (chunk_forward) is written the same way from "Test-Time
+Training Done Right" (abstract): apply with the chunk's starting weight, then
+one gradient step on the chunk's eta-weighted loss.
 """
 from __future__ import annotations
 
@@ -94,4 +98,42 @@ def linear_forward_np(Q, K, V, eta, W0, gamma, beta, *, b, ln, eps=LN_EPS):
     beta = np.zeros((H, d)) if beta is None else beta
     ts = [_t(a) for a in (Q, K, V, eta, W0, gamma, beta)]
     Z, Wo = linear_forward(*ts, b=b, ln=ln, eps=eps)
+    return Z.detach().numpy(), Wo.detach().numpy()
+
+
+def chunk_forward(Q, K, V, eta, W0, *, chunk):
+    """Large-chunk TTT ("Test-Time Training Done Right", abstract): the tokens
+    of chunk c read out with W_c, then W_{c+1} = W_c - grad of
+    sum_t eta_t 1/2 ||k_t W_c - v_t||^2 at W_c (autograd, kept in the graph).
+    f(k) = k W (no LayerNorm). Returns (Z, W_out) as float64 tensors."""
+    B, H, T, d = Q.shape
+    W = W0.expand(B, H, d, d) if W0.dim() == 3 else W0
+    Z = []
+    for c0 in range(0, T, chunk):
+        Wc = W
+        sl = slice(c0, c0 + chunk)
+        Z.append(torch.einsum("bhti,bhij->bhtj", Q[:, :, sl], Wc))
+        r = torch.einsum("bhti,bhij->bhtj", K[:, :, sl], Wc) - V[:, :, sl]
+        loss = 0.5 * (eta[:, :, sl, None] * r * r).sum()
+        W = Wc - torch.autograd.grad(loss, Wc, create_graph=True)[0]
+    return torch.cat(Z, dim=2), W
+
+
+def chunk_grads(Q, K, V, eta, W0, dZ, dW_out=None, *, chunk):
+    """Gradients of L = sum(Z * dZ) + sum(W_out * dW_out) for the large-chunk
+    forward: dict with keys Q, K, V, eta, W0 (float64 numpy)."""
+    ts = {n: _t(a) for n, a in dict(Q=Q, K=K, V=V, eta=eta, W0=W0).items()}
+    Z, Wo = chunk_forward(ts["Q"], ts["K"], ts["V"], ts["eta"], ts["W0"], chunk=chunk)
+    L = (Z * _t(dZ, False)).sum()
+    if dW_out is not None:
+        L = L + (Wo * _t(dW_out, False)).sum()
+    names = ["Q", "K", "V", "eta", "W0"]
+    grads = torch.autograd.grad(L, [ts[n] for n in names], allow_unused=True)
+    return {n: (np.zeros(ts[n].shape) if g is None else g.detach().numpy())
+            for n, g in zip(names, grads)}
+
+
+def chunk_forward_np(Q, K, V, eta, W0, *, chunk):
+    ts = [_t(a) for a in (Q, K, V, eta, W0)]
+    Z, Wo = chunk_forward(*ts, chunk=chunk)
     return Z.detach().numpy(), Wo.detach().numpy()

@@ -1,8 +1,8 @@
 """Pins of the backward oracle (oracle/backward.py) to things other than itself:
-its forward against the C oracle's token-by-token forward, its outer gradients
-against central finite differences (torch.autograd.gradcheck), and special
-cases the method fixes (eta = 0 freezes the weight, so Z cannot depend on K
-or V)."""
+its forwards against the C oracle's forwards, its outer gradients against
+central finite differences (torch.autograd.gradcheck), and special cases the
+method fixes (eta = 0 freezes the weight, so Z cannot depend on K or V; a
+single large chunk reads out with W0 alone)."""
 import os
 import sys
 
@@ -107,3 +107,39 @@ def test_eta_zero_freezes_weight_so_k_and_v_get_no_gradient():
     g = ob.linear_grads(Q, K, V, eta, W0, gamma, beta, dZ, None, b=4, ln=True)
     assert np.abs(g["K"]).max() == 0.0 and np.abs(g["V"]).max() == 0.0
     assert np.abs(g["eta"]).max() > 0.0
+
+
+# ------------------------------------------------------------ large-chunk form
+
+def test_chunk_forward_matches_c_oracle():
+    Q, K, V, eta, W0, _, _ = _inputs(9, 2, 2, 24, 6, eta_scale=0.05)
+    Z, Wo = ob.chunk_forward_np(Q, K, V, eta, W0, chunk=8)
+    Zc, Woc = oracle.chunk_primal(Q, K, V, eta, W0, chunk=8)
+    assert np.abs(Z - Zc).max() <= 1e-12 * max(1.0, np.abs(Zc).max())
+    assert np.abs(Wo - Woc).max() <= 1e-12 * max(1.0, np.abs(Woc).max())
+
+
+def test_chunk_gradients_match_finite_differences():
+    Q, K, V, eta, W0, _, _ = _inputs(10, 1, 1, 6, 3, eta_scale=0.4)
+    ts = [torch.tensor(a, requires_grad=True) for a in (Q, K, V, eta, W0)]
+    r = np.random.default_rng(11)
+    dZ = torch.tensor(r.standard_normal(Q.shape))
+    dW = torch.tensor(r.standard_normal((1, 1, 3, 3)))
+
+    def fn(*a):
+        Z, Wo = ob.chunk_forward(*a, chunk=2)
+        return (Z * dZ).sum() + (Wo * dW).sum()
+
+    assert torch.autograd.gradcheck(fn, tuple(ts), eps=1e-6, atol=1e-7, rtol=1e-6)
+
+
+def test_chunk_single_chunk_closed_form():
+    """One chunk: Z = Q W0 exactly, so with dW_out = 0 the gradients are
+    dQ = dZ W0^T, dW0 = Q^T dZ and nothing reaches K, V or eta."""
+    Q, K, V, eta, W0, _, _ = _inputs(12, 1, 1, 8, 4)
+    dZ = np.random.default_rng(13).standard_normal(Q.shape)
+    g = ob.chunk_grads(Q, K, V, eta, W0, dZ, None, chunk=8)
+    np.testing.assert_allclose(g["Q"][0, 0], dZ[0, 0] @ W0[0].T, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(g["W0"][0], Q[0, 0].T @ dZ[0, 0], rtol=0, atol=1e-13)
+    for k in ("K", "V", "eta"):
+        assert np.abs(g[k]).max() == 0.0
