@@ -562,6 +562,14 @@ def bwd_flops_per_token(d: int) -> float:
     return 20.0 * d * d
 
 
+def chunk_bwd_flops_per_token(d: int, chunk: int) -> float:
+    """Large-chunk backward: the three per-chunk Gram products (A_c, B_c,
+    Q^T dZ: 6 d^2), the two affine scans (2 d^3 each per chunk, spread over
+    the chunk's tokens) and the five per-token products (R, P, dQ and the two
+    terms of dK: 10 d^2)."""
+    return 16.0 * d * d + 4.0 * d ** 3 / chunk
+
+
 def bwd_bytes_per_token(wl) -> float:
     """Algorithmic HBM bytes per token: Q, K, V in once, dZ and eta in, dQ, dK,
     dV and deta out (the W_m checkpoints are the kernel's choice, not counted)."""
@@ -582,7 +590,9 @@ def backward_arm(args, wl):
     x = device_tensors(inp, dev)
     rng = np.random.default_rng(wl.seed + 101)
     dZ = torch.from_numpy(rng.standard_normal((wl.B, wl.H, wl.T, wl.d)).astype(np.float32)).to(dev)
-    need = ttt.ttt_linear_bwd_workspace_bytes(wl.B, wl.H, wl.T, wl.d, wl.b)
+    chunk = wl.kind == "chunk"
+    need = (ttt.ttt_chunk_bwd_workspace_bytes if chunk else ttt.ttt_linear_bwd_workspace_bytes)(
+        wl.B, wl.H, wl.T, wl.d, wl.b)
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
     f32 = dict(dtype=torch.float32, device=dev)
     g = [torch.empty((wl.B, wl.H, wl.T, wl.d), **f32) for _ in range(3)]
@@ -595,9 +605,13 @@ def backward_arm(args, wl):
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def call():
-        ttt.ttt_linear_bwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"], dZ,
-                           None, *g, geta, gW0, gg, gb, wl.B, wl.H, wl.T, wl.d, wl.b, dt, flags, ws,
-                           need, stream.cuda_stream)
+        if chunk:
+            ttt.ttt_chunk_bwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], dZ, None, *g, geta, gW0,
+                              wl.B, wl.H, wl.T, wl.d, wl.b, dt, 0, ws, need, stream.cuda_stream)
+        else:
+            ttt.ttt_linear_bwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
+                               dZ, None, *g, geta, gW0, gg, gb, wl.B, wl.H, wl.T, wl.d, wl.b, dt,
+                               flags, ws, need, stream.cuda_stream)
 
     sampler = ClockSampler(dev)
     sampler.start()
@@ -626,14 +640,20 @@ def backward_arm(args, wl):
         raise RuntimeError("device status error in the timed region")
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     ms = sum(step_ms) / args.steps
-    kern_ms = kern[0] / args.steps
+    # the large-chunk FLOP count covers all three kernels, so it is divided by
+    # their summed time
+    kern_ms = (sum(kern) if chunk else kern[0]) / args.steps
+    knames = (["cb_gram_kernel", "cb_scan_kernel", "cb_tok_kernel", "cb_sum_over_batch_kernel (dW0)"]
+              if chunk else ["linear_bwd_kernel", "sum_over_batch_kernel (dW0)",
+                             "sum_over_batch_kernel (dgamma)", "sum_over_batch_kernel (dbeta)"])
     clocks = sampler.summary(t0, t1)
     mhz = clocks.get("sm_mhz") or 1965
     peak = FP32_LANES * 2 * mhz * 1e6 / 1e12
-    flop = bwd_flops_per_token(wl.d) * wl.tokens
+    flop = (chunk_bwd_flops_per_token(wl.d, wl.b) if chunk else bwd_flops_per_token(wl.d)) * wl.tokens
     achieved = flop / (kern_ms / 1e3) / 1e12
     line = {
-        "metric": "TTT-Linear backward tokens/sec at 1 B200 (outer gradients of every input)",
+        "metric": ("Large-chunk TTT" if chunk else "TTT-Linear") +
+                  " backward tokens/sec at 1 B200 (outer gradients of every input)",
         "value": wl.tokens / (ms / 1e3), "unit": "tokens/s", "higher_is_better": True,
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "dtype": "f32", "data": "synthetic (seeded SplitMix64 normals; bf16-rounded Q/K/V; normal dZ)",
@@ -641,18 +661,17 @@ def backward_arm(args, wl):
                    "mini_batch": wl.b, "layer_norm": wl.ln, "qkv_dtype": wl.dtype,
                    "l2": "flushed between steps (256 MiB write)"},
         "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": "linear_bwd_kernel",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "all backward kernels" if chunk else "linear_bwd_kernel",
                      "peak_source": f"derived: {FP32_LANES} fp32 lanes x 2 FLOP x {mhz} MHz",
                      "algorithmic_per_launch": flop, "kernel_ms": kern_ms,
                      "hbm_bytes_per_token": bwd_bytes_per_token(wl)},
-        "kernels": [{"name": n, "ms_per_launch": t / args.steps} for n, t in
-                    zip(["linear_bwd_kernel", "sum_over_batch_kernel (dW0)",
-                         "sum_over_batch_kernel (dgamma)", "sum_over_batch_kernel (dbeta)"], kern)],
+        "kernels": [{"name": n, "ms_per_launch": t / args.steps} for n, t in zip(knames, kern)],
         "gpu_launches": launches,
         "clocks": clocks,
         "step_ms_min_median": [min(step_ms), statistics.median(step_ms)],
     }
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and not chunk:
         from oracle import backward as ob
         sub = wl.scaled(B=1, H=1, T=min(wl.T, 512))
         si = synth.make_inputs(sub)
@@ -695,8 +714,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
 
     if args.backward:
-        if wl.kind != "linear":
-            ap.error("--backward times the linear workloads")
+        if wl.kind == "mlp":
+            ap.error("--backward times the linear and large-chunk workloads")
         if rank == 0:
             print(json.dumps(backward_arm(args, wl)), flush=True)
         return

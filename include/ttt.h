@@ -151,6 +151,30 @@ TTT_API ttt_status ttt_linear_bwd(const void *Q, const void *K, const void *V, c
                                   ttt_stream stream);
 
 /*
+ * Large-chunk TTT backward: the outer gradients of ttt_chunk_fwd ("Test-Time
+ * Training Done Right", abstract), differentiating through the per-chunk
+ * weight updates. With Om_c = dL/dW_c, R_c = K_c W_c - V_c, P_c = K_c Om_{c+1}:
+ *   Om_c = Om_{c+1} - A_c Om_{c+1} + Q_c^T dZ_c (A_c = K_c^T diag(eta) K_c),
+ *   dQ_c = dZ_c W_c^T, dK_c = -diag(eta)(R_c Om_{c+1}^T + P_c W_c^T),
+ *   dV_c = diag(eta) P_c, deta_t = -P_t . R_t, dW0 = Om_0.
+ * Arguments as ttt_linear_bwd without LayerNorm: inputs Q, K, V (dtype dt),
+ * eta, W0, dZ (fp32, required), dW_out (fp32 or NULL); outputs dQ, dK, dV
+ * [B][H][T][d], deta [B][H][T], dW0 [H][d][d] summed over the batch (or
+ * [B][H][d][d] with TTT_F_W0_PER_SEQ), all fp32, overwritten. workspace:
+ * device memory of at least ttt_chunk_bwd_workspace_bytes() bytes, 256-byte
+ * aligned, owned by the caller (per chunk: A_c, B_c, Q_c^T dZ_c, W_c and
+ * Om_{c+1} in fp32). fp32 CUDA cores; deterministic.
+ * Supported: d in {64, 128}, chunk % 32 == 0, T % chunk == 0; TTT_BF16 or
+ * TTT_FP32. flags: only TTT_F_W0_PER_SEQ.
+ */
+TTT_API size_t ttt_chunk_bwd_workspace_bytes(int B, int H, int T, int d, int chunk);
+TTT_API ttt_status ttt_chunk_bwd(const void *Q, const void *K, const void *V, const float *eta,
+                                 const float *W0, const float *dZ, const float *dW_out, float *dQ,
+                                 float *dK, float *dV, float *deta, float *dW0, int B, int H, int T,
+                                 int d, int chunk, ttt_dtype dt, unsigned flags, void *workspace,
+                                 size_t workspace_bytes, ttt_stream stream);
+
+/*
  * TTT-MLP forward: f(k) = k + LN(GELU(k W1) W2) with W1 [d][dh], W2 [dh][d],
  * GELU the exact erf form; same mini-batch rule as ttt_linear_fwd, with both
  * layers updated ("How to Master Test-Time Training for LLMs": the hidden

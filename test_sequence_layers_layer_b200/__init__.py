@@ -55,6 +55,10 @@ def lib() -> ctypes.CDLL:
         L.ttt_linear_bwd_workspace_bytes.argtypes = [_I] * 5
         L.ttt_linear_bwd.restype = _I
         L.ttt_linear_bwd.argtypes = [_P] * 16 + [_I] * 6 + [ctypes.c_uint, _P, ctypes.c_size_t, _P]
+        L.ttt_chunk_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.ttt_chunk_bwd_workspace_bytes.argtypes = [_I] * 5
+        L.ttt_chunk_bwd.restype = _I
+        L.ttt_chunk_bwd.argtypes = [_P] * 12 + [_I] * 6 + [ctypes.c_uint, _P, ctypes.c_size_t, _P]
         L.ttt_mlp_fwd.restype = _I
         L.ttt_mlp_fwd.argtypes = [_P] * 11 + [_I] * 7 + [ctypes.c_uint, _P]
         L.ttt_chunk_workspace_bytes.restype = ctypes.c_size_t
@@ -143,6 +147,19 @@ def ttt_linear_bwd(Q, K, V, eta, W0, ln_gamma, ln_beta, dZ, dW_out, dQ, dK, dV, 
                               _ptr(deta), _ptr(dW0), _ptr(dgamma), _ptr(dbeta), B, H, T, d, b, dt,
                               flags, _ptr(workspace), workspace_bytes, _stream(stream))
     return _check("ttt_linear_bwd", rc) if check else rc
+
+
+def ttt_chunk_bwd_workspace_bytes(B, H, T, d, chunk) -> int:
+    return int(lib().ttt_chunk_bwd_workspace_bytes(B, H, T, d, chunk))
+
+
+def ttt_chunk_bwd(Q, K, V, eta, W0, dZ, dW_out, dQ, dK, dV, deta, dW0, B, H, T, d, chunk, dt, flags,
+                  workspace, workspace_bytes, stream=None, check=True):
+    rc = lib().ttt_chunk_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(dZ),
+                             _ptr(dW_out), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta), _ptr(dW0), B,
+                             H, T, d, chunk, dt, flags, _ptr(workspace), workspace_bytes,
+                             _stream(stream))
+    return _check("ttt_chunk_bwd", rc) if check else rc
 
 
 def ttt_mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out, B, H, T, d, dh,
@@ -263,6 +280,25 @@ def linear_bwd(Q, K, V, eta, W0, ln_gamma, ln_beta, dZ, dW_out=None, *, b, ln, w
     ttt_linear_bwd(Q, K, V, eta, W0, ln_gamma, ln_beta, dZ, dW_out, g["Q"], g["K"], g["V"],
                    g["eta"], g["W0"], g.get("gamma"), g.get("beta"), B, H, T, d, b, _dtype_code(Q),
                    flags, workspace, workspace.numel() * workspace.element_size(), stream)
+    return g
+
+
+def chunk_bwd(Q, K, V, eta, W0, dZ, dW_out=None, *, chunk, w0_per_seq=False, workspace=None,
+              stream=None):
+    """Large-chunk TTT backward. Returns a dict of fp32 cuda tensors Q, K, V,
+    eta, W0: the gradients of sum(Z * dZ) + sum(W_out * dW_out)."""
+    import torch
+    B, H, T, d = Q.shape
+    f32 = dict(dtype=torch.float32, device=Q.device)
+    need = ttt_chunk_bwd_workspace_bytes(B, H, T, d, chunk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+    g = dict(Q=torch.empty((B, H, T, d), **f32), K=torch.empty((B, H, T, d), **f32),
+             V=torch.empty((B, H, T, d), **f32), eta=torch.empty((B, H, T), **f32),
+             W0=torch.empty(tuple(W0.shape), **f32))
+    ttt_chunk_bwd(Q, K, V, eta, W0, dZ, dW_out, g["Q"], g["K"], g["V"], g["eta"], g["W0"], B, H, T,
+                  d, chunk, _dtype_code(Q), TTT_F_W0_PER_SEQ if w0_per_seq else 0, workspace,
+                  workspace.numel() * workspace.element_size(), stream)
     return g
 
 

@@ -154,6 +154,17 @@ ttt_status launched(cudaError_t e) { return e == cudaSuccess ? TTT_OK : TTT_ERR_
 }  // namespace
 }  // namespace ttt
 
+namespace ttt {
+// Large-chunk backward (ttt_chunk_bwd.cu).
+bool chunk_bwd_supported(int d, int chunk);
+size_t chunk_bwd_workspace_bytes(int B, int H, int T, int d, int chunk);
+cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const float *eta,
+                             const float *W0, const float *dZ, const float *dW_out, float *dQ,
+                             float *dK, float *dV, float *deta, float *dW0, int B, int H, int T,
+                             int d, int chunk, bool bf16, bool w0_per_seq, void *workspace,
+                             cudaStream_t s);
+}  // namespace ttt
+
 using namespace ttt;
 
 extern "C" {
@@ -243,6 +254,39 @@ ttt_status ttt_linear_bwd(const void *Q, const void *K, const void *V, const flo
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
     return launched(launch_linear_bwd(a, cs));
+}
+
+size_t ttt_chunk_bwd_workspace_bytes(int B, int H, int T, int d, int chunk) {
+    return chunk_bwd_workspace_bytes(B, H, T, d, chunk);
+}
+
+ttt_status ttt_chunk_bwd(const void *Q, const void *K, const void *V, const float *eta,
+                         const float *W0, const float *dZ, const float *dW_out, float *dQ, float *dK,
+                         float *dV, float *deta, float *dW0, int B, int H, int T, int d, int chunk,
+                         ttt_dtype dt, unsigned flags, void *workspace, size_t workspace_bytes,
+                         ttt_stream stream) {
+    if (flags & ~TTT_F_W0_PER_SEQ) return TTT_ERR_ARG;
+    if (!Q || !K || !V || !eta || !W0 || !dZ || !dQ || !dK || !dV || !deta || !dW0) return TTT_ERR_PTR;
+    if (B <= 0 || H <= 0 || T <= 0 || chunk <= 0 || T % chunk != 0 || !chunk_bwd_supported(d, chunk))
+        return TTT_ERR_SHAPE;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return TTT_ERR_SHAPE;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(W0) || !aligned16(dZ) ||
+        !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+        return TTT_ERR_ALIGN;
+    const size_t need = chunk_bwd_workspace_bytes(B, H, T, d, chunk);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return TTT_ERR_WORKSPACE;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {Q, K, V, eta, W0, dZ, dW_out, dQ, dK, dV, deta, dW0, workspace};
+    st = check_device_ptrs(ptrs, 13);
+    if (st != TTT_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    return launched(launch_chunk_bwd(Q, K, V, eta, W0, dZ, dW_out, dQ, dK, dV, deta, dW0, B, H, T, d,
+                                     chunk, dt == TTT_BF16, (flags & TTT_F_W0_PER_SEQ) != 0,
+                                     workspace, cs));
 }
 
 ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float *eta,

@@ -1,5 +1,6 @@
-"""TTT-Linear backward (ttt_linear_bwd) against the backward oracle
-(oracle/backward.py: autograd through the float64 unrolled inner loop).
+"""TTT-Linear backward (ttt_linear_bwd) and large-chunk backward
+(ttt_chunk_bwd) against the backward oracle (oracle/backward.py: autograd
+through the float64 unrolled inner loop).
 
 Tolerance: 1e-4 of each gradient's largest magnitude. The kernel works in
 fp32 (unit roundoff 6e-8); a gradient here is a sum over the sequence of
@@ -121,3 +122,66 @@ def test_backward_deterministic_and_rejects_small_workspace():
                             *out, wl.B, wl.H, wl.T + 1, wl.d, wl.b, ttt.TTT_BF16, ttt.TTT_F_LN, ws,
                             need, check=False)
     assert rc == -2  # TTT_ERR_SHAPE
+
+
+# ------------------------------------------------------------ large-chunk TTT
+
+CHUNK_CASES = {
+    # name: (workload changes, w0_per_seq, with dW_out)
+    "chunk_fp32_d64_c32": (dict(B=2, H=2, T=128, d=64, b=32, dtype="fp32"), False, True),
+    "chunk_bf16_d128_c64": (dict(B=1, H=2, T=256, d=128, b=64), False, False),
+    "chunk_fp32_d128_c128_w0seq": (dict(B=2, H=1, T=256, d=128, b=128, dtype="fp32"), True, True),
+}
+
+
+def _chunk_case(name, seed=31):
+    ch, w0seq, with_dw = CHUNK_CASES[name]
+    wl = synth.WORKLOADS["chunk_d128_c2048_b4h8_t32768"].scaled(seed=seed, **ch)
+    inp = synth.make_inputs(wl)
+    r = np.random.default_rng(seed + 1)
+    dZ = r.standard_normal((wl.B, wl.H, wl.T, wl.d)).astype(np.float32)
+    dW = r.standard_normal((wl.B, wl.H, wl.d, wl.d)).astype(np.float32) if with_dw else None
+    W0 = inp.W1
+    if w0seq:
+        W0 = (np.broadcast_to(W0[None], (wl.B,) + W0.shape)
+              + 0.01 * r.standard_normal((wl.B,) + W0.shape)).astype(np.float32)
+    return wl, inp, W0, dZ, dW, w0seq
+
+
+def _chunk_gpu(wl, inp, W0, dZ, dW, w0seq):
+    Q, K, V = _qkv(inp, wl)
+    f = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()  # noqa: E731
+    g = ttt.chunk_bwd(Q, K, V, f(inp.eta), f(W0), f(dZ), f(dW), chunk=wl.b, w0_per_seq=w0seq)
+    torch.cuda.synchronize()
+    assert ttt.ttt_device_status() == 0
+    return {k: v.double().cpu().numpy() for k, v in g.items()}
+
+
+@pytest.mark.parametrize("name", list(CHUNK_CASES))
+def test_chunk_backward_matches_oracle(name):
+    wl, inp, W0, dZ, dW, w0seq = _chunk_case(name)
+    got = _chunk_gpu(wl, inp, W0, dZ, dW, w0seq)
+    ref = ob.chunk_grads(inp.Q, inp.K, inp.V, inp.eta, W0, dZ, dW, chunk=wl.b)
+    if not w0seq:
+        ref["W0"] = ref["W0"].reshape(W0.shape)
+    errs = {k: _rel(got[k], ref[k]) for k in ref}
+    assert set(got) == set(ref)
+    assert max(errs.values()) <= TOL, errs
+
+
+def test_chunk_backward_full_size_sampled_sequences():
+    """The large-chunk bench workload (B=4, H=8, T=32768, d=128, chunk 2048,
+    bf16) in one launch; two sequences' per-token gradients against the
+    oracle run on those sequences alone."""
+    wl = synth.WORKLOADS["chunk_d128_c2048_b4h8_t32768"]
+    inp = synth.make_inputs(wl)
+    r = np.random.default_rng(41)
+    dZ = r.standard_normal((wl.B, wl.H, wl.T, wl.d)).astype(np.float32)
+    got = _chunk_gpu(wl, inp, inp.W1, dZ, None, False)
+    for bb, hh in [(0, 0), (3, 7)]:
+        sl = lambda a: a[bb:bb + 1, hh:hh + 1]  # noqa: E731
+        ref = ob.chunk_grads(sl(inp.Q), sl(inp.K), sl(inp.V), sl(inp.eta), inp.W1[hh:hh + 1],
+                             sl(dZ), None, chunk=wl.b)
+        for k in ("Q", "K", "V", "eta"):
+            e = _rel(sl(got[k]), ref[k])
+            assert e <= TOL, (bb, hh, k, e)
