@@ -86,3 +86,36 @@ def test_no_gpu_means_unsupported_not_fallback():
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert lin() == -8
+
+
+def test_backward_host_validation():
+    """ttt_linear_bwd and ttt_chunk_bwd reject bad arguments before any launch
+    (the workspace check comes before the architecture check, so a too-small
+    workspace is reported even without a GPU)."""
+    A = ALIGNED
+    lb = dict(Q=A, K=A, V=A, eta=A, W0=A, ln_gamma=A, ln_beta=A, dZ=A, dW_out=None, dQ=A, dK=A,
+              dV=A, deta=A, dW0=A, dgamma=A, dbeta=A, B=1, H=2, T=64, d=64, b=16,
+              dt=ttt.TTT_BF16, flags=ttt.TTT_F_LN, workspace=A, workspace_bytes=1 << 30, stream=0)
+    call = lambda **kw: ttt.ttt_linear_bwd(**{**lb, **kw}, check=False)  # noqa: E731
+    need = ttt.ttt_linear_bwd_workspace_bytes(1, 2, 64, 64, 16)
+    assert need == 4 * (2 * 4 * 64 * 64 + 2 * 64 * 64 + 2 * 2 * 64)
+    assert call(flags=ttt.TTT_F_Z_BF16) == -1        # not a backward flag
+    assert call(dgamma=None) == -5                    # LN needs dgamma, dbeta
+    assert call(T=60) == -2                           # backward: T % b == 0
+    assert call(d=48) == -2
+    assert call(workspace_bytes=need - 1) == -9
+    assert call(workspace=A + 16) == -9               # not 256-byte aligned
+    cb = dict(Q=A, K=A, V=A, eta=A, W0=A, dZ=A, dW_out=None, dQ=A, dK=A, dV=A, deta=A, dW0=A,
+              B=1, H=2, T=4096, d=128, chunk=2048, dt=ttt.TTT_BF16, flags=0, workspace=A,
+              workspace_bytes=1 << 34, stream=0)
+    call = lambda **kw: ttt.ttt_chunk_bwd(**{**cb, **kw}, check=False)  # noqa: E731
+    need = ttt.ttt_chunk_bwd_workspace_bytes(1, 2, 4096, 128, 2048)
+    assert need == 4 * (5 * 4 * 128 * 128 + 2 * 128 * 128)
+    assert ttt.ttt_chunk_bwd_workspace_bytes(1, 2, 4096, 96, 2048) == 0
+    assert call(flags=ttt.TTT_F_LN) == -1
+    assert call(dQ=None) == -5
+    assert call(d=96) == -2
+    assert call(chunk=48) == -2                       # chunk % 32 != 0
+    assert call(T=5000) == -2                         # T % chunk != 0
+    assert call(dQ=A + 4) == -4
+    assert call(workspace_bytes=need - 1) == -9
