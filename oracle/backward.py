@@ -1,5 +1,5 @@
-"""Outer gradients of the TTT-Linear layer and of large-chunk TTT (their
-backward passes), for the tests.
+"""Outer gradients of the TTT-Linear layer, of TTT-MLP and of large-chunk TTT
+(their backward passes), for the tests.
 
 TEST INFRASTRUCTURE ONLY: imported by the test suite, never by the library.
 It shares nothing with the CUDA library and does not import it.
@@ -137,3 +137,57 @@ def chunk_forward_np(Q, K, V, eta, W0, *, chunk):
     ts = [_t(a) for a in (Q, K, V, eta, W0)]
     Z, Wo = chunk_forward(*ts, chunk=chunk)
     return Z.detach().numpy(), Wo.detach().numpy()
+
+
+def mlp_forward(Q, K, V, eta, W1_0, W2_0, gamma, beta, *, b, eps=LN_EPS):
+    """TTT-MLP ("How to Master Test-Time Training for LLMs": the fast weight
+    may be an MLP) with the TTT-Linear mini-batch rule: f(k) = k +
+    LN(GELU(k W1) W2) gamma + beta, exact-erf GELU; every token's inner
+    gradient (autograd, kept in the graph) at the mini-batch's starting
+    weights, the read-out of token t after its own step. Returns (Z, W1_out,
+    W2_out) as float64 tensors; W1_0 [H,d,dh] or [B,H,d,dh], W2_0 likewise."""
+    B, H, T, d = Q.shape
+    dh = W1_0.shape[-1]
+    W1 = W1_0.expand(B, H, d, dh) if W1_0.dim() == 3 else W1_0
+    W2 = W2_0.expand(B, H, dh, d) if W2_0.dim() == 3 else W2_0
+    g, be = gamma.view(1, H, d), beta.view(1, H, d)
+
+    def f(k, A1, A2):
+        a = F.gelu(torch.einsum("bhi,bhij->bhj", k, A1))
+        x = torch.einsum("bhi,bhij->bhj", a, A2)
+        return k + F.layer_norm(x, (d,), eps=eps) * g + be
+
+    Z = []
+    for m0 in range(0, T, b):
+        W1m, W2m = W1, W2
+        for t in range(m0, m0 + b):
+            k, v = K[:, :, t], V[:, :, t]
+            loss = 0.5 * ((f(k, W1m, W2m) - v) ** 2).sum()
+            g1, g2 = torch.autograd.grad(loss, (W1m, W2m), create_graph=True)
+            e = eta[:, :, t, None, None]
+            W1, W2 = W1 - e * g1, W2 - e * g2
+            Z.append(f(Q[:, :, t], W1, W2))
+    return torch.stack(Z, dim=2), W1, W2
+
+
+def mlp_forward_np(Q, K, V, eta, W1_0, W2_0, gamma, beta, *, b, eps=LN_EPS):
+    ts = [_t(a) for a in (Q, K, V, eta, W1_0, W2_0, gamma, beta)]
+    Z, W1, W2 = mlp_forward(*ts, b=b, eps=eps)
+    return Z.detach().numpy(), W1.detach().numpy(), W2.detach().numpy()
+
+
+def mlp_grads(Q, K, V, eta, W1_0, W2_0, gamma, beta, dZ, dW1_out=None, dW2_out=None, *, b,
+              eps=LN_EPS):
+    """Gradients of L = sum(Z * dZ) + sum(W1_out * dW1_out) + sum(W2_out *
+    dW2_out) for TTT-MLP: dict with keys Q, K, V, eta, W1, W2, gamma, beta."""
+    names = ["Q", "K", "V", "eta", "W1", "W2", "gamma", "beta"]
+    ts = dict(zip(names, (_t(a) for a in (Q, K, V, eta, W1_0, W2_0, gamma, beta))))
+    Z, W1, W2 = mlp_forward(*(ts[n] for n in names), b=b, eps=eps)
+    L = (Z * _t(dZ, False)).sum()
+    if dW1_out is not None:
+        L = L + (W1 * _t(dW1_out, False)).sum()
+    if dW2_out is not None:
+        L = L + (W2 * _t(dW2_out, False)).sum()
+    grads = torch.autograd.grad(L, [ts[n] for n in names], allow_unused=True)
+    return {n: (np.zeros(ts[n].shape) if gr is None else gr.detach().numpy())
+            for n, gr in zip(names, grads)}

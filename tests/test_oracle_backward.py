@@ -143,3 +143,38 @@ def test_chunk_single_chunk_closed_form():
     np.testing.assert_allclose(g["W0"][0], Q[0, 0].T @ dZ[0, 0], rtol=0, atol=1e-13)
     for k in ("K", "V", "eta"):
         assert np.abs(g[k]).max() == 0.0
+
+
+# ------------------------------------------------------------ TTT-MLP form
+
+def _mlp_inputs(seed, B, H, T, d, dh, eta_scale=0.1):
+    r = np.random.default_rng(seed)
+    Q, K, V = (r.standard_normal((B, H, T, d)) for _ in range(3))
+    eta = eta_scale * r.uniform(0.2, 1.0, (B, H, T))
+    W1 = 0.3 * r.standard_normal((H, d, dh)) / np.sqrt(d)
+    W2 = 0.3 * r.standard_normal((H, dh, d)) / np.sqrt(dh)
+    gamma, beta = 1.0 + 0.2 * r.standard_normal((H, d)), 0.2 * r.standard_normal((H, d))
+    return Q, K, V, eta, W1, W2, gamma, beta
+
+
+@pytest.mark.parametrize("b", [1, 4])
+def test_mlp_forward_matches_c_oracle(b):
+    args = _mlp_inputs(21, 2, 2, 8, 4, 16)
+    Z, W1, W2 = ob.mlp_forward_np(*args, b=b)
+    Zc, W1c, W2c = oracle.mlp_primal(*args, b=b)
+    for x, y in ((Z, Zc), (W1, W1c), (W2, W2c)):
+        assert np.abs(x - y).max() <= 1e-12 * max(1.0, np.abs(y).max())
+
+
+def test_mlp_gradients_match_finite_differences():
+    args = _mlp_inputs(22, 1, 1, 4, 2, 4, eta_scale=0.5)
+    ts = [torch.tensor(a, requires_grad=True) for a in args]
+    r = np.random.default_rng(23)
+    dZ = torch.tensor(r.standard_normal(args[0].shape))
+    dW1 = torch.tensor(r.standard_normal((1, 1, 2, 4)))
+
+    def fn(*a):
+        Z, W1, W2 = ob.mlp_forward(*a, b=2)
+        return (Z * dZ).sum() + (W1 * dW1).sum() + W2.sum()
+
+    assert torch.autograd.gradcheck(fn, tuple(ts), eps=1e-6, atol=1e-7, rtol=1e-6)
