@@ -407,6 +407,7 @@ def gpu_arm(args, wl, rank, world):
                    "tokens_per_step_per_gpu": wl.tokens, "l2": "flushed between steps (256 MiB write)",
                    "parallelism": f"replicas x{world} (independent sequences)"},
         "pct_of_bf16_tensor_peak": 100.0 * tflops / peaks["bf16_tflops"],
+        "pct_of_bf16_tensor_peak_sustained": 100.0 * tflops / peaks["bf16_tflops_sustained"],
         "algorithmic_tflops": tflops,
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
