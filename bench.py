@@ -268,6 +268,38 @@ def aggregate(wl, world, steps, total_ms):
     return tokens, total_ms / steps, tokens * steps / (total_ms / 1e3)
 
 
+SM_COUNT = 148
+
+
+def latency_floor(wl, plan, kern_ms_per_call):
+    """The sequential chain's cost: each sequence scans ceil(T/b) dependent
+    mini-batch (or chunk) steps, one CTA (a 2-CTA cluster for the TTT-MLP
+    tensor-core scan) per sequence, one CTA per SM. With w waves of sequences
+    per launch the scan kernel's time divided by w * ceil(T/b) is the time of
+    one dependent step. Returns a dict for the bench line."""
+    idx = next((i for i, p in enumerate(plan) if "scan" in p[0]), len(plan) - 1)
+    name = plan[idx][0]
+    ctas = 2 if name == "mlp_ln_scan_kernel" else 1
+    nseq = wl.B * wl.H
+    concurrent = min(nseq, SM_COUNT // ctas)
+    waves = -(-nseq // concurrent)
+    steps = -(-wl.T // wl.b)
+    return {"us_per_minibatch_step": kern_ms_per_call[idx] * 1e3 / (waves * steps),
+            "dependent_steps": steps, "concurrent_sequences": concurrent, "waves": waves,
+            "kernel": name}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def gpu_arm(args, wl, rank, world):
     import torch
     import torch.distributed as dist
@@ -419,6 +451,7 @@ def gpu_arm(args, wl, rank, world):
         "gpu_launches": launches,
         "clocks": clocks,
         "step_ms_min_median": [min(step_ms), statistics.median(step_ms)],
+        "latency_floor": latency_floor(wl, plan, [t / args.steps for t in kern_tot]),
     }
     return line
 
@@ -478,7 +511,7 @@ def reference_arm(args, wl):
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "d": wl.d,
                    "mini_batch": wl.b},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -744,7 +777,8 @@ def main():
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             v, cores, desc = oracle_sample(wl, args.cpu_budget)
             line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
-                                    "kind": "oracle", "sample": desc}
+                                    "kind": "oracle", "sample": desc,
+                                    "cpu_model": cpu_model()}
         elif rank == 0:
             line["cpu_baseline"] = None
         if rank == 0:
