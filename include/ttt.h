@@ -252,6 +252,61 @@ TTT_API ttt_status ttt_chunk_fwd_noalloc(const void *Q, const void *K, const voi
                                          ttt_dtype dt, unsigned flags, ttt_stream stream);
 
 /*
+ * Sequence-parallel large-chunk TTT. The weight step of every chunk is
+ * affine in the weight (the gradient step of "Test-Time Training Done Right",
+ * expanded):
+ *   W_{c+1} = (I - A_c) W_c + B_c,  A_c = K_c^T diag(eta) K_c,  B_c = K_c^T diag(eta) V_c,
+ * so a run of whole chunks (a segment) maps its starting weight to its final
+ * weight by W -> M W + N. With every segment's (M, N) known, each segment's
+ * starting weight follows from a short fold (ttt_affine_prefix), and the
+ * segments then run their forwards independently: on separate ranks that each
+ * hold one stretch of the sequence, or on one GPU as more, shorter sequences.
+ *
+ * ttt_chunk_map: (M, N) of every sequence of K, V, eta ([B][H][T][d],
+ *   [B][H][T]), taken as one segment of T / chunk chunks. M and N are
+ *   [B][H][d][d] fp32, 16-byte aligned, distinct, written in full.
+ *   M = (I - A_{n-1}) ... (I - A_0); N is the weight the chunks end with from
+ *   W = 0. Computed with the large-chunk forward's kernels: one forward from
+ *   W = I with V = 0 (its final weight is M) and one from W = 0 (its final
+ *   weight is N), their read-outs discarded.
+ * workspace: at least ttt_chunk_map_workspace_bytes(...) bytes of device
+ *   scratch, 256-byte aligned, owned by the caller, clobbered (a zero V, the
+ *   discarded read-outs as bf16, the starting weights, and the forward's own
+ *   workspace).
+ * Supported shapes, dtypes and errors: those of ttt_chunk_fwd; the workspace
+ *   size is 0 for an unsupported shape.
+ */
+TTT_API size_t ttt_chunk_map_workspace_bytes(int B, int H, int T, int d, int chunk, ttt_dtype dt);
+TTT_API ttt_status ttt_chunk_map(const void *K, const void *V, const float *eta, float *M,
+                                 float *N, int B, int H, int T, int d, int chunk, ttt_dtype dt,
+                                 void *workspace, size_t workspace_bytes, ttt_stream stream);
+
+/*
+ * The fold of segment maps into starting weights, for S sequences of nseg
+ * segments each:
+ *   W_in[s][0] = W0[s],  W_in[s][j+1] = M[s][j] W_in[s][j] + N[s][j],
+ *   W_end[s] = M[s][nseg-1] W_in[s][nseg-1] + N[s][nseg-1]  (if W_end != NULL).
+ * Each (s, j) entry of M, N and W_in is a d x d fp32 row-major block starting
+ * at float offset s * seq_stride + j * seg_stride. Two layouts are meant:
+ * sequence-major (seq_stride = nseg d^2, seg_stride = d^2: the segments of one
+ * sequence adjacent, as when one GPU splits [B][H][T][d] into
+ * [B][H * nseg][T / nseg][d]) and segment-major (seq_stride = d^2,
+ * seg_stride = S d^2: the maps gathered from nseg ranks, rank-major). The
+ * strides must keep the blocks apart: seq_stride >= nseg * seg_stride with
+ * seg_stride >= d^2, or seg_stride >= S * seq_stride with seq_stride >= d^2
+ * (when nseg == 1 only seq_stride >= d^2 is needed); both multiples of 4.
+ * W0 is [H][d][d] (sequence s uses head s % H; S a multiple of H) or, with
+ * TTT_F_W0_PER_SEQ, [S][d][d]. W_end is [S][d][d] or NULL. W_in and W_end must
+ * not overlap M, N or W0. All pointers 16-byte aligned. Supported: d = 64 and
+ * 128, fp32 arithmetic (fused multiply-add, k ascending). One launch, one
+ * block per sequence; nseg - 1 (or nseg, with W_end) dependent d^3 products.
+ */
+TTT_API ttt_status ttt_affine_prefix(const float *M, const float *N, const float *W0, float *W_in,
+                                     float *W_end, int S, int H, int nseg, int d,
+                                     long long seq_stride, long long seg_stride, unsigned flags,
+                                     ttt_stream stream);
+
+/*
  * Synchronises `stream`, then returns TTT_OK, TTT_ERR_DEVICE_TIMEOUT if a
  * kernel of this library ran out of a bounded wait since the last call
  * (the word is then cleared), or TTT_ERR_LAUNCH if the stream reports a CUDA

@@ -67,6 +67,13 @@ def lib() -> ctypes.CDLL:
         L.ttt_chunk_fwd.argtypes = [_P] * 7 + [_I] * 6 + [ctypes.c_uint, _P, ctypes.c_size_t, _P]
         L.ttt_chunk_fwd_noalloc.restype = _I
         L.ttt_chunk_fwd_noalloc.argtypes = [_P] * 7 + [_I] * 6 + [ctypes.c_uint, _P]
+        L.ttt_chunk_map_workspace_bytes.restype = ctypes.c_size_t
+        L.ttt_chunk_map_workspace_bytes.argtypes = [_I] * 6
+        L.ttt_chunk_map.restype = _I
+        L.ttt_chunk_map.argtypes = [_P] * 5 + [_I] * 6 + [_P, ctypes.c_size_t, _P]
+        L.ttt_affine_prefix.restype = _I
+        L.ttt_affine_prefix.argtypes = ([_P] * 5 + [_I] * 4 + [ctypes.c_longlong] * 2
+                                        + [ctypes.c_uint, _P])
         L.ttt_device_status.restype = _I
         L.ttt_device_status.argtypes = [_P]
         L.ttt_launch_count.restype = ctypes.c_ulonglong
@@ -189,6 +196,24 @@ def ttt_chunk_fwd_noalloc(Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, dt, fla
     rc = lib().ttt_chunk_fwd_noalloc(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0), _ptr(Z),
                                      _ptr(W_out), B, H, T, d, chunk, dt, flags, _stream(stream))
     return _check("ttt_chunk_fwd_noalloc", rc) if check else rc
+
+
+def ttt_chunk_map_workspace_bytes(B, H, T, d, chunk, dt) -> int:
+    return int(lib().ttt_chunk_map_workspace_bytes(B, H, T, d, chunk, dt))
+
+
+def ttt_chunk_map(K, V, eta, M, N, B, H, T, d, chunk, dt, workspace, workspace_bytes, stream=None,
+                  check=True):
+    rc = lib().ttt_chunk_map(_ptr(K), _ptr(V), _ptr(eta), _ptr(M), _ptr(N), B, H, T, d, chunk, dt,
+                             _ptr(workspace), workspace_bytes, _stream(stream))
+    return _check("ttt_chunk_map", rc) if check else rc
+
+
+def ttt_affine_prefix(M, N, W0, W_in, W_end, S, H, nseg, d, seq_stride, seg_stride, flags,
+                      stream=None, check=True):
+    rc = lib().ttt_affine_prefix(_ptr(M), _ptr(N), _ptr(W0), _ptr(W_in), _ptr(W_end), S, H, nseg,
+                                 d, seq_stride, seg_stride, flags, _stream(stream))
+    return _check("ttt_affine_prefix", rc) if check else rc
 
 
 def ttt_device_status(stream=None) -> int:
@@ -332,3 +357,28 @@ def chunk_fwd(Q, K, V, eta, W0, *, chunk, w0_per_seq=False, workspace=None, stre
     ttt_chunk_fwd(Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, _dtype_code(Q), flags,
                   workspace, need, stream)
     return Z, W_out
+
+
+def chunk_map(K, V, eta, *, chunk, workspace=None, stream=None):
+    """Affine map W -> M W + N of each sequence's chunks (see ttt_chunk_map).
+    Returns (M, N), each [B, H, d, d] fp32."""
+    import torch
+    B, H, T, d = K.shape
+    M = torch.empty((B, H, d, d), dtype=torch.float32, device=K.device)
+    N = torch.empty_like(M)
+    dt = _dtype_code(K)
+    need = ttt_chunk_map_workspace_bytes(B, H, T, d, chunk, dt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=K.device)
+    ttt_chunk_map(K, V, eta, M, N, B, H, T, d, chunk, dt, workspace,
+                  workspace.numel() * workspace.element_size(), stream)
+    return M, N
+
+
+def affine_prefix(M, N, W0, W_in, W_end=None, *, S, H, nseg, seq_stride, seg_stride,
+                  w0_per_seq=False, stream=None):
+    """Fold segment maps into starting weights (see ttt_affine_prefix); writes
+    W_in and, if given, W_end."""
+    d = M.shape[-1]
+    ttt_affine_prefix(M, N, W0, W_in, W_end, S, H, nseg, d, seq_stride, seg_stride,
+                      TTT_F_W0_PER_SEQ if w0_per_seq else 0, stream)

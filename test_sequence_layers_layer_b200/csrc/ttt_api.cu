@@ -163,9 +163,18 @@ cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const 
                              float *dK, float *dV, float *deta, float *dW0, int B, int H, int T,
                              int d, int chunk, bool bf16, bool w0_per_seq, void *workspace,
                              cudaStream_t s);
+// Affine-map kernels of the sequence-parallel large-chunk forward (ttt_affine.cu).
+cudaError_t launch_affine_eye(float *W, int S, int d, cudaStream_t s);
+cudaError_t launch_affine_prefix(const float *M, const float *N, const float *W0, float *W_in,
+                                 float *W_end, int S, int H, int nseg, int d, long long seq_stride,
+                                 long long seg_stride, bool w0_per_seq, cudaStream_t s);
 }  // namespace ttt
 
 using namespace ttt;
+
+namespace {
+size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
+}  // namespace
 
 extern "C" {
 
@@ -357,6 +366,94 @@ ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, const floa
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
     return launched(tc ? launch_chunk_tc(a, cs) : launch_chunk_simt(a, cs));
+}
+
+size_t ttt_chunk_map_workspace_bytes(int B, int H, int T, int d, int chunk, ttt_dtype dt) {
+    if (B <= 0 || H <= 0 || T <= 0 || chunk <= 0 || T % chunk || chunk % 128) return 0;
+    if ((d != 64 && d != 128) || (dt != TTT_BF16 && dt != TTT_FP32)) return 0;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return 0;
+    const size_t n = (size_t)B * H * T * d, e = dt == TTT_BF16 ? 2 : 4;
+    const size_t fwd = chunk_tc_supported(d, chunk, dt == TTT_BF16)
+                           ? ttt_chunk_workspace_bytes(B, H, T, d, chunk)
+                           : 0;
+    return round256(n * e) + round256(n * 2) + round256((size_t)B * H * d * d * sizeof(float)) + fwd;
+}
+
+ttt_status ttt_chunk_map(const void *K, const void *V, const float *eta, float *M, float *N, int B,
+                         int H, int T, int d, int chunk, ttt_dtype dt, void *workspace,
+                         size_t workspace_bytes, ttt_stream stream) {
+    if (!K || !V || !eta || !M || !N) return TTT_ERR_PTR;
+    if (B <= 0 || H <= 0 || T <= 0 || chunk <= 0 || T % chunk != 0 || chunk % 128 != 0)
+        return TTT_ERR_SHAPE;
+    if (d != 64 && d != 128) return TTT_ERR_SHAPE;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return TTT_ERR_SHAPE;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(M) || !aligned16(N)) return TTT_ERR_ALIGN;
+    if (M == N) return TTT_ERR_ARG;
+    const size_t need = ttt_chunk_map_workspace_bytes(B, H, T, d, chunk, dt);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return TTT_ERR_WORKSPACE;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {K, V, eta, M, N, workspace};
+    st = check_device_ptrs(ptrs, 6);
+    if (st != TTT_OK) return st;
+
+    const size_t S = (size_t)B * H, n = S * T * d, e = dt == TTT_BF16 ? 2 : 4;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    void *v_zero = ws;                                    // [B][H][T][d], V = 0
+    void *z_scratch = ws + round256(n * e);               // discarded read-outs, bf16
+    float *w_start = reinterpret_cast<float *>(ws + round256(n * e) + round256(n * 2));
+    unsigned char *fwd_ws = reinterpret_cast<unsigned char *>(w_start) +
+                            round256(S * d * d * sizeof(float));
+    const size_t fwd_bytes = workspace_bytes - (size_t)(fwd_ws - ws);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const unsigned f = TTT_F_W0_PER_SEQ | TTT_F_Z_BF16;
+    timing_begin(cs);
+    // M: the forward from W = I with V = 0 (every B_c = 0)
+    if (cudaMemsetAsync(v_zero, 0, n * e, cs) != cudaSuccess) return TTT_ERR_LAUNCH;
+    if (launch_affine_eye(w_start, (int)S, d, cs) != cudaSuccess) return TTT_ERR_LAUNCH;
+    st = ttt_chunk_fwd(K, K, v_zero, eta, w_start, z_scratch, M, B, H, T, d, chunk, dt, f, fwd_ws,
+                       fwd_bytes, stream);
+    if (st != TTT_OK) return st;
+    // N: the forward from W = 0
+    if (cudaMemsetAsync(w_start, 0, S * d * d * sizeof(float), cs) != cudaSuccess)
+        return TTT_ERR_LAUNCH;
+    return ttt_chunk_fwd(K, K, V, eta, w_start, z_scratch, N, B, H, T, d, chunk, dt, f, fwd_ws,
+                         fwd_bytes, stream);
+}
+
+ttt_status ttt_affine_prefix(const float *M, const float *N, const float *W0, float *W_in,
+                             float *W_end, int S, int H, int nseg, int d, long long seq_stride,
+                             long long seg_stride, unsigned flags, ttt_stream stream) {
+    if (flags & ~TTT_F_W0_PER_SEQ) return TTT_ERR_ARG;
+    const bool per_seq = flags & TTT_F_W0_PER_SEQ;
+    if (!M || !N || !W0 || !W_in) return TTT_ERR_PTR;
+    if (S <= 0 || H <= 0 || nseg <= 0 || S > (1 << 30) || nseg > (1 << 16)) return TTT_ERR_SHAPE;
+    if ((d != 64 && d != 128) || (!per_seq && S % H)) return TTT_ERR_SHAPE;
+    const long long dd = (long long)d * d;
+    if (seq_stride < 0 || seg_stride < 0 || seq_stride > (1LL << 40) || seg_stride > (1LL << 40))
+        return TTT_ERR_ARG;
+    const bool nested_seq = seg_stride >= dd && seq_stride >= (long long)nseg * seg_stride;
+    const bool nested_seg = seq_stride >= dd && seg_stride >= (long long)S * seq_stride;
+    const bool single = (nseg == 1 && seq_stride >= dd) || (S == 1 && seg_stride >= dd);
+    if (!nested_seq && !nested_seg && !single) return TTT_ERR_ARG;
+    if (seq_stride % 4 || seg_stride % 4) return TTT_ERR_ALIGN;
+    if (!aligned16(M) || !aligned16(N) || !aligned16(W0) || !aligned16(W_in) ||
+        (W_end && !aligned16(W_end)))
+        return TTT_ERR_ALIGN;
+    const float *outs[] = {W_in, W_end};
+    for (const float *o : outs)
+        if (o && (o == M || o == N || o == W0)) return TTT_ERR_ARG;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {M, N, W0, W_in, W_end};
+    st = check_device_ptrs(ptrs, 5);
+    if (st != TTT_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    return launched(launch_affine_prefix(M, N, W0, W_in, W_end, S, H, nseg, d, seq_stride,
+                                         seg_stride, per_seq, cs));
 }
 
 ttt_status ttt_device_status(ttt_stream stream) {

@@ -119,3 +119,53 @@ def test_backward_host_validation():
     assert call(T=5000) == -2                         # T % chunk != 0
     assert call(dQ=A + 4) == -4
     assert call(workspace_bytes=need - 1) == -9
+
+
+def test_chunk_map_and_affine_prefix_host_validation():
+    """ttt_chunk_map and ttt_affine_prefix reject bad arguments before any
+    launch; arguments that pass every host check reach the architecture
+    check, which fails without a GPU."""
+    A = ALIGNED
+    B, H, T, d, C = 1, 2, 4096, 128, 2048
+    need = ttt.ttt_chunk_map_workspace_bytes(B, H, T, d, C, ttt.TTT_BF16)
+    n = B * H * T * d
+    r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert need == (r256(2 * n) + r256(2 * n) + r256(4 * B * H * d * d)
+                    + ttt.ttt_chunk_workspace_bytes(B, H, T, d, C))
+    # fp32 runs the CUDA-core forward, which needs no workspace of its own
+    assert ttt.ttt_chunk_map_workspace_bytes(B, H, T, d, C, ttt.TTT_FP32) == \
+        r256(4 * n) + r256(2 * n) + r256(4 * B * H * d * d)
+    assert ttt.ttt_chunk_map_workspace_bytes(B, H, T, 96, C, ttt.TTT_BF16) == 0
+    assert ttt.ttt_chunk_map_workspace_bytes(B, H, 3000, d, C, ttt.TTT_BF16) == 0
+    cm = dict(K=A, V=A, eta=A, M=A, N=A + (1 << 20), B=B, H=H, T=T, d=d, chunk=C,
+              dt=ttt.TTT_BF16, workspace=A, workspace_bytes=need, stream=0)
+    call = lambda **kw: ttt.ttt_chunk_map(**{**cm, **kw}, check=False)  # noqa: E731
+    assert call(K=None) == -5
+    assert call(T=3000) == -2
+    assert call(chunk=1000) == -2
+    assert call(d=96) == -2
+    assert call(dt=7) == -3
+    assert call(M=A + 4) == -4
+    assert call(N=A) == -1                        # M and N must differ
+    assert call(workspace_bytes=need - 1) == -9
+    assert call(workspace=A + 16) == -9
+    assert call() == -8                           # no GPU here
+    dd = 64 * 64
+    ap = dict(M=A, N=A + (1 << 22), W0=A + (2 << 22), W_in=A + (3 << 22), W_end=None, S=4, H=2,
+              nseg=3, d=64, seq_stride=3 * dd, seg_stride=dd, flags=0, stream=0)
+    call = lambda **kw: ttt.ttt_affine_prefix(**{**ap, **kw}, check=False)  # noqa: E731
+    assert call() == -8                           # sequence-major layout passes
+    assert call(seq_stride=dd, seg_stride=4 * dd) == -8   # segment-major layout passes
+    assert call(seq_stride=dd, seg_stride=dd) == -1       # (s, j) blocks would overlap
+    assert call(seq_stride=2 * dd) == -1                  # 3 segments do not fit
+    assert call(seg_stride=dd - 4) == -1
+    assert call(seq_stride=3 * dd + 2) == -4              # stride not a multiple of 4
+    assert call(nseg=1, seq_stride=dd, seg_stride=0) == -8
+    assert call(S=3) == -2                                # shared W0: S % H == 0
+    assert call(S=3, flags=ttt.TTT_F_W0_PER_SEQ) == -8
+    assert call(d=32) == -2
+    assert call(flags=ttt.TTT_F_LN) == -1
+    assert call(W_in=None) == -5
+    assert call(W_in=A) == -1                             # output aliases M
+    assert call(W_end=A + (1 << 22)) == -1                # output aliases N
+    assert call(W0=A + 8) == -4

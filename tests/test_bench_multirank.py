@@ -40,7 +40,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_ranks_reduce_and_shard():
     world, port = 2, 29500 + os.getpid() % 1000
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
