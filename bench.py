@@ -583,6 +583,86 @@ def decode_arm(args, wl):
     }
 
 
+def segmented_arm(args, wl):
+    """`--segments N` (large-chunk workloads): the forward split into N
+    segments of whole chunks per sequence on one GPU
+    (seqpar.chunk_fwd_segmented: segment maps, their fold, the segments'
+    forwards). L2 flushed between steps. Reports tokens/s of the whole call
+    and the device time of each of its three stages."""
+    import torch
+    import test_sequence_layers_layer_b200 as ttt
+    from test_sequence_layers_layer_b200 import seqpar
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    nseg = args.segments
+    B, H, T, d, C = wl.B, wl.H, wl.T, wl.d, wl.b
+    if T % (nseg * C):
+        raise SystemExit(f"--segments {nseg}: T = {T} does not split into segments of whole "
+                         f"chunks of {C}")
+    x = device_tensors(synth.make_inputs(wl), dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    Ts = T // nseg
+    view = {k: x[k].view(B, H * nseg, Ts, d) for k in ("Q", "K", "V")}
+    view["eta"] = x["eta"].view(B, H * nseg, Ts)
+
+    def call():
+        return seqpar.chunk_fwd_segmented(x["Q"], x["K"], x["V"], x["eta"], x["W1"], chunk=C,
+                                          nseg=nseg, z_bf16=args.z_bf16, stream=stream)
+
+    def stages(ev):
+        ev[0].record(stream)
+        M, N = ttt.chunk_map(view["K"], view["V"], view["eta"], chunk=C, stream=stream)
+        ev[1].record(stream)
+        W_in = torch.empty_like(M)
+        W_out = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+        ttt.affine_prefix(M, N, x["W1"], W_in, W_out, S=B * H, H=H, nseg=nseg,
+                          seq_stride=nseg * d * d, seg_stride=d * d, stream=stream)
+        ev[2].record(stream)
+        ttt.chunk_fwd(view["Q"], view["K"], view["V"], view["eta"], W_in, chunk=C,
+                      w0_per_seq=True, stream=stream, want_w=False, z_bf16=args.z_bf16)
+        ev[3].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            call()
+        stream.synchronize()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        n0 = ttt.ttt_launch_count()
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record(stream)
+            call()
+            ends[k].record(stream)
+        stream.synchronize()
+        launches = ttt.ttt_launch_count() - n0
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        for k in range(args.steps):
+            flush.zero_()
+            stages(evs[k])
+        stream.synchronize()
+    if ttt.ttt_device_status(stream.cuda_stream) != 0:
+        raise RuntimeError("device status error in the segmented loop")
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    stage_ms = [sum(ev[i].elapsed_time(ev[i + 1]) for ev in evs) / args.steps for i in range(3)]
+    return {
+        "metric": "large-chunk TTT forward, sequence split into segments, tokens/s at 1 B200",
+        "value": wl.tokens / (ms / 1e3), "unit": "tokens/s", "higher_is_better": True,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "dtype": wl.dtype, "data": "synthetic (seeded SplitMix64 normals; bf16-rounded Q/K/V)",
+        "config": {"workload": f"{wl.name}_seg{nseg}", "B": B, "H": H, "T": T, "d": d,
+                   "chunk": C, "segments": nseg, "z_dtype": "bf16" if args.z_bf16 else "fp32",
+                   "l2": "flushed between steps (256 MiB write)"},
+        "stages_ms": {"segment_maps": stage_ms[0], "fold": stage_ms[1],
+                      "segment_forwards": stage_ms[2]},
+        "dependent_steps": {"fold": nseg - 1, "chunk_scan": T // (nseg * C)},
+        "gpu_launches": launches,
+    }
+
+
 # fp32 FMA lanes of a B200 (148 SMs x 128 lanes, 2 FLOP per FMA) at the SM clock:
 # the peak of a kernel bound by plain fp32 arithmetic on CUDA cores.
 FP32_LANES = 148 * 128
@@ -736,6 +816,8 @@ def main():
                     help="time the TTT-Linear backward (linear workloads) instead")
     ap.add_argument("--decode", type=int, default=0,
                     help="time N single-token decode steps (linear workloads) instead")
+    ap.add_argument("--segments", type=int, default=0,
+                    help="time the large-chunk forward split into N segments per sequence")
     ap.add_argument("--B", type=int, default=None,
                     help="override the workload's batch size (smaller profiling cases)")
     args = ap.parse_args()
@@ -759,6 +841,13 @@ def main():
             ap.error("--decode times the linear workloads")
         if rank == 0:
             print(json.dumps(decode_arm(args, wl)), flush=True)
+        return
+
+    if args.segments:
+        if wl.kind != "chunk":
+            ap.error("--segments times the large-chunk workloads")
+        if rank == 0:
+            print(json.dumps(segmented_arm(args, wl)), flush=True)
         return
 
     if args.impl == "reference":
