@@ -1,6 +1,8 @@
 /*
  * ttt.h -- C ABI of libttt.so: the forward pass of a Test-Time-Training (TTT)
- * layer on one NVIDIA B200 (sm_100a).
+ * layer on one NVIDIA B200 (sm_100a), the backward passes of TTT-Linear and
+ * large-chunk TTT, and the affine-map calls of a sequence-parallel
+ * large-chunk forward.
  *
  * What the layer computes. The hidden state of a TTT layer is a fast weight W
  * per (batch, head) sequence: a linear map, or a small MLP. Tokens arrive as

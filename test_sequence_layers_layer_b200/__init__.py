@@ -1,12 +1,15 @@
 """Python binding of libttt.so, the B200 library for a Test-Time-Training (TTT)
-layer: its forward pass, and the backward pass of TTT-Linear.
+layer: its forward passes (TTT-Linear, TTT-MLP, large chunk), the backward
+passes of TTT-Linear and large-chunk TTT, and the affine-map calls behind the
+sequence-parallel large-chunk forward (seqpar.py).
 
 The functions named like the C ABI (ttt_linear_fwd, ttt_mlp_fwd,
 ttt_chunk_fwd, ...) take exactly the C arguments; a pointer argument may be a
 torch tensor (its data_ptr() is passed), an int address, or None. They only
 marshal arguments: every step of the computation runs in the library's CUDA
-kernels. linear_fwd / mlp_fwd / chunk_fwd are conveniences that read the
-shapes off torch tensors and allocate the outputs with torch.
+kernels. linear_fwd / mlp_fwd / chunk_fwd / linear_bwd / chunk_bwd /
+chunk_map / affine_prefix are conveniences that read the shapes off torch
+tensors and allocate the outputs (and workspaces) with torch.
 
 There is no fallback: if libttt.so is missing or fails to load, every call
 raises.
