@@ -71,15 +71,26 @@ def max_rel_err(gpu, ref, wl, seqs=None) -> float:
     return float(np.abs(g - r).max() / max(np.abs(r).max(), 1e-30))
 
 
+def elementwise_rel_err(gpu, ref, wl, seqs=None, floor=1e-3) -> float:
+    """Largest per-element relative error, each element's denominator floored
+    at floor * max |ref| (reported beside max_rel_err, not asserted)."""
+    g, r = select(gpu, wl, seqs), select(ref, wl, seqs)
+    den = np.maximum(np.abs(r), floor * max(np.abs(r).max(), 1e-30))
+    return float((np.abs(g - r) / den).max())
+
+
 def check_parity(inp, seqs=None, gpu_out=None):
-    """Runs both sides, asserts every output within tolerance, returns errors."""
+    """Runs both sides, asserts every output within tolerance, returns errors.
+    Prints, per output, the asserted error and the floored per-element one."""
     wl = inp.wl
     gpu_out = gpu_out or run_gpu(inp)
     ref_out = run_oracle(inp, seqs)
     tol = TOL[wl.dtype]
     errs = []
-    for g, r in zip(gpu_out, ref_out):
+    for i, (g, r) in enumerate(zip(gpu_out, ref_out)):
         assert np.all(np.isfinite(select(g, wl, seqs)))
         errs.append(max_rel_err(g, r, wl, seqs))
+        print(f"{wl.name} output {i}: max rel err {errs[-1]:.2e}, per-element (floor 1e-3) "
+              f"{elementwise_rel_err(g, r, wl, seqs):.2e}")
     assert max(errs) <= tol, f"{wl.name}: errors {errs} > {tol}"
     return errs
