@@ -284,6 +284,23 @@ TTT_API ttt_status ttt_chunk_map(const void *K, const void *V, const float *eta,
                                  void *workspace, size_t workspace_bytes, ttt_stream stream);
 
 /*
+ * ttt_linear_map: the same map for TTT-Linear without LayerNorm, whose
+ * mini-batch update ("Key Architectural Mechanics of TTT-Linear", part 4:
+ * every gradient of mini-batch m at its starting weight W_m) is
+ *   W_{m+1} = W_m - K_m^T diag(eta) (K_m W_m - V_m) = (I - A_m) W_m + B_m.
+ * M, N [B][H][d][d] fp32 as for ttt_chunk_map; the segment is T tokens in
+ * mini-batches of b (a last partial mini-batch is a step of its own, as in
+ * ttt_linear_fwd). Computed with ttt_linear_fwd (no TTT_F_LN): from W = I with
+ * V = 0, and from W = 0. workspace: at least ttt_linear_map_workspace_bytes(...)
+ * bytes, 256-byte aligned, clobbered. Supported shapes and dtypes: those of
+ * ttt_linear_fwd; the workspace size is 0 for an unsupported shape.
+ */
+TTT_API size_t ttt_linear_map_workspace_bytes(int B, int H, int T, int d, int b, ttt_dtype dt);
+TTT_API ttt_status ttt_linear_map(const void *K, const void *V, const float *eta, float *M,
+                                  float *N, int B, int H, int T, int d, int b, ttt_dtype dt,
+                                  void *workspace, size_t workspace_bytes, ttt_stream stream);
+
+/*
  * The fold of segment maps into starting weights, for S sequences of nseg
  * segments each:
  *   W_in[s][0] = W0[s],  W_in[s][j+1] = M[s][j] W_in[s][j] + N[s][j],

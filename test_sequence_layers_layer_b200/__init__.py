@@ -74,6 +74,10 @@ def lib() -> ctypes.CDLL:
         L.ttt_chunk_map_workspace_bytes.argtypes = [_I] * 6
         L.ttt_chunk_map.restype = _I
         L.ttt_chunk_map.argtypes = [_P] * 5 + [_I] * 6 + [_P, ctypes.c_size_t, _P]
+        L.ttt_linear_map_workspace_bytes.restype = ctypes.c_size_t
+        L.ttt_linear_map_workspace_bytes.argtypes = [_I] * 6
+        L.ttt_linear_map.restype = _I
+        L.ttt_linear_map.argtypes = [_P] * 5 + [_I] * 6 + [_P, ctypes.c_size_t, _P]
         L.ttt_affine_prefix.restype = _I
         L.ttt_affine_prefix.argtypes = ([_P] * 5 + [_I] * 4 + [ctypes.c_longlong] * 2
                                         + [ctypes.c_uint, _P])
@@ -210,6 +214,17 @@ def ttt_chunk_map(K, V, eta, M, N, B, H, T, d, chunk, dt, workspace, workspace_b
     rc = lib().ttt_chunk_map(_ptr(K), _ptr(V), _ptr(eta), _ptr(M), _ptr(N), B, H, T, d, chunk, dt,
                              _ptr(workspace), workspace_bytes, _stream(stream))
     return _check("ttt_chunk_map", rc) if check else rc
+
+
+def ttt_linear_map_workspace_bytes(B, H, T, d, b, dt) -> int:
+    return int(lib().ttt_linear_map_workspace_bytes(B, H, T, d, b, dt))
+
+
+def ttt_linear_map(K, V, eta, M, N, B, H, T, d, b, dt, workspace, workspace_bytes, stream=None,
+                   check=True):
+    rc = lib().ttt_linear_map(_ptr(K), _ptr(V), _ptr(eta), _ptr(M), _ptr(N), B, H, T, d, b, dt,
+                              _ptr(workspace), workspace_bytes, _stream(stream))
+    return _check("ttt_linear_map", rc) if check else rc
 
 
 def ttt_affine_prefix(M, N, W0, W_in, W_end, S, H, nseg, d, seq_stride, seg_stride, flags,
@@ -375,6 +390,22 @@ def chunk_map(K, V, eta, *, chunk, workspace=None, stream=None):
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=K.device)
     ttt_chunk_map(K, V, eta, M, N, B, H, T, d, chunk, dt, workspace,
                   workspace.numel() * workspace.element_size(), stream)
+    return M, N
+
+
+def linear_map(K, V, eta, *, b, workspace=None, stream=None):
+    """Affine map W -> M W + N of each sequence's mini-batches of TTT-Linear
+    without LayerNorm (see ttt_linear_map). Returns (M, N), each [B, H, d, d]."""
+    import torch
+    B, H, T, d = K.shape
+    M = torch.empty((B, H, d, d), dtype=torch.float32, device=K.device)
+    N = torch.empty_like(M)
+    dt = _dtype_code(K)
+    need = ttt_linear_map_workspace_bytes(B, H, T, d, b, dt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=K.device)
+    ttt_linear_map(K, V, eta, M, N, B, H, T, d, b, dt, workspace,
+                   workspace.numel() * workspace.element_size(), stream)
     return M, N
 
 

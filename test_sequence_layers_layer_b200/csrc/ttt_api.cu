@@ -423,6 +423,54 @@ ttt_status ttt_chunk_map(const void *K, const void *V, const float *eta, float *
                          fwd_bytes, stream);
 }
 
+size_t ttt_linear_map_workspace_bytes(int B, int H, int T, int d, int b, ttt_dtype dt) {
+    if (B <= 0 || H <= 0 || T <= 0 || b <= 0 || b > 64 || !supported_d(d) || b * d > 4096) return 0;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return 0;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return 0;
+    const size_t n = (size_t)B * H * T * d, e = dt == TTT_BF16 ? 2 : 4;
+    return round256(n * e) + round256(n * 2) + round256((size_t)B * H * d * d * sizeof(float));
+}
+
+ttt_status ttt_linear_map(const void *K, const void *V, const float *eta, float *M, float *N,
+                          int B, int H, int T, int d, int b, ttt_dtype dt, void *workspace,
+                          size_t workspace_bytes, ttt_stream stream) {
+    if (!K || !V || !eta || !M || !N) return TTT_ERR_PTR;
+    if (B <= 0 || H <= 0 || T <= 0 || b <= 0 || b > 64) return TTT_ERR_SHAPE;
+    if (!supported_d(d) || b * d > 4096) return TTT_ERR_SHAPE;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return TTT_ERR_SHAPE;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(M) || !aligned16(N)) return TTT_ERR_ALIGN;
+    if (M == N) return TTT_ERR_ARG;
+    const size_t need = ttt_linear_map_workspace_bytes(B, H, T, d, b, dt);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return TTT_ERR_WORKSPACE;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {K, V, eta, M, N, workspace};
+    st = check_device_ptrs(ptrs, 6);
+    if (st != TTT_OK) return st;
+
+    const size_t S = (size_t)B * H, n = S * T * d, e = dt == TTT_BF16 ? 2 : 4;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    void *v_zero = ws;                                    // [B][H][T][d], V = 0
+    void *z_scratch = ws + round256(n * e);               // discarded read-outs, bf16
+    float *w_start = reinterpret_cast<float *>(ws + round256(n * e) + round256(n * 2));
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const unsigned f = TTT_F_W0_PER_SEQ | TTT_F_Z_BF16;  // f(k) = k W: no TTT_F_LN
+    timing_begin(cs);
+    // M: the forward from W = I with V = 0
+    if (cudaMemsetAsync(v_zero, 0, n * e, cs) != cudaSuccess) return TTT_ERR_LAUNCH;
+    if (launch_affine_eye(w_start, (int)S, d, cs) != cudaSuccess) return TTT_ERR_LAUNCH;
+    st = ttt_linear_fwd(K, K, v_zero, eta, w_start, nullptr, nullptr, z_scratch, M, B, H, T, d, b,
+                        dt, f, stream);
+    if (st != TTT_OK) return st;
+    // N: the forward from W = 0
+    if (cudaMemsetAsync(w_start, 0, S * d * d * sizeof(float), cs) != cudaSuccess)
+        return TTT_ERR_LAUNCH;
+    return ttt_linear_fwd(K, K, V, eta, w_start, nullptr, nullptr, z_scratch, N, B, H, T, d, b, dt,
+                          f, stream);
+}
+
 ttt_status ttt_affine_prefix(const float *M, const float *N, const float *W0, float *W_in,
                              float *W_end, int S, int H, int nseg, int d, long long seq_stride,
                              long long seg_stride, unsigned flags, ttt_stream stream) {

@@ -169,3 +169,26 @@ def test_chunk_map_and_affine_prefix_host_validation():
     assert call(W_in=A) == -1                             # output aliases M
     assert call(W_end=A + (1 << 22)) == -1                # output aliases N
     assert call(W0=A + 8) == -4
+
+
+def test_linear_map_host_validation():
+    A = ALIGNED
+    B, H, T, d, b = 1, 2, 256, 64, 16
+    need = ttt.ttt_linear_map_workspace_bytes(B, H, T, d, b, ttt.TTT_BF16)
+    n = B * H * T * d
+    r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert need == r256(2 * n) + r256(2 * n) + r256(4 * B * H * d * d)
+    assert ttt.ttt_linear_map_workspace_bytes(B, H, T, 48, b, ttt.TTT_BF16) == 0
+    assert ttt.ttt_linear_map_workspace_bytes(B, H, T, d, 128, ttt.TTT_BF16) == 0
+    lm = dict(K=A, V=A, eta=A, M=A, N=A + (1 << 20), B=B, H=H, T=T, d=d, b=b, dt=ttt.TTT_BF16,
+              workspace=A, workspace_bytes=need, stream=0)
+    call = lambda **kw: ttt.ttt_linear_map(**{**lm, **kw}, check=False)  # noqa: E731
+    assert call(eta=None) == -5
+    assert call(d=48) == -2
+    assert call(b=0) == -2
+    assert call(dt=5) == -3
+    assert call(N=A) == -1
+    assert call(V=A + 2) == -4
+    assert call(workspace_bytes=need - 1) == -9
+    assert call() == -8                           # no GPU here
+    assert call(T=250) == -8                      # a partial last mini-batch is accepted

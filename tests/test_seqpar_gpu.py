@@ -1,10 +1,11 @@
-"""Sequence-parallel large-chunk forward on one GPU, through the C ABI:
-ttt_chunk_map against the oracle's affine segment maps (oracle/affine.py),
+"""Sequence-parallel forward on one GPU, through the C ABI: ttt_chunk_map and
+ttt_linear_map against the oracle's affine segment maps (oracle/affine.py),
 ttt_affine_prefix against a float64 fold in both stride layouts, and the
-segmented forward (seqpar.chunk_fwd_segmented) against the oracle's forward
-of the whole sequence. Error metric and tolerances as in the other parity
-tests: max |gpu - ref| / max |ref| per output, 2e-3 for bf16 inputs, 1e-5 for
-fp32 inputs (the fold itself, fp32 throughout, within 1e-5)."""
+segmented forwards (seqpar.chunk_fwd_segmented, seqpar.linear_fwd_segmented)
+against the oracle's forward of the whole sequence. Error metric and
+tolerances as in the other parity tests: max |gpu - ref| / max |ref| per
+output, 2e-3 for bf16 inputs, 1e-5 for fp32 inputs (the fold itself, fp32
+throughout, within 1e-5)."""
 import numpy as np
 import pytest
 import torch
@@ -139,3 +140,43 @@ def test_segmented_full_size_sampled_sequences():
     Wo = Wr.reshape(wl.B * wl.H, wl.d, wl.d)
     for s in (0, 31):
         assert _rel(Zg[s], Zo[s]) <= TOL["bf16"] and _rel(Wg[s], Wo[s]) <= TOL["bf16"]
+
+
+# ------------------------------------------------------- TTT-Linear without LN
+L = synth.WORKLOADS["linear_ln_d64_b8h12_t2048"]
+LINEAR_CASES = {
+    # bf16, d = 64, b = 16 runs the tensor-core scan; fp32 the CUDA-core kernel
+    "linear_noln_bf16_d64_b16": L.scaled(B=2, H=2, T=512, ln=False),
+    "linear_noln_fp32_d64_b8": L.scaled(B=1, H=3, T=256, b=8, ln=False, dtype="fp32"),
+}
+
+
+@pytest.mark.parametrize("name", list(LINEAR_CASES))
+def test_linear_map_matches_oracle(name):
+    wl = LINEAR_CASES[name]
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    M, N = ttt.linear_map(x["K"], x["V"], x["eta"], b=wl.b)
+    torch.cuda.synchronize()
+    assert ttt.ttt_device_status() == 0
+    Mr, Nr = affine.segment_map(inp.K, inp.V, inp.eta, chunk=wl.b)
+    assert _rel(_np(M), Mr) <= TOL[wl.dtype]
+    assert _rel(_np(N), Nr) <= TOL[wl.dtype]
+
+
+@pytest.mark.parametrize("name,nseg", [("linear_noln_bf16_d64_b16", 2),
+                                       ("linear_noln_bf16_d64_b16", 8),
+                                       ("linear_noln_fp32_d64_b8", 4)])
+def test_linear_segmented_forward_matches_whole_sequence(name, nseg):
+    wl = LINEAR_CASES[name]
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    Z, W_out = seqpar.linear_fwd_segmented(x["Q"], x["K"], x["V"], x["eta"], x["W1"], b=wl.b,
+                                           nseg=nseg)
+    torch.cuda.synchronize()
+    assert ttt.ttt_device_status() == 0
+    Zr, Wr = oracle.linear_primal(inp.Q, inp.K, inp.V, inp.eta, inp.W1, b=wl.b, ln=False)
+    assert _rel(_np(Z), Zr) <= TOL[wl.dtype]
+    assert _rel(_np(W_out), Wr) <= TOL[wl.dtype]
+    Zc, _ = ttt.linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], b=wl.b, ln=False)
+    assert _rel(_np(Z), _np(Zc)) <= TOL[wl.dtype]
