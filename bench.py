@@ -597,9 +597,6 @@ def segmented_arm(args, wl):
     torch.cuda.set_device(dev)
     nseg = args.segments
     B, H, T, d, C = wl.B, wl.H, wl.T, wl.d, wl.b
-    if T % (nseg * C):
-        raise SystemExit(f"--segments {nseg}: T = {T} does not split into segments of whole "
-                         f"chunks of {C}")
     x = device_tensors(synth.make_inputs(wl), dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
@@ -846,6 +843,9 @@ def main():
     if args.segments:
         if wl.kind != "chunk":
             ap.error("--segments times the large-chunk workloads")
+        if args.segments < 1 or wl.T % (args.segments * wl.b):
+            ap.error(f"--segments {args.segments}: T = {wl.T} does not split into segments of "
+                     f"whole chunks of {wl.b}")
         if rank == 0:
             print(json.dumps(segmented_arm(args, wl)), flush=True)
         return

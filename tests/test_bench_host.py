@@ -73,3 +73,13 @@ def test_latency_floor_accounting():
     f = bench.latency_floor(mlp, bench.kernel_plan(mlp), [1.0])
     assert f["concurrent_sequences"] == 48 and f["waves"] == 1
     assert isinstance(bench.cpu_model(), str)
+
+
+def test_segments_option_is_checked_before_any_gpu_work():
+    import subprocess
+    base = [sys.executable, os.path.join(ROOT, "bench.py"), "--workload",
+            "chunk_d128_c2048_b4h8_t32768"]
+    r = subprocess.run(base + ["--segments", "3"], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 2 and "does not split" in r.stderr
+    r = subprocess.run(base[:2] + ["--segments", "2"], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 2 and "large-chunk" in r.stderr
