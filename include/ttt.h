@@ -84,6 +84,10 @@ typedef void *ttt_stream; /* a cudaStream_t */
 #define TTT_F_W0_PER_SEQ 2u /* W0 is [B][H][...] instead of [H][...]           */
 #define TTT_F_Z_BF16 4u     /* forward entry points: Z is stored as bf16,
                                rounded to nearest even, instead of fp32     */
+#define TTT_F_L2_KEYS 8u    /* ttt_linear_fwd: keys scaled to unit length,
+                               k / max(||k||_2, 1e-12), wherever the inner
+                               loss and its gradient use them (the query is
+                               used as given); runs the fp32 CUDA-core kernel */
 
 #define TTT_ABI_VERSION 1
 
@@ -115,6 +119,11 @@ TTT_API const char *ttt_status_string(int status);
  *   starting weight); d in {16, 32, 64} and 1 <= b <= 64 with b*d <= 4096
  *   for TTT_FP32 and TTT_BF16; TTT_BF16 with d = 64, b = 16 runs the
  *   tensor-core scan, every other case the fp32 CUDA-core kernel.
+ * flags: TTT_F_LN, TTT_F_W0_PER_SEQ, TTT_F_Z_BF16, TTT_F_L2_KEYS. With
+ *   TTT_F_L2_KEYS the key is normalised, as in the PyTorch listing on "Test-
+ *   Time Training: Linear Complexity Beyond Attention"; with LayerNorm, the
+ *   residual k of f(k) = k + LN(k W) is the normalised key too. Every shape
+ *   then runs the fp32 CUDA-core kernel.
  */
 TTT_API ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const float *eta,
                           const float *W0, const float *ln_gamma, const float *ln_beta,

@@ -29,6 +29,7 @@ TTT_BF16, TTT_FP32 = 0, 1
 TTT_F_LN = 1
 TTT_F_W0_PER_SEQ = 2
 TTT_F_Z_BF16 = 4
+TTT_F_L2_KEYS = 8
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -287,15 +288,16 @@ def _dtype_code(t):
 
 
 def linear_fwd(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, w0_per_seq=False,
-               stream=None, want_w=True, z_bf16=False):
+               stream=None, want_w=True, z_bf16=False, l2_keys=False):
     """TTT-Linear forward. Q, K, V: [B,H,T,d] cuda tensors (bf16 or fp32).
+    l2_keys: normalise every key to unit length (TTT_F_L2_KEYS).
     Returns (Z fp32 [B,H,T,d], W_out fp32 [B,H,d,d] or None)."""
     import torch
     B, H, T, d = Q.shape
     Z = torch.empty((B, H, T, d), dtype=torch.bfloat16 if z_bf16 else torch.float32, device=Q.device)
     W_out = torch.empty((B, H, d, d), dtype=torch.float32, device=Q.device) if want_w else None
     flags = (TTT_F_LN if ln else 0) | (TTT_F_W0_PER_SEQ if w0_per_seq else 0) | \
-        (TTT_F_Z_BF16 if z_bf16 else 0)
+        (TTT_F_Z_BF16 if z_bf16 else 0) | (TTT_F_L2_KEYS if l2_keys else 0)
     ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                    _dtype_code(Q), flags, stream)
     return Z, W_out

@@ -163,6 +163,8 @@ cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const 
                              float *dK, float *dV, float *deta, float *dW0, int B, int H, int T,
                              int d, int chunk, bool bf16, bool w0_per_seq, void *workspace,
                              cudaStream_t s);
+// TTT-Linear on the fp32 CUDA-core kernel with L2-normalised keys (ttt_simt.cu).
+cudaError_t launch_linear_simt_keys(const LinearArgs &a, bool l2_keys, cudaStream_t s);
 // Affine-map kernels of the sequence-parallel large-chunk forward (ttt_affine.cu).
 cudaError_t launch_affine_eye(float *W, int S, int d, cudaStream_t s);
 cudaError_t launch_affine_prefix(const float *M, const float *N, const float *W0, float *W_in,
@@ -202,7 +204,7 @@ ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const flo
                           const float *W0, const float *ln_gamma, const float *ln_beta,
                           void *Z, float *W_out, int B, int H, int T, int d, int b,
                           ttt_dtype dt, unsigned flags, ttt_stream stream) {
-    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ | TTT_F_Z_BF16)) return TTT_ERR_ARG;
+    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ | TTT_F_Z_BF16 | TTT_F_L2_KEYS)) return TTT_ERR_ARG;
     const bool ln = flags & TTT_F_LN;
     if (!Q || !K || !V || !eta || !W0 || !Z) return TTT_ERR_PTR;
     if (ln && (!ln_gamma || !ln_beta)) return TTT_ERR_PTR;
@@ -224,6 +226,7 @@ ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const flo
                  dt == TTT_BF16, ln, (flags & TTT_F_W0_PER_SEQ) != 0, (flags & TTT_F_Z_BF16) != 0};
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
+    if (flags & TTT_F_L2_KEYS) return launched(launch_linear_simt_keys(a, true, cs));
     return launched(linear_tc_supported(d, b, dt == TTT_BF16) ? launch_linear_tc(a, cs)
                                                                 : launch_linear_simt(a, cs));
 }

@@ -87,7 +87,11 @@ __device__ __forceinline__ void load_tile(float *dst, const void *src, size_t ba
 // ---------------------------------------------------------------------------
 // TTT-Linear, mini-batch dual form, fp32.
 // Shared memory: W[d*d] | Qs Ks Vs Xs Zs [b*d] | S[b*b] | es[b].
-__global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a) {
+// l2_keys: every key is scaled to unit length, k / max(||k||, 1e-12), before
+// it enters the inner loss, its gradient and the update (the key
+// normalisation of the PyTorch listing on "Test-Time Training: Linear
+// Complexity Beyond Attention"); queries are used as given.
+__global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a, bool l2_keys) {
     extern __shared__ float sm[];
     const int d = a.d, b = a.b, T = a.T;
     const int seq = blockIdx.x, h = seq % a.H;
@@ -110,6 +114,16 @@ __global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a) {
         for (int e = nb * d + threadIdx.x; e < b * d; e += blockDim.x) Qs[e] = Ks[e] = Vs[e] = 0.f;
         for (int e = threadIdx.x; e < b; e += blockDim.x) es[e] = e < nb ? a.eta[(size_t)seq * T + m0 + e] : 0.f;
         __syncthreads();
+        if (l2_keys) {  // one warp per key row; padding rows are zero and stay zero
+            for (int t = warp; t < b; t += kWarps) {
+                float *k = Ks + t * d;
+                float ss = 0.f;
+                for (int j = threadIdx.x & 31; j < d; j += 32) ss = fmaf(k[j], k[j], ss);
+                const float inv = 1.f / fmaxf(sqrtf(warp_sum(ss)), 1e-12f);
+                for (int j = threadIdx.x & 31; j < d; j += 32) k[j] *= inv;
+            }
+            __syncthreads();
+        }
         // X = K W_m and Q W_m
         for (int e = threadIdx.x; e < b * d; e += blockDim.x) {
             const int t = e / d, j = e % d;
@@ -362,15 +376,19 @@ cudaError_t set_smem(K kernel, size_t smem) {
 
 }  // namespace
 
-cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s) {
+cudaError_t launch_linear_simt_keys(const LinearArgs &a, bool l2_keys, cudaStream_t s) {
     const size_t smem = sizeof(float) * ((size_t)a.d * a.d + 5 * (size_t)a.b * a.d +
                                          (size_t)a.b * a.b + a.b);
     cudaError_t e = set_smem(linear_simt_kernel, smem);
     if (e != cudaSuccess) return e;
-    linear_simt_kernel<<<a.B * a.H, kThreads, smem, s>>>(a);
+    linear_simt_kernel<<<a.B * a.H, kThreads, smem, s>>>(a, l2_keys);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch(s);
     return e;
+}
+
+cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s) {
+    return launch_linear_simt_keys(a, false, s);
 }
 
 size_t mlp_simt_smem(int d, int dh, int b) {

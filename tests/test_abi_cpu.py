@@ -41,7 +41,8 @@ def lin(**kw):
     (dict(b=0), -2),
     (dict(B=0), -2),
     (dict(dt=7), -3),
-    (dict(flags=8), -1),           # unknown flag bit
+    (dict(flags=16), -1),          # unknown flag bit
+    (dict(flags=ttt.TTT_F_LN | ttt.TTT_F_L2_KEYS), -8),  # L2 keys pass the host checks
     (dict(Q=None), -5),
     (dict(ln_gamma=None), -5),     # LN requires gamma/beta
     (dict(Q=ALIGNED + 4), -4),     # misaligned
