@@ -131,6 +131,23 @@ TTT_API ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, c
                           ttt_dtype dt, unsigned flags, ttt_stream stream);
 
 /*
+ * TTT-Linear forward, online (b = 1), with n_steps gradient steps per token
+ * ("How to Master Test-Time Training for LLMs", "How TTT Layers Actually
+ * Work": the layer runs one or more steps of gradient descent per token).
+ * At token t the weight takes n_steps steps W <- W - eta_t dl_t/dW, each
+ * gradient at the weight the previous step left, then the token reads out
+ * z_t = f(q_t; W). With n_steps = 1 this is ttt_linear_fwd with b = 1.
+ * Arguments, flags (TTT_F_LN, TTT_F_W0_PER_SEQ, TTT_F_Z_BF16, TTT_F_L2_KEYS)
+ * and errors as ttt_linear_fwd, without b; 1 <= n_steps <= 1024
+ * (TTT_ERR_ARG otherwise); d in {16, 32, 64}. Runs the fp32 CUDA-core kernel.
+ */
+TTT_API ttt_status ttt_linear_fwd_steps(const void *Q, const void *K, const void *V,
+                                        const float *eta, const float *W0, const float *ln_gamma,
+                                        const float *ln_beta, void *Z, float *W_out, int B, int H,
+                                        int T, int d, int n_steps, ttt_dtype dt, unsigned flags,
+                                        ttt_stream stream);
+
+/*
  * TTT-Linear backward: the outer gradients of the forward above ("Key
  * Architectural Mechanics of TTT-Linear", parts 1-4; the inner loop is
  * differentiated through, weight updates included). Given dZ = dL/dZ and,

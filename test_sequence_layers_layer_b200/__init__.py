@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_status_string.argtypes = [_I]
         L.ttt_linear_fwd.restype = _I
         L.ttt_linear_fwd.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_uint, _P]
+        L.ttt_linear_fwd_steps.restype = _I
+        L.ttt_linear_fwd_steps.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_uint, _P]
         L.ttt_linear_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.ttt_linear_bwd_workspace_bytes.argtypes = [_I] * 5
         L.ttt_linear_bwd.restype = _I
@@ -148,6 +150,14 @@ def ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                               _ptr(ln_beta), _ptr(Z), _ptr(W_out), B, H, T, d, b, dt, flags,
                               _stream(stream))
     return _check("ttt_linear_fwd", rc) if check else rc
+
+
+def ttt_linear_fwd_steps(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, n_steps, dt,
+                         flags, stream=None, check=True):
+    rc = lib().ttt_linear_fwd_steps(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W0),
+                                    _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z), _ptr(W_out), B, H, T,
+                                    d, n_steps, dt, flags, _stream(stream))
+    return _check("ttt_linear_fwd_steps", rc) if check else rc
 
 
 def ttt_linear_bwd_workspace_bytes(B, H, T, d, b) -> int:
@@ -300,6 +310,21 @@ def linear_fwd(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, w0_per_s
         (TTT_F_Z_BF16 if z_bf16 else 0) | (TTT_F_L2_KEYS if l2_keys else 0)
     ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                    _dtype_code(Q), flags, stream)
+    return Z, W_out
+
+
+def linear_fwd_steps(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, n_steps, ln,
+                     w0_per_seq=False, stream=None, want_w=True, z_bf16=False, l2_keys=False):
+    """TTT-Linear forward, online, n_steps gradient steps per token before its
+    read-out (ttt_linear_fwd_steps). Returns (Z, W_out) like linear_fwd."""
+    import torch
+    B, H, T, d = Q.shape
+    Z = torch.empty((B, H, T, d), dtype=torch.bfloat16 if z_bf16 else torch.float32, device=Q.device)
+    W_out = torch.empty((B, H, d, d), dtype=torch.float32, device=Q.device) if want_w else None
+    flags = (TTT_F_LN if ln else 0) | (TTT_F_W0_PER_SEQ if w0_per_seq else 0) | \
+        (TTT_F_Z_BF16 if z_bf16 else 0) | (TTT_F_L2_KEYS if l2_keys else 0)
+    ttt_linear_fwd_steps(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, n_steps,
+                         _dtype_code(Q), flags, stream)
     return Z, W_out
 
 

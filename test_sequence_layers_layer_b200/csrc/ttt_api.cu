@@ -165,6 +165,8 @@ cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const 
                              cudaStream_t s);
 // TTT-Linear on the fp32 CUDA-core kernel with L2-normalised keys (ttt_simt.cu).
 cudaError_t launch_linear_simt_keys(const LinearArgs &a, bool l2_keys, cudaStream_t s);
+cudaError_t launch_linear_simt_opts(const LinearArgs &a, bool l2_keys, int n_steps,
+                                   cudaStream_t s);
 // Affine-map kernels of the sequence-parallel large-chunk forward (ttt_affine.cu).
 cudaError_t launch_affine_eye(float *W, int S, int d, cudaStream_t s);
 cudaError_t launch_affine_prefix(const float *M, const float *N, const float *W0, float *W_in,
@@ -229,6 +231,34 @@ ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const flo
     if (flags & TTT_F_L2_KEYS) return launched(launch_linear_simt_keys(a, true, cs));
     return launched(linear_tc_supported(d, b, dt == TTT_BF16) ? launch_linear_tc(a, cs)
                                                                 : launch_linear_simt(a, cs));
+}
+
+ttt_status ttt_linear_fwd_steps(const void *Q, const void *K, const void *V, const float *eta,
+                                const float *W0, const float *ln_gamma, const float *ln_beta,
+                                void *Z, float *W_out, int B, int H, int T, int d, int n_steps,
+                                ttt_dtype dt, unsigned flags, ttt_stream stream) {
+    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ | TTT_F_Z_BF16 | TTT_F_L2_KEYS)) return TTT_ERR_ARG;
+    if (n_steps < 1 || n_steps > 1024) return TTT_ERR_ARG;
+    const bool ln = flags & TTT_F_LN;
+    if (!Q || !K || !V || !eta || !W0 || !Z) return TTT_ERR_PTR;
+    if (ln && (!ln_gamma || !ln_beta)) return TTT_ERR_PTR;
+    if (B <= 0 || H <= 0 || T <= 0 || !supported_d(d)) return TTT_ERR_SHAPE;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return TTT_ERR_SHAPE;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Z) || !aligned16(W0) ||
+        (W_out && !aligned16(W_out)))
+        return TTT_ERR_ALIGN;
+    if (W_out && W_out == W0 && !(flags & TTT_F_W0_PER_SEQ)) return TTT_ERR_ARG;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out};
+    st = check_device_ptrs(ptrs, 9);
+    if (st != TTT_OK) return st;
+    LinearArgs a{Q, K, V, eta, W0, ln_gamma, ln_beta, static_cast<float *>(Z), W_out, B, H, T, d, 1,
+                 dt == TTT_BF16, ln, (flags & TTT_F_W0_PER_SEQ) != 0, (flags & TTT_F_Z_BF16) != 0};
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    return launched(launch_linear_simt_opts(a, (flags & TTT_F_L2_KEYS) != 0, n_steps, cs));
 }
 
 size_t ttt_linear_bwd_workspace_bytes(int B, int H, int T, int d, int b) {

@@ -91,12 +91,19 @@ __device__ __forceinline__ void load_tile(float *dst, const void *src, size_t ba
 // it enters the inner loss, its gradient and the update (the key
 // normalisation of the PyTorch listing on "Test-Time Training: Linear
 // Complexity Beyond Attention"); queries are used as given.
-__global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a, bool l2_keys) {
+// n_steps > 1 (only with b = 1): the token takes n_steps gradient steps, each
+// at the weight the previous one left, before it reads out ("How to Master
+// Test-Time Training for LLMs", "How TTT Layers Actually Work": one or more
+// gradient steps per token). With W' = W_m - k^T (G_1 + ... + G_n), the
+// read-out q W' = q W_m - (q . k) (G_1 + ... + G_n); Gs holds that sum.
+// Shared memory then also holds Gs[b*d] after es.
+__global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a, bool l2_keys,
+                                                               int n_steps) {
     extern __shared__ float sm[];
     const int d = a.d, b = a.b, T = a.T;
     const int seq = blockIdx.x, h = seq % a.H;
     float *W = sm, *Qs = W + d * d, *Ks = Qs + b * d, *Vs = Ks + b * d, *Xs = Vs + b * d,
-          *Zs = Xs + b * d, *S = Zs + b * d, *es = S + b * b;
+          *Zs = Xs + b * d, *S = Zs + b * d, *es = S + b * b, *Gs = es + b;
     const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? seq : h) * d * d;
     const float *gamma = a.ln ? a.gamma + (size_t)h * d : nullptr;
     const float *beta = a.ln ? a.beta + (size_t)h * d : nullptr;
@@ -155,11 +162,37 @@ __global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a, boo
             }
         }
         __syncthreads();
-        // Zpre = Q W_m - S G'
+        // Further steps of the token (b = 1): apply G, sum it, take the next
+        // gradient at the updated weight. The last G is applied below.
+        for (int step = 1; step < n_steps; ++step) {
+            for (int j = threadIdx.x; j < d; j += blockDim.x) Gs[j] = (step == 1 ? 0.f : Gs[j]) + Xs[j];
+            for (int e = threadIdx.x; e < d * d; e += blockDim.x) W[e] -= Ks[e / d] * Xs[e % d];
+            __syncthreads();
+            for (int j = threadIdx.x; j < d; j += blockDim.x) {
+                float ax = 0.f;
+                for (int i = 0; i < d; ++i) ax = fmaf(Ks[i], W[i * d + j], ax);
+                Xs[j] = ax;
+            }
+            __syncthreads();
+            if (warp == 0) {
+                if (a.ln) {
+                    ln_grad_row(Xs, Ks, Vs, gamma, beta, es[0], d);
+                } else {
+                    for (int j = threadIdx.x & 31; j < d; j += 32) Xs[j] = es[0] * (Xs[j] - Vs[j]);
+                }
+            }
+            __syncthreads();
+        }
+        if (n_steps > 1) {
+            for (int j = threadIdx.x; j < d; j += blockDim.x) Gs[j] += Xs[j];
+            __syncthreads();
+        }
+        // Zpre = Q W_m - S G'  (with several steps: - S (G_1 + ... + G_n))
+        const float *Gz = n_steps > 1 ? Gs : Xs;
         for (int e = threadIdx.x; e < b * d; e += blockDim.x) {
             const int t = e / d, j = e % d;
             float acc = Zs[e];
-            for (int s = 0; s <= t; ++s) acc = fmaf(-S[t * b + s], Xs[s * d + j], acc);
+            for (int s = 0; s <= t; ++s) acc = fmaf(-S[t * b + s], Gz[s * d + j], acc);
             Zs[e] = acc;
         }
         // W_{m+1} = W_m - K^T G'
@@ -376,19 +409,24 @@ cudaError_t set_smem(K kernel, size_t smem) {
 
 }  // namespace
 
-cudaError_t launch_linear_simt_keys(const LinearArgs &a, bool l2_keys, cudaStream_t s) {
-    const size_t smem = sizeof(float) * ((size_t)a.d * a.d + 5 * (size_t)a.b * a.d +
+cudaError_t launch_linear_simt_opts(const LinearArgs &a, bool l2_keys, int n_steps,
+                                   cudaStream_t s) {
+    const size_t smem = sizeof(float) * ((size_t)a.d * a.d + 6 * (size_t)a.b * a.d +
                                          (size_t)a.b * a.b + a.b);
     cudaError_t e = set_smem(linear_simt_kernel, smem);
     if (e != cudaSuccess) return e;
-    linear_simt_kernel<<<a.B * a.H, kThreads, smem, s>>>(a, l2_keys);
+    linear_simt_kernel<<<a.B * a.H, kThreads, smem, s>>>(a, l2_keys, n_steps);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch(s);
     return e;
 }
 
+cudaError_t launch_linear_simt_keys(const LinearArgs &a, bool l2_keys, cudaStream_t s) {
+    return launch_linear_simt_opts(a, l2_keys, 1, s);
+}
+
 cudaError_t launch_linear_simt(const LinearArgs &a, cudaStream_t s) {
-    return launch_linear_simt_keys(a, false, s);
+    return launch_linear_simt_opts(a, false, 1, s);
 }
 
 size_t mlp_simt_smem(int d, int dh, int b) {

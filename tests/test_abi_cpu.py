@@ -193,3 +193,19 @@ def test_linear_map_host_validation():
     assert call(workspace_bytes=need - 1) == -9
     assert call() == -8                           # no GPU here
     assert call(T=250) == -8                      # a partial last mini-batch is accepted
+
+
+def test_linear_fwd_steps_host_validation():
+    A = ALIGNED
+    st = dict(Q=A, K=A, V=A, eta=A, W0=A, ln_gamma=A, ln_beta=A, Z=A, W_out=None, B=1, H=2, T=64,
+              d=64, n_steps=2, dt=ttt.TTT_BF16, flags=ttt.TTT_F_LN, stream=0)
+    call = lambda **kw: ttt.ttt_linear_fwd_steps(**{**st, **kw}, check=False)  # noqa: E731
+    assert call(n_steps=0) == -1
+    assert call(n_steps=1025) == -1
+    assert call(flags=16) == -1
+    assert call(d=128) == -2
+    assert call(ln_beta=None) == -5
+    assert call(Z=A + 4) == -4
+    assert call(W_out=A) == -1                  # aliasing W0 without per-sequence W0
+    assert call() == -8                         # no GPU here
+    assert call(flags=ttt.TTT_F_L2_KEYS | ttt.TTT_F_Z_BF16, n_steps=1024) == -8
