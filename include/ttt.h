@@ -224,6 +224,36 @@ TTT_API ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, cons
                        ttt_stream stream);
 
 /*
+ * TTT-MLP backward: the outer gradients of ttt_mlp_fwd (the inner loop is
+ * differentiated through, weight updates included). Given dZ = dL/dZ and,
+ * optionally, dW1_out = dL/dW1_out [B][H][d][dh] and dW2_out = dL/dW2_out
+ * [B][H][dh][d] (NULL: taken as zero), writes dL/d of every input:
+ *   dQ, dK, dV  [B][H][T][d] fp32;  deta [B][H][T] fp32
+ *   dW1_0 [H][d][dh], dW2_0 [H][dh][d] fp32, summed over the batch (or
+ *               [B][H][..] with TTT_F_W0_PER_SEQ)
+ *   dgamma, dbeta [H][d] fp32, summed over the batch.
+ * The kernel re-runs the forward to checkpoint each mini-batch's starting
+ * weights in the workspace (2 d dh floats per mini-batch of every sequence),
+ * then walks the mini-batches and their tokens in reverse; each token adds
+ * the gradient through its own inner gradient (including the LayerNorm
+ * backward's backward and GELU''). fp32 CUDA cores, one block per sequence;
+ * outputs are overwritten, never accumulated into.
+ * workspace: at least ttt_mlp_bwd_workspace_bytes(...) bytes, 256-byte aligned,
+ *   owned by the caller, clobbered (0 for an unsupported shape).
+ * Supported: TTT_F_LN set (TTT-MLP always has its LayerNorm), d in {16, 32, 64},
+ *   dh = 4 d, 1 <= b <= 16, T % b == 0, TTT_BF16 or TTT_FP32 inputs.
+ * flags: TTT_F_LN (required), TTT_F_W0_PER_SEQ.
+ */
+TTT_API size_t ttt_mlp_bwd_workspace_bytes(int B, int H, int T, int d, int dh, int b);
+TTT_API ttt_status ttt_mlp_bwd(const void *Q, const void *K, const void *V, const float *eta,
+                               const float *W1_0, const float *W2_0, const float *ln_gamma,
+                               const float *ln_beta, const float *dZ, const float *dW1_out,
+                               const float *dW2_out, float *dQ, float *dK, float *dV, float *deta,
+                               float *dW1_0, float *dW2_0, float *dgamma, float *dbeta, int B,
+                               int H, int T, int d, int dh, int b, ttt_dtype dt, unsigned flags,
+                               void *workspace, size_t workspace_bytes, ttt_stream stream);
+
+/*
  * Large-chunk TTT forward, apply-then-update ("Test-Time Training Done
  * Right"): the tokens of chunk c all read out with W_c, the weight left by
  * the chunks before it, then

@@ -65,6 +65,10 @@ def lib() -> ctypes.CDLL:
         L.ttt_chunk_bwd_workspace_bytes.argtypes = [_I] * 5
         L.ttt_chunk_bwd.restype = _I
         L.ttt_chunk_bwd.argtypes = [_P] * 12 + [_I] * 6 + [ctypes.c_uint, _P, ctypes.c_size_t, _P]
+        L.ttt_mlp_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.ttt_mlp_bwd_workspace_bytes.argtypes = [_I] * 6
+        L.ttt_mlp_bwd.restype = _I
+        L.ttt_mlp_bwd.argtypes = [_P] * 19 + [_I] * 7 + [ctypes.c_uint, _P, ctypes.c_size_t, _P]
         L.ttt_mlp_fwd.restype = _I
         L.ttt_mlp_fwd.argtypes = [_P] * 11 + [_I] * 7 + [ctypes.c_uint, _P]
         L.ttt_chunk_workspace_bytes.restype = ctypes.c_size_t
@@ -185,6 +189,21 @@ def ttt_chunk_bwd(Q, K, V, eta, W0, dZ, dW_out, dQ, dK, dV, deta, dW0, B, H, T, 
                              H, T, d, chunk, dt, flags, _ptr(workspace), workspace_bytes,
                              _stream(stream))
     return _check("ttt_chunk_bwd", rc) if check else rc
+
+
+def ttt_mlp_bwd_workspace_bytes(B, H, T, d, dh, b) -> int:
+    return int(lib().ttt_mlp_bwd_workspace_bytes(B, H, T, d, dh, b))
+
+
+def ttt_mlp_bwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, dZ, dW1_out, dW2_out, dQ, dK, dV,
+                deta, dW1_0, dW2_0, dgamma, dbeta, B, H, T, d, dh, b, dt, flags, workspace,
+                workspace_bytes, stream=None, check=True):
+    rc = lib().ttt_mlp_bwd(*[_ptr(x) for x in (Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, dZ,
+                                               dW1_out, dW2_out, dQ, dK, dV, deta, dW1_0, dW2_0,
+                                               dgamma, dbeta)],
+                           B, H, T, d, dh, b, dt, flags, _ptr(workspace), workspace_bytes,
+                           _stream(stream))
+    return _check("ttt_mlp_bwd", rc) if check else rc
 
 
 def ttt_mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out, B, H, T, d, dh,
@@ -350,6 +369,29 @@ def linear_bwd(Q, K, V, eta, W0, ln_gamma, ln_beta, dZ, dW_out=None, *, b, ln, w
     ttt_linear_bwd(Q, K, V, eta, W0, ln_gamma, ln_beta, dZ, dW_out, g["Q"], g["K"], g["V"],
                    g["eta"], g["W0"], g.get("gamma"), g.get("beta"), B, H, T, d, b, _dtype_code(Q),
                    flags, workspace, workspace.numel() * workspace.element_size(), stream)
+    return g
+
+
+def mlp_bwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, dZ, dW1_out=None, dW2_out=None, *, b,
+            w0_per_seq=False, workspace=None, stream=None):
+    """TTT-MLP backward. Returns a dict of fp32 gradients with keys Q, K, V,
+    eta, W1, W2, gamma, beta (W1/W2 shaped like W1_0/W2_0)."""
+    import torch
+    B, H, T, d = Q.shape
+    dh = W1_0.shape[-1]
+    f = dict(device=Q.device, dtype=torch.float32)
+    g = {"Q": torch.empty((B, H, T, d), **f), "K": torch.empty((B, H, T, d), **f),
+         "V": torch.empty((B, H, T, d), **f), "eta": torch.empty((B, H, T), **f),
+         "W1": torch.empty(tuple(W1_0.shape), **f), "W2": torch.empty(tuple(W2_0.shape), **f),
+         "gamma": torch.empty((H, d), **f), "beta": torch.empty((H, d), **f)}
+    need = ttt_mlp_bwd_workspace_bytes(B, H, T, d, dh, b)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=Q.device)
+    flags = TTT_F_LN | (TTT_F_W0_PER_SEQ if w0_per_seq else 0)
+    ttt_mlp_bwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, dZ, dW1_out, dW2_out, g["Q"], g["K"],
+                g["V"], g["eta"], g["W1"], g["W2"], g["gamma"], g["beta"], B, H, T, d, dh, b,
+                _dtype_code(Q), flags, workspace, workspace.numel() * workspace.element_size(),
+                stream)
     return g
 
 

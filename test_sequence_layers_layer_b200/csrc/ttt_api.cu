@@ -163,6 +163,16 @@ cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const 
                              float *dK, float *dV, float *deta, float *dW0, int B, int H, int T,
                              int d, int chunk, bool bf16, bool w0_per_seq, void *workspace,
                              cudaStream_t s);
+// TTT-MLP backward (ttt_mlp_bwd.cu).
+bool mlp_bwd_supported(int d, int dh, int b);
+size_t mlp_bwd_workspace_bytes(int B, int H, int T, int d, int b);
+cudaError_t launch_mlp_bwd(const void *Q, const void *K, const void *V, const float *eta,
+                           const float *W1_0, const float *W2_0, const float *gamma,
+                           const float *beta, const float *dZ, const float *dW1_out,
+                           const float *dW2_out, float *dQ, float *dK, float *dV, float *deta,
+                           float *dW1_0, float *dW2_0, float *dgamma, float *dbeta, int B, int H,
+                           int T, int d, int b, bool bf16, bool w0_per_seq, void *workspace,
+                           cudaStream_t s);
 // TTT-Linear on the fp32 CUDA-core kernel with L2-normalised keys (ttt_simt.cu).
 cudaError_t launch_linear_simt_keys(const LinearArgs &a, bool l2_keys, cudaStream_t s);
 cudaError_t launch_linear_simt_opts(const LinearArgs &a, bool l2_keys, int n_steps,
@@ -329,6 +339,45 @@ ttt_status ttt_chunk_bwd(const void *Q, const void *K, const void *V, const floa
     return launched(launch_chunk_bwd(Q, K, V, eta, W0, dZ, dW_out, dQ, dK, dV, deta, dW0, B, H, T, d,
                                      chunk, dt == TTT_BF16, (flags & TTT_F_W0_PER_SEQ) != 0,
                                      workspace, cs));
+}
+
+size_t ttt_mlp_bwd_workspace_bytes(int B, int H, int T, int d, int dh, int b) {
+    if (B <= 0 || H <= 0 || T <= 0 || b <= 0 || T % b || !mlp_bwd_supported(d, dh, b)) return 0;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return 0;
+    return mlp_bwd_workspace_bytes(B, H, T, d, b);
+}
+
+ttt_status ttt_mlp_bwd(const void *Q, const void *K, const void *V, const float *eta,
+                       const float *W1_0, const float *W2_0, const float *ln_gamma,
+                       const float *ln_beta, const float *dZ, const float *dW1_out,
+                       const float *dW2_out, float *dQ, float *dK, float *dV, float *deta,
+                       float *dW1_0, float *dW2_0, float *dgamma, float *dbeta, int B, int H,
+                       int T, int d, int dh, int b, ttt_dtype dt, unsigned flags, void *workspace,
+                       size_t workspace_bytes, ttt_stream stream) {
+    if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ)) return TTT_ERR_ARG;
+    if (!(flags & TTT_F_LN)) return TTT_ERR_ARG;
+    if (!Q || !K || !V || !eta || !W1_0 || !W2_0 || !ln_gamma || !ln_beta || !dZ || !dQ || !dK ||
+        !dV || !deta || !dW1_0 || !dW2_0 || !dgamma || !dbeta)
+        return TTT_ERR_PTR;
+    if (B <= 0 || H <= 0 || T <= 0 || b <= 0 || T % b != 0 || !mlp_bwd_supported(d, dh, b))
+        return TTT_ERR_SHAPE;
+    if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return TTT_ERR_SHAPE;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
+    const size_t need = mlp_bwd_workspace_bytes(B, H, T, d, b);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return TTT_ERR_WORKSPACE;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, dZ, dW1_out, dW2_out, dQ,
+                          dK, dV, deta, dW1_0, dW2_0, dgamma, dbeta, workspace};
+    st = check_device_ptrs(ptrs, 20);
+    if (st != TTT_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    return launched(launch_mlp_bwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, dZ, dW1_out,
+                                   dW2_out, dQ, dK, dV, deta, dW1_0, dW2_0, dgamma, dbeta, B, H, T,
+                                   d, b, dt == TTT_BF16, (flags & TTT_F_W0_PER_SEQ) != 0,
+                                   workspace, cs));
 }
 
 ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float *eta,

@@ -1,0 +1,78 @@
+// Host run of the TTT-MLP backward kernel body (ttt_mlp_bwd_body.inc), for the
+// CPU test of its arithmetic, indexing and barrier placement: each sequence
+// runs as one "block" of nt OS threads, one per CUDA thread, with a
+// std::barrier standing for every __syncthreads(). TEST CODE ONLY: the
+// library never calls it, and it is no fallback for the GPU kernel.
+#include <barrier>
+#include <cstring>
+#include <math.h>
+#include <thread>
+#include <vector>
+
+#define TTT_HD
+#define TTT_HD_SIZES
+#include "../../test_sequence_layers_layer_b200/csrc/ttt_mlp_bwd_body.inc"
+
+namespace {
+
+struct HostCtx {
+    int tid, nt;
+    float *sm;
+    std::barrier<> *bar;
+    void sync() { bar->arrive_and_wait(); }
+};
+
+}  // namespace
+
+extern "C" int ttt_mlp_bwd_host_run(const void *Q, const void *K, const void *V, const float *eta,
+                                    const float *W1_0, const float *W2_0, const float *gamma,
+                                    const float *beta, const float *dZ, const float *dW1_out,
+                                    const float *dW2_out, float *dQ, float *dK, float *dV,
+                                    float *deta, float *dW1_0, float *dW2_0, float *dgamma,
+                                    float *dbeta, int B, int H, int T, int d, int b, int bf16,
+                                    int w0_per_seq, int nt) {
+    if (T % b || nt < 1) return -1;
+    const size_t per = mlp_bwd_body::ws_floats_per_seq(T, d, b);
+    std::vector<float> ws(per * (size_t)B * H, 0.f);
+    std::vector<float> sm(mlp_bwd_body::smem_floats(d, b), 0.f);
+    mlp_bwd_body::Params p{Q, K, V, eta, W1_0, W2_0, gamma, beta, dZ, dW1_out, dW2_out,
+                          dQ, dK, dV, deta, dW1_0, dW2_0, ws.data(), H, T, d, b, bf16 != 0,
+                          w0_per_seq != 0};
+    for (int seq = 0; seq < B * H; ++seq) {
+        std::barrier<> bar(nt);
+        std::vector<std::thread> th;
+        for (int t = 0; t < nt; ++t)
+            th.emplace_back([&, t] {
+                HostCtx cx{t, nt, sm.data(), &bar};
+                mlp_bwd_body::run_sequence(cx, p, seq);
+            });
+        for (auto &x : th) x.join();
+    }
+    // the batch sums the GPU's second kernel makes
+    const size_t dF = (size_t)d * 4 * d;
+    for (int h = 0; h < H; ++h) {
+        for (size_t e = 0; e < dF; ++e) {
+            float a1 = 0.f, a2 = 0.f;
+            for (int bb = 0; bb < B; ++bb) {
+                auto w = mlp_bwd_body::ws_view(ws.data() + (size_t)(bb * H + h) * per, T, d, b);
+                a1 += w.dW1[e];
+                a2 += w.dW2[e];
+            }
+            if (!w0_per_seq) {
+                dW1_0[(size_t)h * dF + e] = a1;
+                dW2_0[(size_t)h * dF + e] = a2;
+            }
+        }
+        for (int c = 0; c < d; ++c) {
+            float g = 0.f, be = 0.f;
+            for (int bb = 0; bb < B; ++bb) {
+                auto w = mlp_bwd_body::ws_view(ws.data() + (size_t)(bb * H + h) * per, T, d, b);
+                g += w.dg[c];
+                be += w.db[c];
+            }
+            dgamma[(size_t)h * d + c] = g;
+            dbeta[(size_t)h * d + c] = be;
+        }
+    }
+    return 0;
+}

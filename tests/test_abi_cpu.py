@@ -209,3 +209,27 @@ def test_linear_fwd_steps_host_validation():
     assert call(W_out=A) == -1                  # aliasing W0 without per-sequence W0
     assert call() == -8                         # no GPU here
     assert call(flags=ttt.TTT_F_L2_KEYS | ttt.TTT_F_Z_BF16, n_steps=1024) == -8
+
+
+def test_mlp_backward_host_validation():
+    A = ALIGNED
+    B, H, T, d, b = 1, 2, 64, 64, 16
+    need = ttt.ttt_mlp_bwd_workspace_bytes(B, H, T, d, 4 * d, b)
+    assert need > 4 * B * H * (T // b) * 2 * d * 4 * d  # the checkpoints and more
+    assert ttt.ttt_mlp_bwd_workspace_bytes(B, H, T, d, 3 * d, b) == 0
+    assert ttt.ttt_mlp_bwd_workspace_bytes(B, H, T, 128, 512, b) == 0
+    mb = dict(Q=A, K=A, V=A, eta=A, W1_0=A, W2_0=A, ln_gamma=A, ln_beta=A, dZ=A, dW1_out=None,
+              dW2_out=None, dQ=A, dK=A, dV=A, deta=A, dW1_0=A, dW2_0=A, dgamma=A, dbeta=A, B=B,
+              H=H, T=T, d=d, dh=4 * d, b=b, dt=ttt.TTT_BF16, flags=ttt.TTT_F_LN, workspace=A,
+              workspace_bytes=need, stream=0)
+    call = lambda **kw: ttt.ttt_mlp_bwd(**{**mb, **kw}, check=False)  # noqa: E731
+    assert call(flags=0) == -1                        # TTT-MLP always has its LayerNorm
+    assert call(flags=ttt.TTT_F_LN | ttt.TTT_F_Z_BF16) == -1
+    assert call(dgamma=None) == -5
+    assert call(T=60) == -2                           # T % b
+    assert call(b=32, T=64) == -2                     # b <= 16
+    assert call(dh=128) == -2
+    assert call(dt=9) == -3
+    assert call(workspace_bytes=need - 1) == -9
+    assert call(workspace=A + 64) == -9
+    assert call() == -8                               # no GPU here

@@ -1,6 +1,6 @@
-"""TTT-Linear backward (ttt_linear_bwd) and large-chunk backward
-(ttt_chunk_bwd) against the backward oracle (oracle/backward.py: autograd
-through the float64 unrolled inner loop).
+"""TTT-Linear backward (ttt_linear_bwd), large-chunk backward (ttt_chunk_bwd)
+and TTT-MLP backward (ttt_mlp_bwd) against the backward oracle
+(oracle/backward.py: autograd through the float64 unrolled inner loop).
 
 Tolerance: 1e-4 of each gradient's largest magnitude. The kernel works in
 fp32 (unit roundoff 6e-8); a gradient here is a sum over the sequence of
@@ -185,3 +185,52 @@ def test_chunk_backward_full_size_sampled_sequences():
         for k in ("Q", "K", "V", "eta"):
             e = _rel(sl(got[k]), ref[k])
             assert e <= TOL, (bb, hh, k, e)
+
+
+# ------------------------------------------------------------------- TTT-MLP
+
+MLP_CASES = {
+    # name: (workload changes, w0_per_seq, with dW1_out / dW2_out)
+    "mlp_bf16_d64_b16": (dict(B=1, H=2, T=64), False, True),
+    "mlp_fp32_d16_b4_w0seq": (dict(B=2, H=1, T=16, d=16, dh=64, b=4, dtype="fp32"), True, False),
+    "mlp_bf16_d32_b8": (dict(B=2, H=1, T=32, d=32, dh=128, b=8), False, True),
+}
+
+
+def _mlp_case(name, seed=51):
+    ch, w0seq, with_dw = MLP_CASES[name]
+    wl = synth.WORKLOADS["mlp_ln_d64_dh256_b4h12_t8192"].scaled(seed=seed, **ch)
+    inp = synth.make_inputs(wl)
+    r = np.random.default_rng(seed + 1)
+    B, H, T, d, dh = wl.B, wl.H, wl.T, wl.d, wl.dh
+    dZ = r.standard_normal((B, H, T, d)).astype(np.float32)
+    dW1 = r.standard_normal((B, H, d, dh)).astype(np.float32) if with_dw else None
+    dW2 = r.standard_normal((B, H, dh, d)).astype(np.float32) if with_dw else None
+    W1, W2 = inp.W1, inp.W2
+    if w0seq:
+        W1 = (np.broadcast_to(W1[None], (B,) + W1.shape)
+              + 0.01 * r.standard_normal((B,) + W1.shape)).astype(np.float32)
+        W2 = (np.broadcast_to(W2[None], (B,) + W2.shape)
+              + 0.01 * r.standard_normal((B,) + W2.shape)).astype(np.float32)
+    return wl, inp, W1, W2, dZ, dW1, dW2, w0seq
+
+
+def _mlp_gpu(wl, inp, W1, W2, dZ, dW1, dW2, w0seq):
+    Q, K, V = _qkv(inp, wl)
+    f = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()  # noqa: E731
+    g = ttt.mlp_bwd(Q, K, V, f(inp.eta), f(W1), f(W2), f(inp.gamma), f(inp.beta), f(dZ), f(dW1),
+                    f(dW2), b=wl.b, w0_per_seq=w0seq)
+    torch.cuda.synchronize()
+    assert ttt.ttt_device_status() == 0
+    return {k: v.double().cpu().numpy() for k, v in g.items()}
+
+
+@pytest.mark.parametrize("name", list(MLP_CASES))
+def test_mlp_backward_matches_oracle(name):
+    wl, inp, W1, W2, dZ, dW1, dW2, w0seq = _mlp_case(name)
+    got = _mlp_gpu(wl, inp, W1, W2, dZ, dW1, dW2, w0seq)
+    ref = ob.mlp_grads(inp.Q, inp.K, inp.V, inp.eta, W1, W2, inp.gamma, inp.beta, dZ, dW1, dW2,
+                       b=wl.b)
+    errs = {k: _rel(got[k], ref[k]) for k in ref}
+    assert set(got) == set(ref)
+    assert max(errs.values()) <= TOL, errs
