@@ -665,6 +665,17 @@ def segmented_arm(args, wl):
 FP32_LANES = 148 * 128
 
 
+def mlp_bwd_flops_per_token(d: int, dh: int) -> float:
+    """Algorithmic FLOPs of the TTT-MLP backward per token, counting its d x dh
+    products (2 d dh FLOPs each): the checkpoint forward (k W1, a W2, Gx W2^T
+    and the two weight updates: 5), the key side and read-out recomputed in the
+    reverse pass (5), the token's read-out backward and second-order term
+    (dxq W2^T, dhq W1^T, the two rank-one Phi updates, k Phi1, a Phi2, dga W2,
+    dx W2^T, Phi2 Gx, Phi1 Gh, dh W1^T: 11) and the end-of-mini-batch weight
+    terms (3): 24 products. The O(b (d + dh)) dual sums are left out."""
+    return 48.0 * d * dh
+
+
 def bwd_flops_per_token(d: int) -> float:
     """Algorithmic FLOPs of the TTT-Linear backward per token: the forward
     re-run (k W, and the K^T G update: 4 d^2) and the reverse step (k W and q W,
@@ -689,8 +700,9 @@ def bwd_bytes_per_token(wl) -> float:
 
 
 def backward_arm(args, wl):
-    """TTT-Linear backward (`--backward`): ttt_linear_bwd on the workload's
-    inputs with a seeded dZ, all resident in HBM, L2 flushed between steps."""
+    """Backward pass (`--backward`): ttt_linear_bwd, ttt_chunk_bwd or
+    ttt_mlp_bwd on the workload's inputs with a seeded dZ, all resident in
+    HBM, L2 flushed between steps."""
     import torch
     import test_sequence_layers_layer_b200 as ttt
 
@@ -701,14 +713,18 @@ def backward_arm(args, wl):
     x = device_tensors(inp, dev)
     rng = np.random.default_rng(wl.seed + 101)
     dZ = torch.from_numpy(rng.standard_normal((wl.B, wl.H, wl.T, wl.d)).astype(np.float32)).to(dev)
-    chunk = wl.kind == "chunk"
-    need = (ttt.ttt_chunk_bwd_workspace_bytes if chunk else ttt.ttt_linear_bwd_workspace_bytes)(
-        wl.B, wl.H, wl.T, wl.d, wl.b)
+    chunk, mlp = wl.kind == "chunk", wl.kind == "mlp"
+    if mlp:
+        need = ttt.ttt_mlp_bwd_workspace_bytes(wl.B, wl.H, wl.T, wl.d, wl.dh, wl.b)
+    else:
+        need = (ttt.ttt_chunk_bwd_workspace_bytes if chunk else ttt.ttt_linear_bwd_workspace_bytes)(
+            wl.B, wl.H, wl.T, wl.d, wl.b)
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
     f32 = dict(dtype=torch.float32, device=dev)
     g = [torch.empty((wl.B, wl.H, wl.T, wl.d), **f32) for _ in range(3)]
     geta = torch.empty((wl.B, wl.H, wl.T), **f32)
     gW0 = torch.empty(tuple(x["W1"].shape), **f32)
+    gW2 = torch.empty(tuple(x["W2"].shape), **f32) if mlp else None
     gg, gb = torch.empty((wl.H, wl.d), **f32), torch.empty((wl.H, wl.d), **f32)
     dt = ttt.TTT_BF16 if wl.dtype == "bf16" else ttt.TTT_FP32
     flags = ttt.TTT_F_LN if wl.ln else 0
@@ -716,7 +732,12 @@ def backward_arm(args, wl):
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def call():
-        if chunk:
+        if mlp:
+            ttt.ttt_mlp_bwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["W2"], x["gamma"],
+                            x["beta"], dZ, None, None, *g, geta, gW0, gW2, gg, gb, wl.B, wl.H,
+                            wl.T, wl.d, wl.dh, wl.b, dt, ttt.TTT_F_LN, ws, need,
+                            stream.cuda_stream)
+        elif chunk:
             ttt.ttt_chunk_bwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], dZ, None, *g, geta, gW0,
                               wl.B, wl.H, wl.T, wl.d, wl.b, dt, 0, ws, need, stream.cuda_stream)
         else:
@@ -755,15 +776,17 @@ def backward_arm(args, wl):
     # their summed time
     kern_ms = (sum(kern) if chunk else kern[0]) / args.steps
     knames = (["cb_gram_kernel", "cb_scan_kernel", "cb_tok_kernel", "cb_sum_over_batch_kernel (dW0)"]
-              if chunk else ["linear_bwd_kernel", "sum_over_batch_kernel (dW0)",
-                             "sum_over_batch_kernel (dgamma)", "sum_over_batch_kernel (dbeta)"])
+              if chunk else ["mlp_bwd_kernel", "mlp_bwd_sum_kernel"] if mlp
+              else ["linear_bwd_kernel", "sum_over_batch_kernel (dW0)",
+                    "sum_over_batch_kernel (dgamma)", "sum_over_batch_kernel (dbeta)"])
     clocks = sampler.summary(t0, t1)
     mhz = clocks.get("sm_mhz") or 1965
     peak = FP32_LANES * 2 * mhz * 1e6 / 1e12
-    flop = (chunk_bwd_flops_per_token(wl.d, wl.b) if chunk else bwd_flops_per_token(wl.d)) * wl.tokens
+    flop = (chunk_bwd_flops_per_token(wl.d, wl.b) if chunk
+            else mlp_bwd_flops_per_token(wl.d, wl.dh) if mlp else bwd_flops_per_token(wl.d)) * wl.tokens
     achieved = flop / (kern_ms / 1e3) / 1e12
     line = {
-        "metric": ("Large-chunk TTT" if chunk else "TTT-Linear") +
+        "metric": ("Large-chunk TTT" if chunk else "TTT-MLP" if mlp else "TTT-Linear") +
                   " backward tokens/sec at 1 B200 (outer gradients of every input)",
         "value": wl.tokens / (ms / 1e3), "unit": "tokens/s", "higher_is_better": True,
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -773,16 +796,28 @@ def backward_arm(args, wl):
                    "l2": "flushed between steps (256 MiB write)"},
         "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None,
-                     "kernel": "all backward kernels" if chunk else "linear_bwd_kernel",
+                     "kernel": ("all backward kernels" if chunk
+                                else "mlp_bwd_kernel" if mlp else "linear_bwd_kernel"),
                      "peak_source": f"derived: {FP32_LANES} fp32 lanes x 2 FLOP x {mhz} MHz",
                      "algorithmic_per_launch": flop, "kernel_ms": kern_ms,
-                     "hbm_bytes_per_token": bwd_bytes_per_token(wl)},
+                     "hbm_bytes_per_token": None if mlp else bwd_bytes_per_token(wl)},
         "kernels": [{"name": n, "ms_per_launch": t / args.steps} for n, t in zip(knames, kern)],
         "gpu_launches": launches,
         "clocks": clocks,
         "step_ms_min_median": [min(step_ms), statistics.median(step_ms)],
     }
-    if not args.no_cpu_baseline and not chunk:
+    if not args.no_cpu_baseline and mlp:
+        from oracle import backward as ob
+        sub = wl.scaled(B=1, H=1, T=min(wl.T, 4 * wl.b))
+        si = synth.make_inputs(sub)
+        dz = rng.standard_normal((1, 1, sub.T, sub.d))
+        t0 = time.perf_counter()
+        ob.mlp_grads(si.Q, si.K, si.V, si.eta, si.W1, si.W2, si.gamma, si.beta, dz, b=sub.b)
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": sub.T / el, "unit": "tokens/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"1 sequence, T={sub.T}: float64 autograd backward"}
+    if not args.no_cpu_baseline and not chunk and not mlp:
         from oracle import backward as ob
         sub = wl.scaled(B=1, H=1, T=min(wl.T, 512))
         si = synth.make_inputs(sub)
@@ -827,8 +862,6 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
 
     if args.backward:
-        if wl.kind == "mlp":
-            ap.error("--backward times the linear and large-chunk workloads")
         if rank == 0:
             print(json.dumps(backward_arm(args, wl)), flush=True)
         return

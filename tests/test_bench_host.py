@@ -83,3 +83,9 @@ def test_segments_option_is_checked_before_any_gpu_work():
     assert r.returncode == 2 and "does not split" in r.stderr
     r = subprocess.run(base[:2] + ["--segments", "2"], capture_output=True, text=True, timeout=120)
     assert r.returncode == 2 and "large-chunk" in r.stderr
+
+
+def test_mlp_backward_flop_count():
+    """24 products of 2 d dh FLOPs per token (checkpoint forward 5, recompute
+    5, token backward 11, end-of-mini-batch weight terms 3)."""
+    assert bench.mlp_bwd_flops_per_token(64, 256) == 24 * 2 * 64 * 256
