@@ -11,9 +11,14 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU; parity tests of the CUDA path")
     config.addinivalue_line("markers", "slow: full-size workloads")
+    config.addinivalue_line(
+        "markers", "late: GPU cases that have not yet passed on a GPU; collected after all the "
+        "others, so that a failure among them (the suite runs with -x) stops none of the rest")
 
 
 def pytest_collection_modifyitems(config, items):
+    # "late" cases last, the order otherwise unchanged (a stable sort)
+    items.sort(key=lambda it: "late" in it.keywords)
     # GPU tests need a device; without one they are reported as skipped rather
     # than silently passing.
     try:

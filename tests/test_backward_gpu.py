@@ -225,6 +225,7 @@ def _mlp_gpu(wl, inp, W1, W2, dZ, dW1, dW2, w0seq):
     return {k: v.double().cpu().numpy() for k, v in g.items()}
 
 
+@pytest.mark.late
 @pytest.mark.parametrize("name", list(MLP_CASES))
 def test_mlp_backward_matches_oracle(name):
     wl, inp, W1, W2, dZ, dW1, dW2, w0seq = _mlp_case(name)

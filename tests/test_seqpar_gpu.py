@@ -151,6 +151,7 @@ LINEAR_CASES = {
 }
 
 
+@pytest.mark.late
 @pytest.mark.parametrize("name", list(LINEAR_CASES))
 def test_linear_map_matches_oracle(name):
     wl = LINEAR_CASES[name]
@@ -164,6 +165,7 @@ def test_linear_map_matches_oracle(name):
     assert _rel(_np(N), Nr) <= TOL[wl.dtype]
 
 
+@pytest.mark.late
 @pytest.mark.parametrize("name,nseg", [("linear_noln_bf16_d64_b16", 2),
                                        ("linear_noln_bf16_d64_b16", 8),
                                        ("linear_noln_fp32_d64_b8", 4)])

@@ -13,7 +13,7 @@ from oracle import variants
 from test_sequence_layers_layer_b200 import synth
 from gpu_helpers import TOL, to_dev
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.late]
 
 L = synth.WORKLOADS["linear_ln_d64_b8h12_t2048"]
 CASES = {
