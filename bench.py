@@ -373,6 +373,7 @@ def gpu_arm(args, wl, rank, world):
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = sum(o.numel() * o.element_size() for o in host_out)
     e2e_steps = max(3, min(args.steps, 10))
+    sliced = args.e2e_slices > 0 and wl.kind == "linear"
     with torch.cuda.stream(stream):
         def e2e_step():
             for k, v in host_in.items():
@@ -380,6 +381,14 @@ def gpu_arm(args, wl, rank, world):
             call_e2e()
             for h, o in zip(host_out, [o for o in outs_e2e if o is not None]):
                 h.copy_(o, non_blocking=True)
+        if sliced:
+            from test_sequence_layers_layer_b200 import hostio
+
+            def e2e_step():  # noqa: F811  (copies overlapped across batch slices)
+                hostio.linear_fwd_host(host_in["Q"], host_in["K"], host_in["V"], host_in["eta"],
+                                       host_in["W1"], host_in.get("gamma"), host_in.get("beta"),
+                                       b=wl.b, ln=wl.ln, slices=args.e2e_slices,
+                                       z_bf16=args.z_bf16)
         e2e_step()
         stream.synchronize()
         barrier()
@@ -447,7 +456,9 @@ def gpu_arm(args, wl, rank, world):
                      "algorithmic_per_launch": per_launch, "kernel_ms": kern_ms},
         "kernels": kernels,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "copies": f"overlapped over {args.e2e_slices} batch slices" if sliced
+                else "in series with the call"},
         "gpu_launches": launches,
         "clocks": clocks,
         "step_ms_min_median": [min(step_ms), statistics.median(step_ms)],
@@ -848,6 +859,9 @@ def main():
                     help="time the TTT-Linear backward (linear workloads) instead")
     ap.add_argument("--decode", type=int, default=0,
                     help="time N single-token decode steps (linear workloads) instead")
+    ap.add_argument("--e2e-slices", type=int, default=0,
+                    help="e2e leg (linear workloads): overlap the host copies with the compute "
+                         "over N batch slices (hostio.linear_fwd_host)")
     ap.add_argument("--segments", type=int, default=0,
                     help="time the large-chunk forward split into N segments per sequence")
     ap.add_argument("--B", type=int, default=None,

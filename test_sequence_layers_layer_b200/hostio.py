@@ -1,0 +1,73 @@
+"""TTT-Linear forward on inputs that live in host memory, with the copies
+overlapped with the compute.
+
+The batch is cut into `slices` groups of whole batch rows (every group holds
+all heads of its rows, so a shared W0 [H, d, d] serves every group). Each
+group runs on its own CUDA stream: its Q, K, V and eta are copied to the
+device, ttt_linear_fwd runs on them, and its Z and W_out are copied back. The
+host-to-device copies of later groups, the device-to-host copies of earlier
+ones and the kernels of the groups in between then proceed at the same time.
+A sequence's result does not depend on which other sequences share its call,
+so the outputs equal those of one ttt_linear_fwd call over the whole batch.
+
+Host tensors must be in pinned (page-locked) memory for the copies to run
+asynchronously. torch provides the memory, the streams and the copies; every
+step of the computation runs in libttt.so's kernels.
+"""
+from __future__ import annotations
+
+import test_sequence_layers_layer_b200 as _lib
+
+
+_STREAMS = {}
+
+
+def _streams(dev, n):
+    """n side streams of device dev, created once and reused."""
+    import torch
+    have = _STREAMS.setdefault(dev.index, [])
+    while len(have) < n:
+        have.append(torch.cuda.Stream(dev))
+    return have[:n]
+
+
+def _bounds(B: int, slices: int):
+    n = max(1, min(slices, B))
+    q, r = divmod(B, n)
+    out, b0 = [], 0
+    for i in range(n):
+        b1 = b0 + q + (1 if i < r else 0)
+        out.append((b0, b1))
+        b0 = b1
+    return out
+
+
+def linear_fwd_host(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, slices=4,
+                    z_bf16=False, device=None):
+    """TTT-Linear forward of host tensors Q, K, V [B, H, T, d] (bf16 or fp32)
+    and eta [B, H, T]; W0 [H, d, d] and the LayerNorm gain and bias [H, d] may
+    be on the host or the device. Returns (Z, W_out) as pinned host tensors,
+    valid once torch's current stream has reached the point of return (for
+    example after torch.cuda.current_stream().synchronize())."""
+    import torch
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    B, H, T, d = Q.shape
+    cur = torch.cuda.current_stream(dev)
+    W0d = W0.to(dev, non_blocking=True)
+    gd = ln_gamma.to(dev, non_blocking=True) if ln_gamma is not None else None
+    bd = ln_beta.to(dev, non_blocking=True) if ln_beta is not None else None
+    Zh = torch.empty((B, H, T, d), dtype=torch.bfloat16 if z_bf16 else torch.float32,
+                     pin_memory=True)
+    Wh = torch.empty((B, H, d, d), dtype=torch.float32, pin_memory=True)
+    bounds = _bounds(B, slices)
+    streams = _streams(dev, len(bounds))
+    for (b0, b1), st in zip(bounds, streams):
+        st.wait_stream(cur)  # W0, gamma, beta are copied on the current stream
+        with torch.cuda.stream(st):
+            q, k, v, e = (x[b0:b1].to(dev, non_blocking=True) for x in (Q, K, V, eta))
+            Z, W = _lib.linear_fwd(q, k, v, e, W0d, gd, bd, b=b, ln=ln, stream=st, z_bf16=z_bf16)
+            Zh[b0:b1].copy_(Z, non_blocking=True)
+            Wh[b0:b1].copy_(W, non_blocking=True)
+    for st in streams:
+        cur.wait_stream(st)
+    return Zh, Wh

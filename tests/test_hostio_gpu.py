@@ -1,0 +1,31 @@
+"""TTT-Linear forward from pinned host buffers with copies overlapped across
+batch slices (hostio.linear_fwd_host): its outputs equal one ttt_linear_fwd
+call on the device over the whole batch, bit for bit (a sequence's result does
+not depend on which sequences share its call)."""
+import pytest
+import torch
+
+import test_sequence_layers_layer_b200 as ttt
+from test_sequence_layers_layer_b200 import hostio, synth
+from gpu_helpers import to_dev
+
+pytestmark = [pytest.mark.gpu, pytest.mark.late]
+
+L = synth.WORKLOADS["linear_ln_d64_b8h12_t2048"]
+
+
+@pytest.mark.parametrize("B,slices,z_bf16,ln", [(3, 1, False, True), (5, 3, False, True),
+                                               (8, 4, True, True), (4, 4, False, False)])
+def test_host_pipeline_equals_device_call(B, slices, z_bf16, ln):
+    wl = L.scaled(B=B, H=3, T=160, ln=ln)
+    x = to_dev(synth.make_inputs(wl))
+    Zd, Wd = ttt.linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
+                            b=wl.b, ln=ln, z_bf16=z_bf16)
+    h = {k: x[k].cpu().pin_memory() for k in ("Q", "K", "V", "eta")}
+    Zh, Wh = hostio.linear_fwd_host(h["Q"], h["K"], h["V"], h["eta"], x["W1"].cpu(),
+                                    x["gamma"].cpu(), x["beta"].cpu(), b=wl.b, ln=ln,
+                                    slices=slices, z_bf16=z_bf16)
+    torch.cuda.current_stream().synchronize()
+    assert ttt.ttt_device_status() == 0
+    assert Zh.is_pinned() and Wh.is_pinned()
+    assert torch.equal(Zh, Zd.cpu()) and torch.equal(Wh, Wd.cpu())
