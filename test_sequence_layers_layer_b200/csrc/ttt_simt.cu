@@ -396,6 +396,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
         for (int e = threadIdx.x; e < d * d; e += blockDim.x) a.W_out[(size_t)seq * d * d + e] = W[e];
 }
 
+#ifndef TTT_HOST_RUN  // launch code (a host build of the kernels for tests leaves it out)
 // Opt a kernel in to more than 48 KB of dynamic shared memory.
 template <typename K>
 cudaError_t set_smem(K kernel, size_t smem) {
@@ -406,9 +407,11 @@ cudaError_t set_smem(K kernel, size_t smem) {
     }
     return cudaSuccess;
 }
+#endif  // TTT_HOST_RUN
 
 }  // namespace
 
+#ifndef TTT_HOST_RUN
 cudaError_t launch_linear_simt_opts(const LinearArgs &a, bool l2_keys, int n_steps,
                                    cudaStream_t s) {
     const size_t smem = sizeof(float) * ((size_t)a.d * a.d + 6 * (size_t)a.b * a.d +
@@ -453,5 +456,7 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s) {
     if (e == cudaSuccess) count_launch(s);
     return e;
 }
+
+#endif  // TTT_HOST_RUN
 
 }  // namespace ttt
