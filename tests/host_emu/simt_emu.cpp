@@ -63,6 +63,47 @@ float sm[1 << 16];
 }  // namespace
 }  // namespace ttt
 
+// Runs fn() as every thread of nblocks blocks of 256 threads, one block at a time.
+template <class Fn>
+static void run_blocks(int nblocks, Fn fn) {
+    const int nt = emu::kMaxThreads;
+    emu::nthreads = nt;
+    blockDim = {(unsigned)nt, 1, 1};
+    gridDim = {(unsigned)nblocks, 1, 1};
+    emu::block_bar = std::make_unique<std::barrier<>>(nt);
+    for (auto &w : emu::warp_bar) w = std::make_unique<std::barrier<>>(32);
+    for (int blk = 0; blk < nblocks; ++blk) {
+        blockIdx = {(unsigned)blk, 0, 0};
+        std::vector<std::thread> th;
+        for (int t = 0; t < nt; ++t)
+            th.emplace_back([&, t] {
+                emu::tid = t;
+                threadIdx = {(unsigned)t, 0, 0};
+                fn();
+            });
+        for (auto &x : th) x.join();
+    }
+}
+
+extern "C" int ttt_mlp_simt_host_run(const void *Q, const void *K, const void *V, const float *eta,
+                                     const float *W1, const float *W2, const float *gamma,
+                                     const float *beta, float *Z, float *W1_out, float *W2_out,
+                                     int B, int H, int T, int d, int dh, int b) {
+    ttt::MlpArgs a{Q, K, V, eta, W1, W2, gamma, beta, Z, W1_out, W2_out, B, H, T, d, dh, b,
+                   false, false, false};
+    run_blocks(B * H, [&] { ttt::mlp_simt_kernel(a); });
+    return 0;
+}
+
+extern "C" int ttt_chunk_simt_host_run(const void *Q, const void *K, const void *V,
+                                       const float *eta, const float *W0, float *Z, float *W_out,
+                                       int B, int H, int T, int d, int chunk) {
+    ttt::ChunkArgs a{Q, K, V, eta, W0, Z, W_out, B, H, T, d, chunk, false, false, false,
+                     nullptr, 0};
+    run_blocks(B * H, [&] { ttt::chunk_simt_kernel(a); });
+    return 0;
+}
+
 extern "C" int ttt_linear_simt_host_run(const void *Q, const void *K, const void *V,
                                         const float *eta, const float *W0, const float *gamma,
                                         const float *beta, float *Z, float *W_out, int B, int H,

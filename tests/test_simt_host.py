@@ -1,6 +1,6 @@
-"""The fp32 CUDA-core TTT-Linear kernel (linear_simt_kernel in ttt_simt.cu)
-run on the host against the oracles: the plain forward (C oracle), with
-L2-normalised keys and with several gradient steps per token (variant oracle).
+"""The fp32 CUDA-core kernels of ttt_simt.cu run on the host against the
+oracles: TTT-Linear (the plain forward, with L2-normalised keys and with
+several gradient steps per token), TTT-MLP and large-chunk TTT.
 The kernel source is compiled with g++ into a test harness
 (tests/host_emu/simt_emu.cpp): 256 OS threads per block, a std::barrier for
 __syncthreads(), warp shuffles through per-warp buffers and barriers. It
@@ -30,6 +30,10 @@ def emu(tmp_path_factory):
     L = ctypes.CDLL(so)
     L.ttt_linear_simt_host_run.restype = ctypes.c_int
     L.ttt_linear_simt_host_run.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 11
+    L.ttt_mlp_simt_host_run.restype = ctypes.c_int
+    L.ttt_mlp_simt_host_run.argtypes = [ctypes.c_void_p] * 11 + [ctypes.c_int] * 6
+    L.ttt_chunk_simt_host_run.restype = ctypes.c_int
+    L.ttt_chunk_simt_host_run.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int] * 5
     return L
 
 
@@ -85,4 +89,36 @@ def test_several_steps_per_token(emu, d, n, ln, l2):
     Kr = variants.normalize_keys(K) if l2 else K
     Zr, Wr = variants.linear_multistep(Q, Kr, V, eta, W0, g if ln else None, be if ln else None,
                                        n_steps=n, ln=ln)
+    assert _rel(Z, Zr) <= TOL and _rel(W, Wr) <= TOL
+
+
+def test_mlp_kernel(emu):
+    r = np.random.default_rng(41)
+    B, H, T, d, dh, b = 1, 2, 32, 16, 64, 8
+    f = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
+    Q, K, V = (f(r.standard_normal((B, H, T, d)) / np.sqrt(d)) for _ in range(3))
+    eta = f(0.1 * r.uniform(0.2, 1.0, (B, H, T)))
+    W1 = f(0.5 * r.standard_normal((H, d, dh)) / np.sqrt(d))
+    W2 = f(0.5 * r.standard_normal((H, dh, d)) / np.sqrt(dh))
+    g, be = f(1 + 0.2 * r.standard_normal((H, d))), f(0.2 * r.standard_normal((H, d)))
+    Z = np.zeros((B, H, T, d), np.float32)
+    W1o, W2o = np.zeros((B, H, d, dh), np.float32), np.zeros((B, H, dh, d), np.float32)
+    assert emu.ttt_mlp_simt_host_run(*[a.ctypes.data for a in (Q, K, V, eta, W1, W2, g, be, Z,
+                                                                W1o, W2o)],
+                                     B, H, T, d, dh, b) == 0
+    Zr, W1r, W2r = oracle.mlp_primal(Q, K, V, eta, W1, W2, g, be, b=b)
+    assert _rel(Z, Zr) <= TOL and _rel(W1o, W1r) <= TOL and _rel(W2o, W2r) <= TOL
+
+
+def test_chunk_kernel(emu):
+    r = np.random.default_rng(43)
+    B, H, T, d, C = 2, 1, 128, 64, 64
+    f = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
+    Q, K, V = (f(r.standard_normal((B, H, T, d)) / np.sqrt(d)) for _ in range(3))
+    eta = f(np.full((B, H, T), 1.0 / C))
+    W0 = f(0.3 * r.standard_normal((H, d, d)) / np.sqrt(d))
+    Z, W = np.zeros((B, H, T, d), np.float32), np.zeros((B, H, d, d), np.float32)
+    assert emu.ttt_chunk_simt_host_run(*[a.ctypes.data for a in (Q, K, V, eta, W0, Z, W)],
+                                       B, H, T, d, C) == 0
+    Zr, Wr = oracle.chunk_primal(Q, K, V, eta, W0, chunk=C)
     assert _rel(Z, Zr) <= TOL and _rel(W, Wr) <= TOL
