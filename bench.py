@@ -300,7 +300,7 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def gpu_arm(args, wl, rank, world):
+def gpu_arm(args, wl, rank, world, keep=None):
     import torch
     import torch.distributed as dist
     import test_sequence_layers_layer_b200 as ttt
@@ -351,6 +351,8 @@ def gpu_arm(args, wl, rank, world):
         torch.cuda.synchronize()
         t1 = time.perf_counter()
         launches = ttt.ttt_launch_count() - n0
+        if keep is not None:
+            keep["outs"] = outs  # the last timed call's outputs, for the parity check
         if multi:
             # summed over the timed calls; read once, after the loop, so the
             # host never waits on the device inside it
@@ -469,10 +471,12 @@ def gpu_arm(args, wl, rank, world):
 
 # ----------------------------------------------------------------------------- CPU (oracle) arm
 
-def oracle_sample(wl, budget_s: float):
+def oracle_sample(wl, budget_s: float, keep=None):
     """Time the oracle on whole sequences of the workload, threaded over the
     host cores, growing the sample until about budget_s of work or the whole
-    workload. Returns (tokens/s, cores, description)."""
+    workload. Returns (tokens/s, cores, description); with `keep` (a dict),
+    also leaves there the sampled sequences ("seqs") and the oracle's outputs
+    of the last, largest sample ("ref")."""
     import oracle
 
     inp = synth.make_inputs(wl)
@@ -484,15 +488,19 @@ def oracle_sample(wl, budget_s: float):
     def run(seqs):
         t0 = time.perf_counter()
         if wl.kind == "linear":
-            oracle.linear_primal(f64["Q"], f64["K"], f64["V"], f64["eta"], f64["W1"], f64["gamma"],
-                                 f64["beta"], b=wl.b, ln=wl.ln, seqs=seqs, with_w=True)
+            out = oracle.linear_primal(f64["Q"], f64["K"], f64["V"], f64["eta"], f64["W1"],
+                                       f64["gamma"], f64["beta"], b=wl.b, ln=wl.ln, seqs=seqs,
+                                       with_w=True)
         elif wl.kind == "mlp":
-            oracle.mlp_primal(f64["Q"], f64["K"], f64["V"], f64["eta"], f64["W1"], f64["W2"],
-                              f64["gamma"], f64["beta"], b=wl.b, seqs=seqs)
+            out = oracle.mlp_primal(f64["Q"], f64["K"], f64["V"], f64["eta"], f64["W1"], f64["W2"],
+                                    f64["gamma"], f64["beta"], b=wl.b, seqs=seqs)
         else:
-            oracle.chunk_primal(f64["Q"], f64["K"], f64["V"], f64["eta"], f64["W1"], chunk=wl.b,
-                                seqs=seqs)
-        return time.perf_counter() - t0
+            out = oracle.chunk_primal(f64["Q"], f64["K"], f64["V"], f64["eta"], f64["W1"],
+                                      chunk=wl.b, seqs=seqs)
+        el = time.perf_counter() - t0
+        if keep is not None:
+            keep["seqs"], keep["ref"] = list(seqs), out
+        return el
 
     n = min(cores, nseq_total)
     dt = run(list(range(n)))
@@ -502,6 +510,27 @@ def oracle_sample(wl, budget_s: float):
     tok = n * wl.T
     desc = f"{n} of {nseq_total} sequences, full length T={wl.T} ({tok} tokens), {cores} threads"
     return tok / dt, cores, desc
+
+
+def bench_parity(wl, outs, sample, z_bf16=False):
+    """Max relative error (max |gpu - oracle| / max |oracle|, per output) of
+    the timed call's outputs on the sequences the CPU-baseline leg ran through
+    the oracle. `outs` are the call's output tensors ([B, H, ...]); `sample`
+    holds "seqs" and "ref" from oracle_sample. Not computed for the TTT-MLP
+    workload, whose exact recurrence is chaotic on some sequences (the
+    parity tests compare it where it is conditioned)."""
+    if wl.kind == "mlp":
+        return {"note": "not computed for TTT-MLP: chaotic sequences (see the parity tests)"}
+    seqs = sample["seqs"]
+    S = wl.B * wl.H
+    res = {"sequences": len(seqs), "of": S,
+           "tolerance": 2e-3 if wl.dtype == "bf16" else 1e-5,
+           "z_dtype": "bf16" if z_bf16 else "fp32"}
+    for name, g, r in zip(("z", "w_out"), outs, sample["ref"]):
+        gs = np.asarray(g.float().reshape(S, -1).cpu().numpy(), dtype=np.float64)[seqs]
+        rs = np.asarray(r, dtype=np.float64).reshape(S, -1)[seqs]
+        res[name + "_max_rel_err"] = float(np.abs(gs - rs).max() / max(np.abs(rs).max(), 1e-30))
+    return res
 
 
 def reference_arm(args, wl):
@@ -909,12 +938,18 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        line = gpu_arm(args, wl, rank, world)
+        kept = {}
+        line = gpu_arm(args, wl, rank, world, kept if (rank == 0 and world == 1) else None)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            v, cores, desc = oracle_sample(wl, args.cpu_budget)
+            sample = {}
+            v, cores, desc = oracle_sample(wl, args.cpu_budget, sample)
             line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
                                     "kind": "oracle", "sample": desc,
                                     "cpu_model": cpu_model()}
+            try:  # a failure here must not cost the bench line
+                line["parity"] = bench_parity(wl, kept["outs"], sample, args.z_bf16)
+            except Exception as e:  # pragma: no cover - reported, not raised
+                line["parity"] = {"error": repr(e)}
         elif rank == 0:
             line["cpu_baseline"] = None
         if rank == 0:

@@ -89,3 +89,25 @@ def test_mlp_backward_flop_count():
     """24 products of 2 d dh FLOPs per token (checkpoint forward 5, recompute
     5, token backward 11, end-of-mini-batch weight terms 3)."""
     assert bench.mlp_bwd_flops_per_token(64, 256) == 24 * 2 * 64 * 256
+
+
+def test_bench_parity_on_the_oracle_sample():
+    """The bench's parity figure compares the sampled sequences only, per
+    output, as max |gpu - ref| / max |ref|."""
+    import numpy as np
+    import torch
+    from test_sequence_layers_layer_b200 import synth
+    wl = synth.WORKLOADS["linear_ln_d64_b8h12_t2048"].scaled(B=2, H=2, T=8)
+    r = np.random.default_rng(0)
+    Zr = r.standard_normal((2, 2, 8, 64))
+    Wr = r.standard_normal((2, 2, 64, 64))
+    Zg, Wg = Zr.copy(), Wr.copy()
+    Zg[0, 1, 3, 5] += 1e-3 * np.abs(Zr).max()      # sequence 1 is sampled
+    Wg[1, 1, 0, 0] += 0.5                           # sequence 3 is not
+    outs = (torch.from_numpy(Zg).float(), torch.from_numpy(Wg).float())
+    p = bench.bench_parity(wl, outs, {"seqs": [0, 1], "ref": (Zr, Wr)})
+    assert p["sequences"] == 2 and p["of"] == 4 and p["tolerance"] == 2e-3
+    assert abs(p["z_max_rel_err"] - 1e-3) < 1e-5
+    assert p["w_out_max_rel_err"] < 1e-6
+    mlp = synth.WORKLOADS["mlp_ln_d64_dh256_b4h12_t8192"]
+    assert "note" in bench.bench_parity(mlp, None, None)
