@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(kPrefixThreads) affine_prefix_kernel(PrefixArg
     }
 }
 
+#ifndef TTT_HOST_RUN  // launch code (a host build of the kernels for tests leaves it out)
 template <int D>
 cudaError_t launch_prefix(const PrefixArgs &a, int S, cudaStream_t s) {
     constexpr size_t smem = prefix_smem_bytes(D);
@@ -142,9 +143,11 @@ cudaError_t launch_prefix(const PrefixArgs &a, int S, cudaStream_t s) {
     count_launch(s);
     return cudaSuccess;
 }
+#endif  // TTT_HOST_RUN
 
 }  // namespace
 
+#ifndef TTT_HOST_RUN
 cudaError_t launch_affine_eye(float *W, int S, int d, cudaStream_t s) {
     const size_t total = (size_t)S * d * d;
     const size_t blocks = (total + 255) / 256;
@@ -160,5 +163,7 @@ cudaError_t launch_affine_prefix(const float *M, const float *N, const float *W0
     const PrefixArgs a{M, N, W0, W_in, W_end, H, nseg, seq_stride, seg_stride, w0_per_seq};
     return d == 64 ? launch_prefix<64>(a, S, s) : launch_prefix<128>(a, S, s);
 }
+
+#endif  // TTT_HOST_RUN
 
 }  // namespace ttt
