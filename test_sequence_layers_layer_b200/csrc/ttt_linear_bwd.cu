@@ -567,6 +567,7 @@ size_t linear_bwd_workspace_bytes(int B, int H, int T, int d, int b) {
     return 4 * (S * (size_t)(T / b) * d * d + S * d * d + 2 * S * d);
 }
 
+#ifndef TTT_HOST_RUN  // launch code (a host build of the kernels for tests leaves it out)
 cudaError_t launch_linear_bwd(const LinearBwdArgs &a, cudaStream_t s) {
     const size_t S = (size_t)a.B * a.H, M = (size_t)(a.T / a.b), dd = (size_t)a.d * a.d;
     float *ws = static_cast<float *>(a.workspace);
@@ -608,5 +609,7 @@ cudaError_t launch_linear_bwd(const LinearBwdArgs &a, cudaStream_t s) {
     }
     return cudaSuccess;
 }
+
+#endif  // TTT_HOST_RUN
 
 }  // namespace ttt
