@@ -3,6 +3,12 @@
 // runs as OS threads (one per CUDA thread), __syncthreads() is a block-wide
 // std::barrier, and warp shuffles and __syncwarp() go through per-warp
 // exchange buffers and barriers. TEST CODE ONLY.
+//
+// Limits: only `extern __shared__` (dynamic) shared memory works -- the
+// including harness defines the array once, in the kernel's namespace; a
+// static `__shared__` array inside a kernel would become a private array per
+// OS thread, so kernels that declare one (the large-chunk backward's Gram
+// kernel) are not run this way. Warp shuffles must be called by all 32 lanes.
 #pragma once
 #include <barrier>
 #include <math.h>
