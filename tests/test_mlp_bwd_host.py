@@ -85,6 +85,7 @@ def _run(L, Q, K, V, eta, W1, W2, g, be, dZ, dW1, dW2, *, b, w0_per_seq, bf16):
     (2, 1, 8, 16, 2, True, False, False),
     (2, 2, 6, 16, 3, False, True, True),
     (1, 1, 4, 32, 4, False, False, True),
+    (1, 1, 32, 64, 16, False, True, True),   # the TTT-MLP workload's shape (d 64, dh 256, b 16)
 ])
 def test_host_run_matches_oracle(emu, B, H, T, d, b, w0_per_seq, bf16, with_dw):
     Q, K, V, eta, W1, W2, g, be, dZ, dW1, dW2 = _inputs(7 + T + d, B, H, T, d, w0_per_seq)
