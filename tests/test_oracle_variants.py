@@ -99,3 +99,26 @@ def test_linear_n_steps_closed_form_and_exact_fit():
     _, W = variants.linear_multistep(one(k), one(k), one(v), np.full((1, 1, 1), eta), W0[None],
                                      n_steps=60, ln=False)
     assert np.abs(k @ W[0, 0] - v).max() < 1e-12 * np.abs(v).max()
+
+
+def test_listing_recurrence_in_column_form():
+    """An independent restatement of the per-token recurrence the PyTorch
+    listing on "Test-Time Training: Linear Complexity Beyond Attention" runs
+    (column form, prediction W k on a unit-length key, error W k - v,
+    W <- W - lr (W k - v) k^T, read-out W q after the update, no LayerNorm
+    inside the loss), against the oracle's b = 1 path on normalised keys with
+    the weight transposed to the row form."""
+    r = np.random.default_rng(12)
+    d, T, lr = 4, 6, 0.05
+    q, k, v = (r.standard_normal((T, d)) for _ in range(3))
+    Wc = r.standard_normal((d, d)) * 0.3          # column form: prediction Wc @ k
+    W = Wc.copy()
+    zs = []
+    for t in range(T):
+        kn = k[t] / np.linalg.norm(k[t])
+        W = W - lr * np.outer(W @ kn - v[t], kn)
+        zs.append(W @ q[t])
+    one = lambda a: a.reshape(1, 1, T, d)  # noqa: E731
+    Zr, Wr = oracle.linear_primal(one(q), variants.normalize_keys(one(k)), one(v),
+                                  np.full((1, 1, T), lr), Wc.T[None], b=1, ln=False)
+    assert _close(Zr[0, 0], np.array(zs)) and _close(Wr[0, 0], W.T)
