@@ -585,6 +585,13 @@ def decode_arm(args, wl):
             ttt.ttt_linear_fwd(t["Q"], t["K"], t["V"], t["eta"], state, x["gamma"], x["beta"], z,
                                state, dwl.B, dwl.H, 1, dwl.d, 1, dt, flags, stream.cuda_stream)
 
+    if args.decode_kernel:  # the one-token kernel (W in registers); same buffers
+        def steps():  # noqa: F811
+            for t in toks:
+                ttt.ttt_linear_decode(t["Q"], t["K"], t["V"], t["eta"], state, x["gamma"],
+                                      x["beta"], z, dwl.B, dwl.H, dwl.d, dt,
+                                      ttt.TTT_F_LN if dwl.ln else 0, stream.cuda_stream)
+
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             steps()
@@ -619,7 +626,9 @@ def decode_arm(args, wl):
         "data": "synthetic (seeded SplitMix64 normals; bf16-rounded Q/K/V)",
         "config": {"workload": wl.name + "_decode", "B": dwl.B, "H": dwl.H, "d": dwl.d,
                    "layer_norm": dwl.ln, "tokens_per_step": dwl.B * dwl.H,
-                   "cuda_graph": graph is not None},
+                   "cuda_graph": graph is not None,
+                   "entry_point": "ttt_linear_decode" if args.decode_kernel
+                   else "ttt_linear_fwd (T = 1, b = 1)"},
     }
 
 
@@ -888,6 +897,8 @@ def main():
                     help="time the TTT-Linear backward (linear workloads) instead")
     ap.add_argument("--decode", type=int, default=0,
                     help="time N single-token decode steps (linear workloads) instead")
+    ap.add_argument("--decode-kernel", action="store_true",
+                    help="with --decode: time ttt_linear_decode (the one-token kernel, d = 64)")
     ap.add_argument("--e2e-slices", type=int, default=0,
                     help="e2e leg (linear workloads): overlap the host copies with the compute "
                          "over N batch slices (hostio.linear_fwd_host)")

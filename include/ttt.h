@@ -131,6 +131,23 @@ TTT_API ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, c
                           ttt_dtype dt, unsigned flags, ttt_stream stream);
 
 /*
+ * One TTT-Linear token per sequence (online decode, b = 1), d = 64, with the
+ * fast weight updated in place: for the token q, k, v [B][H][64] and step size
+ * eta [B][H] of every sequence, and W [B][H][64][64] fp32 (the sequence's
+ * state), computes x = k W, G = eta dl/dx, W <- W - k^T G and z = f(q; W)
+ * after the update ("Key Architectural Mechanics of TTT-Linear", parts 1-3;
+ * the listing's step()). The same result as ttt_linear_fwd with T = 1, b = 1
+ * and TTT_F_W0_PER_SEQ with W_out == W0, from a kernel specialised for it:
+ * one 128-thread block per sequence holding W in registers.
+ * flags: TTT_F_LN (gamma, beta [H][64] required), TTT_F_Z_BF16. z [B][H][64].
+ * Supported: d = 64 (TTT_ERR_SHAPE otherwise), TTT_BF16 or TTT_FP32 inputs.
+ */
+TTT_API ttt_status ttt_linear_decode(const void *q, const void *k, const void *v, const float *eta,
+                                     float *W, const float *ln_gamma, const float *ln_beta,
+                                     void *z, int B, int H, int d, ttt_dtype dt, unsigned flags,
+                                     ttt_stream stream);
+
+/*
  * TTT-Linear forward, online (b = 1), with n_steps gradient steps per token
  * ("How to Master Test-Time Training for LLMs", "How TTT Layers Actually
  * Work": the layer runs one or more steps of gradient descent per token).

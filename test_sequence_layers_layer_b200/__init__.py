@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_status_string.argtypes = [_I]
         L.ttt_linear_fwd.restype = _I
         L.ttt_linear_fwd.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_uint, _P]
+        L.ttt_linear_decode.restype = _I
+        L.ttt_linear_decode.argtypes = [_P] * 8 + [_I] * 4 + [ctypes.c_uint, _P]
         L.ttt_linear_fwd_steps.restype = _I
         L.ttt_linear_fwd_steps.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_uint, _P]
         L.ttt_linear_bwd_workspace_bytes.restype = ctypes.c_size_t
@@ -154,6 +156,13 @@ def ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                               _ptr(ln_beta), _ptr(Z), _ptr(W_out), B, H, T, d, b, dt, flags,
                               _stream(stream))
     return _check("ttt_linear_fwd", rc) if check else rc
+
+
+def ttt_linear_decode(q, k, v, eta, W, ln_gamma, ln_beta, z, B, H, d, dt, flags, stream=None,
+                      check=True):
+    rc = lib().ttt_linear_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(W), _ptr(ln_gamma),
+                                 _ptr(ln_beta), _ptr(z), B, H, d, dt, flags, _stream(stream))
+    return _check("ttt_linear_decode", rc) if check else rc
 
 
 def ttt_linear_fwd_steps(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, n_steps, dt,
@@ -330,6 +339,21 @@ def linear_fwd(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, w0_per_s
     ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                    _dtype_code(Q), flags, stream)
     return Z, W_out
+
+
+def linear_decode(q, k, v, eta, W, ln_gamma=None, ln_beta=None, *, ln, z=None, z_bf16=False,
+                  stream=None):
+    """One TTT-Linear token per sequence, d = 64: q, k, v [B, H, 64], eta [B, H],
+    W [B, H, 64, 64] fp32 updated in place (ttt_linear_decode). Returns z."""
+    import torch
+    B, H, d = q.shape
+    if z is None:
+        z = torch.empty((B, H, d), dtype=torch.bfloat16 if z_bf16 else torch.float32,
+                        device=q.device)
+    flags = (TTT_F_LN if ln else 0) | (TTT_F_Z_BF16 if z_bf16 else 0)
+    ttt_linear_decode(q, k, v, eta, W, ln_gamma, ln_beta, z, B, H, d, _dtype_code(q), flags,
+                      stream)
+    return z
 
 
 def linear_fwd_steps(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, n_steps, ln,

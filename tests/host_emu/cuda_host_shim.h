@@ -57,10 +57,10 @@ inline float __shfl_xor_sync(unsigned, float v, int m) {
 }
 inline float rsqrtf(float x) { return 1.f / sqrtf(x); }
 
-// Runs fn() as every thread of nblocks blocks of 256 threads, one block at a time.
+// Runs fn() as every thread of nblocks blocks of nt threads (a multiple of
+// 32, at most 256), one block at a time.
 template <class Fn>
-static void run_blocks(int nblocks, Fn fn) {
-    const int nt = emu::kMaxThreads;
+static void run_blocks(int nblocks, Fn fn, int nt = emu::kMaxThreads) {
     emu::nthreads = nt;
     blockDim = {(unsigned)nt, 1, 1};
     gridDim = {(unsigned)nblocks, 1, 1};

@@ -233,3 +233,16 @@ def test_mlp_backward_host_validation():
     assert call(workspace_bytes=need - 1) == -9
     assert call(workspace=A + 64) == -9
     assert call() == -8                               # no GPU here
+
+
+def test_decode_host_validation():
+    A = ALIGNED
+    dc = dict(q=A, k=A, v=A, eta=A, W=A, ln_gamma=A, ln_beta=A, z=A, B=2, H=3, d=64,
+              dt=ttt.TTT_BF16, flags=ttt.TTT_F_LN, stream=0)
+    call = lambda **kw: ttt.ttt_linear_decode(**{**dc, **kw}, check=False)  # noqa: E731
+    assert call(d=32) == -2                     # the decode kernel is d = 64
+    assert call(flags=ttt.TTT_F_W0_PER_SEQ) == -1
+    assert call(ln_gamma=None) == -5
+    assert call(W=A + 8) == -4
+    assert call(dt=4) == -3
+    assert call(flags=0, ln_gamma=None, ln_beta=None) == -8   # valid without LN; no GPU here

@@ -67,3 +67,29 @@ def test_mlp_decode_loop():
     Zr, W1r, W2r = run_oracle(inp)
     assert max_rel_err(Z.double().cpu().numpy(), Zr, wl) <= TOL["bf16"]
     assert max_rel_err(s2.double().cpu().numpy(), W2r, wl) <= TOL["bf16"]
+
+
+@pytest.mark.late
+@pytest.mark.parametrize("dtype,ln", [("bf16", True), ("fp32", True), ("bf16", False)])
+def test_decode_kernel_loop(dtype, ln):
+    """ttt_linear_decode (the one-token kernel, W in registers): a token loop
+    against the oracle's online update and against the same loop through
+    ttt_linear_fwd (T = 1), both within the dtype's tolerance."""
+    wl = W["linear_ln_d64_b8h12_t2048"].scaled(B=2, H=3, T=24, b=1, dtype=dtype, ln=ln)
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    state = x["W1"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    Z = torch.empty((wl.B, wl.H, wl.T, wl.d), dtype=torch.float32, device="cuda")
+    for i in range(wl.T):
+        q, k, v = (x[n][:, :, i].contiguous() for n in ("Q", "K", "V"))
+        e = x["eta"][:, :, i].contiguous()
+        Z[:, :, i] = ttt.linear_decode(q, k, v, e, state, x["gamma"], x["beta"], ln=ln)
+    torch.cuda.synchronize()
+    assert ttt.ttt_device_status() == 0
+    Zr, Wr = run_oracle(inp)
+    assert max_rel_err(Z.double().cpu().numpy(), Zr, wl) <= TOL[dtype]
+    assert max_rel_err(state.double().cpu().numpy(), Wr, wl) <= TOL[dtype]
+    Zw, Ww = ttt.linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
+                            b=1, ln=ln)
+    torch.cuda.synchronize()
+    assert max_rel_err(Z.double().cpu().numpy(), Zw.double().cpu().numpy(), wl) <= TOL[dtype]
