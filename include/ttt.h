@@ -139,7 +139,8 @@ TTT_API ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, c
  * the listing's step()). The same result as ttt_linear_fwd with T = 1, b = 1
  * and TTT_F_W0_PER_SEQ with W_out == W0, from a kernel specialised for it:
  * one 128-thread block per sequence holding W in registers.
- * flags: TTT_F_LN (gamma, beta [H][64] required), TTT_F_Z_BF16. z [B][H][64].
+ * flags: TTT_F_LN (gamma, beta [H][64] required), TTT_F_Z_BF16, TTT_F_L2_KEYS.
+ *   z [B][H][64].
  * Supported: d = 64 (TTT_ERR_SHAPE otherwise), TTT_BF16 or TTT_FP32 inputs.
  */
 TTT_API ttt_status ttt_linear_decode(const void *q, const void *k, const void *v, const float *eta,

@@ -342,7 +342,7 @@ def linear_fwd(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, w0_per_s
 
 
 def linear_decode(q, k, v, eta, W, ln_gamma=None, ln_beta=None, *, ln, z=None, z_bf16=False,
-                  stream=None):
+                  l2_keys=False, stream=None):
     """One TTT-Linear token per sequence, d = 64: q, k, v [B, H, 64], eta [B, H],
     W [B, H, 64, 64] fp32 updated in place (ttt_linear_decode). Returns z."""
     import torch
@@ -350,7 +350,8 @@ def linear_decode(q, k, v, eta, W, ln_gamma=None, ln_beta=None, *, ln, z=None, z
     if z is None:
         z = torch.empty((B, H, d), dtype=torch.bfloat16 if z_bf16 else torch.float32,
                         device=q.device)
-    flags = (TTT_F_LN if ln else 0) | (TTT_F_Z_BF16 if z_bf16 else 0)
+    flags = (TTT_F_LN if ln else 0) | (TTT_F_Z_BF16 if z_bf16 else 0) | \
+        (TTT_F_L2_KEYS if l2_keys else 0)
     ttt_linear_decode(q, k, v, eta, W, ln_gamma, ln_beta, z, B, H, d, _dtype_code(q), flags,
                       stream)
     return z

@@ -166,7 +166,8 @@ cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const 
 // One-token TTT-Linear decode, d = 64 (ttt_decode.cu).
 cudaError_t launch_linear_decode(const void *q, const void *k, const void *v, const float *eta,
                                  const float *gamma, const float *beta, float *W, void *z, int B,
-                                 int H, bool bf16, bool ln, bool z_bf16, cudaStream_t s);
+                                 int H, bool bf16, bool ln, bool z_bf16, bool l2_keys,
+                                 cudaStream_t s);
 // TTT-MLP backward (ttt_mlp_bwd.cu).
 bool mlp_bwd_supported(int d, int dh, int b);
 size_t mlp_bwd_workspace_bytes(int B, int H, int T, int d, int b);
@@ -278,7 +279,7 @@ ttt_status ttt_linear_fwd_steps(const void *Q, const void *K, const void *V, con
 ttt_status ttt_linear_decode(const void *q, const void *k, const void *v, const float *eta,
                              float *W, const float *ln_gamma, const float *ln_beta, void *z, int B,
                              int H, int d, ttt_dtype dt, unsigned flags, ttt_stream stream) {
-    if (flags & ~(TTT_F_LN | TTT_F_Z_BF16)) return TTT_ERR_ARG;
+    if (flags & ~(TTT_F_LN | TTT_F_Z_BF16 | TTT_F_L2_KEYS)) return TTT_ERR_ARG;
     const bool ln = flags & TTT_F_LN;
     if (!q || !k || !v || !eta || !W || !z) return TTT_ERR_PTR;
     if (ln && (!ln_gamma || !ln_beta)) return TTT_ERR_PTR;
@@ -294,7 +295,8 @@ ttt_status ttt_linear_decode(const void *q, const void *k, const void *v, const 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
     return launched(launch_linear_decode(q, k, v, eta, ln_gamma, ln_beta, W, z, B, H,
-                                         dt == TTT_BF16, ln, (flags & TTT_F_Z_BF16) != 0, cs));
+                                         dt == TTT_BF16, ln, (flags & TTT_F_Z_BF16) != 0,
+                                         (flags & TTT_F_L2_KEYS) != 0, cs));
 }
 
 size_t ttt_linear_bwd_workspace_bytes(int B, int H, int T, int d, int b) {

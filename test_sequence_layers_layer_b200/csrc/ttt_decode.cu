@@ -26,7 +26,7 @@ struct DecodeArgs {
     float *W;  // [S][64][64], updated in place
     float *z;  // [S][64]; bf16 when z_bf16
     int H;
-    bool bf16, ln, z_bf16;
+    bool bf16, ln, z_bf16, l2_keys;
 };
 
 __device__ __forceinline__ float dec_warp_sum(float v) {
@@ -47,7 +47,7 @@ __device__ __forceinline__ float col_sum(float v, int h, float *slot) {
 
 __global__ void __launch_bounds__(kDecThreads) linear_decode_kernel(DecodeArgs a) {
     extern __shared__ float dsm[];
-    float *ks = dsm, *qs = ks + kDD, *vs = qs + kDD, *slots = vs + kDD;  // slots: 6 x 4 floats
+    float *ks = dsm, *qs = ks + kDD, *vs = qs + kDD, *slots = vs + kDD;  // slots: 7 x 4 floats
     const int seq = blockIdx.x, tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int j = warp * 16 + (lane >> 1), h = lane & 1;
@@ -65,6 +65,12 @@ __global__ void __launch_bounds__(kDecThreads) linear_decode_kernel(DecodeArgs a
     const float g = a.ln ? a.gamma[(size_t)(seq % a.H) * kDD + j] : 1.f;
     const float be = a.ln ? a.beta[(size_t)(seq % a.H) * kDD + j] : 0.f;
     __syncthreads();  // k, q, v staged
+    if (a.l2_keys) {  // k / max(||k||, 1e-12), as the listing normalises its key
+        const float kk = ks[j];
+        const float inv = 1.f / fmaxf(sqrtf(col_sum(kk * kk, h, slots + 24)), 1e-12f);
+        if (h == 0) ks[j] = kk * inv;
+        __syncthreads();
+    }
 
     // x_j = sum_i k_i W[i][j]
     float x = 0.f;
@@ -110,9 +116,11 @@ __global__ void __launch_bounds__(kDecThreads) linear_decode_kernel(DecodeArgs a
 #ifndef TTT_HOST_RUN  // launch code (a host build of the kernels for tests leaves it out)
 cudaError_t launch_linear_decode(const void *q, const void *k, const void *v, const float *eta,
                                  const float *gamma, const float *beta, float *W, void *z, int B,
-                                 int H, bool bf16, bool ln, bool z_bf16, cudaStream_t s) {
-    const DecodeArgs a{q, k, v, eta, gamma, beta, W, static_cast<float *>(z), H, bf16, ln, z_bf16};
-    const size_t smem = sizeof(float) * (3 * kDD + 6 * 4);
+                                 int H, bool bf16, bool ln, bool z_bf16, bool l2_keys,
+                                 cudaStream_t s) {
+    const DecodeArgs a{q, k, v, eta, gamma, beta, W, static_cast<float *>(z), H,
+                       bf16, ln, z_bf16, l2_keys};
+    const size_t smem = sizeof(float) * (3 * kDD + 7 * 4);
     linear_decode_kernel<<<(unsigned)(B * H), kDecThreads, smem, s>>>(a);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launch(s);

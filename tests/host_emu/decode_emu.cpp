@@ -14,8 +14,9 @@ float dsm[1024];  // the decode kernel's dynamic shared memory
 extern "C" int ttt_linear_decode_host_run(const void *q, const void *k, const void *v,
                                           const float *eta, const float *gamma,
                                           const float *beta, float *W, float *z, int B, int H,
-                                          int bf16, int ln) {
-    const ttt::DecodeArgs a{q, k, v, eta, gamma, beta, W, z, H, bf16 != 0, ln != 0, false};
+                                          int bf16, int ln, int l2_keys) {
+    const ttt::DecodeArgs a{q, k, v, eta, gamma, beta, W, z, H, bf16 != 0, ln != 0, false,
+                            l2_keys != 0};
     run_blocks(B * H, [&] { ttt::linear_decode_kernel(a); }, ttt::kDecThreads);
     return 0;
 }

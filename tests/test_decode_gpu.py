@@ -70,8 +70,9 @@ def test_mlp_decode_loop():
 
 
 @pytest.mark.late
-@pytest.mark.parametrize("dtype,ln", [("bf16", True), ("fp32", True), ("bf16", False)])
-def test_decode_kernel_loop(dtype, ln):
+@pytest.mark.parametrize("dtype,ln,l2", [("bf16", True, False), ("fp32", True, False),
+                                         ("bf16", False, False), ("fp32", True, True)])
+def test_decode_kernel_loop(dtype, ln, l2):
     """ttt_linear_decode (the one-token kernel, W in registers): a token loop
     against the oracle's online update and against the same loop through
     ttt_linear_fwd (T = 1), both within the dtype's tolerance."""
@@ -83,13 +84,20 @@ def test_decode_kernel_loop(dtype, ln):
     for i in range(wl.T):
         q, k, v = (x[n][:, :, i].contiguous() for n in ("Q", "K", "V"))
         e = x["eta"][:, :, i].contiguous()
-        Z[:, :, i] = ttt.linear_decode(q, k, v, e, state, x["gamma"], x["beta"], ln=ln)
+        Z[:, :, i] = ttt.linear_decode(q, k, v, e, state, x["gamma"], x["beta"], ln=ln,
+                                       l2_keys=l2)
     torch.cuda.synchronize()
     assert ttt.ttt_device_status() == 0
-    Zr, Wr = run_oracle(inp)
+    if l2:
+        from oracle import variants
+        import oracle
+        Zr, Wr = oracle.linear_primal(inp.Q, variants.normalize_keys(inp.K), inp.V, inp.eta,
+                                      inp.W1, inp.gamma, inp.beta, b=1, ln=ln)
+    else:
+        Zr, Wr = run_oracle(inp)
     assert max_rel_err(Z.double().cpu().numpy(), Zr, wl) <= TOL[dtype]
     assert max_rel_err(state.double().cpu().numpy(), Wr, wl) <= TOL[dtype]
     Zw, Ww = ttt.linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
-                            b=1, ln=ln)
+                            b=1, ln=ln, l2_keys=l2)
     torch.cuda.synchronize()
     assert max_rel_err(Z.double().cpu().numpy(), Zw.double().cpu().numpy(), wl) <= TOL[dtype]

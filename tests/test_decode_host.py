@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 
 import oracle
+from oracle import variants
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "host_emu", "decode_emu.cpp")
@@ -23,12 +24,12 @@ def emu(tmp_path_factory):
                     "-I/usr/local/cuda/include", SRC, "-o", so], check=True)
     L = ctypes.CDLL(so)
     L.ttt_linear_decode_host_run.restype = ctypes.c_int
-    L.ttt_linear_decode_host_run.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int] * 4
+    L.ttt_linear_decode_host_run.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int] * 5
     return L
 
 
-@pytest.mark.parametrize("ln", [True, False])
-def test_token_loop_matches_oracle(emu, ln):
+@pytest.mark.parametrize("ln,l2", [(True, False), (False, False), (True, True)])
+def test_token_loop_matches_oracle(emu, ln, l2):
     B, H, T, d = 2, 3, 12, 64
     r = np.random.default_rng(3 + int(ln))
     f = lambda a: np.ascontiguousarray(a, dtype=np.float32)  # noqa: E731
@@ -43,9 +44,11 @@ def test_token_loop_matches_oracle(emu, ln):
         z = np.zeros((B, H, d), np.float32)
         assert emu.ttt_linear_decode_host_run(q.ctypes.data, k.ctypes.data, v.ctypes.data,
                                               e.ctypes.data, g.ctypes.data, be.ctypes.data,
-                                              W.ctypes.data, z.ctypes.data, B, H, 0, int(ln)) == 0
+                                              W.ctypes.data, z.ctypes.data, B, H, 0, int(ln),
+                                              int(l2)) == 0
         Z[:, :, t] = z
-    Zr, Wr = oracle.linear_primal(Q, K, V, eta, W0, g if ln else None, be if ln else None, b=1,
+    Kr = variants.normalize_keys(K) if l2 else K
+    Zr, Wr = oracle.linear_primal(Q, Kr, V, eta, W0, g if ln else None, be if ln else None, b=1,
                                   ln=ln, w0_per_seq=True)
     assert np.abs(Z - Zr).max() <= 1e-5 * np.abs(Zr).max()
     assert np.abs(W - Wr).max() <= 1e-5 * np.abs(Wr).max()
