@@ -585,6 +585,16 @@ def decode_arm(args, wl):
             ttt.ttt_linear_fwd(t["Q"], t["K"], t["V"], t["eta"], state, x["gamma"], x["beta"], z,
                                state, dwl.B, dwl.H, 1, dwl.d, 1, dt, flags, stream.cuda_stream)
 
+    if dwl.kind == "mlp":  # TTT-MLP: both layers' state per sequence, updated in place
+        state2 = x["W2"].unsqueeze(0).expand(dwl.B, -1, -1, -1).contiguous()
+        W0_2 = state2.clone()
+
+        def steps():  # noqa: F811
+            for t in toks:
+                ttt.ttt_mlp_fwd(t["Q"], t["K"], t["V"], t["eta"], state, state2, x["gamma"],
+                                x["beta"], z, state, state2, dwl.B, dwl.H, 1, dwl.d, dwl.dh, 1, dt,
+                                ttt.TTT_F_LN | ttt.TTT_F_W0_PER_SEQ, stream.cuda_stream)
+
     if args.decode_kernel:  # the one-token kernel (W in registers); same buffers
         def steps():  # noqa: F811
             for t in toks:
@@ -605,6 +615,8 @@ def decode_arm(args, wl):
         except Exception:
             graph = None
         state.copy_(W0)
+        if dwl.kind == "mlp":
+            state2.copy_(W0_2)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         reps = max(1, args.steps)
         e0.record(stream)
@@ -619,7 +631,8 @@ def decode_arm(args, wl):
         raise RuntimeError("device status error in the decode loop")
     us = e0.elapsed_time(e1) * 1e3 / (reps * n)
     return {
-        "metric": "TTT-Linear single-token decode step (b = 1, state updated in place)",
+        "metric": ("TTT-MLP" if dwl.kind == "mlp" else "TTT-Linear")
+                  + " single-token decode step (b = 1, state updated in place)",
         "value": us, "unit": "us/step", "higher_is_better": False,
         "tokens_per_s": dwl.B * dwl.H / (us * 1e-6),
         "n_gpus": 1, "steps": reps * n, "warmup": args.warmup, "dtype": dwl.dtype,
@@ -921,8 +934,10 @@ def main():
         return
 
     if args.decode:
-        if wl.kind != "linear":
-            ap.error("--decode times the linear workloads")
+        if wl.kind == "chunk":
+            ap.error("--decode times the TTT-Linear and TTT-MLP workloads")
+        if args.decode_kernel and wl.kind != "linear":
+            ap.error("--decode-kernel is the TTT-Linear one-token kernel")
         if rank == 0:
             print(json.dumps(decode_arm(args, wl)), flush=True)
         return
