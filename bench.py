@@ -595,7 +595,13 @@ def decode_arm(args, wl):
                                 x["beta"], z, state, state2, dwl.B, dwl.H, 1, dwl.d, dwl.dh, 1, dt,
                                 ttt.TTT_F_LN | ttt.TTT_F_W0_PER_SEQ, stream.cuda_stream)
 
-    if args.decode_kernel:  # the one-token kernel (W in registers); same buffers
+    if args.decode_kernel and dwl.kind == "mlp":  # the one-token TTT-MLP kernel
+        def steps():  # noqa: F811
+            for t in toks:
+                ttt.ttt_mlp_decode(t["Q"], t["K"], t["V"], t["eta"], state, state2, x["gamma"],
+                                   x["beta"], z, dwl.B, dwl.H, dwl.d, dwl.dh, dt, ttt.TTT_F_LN,
+                                   stream.cuda_stream)
+    elif args.decode_kernel:  # the one-token kernel (W in registers); same buffers
         def steps():  # noqa: F811
             for t in toks:
                 ttt.ttt_linear_decode(t["Q"], t["K"], t["V"], t["eta"], state, x["gamma"],
@@ -640,8 +646,10 @@ def decode_arm(args, wl):
         "config": {"workload": wl.name + "_decode", "B": dwl.B, "H": dwl.H, "d": dwl.d,
                    "layer_norm": dwl.ln, "tokens_per_step": dwl.B * dwl.H,
                    "cuda_graph": graph is not None,
-                   "entry_point": "ttt_linear_decode" if args.decode_kernel
-                   else "ttt_linear_fwd (T = 1, b = 1)"},
+                   "entry_point": (("ttt_mlp_decode" if dwl.kind == "mlp" else "ttt_linear_decode")
+                                   if args.decode_kernel else
+                                   ("ttt_mlp_fwd" if dwl.kind == "mlp" else "ttt_linear_fwd")
+                                   + " (T = 1, b = 1)")},
     }
 
 
@@ -911,7 +919,8 @@ def main():
     ap.add_argument("--decode", type=int, default=0,
                     help="time N single-token decode steps (linear workloads) instead")
     ap.add_argument("--decode-kernel", action="store_true",
-                    help="with --decode: time ttt_linear_decode (the one-token kernel, d = 64)")
+                    help="with --decode: time the one-token kernel (ttt_linear_decode, "
+                         "ttt_mlp_decode)")
     ap.add_argument("--e2e-slices", type=int, default=0,
                     help="e2e leg (linear workloads): overlap the host copies with the compute "
                          "over N batch slices (hostio.linear_fwd_host)")
@@ -936,8 +945,7 @@ def main():
     if args.decode:
         if wl.kind == "chunk":
             ap.error("--decode times the TTT-Linear and TTT-MLP workloads")
-        if args.decode_kernel and wl.kind != "linear":
-            ap.error("--decode-kernel is the TTT-Linear one-token kernel")
+
         if rank == 0:
             print(json.dumps(decode_arm(args, wl)), flush=True)
         return

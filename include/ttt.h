@@ -149,6 +149,22 @@ TTT_API ttt_status ttt_linear_decode(const void *q, const void *k, const void *v
                                      ttt_stream stream);
 
 /*
+ * One TTT-MLP token per sequence (online decode, b = 1), d = 64, dh = 256, both
+ * layers updated in place: q, k, v [B][H][64], eta [B][H], W1 [B][H][64][256]
+ * and W2 [B][H][256][64] fp32 (the sequence's state), gamma, beta [H][64],
+ * z [B][H][64]. The same result as ttt_mlp_fwd with T = 1, b = 1 and
+ * TTT_F_W0_PER_SEQ with the outputs aliasing the inputs, from a kernel
+ * specialised for it: one 256-thread block per sequence, thread j holding
+ * column j of W1 and row j of W2 in registers.
+ * flags: TTT_F_LN (required), TTT_F_Z_BF16. Supported: d = 64, dh = 256
+ * (TTT_ERR_SHAPE otherwise); TTT_BF16 or TTT_FP32 inputs; W1 and W2 distinct.
+ */
+TTT_API ttt_status ttt_mlp_decode(const void *q, const void *k, const void *v, const float *eta,
+                                  float *W1, float *W2, const float *ln_gamma,
+                                  const float *ln_beta, void *z, int B, int H, int d, int dh,
+                                  ttt_dtype dt, unsigned flags, ttt_stream stream);
+
+/*
  * TTT-Linear forward, online (b = 1), with n_steps gradient steps per token
  * ("How to Master Test-Time Training for LLMs", "How TTT Layers Actually
  * Work": the layer runs one or more steps of gradient descent per token).

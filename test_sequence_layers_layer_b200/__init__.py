@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_status_string.argtypes = [_I]
         L.ttt_linear_fwd.restype = _I
         L.ttt_linear_fwd.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_uint, _P]
+        L.ttt_mlp_decode.restype = _I
+        L.ttt_mlp_decode.argtypes = [_P] * 9 + [_I] * 5 + [ctypes.c_uint, _P]
         L.ttt_linear_decode.restype = _I
         L.ttt_linear_decode.argtypes = [_P] * 8 + [_I] * 4 + [ctypes.c_uint, _P]
         L.ttt_linear_fwd_steps.restype = _I
@@ -156,6 +158,14 @@ def ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                               _ptr(ln_beta), _ptr(Z), _ptr(W_out), B, H, T, d, b, dt, flags,
                               _stream(stream))
     return _check("ttt_linear_fwd", rc) if check else rc
+
+
+def ttt_mlp_decode(q, k, v, eta, W1, W2, ln_gamma, ln_beta, z, B, H, d, dh, dt, flags,
+                   stream=None, check=True):
+    rc = lib().ttt_mlp_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(W1), _ptr(W2),
+                              _ptr(ln_gamma), _ptr(ln_beta), _ptr(z), B, H, d, dh, dt, flags,
+                              _stream(stream))
+    return _check("ttt_mlp_decode", rc) if check else rc
 
 
 def ttt_linear_decode(q, k, v, eta, W, ln_gamma, ln_beta, z, B, H, d, dt, flags, stream=None,
@@ -339,6 +349,20 @@ def linear_fwd(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, w0_per_s
     ttt_linear_fwd(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, b,
                    _dtype_code(Q), flags, stream)
     return Z, W_out
+
+
+def mlp_decode(q, k, v, eta, W1, W2, ln_gamma, ln_beta, *, z=None, z_bf16=False, stream=None):
+    """One TTT-MLP token per sequence, d = 64, dh = 256: q, k, v [B, H, 64], eta
+    [B, H], W1 [B, H, 64, 256] and W2 [B, H, 256, 64] fp32 updated in place
+    (ttt_mlp_decode). Returns z."""
+    import torch
+    B, H, d = q.shape
+    if z is None:
+        z = torch.empty((B, H, d), dtype=torch.bfloat16 if z_bf16 else torch.float32,
+                        device=q.device)
+    ttt_mlp_decode(q, k, v, eta, W1, W2, ln_gamma, ln_beta, z, B, H, d, W1.shape[-1],
+                   _dtype_code(q), TTT_F_LN | (TTT_F_Z_BF16 if z_bf16 else 0), stream)
+    return z
 
 
 def linear_decode(q, k, v, eta, W, ln_gamma=None, ln_beta=None, *, ln, z=None, z_bf16=False,

@@ -168,6 +168,10 @@ cudaError_t launch_linear_decode(const void *q, const void *k, const void *v, co
                                  const float *gamma, const float *beta, float *W, void *z, int B,
                                  int H, bool bf16, bool ln, bool z_bf16, bool l2_keys,
                                  cudaStream_t s);
+// One-token TTT-MLP decode, d = 64, hidden 256 (ttt_mlp_decode.cu).
+cudaError_t launch_mlp_decode(const void *q, const void *k, const void *v, const float *eta,
+                              const float *gamma, const float *beta, float *W1, float *W2,
+                              void *z, int B, int H, bool bf16, bool z_bf16, cudaStream_t s);
 // TTT-MLP backward (ttt_mlp_bwd.cu).
 bool mlp_bwd_supported(int d, int dh, int b);
 size_t mlp_bwd_workspace_bytes(int B, int H, int T, int d, int b);
@@ -297,6 +301,31 @@ ttt_status ttt_linear_decode(const void *q, const void *k, const void *v, const 
     return launched(launch_linear_decode(q, k, v, eta, ln_gamma, ln_beta, W, z, B, H,
                                          dt == TTT_BF16, ln, (flags & TTT_F_Z_BF16) != 0,
                                          (flags & TTT_F_L2_KEYS) != 0, cs));
+}
+
+ttt_status ttt_mlp_decode(const void *q, const void *k, const void *v, const float *eta,
+                          float *W1, float *W2, const float *ln_gamma, const float *ln_beta,
+                          void *z, int B, int H, int d, int dh, ttt_dtype dt, unsigned flags,
+                          ttt_stream stream) {
+    if (flags & ~(TTT_F_LN | TTT_F_Z_BF16)) return TTT_ERR_ARG;
+    if (!(flags & TTT_F_LN)) return TTT_ERR_ARG;  // TTT-MLP always has its LayerNorm
+    if (!q || !k || !v || !eta || !W1 || !W2 || !ln_gamma || !ln_beta || !z) return TTT_ERR_PTR;
+    if (B <= 0 || H <= 0 || (long long)B * H > (1LL << 30) || d != 64 || dh != 256)
+        return TTT_ERR_SHAPE;
+    if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(W1) || !aligned16(W2) ||
+        !aligned16(z))
+        return TTT_ERR_ALIGN;
+    if (W1 == W2) return TTT_ERR_ARG;
+    ttt_status st = check_arch();
+    if (st != TTT_OK) return st;
+    const void *ptrs[] = {q, k, v, eta, W1, W2, ln_gamma, ln_beta, z};
+    st = check_device_ptrs(ptrs, 9);
+    if (st != TTT_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    return launched(launch_mlp_decode(q, k, v, eta, ln_gamma, ln_beta, W1, W2, z, B, H,
+                                      dt == TTT_BF16, (flags & TTT_F_Z_BF16) != 0, cs));
 }
 
 size_t ttt_linear_bwd_workspace_bytes(int B, int H, int T, int d, int b) {

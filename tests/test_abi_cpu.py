@@ -246,3 +246,16 @@ def test_decode_host_validation():
     assert call(W=A + 8) == -4
     assert call(dt=4) == -3
     assert call(flags=0, ln_gamma=None, ln_beta=None) == -8   # valid without LN; no GPU here
+
+
+def test_mlp_decode_host_validation():
+    A = ALIGNED
+    md = dict(q=A, k=A, v=A, eta=A, W1=A, W2=A + (1 << 20), ln_gamma=A, ln_beta=A, z=A, B=2,
+              H=3, d=64, dh=256, dt=ttt.TTT_BF16, flags=ttt.TTT_F_LN, stream=0)
+    call = lambda **kw: ttt.ttt_mlp_decode(**{**md, **kw}, check=False)  # noqa: E731
+    assert call(flags=0) == -1                  # TTT-MLP always has its LayerNorm
+    assert call(dh=128) == -2 and call(d=32, dh=128) == -2
+    assert call(W2=A) == -1                     # W1 and W2 must differ
+    assert call(ln_beta=None) == -5
+    assert call(z=A + 2) == -4
+    assert call() == -8                         # no GPU here

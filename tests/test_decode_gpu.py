@@ -101,3 +101,31 @@ def test_decode_kernel_loop(dtype, ln, l2):
                             b=1, ln=ln, l2_keys=l2)
     torch.cuda.synchronize()
     assert max_rel_err(Z.double().cpu().numpy(), Zw.double().cpu().numpy(), wl) <= TOL[dtype]
+
+
+@pytest.mark.late
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_mlp_decode_kernel_loop(dtype):
+    """ttt_mlp_decode (the one-token TTT-MLP kernel): a token loop against the
+    oracle's online update and against the same loop through ttt_mlp_fwd
+    (T = 1), within the dtype's tolerance."""
+    wl = W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=1, H=2, T=12, b=1, dtype=dtype)
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    s1 = x["W1"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    s2 = x["W2"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    Z = torch.empty((wl.B, wl.H, wl.T, wl.d), dtype=torch.float32, device="cuda")
+    for i in range(wl.T):
+        q, k, v = (x[n][:, :, i].contiguous() for n in ("Q", "K", "V"))
+        e = x["eta"][:, :, i].contiguous()
+        Z[:, :, i] = ttt.mlp_decode(q, k, v, e, s1, s2, x["gamma"], x["beta"])
+    torch.cuda.synchronize()
+    assert ttt.ttt_device_status() == 0
+    Zr, W1r, W2r = run_oracle(inp)
+    assert max_rel_err(Z.double().cpu().numpy(), Zr, wl) <= TOL[dtype]
+    assert max_rel_err(s1.double().cpu().numpy(), W1r, wl) <= TOL[dtype]
+    assert max_rel_err(s2.double().cpu().numpy(), W2r, wl) <= TOL[dtype]
+    Zw, _, _ = ttt.mlp_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["W2"], x["gamma"],
+                           x["beta"], b=1)
+    torch.cuda.synchronize()
+    assert max_rel_err(Z.double().cpu().numpy(), Zw.double().cpu().numpy(), wl) <= TOL[dtype]
