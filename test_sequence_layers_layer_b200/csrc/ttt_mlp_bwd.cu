@@ -18,6 +18,12 @@ struct DevCtx {
     int tid, nt;
     float *sm;
     __device__ void sync() { __syncthreads(); }
+    // sum over the 32 lanes of the calling warp; every lane must call it
+    __device__ float warp_sum(float v) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        return v;
+    }
 };
 
 __global__ void __launch_bounds__(kBwdThreads) mlp_bwd_kernel(mlp_bwd_body::Params p) {

@@ -6,6 +6,7 @@
 #include <barrier>
 #include <cstring>
 #include <math.h>
+#include <memory>
 #include <thread>
 #include <vector>
 
@@ -19,7 +20,19 @@ struct HostCtx {
     int tid, nt;
     float *sm;
     std::barrier<> *bar;
+    std::unique_ptr<std::barrier<>> *warp_bar;  // one barrier of 32 per warp
+    float *xbuf;               // [warps][32] exchange buffer
     void sync() { bar->arrive_and_wait(); }
+    // sum over the 32 lanes of the calling warp (all lanes call it)
+    float warp_sum(float v) {
+        const int w = tid / 32, l = tid % 32;
+        xbuf[w * 32 + l] = v;
+        warp_bar[w]->arrive_and_wait();
+        float s = 0.f;
+        for (int k = 0; k < 32; ++k) s += xbuf[w * 32 + k];
+        warp_bar[w]->arrive_and_wait();
+        return s;
+    }
 };
 
 }  // namespace
@@ -38,12 +51,16 @@ extern "C" int ttt_mlp_bwd_host_run(const void *Q, const void *K, const void *V,
     mlp_bwd_body::Params p{Q, K, V, eta, W1_0, W2_0, gamma, beta, dZ, dW1_out, dW2_out,
                           dQ, dK, dV, deta, dW1_0, dW2_0, ws.data(), H, T, d, b, bf16 != 0,
                           w0_per_seq != 0};
+    if (nt % 32) return -1;
+    std::vector<float> xbuf(nt);
     for (int seq = 0; seq < B * H; ++seq) {
         std::barrier<> bar(nt);
+        std::vector<std::unique_ptr<std::barrier<>>> wbars;
+        for (int w = 0; w < nt / 32; ++w) wbars.push_back(std::make_unique<std::barrier<>>(32));
         std::vector<std::thread> th;
         for (int t = 0; t < nt; ++t)
             th.emplace_back([&, t] {
-                HostCtx cx{t, nt, sm.data(), &bar};
+                HostCtx cx{t, nt, sm.data(), &bar, wbars.data(), xbuf.data()};
                 mlp_bwd_body::run_sequence(cx, p, seq);
             });
         for (auto &x : th) x.join();
