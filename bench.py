@@ -1,8 +1,11 @@
 #!/usr/bin/env python
 """Benchmark of the TTT-layer forward pass on B200 (libttt.so through its C ABI).
 
-Default workload: TTT-Linear with f(k) = k + LN(k W), d = 64, mini-batch 16,
-B = 8, H = 12, T = 2048, bf16 Q/K/V, per-token eta (196,608 tokens per step).
+Default workload: large-chunk TTT with a linear fast weight, d = 128, chunk
+2048, apply-then-update, eta = 1/2048, B = 4, H = 8, T = 32768, bf16 Q/K/V
+(1,048,576 tokens per step): the largest single-GPU workload. `--workload`
+selects the others (TTT-Linear + LN at d = 64, the long-context TTT-Linear,
+TTT-MLP, the fp32 d = 16 case).
 A step is one library call over one batch of seeded synthetic inputs that
 are already resident in HBM; between timed steps a 256 MiB buffer is written
 to flush the 126 MB L2. Steps are timed with CUDA events on the launching
@@ -34,7 +37,7 @@ sys.path.insert(0, ROOT)
 
 from test_sequence_layers_layer_b200 import synth  # noqa: E402
 
-DEFAULT_WORKLOAD = "linear_ln_d64_b8h12_t2048"
+DEFAULT_WORKLOAD = "chunk_d128_c2048_b4h8_t32768"
 METRIC = "TTT-layer fwd tokens/sec at 1 B200; % of dense bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
@@ -575,7 +578,7 @@ def decode_arm(args, wl):
     dt = ttt.TTT_BF16 if dwl.dtype == "bf16" else ttt.TTT_FP32
     flags = (ttt.TTT_F_LN if dwl.ln else 0) | ttt.TTT_F_W0_PER_SEQ
     toks = [{k: x[k][:, :, i:i + 1].contiguous() for k in ("Q", "K", "V", "eta")} for i in range(n)]
-    state = x["W1"].unsqueeze(0).expand(dwl.B, -1, -1, -1).contiguous()
+    state = x["W1"].unsqueeze(0).repeat(dwl.B, 1, 1, 1)
     W0 = state.clone()
     z = torch.empty((dwl.B, dwl.H, 1, dwl.d), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
@@ -586,7 +589,7 @@ def decode_arm(args, wl):
                                state, dwl.B, dwl.H, 1, dwl.d, 1, dt, flags, stream.cuda_stream)
 
     if dwl.kind == "mlp":  # TTT-MLP: both layers' state per sequence, updated in place
-        state2 = x["W2"].unsqueeze(0).expand(dwl.B, -1, -1, -1).contiguous()
+        state2 = x["W2"].unsqueeze(0).repeat(dwl.B, 1, 1, 1)
         W0_2 = state2.clone()
 
         def steps():  # noqa: F811

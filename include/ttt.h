@@ -327,9 +327,9 @@ TTT_API ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, co
  *     TTT_CHUNK_NOALLOC_SCRATCH_BYTES (24 MiB: 128 chunks of d = 128) return
  *     TTT_ERR_SCRATCH_LIMIT and launch nothing; use ttt_chunk_fwd with a
  *     caller-allocated workspace for them.
- *   - The first call on a device looks up the buffer's device address on
- *     that device (once per device, with the device current); make that first
- *     call before any stream capture on that device.
+ *   - Every call looks up the buffer's device address on the current device
+ *     (a lookup, not an allocation); the first call on a device also loads
+ *     the module there, so make it before any stream capture on that device.
  *   - All calls share the one buffer. Its contents persist between calls and
  *     are fully overwritten before being read, so nothing needs clearing;
  *     but calls whose GPU work overlaps (different streams, or different host

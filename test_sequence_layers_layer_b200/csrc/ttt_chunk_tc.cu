@@ -18,7 +18,6 @@
 // Q/K/V tiles arrive by TMA with the 128-byte swizzle; accumulators live in
 // tensor memory. W_c enters the apply products as two bf16 terms (hi + lo)
 // so the read-out keeps ~16 significant bits of the fp32 state.
-#include <mutex>
 
 #include "../../include/ttt.h"
 #include "sm100.cuh"
@@ -605,27 +604,17 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_chunk_scratch[TTT_CHUNK_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_chunk_scratch on the current device, looked up once per
-// device with that device current. In host code the symbol is only a handle,
-// never an address a kernel may be given.
+// Device address of g_chunk_scratch on the current device. In host code the
+// symbol is only a handle, never an address a kernel may be given. The lookup
+// allocates nothing and is repeated on every call, so an address is never
+// carried over a device reset or a re-created context.
 void *chunk_scratch_on_current_device() {
-    static std::mutex mu;
-    static void *addr[64];
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_chunk_scratch) != cudaSuccess) {
         cudaGetLastError();
         return nullptr;
     }
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_chunk_scratch) != cudaSuccess) {
-            cudaGetLastError();
-            return nullptr;
-        }
-        addr[dev] = p;
-    }
-    return addr[dev];
+    return p;
 }
 
 }  // namespace

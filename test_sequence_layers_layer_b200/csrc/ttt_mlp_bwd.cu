@@ -63,7 +63,7 @@ __global__ void mlp_bwd_sum_kernel(const float *ws, size_t ws_per_seq, int B, in
 }  // namespace
 
 bool mlp_bwd_supported(int d, int dh, int b) {
-    return (d == 16 || d == 32 || d == 64) && dh == 4 * d && b >= 1 && b <= 16;
+    return (d == 16 || d == 32 || d == 64) && dh == 4 * d && b >= 1 && b <= mlp_bwd_body::kMlpBwdMaxB;
 }
 
 size_t mlp_bwd_workspace_bytes(int B, int H, int T, int d, int b) {

@@ -12,8 +12,8 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU; parity tests of the CUDA path")
     config.addinivalue_line("markers", "slow: full-size workloads")
     config.addinivalue_line(
-        "markers", "late: GPU cases that have not yet passed on a GPU; collected after all the "
-        "others, so that a failure among them (the suite runs with -x) stops none of the rest")
+        "markers", "late: collected after all unmarked tests, so that under -x a failure in one "
+        "of these cases stops none of the others")
 
 
 def pytest_collection_modifyitems(config, items):

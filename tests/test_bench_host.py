@@ -81,7 +81,8 @@ def test_segments_option_is_checked_before_any_gpu_work():
             "chunk_d128_c2048_b4h8_t32768"]
     r = subprocess.run(base + ["--segments", "3"], capture_output=True, text=True, timeout=120)
     assert r.returncode == 2 and "does not split" in r.stderr
-    r = subprocess.run(base[:2] + ["--segments", "2"], capture_output=True, text=True, timeout=120)
+    r = subprocess.run(base[:2] + ["--workload", "linear_ln_d64_b8h12_t2048", "--segments", "2"],
+                       capture_output=True, text=True, timeout=120)
     assert r.returncode == 2 and "large-chunk" in r.stderr
 
 

@@ -26,7 +26,7 @@ def test_linear_decode_loop(dtype):
     x = to_dev(inp)
     Zw, Ww = ttt.linear_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["gamma"], x["beta"],
                             b=1, ln=True)
-    state = x["W1"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    state = x["W1"].unsqueeze(0).repeat(wl.B, 1, 1, 1)
     Z = torch.empty_like(Zw)
     for i in range(wl.T):
         z = torch.empty((wl.B, wl.H, 1, wl.d), dtype=torch.float32, device="cuda")
@@ -50,8 +50,8 @@ def test_mlp_decode_loop():
     x = to_dev(inp)
     Zw, W1w, W2w = ttt.mlp_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["W2"], x["gamma"],
                                x["beta"], b=1)
-    s1 = x["W1"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
-    s2 = x["W2"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    s1 = x["W1"].unsqueeze(0).repeat(wl.B, 1, 1, 1)
+    s2 = x["W2"].unsqueeze(0).repeat(wl.B, 1, 1, 1)
     Z = torch.empty_like(Zw)
     for i in range(wl.T):
         z = torch.empty((wl.B, wl.H, 1, wl.d), dtype=torch.float32, device="cuda")
@@ -79,7 +79,7 @@ def test_decode_kernel_loop(dtype, ln, l2):
     wl = W["linear_ln_d64_b8h12_t2048"].scaled(B=2, H=3, T=24, b=1, dtype=dtype, ln=ln)
     inp = synth.make_inputs(wl)
     x = to_dev(inp)
-    state = x["W1"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    state = x["W1"].unsqueeze(0).repeat(wl.B, 1, 1, 1)
     Z = torch.empty((wl.B, wl.H, wl.T, wl.d), dtype=torch.float32, device="cuda")
     for i in range(wl.T):
         q, k, v = (x[n][:, :, i].contiguous() for n in ("Q", "K", "V"))
@@ -112,8 +112,8 @@ def test_mlp_decode_kernel_loop(dtype):
     wl = W["mlp_ln_d64_dh256_b4h12_t8192"].scaled(B=1, H=2, T=12, b=1, dtype=dtype)
     inp = synth.make_inputs(wl)
     x = to_dev(inp)
-    s1 = x["W1"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
-    s2 = x["W2"].unsqueeze(0).expand(wl.B, -1, -1, -1).contiguous()
+    s1 = x["W1"].unsqueeze(0).repeat(wl.B, 1, 1, 1)
+    s2 = x["W2"].unsqueeze(0).repeat(wl.B, 1, 1, 1)
     Z = torch.empty((wl.B, wl.H, wl.T, wl.d), dtype=torch.float32, device="cuda")
     for i in range(wl.T):
         q, k, v = (x[n][:, :, i].contiguous() for n in ("Q", "K", "V"))
