@@ -80,17 +80,17 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_plan(wl, zb: int = 4):
+def kernel_plan(wl, zb: int = 4, tcgen05_mlp: bool = False):
     """Kernels one library call launches, in launch order:
     (name, source file, arithmetic type, algorithmic bytes/token, FLOPs/token)."""
     e = 2 if wl.dtype == "bf16" else 4
     d = wl.d
     if wl.kind == "chunk" and wl.dtype == "bf16" and d == 128 and wl.b % 128 == 0:
         return [
-            # K, V and eta in; A_c | B_c = K^T [eta K | eta V]
-            ("chunk_gram_kernel", "ttt_chunk_tc.cu", "bf16", 2 * d * e + 4, 4 * d * d),
-            # W_{c+1} = W_c - A_c W_c + B_c: d^3 per chunk; W0 in, W_out out
-            ("chunk_scan_kernel", "ttt_chunk_tc.cu", "f32", 8 * d * d / wl.T, 2 * d ** 3 / wl.b),
+            # K, V and eta in, A_c | B_c = K^T [eta K | eta V]; with the scan
+            # W_{c+1} = W_c - A_c W_c + B_c (d^3 per chunk; W0 in, W_out out)
+            ("chunk_gram_scan_kernel", "ttt_chunk_tc.cu", "bf16", 2 * d * e + 4 + 8 * d * d / wl.T,
+             4 * d * d + 2 * d ** 3 / wl.b),
             # Q in, Z (fp32) out; Z = Q W_c
             ("chunk_apply_kernel", "ttt_chunk_tc.cu", "bf16", d * e + zb * d, 2 * d * d),
         ]
@@ -98,6 +98,9 @@ def kernel_plan(wl, zb: int = 4):
         return [("linear_ln_scan_kernel", "ttt_linear_tc.cu", "bf16", algo_bytes_per_token(wl, zb),
                  algo_flops_per_token(wl))]
     if wl.kind == "mlp" and wl.dtype == "bf16" and d == 64 and wl.dh == 256 and wl.b == 16:
+        if tcgen05_mlp:
+            return [("mlp_umma_scan_kernel", "ttt_mlp_umma.cu", "bf16",
+                     algo_bytes_per_token(wl, zb), algo_flops_per_token(wl))]
         return [("mlp_ln_scan_kernel", "ttt_mlp_tc.cu", "bf16", algo_bytes_per_token(wl, zb),
                  algo_flops_per_token(wl))]
     name = {"linear": "linear_simt_kernel", "mlp": "mlp_simt_kernel",
@@ -208,7 +211,7 @@ def device_tensors(inp, dev):
     return x
 
 
-def make_caller(wl, x, stream, z_bf16=False):
+def make_caller(wl, x, stream, z_bf16=False, tcgen05_mlp=False):
     """Returns (call, outputs) where call() enqueues one library call on `stream`."""
     import torch
     import test_sequence_layers_layer_b200 as ttt
@@ -230,9 +233,11 @@ def make_caller(wl, x, stream, z_bf16=False):
         W1o = torch.empty((B, H, d, wl.dh), dtype=torch.float32, device=dev)
         W2o = torch.empty((B, H, wl.dh, d), dtype=torch.float32, device=dev)
 
+        fn = ttt.ttt_diag_mlp_fwd_tcgen05 if tcgen05_mlp else ttt.ttt_mlp_fwd
+
         def call(x=x):
-            ttt.ttt_mlp_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["W2"], x["gamma"],
-                            x["beta"], Z, W1o, W2o, B, H, T, d, wl.dh, wl.b, dt, ttt.TTT_F_LN | zf, sp)
+            fn(x["Q"], x["K"], x["V"], x["eta"], x["W1"], x["W2"], x["gamma"], x["beta"], Z, W1o,
+               W2o, B, H, T, d, wl.dh, wl.b, dt, ttt.TTT_F_LN | zf, sp)
         return call, (Z, W1o, W2o)
     Wo = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
     need = ttt.ttt_chunk_workspace_bytes(B, H, T, d, wl.b)
@@ -276,20 +281,23 @@ SM_COUNT = 148
 
 def latency_floor(wl, plan, kern_ms_per_call):
     """The sequential chain's cost: each sequence scans ceil(T/b) dependent
-    mini-batch (or chunk) steps, one CTA (a 2-CTA cluster for the TTT-MLP
-    tensor-core scan) per sequence, one CTA per SM. With w waves of sequences
-    per launch the scan kernel's time divided by w * ceil(T/b) is the time of
-    one dependent step. Returns a dict for the bench line."""
+    mini-batch (or chunk) steps, one CTA (a 2-CTA cluster for the warp-level
+    MMA TTT-MLP scan) per sequence, one CTA per SM. With w waves of
+    sequences per launch the scan kernel's time divided by w * ceil(T/b) is
+    the time of one dependent step. Returns a dict for the bench line."""
     idx = next((i for i, p in enumerate(plan) if "scan" in p[0]), len(plan) - 1)
-    name = plan[idx][0]
-    ctas = 2 if name == "mlp_ln_scan_kernel" else 1
+    ctas = 2 if plan[idx][0] == "mlp_ln_scan_kernel" else 1
     nseq = wl.B * wl.H
     concurrent = min(nseq, SM_COUNT // ctas)
     waves = -(-nseq // concurrent)
     steps = -(-wl.T // wl.b)
-    return {"us_per_minibatch_step": kern_ms_per_call[idx] * 1e3 / (waves * steps),
-            "dependent_steps": steps, "concurrent_sequences": concurrent, "waves": waves,
-            "kernel": name}
+    out = {"us_per_minibatch_step": kern_ms_per_call[idx] * 1e3 / (waves * steps),
+           "dependent_steps": steps, "concurrent_sequences": concurrent, "waves": waves,
+           "kernel": plan[idx][0]}
+    if plan[idx][0] == "chunk_gram_scan_kernel":
+        out["note"] = ("the scan shares its launch with the Gram products: an upper bound on "
+                       "one chunk step")
+    return out
 
 
 def cpu_model() -> str:
@@ -316,14 +324,14 @@ def gpu_arm(args, wl, rank, world, keep=None):
     x = device_tensors(inp, dev)
     stream = torch.cuda.Stream(dev)
     zb = 2 if args.z_bf16 else 4
-    call, outs = make_caller(wl, x, stream, args.z_bf16)
+    call, outs = make_caller(wl, x, stream, args.z_bf16, args.mlp_kernel == "tcgen05")
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[dev.index])
 
-    plan = kernel_plan(wl, zb)
+    plan = kernel_plan(wl, zb, args.mlp_kernel == "tcgen05")
     multi = len(plan) > 1
     sampler = ClockSampler(dev)
     sampler.start()
@@ -373,7 +381,7 @@ def gpu_arm(args, wl, rank, world, keep=None):
     # the call, device -> pinned host outputs, every step.
     host_in = {k: v.cpu().pin_memory() for k, v in x.items() if v is not None}
     dev_in = {k: torch.empty_like(v) for k, v in x.items() if v is not None}
-    call_e2e, outs_e2e = make_caller(wl, dev_in, stream, args.z_bf16)
+    call_e2e, outs_e2e = make_caller(wl, dev_in, stream, args.z_bf16, args.mlp_kernel == "tcgen05")
     host_out = [o.cpu().pin_memory() for o in outs_e2e if o is not None]
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = sum(o.numel() * o.element_size() for o in host_out)
@@ -429,7 +437,8 @@ def gpu_arm(args, wl, rank, world, keep=None):
         peak, unit = peaks["bf16_tflops"], "TFLOP/s"
     tflops = algo_flops_per_token(wl) * wl.tokens / (ms_per_step / 1e3) / 1e12
     sha = source_sha(ksrc)
-    wname = wl.name + ("_zbf16" if args.z_bf16 else "")
+    wname = (wl.name + ("_zbf16" if args.z_bf16 else "")
+             + ("_tcgen05" if args.mlp_kernel == "tcgen05" and wl.kind == "mlp" else ""))
     traffic = recorded_traffic(kname, wname, sha)
     clocks = sampler.summary(t0, t1)
     kernels = [{"name": p[0], "ms_per_launch": kern_tot[i] / args.steps,
@@ -929,6 +938,9 @@ def main():
                          "over N batch slices (hostio.linear_fwd_host)")
     ap.add_argument("--segments", type=int, default=0,
                     help="time the large-chunk forward split into N segments per sequence")
+    ap.add_argument("--mlp-kernel", default="default", choices=["default", "tcgen05"],
+                    help="TTT-MLP workload: time the single-issuer tensor-core kernel "
+                         "(ttt_diag_mlp_fwd_tcgen05) instead of ttt_mlp_fwd")
     ap.add_argument("--B", type=int, default=None,
                     help="override the workload's batch size (smaller profiling cases)")
     args = ap.parse_args()

@@ -296,13 +296,15 @@ TTT_API ttt_status ttt_mlp_bwd(const void *Q, const void *K, const void *V, cons
  * gradient descent on the chunk's mean loss.
  * Arguments as ttt_linear_fwd without LayerNorm; `chunk` is the chunk length.
  * workspace: device scratch of at least ttt_chunk_workspace_bytes(...) bytes
- *   (192 KiB per chunk of every sequence when d = 128; 0 for the shapes that
- *   need none, when workspace may be NULL), 256-byte aligned, owned by the
- *   caller; its contents on entry do not matter and are clobbered. Calls that
- *   share a workspace must not overlap on the GPU.
+ *   (192 KiB per chunk of every sequence when d = 128, plus 4 bytes per chunk
+ *   and a counter for the chunks' ready flags, rounded up to 256 bytes; 0 for
+ *   the shapes that need none, when workspace may be NULL), 256-byte aligned,
+ *   owned by the caller; its contents on entry do not matter and are
+ *   clobbered. Calls that share a workspace must not overlap on the GPU.
  * Supported: T % chunk == 0, chunk % 128 == 0; d = 128 with TTT_BF16 runs
- *   on the tensor cores (three launches: per-chunk Gram products, the
- *   sequential affine scan over chunks, and the read-out), d in {64, 128}
+ *   on the tensor cores (a memset of the ready flags and two launches: the
+ *   per-chunk Gram products together with the sequential affine scan over
+ *   chunks, then the read-out), d in {64, 128}
  *   with TTT_FP32, and d = 64, run the fp32 CUDA-core kernel.
  * flags: TTT_F_W0_PER_SEQ, TTT_F_Z_BF16.
  */
@@ -324,7 +326,8 @@ TTT_API ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, co
  * GPU that loads libttt.so holds that buffer until the process exits, and no
  * call of this function allocates or frees anything.
  *   - Limit: problems whose ttt_chunk_workspace_bytes(...) exceeds
- *     TTT_CHUNK_NOALLOC_SCRATCH_BYTES (24 MiB: 128 chunks of d = 128) return
+ *     TTT_CHUNK_NOALLOC_SCRATCH_BYTES (24 MiB + 4 KiB: 128 chunks of d = 128
+ *     with their ready flags) return
  *     TTT_ERR_SCRATCH_LIMIT and launch nothing; use ttt_chunk_fwd with a
  *     caller-allocated workspace for them.
  *   - Every call looks up the buffer's device address on the current device
@@ -337,7 +340,7 @@ TTT_API ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, co
  * Arguments, supported shapes and errors are those of ttt_chunk_fwd, without
  * the workspace pair.
  */
-#define TTT_CHUNK_NOALLOC_SCRATCH_BYTES (24u << 20)
+#define TTT_CHUNK_NOALLOC_SCRATCH_BYTES ((24u << 20) + 4096u)
 TTT_API ttt_status ttt_chunk_fwd_noalloc(const void *Q, const void *K, const void *V,
                                          const float *eta, const float *W0, void *Z,
                                          float *W_out, int B, int H, int T, int d, int chunk,

@@ -25,7 +25,7 @@ extern "C" {
  * D[M][N] (fp32, row-major) = A[M][K] * B[K][N] (bf16, row-major), with A
  * and B staged in the given layouts and one 1-CTA tcgen05 MMA chain over K.
  * Supported: M in {64, 128}; N a multiple of 16 in [16, 256] (multiple of 8
- * for M = 64); K a multiple of 16 in [16, 128]. Device pointers; enqueued on
+ * for M = 64); K a multiple of 16 in [16, 256]. Device pointers; enqueued on
  * `stream`. Returns TTT_ERR_SHAPE / TTT_ERR_ARG for unsupported values.
  */
 TTT_API ttt_status ttt_selftest_umma(int M, int N, int K, int a_layout, int b_layout,
@@ -69,6 +69,38 @@ TTT_API ttt_status ttt_diag_wait_timeout(unsigned limit_us, ttt_stream stream);
  */
 TTT_API ttt_status ttt_diag_kernel_timing(int enable);
 TTT_API int ttt_diag_kernel_times(float *ms, int max);
+
+/*
+ * The TTT-MLP forward of ttt_mlp_fwd ("How to Master Test-Time Training for
+ * LLMs": the hidden state as a multi-layer perceptron; the mini-batch dual
+ * form of "Test-Time Training: Linear Complexity Beyond Attention", Key
+ * Architectural Mechanics part 4) computed by the alternative kernel that
+ * runs every dense product as a tcgen05.mma issued by one thread (operands in
+ * shared memory, fp32 accumulators in tensor memory), instead of the
+ * warp-level MMA kernel ttt_mlp_fwd uses for these shapes. Same arguments,
+ * results within the same tolerance; kept to measure one design against the
+ * other. Supported: TTT_BF16, d = 64, dh = 256, b = 16 (TTT_ERR_SHAPE
+ * otherwise).
+ */
+TTT_API ttt_status ttt_diag_mlp_fwd_tcgen05(const void *Q, const void *K, const void *V,
+                                            const float *eta, const float *W1_0,
+                                            const float *W2_0, const float *ln_gamma,
+                                            const float *ln_beta, void *Z, float *W1_out,
+                                            float *W2_out, int B, int H, int T, int d, int dh,
+                                            int b, ttt_dtype dt, unsigned flags,
+                                            ttt_stream stream);
+
+/*
+ * Cost of issuing tcgen05.mma from one thread: one block issues `count`
+ * back-to-back M x N x 16 bf16 products (M in {64, 128}; N a multiple of 16
+ * in [16, 256], of 8 for M = 64; 1 <= count <= 256) into `nacc` accumulators
+ * in turn (1 <= nacc <= 4), twice, and writes the SM clock cycles of the
+ * second round to cycles[0] (issuing the instructions) and cycles[1] (issue
+ * until their commit's mbarrier completes). cycles: two device int64.
+ * Operands are zero; the products themselves are discarded.
+ */
+TTT_API ttt_status ttt_diag_umma_issue_cycles(int M, int N, int count, int nacc,
+                                              long long *cycles, ttt_stream stream);
 
 #ifdef __cplusplus
 }

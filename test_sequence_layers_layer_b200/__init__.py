@@ -106,6 +106,10 @@ def lib() -> ctypes.CDLL:
         L.ttt_diag_gelu.argtypes = [_P, _P, _P, _I, _P]
         L.ttt_diag_wait_timeout.restype = _I
         L.ttt_diag_wait_timeout.argtypes = [ctypes.c_uint, _P]
+        L.ttt_diag_mlp_fwd_tcgen05.restype = _I
+        L.ttt_diag_mlp_fwd_tcgen05.argtypes = [_P] * 11 + [_I] * 7 + [ctypes.c_uint, _P]
+        L.ttt_diag_umma_issue_cycles.restype = _I
+        L.ttt_diag_umma_issue_cycles.argtypes = [_I] * 4 + [_P, _P]
         _lib = L
     return _lib
 
@@ -231,6 +235,20 @@ def ttt_mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out, 
                            _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z), _ptr(W1_out), _ptr(W2_out),
                            B, H, T, d, dh, b, dt, flags, _stream(stream))
     return _check("ttt_mlp_fwd", rc) if check else rc
+
+
+def ttt_diag_mlp_fwd_tcgen05(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out, B, H,
+                             T, d, dh, b, dt, flags, stream=None, check=True):
+    rc = lib().ttt_diag_mlp_fwd_tcgen05(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(W1_0),
+                                        _ptr(W2_0), _ptr(ln_gamma), _ptr(ln_beta), _ptr(Z),
+                                        _ptr(W1_out), _ptr(W2_out), B, H, T, d, dh, b, dt, flags,
+                                        _stream(stream))
+    return _check("ttt_diag_mlp_fwd_tcgen05", rc) if check else rc
+
+
+def ttt_diag_umma_issue_cycles(M, N, count, nacc, cycles, stream=None, check=True):
+    rc = lib().ttt_diag_umma_issue_cycles(M, N, count, nacc, _ptr(cycles), _stream(stream))
+    return _check("ttt_diag_umma_issue_cycles", rc) if check else rc
 
 
 def ttt_chunk_workspace_bytes(B, H, T, d, chunk) -> int:
@@ -464,8 +482,9 @@ def chunk_bwd(Q, K, V, eta, W0, dZ, dW_out=None, *, chunk, w0_per_seq=False, wor
 
 
 def mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, *, b, w0_per_seq=False, stream=None,
-            want_w=True, z_bf16=False):
-    """TTT-MLP forward. Returns (Z, W1_out, W2_out)."""
+            want_w=True, z_bf16=False, kernel="default"):
+    """TTT-MLP forward. Returns (Z, W1_out, W2_out). kernel="tcgen05" runs the
+    diagnostic single-issuer tensor-core kernel (ttt_diag_mlp_fwd_tcgen05)."""
     import torch
     B, H, T, d = Q.shape
     dh = W1_0.shape[-1]
@@ -473,8 +492,9 @@ def mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, *, b, w0_per_seq=False,
     W1o = torch.empty((B, H, d, dh), dtype=torch.float32, device=Q.device) if want_w else None
     W2o = torch.empty((B, H, dh, d), dtype=torch.float32, device=Q.device) if want_w else None
     flags = TTT_F_LN | (TTT_F_W0_PER_SEQ if w0_per_seq else 0) | (TTT_F_Z_BF16 if z_bf16 else 0)
-    ttt_mlp_fwd(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1o, W2o, B, H, T, d, dh, b,
-                _dtype_code(Q), flags, stream)
+    fn = ttt_diag_mlp_fwd_tcgen05 if kernel == "tcgen05" else ttt_mlp_fwd
+    fn(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1o, W2o, B, H, T, d, dh, b,
+       _dtype_code(Q), flags, stream)
     return Z, W1o, W2o
 
 

@@ -444,3 +444,23 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t cluster_dst, uint3
 
 }  // namespace sm100
 }  // namespace ttt
+
+// ----------------------------------------------------------------- narrow TMEM loads
+namespace ttt {
+namespace sm100 {
+
+// Warp-collective 32-lane x 32-bit load of 8 consecutive columns: thread i
+// receives columns col..col+7 of lane (base lane + i).
+__device__ __forceinline__ void tmem_ld8(uint32_t ta, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(ta));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+}  // namespace sm100
+}  // namespace ttt

@@ -437,11 +437,13 @@ ttt_status ttt_mlp_bwd(const void *Q, const void *K, const void *V, const float 
                                    workspace, cs));
 }
 
-ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float *eta,
+namespace {
+
+// Validation shared by the TTT-MLP forward entry points; fills `a` on success.
+ttt_status mlp_prepare(const void *Q, const void *K, const void *V, const float *eta,
                        const float *W1_0, const float *W2_0, const float *ln_gamma,
-                       const float *ln_beta, void *Z, float *W1_out, float *W2_out, int B,
-                       int H, int T, int d, int dh, int b, ttt_dtype dt, unsigned flags,
-                       ttt_stream stream) {
+                       const float *ln_beta, void *Z, float *W1_out, float *W2_out, int B, int H,
+                       int T, int d, int dh, int b, ttt_dtype dt, unsigned flags, ttt::MlpArgs &a) {
     if (flags & ~(TTT_F_LN | TTT_F_W0_PER_SEQ | TTT_F_Z_BF16)) return TTT_ERR_ARG;
     if (!(flags & TTT_F_LN)) return TTT_ERR_ARG;
     if (!Q || !K || !V || !eta || !W1_0 || !W2_0 || !ln_gamma || !ln_beta || !Z) return TTT_ERR_PTR;
@@ -459,14 +461,44 @@ ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float 
     const void *ptrs[] = {Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out, W2_out};
     st = check_device_ptrs(ptrs, 11);
     if (st != TTT_OK) return st;
+    a = ttt::MlpArgs{Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, static_cast<float *>(Z), W1_out,
+                     W2_out, B, H, T, d, dh, b, dt == TTT_BF16, per_seq,
+                     (flags & TTT_F_Z_BF16) != 0};
+    return TTT_OK;
+}
 
-    MlpArgs a{Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, static_cast<float *>(Z), W1_out, W2_out,
-              B, H, T, d, dh, b, dt == TTT_BF16, per_seq, (flags & TTT_F_Z_BF16) != 0};
+}  // namespace
+
+ttt_status ttt_mlp_fwd(const void *Q, const void *K, const void *V, const float *eta,
+                       const float *W1_0, const float *W2_0, const float *ln_gamma,
+                       const float *ln_beta, void *Z, float *W1_out, float *W2_out, int B,
+                       int H, int T, int d, int dh, int b, ttt_dtype dt, unsigned flags,
+                       ttt_stream stream) {
+    MlpArgs a;
+    const ttt_status st = mlp_prepare(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out,
+                                      W2_out, B, H, T, d, dh, b, dt, flags, a);
+    if (st != TTT_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
     return launched(mlp_tc_supported(d, dh, b, dt == TTT_BF16, (long long)B * H * T)
                         ? launch_mlp_tc(a, cs)
                         : launch_mlp_simt(a, cs));
+}
+
+ttt_status ttt_diag_mlp_fwd_tcgen05(const void *Q, const void *K, const void *V,
+                                    const float *eta, const float *W1_0, const float *W2_0,
+                                    const float *ln_gamma, const float *ln_beta, void *Z,
+                                    float *W1_out, float *W2_out, int B, int H, int T, int d,
+                                    int dh, int b, ttt_dtype dt, unsigned flags,
+                                    ttt_stream stream) {
+    MlpArgs a;
+    const ttt_status st = mlp_prepare(Q, K, V, eta, W1_0, W2_0, ln_gamma, ln_beta, Z, W1_out,
+                                      W2_out, B, H, T, d, dh, b, dt, flags, a);
+    if (st != TTT_OK) return st;
+    if (!mlp_tc_supported(d, dh, b, dt == TTT_BF16, (long long)B * H * T)) return TTT_ERR_SHAPE;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    return launched(launch_mlp_umma(a, cs));
 }
 
 size_t ttt_chunk_workspace_bytes(int B, int H, int T, int d, int chunk) {

@@ -6,13 +6,18 @@
 // chunk c reads out with W_c, then
 //   W_{c+1} = W_c - sum_{s in c} eta_s k_s^T (k_s W_c - v_s)
 //           = W_c - A_c W_c + B_c,   A_c = K_c^T diag(eta) K_c,  B_c = K_c^T diag(eta) V_c.
-// The update is affine in W, so the work splits into three launches:
-//   1. gram:  A_c | B_c for every chunk of every sequence at once (the only
-//             pass over K and V; tcgen05, M = d_in = 128, N = 256, K = tokens);
-//   2. scan:  W_{c+1} = W_c - A_c W_c + B_c, 16 steps per sequence (tcgen05,
-//             M = N = K = 128, hi/lo operands; the state and the update in
-//             fp32), writing each W_c as the ready-made bf16 hi/lo operand image;
-//   3. apply: Z_c = Q_c W_c for every chunk at once (the only pass over Q and
+// The update is affine in W, so the work splits into two launches:
+//   1. gram + scan, one launch with two block roles taken in start order:
+//      gram:  A_c | B_c for every chunk of every sequence (the only pass over
+//             K and V; tcgen05, M = d_in = 128, N = 256, K = tokens), each
+//             chunk published by a ready flag;
+//      scan:  W_{c+1} = W_c - A_c W_c + B_c, 16 steps per sequence, split by
+//             32-column slices of W over 4 blocks (columns evolve
+//             independently; tcgen05, M = 128, N = 32, K = 128, hi/lo
+//             operands; state and update in fp32), each step as soon as its
+//             chunk is published, writing each W_c as the ready-made bf16
+//             hi/lo operand image of the read-out;
+//   2. apply: Z_c = Q_c W_c for every chunk at once (the only pass over Q and
 //             the only write of Z; tcgen05, M = 128 tokens, N = d_out, K = d_in;
 //             W_c arrives by one bulk copy).
 // Q/K/V tiles arrive by TMA with the 128-byte swizzle; accumulators live in
@@ -32,232 +37,270 @@ constexpr int kD = 128;
 constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: math/epilogue
 
 // Workspace per chunk: A_c as a bf16 hi | lo operand image (K-major, 32 KB
-// each) and B_c in fp32 (64 KB; column quad q of row i at float4 q * 128 + i); after all chunks, each W_c as the
-// apply kernel's bf16 hi | lo image (MN-major, 64 KB).
+// each) and B_c in fp32 (64 KB; column quad q of row i at float4 q * 128 + i);
+// after all chunks, each W_c as the apply kernel's bf16 hi | lo image
+// (MN-major, 64 KB); then the ticket counter and the chunks' ready flags.
 constexpr int kImgBytes = kD * kD * 2;            // one bf16 128 x 128 image
 constexpr int kChunkWs = 2 * kImgBytes + kD * kD * 4;
 
 // ---------------------------------------------------------------------------
-// 1. gram: A_c | B_c = (diag(eta) K_c)^T [K_c | V_c]
+// 1 + 2. gram and scan in one launch. Each block takes a ticket from a
+// counter in the workspace (tickets follow the order in which blocks start)
+// and from it a role:
+//   tickets [0, n):  gram of one chunk, chunks in chunk-major order (chunk 0 of
+//     every sequence first): A_c | B_c = (diag(eta) K_c)^T [K_c | V_c], then a
+//     ready flag for the chunk;
+//   tickets [n, n + 4 S): scan of one 32-column slice of one sequence's
+//     weight: W_{c+1}[:, j] = W_c[:, j] - A_c W_c[:, j] + B_c[:, j] (columns of
+//     W evolve independently), waiting on each chunk's ready flag.
+// A scan block only ever waits on gram blocks; every gram block started
+// before any scan block (smaller ticket) and waits on nothing, so the wait
+// always ends. The scans run while the last grams stream, instead of after
+// them.
 constexpr int kGramRows = 32;                    // tokens per pipeline stage
 constexpr int kGramStages = 4;
 constexpr int kGramBox = kGramRows * 128;        // one 64-column box of a stage (4 KB)
 constexpr int kGramStageBytes = 6 * kGramBox;    // K (2 boxes) | V (2) | eta*K (2)
 constexpr size_t kGramSmem = 1024 + kGramStages * kGramStageBytes;  // 97 KB: two blocks per SM
+constexpr int kSlice = 64, kSlices = kD / kSlice;  // scan: output columns per block
+constexpr int kSliceImg = 2 * kSlice * kD * 2;     // [W hi | W lo] slice image [128][128] bf16: 32 KB
+static_assert(2 * kImgBytes / 2 + kSliceImg + 1024 <= (int)kGramSmem, "scan role fits the gram's smem");
 
-struct GramArgs {
+// Ready flags and the ticket counter sit after the per-chunk workspace.
+__host__ __device__ constexpr size_t sync_offset(size_t n) { return n * ((size_t)kChunkWs + 65536); }
+__host__ __device__ constexpr size_t sync_bytes(size_t n) { return ((n + 1) * 4 + 255) / 256 * 256; }
+
+struct GramScanArgs {
     const float *eta;
-    float *AB;  // [chunks][kChunkWs bytes]: A_c hi | A_c lo | B_c
-    int chunk;
-    int *status;
-};
-
-__global__ void __launch_bounds__(kThreads, 2)
-    chunk_gram_kernel(const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, GramArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t full[kGramStages], conv[kGramStages], empty[kGramStages], done, drain;
-    __shared__ uint32_t tmem_base;
-    __shared__ int abort_flag;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = blockIdx.x;
-    const long row0 = (long)g * a.chunk;  // first token row of this chunk in [B*H*T][d]
-    const int nst = a.chunk / kGramRows;
-
-    if (threadIdx.x == 0) {
-        abort_flag = 0;
-        for (int s = 0; s < kGramStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&conv[s], 128);
-            mbar_init(&empty[s], 1);
-        }
-        mbar_init(&done, 1);
-        mbar_init(&drain, 1);
-        fence_mbar_init();
-    }
-    if (warp == 1) tmem_alloc(&tmem_base, 256);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tm = tmem_base;
-    int issued = 0;
-
-    if (warp == 0 && lane == 0) {
-        // TMA producer: K rows and V rows of each stage, two 64-column boxes each.
-        for (int r = 0; r < nst; ++r) {
-            const int s = r % kGramStages;
-            if (r >= kGramStages &&
-                !mbar_wait(&empty[s], ((r / kGramStages) - 1) & 1, &abort_flag, a.status, 11))
-                break;
-            uint8_t *st = smem + s * kGramStageBytes;
-            const int y = (int)(row0 + (long)r * kGramRows);
-            mbar_arrive_expect_tx(&full[s], 4 * kGramBox);
-            tma_load_2d(st, &tmK, 0, y, &full[s]);
-            tma_load_2d(st + kGramBox, &tmK, 64, y, &full[s]);
-            tma_load_2d(st + 2 * kGramBox, &tmV, 0, y, &full[s]);
-            tma_load_2d(st + 3 * kGramBox, &tmV, 64, y, &full[s]);
-            issued = r + 1;
-        }
-    } else if (warp == 1 && lane == 0) {
-        // MMA issuer: D[d_in][0:128) += (eta K)^T K, D[d_in][128:256) += (eta K)^T V.
-        const uint32_t idesc = make_idesc_bf16(128, 256, true, true);
-        for (int r = 0; r < nst; ++r) {
-            const int s = r % kGramStages;
-            if (!mbar_wait(&conv[s], (r / kGramStages) & 1, &abort_flag, a.status, 12)) break;
-            tc_fence_after();
-            const uint32_t ab = smem_u32(smem + s * kGramStageBytes);
-#pragma unroll
-            for (int k = 0; k < kGramRows / 16; ++k) {
-                const uint64_t ad = make_sdesc(ab + 4 * kGramBox + k * 2048, kGramBox, 1024, kSw128);
-                const uint64_t bd = make_sdesc(ab + k * 2048, kGramBox, 1024, kSw128);
-                mma_bf16(tm, ad, bd, idesc, (r | k) != 0);
-            }
-            mma_commit(&empty[s]);
-        }
-        mma_commit(&done);
-    } else if (warp >= 2) {
-        // Scale K's rows by eta into the A operand's buffer (K and V stay raw
-        // as the B operand). Swizzling permutes 16-byte chunks inside a
-        // 128-byte row only, so a chunk's row (token) is offset / 128.
-        const int c = threadIdx.x - 64;
-        constexpr int kChunks = 2 * kGramBox / 16;  // 16-byte chunks of K per stage
-        for (int r = 0; r < nst; ++r) {
-            const int s = r % kGramStages;
-            // This thread's eta values for the stage, loaded before the wait.
-            float ev[kChunks / 128];
-#pragma unroll
-            for (int i = 0; i < kChunks / 128; ++i) {
-                const int o = (c + 128 * i) * 16;
-                ev[i] = a.eta[row0 + (long)r * kGramRows + ((o % kGramBox) >> 7)];
-            }
-            if (!mbar_wait(&full[s], (r / kGramStages) & 1, &abort_flag, a.status, 13)) break;
-            uint8_t *st = smem + s * kGramStageBytes;
-#pragma unroll
-            for (int i = 0; i < kChunks / 128; ++i) {
-                const int o = (c + 128 * i) * 16;
-                const float e = ev[i];
-                const uint4 v = *reinterpret_cast<const uint4 *>(st + o);
-                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
-                uint4 out;
-                __nv_bfloat162 *ho = reinterpret_cast<__nv_bfloat162 *>(&out);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = __bfloat1622float2(h[i]);
-                    ho[i] = __floats2bfloat162_rn(f.x * e, f.y * e);
-                }
-                *reinterpret_cast<uint4 *>(st + 4 * kGramBox + o) = out;
-            }
-            fence_async_smem();
-            mbar_arrive(&conv[s]);
-        }
-        // Epilogue: lanes are d_in rows i. A_c goes out as the scan's bf16
-        // hi/lo operand image (K-major, 128-byte swizzle: row i = 128 bytes
-        // per 64 columns j), B_c as fp32 rows. (__all_sync reconverges the
-        // warp for the warp-collective TMEM loads.)
-        if (__all_sync(0xffffffffu, mbar_wait(&done, 0, &abort_flag, a.status, 14))) {
-            tc_fence_after();
-            const int sp = warp & 3;
-            const int row = 32 * sp + lane;
-            uint8_t *blk = reinterpret_cast<uint8_t *>(a.AB) + (size_t)g * kChunkWs;
-            float4 *bdst = reinterpret_cast<float4 *>(blk + 2 * kImgBytes);
-            for (int q = 0; q < 16; ++q) {
-                float v[16];
-                tmem_ld16(taddr(tm, 32 * sp, 16 * q), v);
-                tmem_ld_wait();
-                if (q < 8) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint4 hi, lo;
-                        __nv_bfloat16 *hb = reinterpret_cast<__nv_bfloat16 *>(&hi);
-                        __nv_bfloat16 *lb = reinterpret_cast<__nv_bfloat16 *>(&lo);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) split_bf16(v[8 * h + e], hb[e], lb[e]);
-                        const uint32_t off = off_kmajor_sw128(row, 16 * q + 8 * h, kD);
-                        *reinterpret_cast<uint4 *>(blk + off) = hi;
-                        *reinterpret_cast<uint4 *>(blk + kImgBytes + off) = lo;
-                    }
-                } else {  // B_c: column quad q4 of row i at float4 q4 * 128 + i
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        bdst[(4 * (q - 8) + i) * kD + row] =
-                            make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                }
-            }
-        }
-    }
-    // Teardown: after an abort, let this block's own copies and MMAs land
-    // before the shared memory and tensor memory are released.
-    if (abort_flag) {
-        if (warp == 0 && lane == 0)
-            for (int r = issued - kGramStages < 0 ? 0 : issued - kGramStages; r < issued; ++r)
-                mbar_drain(&full[r % kGramStages], (r / kGramStages) & 1);
-        if (warp == 1 && lane == 0) {
-            mma_commit(&drain);
-            mbar_drain(&drain, 0);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) tmem_dealloc(tm, 256);
-}
-
-// ---------------------------------------------------------------------------
-// 2. scan: W_{c+1} = W_c - A_c W_c + B_c, one block per sequence, on the
-// tensor cores. The fp32 state W lives in the registers of 8 epilogue warps
-// (row i = TMEM lane, 64 columns each); per chunk the MMA thread forms
-// D = A_c W_c from the bf16 hi/lo images of A_c (written by the gram kernel,
-// brought in by bulk copy, double-buffered) and of W_c (in shared memory):
-// A_hi W_hi + A_hi W_lo + A_lo W_hi, M = N = 128, K = 128, fp32 in TMEM. The
-// epilogue adds W_c + B_c - D in fp32 (B_c read from global ahead of time),
-// rewrites the W image for the next chunk and bulk-stores it to global as the
-// apply kernel's operand for that chunk.
-constexpr int kScanThreads = 320;  // warp 0: A loads, warp 1: MMA + TMEM, warps 2-9: epilogue
-constexpr size_t kScanSmem = 1024 + 2 * (size_t)kImgBytes /* W */ + 4 * (size_t)kImgBytes /* A x2 */;
-
-struct ScanArgs {
-    const uint8_t *AB;  // per chunk: A_c hi | lo image, B_c fp32
+    uint8_t *ws;        // per chunk: A_c hi | lo image, B_c fp32; then W_c images; then sync
     const float *W0;
-    uint8_t *Wimg;      // [chunks][hi 32 KB | lo 32 KB]: MN-major, 128-byte swizzle
     float *W_out;
-    int H, chunks_per_seq;
+    int chunk, H, nseq, cps;
     bool w0_per_seq;
     int *status;
 };
 
-__device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
-                 "r"(smem_u32(ssrc)), "r"(bytes)
-                 : "memory");
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-__global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(ScanArgs a) {
-    extern __shared__ uint8_t scan_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(scan_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sW = smem;                  // W image: hi | lo (MN-major)
-    uint8_t *sA = smem + 2 * kImgBytes;  // A images: [2 buffers][hi | lo] (K-major)
-    __shared__ uint64_t aready[2], afree[2], dfull, wready, drain;
-    __shared__ uint32_t tmem_base;
-    __shared__ int abort_flag;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int seq = blockIdx.x, cps = a.chunks_per_seq;
-    const size_t g0 = (size_t)seq * cps;
-
-    if (threadIdx.x == 0) {
-        abort_flag = 0;
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&aready[b], 1);
-            mbar_init(&afree[b], 1);
+// Waits (bounded) until *flag != 0. On timeout sets *abort and the status.
+__device__ bool wait_flag(const int *flag, volatile int *abort, int *status, int code) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 0;; ++i) {
+        if (ld_acquire(flag)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicExch(status, code);
+            return false;
         }
-        mbar_init(&dfull, 1);
-        mbar_init(&wready, 1);
-        mbar_init(&drain, 1);
+        __nanosleep(i < 16 ? 64 : 512);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+    chunk_gram_scan_kernel(const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, GramScanArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bars[3 * kGramStages + 2];
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag, ticket;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = a.nseq * a.cps;
+    int *sync = reinterpret_cast<int *>(a.ws + sync_offset(n));  // [0]: ticket counter, [1 + g]: flags
+    if (threadIdx.x == 0) {
+        ticket = atomicAdd(sync, 1);
+        abort_flag = 0;
+    }
+    __syncthreads();
+    const int tk = ticket;
+    const bool gram = tk < n;
+    const uint32_t ncols = 256;  // the gram role's accumulator
+    uint64_t *drain = &bars[3 * kGramStages + 1];
+
+    if (gram) {
+        // ---- gram of chunk c of sequence s (chunk-major ticket order)
+        const int c = tk / a.nseq, s = tk % a.nseq, g = s * a.cps + c;
+        uint64_t *full = bars, *conv = bars + kGramStages, *empty = bars + 2 * kGramStages;
+        uint64_t *done = &bars[3 * kGramStages];
+        const long row0 = (long)g * a.chunk;  // first token row of this chunk in [B*H*T][d]
+        const int nst = a.chunk / kGramRows;
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < kGramStages; ++i) {
+                mbar_init(&full[i], 1);
+                mbar_init(&conv[i], 128);
+                mbar_init(&empty[i], 1);
+            }
+            mbar_init(done, 1);
+            mbar_init(drain, 1);
+            fence_mbar_init();
+        }
+        if (warp == 1) tmem_alloc(&tmem_base, ncols);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        const uint32_t tm = tmem_base;
+        int issued = 0;
+        if (warp == 0 && lane == 0) {
+            // TMA producer: K rows and V rows of each stage, two 64-column boxes each.
+            for (int r = 0; r < nst; ++r) {
+                const int st = r % kGramStages;
+                if (r >= kGramStages &&
+                    !mbar_wait(&empty[st], ((r / kGramStages) - 1) & 1, &abort_flag, a.status, 11))
+                    break;
+                uint8_t *sb = smem + st * kGramStageBytes;
+                const int y = (int)(row0 + (long)r * kGramRows);
+                mbar_arrive_expect_tx(&full[st], 4 * kGramBox);
+                tma_load_2d(sb, &tmK, 0, y, &full[st]);
+                tma_load_2d(sb + kGramBox, &tmK, 64, y, &full[st]);
+                tma_load_2d(sb + 2 * kGramBox, &tmV, 0, y, &full[st]);
+                tma_load_2d(sb + 3 * kGramBox, &tmV, 64, y, &full[st]);
+                issued = r + 1;
+            }
+        } else if (warp == 1 && lane == 0) {
+            // MMA issuer: D[d_in][0:128) += (eta K)^T K, D[d_in][128:256) += (eta K)^T V.
+            const uint32_t idesc = make_idesc_bf16(128, 256, true, true);
+            for (int r = 0; r < nst; ++r) {
+                const int st = r % kGramStages;
+                if (!mbar_wait(&conv[st], (r / kGramStages) & 1, &abort_flag, a.status, 12)) break;
+                tc_fence_after();
+                const uint32_t ab = smem_u32(smem + st * kGramStageBytes);
+#pragma unroll
+                for (int k = 0; k < kGramRows / 16; ++k) {
+                    const uint64_t ad = make_sdesc(ab + 4 * kGramBox + k * 2048, kGramBox, 1024, kSw128);
+                    const uint64_t bd = make_sdesc(ab + k * 2048, kGramBox, 1024, kSw128);
+                    mma_bf16(tm, ad, bd, idesc, (r | k) != 0);
+                }
+                mma_commit(&empty[st]);
+            }
+            mma_commit(done);
+        } else if (warp >= 2) {
+            // Scale K's rows by eta into the A operand's buffer (K and V stay raw
+            // as the B operand). Swizzling permutes 16-byte chunks inside a
+            // 128-byte row only, so a chunk's row (token) is offset / 128.
+            const int t = threadIdx.x - 64;
+            constexpr int kChunks = 2 * kGramBox / 16;  // 16-byte chunks of K per stage
+            for (int r = 0; r < nst; ++r) {
+                const int st = r % kGramStages;
+                // This thread's eta values for the stage, loaded before the wait.
+                float ev[kChunks / 128];
+#pragma unroll
+                for (int i = 0; i < kChunks / 128; ++i) {
+                    const int o = (t + 128 * i) * 16;
+                    ev[i] = a.eta[row0 + (long)r * kGramRows + ((o % kGramBox) >> 7)];
+                }
+                if (!mbar_wait(&full[st], (r / kGramStages) & 1, &abort_flag, a.status, 13)) break;
+                uint8_t *sb = smem + st * kGramStageBytes;
+#pragma unroll
+                for (int i = 0; i < kChunks / 128; ++i) {
+                    const int o = (t + 128 * i) * 16;
+                    const float e = ev[i];
+                    const uint4 v = *reinterpret_cast<const uint4 *>(sb + o);
+                    const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&v);
+                    uint4 out;
+                    __nv_bfloat162 *ho = reinterpret_cast<__nv_bfloat162 *>(&out);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float2 f = __bfloat1622float2(hv[q]);
+                        ho[q] = __floats2bfloat162_rn(f.x * e, f.y * e);
+                    }
+                    *reinterpret_cast<uint4 *>(sb + 4 * kGramBox + o) = out;
+                }
+                fence_async_smem();
+                mbar_arrive(&conv[st]);
+            }
+            // Epilogue: lanes are d_in rows i. A_c goes out as the scan's bf16
+            // hi/lo operand image (K-major, 128-byte swizzle: row i = 128 bytes
+            // per 64 columns j), B_c as fp32 rows. (__all_sync reconverges the
+            // warp for the warp-collective TMEM loads.)
+            if (__all_sync(0xffffffffu, mbar_wait(done, 0, &abort_flag, a.status, 14))) {
+                tc_fence_after();
+                const int sp = warp & 3;
+                const int row = 32 * sp + lane;
+                uint8_t *blk = a.ws + (size_t)g * kChunkWs;
+                float4 *bdst = reinterpret_cast<float4 *>(blk + 2 * kImgBytes);
+                for (int q = 0; q < 16; ++q) {
+                    float v[16];
+                    tmem_ld16(taddr(tm, 32 * sp, 16 * q), v);
+                    tmem_ld_wait();
+                    if (q < 8) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint4 hi, lo;
+                            __nv_bfloat16 *hb = reinterpret_cast<__nv_bfloat16 *>(&hi);
+                            __nv_bfloat16 *lb = reinterpret_cast<__nv_bfloat16 *>(&lo);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) split_bf16(v[8 * h + e], hb[e], lb[e]);
+                            const uint32_t off = off_kmajor_sw128(row, 16 * q + 8 * h, kD);
+                            *reinterpret_cast<uint4 *>(blk + off) = hi;
+                            *reinterpret_cast<uint4 *>(blk + kImgBytes + off) = lo;
+                        }
+                    } else {  // B_c: column quad q4 of row i at float4 q4 * 128 + i
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            bdst[(4 * (q - 8) + i) * kD + row] =
+                                make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    }
+                }
+                __threadfence();  // ordered before the chunk's ready flag
+            }
+        }
+        // Teardown: after an abort, let this block's own copies and MMAs land
+        // before the shared memory and tensor memory are released.
+        if (abort_flag) {
+            if (warp == 0 && lane == 0)
+                for (int r = issued - kGramStages < 0 ? 0 : issued - kGramStages; r < issued; ++r)
+                    mbar_drain(&full[r % kGramStages], (r / kGramStages) & 1);
+            if (warp == 1 && lane == 0) {
+                mma_commit(drain);
+                mbar_drain(drain, 0);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        // A_c and B_c are written: publish the chunk (release, device scope).
+        if (threadIdx.x == 0 && !abort_flag) {
+            __threadfence();
+            atomicExch(sync + 1 + g, 1);
+        }
+        if (warp == 1) tmem_dealloc(tm, ncols);
+        return;
+    }
+
+    // ---- scan of columns [64 r, 64 r + 64) of sequence s, on the tensor
+    // cores. One product per chunk, D = A_c [W_c,hi | W_c,lo] (M = 128 rows
+    // i, N = 128: the slice's hi and lo terms side by side, K = 128), from
+    // the bf16 image of A_c (its hi term; A_c ~ I / chunk-scale, so its lo
+    // term moves W by ~2^-9 of the ~1% step) and the slice's image in shared
+    // memory (K-major: rows 0-63 W_hi^T, rows 64-127 W_lo^T). A_c and the
+    // slice of B_c arrive by bulk copy as soon as the chunk is published and
+    // their previous readers are done, so they land while the previous
+    // chunk's epilogue or this chunk's product runs. The fp32 state is in
+    // the registers of 4 epilogue warps (row i = TMEM lane, 64 columns); they
+    // form W_c + B_c - (D_hi + D_lo) and write W_c's columns into the
+    // read-out's operand image of chunk c in the workspace.
+    const int si = tk - n, s = si / kSlices, r = si % kSlices, j0 = kSlice * r;
+    const int cps = a.cps;
+    const size_t g0 = (size_t)s * cps;
+    uint8_t *sA = smem;                   // A_c hi (K-major, 32 KB)
+    uint8_t *sB = smem + kImgBytes;       // B_c columns j0.. (quad q of row i at float4 q * 128 + i)
+    uint8_t *sWs = smem + 2 * kImgBytes;  // slice image: 2 column blocks of 16 KB
+    uint64_t *aready = bars, *bready = bars + 1, *afree = bars + 2, *bfree = bars + 3,
+             *dfull = bars + 4, *wready = bars + 5;
+    uint8_t *Wimg = a.ws + (size_t)n * kChunkWs;
+    if (threadIdx.x == 0) {
+        mbar_init(aready, 1);
+        mbar_init(bready, 1);
+        mbar_init(afree, 1);
+        mbar_init(bfree, 4);  // one arrival per epilogue warp
+        mbar_init(dfull, 1);
+        mbar_init(wready, 1);
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(&tmem_base, 128);
@@ -268,130 +311,142 @@ __global__ void __launch_bounds__(kScanThreads, 1) chunk_scan_kernel(ScanArgs a)
     int issued = 0;
 
     if (warp == 0 && lane == 0) {
-        // A_c images, two chunks ahead of nothing: buffer c & 1 is reused once
-        // the MMAs of chunk c - 2 have completed.
+        // A_c once chunk c's gram is published and the product of chunk
+        // c - 1 is done with the buffer; B_c once the epilogue of c - 1 has
+        // read the previous one.
         for (int c = 0; c < cps; ++c) {
-            const int b = c & 1;
-            if (c >= 2 && !mbar_wait(&afree[b], ((c >> 1) - 1) & 1, &abort_flag, a.status, 16)) break;
-            mbar_arrive_expect_tx(&aready[b], 2 * kImgBytes);
-            bulk_load(sA + b * 2 * kImgBytes, a.AB + (g0 + c) * kChunkWs, 2 * kImgBytes, &aready[b]);
-            issued = c + 1;
+            if (!wait_flag(sync + 1 + g0 + c, &abort_flag, a.status, 15)) break;
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            const uint8_t *blk = a.ws + (g0 + c) * kChunkWs;
+            if (c >= 1 && !mbar_wait(afree, (c - 1) & 1, &abort_flag, a.status, 16)) break;
+            mbar_arrive_expect_tx(aready, kImgBytes);
+            bulk_load(sA, blk, kImgBytes, aready);
+            issued = 2 * c + 1;
+            if (c >= 1 && !mbar_wait(bfree, (c - 1) & 1, &abort_flag, a.status, 16)) break;
+            mbar_arrive_expect_tx(bready, kImgBytes);
+            bulk_load(sB, blk + 2 * kImgBytes + (size_t)j0 * kD * 4, kImgBytes, bready);
+            issued = 2 * c + 2;
         }
     } else if (warp == 1 && lane == 0) {
-        const uint32_t idesc = make_idesc_bf16(128, 128, false, true);
-        const uint32_t wb = smem_u32(sW);
+        const uint32_t idesc = make_idesc_bf16(128, 2 * kSlice, false, false);
+        const uint32_t wb = smem_u32(sWs);
+        const uint32_t ab = smem_u32(sA);
         for (int c = 0; c < cps; ++c) {
-            const int b = c & 1;
-            if (!mbar_wait(&aready[b], (c >> 1) & 1, &abort_flag, a.status, 17)) break;
-            if (!mbar_wait(&wready, c & 1, &abort_flag, a.status, 18)) break;
+            if (!mbar_wait(aready, c & 1, &abort_flag, a.status, 17)) break;
+            if (!mbar_wait(wready, c & 1, &abort_flag, a.status, 18)) break;
             tc_fence_after();
-            const uint32_t ab = smem_u32(sA + b * 2 * kImgBytes);
-            // (A, W) term pairs: hi hi, hi lo, lo hi
-            const uint32_t aoff[3] = {0, 0, (uint32_t)kImgBytes}, woff[3] = {0, (uint32_t)kImgBytes, 0};
 #pragma unroll
-            for (int p = 0; p < 3; ++p)
-#pragma unroll
-                for (int k = 0; k < kD / 16; ++k) {
-                    const int k0 = 16 * k;
-                    const uint64_t ad = make_sdesc(ab + aoff[p] + (k0 >> 6) * 16384 + (k0 & 63) * 2, 16, 1024, kSw128);
-                    const uint64_t bd = make_sdesc(wb + woff[p] + (k0 >> 3) * 1024, 16384, 1024, kSw128);
-                    mma_bf16(tm, ad, bd, idesc, (p | k) != 0);
-                }
-            mma_commit(&afree[b]);
-            mma_commit(&dfull);
+            for (int k = 0; k < kD / 16; ++k) {
+                const int k0 = 16 * k;
+                const uint32_t o = (uint32_t)((k0 >> 6) * 16384 + (k0 & 63) * 2);
+                mma_bf16(tm, make_sdesc(ab + o, 16, 1024, kSw128), make_sdesc(wb + o, 16, 1024, kSw128),
+                         idesc, k != 0);
+            }
+            mma_commit(afree);
+            mma_commit(dfull);
         }
     } else if (warp >= 2) {
-        // Epilogue: row i = 32 (warp & 3) + lane, columns 64 half .. +63.
-        const int sp = warp & 3, half = (warp - 2) >> 2;
-        const int row = 32 * sp + lane, col0 = 64 * half;
-        const bool leader = warp == 2 && lane == 0;
-        const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? seq : seq % a.H) * kD * kD;
-        float w[64];
+        // Epilogue: row i = 32 (warp & 3) + lane, columns j0 .. j0 + 63.
+        const int sp = warp & 3, row = 32 * sp + lane;
+        const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? s : s % a.H) * kD * kD;
+        float w[kSlice];
 #pragma unroll
-        for (int j4 = 0; j4 < 16; ++j4) {
-            const float4 u = *reinterpret_cast<const float4 *>(W0 + (size_t)row * kD + col0 + 4 * j4);
-            w[4 * j4] = u.x;
-            w[4 * j4 + 1] = u.y;
-            w[4 * j4 + 2] = u.z;
-            w[4 * j4 + 3] = u.w;
+        for (int q = 0; q < kSlice / 4; ++q) {
+            const float4 u = *reinterpret_cast<const float4 *>(W0 + (size_t)row * kD + j0 + 4 * q);
+            w[4 * q] = u.x;
+            w[4 * q + 1] = u.y;
+            w[4 * q + 2] = u.z;
+            w[4 * q + 3] = u.w;
         }
-        // Write this thread's 64 values of W as its row of the MN-major image
-        // (k = row, 64-column atom = half): 8 chunks of 8 bf16, hi and lo.
-        auto emit = [&]() {
+        // This thread's column i of the slice image (rows n: W_hi^T then
+        // W_lo^T; 128-byte swizzle, 16 KB per 64 values of i) and row i of
+        // chunk c's read-out image (MN-major [i][j], 16 KB per 64 columns j).
+        auto emit = [&](int c) {
+            const uint32_t cb = (uint32_t)((row >> 6) * 16384 + (row & 7) * 2);
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
+            for (int jj = 0; jj < kSlice; ++jj) {
+                __nv_bfloat16 hb, lb;
+                split_bf16(w[jj], hb, lb);
+                const int nh = jj, nl = kSlice + jj;
+                *reinterpret_cast<__nv_bfloat16 *>(sWs + cb + (nh >> 3) * 1024 + (nh & 7) * 128 +
+                                                   ((((row & 63) >> 3) ^ (nh & 7)) << 4)) = hb;
+                *reinterpret_cast<__nv_bfloat16 *>(sWs + cb + (nl >> 3) * 1024 + (nl & 7) * 128 +
+                                                   ((((row & 63) >> 3) ^ (nl & 7)) << 4)) = lb;
+            }
+            uint8_t *img = Wimg + (g0 + c) * 65536;
+#pragma unroll
+            for (int h8 = 0; h8 < kSlice / 8; ++h8) {
                 uint4 hi, lo;
                 __nv_bfloat16 *hb = reinterpret_cast<__nv_bfloat16 *>(&hi);
                 __nv_bfloat16 *lb = reinterpret_cast<__nv_bfloat16 *>(&lo);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) split_bf16(w[8 * ch + e], hb[e], lb[e]);
-                const uint32_t off = off_mnmajor_sw128(row, col0 + 8 * ch, kD);
-                *reinterpret_cast<uint4 *>(sW + off) = hi;
-                *reinterpret_cast<uint4 *>(sW + kImgBytes + off) = lo;
+                for (int e = 0; e < 8; ++e) split_bf16(w[8 * h8 + e], hb[e], lb[e]);
+                const uint32_t off = off_mnmajor_sw128(row, j0 + 8 * h8, kD);
+                *reinterpret_cast<uint4 *>(img + off) = hi;
+                *reinterpret_cast<uint4 *>(img + kImgBytes + off) = lo;
             }
             fence_async_smem();
         };
-        // image of W_c -> global (apply's operand for chunk c); W ready for the MMA
-        auto publish = [&](int c) {
-            if (leader) {
-                bulk_store(a.Wimg + (g0 + c) * 65536, sW, 2 * kImgBytes);
-                bulk_commit();
-                mbar_arrive(&wready);
-            }
-        };
-        emit();
-        bool ok = !named_bar_or(1, 256, false);
-        if (ok) publish(0);
+        emit(0);
+        bool ok = !named_bar_or(1, 128, false);
+        if (ok && warp == 2 && lane == 0) mbar_arrive(wready);
         for (int c = 0; ok && c < cps; ++c) {
-            // B_c row of this thread, read ahead of the product
-            // (column quad q4 of row i at float4 q4 * 128 + i: a warp reads 512
-            // contiguous bytes per load)
-            const float4 *Bc = reinterpret_cast<const float4 *>(a.AB + (g0 + c) * kChunkWs + 2 * kImgBytes);
-            float bv[64];
-#pragma unroll
-            for (int j4 = 0; j4 < 16; ++j4) {
-                const float4 u = Bc[(col0 / 4 + j4) * kD + row];
-                bv[4 * j4] = u.x;
-                bv[4 * j4 + 1] = u.y;
-                bv[4 * j4 + 2] = u.z;
-                bv[4 * j4 + 3] = u.w;
+            bool got = mbar_wait(bready, c & 1, &abort_flag, a.status, 19);
+            got = got && mbar_wait(dfull, c & 1, &abort_flag, a.status, 20);
+            if (named_bar_or(1, 128, !__all_sync(0xffffffffu, got))) {
+                ok = false;
+                break;
             }
-            bool got = mbar_wait(&dfull, c & 1, &abort_flag, a.status, 19);
-            if (leader) bulk_wait_read();  // the image's last store has read it
-            // every epilogue warp agrees before anyone moves on
-            if (named_bar_or(1, 256, !__all_sync(0xffffffffu, got))) break;
             tc_fence_after();
+            const float4 *Bc = reinterpret_cast<const float4 *>(sB);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float v[16];
-                tmem_ld16(taddr(tm, 32 * sp, col0 + 16 * q), v);
+            for (int q = 0; q < kSlice / 16; ++q) {
+                float dh[16], dl[16];
+                tmem_ld16(taddr(tm, 32 * sp, 16 * q), dh);
+                tmem_ld16(taddr(tm, 32 * sp, kSlice + 16 * q), dl);
+                float bv[16];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 f = Bc[(4 * q + u) * kD + row];
+                    bv[4 * u] = f.x;
+                    bv[4 * u + 1] = f.y;
+                    bv[4 * u + 2] = f.z;
+                    bv[4 * u + 3] = f.w;
+                }
                 tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) w[16 * q + e] = (w[16 * q + e] + bv[16 * q + e]) - v[e];
+                for (int e = 0; e < 16; ++e)
+                    w[16 * q + e] = (w[16 * q + e] + bv[e]) - (dh[e] + dl[e]);
             }
             tc_fence_before();
-            if (c + 1 < cps) emit();
-            if (named_bar_or(1, 256, false)) break;
-            if (c + 1 < cps) publish(c + 1);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bfree);  // this warp has read B_c
+            if (c + 1 < cps) emit(c + 1);
+            if (named_bar_or(1, 128, false)) {
+                ok = false;
+                break;
+            }
+            if (c + 1 < cps && warp == 2 && lane == 0) mbar_arrive(wready);
         }
-        if (leader) bulk_wait_all();
         if (ok && !abort_flag && a.W_out) {
-            float *o = a.W_out + (size_t)seq * kD * kD + (size_t)row * kD + col0;
+            float *o = a.W_out + (size_t)s * kD * kD + (size_t)row * kD + j0;
 #pragma unroll
-            for (int j4 = 0; j4 < 16; ++j4)
-                *reinterpret_cast<float4 *>(o + 4 * j4) =
-                    make_float4(w[4 * j4], w[4 * j4 + 1], w[4 * j4 + 2], w[4 * j4 + 3]);
+            for (int q = 0; q < kSlice / 4; ++q)
+                *reinterpret_cast<float4 *>(o + 4 * q) =
+                    make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
     }
     // Teardown: after an abort, let this block's own copies and MMAs land
     // before the shared memory and tensor memory are released.
     if (abort_flag) {
-        if (warp == 0 && lane == 0)
-            for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
-                mbar_drain(&aready[c & 1], (c >> 1) & 1);
+        if (warp == 0 && lane == 0 && issued > 0) {
+            const int c = (issued - 1) / 2;  // the last chunk whose copies were issued
+            mbar_drain(aready, c & 1);
+            if (issued % 2 == 0) mbar_drain(bready, c & 1);
+        }
         if (warp == 1 && lane == 0) {
-            mma_commit(&drain);
-            mbar_drain(&drain, 0);
+            mma_commit(drain);
+            mbar_drain(drain, 0);
         }
     }
     tc_fence_before();
@@ -555,36 +610,32 @@ bool chunk_tc_supported(int d, int chunk, bool bf16) {
 size_t chunk_tc_workspace_bytes(int B, int H, int T, int d, int chunk) {
     if (d != kD || chunk <= 0 || T % chunk) return 0;
     const size_t n = (size_t)B * H * (T / chunk);
-    return n * (kD * 256 + kD * kD) * sizeof(float);
+    return sync_offset(n) + sync_bytes(n);
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     const int cps = a.T / a.chunk;
-    const int n = a.B * a.H * cps;
-    float *AB = static_cast<float *>(a.workspace);
-    uint8_t *Wimg = reinterpret_cast<uint8_t *>(AB + (size_t)n * kD * 256);
+    const int nseq = a.B * a.H, n = nseq * cps;
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+    uint8_t *Wimg = ws + (size_t)n * kChunkWs;
     const uint64_t rows = (uint64_t)a.B * a.H * a.T;
     alignas(64) CUtensorMap tmK, tmV, tmQ;
     if (!encode_tmap_bf16_2d(&tmK, a.K, kD, rows, 64, kGramRows) ||
         !encode_tmap_bf16_2d(&tmV, a.V, kD, rows, 64, kGramRows) ||
         !encode_tmap_bf16_2d(&tmQ, a.Q, kD, rows, 64, kApplyRows))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chunk_gram_kernel,
+    cudaError_t e = cudaFuncSetAttribute(chunk_gram_scan_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGramSmem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(chunk_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kApplySmem);
     if (e != cudaSuccess) return e;
     int *status = device_status_word();
-    chunk_gram_kernel<<<n, kThreads, kGramSmem, s>>>(tmK, tmV, GramArgs{a.eta, AB, a.chunk, status});
-    e = cudaGetLastError();
+    // ticket counter and ready flags start at zero
+    e = cudaMemsetAsync(ws + sync_offset(n), 0, sync_bytes(n), s);
     if (e != cudaSuccess) return e;
-    count_launch(s);
-    e = cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kScanSmem);
-    if (e != cudaSuccess) return e;
-    chunk_scan_kernel<<<a.B * a.H, kScanThreads, kScanSmem, s>>>(
-        ScanArgs{reinterpret_cast<const uint8_t *>(AB), a.W0, Wimg, a.W_out, a.H, cps, a.w0_per_seq, status});
+    chunk_gram_scan_kernel<<<n + nseq * kSlices, kThreads, kGramSmem, s>>>(
+        tmK, tmV, GramScanArgs{a.eta, ws, a.W0, a.W_out, a.chunk, a.H, nseq, cps, a.w0_per_seq, status});
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);

@@ -88,6 +88,7 @@ cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s);
 // TTT-MLP warp-MMA scan (bf16, d = 64, hidden 256, b = 16; rows = B*H*T).
 bool mlp_tc_supported(int d, int dh, int b, bool bf16, long long rows);
 cudaError_t launch_mlp_tc(const MlpArgs &a, cudaStream_t s);
+cudaError_t launch_mlp_umma(const MlpArgs &a, cudaStream_t s);
 
 // Large-chunk tensor-core path (bf16, d = 128, chunk % 128 == 0).
 bool chunk_tc_supported(int d, int chunk, bool bf16);

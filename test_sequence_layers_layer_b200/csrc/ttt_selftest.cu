@@ -112,6 +112,57 @@ __global__ void gelu_kernel(const float *h, float *g, float *gp, int n) {
     }
 }
 
+// Issue cost of tcgen05.mma: thread 0 issues `count` M x N x 16 products
+// (zero operands, K-major, 128-byte swizzle) into `nacc` accumulators in
+// turn, twice; the second round's cycles are written out.
+constexpr int kIssueSmem = 1024 + 16384 + 32768;
+
+__global__ void __launch_bounds__(128) umma_issue_kernel(int M, int N, int count, int nacc,
+                                                         long long *cycles, int *status) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    for (int i = threadIdx.x; i < (16384 + 32768) / 16; i += blockDim.x)
+        reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    if (threadIdx.x < 32) tmem_alloc(&tmem_base, 512);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = tmem_base;
+    bool ok = true;
+    for (int round = 0; round < 2 && ok; ++round) {
+        if (threadIdx.x == 0) {
+            const uint32_t idesc = make_idesc_bf16(M, N, false, false);
+            const uint32_t a = smem_u32(smem), b = smem_u32(smem + 16384);
+            const long long t0 = clock64();
+            for (int i = 0; i < count; ++i)
+                mma_bf16(tb + (uint32_t)((i % nacc) * N), make_sdesc(a + 32 * (i & 3), 16, 1024, kSw128),
+                         make_sdesc(b + 32 * (i & 3), 16, 1024, kSw128), idesc, i >= nacc);
+            const long long t1 = clock64();
+            mma_commit(&bar);
+            ok = mbar_wait(&bar, round & 1, &abort_flag, status, 91);
+            const long long t2 = clock64();
+            if (ok && round == 1) {
+                cycles[0] = t1 - t0;
+                cycles[1] = t2 - t0;
+            }
+        }
+        ok = __syncthreads_or(!ok) == 0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(tb, 512);
+}
+
 // One warp waits on an mbarrier nobody arrives on, with a short limit.
 __global__ void wait_timeout_kernel(uint64_t limit_ns, int *status) {
     __shared__ uint64_t bar;
@@ -158,7 +209,7 @@ extern "C" ttt_status ttt_selftest_umma(int M, int N, int K, int a_layout, int b
     using namespace ttt;
     if (M != 64 && M != 128) return TTT_ERR_SHAPE;
     if (N < 16 || N > 256 || N % (M == 64 ? 8 : 16) != 0 || N % 16 != 0) return TTT_ERR_SHAPE;
-    if (K < 16 || K > 128 || K % 16 != 0) return TTT_ERR_SHAPE;
+    if (K < 16 || K > 256 || K % 16 != 0) return TTT_ERR_SHAPE;
     if (a_layout < 0 || a_layout > 2 || b_layout < 0 || b_layout > 2) return TTT_ERR_ARG;
     if ((a_layout == TTT_DIAG_MNMAJOR_SW128 && M % 64) || (b_layout == TTT_DIAG_MNMAJOR_SW128 && N % 64))
         return TTT_ERR_SHAPE;
@@ -173,6 +224,23 @@ extern "C" ttt_status ttt_selftest_umma(int M, int N, int K, int a_layout, int b
     selftest_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return TTT_ERR_LAUNCH;
+    count_launch(1);
+    return TTT_OK;
+}
+
+extern "C" ttt_status ttt_diag_umma_issue_cycles(int M, int N, int count, int nacc,
+                                                 long long *cycles, ttt_stream stream) {
+    using namespace ttt;
+    if (M != 64 && M != 128) return TTT_ERR_SHAPE;
+    if (N < 16 || N > 256 || N % (M == 64 ? 8 : 16) != 0) return TTT_ERR_SHAPE;
+    if (count < 1 || count > 256 || nacc < 1 || nacc > 4 || nacc * N > 512) return TTT_ERR_SHAPE;
+    if (!cycles) return TTT_ERR_PTR;
+    if (cudaFuncSetAttribute(umma_issue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kIssueSmem) != cudaSuccess)
+        return TTT_ERR_LAUNCH;
+    umma_issue_kernel<<<1, 128, kIssueSmem, static_cast<cudaStream_t>(stream)>>>(
+        M, N, count, nacc, cycles, device_status_word());
+    if (cudaGetLastError() != cudaSuccess) return TTT_ERR_LAUNCH;
     count_launch(1);
     return TTT_OK;
 }

@@ -49,14 +49,14 @@ def test_workload_accounting():
     plan16 = {p[0]: p for p in bench.kernel_plan(ch, 2)}
     assert plan["chunk_apply_kernel"][3] == ch.d * 2 + 4 * ch.d
     assert plan16["chunk_apply_kernel"][3] == ch.d * 2 + 2 * ch.d
-    assert plan["chunk_gram_kernel"][3] == plan16["chunk_gram_kernel"][3]
+    assert plan["chunk_gram_scan_kernel"][3] == plan16["chunk_gram_scan_kernel"][3]
     assert bench.bwd_flops_per_token(64) == 20 * 64 * 64
     assert bench.bwd_bytes_per_token(lin) == 3 * d * 2 + 4 * d + 4 + 3 * 4 * d + 4
 
 
 def test_latency_floor_accounting():
     """One dependent step = scan time / (waves * ceil(T/b)): one CTA per
-    sequence (two for the TTT-MLP cluster scan), one CTA per SM."""
+    sequence, one CTA per SM."""
     from test_sequence_layers_layer_b200 import synth
     lin = synth.WORKLOADS["linear_ln_d64_b8h12_t2048"]
     f = bench.latency_floor(lin, bench.kernel_plan(lin), [0.256])
@@ -66,9 +66,9 @@ def test_latency_floor_accounting():
     f = bench.latency_floor(big, bench.kernel_plan(big), [3.0])
     assert f["waves"] == 3 and f["dependent_steps"] == 128
     ch = synth.WORKLOADS["chunk_d128_c2048_b4h8_t32768"]
-    f = bench.latency_floor(ch, bench.kernel_plan(ch), [0.1, 0.032, 0.2])
-    assert f["kernel"] == "chunk_scan_kernel" and f["dependent_steps"] == 16
-    assert abs(f["us_per_minibatch_step"] - 2.0) < 1e-12
+    f = bench.latency_floor(ch, bench.kernel_plan(ch), [0.032, 0.2])
+    assert f["kernel"] == "chunk_gram_scan_kernel" and f["dependent_steps"] == 16
+    assert abs(f["us_per_minibatch_step"] - 2.0) < 1e-12 and "upper bound" in f["note"]
     mlp = synth.WORKLOADS["mlp_ln_d64_dh256_b4h12_t8192"]
     f = bench.latency_floor(mlp, bench.kernel_plan(mlp), [1.0])
     assert f["concurrent_sequences"] == 48 and f["waves"] == 1

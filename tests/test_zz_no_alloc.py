@@ -43,7 +43,7 @@ def test_noalloc_matches_workspace_entry_point_twice():
     for seed in (3, 4):  # two calls in a row, different inputs, one shared buffer
         wl, x = _case(seed)
         need = ttt.ttt_chunk_workspace_bytes(wl.B, wl.H, wl.T, wl.d, wl.b)
-        assert 0 < need <= (24 << 20)
+        assert 0 < need <= (24 << 20) + 4096
         Zr, Wr = _with_workspace(wl, x)
         Z, W = _noalloc(wl, x)
         torch.cuda.synchronize()
@@ -55,7 +55,7 @@ def test_noalloc_matches_workspace_entry_point_twice():
 
 def test_noalloc_refuses_problems_beyond_its_buffer():
     wl, x = _case(5)
-    big_T = 129 * 256  # 2 * 3 * 129 chunks of 192 KiB > 24 MiB
+    big_T = 129 * 256  # 2 * 3 * 129 chunks of 192 KiB > 24 MiB + 4 KiB
     Z = torch.empty(1, device="cuda")
     n0 = ttt.ttt_launch_count()
     rc = ttt.ttt_chunk_fwd_noalloc(x["Q"], x["K"], x["V"], x["eta"], x["W1"], Z, None, wl.B,
