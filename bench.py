@@ -607,7 +607,21 @@ def decode_arm(args, wl):
                                 x["beta"], z, state, state2, dwl.B, dwl.H, 1, dwl.d, dwl.dh, 1, dt,
                                 ttt.TTT_F_LN | ttt.TTT_F_W0_PER_SEQ, stream.cuda_stream)
 
-    if args.decode_kernel and dwl.kind == "mlp":  # the one-token TTT-MLP kernel
+    if args.decode_one_call:  # all n tokens in one call, the weight on chip across them
+        qkv = {k: x[k].contiguous() for k in ("Q", "K", "V", "eta")}
+        zn = torch.empty((dwl.B, dwl.H, n, dwl.d), dtype=torch.float32, device=dev)
+
+        def steps():  # noqa: F811
+            if dwl.kind == "mlp":
+                ttt.ttt_mlp_decode_tokens(qkv["Q"], qkv["K"], qkv["V"], qkv["eta"], state, state2,
+                                          x["gamma"], x["beta"], zn, dwl.B, dwl.H, n, dwl.d,
+                                          dwl.dh, dt, ttt.TTT_F_LN, stream.cuda_stream)
+            else:
+                ttt.ttt_linear_decode_tokens(qkv["Q"], qkv["K"], qkv["V"], qkv["eta"], state,
+                                             x["gamma"], x["beta"], zn, dwl.B, dwl.H, n, dwl.d,
+                                             dt, ttt.TTT_F_LN if dwl.ln else 0,
+                                             stream.cuda_stream)
+    elif args.decode_kernel and dwl.kind == "mlp":  # the one-token TTT-MLP kernel
         def steps():  # noqa: F811
             for t in toks:
                 ttt.ttt_mlp_decode(t["Q"], t["K"], t["V"], t["eta"], state, state2, x["gamma"],
@@ -658,7 +672,10 @@ def decode_arm(args, wl):
         "config": {"workload": wl.name + "_decode", "B": dwl.B, "H": dwl.H, "d": dwl.d,
                    "layer_norm": dwl.ln, "tokens_per_step": dwl.B * dwl.H,
                    "cuda_graph": graph is not None,
-                   "entry_point": (("ttt_mlp_decode" if dwl.kind == "mlp" else "ttt_linear_decode")
+                   "entry_point": ((("ttt_mlp_decode_tokens" if dwl.kind == "mlp"
+                                     else "ttt_linear_decode_tokens") + f" ({n} tokens, one call)")
+                                   if args.decode_one_call else
+                                   ("ttt_mlp_decode" if dwl.kind == "mlp" else "ttt_linear_decode")
                                    if args.decode_kernel else
                                    ("ttt_mlp_fwd" if dwl.kind == "mlp" else "ttt_linear_fwd")
                                    + " (T = 1, b = 1)")},
@@ -933,6 +950,9 @@ def main():
     ap.add_argument("--decode-kernel", action="store_true",
                     help="with --decode: time the one-token kernel (ttt_linear_decode, "
                          "ttt_mlp_decode)")
+    ap.add_argument("--decode-one-call", action="store_true",
+                    help="with --decode N: all N tokens in one call with the weight on chip "
+                         "(ttt_linear_decode_tokens, ttt_mlp_decode_tokens)")
     ap.add_argument("--e2e-slices", type=int, default=0,
                     help="e2e leg (linear workloads): overlap the host copies with the compute "
                          "over N batch slices (hostio.linear_fwd_host)")

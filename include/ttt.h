@@ -165,6 +165,28 @@ TTT_API ttt_status ttt_mlp_decode(const void *q, const void *k, const void *v, c
                                   ttt_dtype dt, unsigned flags, ttt_stream stream);
 
 /*
+ * Decode of n tokens per sequence in one call, the fast weight kept on chip
+ * across them (the token loop of the listing's step() run inside one kernel,
+ * "Test-Time Training: Linear Complexity Beyond Attention"): the tokens of
+ * sequence s are q, k, v [B][H][n][64] and eta [B][H][n]; each takes its
+ * update and reads out with the updated weight, exactly as n successive
+ * ttt_linear_decode / ttt_mlp_decode calls would, and z is [B][H][n][64].
+ * The weight lives in the registers of the sequence's block for the whole
+ * call and is read and written once. Arguments, flags and errors as
+ * ttt_linear_decode / ttt_mlp_decode, plus n >= 1 (TTT_ERR_SHAPE otherwise).
+ */
+TTT_API ttt_status ttt_linear_decode_tokens(const void *q, const void *k, const void *v,
+                                            const float *eta, float *W, const float *ln_gamma,
+                                            const float *ln_beta, void *z, int B, int H, int n,
+                                            int d, ttt_dtype dt, unsigned flags,
+                                            ttt_stream stream);
+TTT_API ttt_status ttt_mlp_decode_tokens(const void *q, const void *k, const void *v,
+                                         const float *eta, float *W1, float *W2,
+                                         const float *ln_gamma, const float *ln_beta, void *z,
+                                         int B, int H, int n, int d, int dh, ttt_dtype dt,
+                                         unsigned flags, ttt_stream stream);
+
+/*
  * TTT-Linear forward, online (b = 1), with n_steps gradient steps per token
  * ("How to Master Test-Time Training for LLMs", "How TTT Layers Actually
  * Work": the layer runs one or more steps of gradient descent per token).

@@ -106,6 +106,10 @@ def lib() -> ctypes.CDLL:
         L.ttt_diag_gelu.argtypes = [_P, _P, _P, _I, _P]
         L.ttt_diag_wait_timeout.restype = _I
         L.ttt_diag_wait_timeout.argtypes = [ctypes.c_uint, _P]
+        L.ttt_linear_decode_tokens.restype = _I
+        L.ttt_linear_decode_tokens.argtypes = [_P] * 8 + [_I] * 5 + [ctypes.c_uint, _P]
+        L.ttt_mlp_decode_tokens.restype = _I
+        L.ttt_mlp_decode_tokens.argtypes = [_P] * 9 + [_I] * 6 + [ctypes.c_uint, _P]
         L.ttt_diag_mlp_fwd_tcgen05.restype = _I
         L.ttt_diag_mlp_fwd_tcgen05.argtypes = [_P] * 11 + [_I] * 7 + [ctypes.c_uint, _P]
         L.ttt_diag_umma_issue_cycles.restype = _I
@@ -177,6 +181,22 @@ def ttt_linear_decode(q, k, v, eta, W, ln_gamma, ln_beta, z, B, H, d, dt, flags,
     rc = lib().ttt_linear_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(W), _ptr(ln_gamma),
                                  _ptr(ln_beta), _ptr(z), B, H, d, dt, flags, _stream(stream))
     return _check("ttt_linear_decode", rc) if check else rc
+
+
+def ttt_linear_decode_tokens(q, k, v, eta, W, ln_gamma, ln_beta, z, B, H, n, d, dt, flags,
+                             stream=None, check=True):
+    rc = lib().ttt_linear_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(W),
+                                        _ptr(ln_gamma), _ptr(ln_beta), _ptr(z), B, H, n, d, dt,
+                                        flags, _stream(stream))
+    return _check("ttt_linear_decode_tokens", rc) if check else rc
+
+
+def ttt_mlp_decode_tokens(q, k, v, eta, W1, W2, ln_gamma, ln_beta, z, B, H, n, d, dh, dt, flags,
+                          stream=None, check=True):
+    rc = lib().ttt_mlp_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(W1), _ptr(W2),
+                                     _ptr(ln_gamma), _ptr(ln_beta), _ptr(z), B, H, n, d, dh, dt,
+                                     flags, _stream(stream))
+    return _check("ttt_mlp_decode_tokens", rc) if check else rc
 
 
 def ttt_linear_fwd_steps(Q, K, V, eta, W0, ln_gamma, ln_beta, Z, W_out, B, H, T, d, n_steps, dt,
@@ -397,6 +417,36 @@ def linear_decode(q, k, v, eta, W, ln_gamma=None, ln_beta=None, *, ln, z=None, z
     ttt_linear_decode(q, k, v, eta, W, ln_gamma, ln_beta, z, B, H, d, _dtype_code(q), flags,
                       stream)
     return z
+
+
+def linear_decode_tokens(Q, K, V, eta, W, ln_gamma=None, ln_beta=None, *, ln, z_bf16=False,
+                         l2_keys=False, stream=None):
+    """n TTT-Linear tokens per sequence in one call, d = 64: Q, K, V [B, H, n, 64],
+    eta [B, H, n], W [B, H, 64, 64] fp32 updated in place, the weight on chip
+    across the tokens (ttt_linear_decode_tokens). Returns Z [B, H, n, 64]."""
+    import torch
+    B, H, n, d = Q.shape
+    Z = torch.empty((B, H, n, d), dtype=torch.bfloat16 if z_bf16 else torch.float32,
+                    device=Q.device)
+    flags = (TTT_F_LN if ln else 0) | (TTT_F_Z_BF16 if z_bf16 else 0) | \
+        (TTT_F_L2_KEYS if l2_keys else 0)
+    ttt_linear_decode_tokens(Q, K, V, eta, W, ln_gamma, ln_beta, Z, B, H, n, d, _dtype_code(Q),
+                             flags, stream)
+    return Z
+
+
+def mlp_decode_tokens(Q, K, V, eta, W1, W2, ln_gamma, ln_beta, *, z_bf16=False, stream=None):
+    """n TTT-MLP tokens per sequence in one call, d = 64, dh = 256: Q, K, V
+    [B, H, n, 64], eta [B, H, n], W1 [B, H, 64, 256] and W2 [B, H, 256, 64] fp32
+    updated in place, both on chip across the tokens (ttt_mlp_decode_tokens).
+    Returns Z [B, H, n, 64]."""
+    import torch
+    B, H, n, d = Q.shape
+    Z = torch.empty((B, H, n, d), dtype=torch.bfloat16 if z_bf16 else torch.float32,
+                    device=Q.device)
+    ttt_mlp_decode_tokens(Q, K, V, eta, W1, W2, ln_gamma, ln_beta, Z, B, H, n, d, W1.shape[-1],
+                          _dtype_code(Q), TTT_F_LN | (TTT_F_Z_BF16 if z_bf16 else 0), stream)
+    return Z
 
 
 def linear_fwd_steps(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, n_steps, ln,

@@ -163,15 +163,16 @@ cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const 
                              float *dK, float *dV, float *deta, float *dW0, int B, int H, int T,
                              int d, int chunk, bool bf16, bool w0_per_seq, void *workspace,
                              cudaStream_t s);
-// One-token TTT-Linear decode, d = 64 (ttt_decode.cu).
+// TTT-Linear decode of n tokens per sequence, d = 64 (ttt_decode.cu).
 cudaError_t launch_linear_decode(const void *q, const void *k, const void *v, const float *eta,
                                  const float *gamma, const float *beta, float *W, void *z, int B,
-                                 int H, bool bf16, bool ln, bool z_bf16, bool l2_keys,
+                                 int H, int n, bool bf16, bool ln, bool z_bf16, bool l2_keys,
                                  cudaStream_t s);
-// One-token TTT-MLP decode, d = 64, hidden 256 (ttt_mlp_decode.cu).
+// TTT-MLP decode of n tokens per sequence, d = 64, hidden 256 (ttt_mlp_decode.cu).
 cudaError_t launch_mlp_decode(const void *q, const void *k, const void *v, const float *eta,
                               const float *gamma, const float *beta, float *W1, float *W2,
-                              void *z, int B, int H, bool bf16, bool z_bf16, cudaStream_t s);
+                              void *z, int B, int H, int n, bool bf16, bool z_bf16,
+                              cudaStream_t s);
 // TTT-MLP backward (ttt_mlp_bwd.cu).
 bool mlp_bwd_supported(int d, int dh, int b);
 size_t mlp_bwd_workspace_bytes(int B, int H, int T, int d, int b);
@@ -280,14 +281,17 @@ ttt_status ttt_linear_fwd_steps(const void *Q, const void *K, const void *V, con
     return launched(launch_linear_simt_opts(a, (flags & TTT_F_L2_KEYS) != 0, n_steps, cs));
 }
 
-ttt_status ttt_linear_decode(const void *q, const void *k, const void *v, const float *eta,
-                             float *W, const float *ln_gamma, const float *ln_beta, void *z, int B,
-                             int H, int d, ttt_dtype dt, unsigned flags, ttt_stream stream) {
+ttt_status ttt_linear_decode_tokens(const void *q, const void *k, const void *v,
+                                    const float *eta, float *W, const float *ln_gamma,
+                                    const float *ln_beta, void *z, int B, int H, int n, int d,
+                                    ttt_dtype dt, unsigned flags, ttt_stream stream) {
     if (flags & ~(TTT_F_LN | TTT_F_Z_BF16 | TTT_F_L2_KEYS)) return TTT_ERR_ARG;
     const bool ln = flags & TTT_F_LN;
     if (!q || !k || !v || !eta || !W || !z) return TTT_ERR_PTR;
     if (ln && (!ln_gamma || !ln_beta)) return TTT_ERR_PTR;
-    if (B <= 0 || H <= 0 || (long long)B * H > (1LL << 30) || d != 64) return TTT_ERR_SHAPE;
+    if (B <= 0 || H <= 0 || n <= 0 || (long long)B * H > (1LL << 30) || d != 64 ||
+        (long long)B * H * n > (1LL << 34))
+        return TTT_ERR_SHAPE;
     if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(W) || !aligned16(z))
         return TTT_ERR_ALIGN;
@@ -298,19 +302,27 @@ ttt_status ttt_linear_decode(const void *q, const void *k, const void *v, const 
     if (st != TTT_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
-    return launched(launch_linear_decode(q, k, v, eta, ln_gamma, ln_beta, W, z, B, H,
+    return launched(launch_linear_decode(q, k, v, eta, ln_gamma, ln_beta, W, z, B, H, n,
                                          dt == TTT_BF16, ln, (flags & TTT_F_Z_BF16) != 0,
                                          (flags & TTT_F_L2_KEYS) != 0, cs));
 }
 
-ttt_status ttt_mlp_decode(const void *q, const void *k, const void *v, const float *eta,
-                          float *W1, float *W2, const float *ln_gamma, const float *ln_beta,
-                          void *z, int B, int H, int d, int dh, ttt_dtype dt, unsigned flags,
-                          ttt_stream stream) {
+ttt_status ttt_linear_decode(const void *q, const void *k, const void *v, const float *eta,
+                             float *W, const float *ln_gamma, const float *ln_beta, void *z, int B,
+                             int H, int d, ttt_dtype dt, unsigned flags, ttt_stream stream) {
+    return ttt_linear_decode_tokens(q, k, v, eta, W, ln_gamma, ln_beta, z, B, H, 1, d, dt, flags,
+                                    stream);
+}
+
+ttt_status ttt_mlp_decode_tokens(const void *q, const void *k, const void *v, const float *eta,
+                                 float *W1, float *W2, const float *ln_gamma,
+                                 const float *ln_beta, void *z, int B, int H, int n, int d,
+                                 int dh, ttt_dtype dt, unsigned flags, ttt_stream stream) {
     if (flags & ~(TTT_F_LN | TTT_F_Z_BF16)) return TTT_ERR_ARG;
     if (!(flags & TTT_F_LN)) return TTT_ERR_ARG;  // TTT-MLP always has its LayerNorm
     if (!q || !k || !v || !eta || !W1 || !W2 || !ln_gamma || !ln_beta || !z) return TTT_ERR_PTR;
-    if (B <= 0 || H <= 0 || (long long)B * H > (1LL << 30) || d != 64 || dh != 256)
+    if (B <= 0 || H <= 0 || n <= 0 || (long long)B * H > (1LL << 30) || d != 64 || dh != 256 ||
+        (long long)B * H * n > (1LL << 34))
         return TTT_ERR_SHAPE;
     if (dt != TTT_BF16 && dt != TTT_FP32) return TTT_ERR_DTYPE;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(W1) || !aligned16(W2) ||
@@ -324,8 +336,16 @@ ttt_status ttt_mlp_decode(const void *q, const void *k, const void *v, const flo
     if (st != TTT_OK) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
-    return launched(launch_mlp_decode(q, k, v, eta, ln_gamma, ln_beta, W1, W2, z, B, H,
+    return launched(launch_mlp_decode(q, k, v, eta, ln_gamma, ln_beta, W1, W2, z, B, H, n,
                                       dt == TTT_BF16, (flags & TTT_F_Z_BF16) != 0, cs));
+}
+
+ttt_status ttt_mlp_decode(const void *q, const void *k, const void *v, const float *eta,
+                          float *W1, float *W2, const float *ln_gamma, const float *ln_beta,
+                          void *z, int B, int H, int d, int dh, ttt_dtype dt, unsigned flags,
+                          ttt_stream stream) {
+    return ttt_mlp_decode_tokens(q, k, v, eta, W1, W2, ln_gamma, ln_beta, z, B, H, 1, d, dh, dt,
+                                 flags, stream);
 }
 
 size_t ttt_linear_bwd_workspace_bytes(int B, int H, int T, int d, int b) {

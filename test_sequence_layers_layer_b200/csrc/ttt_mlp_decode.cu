@@ -14,7 +14,9 @@
 // read-out's) are reduced across the block by a warp reduce-scatter (lane l
 // ends with outputs 2l and 2l+1 of its warp's sum, 62 shuffles) and a sum of
 // the 8 warps' partials through shared memory. The LayerNorm work runs on
-// threads 0-63, one output each.
+// threads 0-63, one output each. The weights stay in registers over all n
+// tokens of a call (the next token's q, k, v are loaded one token ahead) and
+// are read once and written once per call.
 #include "../../include/ttt.h"
 #include "ttt_common.cuh"
 
@@ -27,9 +29,10 @@ struct MlpDecodeArgs {
     const void *q, *k, *v;
     const float *eta, *gamma, *beta;
     float *W1, *W2;  // [S][64][256], [S][256][64], updated in place
-    float *z;        // [S][64]; bf16 when z_bf16
+    float *z;        // [S][n][64]; bf16 when z_bf16
     int H;
     bool bf16, z_bf16;
+    int n = 1;  // tokens per sequence in this call (q, k, v [S][n][64], eta [S][n])
 };
 
 __device__ __forceinline__ float md_gelu(float h) {
@@ -77,14 +80,8 @@ __global__ void __launch_bounds__(kMThreads, 1) mlp_decode_kernel(MlpDecodeArgs 
     float *ks = msm, *qs = ks + kMD, *vs = qs + kMD, *xs = vs + kMD, *gx = xs + kMD;
     float *R = gx + kMD;                 // [8][64] warp partials
     float *slots = R + kMWarps * kMD;    // 8 reductions x 2 floats
-    const int seq = blockIdx.x, j = threadIdx.x, lane = j & 31, warp = j >> 5;
-    const size_t row = (size_t)seq * kMD;
+    const int seq = blockIdx.x, j = threadIdx.x, lane = j & 31, warp = j >> 5, n = a.n;
     float *W1 = a.W1 + (size_t)seq * kMD * kMF, *W2 = a.W2 + (size_t)seq * kMF * kMD;
-    if (j < kMD) {
-        ks[j] = load_elem(a.k, row + j, a.bf16);
-        qs[j] = load_elem(a.q, row + j, a.bf16);
-        vs[j] = load_elem(a.v, row + j, a.bf16);
-    }
     float w1[kMD], w2[kMD];  // column j of W1, row j of W2
 #pragma unroll
     for (int i = 0; i < kMD; ++i) w1[i] = W1[i * kMF + j];
@@ -96,10 +93,35 @@ __global__ void __launch_bounds__(kMThreads, 1) mlp_decode_kernel(MlpDecodeArgs 
         w2[c + 2] = u.z;
         w2[c + 3] = u.w;
     }
-    const float eta = a.eta[seq];
     const int hh = seq % a.H;
     const float g = j < kMD ? a.gamma[(size_t)hh * kMD + j] : 0.f;
     const float be = j < kMD ? a.beta[(size_t)hh * kMD + j] : 0.f;
+    // token 0's q, k, v and eta; later tokens are loaded one token ahead
+    float kn = 0.f, qn = 0.f, vn = 0.f;
+    if (j < kMD) {
+        const size_t r0 = (size_t)seq * n * kMD + j;
+        kn = load_elem(a.k, r0, a.bf16);
+        qn = load_elem(a.q, r0, a.bf16);
+        vn = load_elem(a.v, r0, a.bf16);
+    }
+    float etan = a.eta[(size_t)seq * n];
+    for (int t = 0; t < n; ++t) {
+    const size_t row = ((size_t)seq * n + t) * kMD;
+    if (t > 0) __syncthreads();  // every reader of the previous token's staging is done
+    if (j < kMD) {
+        ks[j] = kn;
+        qs[j] = qn;
+        vs[j] = vn;
+    }
+    const float eta = etan;
+    if (t + 1 < n) {
+        if (j < kMD) {
+            kn = load_elem(a.k, row + kMD + j, a.bf16);
+            qn = load_elem(a.q, row + kMD + j, a.bf16);
+            vn = load_elem(a.v, row + kMD + j, a.bf16);
+        }
+        etan = a.eta[(size_t)seq * n + t + 1];
+    }
     __syncthreads();  // k, q, v staged
 
     // layer 1 (local): h_j = k . W1[:, j]
@@ -165,6 +187,7 @@ __global__ void __launch_bounds__(kMThreads, 1) mlp_decode_kernel(MlpDecodeArgs 
     const float cq = xq - muq;
     const float rq = rsqrtf(sum64(cq * cq, slots + 10) * (1.f / kMD) + kLnEps);
     if (j < kMD) store_z1(a.z, a.z_bf16, row + j, qs[j] + g * (cq * rq) + be);
+    }
 #pragma unroll
     for (int i = 0; i < kMD; ++i) W1[i * kMF + j] = w1[i];
 #pragma unroll
@@ -178,9 +201,10 @@ __global__ void __launch_bounds__(kMThreads, 1) mlp_decode_kernel(MlpDecodeArgs 
 #ifndef TTT_HOST_RUN  // launch code (a host build of the kernels for tests leaves it out)
 cudaError_t launch_mlp_decode(const void *q, const void *k, const void *v, const float *eta,
                               const float *gamma, const float *beta, float *W1, float *W2,
-                              void *z, int B, int H, bool bf16, bool z_bf16, cudaStream_t s) {
+                              void *z, int B, int H, int n, bool bf16, bool z_bf16,
+                              cudaStream_t s) {
     const MlpDecodeArgs a{q, k, v, eta, gamma, beta, W1, W2, static_cast<float *>(z), H, bf16,
-                          z_bf16};
+                          z_bf16, n};
     const size_t smem = sizeof(float) * (5 * kMD + kMWarps * kMD + 16);
     mlp_decode_kernel<<<(unsigned)(B * H), kMThreads, smem, s>>>(a);
     const cudaError_t e = cudaGetLastError();

@@ -129,3 +129,50 @@ def test_mlp_decode_kernel_loop(dtype):
                            x["beta"], b=1)
     torch.cuda.synchronize()
     assert max_rel_err(Z.double().cpu().numpy(), Zw.double().cpu().numpy(), wl) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("kind,dtype", [("linear", "bf16"), ("linear", "fp32"), ("mlp", "bf16")])
+def test_decode_tokens_in_one_call(kind, dtype):
+    """ttt_linear_decode_tokens / ttt_mlp_decode_tokens (all tokens of the
+    call with the weight kept on chip) equal the loop of one-token calls bit
+    for bit, and match the oracle's online update."""
+    name = "linear_ln_d64_b8h12_t2048" if kind == "linear" else "mlp_ln_d64_dh256_b4h12_t8192"
+    wl = W[name].scaled(B=2, H=3, T=20, b=1, dtype=dtype)
+    inp = synth.make_inputs(wl)
+    x = to_dev(inp)
+    s1 = x["W1"].unsqueeze(0).repeat(wl.B, 1, 1, 1)
+    t1 = s1.clone()
+    if kind == "mlp":
+        s2 = x["W2"].unsqueeze(0).repeat(wl.B, 1, 1, 1)
+        t2 = s2.clone()
+        Z = ttt.mlp_decode_tokens(x["Q"], x["K"], x["V"], x["eta"], s1, s2, x["gamma"], x["beta"])
+    else:
+        Z = ttt.linear_decode_tokens(x["Q"], x["K"], x["V"], x["eta"], s1, x["gamma"], x["beta"],
+                                     ln=True)
+    Zl = torch.empty_like(Z)
+    for i in range(wl.T):
+        q, k, v = (x[n][:, :, i].contiguous() for n in ("Q", "K", "V"))
+        e = x["eta"][:, :, i].contiguous()
+        if kind == "mlp":
+            Zl[:, :, i] = ttt.mlp_decode(q, k, v, e, t1, t2, x["gamma"], x["beta"])
+        else:
+            Zl[:, :, i] = ttt.linear_decode(q, k, v, e, t1, x["gamma"], x["beta"], ln=True)
+    torch.cuda.synchronize()
+    assert ttt.ttt_device_status() == 0
+    assert torch.equal(Z, Zl) and torch.equal(s1, t1)
+    outs = run_oracle(inp)
+    assert max_rel_err(Z.double().cpu().numpy(), outs[0], wl) <= TOL[dtype]
+    assert max_rel_err(s1.double().cpu().numpy(), outs[1], wl) <= TOL[dtype]
+    if kind == "mlp":
+        assert torch.equal(s2, t2)
+        assert max_rel_err(s2.double().cpu().numpy(), outs[2], wl) <= TOL[dtype]
+
+
+def test_decode_tokens_rejects_bad_n():
+    wl = W["linear_ln_d64_b8h12_t2048"].scaled(B=1, H=1, T=4, b=1)
+    x = to_dev(synth.make_inputs(wl))
+    s = x["W1"].unsqueeze(0).repeat(1, 1, 1, 1)
+    z = torch.empty((1, 1, 4, 64), device="cuda")
+    rc = ttt.ttt_linear_decode_tokens(x["Q"], x["K"], x["V"], x["eta"], s, x["gamma"], x["beta"],
+                                      z, 1, 1, 0, 64, ttt.TTT_BF16, ttt.TTT_F_LN, check=False)
+    assert rc == -2
