@@ -563,11 +563,11 @@ size_t ttt_chunk_map_workspace_bytes(int B, int H, int T, int d, int chunk, ttt_
     if (B <= 0 || H <= 0 || T <= 0 || chunk <= 0 || T % chunk || chunk % 128) return 0;
     if ((d != 64 && d != 128) || (dt != TTT_BF16 && dt != TTT_FP32)) return 0;
     if ((long long)B * H > (1LL << 30) || (long long)B * H * T * d > (1LL << 40)) return 0;
+    // tensor-core shapes: one Gram pass and one scan of [M | N] (the forward's workspace)
+    if (chunk_tc_supported(d, chunk, dt == TTT_BF16)) return ttt_chunk_workspace_bytes(B, H, T, d, chunk);
+    // others: two forwards, from W = I with V = 0 and from W = 0
     const size_t n = (size_t)B * H * T * d, e = dt == TTT_BF16 ? 2 : 4;
-    const size_t fwd = chunk_tc_supported(d, chunk, dt == TTT_BF16)
-                           ? ttt_chunk_workspace_bytes(B, H, T, d, chunk)
-                           : 0;
-    return round256(n * e) + round256(n * 2) + round256((size_t)B * H * d * d * sizeof(float)) + fwd;
+    return round256(n * e) + round256(n * 2) + round256((size_t)B * H * d * d * sizeof(float));
 }
 
 ttt_status ttt_chunk_map(const void *K, const void *V, const float *eta, float *M, float *N, int B,
@@ -590,28 +590,27 @@ ttt_status ttt_chunk_map(const void *K, const void *V, const float *eta, float *
     st = check_device_ptrs(ptrs, 6);
     if (st != TTT_OK) return st;
 
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    timing_begin(cs);
+    if (chunk_tc_supported(d, chunk, dt == TTT_BF16))
+        return launched(launch_chunk_map_tc(K, V, eta, M, N, B, H, T, chunk, workspace, cs));
     const size_t S = (size_t)B * H, n = S * T * d, e = dt == TTT_BF16 ? 2 : 4;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     void *v_zero = ws;                                    // [B][H][T][d], V = 0
     void *z_scratch = ws + round256(n * e);               // discarded read-outs, bf16
     float *w_start = reinterpret_cast<float *>(ws + round256(n * e) + round256(n * 2));
-    unsigned char *fwd_ws = reinterpret_cast<unsigned char *>(w_start) +
-                            round256(S * d * d * sizeof(float));
-    const size_t fwd_bytes = workspace_bytes - (size_t)(fwd_ws - ws);
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const unsigned f = TTT_F_W0_PER_SEQ | TTT_F_Z_BF16;
-    timing_begin(cs);
     // M: the forward from W = I with V = 0 (every B_c = 0)
     if (cudaMemsetAsync(v_zero, 0, n * e, cs) != cudaSuccess) return TTT_ERR_LAUNCH;
     if (launch_affine_eye(w_start, (int)S, d, cs) != cudaSuccess) return TTT_ERR_LAUNCH;
-    st = ttt_chunk_fwd(K, K, v_zero, eta, w_start, z_scratch, M, B, H, T, d, chunk, dt, f, fwd_ws,
-                       fwd_bytes, stream);
+    st = ttt_chunk_fwd(K, K, v_zero, eta, w_start, z_scratch, M, B, H, T, d, chunk, dt, f, nullptr,
+                       0, stream);
     if (st != TTT_OK) return st;
     // N: the forward from W = 0
     if (cudaMemsetAsync(w_start, 0, S * d * d * sizeof(float), cs) != cudaSuccess)
         return TTT_ERR_LAUNCH;
-    return ttt_chunk_fwd(K, K, V, eta, w_start, z_scratch, N, B, H, T, d, chunk, dt, f, fwd_ws,
-                         fwd_bytes, stream);
+    return ttt_chunk_fwd(K, K, V, eta, w_start, z_scratch, N, B, H, T, d, chunk, dt, f, nullptr, 0,
+                         stream);
 }
 
 size_t ttt_linear_map_workspace_bytes(int B, int H, int T, int d, int b, ttt_dtype dt) {

@@ -78,6 +78,10 @@ struct GramScanArgs {
     int chunk, H, nseq, cps;
     bool w0_per_seq;
     int *status;
+    // Map mode: no read-out; the scan runs the map W -> M W + N of the whole
+    // sequence instead of the forward: M from W = I without B_c, N from
+    // W = 0 with B_c, 4 slices per sequence (M's two, then N's two).
+    float *M = nullptr, *N = nullptr;
 };
 
 __device__ __forceinline__ int ld_acquire(const int *p) {
@@ -284,7 +288,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     // the registers of 4 epilogue warps (row i = TMEM lane, 64 columns); they
     // form W_c + B_c - (D_hi + D_lo) and write W_c's columns into the
     // read-out's operand image of chunk c in the workspace.
-    const int si = tk - n, s = si / kSlices, r = si % kSlices, j0 = kSlice * r;
+    const bool map = a.M != nullptr;
+    const int per_seq = map ? 2 * kSlices : kSlices;
+    const int si = tk - n, s = si / per_seq, r = si % per_seq, j0 = kSlice * (r % kSlices);
+    const bool ident = map && r < kSlices;  // M: starts at I, takes no B_c
+    float *out = map ? (ident ? a.M : a.N) : a.W_out;
     const int cps = a.cps;
     const size_t g0 = (size_t)s * cps;
     uint8_t *sA = smem;                   // A_c hi (K-major, 32 KB)
@@ -348,16 +356,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else if (warp >= 2) {
         // Epilogue: row i = 32 (warp & 3) + lane, columns j0 .. j0 + 63.
         const int sp = warp & 3, row = 32 * sp + lane;
-        const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? s : s % a.H) * kD * kD;
         float w[kSlice];
+        if (map) {
 #pragma unroll
-        for (int q = 0; q < kSlice / 4; ++q) {
-            const float4 u = *reinterpret_cast<const float4 *>(W0 + (size_t)row * kD + j0 + 4 * q);
-            w[4 * q] = u.x;
-            w[4 * q + 1] = u.y;
-            w[4 * q + 2] = u.z;
-            w[4 * q + 3] = u.w;
+            for (int q = 0; q < kSlice; ++q) w[q] = (ident && row == j0 + q) ? 1.f : 0.f;
+        } else {
+            const float *W0 = a.W0 + (size_t)(a.w0_per_seq ? s : s % a.H) * kD * kD;
+#pragma unroll
+            for (int q = 0; q < kSlice / 4; ++q) {
+                const float4 u = *reinterpret_cast<const float4 *>(W0 + (size_t)row * kD + j0 + 4 * q);
+                w[4 * q] = u.x;
+                w[4 * q + 1] = u.y;
+                w[4 * q + 2] = u.z;
+                w[4 * q + 3] = u.w;
+            }
         }
+        const float bscale = ident ? 0.f : 1.f;
         // This thread's column i of the slice image (rows n: W_hi^T then
         // W_lo^T; 128-byte swizzle, 16 KB per 64 values of i) and row i of
         // chunk c's read-out image (MN-major [i][j], 16 KB per 64 columns j).
@@ -375,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             uint8_t *img = Wimg + (g0 + c) * 65536;
 #pragma unroll
-            for (int h8 = 0; h8 < kSlice / 8; ++h8) {
+            for (int h8 = 0; h8 < kSlice / 8 && !map; ++h8) {
                 uint4 hi, lo;
                 __nv_bfloat16 *hb = reinterpret_cast<__nv_bfloat16 *>(&hi);
                 __nv_bfloat16 *lb = reinterpret_cast<__nv_bfloat16 *>(&lo);
@@ -416,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    w[16 * q + e] = (w[16 * q + e] + bv[e]) - (dh[e] + dl[e]);
+                    w[16 * q + e] = fmaf(bscale, bv[e], w[16 * q + e]) - (dh[e] + dl[e]);
             }
             tc_fence_before();
             __syncwarp();
@@ -428,8 +442,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             if (c + 1 < cps && warp == 2 && lane == 0) mbar_arrive(wready);
         }
-        if (ok && !abort_flag && a.W_out) {
-            float *o = a.W_out + (size_t)s * kD * kD + (size_t)row * kD + j0;
+        if (ok && !abort_flag && out) {
+            float *o = out + (size_t)s * kD * kD + (size_t)row * kD + j0;
 #pragma unroll
             for (int q = 0; q < kSlice / 4; ++q)
                 *reinterpret_cast<float4 *>(o + 4 * q) =
@@ -611,6 +625,33 @@ size_t chunk_tc_workspace_bytes(int B, int H, int T, int d, int chunk) {
     if (d != kD || chunk <= 0 || T % chunk) return 0;
     const size_t n = (size_t)B * H * (T / chunk);
     return sync_offset(n) + sync_bytes(n);
+}
+
+// Map mode: the Gram products and the scan of [M | N] in one launch, no
+// read-out (d = 128, bf16, chunk % 128 == 0; workspace as the forward's).
+cudaError_t launch_chunk_map_tc(const void *K, const void *V, const float *eta, float *M, float *N,
+                                int B, int H, int T, int chunk, void *workspace, cudaStream_t s) {
+    const int cps = T / chunk;
+    const int nseq = B * H, n = nseq * cps;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const uint64_t rows = (uint64_t)B * H * T;
+    alignas(64) CUtensorMap tmK, tmV;
+    if (!encode_tmap_bf16_2d(&tmK, K, kD, rows, 64, kGramRows) ||
+        !encode_tmap_bf16_2d(&tmV, V, kD, rows, 64, kGramRows))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(chunk_gram_scan_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGramSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(ws + sync_offset(n), 0, sync_bytes(n), s);
+    if (e != cudaSuccess) return e;
+    GramScanArgs g{eta, ws, nullptr, nullptr, chunk, H, nseq, cps, false, device_status_word()};
+    g.M = M;
+    g.N = N;
+    chunk_gram_scan_kernel<<<n + nseq * 2 * kSlices, kThreads, kGramSmem, s>>>(tmK, tmV, g);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launch(s);
+    return cudaSuccess;
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {

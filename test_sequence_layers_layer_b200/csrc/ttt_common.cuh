@@ -94,6 +94,8 @@ cudaError_t launch_mlp_umma(const MlpArgs &a, cudaStream_t s);
 bool chunk_tc_supported(int d, int chunk, bool bf16);
 size_t chunk_tc_workspace_bytes(int B, int H, int T, int d, int chunk);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
+cudaError_t launch_chunk_map_tc(const void *K, const void *V, const float *eta, float *M, float *N,
+                                int B, int H, int T, int chunk, void *workspace, cudaStream_t s);
 
 // Encodes a 2-D bf16 TMA descriptor (CUtensorMap, 128 bytes) over a
 // row-major [rows][cols] tensor with a box of box_rows x box_cols elements and
