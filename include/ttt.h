@@ -87,7 +87,7 @@ typedef void *ttt_stream; /* a cudaStream_t */
 #define TTT_F_L2_KEYS 8u    /* ttt_linear_fwd: keys scaled to unit length,
                                k / max(||k||_2, 1e-12), wherever the inner
                                loss and its gradient use them (the query is
-                               used as given); runs the fp32 CUDA-core kernel */
+                               used as given) */
 
 #define TTT_ABI_VERSION 1
 
@@ -122,8 +122,10 @@ TTT_API const char *ttt_status_string(int status);
  * flags: TTT_F_LN, TTT_F_W0_PER_SEQ, TTT_F_Z_BF16, TTT_F_L2_KEYS. With
  *   TTT_F_L2_KEYS the key is normalised, as in the PyTorch listing on "Test-
  *   Time Training: Linear Complexity Beyond Attention"; with LayerNorm, the
- *   residual k of f(k) = k + LN(k W) is the normalised key too. Every shape
- *   then runs the fp32 CUDA-core kernel.
+ *   residual k of f(k) = k + LN(k W) is the normalised key too. The
+ *   tensor-core scan keeps the raw bf16 keys in its products and applies
+ *   the per-token scales 1 / ||k|| as row and column scalings in fp32; the
+ *   other shapes scale the keys in the fp32 kernel.
  */
 TTT_API ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const float *eta,
                           const float *W0, const float *ln_gamma, const float *ln_beta,

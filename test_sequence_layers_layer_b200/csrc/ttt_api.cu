@@ -248,9 +248,9 @@ ttt_status ttt_linear_fwd(const void *Q, const void *K, const void *V, const flo
                  dt == TTT_BF16, ln, (flags & TTT_F_W0_PER_SEQ) != 0, (flags & TTT_F_Z_BF16) != 0};
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     timing_begin(cs);
-    if (flags & TTT_F_L2_KEYS) return launched(launch_linear_simt_keys(a, true, cs));
-    return launched(linear_tc_supported(d, b, dt == TTT_BF16) ? launch_linear_tc(a, cs)
-                                                                : launch_linear_simt(a, cs));
+    const bool l2 = flags & TTT_F_L2_KEYS;
+    if (linear_tc_supported(d, b, dt == TTT_BF16)) return launched(launch_linear_tc(a, cs, l2));
+    return launched(l2 ? launch_linear_simt_keys(a, true, cs) : launch_linear_simt(a, cs));
 }
 
 ttt_status ttt_linear_fwd_steps(const void *Q, const void *K, const void *V, const float *eta,

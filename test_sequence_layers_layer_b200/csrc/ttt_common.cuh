@@ -83,7 +83,7 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
 
 // TTT-Linear tensor-core scan (bf16, d = 64, b = 16).
 bool linear_tc_supported(int d, int b, bool bf16);
-cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s);
+cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s, bool l2_keys = false);
 
 // TTT-MLP warp-MMA scan (bf16, d = 64, hidden 256, b = 16; rows = B*H*T).
 bool mlp_tc_supported(int d, int dh, int b, bool bf16, long long rows);

@@ -80,7 +80,8 @@ constexpr int OFF_GF = OFF_CF + 2 * 16 * kCStride * 4;  // G fp32 [4][16][64]
 constexpr int OFF_ZQ = OFF_GF + 4 * 16 * 64 * 4;      // Q W fp32 [4][16][64], float4-swizzled
 constexpr int OFF_SF = OFF_ZQ + 4 * 16 * 64 * 4;      // Q K^T fp32 [4][16][kCStride]
 constexpr int OFF_ETA = OFF_SF + 4 * 16 * kCStride * 4;  // eta fp32 [kSlots][64], one row per chunk
-constexpr int OFF_TRACE = OFF_ETA + kSlots * kChunkTok * 4;
+constexpr int OFF_KS = OFF_ETA + kSlots * kChunkTok * 4;  // 1 / |k| fp32 [kSlots][64] (L2 keys)
+constexpr int OFF_TRACE = OFF_KS + kSlots * kChunkTok * 4;
 #ifdef TTT_TRACE
 constexpr int kTraceBytes = kTraceEvents * kTraceSteps * 4;
 #else
@@ -171,6 +172,7 @@ __device__ __forceinline__ void split4(float a, float b, float c, float d, uint2
     split2(c, d, hi.y, lo.y);
 }
 
+template <bool kL2>  // L2-normalised keys: compiled as its own kernel
 __global__ void __launch_bounds__(kThreads, 1)
     linear_ln_scan_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmQ,
@@ -186,6 +188,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *Zqf = reinterpret_cast<float *>(smem + OFF_ZQ);
     float *Sf = reinterpret_cast<float *>(smem + OFF_SF);
     float *etas = reinterpret_cast<float *>(smem + OFF_ETA);
+    // Key scales s_t = 1 / max(|k_t|, 1e-12) with L2-normalised keys, else 1.
+    // The kernel keeps the raw bf16 keys in every product and applies s as
+    // row / column scalings: P and C rows by the key token's s, C and Q K^T
+    // columns by the source token's s, the key residual of the LayerNorm
+    // backward and the G rows of the weight update by s.
+    float *kscale = reinterpret_cast<float *>(smem + OFF_KS);
 #ifdef TTT_TRACE
     volatile unsigned *trace_smem = reinterpret_cast<volatile unsigned *>(smem + OFF_TRACE);
     for (int e = threadIdx.x; e < kTraceEvents * kTraceSteps; e += blockDim.x) trace_smem[e] = 0;
@@ -237,6 +245,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Row r of mini-batch m in a K/Q/V ring (generic pointer to its 128 bytes).
     auto ring_row = [&](uint8_t *ring, int m, int r) -> uint8_t * {
         return ring + ((m / kMbPerChunk) % kSlots) * kTile + ((m % kMbPerChunk) * kMB + r) * 128;
+    };
+    // key scale of token t of mini-batch m (staged with the chunk's etas)
+    auto kscale_of = [&](int m, int t) -> float {
+        return kscale[((m / kMbPerChunk) % kSlots) * kChunkTok + (m % kMbPerChunk) * kMB + t];
     };
     auto chunk_wait = [&](int m, int code) -> bool {  // warp-uniform wait for m's chunk
         const int c = m / kMbPerChunk;
@@ -320,6 +332,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = lane; e < kChunkTok; e += 32) {
                     const long tok = (long)c * kChunkTok + e;
                     etas[(c % kSlots) * kChunkTok + e] = tok < T ? a.eta[tok0 + tok] : 0.f;
+                    if constexpr (kL2) {  // the row's 16-byte chunks in any order: sum of squares
+                        const uint8_t *kr = sK + (c % kSlots) * kTile + e * 128;
+                        float ss = 0.f;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const uint4 u = *reinterpret_cast<const uint4 *>(kr + 16 * q);
+                            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[h]));
+                                ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                            }
+                        }
+                        kscale[(c % kSlots) * kChunkTok + e] = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+                    }
                 }
             }
             uint8_t *dst = sA + s * 4096;
@@ -351,6 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t col = TM_B + ((i + 2) & 1) * kBRows;
             float *dst = qrow ? Zqf + (mz & 3) * 1024 : Pf + (mp & 1) * 1024;
             const bool live = qrow ? mz >= 0 : mp < NM;
+            // key scales: this K row's (P and C rows), the source keys' (columns)
+            const int msrc = i + 1;  // B rows 128-143 hold K_{i+1}
+            const float rs = (kL2 && !qrow && live) ? kscale_of(mp, row) : 1.f;
             float v0[16], v1[16];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {  // hi + lo, 16 columns at a time
@@ -362,14 +392,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         d4[swz4(row, 4 * c + q)] =
-                            make_float4(v0[4 * q] + v1[4 * q], v0[4 * q + 1] + v1[4 * q + 1],
-                                        v0[4 * q + 2] + v1[4 * q + 2], v0[4 * q + 3] + v1[4 * q + 3]);
+                            kL2
+                                ? make_float4(rs * (v0[4 * q] + v1[4 * q]), rs * (v0[4 * q + 1] + v1[4 * q + 1]),
+                                              rs * (v0[4 * q + 2] + v1[4 * q + 2]),
+                                              rs * (v0[4 * q + 3] + v1[4 * q + 3]))
+                                : make_float4(v0[4 * q] + v1[4 * q], v0[4 * q + 1] + v1[4 * q + 1],
+                                              v0[4 * q + 2] + v1[4 * q + 2], v0[4 * q + 3] + v1[4 * q + 3]);
                 }
             }
             tmem_ld16(taddr(tm, 96, col + 128), v0);
             tmem_ld_wait();
             if (live) {
                 float *g16 = qrow ? Sf + ((mz & 3) * 16 + row) * kCStride : Cf + ((mp & 1) * 16 + row) * kCStride;
+                if (kL2 && msrc >= 0) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v0[e] *= rs * kscale_of(msrc, e);
+                }
                 float4 *c4 = reinterpret_cast<float4 *>(g16);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) c4[q] = make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
@@ -430,9 +468,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float eta = etas[((j / kMbPerChunk) % kSlots) * kChunkTok + (j % kMbPerChunk) * kMB + t];
             float vv[8], G[8];
             load_quads_bf16(ring_row(sV, j, 0), t, g, vv);
+            const float ksc = kL2 ? kscale_of(j, t) : 1.f;
             if (a.ln) {
                 float kv[8];
                 load_quads_bf16(ring_row(sK, j, 0), t, g, kv);
+                if constexpr (kL2) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) kv[i] *= ksc;
+                }
                 float mu, rstd;
                 row_stats(x, mu, rstd);
                 float xh[8], gh[8], s1 = 0.f, s2 = 0.f;
@@ -467,7 +510,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint2 hi, lo;
-                split4(-G[4 * h], -G[4 * h + 1], -G[4 * h + 2], -G[4 * h + 3], hi, lo);
+                if constexpr (kL2)
+                    split4(-ksc * G[4 * h], -ksc * G[4 * h + 1], -ksc * G[4 * h + 2],
+                           -ksc * G[4 * h + 3], hi, lo);
+                else
+                    split4(-G[4 * h], -G[4 * h + 1], -G[4 * h + 2], -G[4 * h + 3], hi, lo);
                 const uint32_t off = off_mnmajor_sw128(t, 32 * h + 4 * g, kMB);
                 *reinterpret_cast<uint2 *>(gb + off) = hi;
                 *reinterpret_cast<uint2 *>(gb + 2048 + off) = lo;
@@ -640,19 +687,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool linear_tc_supported(int d, int b, bool bf16) { return bf16 && d == kD && b == kMB; }
 
-cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s) {
+cudaError_t launch_linear_tc(const LinearArgs &a, cudaStream_t s, bool l2_keys) {
     const uint64_t rows = (uint64_t)a.B * a.H * a.T;
     alignas(64) CUtensorMap tmK, tmQ, tmV;
     if (!encode_tmap_bf16_2d(&tmK, a.K, kD, rows, kD, kChunkTok) ||
         !encode_tmap_bf16_2d(&tmQ, a.Q, kD, rows, kD, kChunkTok) ||
         !encode_tmap_bf16_2d(&tmV, a.V, kD, rows, kD, kChunkTok))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(linear_ln_scan_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    auto kernel = l2_keys ? linear_ln_scan_kernel<true> : linear_ln_scan_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
     if (e != cudaSuccess) return e;
     Args args{a.eta, a.W0, a.gamma, a.beta, a.Z, a.W_out, a.H, a.T, a.ln, a.w0_per_seq,
               a.z_bf16, device_status_word()};
-    linear_ln_scan_kernel<<<a.B * a.H, kThreads, kSmemBytes, s>>>(tmK, tmQ, tmV, args);
+    kernel<<<a.B * a.H, kThreads, kSmemBytes, s>>>(tmK, tmQ, tmV, args);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch(s);
     return e;
