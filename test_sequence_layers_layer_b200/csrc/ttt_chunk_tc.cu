@@ -62,6 +62,11 @@ constexpr int kGramStages = 4;
 constexpr int kGramBox = kGramRows * 128;        // one 64-column box of a stage (4 KB)
 constexpr int kGramStageBytes = 6 * kGramBox;    // K (2 boxes) | V (2) | eta*K (2)
 constexpr size_t kGramSmem = 1024 + kGramStages * kGramStageBytes;  // 97 KB: two blocks per SM
+// With one step size for the whole chunk, K itself is the A operand (no eta*K
+// copy, no conversion pass) and the accumulator is scaled by eta once: the
+// same 96 KB then hold 6 stages of K | V.
+constexpr int kGramStagesU = 6, kGramStageBytesU = 4 * kGramBox;
+static_assert(kGramStagesU * kGramStageBytesU <= kGramStages * kGramStageBytes, "uniform-eta ring");
 constexpr int kSlice = 64, kSlices = kD / kSlice;  // scan: output columns per block
 constexpr int kSliceImg = 2 * kSlice * kD * 2;     // [W hi | W lo] slice image [128][128] bf16: 32 KB
 static_assert(2 * kImgBytes / 2 + kSliceImg + 1024 <= (int)kGramSmem, "scan role fits the gram's smem");
@@ -111,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bars[3 * kGramStages + 2];
+    __shared__ uint64_t bars[3 * kGramStagesU + 2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag, ticket;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -125,17 +130,25 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int tk = ticket;
     const bool gram = tk < n;
     const uint32_t ncols = 256;  // the gram role's accumulator
-    uint64_t *drain = &bars[3 * kGramStages + 1];
+    uint64_t *drain = &bars[3 * kGramStagesU + 1];
 
     if (gram) {
         // ---- gram of chunk c of sequence s (chunk-major ticket order)
         const int c = tk / a.nseq, s = tk % a.nseq, g = s * a.cps + c;
-        uint64_t *full = bars, *conv = bars + kGramStages, *empty = bars + 2 * kGramStages;
-        uint64_t *done = &bars[3 * kGramStages];
+        uint64_t *full = bars, *conv = bars + kGramStagesU, *empty = bars + 2 * kGramStagesU;
+        uint64_t *done = &bars[3 * kGramStagesU];
         const long row0 = (long)g * a.chunk;  // first token row of this chunk in [B*H*T][d]
         const int nst = a.chunk / kGramRows;
+        // one step size over the whole chunk?
+        const float eta0 = a.eta[row0];
+        bool differs = false;
+        for (int i = threadIdx.x; i < a.chunk; i += kThreads)
+            differs |= __float_as_uint(a.eta[row0 + i]) != __float_as_uint(eta0);
+        const bool uniform = !__syncthreads_or(differs);
+        const int stages = uniform ? kGramStagesU : kGramStages;
+        const int stage_bytes = uniform ? kGramStageBytesU : kGramStageBytes;
         if (threadIdx.x == 0) {
-            for (int i = 0; i < kGramStages; ++i) {
+            for (int i = 0; i < stages; ++i) {
                 mbar_init(&full[i], 1);
                 mbar_init(&conv[i], 128);
                 mbar_init(&empty[i], 1);
@@ -153,11 +166,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (warp == 0 && lane == 0) {
             // TMA producer: K rows and V rows of each stage, two 64-column boxes each.
             for (int r = 0; r < nst; ++r) {
-                const int st = r % kGramStages;
-                if (r >= kGramStages &&
-                    !mbar_wait(&empty[st], ((r / kGramStages) - 1) & 1, &abort_flag, a.status, 11))
+                const int st = r % stages;
+                if (r >= stages &&
+                    !mbar_wait(&empty[st], ((r / stages) - 1) & 1, &abort_flag, a.status, 11))
                     break;
-                uint8_t *sb = smem + st * kGramStageBytes;
+                uint8_t *sb = smem + st * stage_bytes;
                 const int y = (int)(row0 + (long)r * kGramRows);
                 mbar_arrive_expect_tx(&full[st], 4 * kGramBox);
                 tma_load_2d(sb, &tmK, 0, y, &full[st]);
@@ -167,16 +180,20 @@ __global__ void __launch_bounds__(kThreads, 2)
                 issued = r + 1;
             }
         } else if (warp == 1 && lane == 0) {
-            // MMA issuer: D[d_in][0:128) += (eta K)^T K, D[d_in][128:256) += (eta K)^T V.
+            // MMA issuer: D[d_in][0:128) += (eta K)^T K, D[d_in][128:256) += (eta K)^T V
+            // (uniform eta: K^T K | K^T V, scaled by eta in the epilogue).
             const uint32_t idesc = make_idesc_bf16(128, 256, true, true);
+            const uint32_t aoff = uniform ? 0u : 4u * kGramBox;
             for (int r = 0; r < nst; ++r) {
-                const int st = r % kGramStages;
-                if (!mbar_wait(&conv[st], (r / kGramStages) & 1, &abort_flag, a.status, 12)) break;
+                const int st = r % stages;
+                if (!mbar_wait(uniform ? &full[st] : &conv[st], (r / stages) & 1, &abort_flag,
+                               a.status, 12))
+                    break;
                 tc_fence_after();
-                const uint32_t ab = smem_u32(smem + st * kGramStageBytes);
+                const uint32_t ab = smem_u32(smem + st * stage_bytes);
 #pragma unroll
                 for (int k = 0; k < kGramRows / 16; ++k) {
-                    const uint64_t ad = make_sdesc(ab + 4 * kGramBox + k * 2048, kGramBox, 1024, kSw128);
+                    const uint64_t ad = make_sdesc(ab + aoff + k * 2048, kGramBox, 1024, kSw128);
                     const uint64_t bd = make_sdesc(ab + k * 2048, kGramBox, 1024, kSw128);
                     mma_bf16(tm, ad, bd, idesc, (r | k) != 0);
                 }
@@ -189,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             // 128-byte row only, so a chunk's row (token) is offset / 128.
             const int t = threadIdx.x - 64;
             constexpr int kChunks = 2 * kGramBox / 16;  // 16-byte chunks of K per stage
-            for (int r = 0; r < nst; ++r) {
+            for (int r = 0; r < nst && !uniform; ++r) {
                 const int st = r % kGramStages;
                 // This thread's eta values for the stage, loaded before the wait.
                 float ev[kChunks / 128];
@@ -228,10 +245,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int row = 32 * sp + lane;
                 uint8_t *blk = a.ws + (size_t)g * kChunkWs;
                 float4 *bdst = reinterpret_cast<float4 *>(blk + 2 * kImgBytes);
+                const float scale = uniform ? eta0 : 1.f;
                 for (int q = 0; q < 16; ++q) {
                     float v[16];
                     tmem_ld16(taddr(tm, 32 * sp, 16 * q), v);
                     tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] *= scale;
                     if (q < 8) {
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
@@ -258,8 +278,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         // before the shared memory and tensor memory are released.
         if (abort_flag) {
             if (warp == 0 && lane == 0)
-                for (int r = issued - kGramStages < 0 ? 0 : issued - kGramStages; r < issued; ++r)
-                    mbar_drain(&full[r % kGramStages], (r / kGramStages) & 1);
+                for (int r = issued - stages < 0 ? 0 : issued - stages; r < issued; ++r)
+                    mbar_drain(&full[r % stages], (r / stages) & 1);
             if (warp == 1 && lane == 0) {
                 mma_commit(drain);
                 mbar_drain(drain, 0);
