@@ -86,14 +86,11 @@ def kernel_plan(wl, zb: int = 4, tcgen05_mlp: bool = False):
     e = 2 if wl.dtype == "bf16" else 4
     d = wl.d
     if wl.kind == "chunk" and wl.dtype == "bf16" and d == 128 and wl.b % 128 == 0:
-        return [
-            # K, V and eta in, A_c | B_c = K^T [eta K | eta V]; with the scan
-            # W_{c+1} = W_c - A_c W_c + B_c (d^3 per chunk; W0 in, W_out out)
-            ("chunk_gram_scan_kernel", "ttt_chunk_tc.cu", "bf16", 2 * d * e + 4 + 8 * d * d / wl.T,
-             4 * d * d + 2 * d ** 3 / wl.b),
-            # Q in, Z (fp32) out; Z = Q W_c
-            ("chunk_apply_kernel", "ttt_chunk_tc.cu", "bf16", d * e + zb * d, 2 * d * d),
-        ]
+        # One launch: K, V and eta in, A_c | B_c = K^T [eta K | eta V]; the
+        # scan W_{c+1} = W_c - A_c W_c + B_c (d^3 per chunk; W0 in, W_out
+        # out); Q in, Z = Q W_c out.
+        return [("chunk_fwd_kernel", "ttt_chunk_tc.cu", "bf16",
+                 3 * d * e + 4 + zb * d + 8 * d * d / wl.T, 6 * d * d + 2 * d ** 3 / wl.b)]
     if wl.kind == "linear" and wl.dtype == "bf16" and d == 64 and wl.b == 16:
         return [("linear_ln_scan_kernel", "ttt_linear_tc.cu", "bf16", algo_bytes_per_token(wl, zb),
                  algo_flops_per_token(wl))]
@@ -294,9 +291,9 @@ def latency_floor(wl, plan, kern_ms_per_call):
     out = {"us_per_minibatch_step": kern_ms_per_call[idx] * 1e3 / (waves * steps),
            "dependent_steps": steps, "concurrent_sequences": concurrent, "waves": waves,
            "kernel": plan[idx][0]}
-    if plan[idx][0] == "chunk_gram_scan_kernel":
-        out["note"] = ("the scan shares its launch with the Gram products: an upper bound on "
-                       "one chunk step")
+    if plan[idx][0] == "chunk_fwd_kernel":
+        out["note"] = ("the scan shares its launch with the Gram products and the read-out: an "
+                       "upper bound on one chunk step")
     return out
 
 

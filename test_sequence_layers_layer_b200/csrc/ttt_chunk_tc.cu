@@ -6,20 +6,22 @@
 // chunk c reads out with W_c, then
 //   W_{c+1} = W_c - sum_{s in c} eta_s k_s^T (k_s W_c - v_s)
 //           = W_c - A_c W_c + B_c,   A_c = K_c^T diag(eta) K_c,  B_c = K_c^T diag(eta) V_c.
-// The update is affine in W, so the work splits into two launches:
-//   1. gram + scan, one launch with two block roles taken in start order:
-//      gram:  A_c | B_c for every chunk of every sequence (the only pass over
+// The update is affine in W, so the work splits into three block roles of
+// one launch, taken in start order (a ticket counter), each waiting only on
+// blocks that started before it:
+//   gram:     A_c | B_c for every chunk of every sequence (the only pass over
 //             K and V; tcgen05, M = d_in = 128, N = 256, K = tokens), each
 //             chunk published by a ready flag;
-//      scan:  W_{c+1} = W_c - A_c W_c + B_c, 16 steps per sequence, split by
-//             32-column slices of W over 4 blocks (columns evolve
-//             independently; tcgen05, M = 128, N = 32, K = 128, hi/lo
-//             operands; state and update in fp32), each step as soon as its
-//             chunk is published, writing each W_c as the ready-made bf16
+//   scan:     W_{c+1} = W_c - A_c W_c + B_c, one step per chunk, split by
+//             64-column slices of W over 2 blocks per sequence (columns evolve
+//             independently; tcgen05, M = 128, N = 128 = the slice's hi and lo
+//             terms, K = 128; state and update in fp32), each step as soon as
+//             its chunk is published, writing each W_c as the ready-made bf16
 //             hi/lo operand image of the read-out;
-//   2. apply: Z_c = Q_c W_c for every chunk at once (the only pass over Q and
-//             the only write of Z; tcgen05, M = 128 tokens, N = d_out, K = d_in;
-//             W_c arrives by one bulk copy).
+//   read-out: Z_c = Q_c W_c once both slices of W_c are written (the only
+//             pass over Q and the only write of Z; tcgen05, M = 64 tokens,
+//             N = 256 = hi | lo side by side, K = d_in; W_c arrives by one
+//             bulk copy). Their HBM traffic overlaps the Gram's.
 // Q/K/V tiles arrive by TMA with the 128-byte swizzle; accumulators live in
 // tensor memory. W_c enters the apply products as two bf16 terms (hi + lo)
 // so the read-out keeps ~16 significant bits of the fp32 state.
@@ -73,7 +75,9 @@ static_assert(2 * kImgBytes / 2 + kSliceImg + 1024 <= (int)kGramSmem, "scan role
 
 // Ready flags and the ticket counter sit after the per-chunk workspace.
 __host__ __device__ constexpr size_t sync_offset(size_t n) { return n * ((size_t)kChunkWs + 65536); }
-__host__ __device__ constexpr size_t sync_bytes(size_t n) { return ((n + 1) * 4 + 255) / 256 * 256; }
+// [0]: ticket counter, [1 + g]: chunk g's Gram published, [1 + n + g]: the
+// number of scan blocks that have written their columns of W_g's read-out image.
+__host__ __device__ constexpr size_t sync_bytes(size_t n) { return ((2 * n + 1) * 4 + 255) / 256 * 256; }
 
 struct GramScanArgs {
     const float *eta;
@@ -87,7 +91,20 @@ struct GramScanArgs {
     // sequence instead of the forward: M from W = I without B_c, N from
     // W = 0 with B_c, 4 slices per sequence (M's two, then N's two).
     float *M = nullptr, *N = nullptr;
+    // Forward: the read-out's output (bf16 instead when z_bf16) and the
+    // number of read-out blocks per chunk (each takes chunk / parts tokens, a
+    // multiple of 128).
+    float *Z = nullptr;
+    bool z_bf16 = false;
+    int parts = 1;
 };
+
+// Read-out blocks per chunk: about 512 tokens each, in whole 128-token tiles.
+int readout_parts(int chunk) {
+    for (int p = chunk / 512; p > 1; --p)
+        if ((chunk / 128) % p == 0) return p;
+    return 1;
+}
 
 __device__ __forceinline__ int ld_acquire(const int *p) {
     int v;
@@ -110,9 +127,33 @@ __device__ bool wait_flag(const int *flag, volatile int *abort, int *status, int
     }
 }
 
+// Read-out role: Z_c^T = W_c^T Q_c^T per 128-token tile, with W_c^T (hi and
+// lo bf16 terms, 64 + 64 columns) as the A operand in tensor memory and the Q
+// tile as the K-major B operand, so that shared memory holds only a 3-stage
+// Q ring (3 x 32 KB).
+constexpr int kApplyTile = 128, kApplyTileBytes = kApplyTile * kD * 2;  // 32 KB
+constexpr int kApplyStages = 3;
+static_assert(kApplyStages * kApplyTileBytes <= kGramStages * kGramStageBytes,
+              "read-out role fits the shared memory of the launch");
+
+__device__ bool wait_count(const int *p, int want, volatile int *abort, int *status, int code) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 0;; ++i) {
+        if (ld_acquire(p) >= want) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicExch(status, code);
+            return false;
+        }
+        __nanosleep(i < 16 ? 64 : 512);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 2)
-    chunk_gram_scan_kernel(const __grid_constant__ CUtensorMap tmK,
-                           const __grid_constant__ CUtensorMap tmV, GramScanArgs a) {
+    chunk_fwd_kernel(const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmQ, GramScanArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -129,8 +170,156 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     const int tk = ticket;
     const bool gram = tk < n;
-    const uint32_t ncols = 256;  // the gram role's accumulator
+    const int nscan = a.nseq * (a.M ? 2 * kSlices : kSlices);
+    const uint32_t ncols = 256;  // the gram and read-out roles' accumulator
     uint64_t *drain = &bars[3 * kGramStagesU + 1];
+
+    if (tk >= n + nscan) {
+        // ---- read-out of part `part` of chunk c of sequence s (chunk-major
+        // ticket order): Z_c = Q_c W_c once both scan blocks of s have written
+        // W_c's image. A chunk's tokens are split over a.parts blocks, so that
+        // the last chunk's read-out, which waits for the whole scan, is short.
+        // Q does not depend on the scan: its first tiles load while the block
+        // waits for W_c.
+        const int ai = tk - n - nscan, per_c = a.nseq * a.parts;
+        const int c = ai / per_c, s = (ai % per_c) / a.parts, part = ai % a.parts;
+        const int g = s * a.cps + c;
+        const int ntile = a.chunk / a.parts / kApplyTile;
+        const long row0 = (long)g * a.chunk + (long)part * ntile * kApplyTile;
+        uint64_t *qfull = bars, *qempty = bars + kApplyStages, *wfull = bars + 2 * kApplyStages,
+                 *tfull = wfull + 1, *tempty = wfull + 2;
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < kApplyStages; ++i) {
+                mbar_init(&qfull[i], 1);
+                mbar_init(&qempty[i], 1);
+            }
+            mbar_init(wfull, 128);
+            mbar_init(tfull, 1);
+            mbar_init(tempty, 128);
+            mbar_init(drain, 1);
+            fence_mbar_init();
+        }
+        if (warp == 1) tmem_alloc(&tmem_base, ncols);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // tensor memory: [0, 64) W^T hi, [64, 128) W^T lo (lane j = output
+        // column j, column q = inputs 2q, 2q + 1), [128, 256) the accumulator
+        // (lane j, column = token of the tile)
+        const uint32_t tm = tmem_base, tA = tm, tD = tm + 128;
+        int issued = 0;
+        if (warp == 0 && lane == 0) {
+            for (int t = 0; t < ntile; ++t) {
+                const int st = t % kApplyStages;
+                if (t >= kApplyStages &&
+                    !mbar_wait(&qempty[st], ((t / kApplyStages) - 1) & 1, &abort_flag, a.status, 21))
+                    break;
+                uint8_t *sb = smem + st * kApplyTileBytes;
+                const int y = (int)(row0 + (long)t * kApplyTile);
+                mbar_arrive_expect_tx(&qfull[st], kApplyTileBytes);
+                tma_load_2d(sb, &tmQ, 0, y, &qfull[st]);
+                tma_load_2d(sb + kApplyTileBytes / 2, &tmQ, 64, y, &qfull[st]);
+                issued = t + 1;
+            }
+        } else if (warp == 1 && lane == 0) {
+            const uint32_t idesc = make_idesc_bf16(128, kApplyTile, false, false);
+            if (mbar_wait(wfull, 0, &abort_flag, a.status, 22)) {
+                for (int t = 0; t < ntile; ++t) {
+                    const int st = t % kApplyStages;
+                    if (!mbar_wait(&qfull[st], (t / kApplyStages) & 1, &abort_flag, a.status, 23)) break;
+                    if (t >= 1 && !mbar_wait(tempty, (t - 1) & 1, &abort_flag, a.status, 24)) break;
+                    tc_fence_after();
+                    const uint32_t qb = smem_u32(smem + st * kApplyTileBytes);
+#pragma unroll
+                    for (int k = 0; k < kD / 16; ++k) {
+                        const int k0 = 16 * k;
+                        const uint64_t bd = make_sdesc(qb + (k0 >> 6) * (kApplyTileBytes / 2) + (k0 & 63) * 2,
+                                                       16, 1024, kSw128);
+                        mma_bf16_tmem_a(tD, tA + 8 * k, bd, idesc, k != 0);
+                        mma_bf16_tmem_a(tD, tA + 64 + 8 * k, bd, idesc, true);
+                    }
+                    mma_commit(&qempty[st]);
+                    mma_commit(tfull);
+                }
+            }
+        } else if (warp >= 2) {
+            // Thread j = 32 (warp & 3) + lane: output column j. W_c^T row j
+            // from the image (K-major rows n: hi j at n = 128 (j / 64) + j % 64,
+            // lo 64 rows further; 16-byte chunk q of row n at q ^ (n & 7))
+            // into tensor memory.
+            const int j = 32 * (warp & 3) + lane;
+            bool ok = true;
+            if (warp == 2 && lane == 0) ok = wait_count(sync + 1 + n + g, kSlices, &abort_flag, a.status, 26);
+            ok = !named_bar_or(1, 128, !ok);
+            if (ok) {
+                const uint8_t *img = a.ws + (size_t)n * kChunkWs + (size_t)g * 65536;
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {  // hi, lo
+                    const int nr = 128 * (j >> 6) + 64 * p + (j & 63);
+#pragma unroll
+                    for (int kb = 0; kb < 2; ++kb) {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(
+                            img + kb * kImgBytes + (nr >> 3) * 1024 + (nr & 7) * 128);
+                        float v[32];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const uint4 u = src[q ^ (nr & 7)];
+                            v[4 * q] = __uint_as_float(u.x);
+                            v[4 * q + 1] = __uint_as_float(u.y);
+                            v[4 * q + 2] = __uint_as_float(u.z);
+                            v[4 * q + 3] = __uint_as_float(u.w);
+                        }
+                        const uint32_t ta = taddr(tA, 32 * (warp & 3), 64 * p + 32 * kb);
+                        tmem_st16(ta, *reinterpret_cast<float(*)[16]>(v));
+                        tmem_st16(ta + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+                    }
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(wfull);
+            }
+            // Epilogue: thread j stores column j of each token row of the tile.
+            for (int t = 0; ok && t < ntile; ++t) {
+                if (!__all_sync(0xffffffffu, mbar_wait(tfull, t & 1, &abort_flag, a.status, 25))) break;
+                tc_fence_after();
+                const size_t z0 = (size_t)(row0 + (long)t * kApplyTile) * kD + j;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float v[4][16];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) tmem_ld16(taddr(tD, 32 * (warp & 3), 64 * h + 16 * q), v[q]);
+                    tmem_ld_wait();
+                    if (h == 1) {
+                        tc_fence_before();
+                        mbar_arrive(tempty);  // the accumulator is read; the next tile's MMA may start
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const size_t o = z0 + (size_t)(64 * h + 16 * q + e) * kD;
+                            if (a.z_bf16)
+                                reinterpret_cast<__nv_bfloat16 *>(a.Z)[o] = __float2bfloat16_rn(v[q][e]);
+                            else
+                                a.Z[o] = v[q][e];
+                        }
+                }
+            }
+        }
+        if (abort_flag) {
+            if (warp == 0 && lane == 0)
+                for (int t = issued - kApplyStages < 0 ? 0 : issued - kApplyStages; t < issued; ++t)
+                    mbar_drain(&qfull[t % kApplyStages], (t / kApplyStages) & 1);
+            if (warp == 1 && lane == 0) {
+                mma_commit(drain);
+                mbar_drain(drain, 0);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 1) tmem_dealloc(tm, ncols);
+        return;
+    }
 
     if (gram) {
         // ---- gram of chunk c of sequence s (chunk-major ticket order)
@@ -342,9 +531,25 @@ __global__ void __launch_bounds__(kThreads, 2)
         // A_c once chunk c's gram is published and the product of chunk
         // c - 1 is done with the buffer; B_c once the epilogue of c - 1 has
         // read the previous one.
+        // Each chunk's A_c and B_c slice are also prefetched into L2 as soon
+        // as the chunk is published (and the next chunk's too when it already
+        // is), so that the copies into shared memory, which wait for the
+        // previous step, hit L2 instead of waiting on HBM behind the streams.
+        auto prefetch = [&](int c) {
+            const uint8_t *blk = a.ws + (g0 + c) * kChunkWs;
+            bulk_prefetch_l2(blk, kImgBytes);
+            bulk_prefetch_l2(blk + 2 * kImgBytes + (size_t)j0 * kD * 4, kImgBytes);
+        };
+        int prefetched = 0;  // chunks [0, prefetched) are prefetched
         for (int c = 0; c < cps; ++c) {
             if (!wait_flag(sync + 1 + g0 + c, &abort_flag, a.status, 15)) break;
             asm volatile("fence.proxy.async.global;" ::: "memory");
+            if (prefetched <= c) prefetch(c), prefetched = c + 1;
+            if (c + 1 < cps && prefetched == c + 1 && ld_acquire(sync + 1 + g0 + c + 1)) {
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                prefetch(c + 1);
+                prefetched = c + 2;
+            }
             const uint8_t *blk = a.ws + (g0 + c) * kChunkWs;
             if (c >= 1 && !mbar_wait(afree, (c - 1) & 1, &abort_flag, a.status, 16)) break;
             mbar_arrive_expect_tx(aready, kImgBytes);
@@ -393,8 +598,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         const float bscale = ident ? 0.f : 1.f;
         // This thread's column i of the slice image (rows n: W_hi^T then
-        // W_lo^T; 128-byte swizzle, 16 KB per 64 values of i) and row i of
-        // chunk c's read-out image (MN-major [i][j], 16 KB per 64 columns j).
+        // W_lo^T; 128-byte swizzle, 16 KB per 64 values of i).
         auto emit = [&](int c) {
             const uint32_t cb = (uint32_t)((row >> 6) * 16384 + (row & 7) * 2);
 #pragma unroll
@@ -407,26 +611,40 @@ __global__ void __launch_bounds__(kThreads, 2)
                 *reinterpret_cast<__nv_bfloat16 *>(sWs + cb + (nl >> 3) * 1024 + (nl & 7) * 128 +
                                                    ((((row & 63) >> 3) ^ (nl & 7)) << 4)) = lb;
             }
-            uint8_t *img = Wimg + (g0 + c) * 65536;
-#pragma unroll
-            for (int h8 = 0; h8 < kSlice / 8 && !map; ++h8) {
-                uint4 hi, lo;
-                __nv_bfloat16 *hb = reinterpret_cast<__nv_bfloat16 *>(&hi);
-                __nv_bfloat16 *lb = reinterpret_cast<__nv_bfloat16 *>(&lo);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) split_bf16(w[8 * h8 + e], hb[e], lb[e]);
-                const uint32_t off = off_mnmajor_sw128(row, j0 + 8 * h8, kD);
-                *reinterpret_cast<uint4 *>(img + off) = hi;
-                *reinterpret_cast<uint4 *>(img + kImgBytes + off) = lo;
-            }
             fence_async_smem();
+        };
+        // The slice image is also W_c's share of the read-out operand: one
+        // thread copies its two 16 KB K blocks into chunk c's image in the
+        // workspace (K block kb of slice r at 32 KB kb + 16 KB r) by bulk
+        // store, and counts the chunk for the read-out once the store is
+        // complete, a step later, so that neither the wait nor a memory fence
+        // lands on the scan's chain.
+        const bool pub = !map && warp == 2 && lane == 0;
+        auto store_image = [&](int c) {
+            uint8_t *img = Wimg + (g0 + c) * 65536 + (size_t)r * (kImgBytes / 2);
+            bulk_store(img, sWs, kImgBytes / 2);
+            bulk_store(img + kImgBytes, sWs + kImgBytes / 2, kImgBytes / 2);
+            bulk_commit();
+        };
+        int released = 0;  // chunks whose image share is counted
+        auto release_upto = [&](int c_end) {
+            if (released >= c_end) return;
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __threadfence();
+            for (; released < c_end; ++released) atomicAdd(sync + 1 + n + g0 + released, 1);
         };
         emit(0);
         bool ok = !named_bar_or(1, 128, false);
+        if (ok && pub) store_image(0);
         if (ok && warp == 2 && lane == 0) mbar_arrive(wready);
         for (int c = 0; ok && c < cps; ++c) {
             bool got = mbar_wait(bready, c & 1, &abort_flag, a.status, 19);
             got = got && mbar_wait(dfull, c & 1, &abort_flag, a.status, 20);
+            if (pub) {
+                bulk_wait_read<0>();  // the slice image may be rewritten after the barrier
+                bulk_wait<1>();       // images of chunks < c are stored
+                release_upto(c);
+            }
             if (named_bar_or(1, 128, !__all_sync(0xffffffffu, got))) {
                 ok = false;
                 break;
@@ -460,7 +678,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 ok = false;
                 break;
             }
+            if (c + 1 < cps && pub) store_image(c + 1);
             if (c + 1 < cps && warp == 2 && lane == 0) mbar_arrive(wready);
+        }
+        if (pub) {
+            bulk_wait<0>();
+            if (ok && !abort_flag) release_upto(cps);
         }
         if (ok && !abort_flag && out) {
             float *o = out + (size_t)s * kD * kD + (size_t)row * kD + j0;
@@ -488,157 +711,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == 1) tmem_dealloc(tm, 128);
 }
 
-// ---------------------------------------------------------------------------
-// 3. apply: Z_c = Q_c (W_c,hi + W_c,lo), one block per chunk, 128-token tiles.
-constexpr int kApplyRows = 128;
-constexpr int kApplyStages = 3;
-constexpr int kApplyThreads = 320;  // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
-constexpr int kApplyStageOff = 65536 + kApplyStages * 32768;  // epilogue staging, 8 KB per warp
-constexpr size_t kApplySmem = 1024 + kApplyStageOff + 8 * 8192;
-
-struct ApplyArgs {
-    const uint8_t *Wimg;
-    float *Z;  // bf16 instead when z_bf16
-    int chunk;
-    bool z_bf16;
-    int *status;
-};
-
-__global__ void __launch_bounds__(kApplyThreads, 1)
-    chunk_apply_kernel(const __grid_constant__ CUtensorMap tmQ, ApplyArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sW = smem;          // hi [0, 32K), lo [32K, 64K): MN-major, d_in rows
-    uint8_t *sQ = smem + 65536;  // stages of 128 tokens x 128 d (two 64-column boxes)
-    __shared__ uint64_t full[kApplyStages], empty[kApplyStages], tfull[2], tempty[2], wfull, drain;
-    __shared__ uint32_t tmem_base;
-    __shared__ int abort_flag;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = blockIdx.x;
-    const long row0 = (long)g * a.chunk;
-    const int ntile = a.chunk / kApplyRows;
-
-    if (threadIdx.x == 0) {
-        abort_flag = 0;
-        for (int s = 0; s < kApplyStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 256);
-        }
-        mbar_init(&wfull, 1);
-        mbar_init(&drain, 1);
-        fence_mbar_init();
-    }
-    if (warp == 1) tmem_alloc(&tmem_base, 256);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tm = tmem_base;
-    int issued = 0;
-    bool w_issued = false;
-
-    if (warp == 0 && lane == 0) {
-        mbar_arrive_expect_tx(&wfull, 65536);
-        bulk_load(sW, a.Wimg + (size_t)g * 65536, 32768, &wfull);
-        bulk_load(sW + 32768, a.Wimg + (size_t)g * 65536 + 32768, 32768, &wfull);
-        w_issued = true;
-        for (int t = 0; t < ntile; ++t) {
-            const int s = t % kApplyStages;
-            if (t >= kApplyStages &&
-                !mbar_wait(&empty[s], ((t / kApplyStages) - 1) & 1, &abort_flag, a.status, 21))
-                break;
-            uint8_t *st = sQ + s * 32768;
-            const int y = (int)(row0 + (long)t * kApplyRows);
-            mbar_arrive_expect_tx(&full[s], 32768);
-            tma_load_2d(st, &tmQ, 0, y, &full[s]);
-            tma_load_2d(st + 16384, &tmQ, 64, y, &full[s]);
-            issued = t + 1;
-        }
-    } else if (warp == 1 && lane == 0) {
-        const uint32_t idesc = make_idesc_bf16(128, 128, false, true);
-        const uint32_t wb = smem_u32(sW);
-        if (mbar_wait(&wfull, 0, &abort_flag, a.status, 22)) {
-            for (int t = 0; t < ntile; ++t) {
-                const int s = t % kApplyStages, acc = t & 1;
-                if (!mbar_wait(&full[s], (t / kApplyStages) & 1, &abort_flag, a.status, 23)) break;
-                if (t >= 2 && !mbar_wait(&tempty[acc], ((t >> 1) - 1) & 1, &abort_flag, a.status, 24))
-                    break;
-                tc_fence_after();
-                const uint32_t qb = smem_u32(sQ + s * 32768);
-#pragma unroll
-                for (int k = 0; k < kD / 16; ++k) {
-                    const int k0 = 16 * k;
-                    const uint64_t ad = make_sdesc(qb + (k0 >> 6) * 16384 + (k0 & 63) * 2, 16, 1024, kSw128);
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        const uint64_t bd = make_sdesc(wb + p * 32768 + (k0 >> 3) * 1024, 16384, 1024, kSw128);
-                        mma_bf16(tm + acc * 128, ad, bd, idesc, (k | p) != 0);
-                    }
-                }
-                mma_commit(&empty[s]);
-                mma_commit(&tfull[acc]);
-            }
-        }
-    } else if (warp >= 2) {
-        // Epilogue: lane = token row of the tile; each warp pair splits the
-        // 128 fp32 columns of its subpartition's 32 rows. The warp's 32 x 64
-        // block goes through shared memory (16-byte chunk c of row r at chunk
-        // c ^ (r & 7): conflict-free both ways) so that every global store
-        // writes two whole 256-byte half-rows of Z.
-        const int sp = warp & 3, half = (warp - 2) >> 2;
-        float *stage = reinterpret_cast<float *>(smem + kApplyStageOff) + (warp - 2) * 2048;
-        for (int t = 0; t < ntile; ++t) {
-            const int acc = t & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (t >> 1) & 1, &abort_flag, a.status, 25)))
-                break;
-            tc_fence_after();
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float v[16];
-                tmem_ld16(taddr(tm, 32 * sp, acc * 128 + 64 * half + 16 * q), v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    *reinterpret_cast<float4 *>(stage + lane * 64 + (((4 * q + i) ^ (lane & 7)) << 2)) =
-                        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            }
-            tc_fence_before();
-            mbar_arrive(&tempty[acc]);  // the accumulator is read; the MMA may reuse it
-            __syncwarp();
-            const size_t zbase = ((size_t)(row0 + (long)t * kApplyRows) + 32 * sp) * kD + 64 * half;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 2 * i + (lane >> 4), c = lane & 15;
-                const float4 f = *reinterpret_cast<const float4 *>(stage + r * 64 + ((c ^ (r & 7)) << 2));
-                store_z4(a.Z, a.z_bf16, zbase + (size_t)r * kD + 4 * c, f.x, f.y, f.z, f.w);
-            }
-            __syncwarp();
-        }
-    }
-    if (abort_flag) {
-        if (warp == 0 && lane == 0) {
-            if (w_issued) mbar_drain(&wfull, 0);
-            for (int t = issued - kApplyStages < 0 ? 0 : issued - kApplyStages; t < issued; ++t)
-                mbar_drain(&full[t % kApplyStages], (t / kApplyStages) & 1);
-        }
-        if (warp == 1 && lane == 0) {
-            mma_commit(&drain);
-            mbar_drain(&drain, 0);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) tmem_dealloc(tm, 256);
-}
-
 }  // namespace
 
 bool chunk_tc_supported(int d, int chunk, bool bf16) {
-    return bf16 && d == kD && chunk >= kApplyRows && chunk % kApplyRows == 0;
+    return bf16 && d == kD && chunk >= 128 && chunk % 128 == 0;
 }
 
 size_t chunk_tc_workspace_bytes(int B, int H, int T, int d, int chunk) {
@@ -659,7 +735,7 @@ cudaError_t launch_chunk_map_tc(const void *K, const void *V, const float *eta, 
     if (!encode_tmap_bf16_2d(&tmK, K, kD, rows, 64, kGramRows) ||
         !encode_tmap_bf16_2d(&tmV, V, kD, rows, 64, kGramRows))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chunk_gram_scan_kernel,
+    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGramSmem);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(ws + sync_offset(n), 0, sync_bytes(n), s);
@@ -667,7 +743,8 @@ cudaError_t launch_chunk_map_tc(const void *K, const void *V, const float *eta, 
     GramScanArgs g{eta, ws, nullptr, nullptr, chunk, H, nseq, cps, false, device_status_word()};
     g.M = M;
     g.N = N;
-    chunk_gram_scan_kernel<<<n + nseq * 2 * kSlices, kThreads, kGramSmem, s>>>(tmK, tmV, g);
+    // no read-out blocks: the Q map is never read (K's stands in)
+    chunk_fwd_kernel<<<n + nseq * 2 * kSlices, kThreads, kGramSmem, s>>>(tmK, tmV, tmK, g);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
@@ -678,29 +755,24 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     const int cps = a.T / a.chunk;
     const int nseq = a.B * a.H, n = nseq * cps;
     uint8_t *ws = static_cast<uint8_t *>(a.workspace);
-    uint8_t *Wimg = ws + (size_t)n * kChunkWs;
     const uint64_t rows = (uint64_t)a.B * a.H * a.T;
     alignas(64) CUtensorMap tmK, tmV, tmQ;
     if (!encode_tmap_bf16_2d(&tmK, a.K, kD, rows, 64, kGramRows) ||
         !encode_tmap_bf16_2d(&tmV, a.V, kD, rows, 64, kGramRows) ||
-        !encode_tmap_bf16_2d(&tmQ, a.Q, kD, rows, 64, kApplyRows))
+        !encode_tmap_bf16_2d(&tmQ, a.Q, kD, rows, 64, kApplyTile))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chunk_gram_scan_kernel,
+    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGramSmem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kApplySmem);
-    if (e != cudaSuccess) return e;
-    int *status = device_status_word();
-    // ticket counter and ready flags start at zero
+    // ticket counter, ready flags and read-out counts start at zero
     e = cudaMemsetAsync(ws + sync_offset(n), 0, sync_bytes(n), s);
     if (e != cudaSuccess) return e;
-    chunk_gram_scan_kernel<<<n + nseq * kSlices, kThreads, kGramSmem, s>>>(
-        tmK, tmV, GramScanArgs{a.eta, ws, a.W0, a.W_out, a.chunk, a.H, nseq, cps, a.w0_per_seq, status});
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    count_launch(s);
-    chunk_apply_kernel<<<n, kApplyThreads, kApplySmem, s>>>(tmQ, ApplyArgs{Wimg, a.Z, a.chunk, a.z_bf16, status});
+    GramScanArgs g{a.eta, ws, a.W0, a.W_out, a.chunk, a.H, nseq, cps, a.w0_per_seq, device_status_word()};
+    g.Z = a.Z;
+    g.z_bf16 = a.z_bf16;
+    g.parts = readout_parts(a.chunk);
+    // n Gram blocks, 2 scan blocks per sequence, parts read-out blocks per chunk
+    chunk_fwd_kernel<<<n + nseq * kSlices + n * g.parts, kThreads, kGramSmem, s>>>(tmK, tmV, tmQ, g);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
@@ -710,7 +782,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
 }  // namespace ttt
 
 // ---------------------------------------------------------------------------
-// Allocation-free entry point: the same three kernels, with their scratch in a
+// Allocation-free entry point: the same launch, with its scratch in a
 // statically declared device buffer instead of a caller workspace.
 namespace {
 

@@ -47,9 +47,10 @@ def test_workload_accounting():
     ch = synth.WORKLOADS["chunk_d128_c2048_b4h8_t32768"]
     plan = {p[0]: p for p in bench.kernel_plan(ch)}
     plan16 = {p[0]: p for p in bench.kernel_plan(ch, 2)}
-    assert plan["chunk_apply_kernel"][3] == ch.d * 2 + 4 * ch.d
-    assert plan16["chunk_apply_kernel"][3] == ch.d * 2 + 2 * ch.d
-    assert plan["chunk_gram_scan_kernel"][3] == plan16["chunk_gram_scan_kernel"][3]
+    kv_eta_w = 2 * ch.d * 2 + 4 + 8 * ch.d * ch.d / ch.T  # K, V, eta in; W0 in, W_out out
+    assert plan["chunk_fwd_kernel"][3] == kv_eta_w + ch.d * 2 + 4 * ch.d  # Q in, Z out
+    assert plan16["chunk_fwd_kernel"][3] == kv_eta_w + ch.d * 2 + 2 * ch.d
+    assert plan["chunk_fwd_kernel"][4] == 6 * ch.d ** 2 + 2 * ch.d ** 3 / ch.b
     assert bench.bwd_flops_per_token(64) == 20 * 64 * 64
     assert bench.bwd_bytes_per_token(lin) == 3 * d * 2 + 4 * d + 4 + 3 * 4 * d + 4
 
@@ -66,8 +67,8 @@ def test_latency_floor_accounting():
     f = bench.latency_floor(big, bench.kernel_plan(big), [3.0])
     assert f["waves"] == 3 and f["dependent_steps"] == 128
     ch = synth.WORKLOADS["chunk_d128_c2048_b4h8_t32768"]
-    f = bench.latency_floor(ch, bench.kernel_plan(ch), [0.032, 0.2])
-    assert f["kernel"] == "chunk_gram_scan_kernel" and f["dependent_steps"] == 16
+    f = bench.latency_floor(ch, bench.kernel_plan(ch), [0.032])
+    assert f["kernel"] == "chunk_fwd_kernel" and f["dependent_steps"] == 16
     assert abs(f["us_per_minibatch_step"] - 2.0) < 1e-12 and "upper bound" in f["note"]
     mlp = synth.WORKLOADS["mlp_ln_d64_dh256_b4h12_t8192"]
     f = bench.latency_floor(mlp, bench.kernel_plan(mlp), [1.0])

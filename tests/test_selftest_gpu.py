@@ -82,26 +82,33 @@ def test_bounded_wait_times_out_and_context_survives():
 def test_kernel_timing_sums_over_calls_without_sync():
     """Per-kernel event timing kept across several calls: one read after the
     loop returns, per kernel position, the summed durations; each is positive
-    and together they fit inside the outer events around the calls."""
+    and together they fit inside the outer events around the calls. The
+    large-chunk backward with a shared W0 launches four kernels (Gram, scan,
+    token pass, sum over the batch)."""
     from test_sequence_layers_layer_b200 import synth
     from gpu_helpers import to_dev
     wl = synth.WORKLOADS["chunk_d128_c2048_b4h8_t32768"].scaled(B=1, H=2, T=1024, b=256)
     x = to_dev(synth.make_inputs(wl))
-    ws = torch.empty(ttt.ttt_chunk_workspace_bytes(wl.B, wl.H, wl.T, wl.d, wl.b),
+    dZ = torch.randn((wl.B, wl.H, wl.T, wl.d), device="cuda")
+    ws = torch.empty(ttt.ttt_chunk_bwd_workspace_bytes(wl.B, wl.H, wl.T, wl.d, wl.b),
                      dtype=torch.uint8, device="cuda")
-    ttt.chunk_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], chunk=wl.b, workspace=ws)
+
+    def call():
+        return ttt.chunk_bwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], dZ, chunk=wl.b, workspace=ws)
+
+    call()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ttt.ttt_diag_kernel_timing(True)
     try:
         e0.record()
         for _ in range(3):
-            ttt.chunk_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W1"], chunk=wl.b, workspace=ws)
+            call()
         e1.record()
         times = ttt.ttt_diag_kernel_times(8)
     finally:
         ttt.ttt_diag_kernel_timing(False)
     torch.cuda.synchronize()
-    assert len(times) == 2 and all(t > 0 for t in times), times
+    assert len(times) == 4 and all(t > 0 for t in times), times
     assert sum(times) <= e0.elapsed_time(e1) * 1.001 + 1e-3
     assert ttt.ttt_diag_kernel_times(8) == []  # disabled: nothing recorded
