@@ -26,6 +26,8 @@
 // tensor memory. W_c enters the apply products as two bf16 terms (hi + lo)
 // so the read-out keeps ~16 significant bits of the fp32 state.
 
+#include <algorithm>
+
 #include "../../include/ttt.h"
 #include "sm100.cuh"
 #include "ttt_common.cuh"
@@ -99,9 +101,15 @@ struct GramScanArgs {
     int parts = 1;
 };
 
-// Read-out blocks per chunk: about 512 tokens each, in whole 128-token tiles.
-int readout_parts(int chunk) {
-    for (int p = chunk / 512; p > 1; --p)
+// Read-out blocks per chunk, for n chunks: about 1024 read-out blocks in all
+// (3.5 waves of the 296 resident blocks: enough to keep HBM busy while the
+// last chunks wait for the scan, few enough that each block's W_c set-up is
+// spread over several tiles), at least two 128-token tiles per block, and a
+// divisor of the chunk's tiles.
+int readout_parts(int chunk, int n) {
+    int want = n >= 1024 ? 1 : 1024 / n;
+    want = std::min(want, std::max(1, chunk / 256));
+    for (int p = want; p > 1; --p)
         if ((chunk / 128) % p == 0) return p;
     return 1;
 }
@@ -770,7 +778,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     GramScanArgs g{a.eta, ws, a.W0, a.W_out, a.chunk, a.H, nseq, cps, a.w0_per_seq, device_status_word()};
     g.Z = a.Z;
     g.z_bf16 = a.z_bf16;
-    g.parts = readout_parts(a.chunk);
+    g.parts = readout_parts(a.chunk, n);
     // n Gram blocks, 2 scan blocks per sequence, parts read-out blocks per chunk
     chunk_fwd_kernel<<<n + nseq * kSlices + n * g.parts, kThreads, kGramSmem, s>>>(tmK, tmV, tmQ, g);
     e = cudaGetLastError();
