@@ -287,31 +287,29 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mbar_arrive(wfull);
             }
             // Epilogue: thread j stores column j of each token row of the tile.
+            // All of the tile's accumulator columns are loaded before the one
+            // wait, so that the accumulator is released to the next tile's MMA
+            // before any store.
             for (int t = 0; ok && t < ntile; ++t) {
                 if (!__all_sync(0xffffffffu, mbar_wait(tfull, t & 1, &abort_flag, a.status, 25))) break;
                 tc_fence_after();
+                float v[kApplyTile / 16][16];
+#pragma unroll
+                for (int q = 0; q < kApplyTile / 16; ++q) tmem_ld16(taddr(tD, 32 * (warp & 3), 16 * q), v[q]);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(tempty);  // the accumulator is read; the next tile's MMA may start
                 const size_t z0 = (size_t)(row0 + (long)t * kApplyTile) * kD + j;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    float v[4][16];
+                for (int q = 0; q < kApplyTile / 16; ++q)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) tmem_ld16(taddr(tD, 32 * (warp & 3), 64 * h + 16 * q), v[q]);
-                    tmem_ld_wait();
-                    if (h == 1) {
-                        tc_fence_before();
-                        mbar_arrive(tempty);  // the accumulator is read; the next tile's MMA may start
+                    for (int e = 0; e < 16; ++e) {
+                        const size_t o = z0 + (size_t)(16 * q + e) * kD;
+                        if (a.z_bf16)
+                            reinterpret_cast<__nv_bfloat16 *>(a.Z)[o] = __float2bfloat16_rn(v[q][e]);
+                        else
+                            a.Z[o] = v[q][e];
                     }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const size_t o = z0 + (size_t)(64 * h + 16 * q + e) * kD;
-                            if (a.z_bf16)
-                                reinterpret_cast<__nv_bfloat16 *>(a.Z)[o] = __float2bfloat16_rn(v[q][e]);
-                            else
-                                a.Z[o] = v[q][e];
-                        }
-                }
             }
         }
         if (abort_flag) {
