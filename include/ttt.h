@@ -320,15 +320,17 @@ TTT_API ttt_status ttt_mlp_bwd(const void *Q, const void *K, const void *V, cons
  * gradient descent on the chunk's mean loss.
  * Arguments as ttt_linear_fwd without LayerNorm; `chunk` is the chunk length.
  * workspace: device scratch of at least ttt_chunk_workspace_bytes(...) bytes
- *   (192 KiB per chunk of every sequence when d = 128, plus 4 bytes per chunk
- *   and a counter for the chunks' ready flags, rounded up to 256 bytes; 0 for
+ *   (192 KiB per chunk of every sequence when d = 128, plus 8 bytes per chunk
+ *   for its ready flag and read-out count and a ticket counter, rounded up to
+ *   256 bytes; 0 for
  *   the shapes that need none, when workspace may be NULL), 256-byte aligned,
  *   owned by the caller; its contents on entry do not matter and are
  *   clobbered. Calls that share a workspace must not overlap on the GPU.
  * Supported: T % chunk == 0, chunk % 128 == 0; d = 128 with TTT_BF16 runs
- *   on the tensor cores (a memset of the ready flags and two launches: the
- *   per-chunk Gram products together with the sequential affine scan over
- *   chunks, then the read-out), d in {64, 128}
+ *   on the tensor cores (a memset of the flags and one launch whose blocks
+ *   take three roles in start order: the per-chunk Gram products, the
+ *   sequential affine scan over chunks, and the read-out of each chunk as
+ *   soon as its weight is known), d in {64, 128}
  *   with TTT_FP32, and d = 64, run the fp32 CUDA-core kernel.
  * flags: TTT_F_W0_PER_SEQ, TTT_F_Z_BF16.
  */
