@@ -383,7 +383,8 @@ def gpu_arm(args, wl, rank, world, keep=None):
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = sum(o.numel() * o.element_size() for o in host_out)
     e2e_steps = max(3, min(args.steps, 10))
-    sliced = args.e2e_slices > 0 and wl.kind == "linear"
+    slices = args.e2e_slices if args.e2e_slices is not None else 4
+    sliced = slices > 0 and wl.kind in ("linear", "chunk")
     with torch.cuda.stream(stream):
         def e2e_step():
             for k, v in host_in.items():
@@ -394,11 +395,18 @@ def gpu_arm(args, wl, rank, world, keep=None):
         if sliced:
             from test_sequence_layers_layer_b200 import hostio
 
+            host_pair = (host_out[0], host_out[1])
+
             def e2e_step():  # noqa: F811  (copies overlapped across batch slices)
-                hostio.linear_fwd_host(host_in["Q"], host_in["K"], host_in["V"], host_in["eta"],
-                                       host_in["W1"], host_in.get("gamma"), host_in.get("beta"),
-                                       b=wl.b, ln=wl.ln, slices=args.e2e_slices,
-                                       z_bf16=args.z_bf16)
+                if wl.kind == "chunk":
+                    hostio.chunk_fwd_host(host_in["Q"], host_in["K"], host_in["V"], host_in["eta"],
+                                          host_in["W1"], chunk=wl.b, slices=slices,
+                                          z_bf16=args.z_bf16, out=host_pair)
+                else:
+                    hostio.linear_fwd_host(host_in["Q"], host_in["K"], host_in["V"], host_in["eta"],
+                                           host_in["W1"], host_in.get("gamma"), host_in.get("beta"),
+                                           b=wl.b, ln=wl.ln, slices=slices,
+                                           z_bf16=args.z_bf16, out=host_pair)
         e2e_step()
         stream.synchronize()
         barrier()
@@ -468,7 +476,7 @@ def gpu_arm(args, wl, rank, world, keep=None):
         "kernels": kernels,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "copies": f"overlapped over {args.e2e_slices} batch slices" if sliced
+                "copies": f"overlapped over {slices} batch slices (hostio)" if sliced
                 else "in series with the call"},
         "gpu_launches": launches,
         "clocks": clocks,
@@ -950,9 +958,10 @@ def main():
     ap.add_argument("--decode-one-call", action="store_true",
                     help="with --decode N: all N tokens in one call with the weight on chip "
                          "(ttt_linear_decode_tokens, ttt_mlp_decode_tokens)")
-    ap.add_argument("--e2e-slices", type=int, default=0,
-                    help="e2e leg (linear workloads): overlap the host copies with the compute "
-                         "over N batch slices (hostio.linear_fwd_host)")
+    ap.add_argument("--e2e-slices", type=int, default=None,
+                    help="e2e leg (linear and large-chunk workloads): overlap the host copies with "
+                         "the compute over N batch slices (hostio.linear_fwd_host, "
+                         "hostio.chunk_fwd_host); default 4, 0 = copies in series with one call")
     ap.add_argument("--segments", type=int, default=0,
                     help="time the large-chunk forward split into N segments per sequence")
     ap.add_argument("--mlp-kernel", default="default", choices=["default", "tcgen05"],

@@ -1,5 +1,5 @@
-"""TTT-Linear forward on inputs that live in host memory, with the copies
-overlapped with the compute.
+"""TTT-Linear and large-chunk forwards on inputs that live in host memory,
+with the copies overlapped with the compute.
 
 The batch is cut into `slices` groups of whole batch rows (every group holds
 all heads of its rows, so a shared W0 [H, d, d] serves every group). Each
@@ -8,7 +8,8 @@ device, ttt_linear_fwd runs on them, and its Z and W_out are copied back. The
 host-to-device copies of later groups, the device-to-host copies of earlier
 ones and the kernels of the groups in between then proceed at the same time.
 A sequence's result does not depend on which other sequences share its call,
-so the outputs equal those of one ttt_linear_fwd call over the whole batch.
+so the outputs equal those of one ttt_linear_fwd (ttt_chunk_fwd) call over
+the whole batch.
 
 Host tensors must be in pinned (page-locked) memory for the copies to run
 asynchronously. torch provides the memory, the streams and the copies; every
@@ -42,13 +43,26 @@ def _bounds(B: int, slices: int):
     return out
 
 
+def _outputs(Q, z_bf16, out):
+    """(Z, W_out) pinned host tensors: the caller's `out` pair, else new ones."""
+    import torch
+    if out is not None:
+        return out
+    B, H, T, d = Q.shape
+    Zh = torch.empty((B, H, T, d), dtype=torch.bfloat16 if z_bf16 else torch.float32,
+                     pin_memory=True)
+    Wh = torch.empty((B, H, d, d), dtype=torch.float32, pin_memory=True)
+    return Zh, Wh
+
+
 def linear_fwd_host(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, slices=4,
-                    z_bf16=False, device=None):
+                    z_bf16=False, device=None, out=None):
     """TTT-Linear forward of host tensors Q, K, V [B, H, T, d] (bf16 or fp32)
     and eta [B, H, T]; W0 [H, d, d] and the LayerNorm gain and bias [H, d] may
-    be on the host or the device. Returns (Z, W_out) as pinned host tensors,
-    valid once torch's current stream has reached the point of return (for
-    example after torch.cuda.current_stream().synchronize())."""
+    be on the host or the device. Returns (Z, W_out) as pinned host tensors
+    (`out`, a pinned (Z, W_out) pair of the right shapes, if given), valid once
+    torch's current stream has reached the point of return (for example after
+    torch.cuda.current_stream().synchronize())."""
     import torch
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     B, H, T, d = Q.shape
@@ -56,9 +70,7 @@ def linear_fwd_host(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, sli
     W0d = W0.to(dev, non_blocking=True)
     gd = ln_gamma.to(dev, non_blocking=True) if ln_gamma is not None else None
     bd = ln_beta.to(dev, non_blocking=True) if ln_beta is not None else None
-    Zh = torch.empty((B, H, T, d), dtype=torch.bfloat16 if z_bf16 else torch.float32,
-                     pin_memory=True)
-    Wh = torch.empty((B, H, d, d), dtype=torch.float32, pin_memory=True)
+    Zh, Wh = _outputs(Q, z_bf16, out)
     bounds = _bounds(B, slices)
     streams = _streams(dev, len(bounds))
     for (b0, b1), st in zip(bounds, streams):
@@ -66,6 +78,36 @@ def linear_fwd_host(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, sli
         with torch.cuda.stream(st):
             q, k, v, e = (x[b0:b1].to(dev, non_blocking=True) for x in (Q, K, V, eta))
             Z, W = _lib.linear_fwd(q, k, v, e, W0d, gd, bd, b=b, ln=ln, stream=st, z_bf16=z_bf16)
+            Zh[b0:b1].copy_(Z, non_blocking=True)
+            Wh[b0:b1].copy_(W, non_blocking=True)
+    for st in streams:
+        cur.wait_stream(st)
+    return Zh, Wh
+
+
+def chunk_fwd_host(Q, K, V, eta, W0, *, chunk, slices=4, w0_per_seq=False, z_bf16=False,
+                   device=None, out=None):
+    """Large-chunk forward of host tensors Q, K, V [B, H, T, d] and eta
+    [B, H, T]; W0 ([H, d, d], or [B, H, d, d] with w0_per_seq) on the host or
+    the device. Each group of batch rows gets its own workspace (allocated by
+    torch on its stream), so the groups' kernels may overlap. Returns (Z, W_out)
+    as pinned host tensors (`out` if given), valid once torch's current stream
+    has reached the point of return."""
+    import torch
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    B = Q.shape[0]
+    cur = torch.cuda.current_stream(dev)
+    W0d = W0.to(dev, non_blocking=True)
+    Zh, Wh = _outputs(Q, z_bf16, out)
+    bounds = _bounds(B, slices)
+    streams = _streams(dev, len(bounds))
+    for (b0, b1), st in zip(bounds, streams):
+        st.wait_stream(cur)  # W0 is copied on the current stream
+        with torch.cuda.stream(st):
+            q, k, v, e = (x[b0:b1].to(dev, non_blocking=True) for x in (Q, K, V, eta))
+            w0 = W0d[b0:b1] if w0_per_seq else W0d
+            Z, W = _lib.chunk_fwd(q, k, v, e, w0, chunk=chunk, w0_per_seq=w0_per_seq, stream=st,
+                                  z_bf16=z_bf16)
             Zh[b0:b1].copy_(Z, non_blocking=True)
             Wh[b0:b1].copy_(W, non_blocking=True)
     for st in streams:

@@ -29,3 +29,28 @@ def test_host_pipeline_equals_device_call(B, slices, z_bf16, ln):
     assert ttt.ttt_device_status() == 0
     assert Zh.is_pinned() and Wh.is_pinned()
     assert torch.equal(Zh, Zd.cpu()) and torch.equal(Wh, Wd.cpu())
+
+
+C = synth.WORKLOADS["chunk_d128_c2048_b4h8_t32768"]
+
+
+@pytest.mark.parametrize("B,slices,z_bf16,per_seq", [(3, 3, False, False), (4, 2, True, False),
+                                                    (2, 2, False, True)])
+def test_chunk_host_pipeline_equals_device_call(B, slices, z_bf16, per_seq):
+    """Large-chunk forward from pinned host buffers, one workspace per slice,
+    outputs written into caller-given pinned buffers: equal to one
+    ttt_chunk_fwd call on the device, bit for bit."""
+    wl = C.scaled(B=B, H=2, T=1024, b=256)
+    x = to_dev(synth.make_inputs(wl))
+    W0 = x["W1"].unsqueeze(0).repeat(B, 1, 1, 1) if per_seq else x["W1"]
+    Zd, Wd = ttt.chunk_fwd(x["Q"], x["K"], x["V"], x["eta"], W0, chunk=wl.b, w0_per_seq=per_seq,
+                           z_bf16=z_bf16)
+    h = {k: x[k].cpu().pin_memory() for k in ("Q", "K", "V", "eta")}
+    out = (torch.empty(tuple(Zd.shape), dtype=Zd.dtype, pin_memory=True),
+           torch.empty(tuple(Wd.shape), dtype=torch.float32, pin_memory=True))
+    Zh, Wh = hostio.chunk_fwd_host(h["Q"], h["K"], h["V"], h["eta"], W0.cpu(), chunk=wl.b,
+                                   slices=slices, w0_per_seq=per_seq, z_bf16=z_bf16, out=out)
+    torch.cuda.current_stream().synchronize()
+    assert ttt.ttt_device_status() == 0
+    assert Zh is out[0] and Wh is out[1]
+    assert torch.equal(Zh, Zd.cpu()) and torch.equal(Wh, Wd.cpu())
