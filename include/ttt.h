@@ -320,7 +320,7 @@ TTT_API ttt_status ttt_mlp_bwd(const void *Q, const void *K, const void *V, cons
  * gradient descent on the chunk's mean loss.
  * Arguments as ttt_linear_fwd without LayerNorm; `chunk` is the chunk length.
  * workspace: device scratch of at least ttt_chunk_workspace_bytes(...) bytes
- *   (192 KiB per chunk of every sequence when d = 128, plus 8 bytes per chunk
+ *   (160 KiB per chunk of every sequence when d = 128, plus 8 bytes per chunk
  *   for its ready flag and read-out count and a ticket counter, rounded up to
  *   256 bytes; 0 for
  *   the shapes that need none, when workspace may be NULL), 256-byte aligned,
@@ -352,8 +352,8 @@ TTT_API ttt_status ttt_chunk_fwd(const void *Q, const void *K, const void *V, co
  * GPU that loads libttt.so holds that buffer until the process exits, and no
  * call of this function allocates or frees anything.
  *   - Limit: problems whose ttt_chunk_workspace_bytes(...) exceeds
- *     TTT_CHUNK_NOALLOC_SCRATCH_BYTES (24 MiB + 4 KiB: 128 chunks of d = 128
- *     with their ready flags) return
+ *     TTT_CHUNK_NOALLOC_SCRATCH_BYTES (24 MiB + 4 KiB: 153 chunks of d = 128
+ *     with their flags) return
  *     TTT_ERR_SCRATCH_LIMIT and launch nothing; use ttt_chunk_fwd with a
  *     caller-allocated workspace for them.
  *   - Every call looks up the buffer's device address on the current device

@@ -40,27 +40,26 @@ using namespace sm100;
 constexpr int kD = 128;
 constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: math/epilogue
 
-// Workspace per chunk: A_c as a bf16 hi | lo operand image (K-major, 32 KB
-// each) and B_c in fp32 (64 KB; column quad q of row i at float4 q * 128 + i);
-// after all chunks, each W_c as the apply kernel's bf16 hi | lo image
-// (MN-major, 64 KB); then the ticket counter and the chunks' ready flags.
+// Workspace per chunk: A_c as a bf16 operand image (K-major, 32 KB; the scan
+// takes A_c's rounded-to-nearest bf16 term only) and B_c in fp32 (64 KB;
+// column quad q of row i at float4 q * 128 + i); after all chunks, each W_c
+// as the read-out's bf16 hi | lo image (64 KB, layout at the read-out role);
+// then the ticket counter, the chunks' ready flags and read-out counts.
 constexpr int kImgBytes = kD * kD * 2;            // one bf16 128 x 128 image
-constexpr int kChunkWs = 2 * kImgBytes + kD * kD * 4;
+constexpr int kChunkWs = kImgBytes + kD * kD * 4;
 
 // ---------------------------------------------------------------------------
-// 1 + 2. gram and scan in one launch. Each block takes a ticket from a
-// counter in the workspace (tickets follow the order in which blocks start)
-// and from it a role:
-//   tickets [0, n):  gram of one chunk, chunks in chunk-major order (chunk 0 of
-//     every sequence first): A_c | B_c = (diag(eta) K_c)^T [K_c | V_c], then a
-//     ready flag for the chunk;
-//   tickets [n, n + 4 S): scan of one 32-column slice of one sequence's
-//     weight: W_{c+1}[:, j] = W_c[:, j] - A_c W_c[:, j] + B_c[:, j] (columns of
-//     W evolve independently), waiting on each chunk's ready flag.
-// A scan block only ever waits on gram blocks; every gram block started
-// before any scan block (smaller ticket) and waits on nothing, so the wait
-// always ends. The scans run while the last grams stream, instead of after
-// them.
+// One launch, three block roles by ticket (a counter in the workspace;
+// tickets follow the order in which blocks start):
+//   tickets [0, n): Gram of one chunk, chunk-major (chunk 0 of every sequence
+//     first): A_c | B_c = (diag(eta) K_c)^T [K_c | V_c], then a ready flag;
+//   next 2 per sequence (4 in map mode): scan of one 64-column slice of one
+//     sequence's weight, W_{c+1}[:, j] = W_c[:, j] - A_c W_c[:, j] + B_c[:, j]
+//     (columns of W evolve independently), waiting on each chunk's flag;
+//   the rest (forward only): read-out of part of one chunk, waiting on the
+//     count of scan slices that have stored W_c.
+// Every wait is on blocks with smaller tickets, which have started and wait
+// only on blocks before them, so the waits always end.
 constexpr int kGramRows = 32;                    // tokens per pipeline stage
 constexpr int kGramStages = 4;
 constexpr int kGramBox = kGramRows * 128;        // one 64-column box of a stage (4 KB)
@@ -431,33 +430,28 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mbar_arrive(&conv[st]);
             }
             // Epilogue: lanes are d_in rows i. A_c goes out as the scan's bf16
-            // hi/lo operand image (K-major, 128-byte swizzle: row i = 128 bytes
-            // per 64 columns j), B_c as fp32 rows. (__all_sync reconverges the
-            // warp for the warp-collective TMEM loads.)
+            // operand image (K-major, 128-byte swizzle: row i = 128 bytes per
+            // 64 columns j), B_c as fp32 rows; two accumulator loads per wait.
+            // (__all_sync reconverges the warp for the warp-collective TMEM
+            // loads.)
             if (__all_sync(0xffffffffu, mbar_wait(done, 0, &abort_flag, a.status, 14))) {
                 tc_fence_after();
                 const int sp = warp & 3;
                 const int row = 32 * sp + lane;
                 uint8_t *blk = a.ws + (size_t)g * kChunkWs;
-                float4 *bdst = reinterpret_cast<float4 *>(blk + 2 * kImgBytes);
+                float4 *bdst = reinterpret_cast<float4 *>(blk + kImgBytes);
                 const float scale = uniform ? eta0 : 1.f;
-                for (int q = 0; q < 16; ++q) {
-                    float v[16];
-                    tmem_ld16(taddr(tm, 32 * sp, 16 * q), v);
-                    tmem_ld_wait();
+                auto emit16 = [&](int q, float (&v)[16]) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) v[e] *= scale;
                     if (q < 8) {
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            uint4 hi, lo;
+                            uint4 hi;
                             __nv_bfloat16 *hb = reinterpret_cast<__nv_bfloat16 *>(&hi);
-                            __nv_bfloat16 *lb = reinterpret_cast<__nv_bfloat16 *>(&lo);
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) split_bf16(v[8 * h + e], hb[e], lb[e]);
-                            const uint32_t off = off_kmajor_sw128(row, 16 * q + 8 * h, kD);
-                            *reinterpret_cast<uint4 *>(blk + off) = hi;
-                            *reinterpret_cast<uint4 *>(blk + kImgBytes + off) = lo;
+                            for (int e = 0; e < 8; ++e) hb[e] = __float2bfloat16_rn(v[8 * h + e]);
+                            *reinterpret_cast<uint4 *>(blk + off_kmajor_sw128(row, 16 * q + 8 * h, kD)) = hi;
                         }
                     } else {  // B_c: column quad q4 of row i at float4 q4 * 128 + i
 #pragma unroll
@@ -465,6 +459,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                             bdst[(4 * (q - 8) + i) * kD + row] =
                                 make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                     }
+                };
+                for (int q = 0; q < 16; q += 2) {
+                    float v0[16], v1[16];
+                    tmem_ld16(taddr(tm, 32 * sp, 16 * q), v0);
+                    tmem_ld16(taddr(tm, 32 * sp, 16 * q + 16), v1);
+                    tmem_ld_wait();
+                    emit16(q, v0);
+                    emit16(q + 1, v1);
                 }
                 __threadfence();  // ordered before the chunk's ready flag
             }
@@ -544,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         auto prefetch = [&](int c) {
             const uint8_t *blk = a.ws + (g0 + c) * kChunkWs;
             bulk_prefetch_l2(blk, kImgBytes);
-            bulk_prefetch_l2(blk + 2 * kImgBytes + (size_t)j0 * kD * 4, kImgBytes);
+            bulk_prefetch_l2(blk + kImgBytes + (size_t)j0 * kD * 4, kImgBytes);
         };
         int prefetched = 0;  // chunks [0, prefetched) are prefetched
         for (int c = 0; c < cps; ++c) {
@@ -563,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             issued = 2 * c + 1;
             if (c >= 1 && !mbar_wait(bfree, (c - 1) & 1, &abort_flag, a.status, 16)) break;
             mbar_arrive_expect_tx(bready, kImgBytes);
-            bulk_load(sB, blk + 2 * kImgBytes + (size_t)j0 * kD * 4, kImgBytes, bready);
+            bulk_load(sB, blk + kImgBytes + (size_t)j0 * kD * 4, kImgBytes, bready);
             issued = 2 * c + 2;
         }
     } else if (warp == 1 && lane == 0) {

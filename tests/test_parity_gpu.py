@@ -310,7 +310,7 @@ def test_chunk_rejects_small_workspace():
     Z = torch.empty((wl.B, wl.H, wl.T, wl.d), device="cuda")
     need = ttt.ttt_chunk_workspace_bytes(wl.B, wl.H, wl.T, wl.d, wl.b)
     n = wl.B * wl.H * (wl.T // wl.b)
-    assert need == n * 192 * 1024 + 256  # per chunk 192 KiB; ready flags and counter: 256 B
+    assert need == n * 160 * 1024 + 256  # per chunk 160 KiB; flags, counts and counter: 256 B
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     args = (x["Q"], x["K"], x["V"], x["eta"], x["W1"], Z, None, wl.B, wl.H, wl.T, wl.d, wl.b,
             ttt.TTT_BF16, 0)

@@ -55,7 +55,7 @@ def test_noalloc_matches_workspace_entry_point_twice():
 
 def test_noalloc_refuses_problems_beyond_its_buffer():
     wl, x = _case(5)
-    big_T = 129 * 256  # 2 * 3 * 129 chunks of 192 KiB > 24 MiB + 4 KiB
+    big_T = 129 * 256  # 2 * 3 * 129 chunks of 160 KiB > 24 MiB + 4 KiB
     Z = torch.empty(1, device="cuda")
     n0 = ttt.ttt_launch_count()
     rc = ttt.ttt_chunk_fwd_noalloc(x["Q"], x["K"], x["V"], x["eta"], x["W1"], Z, None, wl.B,
