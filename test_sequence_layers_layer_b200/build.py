@@ -23,6 +23,9 @@ NVCC_FLAGS = [
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
     "-I", INCLUDE, "-I", CSRC,
 ]
+# Extra preprocessor definitions for a profiling build, e.g. TTT_NVCC_DEFINES=TTT_TRACE
+# (the TTT-Linear scan's phase trace, read by trace_linear.py). Rebuild with --force.
+NVCC_FLAGS += ["-D" + d for d in os.environ.get("TTT_NVCC_DEFINES", "").split()]
 
 
 def _deps_mtime() -> float:

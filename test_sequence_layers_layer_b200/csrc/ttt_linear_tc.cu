@@ -436,6 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (j > 0) {  // X_j = P_j - C_j G_{j-1}: coefficients in registers, two chains
                 // G_{j-1} comes from all four scan warps: wait for all of it.
                 if (!mbar_wait_warp(&gready[(j - 1) & 3], ((j - 1) >> 2) & 1, abrt, status, 44)) break;
+                if (threadIdx.x == 128) TRACE(21, j);
                 const float4 *c4 = reinterpret_cast<const float4 *>(Cf + ((j & 1) * 16 + t) * kCStride);
                 float c[16];
 #pragma unroll
@@ -478,6 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 float mu, rstd;
                 row_stats(x, mu, rstd);
+                if (threadIdx.x == 128) TRACE(24, j);
                 float xh[8], gh[8], s1 = 0.f, s2 = 0.f;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -505,6 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float *gf = Gf + (j & 3) * 1024 + t * kD;
             *reinterpret_cast<float4 *>(gf + 4 * g) = make_float4(G[0], G[1], G[2], G[3]);
             *reinterpret_cast<float4 *>(gf + 32 + 4 * g) = make_float4(G[4], G[5], G[6], G[7]);
+            if (threadIdx.x == 128) TRACE(25, j);
             // -G as bf16 hi + lo, MN-major (rows = tokens, 128-byte swizzle)
             uint8_t *gb = sG + (j & 1) * 4096;
 #pragma unroll
@@ -519,7 +522,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint2 *>(gb + off) = hi;
                 *reinterpret_cast<uint2 *>(gb + 2048 + off) = lo;
             }
+            if (threadIdx.x == 128) TRACE(26, j);
             fence_async_smem();
+            if (threadIdx.x == 128) TRACE(27, j);
             mbar_arrive(&gready[j & 3]);
             if (threadIdx.x == 128) TRACE(8, j);
         }
