@@ -877,9 +877,12 @@ def backward_arm(args, wl):
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     ms = sum(step_ms) / args.steps
     # the large-chunk FLOP count covers all three kernels, so it is divided by
-    # their summed time
+    # their summed time (against the fp32 CUDA-core peak; the Gram kernel runs
+    # on the tensor cores for d = 128 with bf16 inputs)
     kern_ms = (sum(kern) if chunk else kern[0]) / args.steps
-    knames = (["cb_gram_kernel", "cb_scan_kernel", "cb_tok_kernel", "cb_sum_over_batch_kernel (dW0)"]
+    gram_name = ("cb_gram_tc_kernel" if wl.d == 128 and wl.dtype == "bf16" and wl.b % 32 == 0
+                 else "cb_gram_kernel")
+    knames = ([gram_name, "cb_scan_kernel", "cb_tok_kernel", "cb_sum_over_batch_kernel (dW0)"]
               if chunk else ["mlp_bwd_kernel", "mlp_bwd_sum_kernel"] if mlp
               else ["linear_bwd_kernel", "sum_over_batch_kernel (dW0)",
                     "sum_over_batch_kernel (dgamma)", "sum_over_batch_kernel (dbeta)"])

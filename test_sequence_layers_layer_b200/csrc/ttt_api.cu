@@ -83,8 +83,10 @@ int *device_status_word() {
     return p;
 }
 
-bool encode_tmap_bf16_2d(void *map, const void *base, uint64_t cols, uint64_t rows,
-                         uint32_t box_cols, uint32_t box_rows) {
+// 2-D TMA descriptor over a row-major [rows][cols] bf16 (or fp32) tensor,
+// box of box_rows x box_cols elements, 128-byte swizzle.
+bool encode_tmap_2d(void *map, const void *base, bool f32, uint64_t cols, uint64_t rows,
+                    uint32_t box_cols, uint32_t box_rows) {
     using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -100,13 +102,19 @@ bool encode_tmap_bf16_2d(void *map, const void *base, uint64_t cols, uint64_t ro
         fn = reinterpret_cast<EncodeFn>(p);
     }
     const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint64_t strides[1] = {cols * (f32 ? 4 : 2)};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(static_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+    return fn(static_cast<CUtensorMap *>(map),
+              f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_tmap_bf16_2d(void *map, const void *base, uint64_t cols, uint64_t rows,
+                         uint32_t box_cols, uint32_t box_rows) {
+    return encode_tmap_2d(map, base, false, cols, rows, box_cols, box_rows);
 }
 
 namespace {

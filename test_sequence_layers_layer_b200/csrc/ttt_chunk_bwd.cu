@@ -17,13 +17,22 @@
 // forward's: per-chunk Gram products (A_c, B_c, D_c) in parallel, one scan per
 // sequence in each direction (W_c forward, Om_{c+1} backward), and the
 // per-token gradients of every chunk in parallel from W_c and Om_{c+1}.
+#include <type_traits>
+
 #include "../../include/ttt.h"
 #include "ttt_common.cuh"
 
 namespace ttt {
+
+// ttt_chunk_bwd_tc.cu
+bool chunk_bwd_gram_tc_supported(int d, int chunk, bool bf16);
+cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V, const float *eta,
+                                     const float *dZ, int B, int H, int T, int chunk, float *gram,
+                                     cudaStream_t s);
+
 namespace {
 
-constexpr int kT = 256;  // threads per block in every kernel here
+constexpr int kT = 256;  // threads per block in every kernel here (CUDA-core path)
 
 template <typename T>
 __device__ __forceinline__ float ldv(const T *p, size_t i);
@@ -290,11 +299,17 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
     const WsView w = ws_view(static_cast<float *>(workspace), nch, S, D);
     const TIn *q = static_cast<const TIn *>(Q), *k = static_cast<const TIn *>(K),
               *v = static_cast<const TIn *>(V);
-    cb_gram_kernel<TIn, D><<<dim3((unsigned)nch, 3, (D / 64) * (D / 64)), kT, 0, s>>>(
-        q, k, v, eta, dZ, T, C, w.gram);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    count_launch(s);
+    cudaError_t e;
+    if (std::is_same<TIn, __nv_bfloat16>::value && chunk_bwd_gram_tc_supported(D, C, true)) {
+        // d = 128, bf16: the Gram products on the tensor cores
+        if ((e = launch_chunk_bwd_gram_tc(Q, K, V, eta, dZ, B, H, T, C, w.gram, s)) != cudaSuccess)
+            return e;
+    } else {
+        cb_gram_kernel<TIn, D><<<dim3((unsigned)nch, 3, (D / 64) * (D / 64)), kT, 0, s>>>(
+            q, k, v, eta, dZ, T, C, w.gram);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        count_launch(s);
+    }
     const size_t scan_smem = (size_t)D * D * sizeof(float);
     if ((e = cudaFuncSetAttribute(cb_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)scan_smem)) != cudaSuccess)

@@ -131,6 +131,12 @@ CHUNK_CASES = {
     "chunk_fp32_d64_c32": (dict(B=2, H=2, T=128, d=64, b=32, dtype="fp32"), False, True),
     "chunk_bf16_d128_c64": (dict(B=1, H=2, T=256, d=128, b=64), False, False),
     "chunk_fp32_d128_c128_w0seq": (dict(B=2, H=1, T=256, d=128, b=128, dtype="fp32"), True, True),
+    # d = 128, bf16: the Gram products on the tensor cores (one eta per chunk:
+    # raw K with eta on the fp32 accumulator; a varying eta: eta K as hi + lo)
+    "chunk_bf16_d128_c64_eta_varied": (dict(B=1, H=2, T=256, d=128, b=64, eta="sigmoid_over_d"),
+                                       False, True),
+    "chunk_bf16_d128_c128_w0seq": (dict(B=2, H=1, T=512, d=128, b=128), True, True),
+    "chunk_bf16_d128_c32_one_chunk": (dict(B=1, H=3, T=32, d=128, b=32), False, True),
 }
 
 
