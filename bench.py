@@ -488,17 +488,24 @@ def gpu_arm(args, wl, rank, world, keep=None):
 
 # ----------------------------------------------------------------------------- CPU (oracle) arm
 
-def oracle_sample(wl, budget_s: float, keep=None):
+def oracle_inputs(wl):
+    """The workload's seeded inputs as float64 arrays, the oracle's input form."""
+    inp = synth.make_inputs(wl)
+    return {k: (np.asarray(getattr(inp, k), dtype=np.float64) if getattr(inp, k) is not None else None)
+            for k in ("Q", "K", "V", "eta", "W1", "W2", "gamma", "beta")}
+
+
+def oracle_sample(wl, budget_s: float, keep=None, f64=None):
     """Time the oracle on whole sequences of the workload, threaded over the
     host cores, growing the sample until about budget_s of work or the whole
     workload. Returns (tokens/s, cores, description); with `keep` (a dict),
     also leaves there the sampled sequences ("seqs") and the oracle's outputs
-    of the last, largest sample ("ref")."""
+    of the last, largest sample ("ref"). `f64`: the inputs from
+    oracle_inputs(wl), made here if not given (not part of the timing)."""
     import oracle
 
-    inp = synth.make_inputs(wl)
-    f64 = {k: (np.asarray(getattr(inp, k), dtype=np.float64) if getattr(inp, k) is not None else None)
-           for k in ("Q", "K", "V", "eta", "W1", "W2", "gamma", "beta")}
+    if f64 is None:
+        f64 = oracle_inputs(wl)
     cores = oracle.num_threads()
     nseq_total = wl.B * wl.H
 
@@ -554,8 +561,9 @@ def reference_arm(args, wl):
     vals = []
     cores, desc = None, None
     per_step_budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    f64 = oracle_inputs(wl)  # once: every step times the oracle on the same inputs
     for k in range(args.warmup + args.steps):
-        v, cores, desc = oracle_sample(wl, per_step_budget)
+        v, cores, desc = oracle_sample(wl, per_step_budget, f64=f64)
         if k >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
