@@ -19,12 +19,13 @@
 //             its chunk is published, writing each W_c as the ready-made bf16
 //             hi/lo operand image of the read-out;
 //   read-out: Z_c = Q_c W_c once both slices of W_c are written (the only
-//             pass over Q and the only write of Z; tcgen05, M = 64 tokens,
-//             N = 256 = hi | lo side by side, K = d_in; W_c arrives by one
-//             bulk copy). Their HBM traffic overlaps the Gram's.
+//             pass over Q and the only write of Z), as Z_c^T = W_c^T Q_c^T on
+//             tcgen05: M = d_out = 128 with W_c^T (hi and lo terms) as the A
+//             operand in tensor memory, N = 128 tokens per tile, K = d_in.
+//             Their HBM traffic overlaps the Gram's.
 // Q/K/V tiles arrive by TMA with the 128-byte swizzle; accumulators live in
-// tensor memory. W_c enters the apply products as two bf16 terms (hi + lo)
-// so the read-out keeps ~16 significant bits of the fp32 state.
+// tensor memory. W_c enters the read-out as two bf16 terms (hi + lo) so it
+// keeps ~16 significant bits of the fp32 state.
 
 #include <algorithm>
 
