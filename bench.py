@@ -884,13 +884,15 @@ def backward_arm(args, wl):
         raise RuntimeError("device status error in the timed region")
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     ms = sum(step_ms) / args.steps
-    # the large-chunk FLOP count covers all three kernels, so it is divided by
-    # their summed time (against the fp32 CUDA-core peak; the Gram kernel runs
-    # on the tensor cores for d = 128 with bf16 inputs)
+    # the large-chunk FLOP count covers all its kernels, so it is divided by
+    # their summed time
     kern_ms = (sum(kern) if chunk else kern[0]) / args.steps
-    gram_name = ("cb_gram_tc_kernel" if wl.d == 128 and wl.dtype == "bf16" and wl.b % 32 == 0
-                 else "cb_gram_kernel")
-    knames = ([gram_name, "cb_scan_kernel", "cb_tok_kernel", "cb_sum_over_batch_kernel (dW0)"]
+    tc_gram = chunk and wl.d == 128 and wl.dtype == "bf16" and wl.b % 32 == 0
+    tc_tok = tc_gram and wl.b % 128 == 0
+    chunk_names = (["cb_gram_tc_kernel" if tc_gram else "cb_gram_kernel", "cb_scan_kernel"]
+                   + (["cb_tok_tc_kernel<RP>", "cb_tok_tc_kernel<DK>", "cb_tok_tc_kernel<DQ>"]
+                      if tc_tok else ["cb_tok_kernel"]) + ["cb_sum_over_batch_kernel (dW0)"])
+    knames = (chunk_names
               if chunk else ["mlp_bwd_kernel", "mlp_bwd_sum_kernel"] if mlp
               else ["linear_bwd_kernel", "sum_over_batch_kernel (dW0)",
                     "sum_over_batch_kernel (dgamma)", "sum_over_batch_kernel (dbeta)"])
@@ -916,11 +918,30 @@ def backward_arm(args, wl):
                      "peak_source": f"derived: {FP32_LANES} fp32 lanes x 2 FLOP x {mhz} MHz",
                      "algorithmic_per_launch": flop, "kernel_ms": kern_ms,
                      "hbm_bytes_per_token": None if mlp else bwd_bytes_per_token(wl)},
+    }
+    # With the products on the tensor cores the fp32 ALU roofline no longer
+    # bounds the call: the unavoidable HBM traffic against the copy peak.
+    if tc_tok:
+        peaks, peaks_src = load_peaks()
+        hb = bwd_bytes_per_token(wl) * wl.tokens
+        ach = hb / (kern_ms / 1e3) / 1e9
+        line_roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "all backward kernels", "peak_source": peaks_src,
+                     "algorithmic_per_launch": hb, "kernel_ms": kern_ms,
+                     "note": ("Gram and per-token products on the tensor cores; bytes are the "
+                              "inputs and gradients only (not the workspace round trips)"),
+                     "tflops_algorithmic": achieved}
+    else:
+        line_roof = None
+    line.update({
         "kernels": [{"name": n, "ms_per_launch": t / args.steps} for n, t in zip(knames, kern)],
         "gpu_launches": launches,
         "clocks": clocks,
         "step_ms_min_median": [min(step_ms), statistics.median(step_ms)],
-    }
+    })
+    if line_roof is not None:
+        line["roofline"] = line_roof
     if not args.no_cpu_baseline and mlp:
         from oracle import backward as ob
         sub = wl.scaled(B=1, H=1, T=min(wl.T, 4 * wl.b))

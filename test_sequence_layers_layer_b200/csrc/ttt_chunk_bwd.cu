@@ -29,6 +29,12 @@ bool chunk_bwd_gram_tc_supported(int d, int chunk, bool bf16);
 cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V, const float *eta,
                                      const float *dZ, int B, int H, int T, int chunk, float *gram,
                                      cudaStream_t s);
+bool chunk_bwd_tok_tc_supported(int d, int chunk, bool bf16);
+size_t chunk_bwd_tok_tc_scratch_bytes(size_t tokens);
+cudaError_t launch_chunk_bwd_tok_tc(const void *K, const void *V, const float *eta, const float *dZ,
+                                    const float *W, const float *Om, int B, int H, int T, int chunk,
+                                    void *scratch, float *dQ, float *dK, float *dV, float *deta,
+                                    cudaStream_t s);
 
 namespace {
 
@@ -319,13 +325,24 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
                                                                   dW0_seq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launch(s);
-    const size_t tsm = tok_smem_bytes(D);
-    if ((e = cudaFuncSetAttribute(cb_tok_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)tsm)) != cudaSuccess)
-        return e;
-    cb_tok_kernel<TIn, D><<<(unsigned)nch, kT, tsm, s>>>(k, v, eta, dZ, T, C, w, dQ, dK, dV, deta);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    count_launch(s);
+    if (std::is_same<TIn, __nv_bfloat16>::value && chunk_bwd_tok_tc_supported(D, C, true)) {
+        // d = 128, bf16, chunk % 128 == 0: the per-token products on the tensor
+        // cores; their bf16 operand rows follow the fp32 part of the workspace
+        void *scratch = reinterpret_cast<float *>(workspace) + (5 * nch + S) * (size_t)D * D;
+        if ((e = launch_chunk_bwd_tok_tc(K, V, eta, dZ, w.W, w.Om, B, H, T, C, scratch, dQ, dK, dV,
+                                         deta, s)) != cudaSuccess)
+            return e;
+    } else {
+        const size_t tsm = tok_smem_bytes(D);
+        if ((e = cudaFuncSetAttribute(cb_tok_kernel<TIn, D>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm)) !=
+            cudaSuccess)
+            return e;
+        cb_tok_kernel<TIn, D><<<(unsigned)nch, kT, tsm, s>>>(k, v, eta, dZ, T, C, w, dQ, dK, dV,
+                                                             deta);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        count_launch(s);
+    }
     if (!w0_per_seq) {
         cb_sum_over_batch_kernel<<<H, 256, 0, s>>>(w.dW0s, dW0, B, H, D * D);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -344,7 +361,11 @@ size_t chunk_bwd_workspace_bytes(int B, int H, int T, int d, int chunk) {
     if (B <= 0 || H <= 0 || T <= 0 || chunk <= 0 || T % chunk || !chunk_bwd_supported(d, chunk))
         return 0;
     const size_t S = (size_t)B * H, nch = S * (T / chunk), dd = (size_t)d * d;
-    return sizeof(float) * (5 * nch * dd + S * dd);
+    // d = 128, chunk % 128 == 0: the tensor-core token passes' operand rows
+    // (used with bf16 inputs; the size does not depend on the dtype)
+    const size_t tc = chunk_bwd_tok_tc_supported(d, chunk, true)
+                          ? chunk_bwd_tok_tc_scratch_bytes(S * (size_t)T) : 0;
+    return sizeof(float) * (5 * nch * dd + S * dd) + tc;
 }
 
 cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const float *eta,

@@ -264,4 +264,344 @@ cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V
     return cudaSuccess;
 }
 
+
+// ---------------------------------------------------------------------------
+// Per-token gradients of the large-chunk backward on the tensor cores (d =
+// 128, bf16 inputs, chunk a multiple of 128), with W = W_c and Om = Om_{c+1}
+// of each token's chunk:
+//   R = K W - V,  P = K Om,  dV = diag(eta) P,  deta_t = -P_t . R_t,
+//   dK = -diag(eta) [R | P] [Om | W]^T,  dQ = dZ W^T,
+// as three passes of one kernel over 128-token tiles, a block per chunk:
+//   RP: D = K [W | Om] (N = 256, K = d_in): A = K (exact), B = [W | Om]^T as
+//       hi and lo terms; the epilogue forms R, dV, deta and writes R, P (and
+//       dZ) as bf16 hi/lo operand rows into the workspace;
+//   DK: D = [R | P]_{hi,lo} [Om | W]^T (K = 256);  DQ: D = dZ_{hi,lo} W^T (K = 128):
+//       B stacked as [hi rows | lo rows] (N = 256), so A_hi x B gives the hi.hi
+//       and hi.lo terms side by side and A_lo x B_hi adds lo.hi to the first half.
+// A tiles arrive by TMA one 64-wide K block at a time (3-stage ring); B is
+// built once per block in shared memory from the fp32 W and Om (K-major,
+// 128-byte swizzle); accumulators double-buffered in tensor memory.
+namespace {
+
+enum { kModeRP = 0, kModeDK = 1, kModeDQ = 2 };
+constexpr int kTokTile = 128, kTokThreads = 192, kTokStages = 3;
+constexpr int kTokStage = 2 * kTokTile * 128;            // A hi | lo for one 64-wide K block: 32 KB
+constexpr int kTokBBytes = 4 * 2 * kD * 128;             // up to 4 K blocks x 256 rows: 128 KB
+constexpr size_t kTokSmem = 1024 + kTokBBytes + kTokStages * kTokStage;  // 225 KB
+static_assert(kTokSmem <= 232448, "shared memory budget");
+
+struct TokArgs {
+    const float *W, *Om;  // per chunk [d][d] fp32, row-major [i][j]
+    const __nv_bfloat16 *V;
+    const float *eta, *dZ;
+    float *out;           // RP: dV; DK: dK; DQ: dQ   ([tokens][d] fp32)
+    float *deta;          // RP only
+    __nv_bfloat16 *rp_hi, *rp_lo, *z_hi, *z_lo;  // RP writes them; DK and DQ read them by TMA
+    int chunk;
+    int *status;
+};
+
+// Byte offset of element (n, k) in a K-major, 128-byte-swizzled image of
+// `rows` rows per 64-wide K block.
+__device__ __forceinline__ uint32_t kmajor_off(int n, int k, int rows) {
+    return (uint32_t)((k >> 6) * rows * 128 + n * 128 + ((((k & 63) >> 3) ^ (n & 7)) << 4) + (k & 7) * 2);
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kTokThreads, 1)
+    cb_tok_tc_kernel(const __grid_constant__ CUtensorMap tmA_hi, const __grid_constant__ CUtensorMap tmA_lo,
+                     TokArgs a) {
+    constexpr int KD = kMode == kModeDK ? 2 * kD : kD;  // reduction length
+    constexpr int NKB = KD / 64;                         // 64-wide K blocks per tile
+    constexpr bool kTwoA = kMode != kModeRP;             // A as hi and lo terms
+    // B image rows per K block: RP keeps hi and lo as two images of 256 rows
+    // ([W | Om]^T); DK and DQ stack [hi rows | lo rows] of their 128 rows.
+    constexpr int BR = 2 * kD;
+    constexpr uint32_t kBLoOff = kMode == kModeRP ? (uint32_t)NKB * BR * 128 : 0u;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sB = smem, *sA = smem + kTokBBytes;
+    __shared__ uint64_t full[kTokStages], empty[kTokStages], bready, tfull[2], tempty[2], drain;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = blockIdx.x;
+    const long row0 = (long)g * a.chunk;
+    const int ntile = a.chunk / kTokTile;
+    const size_t dd = (size_t)kD * kD;
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < kTokStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&bready, 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 128);
+        }
+        mbar_init(&drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&tmem_base, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_base;
+    int issued = 0;
+
+    if (warp == 0 && lane == 0) {
+        // A tiles, one K block per stage
+        for (int t = 0, u = 0; t < ntile; ++t) {
+            for (int kb = 0; kb < NKB; ++kb, ++u) {
+                const int st = u % kTokStages;
+                if (u >= kTokStages &&
+                    !mbar_wait(&empty[st], ((u / kTokStages) - 1) & 1, &abort_flag, a.status, 101))
+                    goto producer_done;
+                uint8_t *sb = sA + st * kTokStage;
+                const int y = (int)(row0 + (long)t * kTokTile);
+                mbar_arrive_expect_tx(&full[st], kTwoA ? kTokStage : kTokStage / 2);
+                tma_load_2d(sb, &tmA_hi, 64 * kb, y, &full[st]);
+                if (kTwoA) tma_load_2d(sb + kTokStage / 2, &tmA_lo, 64 * kb, y, &full[st]);
+                issued = u + 1;
+            }
+        }
+    producer_done:;
+    } else if (warp == 1 && lane == 0) {
+        const uint32_t id256 = make_idesc_bf16(128, 256, false, false);
+        const uint32_t id128 = make_idesc_bf16(128, 128, false, false);
+        const uint32_t bb = smem_u32(sB), ab = smem_u32(sA);
+        if (mbar_wait(&bready, 0, &abort_flag, a.status, 102)) {
+            for (int t = 0, u = 0; t < ntile; ++t) {
+                const int acc = t & 1;
+                if (t >= 2 && !mbar_wait(&tempty[acc], ((t >> 1) - 1) & 1, &abort_flag, a.status, 103))
+                    break;
+                tc_fence_after();
+                const uint32_t d = tm + 256 * acc;
+                bool ok = true;
+                for (int kb = 0; kb < NKB; ++kb, ++u) {
+                    const int st = u % kTokStages;
+                    if (!mbar_wait(&full[st], (u / kTokStages) & 1, &abort_flag, a.status, 104)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = ab + st * kTokStage;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t ko = (uint32_t)(16 * k * 2);
+                        const uint64_t ahi = make_sdesc(a0 + ko, 16, 1024, kSw128);
+                        const uint64_t bhi = make_sdesc(bb + kb * BR * 128 + ko, 16, 1024, kSw128);
+                        const bool accum = (kb | k) != 0;
+                        if (kMode == kModeRP) {
+                            const uint64_t blo = make_sdesc(bb + kBLoOff + kb * BR * 128 + ko, 16, 1024, kSw128);
+                            mma_bf16(d, ahi, bhi, id256, accum);
+                            mma_bf16(d, ahi, blo, id256, true);
+                        } else {
+                            const uint64_t alo = make_sdesc(a0 + kTokStage / 2 + ko, 16, 1024, kSw128);
+                            mma_bf16(d, ahi, bhi, id256, accum);  // hi.hi | hi.lo
+                            mma_bf16(d, alo, bhi, id128, true);   // + lo.hi (first half)
+                        }
+                    }
+                    mma_commit(&empty[st]);
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+            }
+        }
+    } else if (warp >= 2) {
+        const int tt = threadIdx.x - 64;  // 0..127
+        // ---- B operand images from the fp32 W and Om of the chunk
+        {
+            const float *Wc = a.W + (size_t)g * dd, *Oc = a.Om + (size_t)g * dd;
+            // units: (row n, 8 consecutive k)
+            constexpr int NROWS = kMode == kModeRP ? 2 * kD : kD;
+            for (int uidx = tt; uidx < NROWS * (KD / 8); uidx += 128) {
+                const int n = uidx / (KD / 8), k0 = 8 * (uidx % (KD / 8));
+                float f[8];
+                if (kMode == kModeRP) {
+                    // B[n][k]: n < 128: W[k][n]; else Om[k][n - 128]  (K = d_in)
+                    const float *src = n < kD ? Wc + n : Oc + (n - kD);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = src[(size_t)(k0 + e) * kD];
+                } else {
+                    // B[n][k]: DK: k < 128: Om[n][k], else W[n][k - 128]; DQ: W[n][k]
+                    const float *src = (kMode == kModeDK && k0 < kD) ? Oc + (size_t)n * kD + k0
+                                       : Wc + (size_t)n * kD + (k0 & (kD - 1));
+                    const float4 u0 = *reinterpret_cast<const float4 *>(src);
+                    const float4 u1 = *reinterpret_cast<const float4 *>(src + 4);
+                    f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w;
+                    f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
+                }
+                uint2 h0, l0, h1, l1;
+                split4(f[0], f[1], f[2], f[3], h0, l0);
+                split4(f[4], f[5], f[6], f[7], h1, l1);
+                if (kMode == kModeRP) {
+                    const uint32_t o = kmajor_off(n, k0, BR);
+                    *reinterpret_cast<uint4 *>(sB + o) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                    *reinterpret_cast<uint4 *>(sB + kBLoOff + o) = make_uint4(l0.x, l0.y, l1.x, l1.y);
+                } else {
+                    *reinterpret_cast<uint4 *>(sB + kmajor_off(n, k0, BR)) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                    *reinterpret_cast<uint4 *>(sB + kmajor_off(kD + n, k0, BR)) =
+                        make_uint4(l0.x, l0.y, l1.x, l1.y);
+                }
+            }
+            fence_async_smem();
+            mbar_arrive(&bready);
+        }
+        // ---- epilogue: lane = token row of the tile
+        const int sp = warp & 3;
+        for (int t = 0; t < ntile; ++t) {
+            const int acc = t & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (t >> 1) & 1, &abort_flag, a.status, 105)))
+                break;
+            tc_fence_after();
+            const uint32_t dcol = 256 * acc;
+            const long tok = row0 + (long)t * kTokTile + 32 * sp + lane;
+            const float et = a.eta[tok];
+            if (kMode == kModeRP) {
+                float de = 0.f;
+#pragma unroll 1
+                for (int q = 0; q < kD / 16; ++q) {
+                    float r[16], p[16];
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + 16 * q), r);
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + kD + 16 * q), p);
+                    const uint4 *vq = reinterpret_cast<const uint4 *>(a.V + tok * kD + 16 * q);
+                    const uint4 v0 = vq[0], v1 = vq[1];
+                    tmem_ld_wait();
+                    const __nv_bfloat162 *vh0 = reinterpret_cast<const __nv_bfloat162 *>(&v0);
+                    const __nv_bfloat162 *vh1 = reinterpret_cast<const __nv_bfloat162 *>(&v1);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x0 = __bfloat1622float2(vh0[e]), x1 = __bfloat1622float2(vh1[e]);
+                        r[2 * e] -= x0.x;
+                        r[2 * e + 1] -= x0.y;
+                        r[8 + 2 * e] -= x1.x;
+                        r[8 + 2 * e + 1] -= x1.y;
+                    }
+                    float4 *dv = reinterpret_cast<float4 *>(a.out + tok * kD + 16 * q);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        dv[e] = make_float4(et * p[4 * e], et * p[4 * e + 1], et * p[4 * e + 2], et * p[4 * e + 3]);
+                        de = fmaf(p[4 * e], r[4 * e], de);
+                        de = fmaf(p[4 * e + 1], r[4 * e + 1], de);
+                        de = fmaf(p[4 * e + 2], r[4 * e + 2], de);
+                        de = fmaf(p[4 * e + 3], r[4 * e + 3], de);
+                    }
+                    // R and P as bf16 hi/lo operand rows ([t][R (128) | P (128)])
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint2 rh0, rl0, rh1, rl1, ph0, pl0, ph1, pl1;
+                        split4(r[8 * h], r[8 * h + 1], r[8 * h + 2], r[8 * h + 3], rh0, rl0);
+                        split4(r[8 * h + 4], r[8 * h + 5], r[8 * h + 6], r[8 * h + 7], rh1, rl1);
+                        split4(p[8 * h], p[8 * h + 1], p[8 * h + 2], p[8 * h + 3], ph0, pl0);
+                        split4(p[8 * h + 4], p[8 * h + 5], p[8 * h + 6], p[8 * h + 7], ph1, pl1);
+                        const size_t ro = (size_t)tok * 2 * kD + 16 * q + 8 * h;
+                        *reinterpret_cast<uint4 *>(a.rp_hi + ro) = make_uint4(rh0.x, rh0.y, rh1.x, rh1.y);
+                        *reinterpret_cast<uint4 *>(a.rp_lo + ro) = make_uint4(rl0.x, rl0.y, rl1.x, rl1.y);
+                        *reinterpret_cast<uint4 *>(a.rp_hi + ro + kD) = make_uint4(ph0.x, ph0.y, ph1.x, ph1.y);
+                        *reinterpret_cast<uint4 *>(a.rp_lo + ro + kD) = make_uint4(pl0.x, pl0.y, pl1.x, pl1.y);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
+                a.deta[tok] = -de;
+                // dZ as bf16 hi/lo operand rows for the dQ pass
+#pragma unroll 1
+                for (int q = 0; q < kD / 8; ++q) {
+                    const float4 *zq = reinterpret_cast<const float4 *>(a.dZ + tok * kD + 8 * q);
+                    const float4 z0 = zq[0], z1 = zq[1];
+                    uint2 zh0, zl0, zh1, zl1;
+                    split4(z0.x, z0.y, z0.z, z0.w, zh0, zl0);
+                    split4(z1.x, z1.y, z1.z, z1.w, zh1, zl1);
+                    *reinterpret_cast<uint4 *>(a.z_hi + tok * kD + 8 * q) = make_uint4(zh0.x, zh0.y, zh1.x, zh1.y);
+                    *reinterpret_cast<uint4 *>(a.z_lo + tok * kD + 8 * q) = make_uint4(zl0.x, zl0.y, zl1.x, zl1.y);
+                }
+            } else {
+                const float sc = kMode == kModeDK ? -et : 1.f;
+                float4 *o = reinterpret_cast<float4 *>(a.out + tok * kD);
+#pragma unroll 1
+                for (int q = 0; q < kD / 16; ++q) {
+                    float x[16], y[16];
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + 16 * q), x);
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + kD + 16 * q), y);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        o[4 * q + e] = make_float4(sc * (x[4 * e] + y[4 * e]), sc * (x[4 * e + 1] + y[4 * e + 1]),
+                                                   sc * (x[4 * e + 2] + y[4 * e + 2]),
+                                                   sc * (x[4 * e + 3] + y[4 * e + 3]));
+                }
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
+            }
+        }
+    }
+    if (abort_flag) {
+        if (warp == 0 && lane == 0)
+            for (int u = issued - kTokStages < 0 ? 0 : issued - kTokStages; u < issued; ++u)
+                mbar_drain(&full[u % kTokStages], (u / kTokStages) & 1);
+        if (warp == 1 && lane == 0) {
+            mma_commit(&drain);
+            mbar_drain(&drain, 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tm, 512);
+}
+
+template <int kMode>
+cudaError_t launch_tok_mode(const CUtensorMap &hi, const CUtensorMap &lo, const TokArgs &a, int nch,
+                            cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(cb_tok_tc_kernel<kMode>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTokSmem);
+    if (e != cudaSuccess) return e;
+    cb_tok_tc_kernel<kMode><<<nch, kTokThreads, kTokSmem, s>>>(hi, lo, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launch(s);
+    return cudaSuccess;
+}
+
+}  // namespace
+
+bool chunk_bwd_tok_tc_supported(int d, int chunk, bool bf16) {
+    return bf16 && d == kD && chunk >= kTokTile && chunk % kTokTile == 0;
+}
+
+// Workspace bytes of the tensor-core token passes: R | P and dZ as bf16 hi
+// and lo rows (1.5 KiB per token).
+size_t chunk_bwd_tok_tc_scratch_bytes(size_t tokens) { return tokens * (2 * 2 * kD + 2 * kD) * 2; }
+
+cudaError_t launch_chunk_bwd_tok_tc(const void *K, const void *V, const float *eta, const float *dZ,
+                                    const float *W, const float *Om, int B, int H, int T, int chunk,
+                                    void *scratch, float *dQ, float *dK, float *dV, float *deta,
+                                    cudaStream_t s) {
+    const uint64_t rows = (uint64_t)B * H * T;
+    const int nch = B * H * (T / chunk);
+    __nv_bfloat16 *rp_hi = static_cast<__nv_bfloat16 *>(scratch);
+    __nv_bfloat16 *rp_lo = rp_hi + rows * 2 * kD;
+    __nv_bfloat16 *z_hi = rp_lo + rows * 2 * kD;
+    __nv_bfloat16 *z_lo = z_hi + rows * kD;
+    int *status = device_status_word();
+    alignas(64) CUtensorMap tmK, tmRPh, tmRPl, tmZh, tmZl;
+    if (!encode_tmap_2d(&tmK, K, false, kD, rows, 64, kTokTile) ||
+        !encode_tmap_2d(&tmRPh, rp_hi, false, 2 * kD, rows, 64, kTokTile) ||
+        !encode_tmap_2d(&tmRPl, rp_lo, false, 2 * kD, rows, 64, kTokTile) ||
+        !encode_tmap_2d(&tmZh, z_hi, false, kD, rows, 64, kTokTile) ||
+        !encode_tmap_2d(&tmZl, z_lo, false, kD, rows, 64, kTokTile))
+        return cudaErrorInvalidValue;
+    TokArgs a{W, Om, static_cast<const __nv_bfloat16 *>(V), eta, dZ, dV, deta,
+              rp_hi, rp_lo, z_hi, z_lo, chunk, status};
+    cudaError_t e = launch_tok_mode<kModeRP>(tmK, tmK, a, nch, s);
+    if (e != cudaSuccess) return e;
+    a.out = dK;
+    if ((e = launch_tok_mode<kModeDK>(tmRPh, tmRPl, a, nch, s)) != cudaSuccess) return e;
+    a.out = dQ;
+    return launch_tok_mode<kModeDQ>(tmZh, tmZl, a, nch, s);
+}
+
 }  // namespace ttt

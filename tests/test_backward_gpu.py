@@ -137,6 +137,10 @@ CHUNK_CASES = {
                                        False, True),
     "chunk_bf16_d128_c128_w0seq": (dict(B=2, H=1, T=512, d=128, b=128), True, True),
     "chunk_bf16_d128_c32_one_chunk": (dict(B=1, H=3, T=32, d=128, b=32), False, True),
+    # chunk % 128 == 0: the per-token products on the tensor cores too
+    "chunk_bf16_d128_c256_eta_varied": (dict(B=1, H=2, T=768, d=128, b=256, eta="sigmoid_over_d"),
+                                        False, True),
+    "chunk_bf16_d128_c128_one_chunk": (dict(B=2, H=1, T=128, d=128, b=128), True, False),
 }
 
 
