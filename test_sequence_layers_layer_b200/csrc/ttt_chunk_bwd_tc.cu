@@ -307,6 +307,29 @@ __device__ __forceinline__ uint32_t kmajor_off(int n, int k, int rows) {
     return (uint32_t)((k >> 6) * rows * 128 + n * 128 + ((((k & 63) >> 3) ^ (n & 7)) << 4) + (k & 7) * 2);
 }
 
+// A warp's 32 token rows written through padded shared memory (16-byte
+// accesses conflict-free) so that global memory sees whole row segments:
+// lane l holds row l's NP consecutive 16-byte pieces.
+constexpr int kStgWarp = 32 * (8 * 16 + 16);  // staging per warp: 32 rows of up to 128 bytes
+template <int NP>
+__device__ __forceinline__ void warp_rows_out(uint8_t *stg, const uint4 (&v)[NP], uint8_t *g0,
+                                              size_t pitch, int lane) {
+    constexpr int SP = NP * 16 + 16, RPI = 32 / NP;
+#pragma unroll
+    for (int i = 0; i < NP; ++i) *reinterpret_cast<uint4 *>(stg + lane * SP + 16 * i) = v[i];
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < NP; ++k) {
+        const int row = k * RPI + lane / NP, pc = lane % NP;
+        *reinterpret_cast<uint4 *>(g0 + (size_t)row * pitch + 16 * pc) =
+            *reinterpret_cast<const uint4 *>(stg + row * SP + 16 * pc);
+    }
+    __syncwarp();
+}
+__device__ __forceinline__ uint4 pack4f(float a, float b, float c, float d) {
+    return make_uint4(__float_as_uint(a), __float_as_uint(b), __float_as_uint(c), __float_as_uint(d));
+}
+
 template <int kMode>
 __global__ void __launch_bounds__(kTokThreads, 1)
     cb_tok_tc_kernel(const __grid_constant__ CUtensorMap tmA_hi, const __grid_constant__ CUtensorMap tmA_lo,
@@ -318,10 +341,16 @@ __global__ void __launch_bounds__(kTokThreads, 1)
     // ([W | Om]^T); DK and DQ stack [hi rows | lo rows] of their 128 rows.
     constexpr int BR = 2 * kD;
     constexpr uint32_t kBLoOff = kMode == kModeRP ? (uint32_t)NKB * BR * 128 : 0u;
+    // A ring: one or two terms of a 64-wide K block per stage; DK's B images
+    // (128 KB) leave room for two stages beside the epilogue's staging.
+    constexpr int STAGES = kMode == kModeDK ? 2 : 3;
+    constexpr int SBYTES = kTwoA ? kTokStage : kTokStage / 2;
+    constexpr int BBYTES = NKB * BR * 128 * (kMode == kModeRP ? 2 : 1);  // B images
+    static_assert(BBYTES + STAGES * SBYTES + 4 * kStgWarp + 1024 <= (int)kTokSmem, "smem plan");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sB = smem, *sA = smem + kTokBBytes;
+    uint8_t *sB = smem, *sA = smem + BBYTES;
     __shared__ uint64_t full[kTokStages], empty[kTokStages], bready, tfull[2], tempty[2], drain;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
@@ -356,13 +385,13 @@ __global__ void __launch_bounds__(kTokThreads, 1)
         // A tiles, one K block per stage
         for (int t = 0, u = 0; t < ntile; ++t) {
             for (int kb = 0; kb < NKB; ++kb, ++u) {
-                const int st = u % kTokStages;
-                if (u >= kTokStages &&
-                    !mbar_wait(&empty[st], ((u / kTokStages) - 1) & 1, &abort_flag, a.status, 101))
+                const int st = u % STAGES;
+                if (u >= STAGES &&
+                    !mbar_wait(&empty[st], ((u / STAGES) - 1) & 1, &abort_flag, a.status, 101))
                     goto producer_done;
-                uint8_t *sb = sA + st * kTokStage;
+                uint8_t *sb = sA + st * SBYTES;
                 const int y = (int)(row0 + (long)t * kTokTile);
-                mbar_arrive_expect_tx(&full[st], kTwoA ? kTokStage : kTokStage / 2);
+                mbar_arrive_expect_tx(&full[st], SBYTES);
                 tma_load_2d(sb, &tmA_hi, 64 * kb, y, &full[st]);
                 if (kTwoA) tma_load_2d(sb + kTokStage / 2, &tmA_lo, 64 * kb, y, &full[st]);
                 issued = u + 1;
@@ -382,13 +411,13 @@ __global__ void __launch_bounds__(kTokThreads, 1)
                 const uint32_t d = tm + 256 * acc;
                 bool ok = true;
                 for (int kb = 0; kb < NKB; ++kb, ++u) {
-                    const int st = u % kTokStages;
-                    if (!mbar_wait(&full[st], (u / kTokStages) & 1, &abort_flag, a.status, 104)) {
+                    const int st = u % STAGES;
+                    if (!mbar_wait(&full[st], (u / STAGES) & 1, &abort_flag, a.status, 104)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = ab + st * kTokStage;
+                    const uint32_t a0 = ab + st * SBYTES;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t ko = (uint32_t)(16 * k * 2);
@@ -419,7 +448,11 @@ __global__ void __launch_bounds__(kTokThreads, 1)
             // units: (row n, 8 consecutive k)
             constexpr int NROWS = kMode == kModeRP ? 2 * kD : kD;
             for (int uidx = tt; uidx < NROWS * (KD / 8); uidx += 128) {
-                const int n = uidx / (KD / 8), k0 = 8 * (uidx % (KD / 8));
+                // RP reads W and Om transposed: consecutive threads take
+                // consecutive n (one 128-byte row segment per warp load);
+                // DK and DQ read rows: consecutive threads take consecutive k
+                const int n = kMode == kModeRP ? uidx % NROWS : uidx / (KD / 8);
+                const int k0 = kMode == kModeRP ? 8 * (uidx / NROWS) : 8 * (uidx % (KD / 8));
                 float f[8];
                 if (kMode == kModeRP) {
                     // B[n][k]: n < 128: W[k][n]; else Om[k][n - 128]  (K = d_in)
@@ -451,28 +484,39 @@ __global__ void __launch_bounds__(kTokThreads, 1)
             fence_async_smem();
             mbar_arrive(&bready);
         }
-        // ---- epilogue: lane = token row of the tile
+        // ---- epilogue: lane = token row of the tile; every global row access
+        // goes through the warp's staging rows (whole row segments)
         const int sp = warp & 3;
+        uint8_t *stg = sA + STAGES * SBYTES + (warp - 2) * kStgWarp;
         for (int t = 0; t < ntile; ++t) {
             const int acc = t & 1;
+            const long tokw = row0 + (long)t * kTokTile + 32 * sp;  // the warp's first token
+            const long tok = tokw + lane;
+            const float et = a.eta[tok];
+            // RP: the token's V row (256 B) loads while the tile's products run
+            uint4 vr[kMode == kModeRP ? kD / 8 : 1];
+            if (kMode == kModeRP) {
+                const uint4 *vq = reinterpret_cast<const uint4 *>(a.V + tok * kD);
+#pragma unroll
+                for (int q = 0; q < kD / 8; ++q) vr[q] = vq[q];
+            }
             if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (t >> 1) & 1, &abort_flag, a.status, 105)))
                 break;
             tc_fence_after();
             const uint32_t dcol = 256 * acc;
-            const long tok = row0 + (long)t * kTokTile + 32 * sp + lane;
-            const float et = a.eta[tok];
             if (kMode == kModeRP) {
+                // A thread per token row: its stores are 16-byte pieces of its own
+                // rows (staging them through shared memory measured slower here:
+                // the pass waits on its loads, not on the number of store requests).
                 float de = 0.f;
-#pragma unroll 1
+#pragma unroll
                 for (int q = 0; q < kD / 16; ++q) {
                     float r[16], p[16];
                     tmem_ld16(taddr(tm, 32 * sp, dcol + 16 * q), r);
                     tmem_ld16(taddr(tm, 32 * sp, dcol + kD + 16 * q), p);
-                    const uint4 *vq = reinterpret_cast<const uint4 *>(a.V + tok * kD + 16 * q);
-                    const uint4 v0 = vq[0], v1 = vq[1];
                     tmem_ld_wait();
-                    const __nv_bfloat162 *vh0 = reinterpret_cast<const __nv_bfloat162 *>(&v0);
-                    const __nv_bfloat162 *vh1 = reinterpret_cast<const __nv_bfloat162 *>(&v1);
+                    const __nv_bfloat162 *vh0 = reinterpret_cast<const __nv_bfloat162 *>(&vr[2 * q]);
+                    const __nv_bfloat162 *vh1 = reinterpret_cast<const __nv_bfloat162 *>(&vr[2 * q + 1]);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 x0 = __bfloat1622float2(vh0[e]), x1 = __bfloat1622float2(vh1[e]);
@@ -508,41 +552,53 @@ __global__ void __launch_bounds__(kTokThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&tempty[acc]);
                 a.deta[tok] = -de;
-                // dZ as bf16 hi/lo operand rows for the dQ pass
+                // dZ as bf16 hi/lo operand rows for the dQ pass, 32 columns per
+                // round with all of a round's loads in flight
+                const float4 *zq = reinterpret_cast<const float4 *>(a.dZ + tok * kD);
 #pragma unroll 1
-                for (int q = 0; q < kD / 8; ++q) {
-                    const float4 *zq = reinterpret_cast<const float4 *>(a.dZ + tok * kD + 8 * q);
-                    const float4 z0 = zq[0], z1 = zq[1];
-                    uint2 zh0, zl0, zh1, zl1;
-                    split4(z0.x, z0.y, z0.z, z0.w, zh0, zl0);
-                    split4(z1.x, z1.y, z1.z, z1.w, zh1, zl1);
-                    *reinterpret_cast<uint4 *>(a.z_hi + tok * kD + 8 * q) = make_uint4(zh0.x, zh0.y, zh1.x, zh1.y);
-                    *reinterpret_cast<uint4 *>(a.z_lo + tok * kD + 8 * q) = make_uint4(zl0.x, zl0.y, zl1.x, zl1.y);
+                for (int h = 0; h < kD / 32; ++h) {
+                    float4 z[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) z[e] = zq[8 * h + e];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        uint2 zh0, zl0, zh1, zl1;
+                        split4(z[2 * e].x, z[2 * e].y, z[2 * e].z, z[2 * e].w, zh0, zl0);
+                        split4(z[2 * e + 1].x, z[2 * e + 1].y, z[2 * e + 1].z, z[2 * e + 1].w, zh1, zl1);
+                        const size_t zo = (size_t)tok * kD + 32 * h + 8 * e;
+                        *reinterpret_cast<uint4 *>(a.z_hi + zo) = make_uint4(zh0.x, zh0.y, zh1.x, zh1.y);
+                        *reinterpret_cast<uint4 *>(a.z_lo + zo) = make_uint4(zl0.x, zl0.y, zl1.x, zl1.y);
+                    }
                 }
             } else {
                 const float sc = kMode == kModeDK ? -et : 1.f;
-                float4 *o = reinterpret_cast<float4 *>(a.out + tok * kD);
 #pragma unroll 1
-                for (int q = 0; q < kD / 16; ++q) {
-                    float x[16], y[16];
-                    tmem_ld16(taddr(tm, 32 * sp, dcol + 16 * q), x);
-                    tmem_ld16(taddr(tm, 32 * sp, dcol + kD + 16 * q), y);
+                for (int q = 0; q < kD / 32; ++q) {
+                    float x[32], y[32];
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + 32 * q), *reinterpret_cast<float(*)[16]>(&x[0]));
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + 32 * q + 16), *reinterpret_cast<float(*)[16]>(&x[16]));
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + kD + 32 * q), *reinterpret_cast<float(*)[16]>(&y[0]));
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + kD + 32 * q + 16), *reinterpret_cast<float(*)[16]>(&y[16]));
                     tmem_ld_wait();
+                    if (q == kD / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(&tempty[acc]);  // the accumulator is read
+                    }
+                    uint4 o8[8];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        o[4 * q + e] = make_float4(sc * (x[4 * e] + y[4 * e]), sc * (x[4 * e + 1] + y[4 * e + 1]),
-                                                   sc * (x[4 * e + 2] + y[4 * e + 2]),
-                                                   sc * (x[4 * e + 3] + y[4 * e + 3]));
+                    for (int e = 0; e < 8; ++e)
+                        o8[e] = pack4f(sc * (x[4 * e] + y[4 * e]), sc * (x[4 * e + 1] + y[4 * e + 1]),
+                                       sc * (x[4 * e + 2] + y[4 * e + 2]), sc * (x[4 * e + 3] + y[4 * e + 3]));
+                    warp_rows_out<8>(stg, o8, reinterpret_cast<uint8_t *>(a.out + tokw * kD + 32 * q),
+                                     4 * kD, lane);
                 }
-                tc_fence_before();
-                mbar_arrive(&tempty[acc]);
             }
         }
     }
     if (abort_flag) {
         if (warp == 0 && lane == 0)
-            for (int u = issued - kTokStages < 0 ? 0 : issued - kTokStages; u < issued; ++u)
-                mbar_drain(&full[u % kTokStages], (u / kTokStages) & 1);
+            for (int u = issued - STAGES < 0 ? 0 : issued - STAGES; u < issued; ++u)
+                mbar_drain(&full[u % STAGES], (u / STAGES) & 1);
         if (warp == 1 && lane == 0) {
             mma_commit(&drain);
             mbar_drain(&drain, 0);
