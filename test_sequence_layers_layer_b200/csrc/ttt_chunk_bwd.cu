@@ -124,12 +124,14 @@ __global__ void __launch_bounds__(kT) cb_gram_kernel(const TIn *Q, const TIn *K,
 //    blockIdx.y = 1: M = Om_{c+1} backward from dW_out, E = D_c, storing
 //    Om_{c+1}, and at the end Om_0 = dW0 of the sequence.
 // A thread owns an RB x RB block of M. A_c is symmetric (K^T diag(eta) K), so
-// its row k stands for its column k.
+// its row k stands for its column k. Each step first copies A_c into shared
+// memory (coalesced), so the product's inner loop reads shared memory only.
 template <int D>
 __global__ void __launch_bounds__(kT) cb_scan_kernel(const float *W0, const float *dW_out,
                                                      int H, int NC, bool w0_per_seq, WsView w,
                                                      float *dW0_out) {
-    extern __shared__ __align__(16) float Ms[];  // D x D
+    extern __shared__ __align__(16) float Ms[];  // D x D, then A_c (D x D)
+    float *As = Ms + D * D;
     constexpr int RB = D / 16;
     const int seq = blockIdx.x, dir = blockIdx.y, tid = threadIdx.x;
     const int i0 = RB * (tid / 16), j0 = RB * (tid % 16);
@@ -146,14 +148,17 @@ __global__ void __launch_bounds__(kT) cb_scan_kernel(const float *W0, const floa
         const size_t g = (size_t)seq * NC + c;
         float *store = (dir == 0 ? w.W : w.Om) + g * dd;
         for (int e = tid; e < D * D; e += kT) store[e] = Ms[e];
-        const float *A = w.gram + (g * 3 + 0) * dd;
+        const float *Ag = w.gram + (g * 3 + 0) * dd;
         const float *E = w.gram + (g * 3 + (dir == 0 ? 1 : 2)) * dd;
+        for (int e = 4 * tid; e < D * D; e += 4 * kT)
+            *reinterpret_cast<float4 *>(As + e) = *reinterpret_cast<const float4 *>(Ag + e);
+        __syncthreads();  // A_c is in shared memory
         float acc[RB][RB] = {};
         for (int k = 0; k < D; ++k) {
             float av[RB], mv[RB];
 #pragma unroll
             for (int r = 0; r < RB; r += 4) {
-                const float4 u = *reinterpret_cast<const float4 *>(A + (size_t)k * D + i0 + r);
+                const float4 u = *reinterpret_cast<const float4 *>(As + k * D + i0 + r);
                 const float4 v = *reinterpret_cast<const float4 *>(Ms + k * D + j0 + r);
                 av[r] = u.x; av[r + 1] = u.y; av[r + 2] = u.z; av[r + 3] = u.w;
                 mv[r] = v.x; mv[r + 1] = v.y; mv[r + 2] = v.z; mv[r + 3] = v.w;
@@ -316,7 +321,7 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         count_launch(s);
     }
-    const size_t scan_smem = (size_t)D * D * sizeof(float);
+    const size_t scan_smem = 2 * (size_t)D * D * sizeof(float);  // M and A_c
     if ((e = cudaFuncSetAttribute(cb_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)scan_smem)) != cudaSuccess)
         return e;
