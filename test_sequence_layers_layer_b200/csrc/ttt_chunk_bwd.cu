@@ -28,7 +28,7 @@ namespace ttt {
 bool chunk_bwd_gram_tc_supported(int d, int chunk, bool bf16);
 cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V, const float *eta,
                                      const float *dZ, int B, int H, int T, int chunk, float *gram,
-                                     cudaStream_t s);
+                                     void *tok_scratch, cudaStream_t s);
 bool chunk_bwd_tok_tc_supported(int d, int chunk, bool bf16);
 size_t chunk_bwd_tok_tc_scratch_bytes(size_t tokens);
 cudaError_t launch_chunk_bwd_tok_tc(const void *K, const void *V, const float *eta, const float *dZ,
@@ -311,9 +311,15 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
     const TIn *q = static_cast<const TIn *>(Q), *k = static_cast<const TIn *>(K),
               *v = static_cast<const TIn *>(V);
     cudaError_t e;
+    // d = 128, bf16, chunk % 128 == 0: the per-token products on the tensor
+    // cores; their bf16 operand rows follow the fp32 part of the workspace
+    const bool tok_tc = std::is_same<TIn, __nv_bfloat16>::value && chunk_bwd_tok_tc_supported(D, C, true);
+    void *scratch = tok_tc ? reinterpret_cast<float *>(workspace) + (5 * nch + S) * (size_t)D * D : nullptr;
     if (std::is_same<TIn, __nv_bfloat16>::value && chunk_bwd_gram_tc_supported(D, C, true)) {
-        // d = 128, bf16: the Gram products on the tensor cores
-        if ((e = launch_chunk_bwd_gram_tc(Q, K, V, eta, dZ, B, H, T, C, w.gram, s)) != cudaSuccess)
+        // d = 128, bf16: the Gram products on the tensor cores (also writing
+        // dZ's operand rows for the token passes)
+        if ((e = launch_chunk_bwd_gram_tc(Q, K, V, eta, dZ, B, H, T, C, w.gram, scratch, s)) !=
+            cudaSuccess)
             return e;
     } else {
         cb_gram_kernel<TIn, D><<<dim3((unsigned)nch, 3, (D / 64) * (D / 64)), kT, 0, s>>>(
@@ -330,10 +336,7 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
                                                                   dW0_seq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launch(s);
-    if (std::is_same<TIn, __nv_bfloat16>::value && chunk_bwd_tok_tc_supported(D, C, true)) {
-        // d = 128, bf16, chunk % 128 == 0: the per-token products on the tensor
-        // cores; their bf16 operand rows follow the fp32 part of the workspace
-        void *scratch = reinterpret_cast<float *>(workspace) + (5 * nch + S) * (size_t)D * D;
+    if (tok_tc) {
         if ((e = launch_chunk_bwd_tok_tc(K, V, eta, dZ, w.W, w.Om, B, H, T, C, scratch, dQ, dK, dV,
                                          deta, s)) != cudaSuccess)
             return e;

@@ -48,6 +48,9 @@ struct GramArgs {
     float *gram;  // [chunk][3][d][d]
     int chunk;
     int *status;
+    // optional: dZ's bf16 hi and lo rows ([tokens][d]) for the token passes,
+    // written from the terms this kernel forms anyway
+    __nv_bfloat16 *z_hi = nullptr, *z_lo = nullptr;
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -168,6 +171,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_uint4(h0.x, h0.y, h1.x, h1.y);
                 *reinterpret_cast<uint4 *>(sb + OFF_ZB + (2 + (col0 >> 6)) * kBox + off) =
                     make_uint4(l0.x, l0.y, l1.x, l1.y);
+                if (a.z_hi) {
+                    const size_t zo = (size_t)(row0 + (long)r * kRows + row) * kD + col0;
+                    *reinterpret_cast<uint4 *>(a.z_hi + zo) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                    *reinterpret_cast<uint4 *>(a.z_lo + zo) = make_uint4(l0.x, l0.y, l1.x, l1.y);
+                }
                 if (!uniform) {
                     const uint4 kq = *reinterpret_cast<const uint4 *>(sb + OFF_K + (col0 >> 6) * kBox + off);
                     const __nv_bfloat162 *kh = reinterpret_cast<const __nv_bfloat162 *>(&kq);
@@ -241,10 +249,25 @@ bool chunk_bwd_gram_tc_supported(int d, int chunk, bool bf16) {
     return bf16 && d == kD && chunk >= kRows && chunk % kRows == 0;
 }
 
-// gram: [B*H*(T/chunk)][3][128][128] fp32, written in full.
+// The token passes' operand rows in their scratch: R | P hi and lo
+// ([tokens][2d]), then dZ hi and lo ([tokens][d]), all bf16.
+struct TokScratch {
+    __nv_bfloat16 *rp_hi, *rp_lo, *z_hi, *z_lo;
+};
+TokScratch tok_scratch(void *scratch, uint64_t rows) {
+    TokScratch t;
+    t.rp_hi = static_cast<__nv_bfloat16 *>(scratch);
+    t.rp_lo = t.rp_hi + rows * 2 * kD;
+    t.z_hi = t.rp_lo + rows * 2 * kD;
+    t.z_lo = t.z_hi + rows * kD;
+    return t;
+}
+
+// gram: [B*H*(T/chunk)][3][128][128] fp32, written in full. tok_scratch:
+// the token passes' scratch (or nullptr), whose dZ rows this kernel fills.
 cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V, const float *eta,
                                      const float *dZ, int B, int H, int T, int chunk, float *gram,
-                                     cudaStream_t s) {
+                                     void *tok_scratch_ptr, cudaStream_t s) {
     const uint64_t rows = (uint64_t)B * H * T;
     const int nch = B * H * (T / chunk);
     alignas(64) CUtensorMap tmK, tmV, tmQ, tmZ;
@@ -256,8 +279,13 @@ cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V
     cudaError_t e = cudaFuncSetAttribute(cb_gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmem);
     if (e != cudaSuccess) return e;
-    cb_gram_tc_kernel<<<nch, kThreads, kSmem, s>>>(tmK, tmV, tmQ, tmZ,
-                                                   GramArgs{eta, gram, chunk, device_status_word()});
+    GramArgs ga{eta, gram, chunk, device_status_word()};
+    if (tok_scratch_ptr) {
+        const TokScratch ts = tok_scratch(tok_scratch_ptr, rows);
+        ga.z_hi = ts.z_hi;
+        ga.z_lo = ts.z_lo;
+    }
+    cb_gram_tc_kernel<<<nch, kThreads, kSmem, s>>>(tmK, tmV, tmQ, tmZ, ga);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
@@ -273,8 +301,9 @@ cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V
 //   dK = -diag(eta) [R | P] [Om | W]^T,  dQ = dZ W^T,
 // as three passes of one kernel over 128-token tiles, a block per chunk:
 //   RP: D = K [W | Om] (N = 256, K = d_in): A = K (exact), B = [W | Om]^T as
-//       hi and lo terms; the epilogue forms R, dV, deta and writes R, P (and
-//       dZ) as bf16 hi/lo operand rows into the workspace;
+//       hi and lo terms; the epilogue forms R, dV, deta and writes R, P as
+//       bf16 hi/lo operand rows into the workspace (dZ's rows come from the
+//       Gram kernel, which splits dZ anyway);
 //   DK: D = [R | P]_{hi,lo} [Om | W]^T (K = 256);  DQ: D = dZ_{hi,lo} W^T (K = 128):
 //       B stacked as [hi rows | lo rows] (N = 256), so A_hi x B gives the hi.hi
 //       and hi.lo terms side by side and A_lo x B_hi adds lo.hi to the first half.
@@ -552,24 +581,6 @@ __global__ void __launch_bounds__(kTokThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&tempty[acc]);
                 a.deta[tok] = -de;
-                // dZ as bf16 hi/lo operand rows for the dQ pass, 32 columns per
-                // round with all of a round's loads in flight
-                const float4 *zq = reinterpret_cast<const float4 *>(a.dZ + tok * kD);
-#pragma unroll 1
-                for (int h = 0; h < kD / 32; ++h) {
-                    float4 z[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) z[e] = zq[8 * h + e];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        uint2 zh0, zl0, zh1, zl1;
-                        split4(z[2 * e].x, z[2 * e].y, z[2 * e].z, z[2 * e].w, zh0, zl0);
-                        split4(z[2 * e + 1].x, z[2 * e + 1].y, z[2 * e + 1].z, z[2 * e + 1].w, zh1, zl1);
-                        const size_t zo = (size_t)tok * kD + 32 * h + 8 * e;
-                        *reinterpret_cast<uint4 *>(a.z_hi + zo) = make_uint4(zh0.x, zh0.y, zh1.x, zh1.y);
-                        *reinterpret_cast<uint4 *>(a.z_lo + zo) = make_uint4(zl0.x, zl0.y, zl1.x, zl1.y);
-                    }
-                }
             } else {
                 const float sc = kMode == kModeDK ? -et : 1.f;
 #pragma unroll 1
@@ -638,10 +649,8 @@ cudaError_t launch_chunk_bwd_tok_tc(const void *K, const void *V, const float *e
                                     cudaStream_t s) {
     const uint64_t rows = (uint64_t)B * H * T;
     const int nch = B * H * (T / chunk);
-    __nv_bfloat16 *rp_hi = static_cast<__nv_bfloat16 *>(scratch);
-    __nv_bfloat16 *rp_lo = rp_hi + rows * 2 * kD;
-    __nv_bfloat16 *z_hi = rp_lo + rows * 2 * kD;
-    __nv_bfloat16 *z_lo = z_hi + rows * kD;
+    const TokScratch ts = tok_scratch(scratch, rows);
+    __nv_bfloat16 *rp_hi = ts.rp_hi, *rp_lo = ts.rp_lo, *z_hi = ts.z_hi, *z_lo = ts.z_lo;
     int *status = device_status_word();
     alignas(64) CUtensorMap tmK, tmRPh, tmRPl, tmZh, tmZl;
     if (!encode_tmap_2d(&tmK, K, false, kD, rows, 64, kTokTile) ||
