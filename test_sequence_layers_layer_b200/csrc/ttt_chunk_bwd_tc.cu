@@ -534,49 +534,57 @@ __global__ void __launch_bounds__(kTokThreads, 1)
             tc_fence_after();
             const uint32_t dcol = 256 * acc;
             if (kMode == kModeRP) {
-                // A thread per token row: its stores are 16-byte pieces of its own
-                // rows (staging them through shared memory measured slower here:
-                // the pass waits on its loads, not on the number of store requests).
+                // A thread per token row; its output rows leave through the warp's
+                // staging rows as whole segments (32 columns a round).
                 float de = 0.f;
 #pragma unroll
-                for (int q = 0; q < kD / 16; ++q) {
-                    float r[16], p[16];
-                    tmem_ld16(taddr(tm, 32 * sp, dcol + 16 * q), r);
-                    tmem_ld16(taddr(tm, 32 * sp, dcol + kD + 16 * q), p);
+                for (int q = 0; q < kD / 32; ++q) {
+                    float r[32], p[32];
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + 32 * q), *reinterpret_cast<float(*)[16]>(&r[0]));
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + 32 * q + 16), *reinterpret_cast<float(*)[16]>(&r[16]));
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + kD + 32 * q), *reinterpret_cast<float(*)[16]>(&p[0]));
+                    tmem_ld16(taddr(tm, 32 * sp, dcol + kD + 32 * q + 16), *reinterpret_cast<float(*)[16]>(&p[16]));
                     tmem_ld_wait();
-                    const __nv_bfloat162 *vh0 = reinterpret_cast<const __nv_bfloat162 *>(&vr[2 * q]);
-                    const __nv_bfloat162 *vh1 = reinterpret_cast<const __nv_bfloat162 *>(&vr[2 * q + 1]);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 x0 = __bfloat1622float2(vh0[e]), x1 = __bfloat1622float2(vh1[e]);
-                        r[2 * e] -= x0.x;
-                        r[2 * e + 1] -= x0.y;
-                        r[8 + 2 * e] -= x1.x;
-                        r[8 + 2 * e + 1] -= x1.y;
+                    for (int c = 0; c < 4; ++c) {
+                        const __nv_bfloat162 *vh = reinterpret_cast<const __nv_bfloat162 *>(&vr[4 * q + c]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 x = __bfloat1622float2(vh[e]);
+                            r[8 * c + 2 * e] -= x.x;
+                            r[8 * c + 2 * e + 1] -= x.y;
+                        }
                     }
-                    float4 *dv = reinterpret_cast<float4 *>(a.out + tok * kD + 16 * q);
+                    uint4 o8[8];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        dv[e] = make_float4(et * p[4 * e], et * p[4 * e + 1], et * p[4 * e + 2], et * p[4 * e + 3]);
+                    for (int e = 0; e < 8; ++e) {
+                        o8[e] = pack4f(et * p[4 * e], et * p[4 * e + 1], et * p[4 * e + 2], et * p[4 * e + 3]);
                         de = fmaf(p[4 * e], r[4 * e], de);
                         de = fmaf(p[4 * e + 1], r[4 * e + 1], de);
                         de = fmaf(p[4 * e + 2], r[4 * e + 2], de);
                         de = fmaf(p[4 * e + 3], r[4 * e + 3], de);
                     }
+                    warp_rows_out<8>(stg, o8, reinterpret_cast<uint8_t *>(a.out + tokw * kD + 32 * q),
+                                     4 * kD, lane);  // dV
                     // R and P as bf16 hi/lo operand rows ([t][R (128) | P (128)])
+                    uint4 rh[4], rl[4], ph[4], pl[4];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint2 rh0, rl0, rh1, rl1, ph0, pl0, ph1, pl1;
-                        split4(r[8 * h], r[8 * h + 1], r[8 * h + 2], r[8 * h + 3], rh0, rl0);
-                        split4(r[8 * h + 4], r[8 * h + 5], r[8 * h + 6], r[8 * h + 7], rh1, rl1);
-                        split4(p[8 * h], p[8 * h + 1], p[8 * h + 2], p[8 * h + 3], ph0, pl0);
-                        split4(p[8 * h + 4], p[8 * h + 5], p[8 * h + 6], p[8 * h + 7], ph1, pl1);
-                        const size_t ro = (size_t)tok * 2 * kD + 16 * q + 8 * h;
-                        *reinterpret_cast<uint4 *>(a.rp_hi + ro) = make_uint4(rh0.x, rh0.y, rh1.x, rh1.y);
-                        *reinterpret_cast<uint4 *>(a.rp_lo + ro) = make_uint4(rl0.x, rl0.y, rl1.x, rl1.y);
-                        *reinterpret_cast<uint4 *>(a.rp_hi + ro + kD) = make_uint4(ph0.x, ph0.y, ph1.x, ph1.y);
-                        *reinterpret_cast<uint4 *>(a.rp_lo + ro + kD) = make_uint4(pl0.x, pl0.y, pl1.x, pl1.y);
+                    for (int e = 0; e < 4; ++e) {
+                        uint2 a0, b0, a1, b1;
+                        split4(r[8 * e], r[8 * e + 1], r[8 * e + 2], r[8 * e + 3], a0, b0);
+                        split4(r[8 * e + 4], r[8 * e + 5], r[8 * e + 6], r[8 * e + 7], a1, b1);
+                        rh[e] = make_uint4(a0.x, a0.y, a1.x, a1.y);
+                        rl[e] = make_uint4(b0.x, b0.y, b1.x, b1.y);
+                        split4(p[8 * e], p[8 * e + 1], p[8 * e + 2], p[8 * e + 3], a0, b0);
+                        split4(p[8 * e + 4], p[8 * e + 5], p[8 * e + 6], p[8 * e + 7], a1, b1);
+                        ph[e] = make_uint4(a0.x, a0.y, a1.x, a1.y);
+                        pl[e] = make_uint4(b0.x, b0.y, b1.x, b1.y);
                     }
+                    const size_t rpo = (size_t)tokw * 2 * kD + 32 * q;
+                    warp_rows_out<4>(stg, rh, reinterpret_cast<uint8_t *>(a.rp_hi + rpo), 4 * kD, lane);
+                    warp_rows_out<4>(stg, rl, reinterpret_cast<uint8_t *>(a.rp_lo + rpo), 4 * kD, lane);
+                    warp_rows_out<4>(stg, ph, reinterpret_cast<uint8_t *>(a.rp_hi + rpo + kD), 4 * kD, lane);
+                    warp_rows_out<4>(stg, pl, reinterpret_cast<uint8_t *>(a.rp_lo + rpo + kD), 4 * kD, lane);
                 }
                 tc_fence_before();
                 mbar_arrive(&tempty[acc]);
