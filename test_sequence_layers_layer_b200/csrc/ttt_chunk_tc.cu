@@ -334,6 +334,26 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint64_t *done = &bars[3 * kGramStagesU];
         const long row0 = (long)g * a.chunk;  // first token row of this chunk in [B*H*T][d]
         const int nst = a.chunk / kGramRows;
+        int issued = 0;
+        // Barriers for either ring, and stage 0's K and V loads (at the same
+        // place in both layouts) on their way before the step-size check.
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < kGramStagesU; ++i) {
+                mbar_init(&full[i], 1);
+                mbar_init(&conv[i], 128);
+                mbar_init(&empty[i], 1);
+            }
+            mbar_init(done, 1);
+            mbar_init(drain, 1);
+            fence_mbar_init();
+            const int y = (int)row0;
+            mbar_arrive_expect_tx(&full[0], 4 * kGramBox);
+            tma_load_2d(smem, &tmK, 0, y, &full[0]);
+            tma_load_2d(smem + kGramBox, &tmK, 64, y, &full[0]);
+            tma_load_2d(smem + 2 * kGramBox, &tmV, 0, y, &full[0]);
+            tma_load_2d(smem + 3 * kGramBox, &tmV, 64, y, &full[0]);
+            issued = 1;
+        }
         // one step size over the whole chunk?
         const float eta0 = a.eta[row0];
         bool differs = false;
@@ -342,25 +362,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         const bool uniform = !__syncthreads_or(differs);
         const int stages = uniform ? kGramStagesU : kGramStages;
         const int stage_bytes = uniform ? kGramStageBytesU : kGramStageBytes;
-        if (threadIdx.x == 0) {
-            for (int i = 0; i < stages; ++i) {
-                mbar_init(&full[i], 1);
-                mbar_init(&conv[i], 128);
-                mbar_init(&empty[i], 1);
-            }
-            mbar_init(done, 1);
-            mbar_init(drain, 1);
-            fence_mbar_init();
-        }
         if (warp == 1) tmem_alloc(&tmem_base, ncols);
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         const uint32_t tm = tmem_base;
-        int issued = 0;
         if (warp == 0 && lane == 0) {
             // TMA producer: K rows and V rows of each stage, two 64-column boxes each.
-            for (int r = 0; r < nst; ++r) {
+            for (int r = 1; r < nst; ++r) {
                 const int st = r % stages;
                 if (r >= stages &&
                     !mbar_wait(&empty[st], ((r / stages) - 1) & 1, &abort_flag, a.status, 11))
