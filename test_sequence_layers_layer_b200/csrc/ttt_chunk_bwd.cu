@@ -123,31 +123,40 @@ __global__ void __launch_bounds__(kT) cb_gram_kernel(const TIn *Q, const TIn *K,
 //    blockIdx.y = 0: M = W_c forward from W0, E = B_c, storing W_c;
 //    blockIdx.y = 1: M = Om_{c+1} backward from dW_out, E = D_c, storing
 //    Om_{c+1}, and at the end Om_0 = dW0 of the sequence.
-// A thread owns an RB x RB block of M. A_c is symmetric (K^T diag(eta) K), so
-// its row k stands for its column k. Each step first copies A_c into shared
-// memory (coalesced), so the product's inner loop reads shared memory only.
+// The columns of M evolve independently, so blockIdx.z picks a slice of
+// scan_cols(D) columns (more blocks on the 16-step chains: 32 columns at
+// d = 128). A thread owns a 4 x 4 block of the slice. A_c is symmetric
+// (K^T diag(eta) K), so its row k stands for its column k. Each step first
+// copies A_c into shared memory (coalesced), so the product's inner loop
+// reads shared memory only.
+__host__ __device__ constexpr int scan_cols(int D) { return 16 * kT / D; }
 template <int D>
 __global__ void __launch_bounds__(kT) cb_scan_kernel(const float *W0, const float *dW_out,
                                                      int H, int NC, bool w0_per_seq, WsView w,
                                                      float *dW0_out) {
-    extern __shared__ __align__(16) float Ms[];  // D x D, then A_c (D x D)
-    float *As = Ms + D * D;
-    constexpr int RB = D / 16;
-    const int seq = blockIdx.x, dir = blockIdx.y, tid = threadIdx.x;
-    const int i0 = RB * (tid / 16), j0 = RB * (tid % 16);
+    constexpr int kScanCols = scan_cols(D);
+    extern __shared__ __align__(16) float As[];  // A_c (D x D), then the slice of M (D x kScanCols)
+    float *Ms = As + D * D;
+    constexpr int RB = 4, CG = kScanCols / RB;   // CG column groups of 4
+    static_assert(D / RB * CG == kT && D % kScanCols == 0, "a 4 x 4 block per thread");
+    const int seq = blockIdx.x, dir = blockIdx.y, c0 = kScanCols * blockIdx.z, tid = threadIdx.x;
+    const int i0 = RB * (tid / CG), j0 = RB * (tid % CG);  // within the slice
     const size_t dd = (size_t)D * D;
-    if (dir == 0) {
-        const float *w0 = W0 + (size_t)(w0_per_seq ? seq : seq % H) * dd;
-        for (int e = tid; e < D * D; e += kT) Ms[e] = w0[e];
-    } else {
-        for (int e = tid; e < D * D; e += kT) Ms[e] = dW_out ? dW_out[(size_t)seq * dd + e] : 0.f;
+    const float *src0 = dir == 0 ? W0 + (size_t)(w0_per_seq ? seq : seq % H) * dd
+                                 : (dW_out ? dW_out + (size_t)seq * dd : nullptr);
+    for (int e = tid; e < D * kScanCols; e += kT) {
+        const int i = e / kScanCols, j = e % kScanCols;
+        Ms[e] = src0 ? src0[(size_t)i * D + c0 + j] : 0.f;
     }
     __syncthreads();
     for (int s = 0; s < NC; ++s) {
         const int c = dir == 0 ? s : NC - 1 - s;
         const size_t g = (size_t)seq * NC + c;
         float *store = (dir == 0 ? w.W : w.Om) + g * dd;
-        for (int e = tid; e < D * D; e += kT) store[e] = Ms[e];
+        for (int e = tid; e < D * kScanCols; e += kT) {
+            const int i = e / kScanCols, j = e % kScanCols;
+            store[(size_t)i * D + c0 + j] = Ms[e];
+        }
         const float *Ag = w.gram + (g * 3 + 0) * dd;
         const float *E = w.gram + (g * 3 + (dir == 0 ? 1 : 2)) * dd;
         for (int e = 4 * tid; e < D * D; e += 4 * kT)
@@ -155,31 +164,29 @@ __global__ void __launch_bounds__(kT) cb_scan_kernel(const float *W0, const floa
         __syncthreads();  // A_c is in shared memory
         float acc[RB][RB] = {};
         for (int k = 0; k < D; ++k) {
-            float av[RB], mv[RB];
-#pragma unroll
-            for (int r = 0; r < RB; r += 4) {
-                const float4 u = *reinterpret_cast<const float4 *>(As + k * D + i0 + r);
-                const float4 v = *reinterpret_cast<const float4 *>(Ms + k * D + j0 + r);
-                av[r] = u.x; av[r + 1] = u.y; av[r + 2] = u.z; av[r + 3] = u.w;
-                mv[r] = v.x; mv[r + 1] = v.y; mv[r + 2] = v.z; mv[r + 3] = v.w;
-            }
+            const float4 u = *reinterpret_cast<const float4 *>(As + k * D + i0);
+            const float4 v = *reinterpret_cast<const float4 *>(Ms + k * kScanCols + j0);
+            const float av[RB] = {u.x, u.y, u.z, u.w}, mv[RB] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int a = 0; a < RB; ++a)
 #pragma unroll
                 for (int b = 0; b < RB; ++b) acc[a][b] = fmaf(av[a], mv[b], acc[a][b]);
         }
-        __syncthreads();  // every thread has read M
+        __syncthreads();  // every thread has read M and A_c
 #pragma unroll
         for (int a = 0; a < RB; ++a)
 #pragma unroll
             for (int b = 0; b < RB; ++b) {
-                const int e = (i0 + a) * D + j0 + b;
-                Ms[e] = Ms[e] - acc[a][b] + E[e];
+                const int e = (i0 + a) * kScanCols + j0 + b;
+                Ms[e] = Ms[e] - acc[a][b] + E[(size_t)(i0 + a) * D + c0 + j0 + b];
             }
         __syncthreads();
     }
     if (dir == 1)
-        for (int e = tid; e < D * D; e += kT) dW0_out[(size_t)seq * dd + e] = Ms[e];
+        for (int e = tid; e < D * kScanCols; e += kT) {
+            const int i = e / kScanCols, j = e % kScanCols;
+            dW0_out[(size_t)seq * dd + (size_t)i * D + c0 + j] = Ms[e];
+        }
 }
 
 // ---------------------------------------------------------------------------
@@ -327,13 +334,13 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         count_launch(s);
     }
-    const size_t scan_smem = 2 * (size_t)D * D * sizeof(float);  // M and A_c
+    const size_t scan_smem = ((size_t)D * D + (size_t)D * scan_cols(D)) * sizeof(float);  // A_c, M slice
     if ((e = cudaFuncSetAttribute(cb_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)scan_smem)) != cudaSuccess)
         return e;
     float *dW0_seq = w0_per_seq ? dW0 : w.dW0s;
-    cb_scan_kernel<D><<<dim3((unsigned)S, 2), kT, scan_smem, s>>>(W0, dW_out, H, NC, w0_per_seq, w,
-                                                                  dW0_seq);
+    cb_scan_kernel<D><<<dim3((unsigned)S, 2, D / scan_cols(D)), kT, scan_smem, s>>>(
+        W0, dW_out, H, NC, w0_per_seq, w, dW0_seq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launch(s);
     if (tok_tc) {
