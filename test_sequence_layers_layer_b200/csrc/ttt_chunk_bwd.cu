@@ -126,9 +126,9 @@ __global__ void __launch_bounds__(kT) cb_gram_kernel(const TIn *Q, const TIn *K,
 // The columns of M evolve independently, so blockIdx.z picks a slice of
 // scan_cols(D) columns (more blocks on the 16-step chains: 32 columns at
 // d = 128). A thread owns a 4 x 4 block of the slice. A_c is symmetric
-// (K^T diag(eta) K), so its row k stands for its column k. Each step first
-// copies A_c into shared memory (coalesced), so the product's inner loop
-// reads shared memory only.
+// (K^T diag(eta) K), so its row k stands for its column k. A_c sits in
+// shared memory for the step's product; the next step's A_c and this step's
+// E_c are loaded into registers while the product runs.
 __host__ __device__ constexpr int scan_cols(int D) { return 16 * kT / D; }
 template <int D>
 __global__ void __launch_bounds__(kT) cb_scan_kernel(const float *W0, const float *dW_out,
@@ -149,19 +149,36 @@ __global__ void __launch_bounds__(kT) cb_scan_kernel(const float *W0, const floa
         Ms[e] = src0 ? src0[(size_t)i * D + c0 + j] : 0.f;
     }
     __syncthreads();
+    // A_c of the first step into shared memory; each later step's A_c is
+    // loaded into registers while the previous step's product runs
+    constexpr int NPF = D * D / 4 / kT;  // float4 of A_c per thread
+    auto chunk_of = [&](int st) { return (size_t)seq * NC + (dir == 0 ? st : NC - 1 - st); };
+    {
+        const float *Ag = w.gram + (chunk_of(0) * 3 + 0) * dd;
+#pragma unroll
+        for (int q = 0; q < NPF; ++q)
+            *reinterpret_cast<float4 *>(As + 4 * (tid + q * kT)) =
+                *reinterpret_cast<const float4 *>(Ag + 4 * (tid + q * kT));
+    }
     for (int s = 0; s < NC; ++s) {
-        const int c = dir == 0 ? s : NC - 1 - s;
-        const size_t g = (size_t)seq * NC + c;
+        const size_t g = chunk_of(s);
         float *store = (dir == 0 ? w.W : w.Om) + g * dd;
         for (int e = tid; e < D * kScanCols; e += kT) {
             const int i = e / kScanCols, j = e % kScanCols;
             store[(size_t)i * D + c0 + j] = Ms[e];
         }
-        const float *Ag = w.gram + (g * 3 + 0) * dd;
         const float *E = w.gram + (g * 3 + (dir == 0 ? 1 : 2)) * dd;
-        for (int e = 4 * tid; e < D * D; e += 4 * kT)
-            *reinterpret_cast<float4 *>(As + e) = *reinterpret_cast<const float4 *>(Ag + e);
         __syncthreads();  // A_c is in shared memory
+        float4 pf[NPF];   // the next step's A
+        if (s + 1 < NC) {
+            const float *An = w.gram + (chunk_of(s + 1) * 3 + 0) * dd;
+#pragma unroll
+            for (int q = 0; q < NPF; ++q) pf[q] = *reinterpret_cast<const float4 *>(An + 4 * (tid + q * kT));
+        }
+        float4 ev[RB];  // this thread's 4 x 4 block of E
+#pragma unroll
+        for (int a = 0; a < RB; ++a)
+            ev[a] = *reinterpret_cast<const float4 *>(E + (size_t)(i0 + a) * D + c0 + j0);
         float acc[RB][RB] = {};
         for (int k = 0; k < D; ++k) {
             const float4 u = *reinterpret_cast<const float4 *>(As + k * D + i0);
@@ -174,12 +191,16 @@ __global__ void __launch_bounds__(kT) cb_scan_kernel(const float *W0, const floa
         }
         __syncthreads();  // every thread has read M and A_c
 #pragma unroll
-        for (int a = 0; a < RB; ++a)
+        for (int a = 0; a < RB; ++a) {
+            float4 *m = reinterpret_cast<float4 *>(Ms + (i0 + a) * kScanCols + j0);
+            const float4 o = *m;
+            *m = make_float4(o.x - acc[a][0] + ev[a].x, o.y - acc[a][1] + ev[a].y,
+                             o.z - acc[a][2] + ev[a].z, o.w - acc[a][3] + ev[a].w);
+        }
+        if (s + 1 < NC) {
 #pragma unroll
-            for (int b = 0; b < RB; ++b) {
-                const int e = (i0 + a) * kScanCols + j0 + b;
-                Ms[e] = Ms[e] - acc[a][b] + E[(size_t)(i0 + a) * D + c0 + j0 + b];
-            }
+            for (int q = 0; q < NPF; ++q) *reinterpret_cast<float4 *>(As + 4 * (tid + q * kT)) = pf[q];
+        }
         __syncthreads();
     }
     if (dir == 1)
