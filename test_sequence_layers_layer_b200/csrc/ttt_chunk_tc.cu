@@ -61,15 +61,15 @@ constexpr int kChunkWs = kImgBytes + kD * kD * 4;
 //     count of scan slices that have stored W_c.
 // Every wait is on blocks with smaller tickets, which have started and wait
 // only on blocks before them, so the waits always end.
-constexpr int kGramRows = 32;                    // tokens per pipeline stage
-constexpr int kGramStages = 4;
-constexpr int kGramBox = kGramRows * 128;        // one 64-column box of a stage (4 KB)
+constexpr int kGramRows = 64;                    // tokens per pipeline stage
+constexpr int kGramStages = 2;
+constexpr int kGramBox = kGramRows * 128;        // one 64-column box of a stage (8 KB)
 constexpr int kGramStageBytes = 6 * kGramBox;    // K (2 boxes) | V (2) | eta*K (2)
 constexpr size_t kGramSmem = 1024 + kGramStages * kGramStageBytes;  // 97 KB: two blocks per SM
 // With one step size for the whole chunk, K itself is the A operand (no eta*K
 // copy, no conversion pass) and the accumulator is scaled by eta once: the
-// same 96 KB then hold 6 stages of K | V.
-constexpr int kGramStagesU = 6, kGramStageBytesU = 4 * kGramBox;
+// same 96 KB then hold 3 stages of K | V.
+constexpr int kGramStagesU = 3, kGramStageBytesU = 4 * kGramBox;
 static_assert(kGramStagesU * kGramStageBytesU <= kGramStages * kGramStageBytes, "uniform-eta ring");
 constexpr int kSlice = 64, kSlices = kD / kSlice;  // scan: output columns per block
 constexpr int kSliceImg = 2 * kSlice * kD * 2;     // [W hi | W lo] slice image [128][128] bf16: 32 KB
@@ -95,10 +95,11 @@ struct GramScanArgs {
     float *M = nullptr, *N = nullptr;
     // Forward: the read-out's output (bf16 instead when z_bf16) and the
     // number of read-out blocks per chunk (each takes chunk / parts tokens, a
-    // multiple of 128).
+    // multiple of 128); the last chunk of each sequence, read last, is split
+    // over parts_last blocks.
     float *Z = nullptr;
     bool z_bf16 = false;
-    int parts = 1;
+    int parts = 1, parts_last = 1;
 };
 
 // Read-out blocks per chunk, for n chunks: about 1024 read-out blocks in all
@@ -112,6 +113,15 @@ int readout_parts(int chunk, int n) {
     for (int p = want; p > 1; --p)
         if ((chunk / 128) % p == 0) return p;
     return 1;
+}
+
+// The last chunk's read-outs are the kernel's tail, run while fewer and
+// fewer blocks are left: up to 4x finer (one 128-token tile per block at
+// most), again a divisor of the chunk's tiles.
+int readout_parts_last(int chunk, int parts) {
+    for (int p = std::min(chunk / 128, 4 * parts); p > parts; --p)
+        if ((chunk / 128) % p == 0) return p;
+    return parts;
 }
 
 __device__ __forceinline__ int ld_acquire(const int *p) {
@@ -185,14 +195,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (tk >= n + nscan) {
         // ---- read-out of part `part` of chunk c of sequence s (chunk-major
         // ticket order): Z_c = Q_c W_c once both scan blocks of s have written
-        // W_c's image. A chunk's tokens are split over a.parts blocks, so that
-        // the last chunk's read-out, which waits for the whole scan, is short.
-        // Q does not depend on the scan: its first tiles load while the block
-        // waits for W_c.
-        const int ai = tk - n - nscan, per_c = a.nseq * a.parts;
-        const int c = ai / per_c, s = (ai % per_c) / a.parts, part = ai % a.parts;
+        // W_c's image. A chunk's tokens are split over a.parts blocks (the
+        // last chunk's over a.parts_last), so that the last chunk's read-out,
+        // which waits for the whole scan, is short. Q does not depend on the
+        // scan: its first tiles load while the block waits for W_c.
+        const int ai = tk - n - nscan, per_c = a.nseq * a.parts, head = (a.cps - 1) * per_c;
+        const bool last = ai >= head;
+        const int nparts = last ? a.parts_last : a.parts;
+        const int c = last ? a.cps - 1 : ai / per_c;
+        const int s = last ? (ai - head) / nparts : (ai % per_c) / nparts;
+        const int part = last ? (ai - head) % nparts : ai % nparts;
         const int g = s * a.cps + c;
-        const int ntile = a.chunk / a.parts / kApplyTile;
+        const int ntile = a.chunk / nparts / kApplyTile;
         const long row0 = (long)g * a.chunk + (long)part * ntile * kApplyTile;
         uint64_t *qfull = bars, *qempty = bars + kApplyStages, *wfull = bars + 2 * kApplyStages,
                  *tfull = wfull + 1, *tempty = wfull + 2;
@@ -526,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint8_t *sB = smem + kImgBytes;       // B_c columns j0.. (quad q of row i at float4 q * 128 + i)
     uint8_t *sWs = smem + 2 * kImgBytes;  // slice image: 2 column blocks of 16 KB
     uint64_t *aready = bars, *bready = bars + 1, *afree = bars + 2, *bfree = bars + 3,
-             *dfull = bars + 4, *wready = bars + 5;
+             *dfull = bars + 4, *wready = bars + 5, *imgfree = bars + 6;
     uint8_t *Wimg = a.ws + (size_t)n * kChunkWs;
     if (threadIdx.x == 0) {
         mbar_init(aready, 1);
@@ -535,6 +549,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(bfree, 4);  // one arrival per epilogue warp
         mbar_init(dfull, 1);
         mbar_init(wready, 1);
+        mbar_init(imgfree, 1);
         mbar_init(drain, 1);
         fence_mbar_init();
     }
@@ -579,9 +594,25 @@ __global__ void __launch_bounds__(kThreads, 2)
             issued = 2 * c + 2;
         }
     } else if (warp == 1 && lane == 0) {
+        // The product of each chunk, and W_c's share of the read-out operand:
+        // the slice image, read by the product, is also copied into chunk
+        // c's image in the workspace (K block kb of slice r at
+        // 32 KB kb + 16 KB r) by bulk store. The epilogue may rewrite the
+        // slice image once the store has read it (imgfree); the chunk is
+        // counted for the read-out once its store is complete, a step later.
+        // The waits and the memory fence are on this thread, which next
+        // waits for the epilogue, not on the epilogue's chain.
         const uint32_t idesc = make_idesc_bf16(128, 2 * kSlice, false, false);
         const uint32_t wb = smem_u32(sWs);
         const uint32_t ab = smem_u32(sA);
+        int released = 0;  // chunks whose image share is counted
+        auto release_upto = [&](int c_end) {
+            if (released >= c_end) return;
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __threadfence();
+            for (; released < c_end; ++released) atomicAdd(sync + 1 + n + g0 + released, 1);
+        };
+        int stored = 0;  // chunks whose image store is issued
         for (int c = 0; c < cps; ++c) {
             if (!mbar_wait(aready, c & 1, &abort_flag, a.status, 17)) break;
             if (!mbar_wait(wready, c & 1, &abort_flag, a.status, 18)) break;
@@ -595,6 +626,23 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             mma_commit(afree);
             mma_commit(dfull);
+            if (!map) {
+                uint8_t *img = Wimg + (g0 + c) * 65536 + (size_t)r * (kImgBytes / 2);
+                bulk_store(img, sWs, kImgBytes / 2);
+                bulk_store(img + kImgBytes, sWs + kImgBytes / 2, kImgBytes / 2);
+                bulk_commit();
+                stored = c + 1;
+            }
+            bulk_wait_read<0>();  // the slice image may be rewritten
+            mbar_arrive(imgfree);
+            if (!map) {
+                bulk_wait<1>();  // images of chunks < c are stored
+                release_upto(c);
+            }
+        }
+        if (!map) {
+            bulk_wait<0>();
+            if (stored == cps && !abort_flag) release_upto(cps);
         }
     } else if (warp >= 2) {
         // Epilogue: row i = 32 (warp & 3) + lane, columns j0 .. j0 + 63.
@@ -631,38 +679,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             fence_async_smem();
         };
-        // The slice image is also W_c's share of the read-out operand: one
-        // thread copies its two 16 KB K blocks into chunk c's image in the
-        // workspace (K block kb of slice r at 32 KB kb + 16 KB r) by bulk
-        // store, and counts the chunk for the read-out once the store is
-        // complete, a step later, so that neither the wait nor a memory fence
-        // lands on the scan's chain.
-        const bool pub = !map && warp == 2 && lane == 0;
-        auto store_image = [&](int c) {
-            uint8_t *img = Wimg + (g0 + c) * 65536 + (size_t)r * (kImgBytes / 2);
-            bulk_store(img, sWs, kImgBytes / 2);
-            bulk_store(img + kImgBytes, sWs + kImgBytes / 2, kImgBytes / 2);
-            bulk_commit();
-        };
-        int released = 0;  // chunks whose image share is counted
-        auto release_upto = [&](int c_end) {
-            if (released >= c_end) return;
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            __threadfence();
-            for (; released < c_end; ++released) atomicAdd(sync + 1 + n + g0 + released, 1);
-        };
         emit(0);
         bool ok = !named_bar_or(1, 128, false);
-        if (ok && pub) store_image(0);
         if (ok && warp == 2 && lane == 0) mbar_arrive(wready);
         for (int c = 0; ok && c < cps; ++c) {
             bool got = mbar_wait(bready, c & 1, &abort_flag, a.status, 19);
             got = got && mbar_wait(dfull, c & 1, &abort_flag, a.status, 20);
-            if (pub) {
-                bulk_wait_read<0>();  // the slice image may be rewritten after the barrier
-                bulk_wait<1>();       // images of chunks < c are stored
-                release_upto(c);
-            }
             if (named_bar_or(1, 128, !__all_sync(0xffffffffu, got))) {
                 ok = false;
                 break;
@@ -691,17 +713,17 @@ __global__ void __launch_bounds__(kThreads, 2)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bfree);  // this warp has read B_c
-            if (c + 1 < cps) emit(c + 1);
-            if (named_bar_or(1, 128, false)) {
+            // the next slice image, once the store of this one has read it
+            bool fr = true;
+            if (c + 1 < cps) {
+                fr = __all_sync(0xffffffffu, mbar_wait(imgfree, c & 1, &abort_flag, a.status, 27));
+                if (fr) emit(c + 1);
+            }
+            if (named_bar_or(1, 128, !fr)) {
                 ok = false;
                 break;
             }
-            if (c + 1 < cps && pub) store_image(c + 1);
             if (c + 1 < cps && warp == 2 && lane == 0) mbar_arrive(wready);
-        }
-        if (pub) {
-            bulk_wait<0>();
-            if (ok && !abort_flag) release_upto(cps);
         }
         if (ok && !abort_flag && out) {
             float *o = out + (size_t)s * kD * kD + (size_t)row * kD + j0;
@@ -789,8 +811,11 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     g.Z = a.Z;
     g.z_bf16 = a.z_bf16;
     g.parts = readout_parts(a.chunk, n);
-    // n Gram blocks, 2 scan blocks per sequence, parts read-out blocks per chunk
-    chunk_fwd_kernel<<<n + nseq * kSlices + n * g.parts, kThreads, kGramSmem, s>>>(tmK, tmV, tmQ, g);
+    g.parts_last = readout_parts_last(a.chunk, g.parts);
+    // n Gram blocks, 2 scan blocks per sequence, parts read-out blocks per
+    // chunk (parts_last for the last chunk of each sequence)
+    const int nread = nseq * ((cps - 1) * g.parts + g.parts_last);
+    chunk_fwd_kernel<<<n + nseq * kSlices + nread, kThreads, kGramSmem, s>>>(tmK, tmV, tmQ, g);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
