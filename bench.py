@@ -476,7 +476,7 @@ def gpu_arm(args, wl, rank, world, keep=None):
         "kernels": kernels,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "copies": f"overlapped over {slices} batch slices (hostio)" if sliced
+                "copies": f"overlapped over {slices} slices of the (batch, head) grid (hostio)" if sliced
                 else "in series with the call"},
         "gpu_launches": launches,
         "clocks": clocks,
@@ -992,7 +992,7 @@ def main():
                          "(ttt_linear_decode_tokens, ttt_mlp_decode_tokens)")
     ap.add_argument("--e2e-slices", type=int, default=None,
                     help="e2e leg (linear and large-chunk workloads): overlap the host copies with "
-                         "the compute over N batch slices (hostio.linear_fwd_host, "
+                         "the compute over N slices of the (batch, head) grid (hostio.linear_fwd_host, "
                          "hostio.chunk_fwd_host); default 4, 0 = copies in series with one call")
     ap.add_argument("--segments", type=int, default=0,
                     help="time the large-chunk forward split into N segments per sequence")

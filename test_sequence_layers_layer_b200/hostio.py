@@ -1,10 +1,14 @@
 """TTT-Linear and large-chunk forwards on inputs that live in host memory,
 with the copies overlapped with the compute.
 
-The batch is cut into `slices` groups of whole batch rows (every group holds
-all heads of its rows, so a shared W0 [H, d, d] serves every group). Each
-group runs on its own CUDA stream: its Q, K, V and eta are copied to the
-device, ttt_linear_fwd runs on them, and its Z and W_out are copied back. The
+The (batch, head) grid is cut into `slices` groups: whole batch rows while
+there are at least as many rows as groups, else each row's heads split into
+runs (a run of heads of one row is contiguous in [B, H, T, d], and W0, gamma
+and beta are cut to the same heads). Each group runs on its own CUDA stream:
+its Q, K, V and eta are copied to the device, ttt_linear_fwd runs on them,
+and its Z and W_out are copied back. The host-to-device copies are issued in
+group order, each after the previous group's (so the first group's kernel
+starts after 1/slices of the input has crossed, not all of it); the
 host-to-device copies of later groups, the device-to-host copies of earlier
 ones and the kernels of the groups in between then proceed at the same time.
 A sequence's result does not depend on which other sequences share its call,
@@ -32,15 +36,24 @@ def _streams(dev, n):
     return have[:n]
 
 
-def _bounds(B: int, slices: int):
-    n = max(1, min(slices, B))
-    q, r = divmod(B, n)
-    out, b0 = [], 0
-    for i in range(n):
-        b1 = b0 + q + (1 if i < r else 0)
-        out.append((b0, b1))
-        b0 = b1
+def _split(n: int, parts: int):
+    """[0, n) cut into `parts` runs whose lengths differ by at most one."""
+    q, r = divmod(n, parts)
+    out, a = [], 0
+    for i in range(parts):
+        b = a + q + (1 if i < r else 0)
+        out.append((a, b))
+        a = b
     return out
+
+
+def _bounds(B: int, H: int, slices: int):
+    """Groups (b0, b1, h0, h1): whole batch rows when slices <= B, else runs
+    of heads of one batch row each (about slices / B runs per row)."""
+    if slices <= B:
+        return [(b0, b1, 0, H) for b0, b1 in _split(B, max(1, slices))]
+    per_row = min(H, -(-slices // B))
+    return [(b, b + 1, h0, h1) for b in range(B) for h0, h1 in _split(H, per_row)]
 
 
 def _outputs(Q, z_bf16, out):
@@ -71,15 +84,23 @@ def linear_fwd_host(Q, K, V, eta, W0, ln_gamma=None, ln_beta=None, *, b, ln, sli
     gd = ln_gamma.to(dev, non_blocking=True) if ln_gamma is not None else None
     bd = ln_beta.to(dev, non_blocking=True) if ln_beta is not None else None
     Zh, Wh = _outputs(Q, z_bf16, out)
-    bounds = _bounds(B, slices)
+    bounds = _bounds(B, H, slices)
     streams = _streams(dev, len(bounds))
-    for (b0, b1), st in zip(bounds, streams):
+    prev = None  # the previous group's input copies
+    for (b0, b1, h0, h1), st in zip(bounds, streams):
         st.wait_stream(cur)  # W0, gamma, beta are copied on the current stream
+        if prev is not None:
+            st.wait_event(prev)
         with torch.cuda.stream(st):
-            q, k, v, e = (x[b0:b1].to(dev, non_blocking=True) for x in (Q, K, V, eta))
-            Z, W = _lib.linear_fwd(q, k, v, e, W0d, gd, bd, b=b, ln=ln, stream=st, z_bf16=z_bf16)
-            Zh[b0:b1].copy_(Z, non_blocking=True)
-            Wh[b0:b1].copy_(W, non_blocking=True)
+            q, k, v, e = (x[b0:b1, h0:h1].to(dev, non_blocking=True) for x in (Q, K, V, eta))
+            prev = torch.cuda.Event()
+            prev.record(st)
+            Z, W = _lib.linear_fwd(q, k, v, e, W0d[h0:h1],
+                                   gd[h0:h1] if gd is not None else None,
+                                   bd[h0:h1] if bd is not None else None,
+                                   b=b, ln=ln, stream=st, z_bf16=z_bf16)
+            Zh[b0:b1, h0:h1].copy_(Z, non_blocking=True)
+            Wh[b0:b1, h0:h1].copy_(W, non_blocking=True)
     for st in streams:
         cur.wait_stream(st)
     return Zh, Wh
@@ -99,17 +120,23 @@ def chunk_fwd_host(Q, K, V, eta, W0, *, chunk, slices=4, w0_per_seq=False, z_bf1
     cur = torch.cuda.current_stream(dev)
     W0d = W0.to(dev, non_blocking=True)
     Zh, Wh = _outputs(Q, z_bf16, out)
-    bounds = _bounds(B, slices)
+    H = Q.shape[1]
+    bounds = _bounds(B, H, slices)
     streams = _streams(dev, len(bounds))
-    for (b0, b1), st in zip(bounds, streams):
+    prev = None  # the previous group's input copies
+    for (b0, b1, h0, h1), st in zip(bounds, streams):
         st.wait_stream(cur)  # W0 is copied on the current stream
+        if prev is not None:
+            st.wait_event(prev)
         with torch.cuda.stream(st):
-            q, k, v, e = (x[b0:b1].to(dev, non_blocking=True) for x in (Q, K, V, eta))
-            w0 = W0d[b0:b1] if w0_per_seq else W0d
+            q, k, v, e = (x[b0:b1, h0:h1].to(dev, non_blocking=True) for x in (Q, K, V, eta))
+            prev = torch.cuda.Event()
+            prev.record(st)
+            w0 = W0d[b0:b1, h0:h1] if w0_per_seq else W0d[h0:h1]
             Z, W = _lib.chunk_fwd(q, k, v, e, w0, chunk=chunk, w0_per_seq=w0_per_seq, stream=st,
                                   z_bf16=z_bf16)
-            Zh[b0:b1].copy_(Z, non_blocking=True)
-            Wh[b0:b1].copy_(W, non_blocking=True)
+            Zh[b0:b1, h0:h1].copy_(Z, non_blocking=True)
+            Wh[b0:b1, h0:h1].copy_(W, non_blocking=True)
     for st in streams:
         cur.wait_stream(st)
     return Zh, Wh

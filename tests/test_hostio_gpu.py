@@ -1,7 +1,7 @@
 """TTT-Linear forward from pinned host buffers with copies overlapped across
-batch slices (hostio.linear_fwd_host): its outputs equal one ttt_linear_fwd
-call on the device over the whole batch, bit for bit (a sequence's result does
-not depend on which sequences share its call)."""
+slices of the (batch, head) grid (hostio.linear_fwd_host): its outputs equal
+one ttt_linear_fwd call on the device over the whole batch, bit for bit (a
+sequence's result does not depend on which sequences share its call)."""
 import pytest
 import torch
 
@@ -15,7 +15,8 @@ L = synth.WORKLOADS["linear_ln_d64_b8h12_t2048"]
 
 
 @pytest.mark.parametrize("B,slices,z_bf16,ln", [(3, 1, False, True), (5, 3, False, True),
-                                               (8, 4, True, True), (4, 4, False, False)])
+                                               (8, 4, True, True), (4, 4, False, False),
+                                               (2, 5, False, True)])
 def test_host_pipeline_equals_device_call(B, slices, z_bf16, ln):
     wl = L.scaled(B=B, H=3, T=160, ln=ln)
     x = to_dev(synth.make_inputs(wl))
@@ -35,7 +36,8 @@ C = synth.WORKLOADS["chunk_d128_c2048_b4h8_t32768"]
 
 
 @pytest.mark.parametrize("B,slices,z_bf16,per_seq", [(3, 3, False, False), (4, 2, True, False),
-                                                    (2, 2, False, True)])
+                                                    (2, 2, False, True), (2, 4, False, False),
+                                                    (1, 2, True, True)])
 def test_chunk_host_pipeline_equals_device_call(B, slices, z_bf16, per_seq):
     """Large-chunk forward from pinned host buffers, one workspace per slice,
     outputs written into caller-given pinned buffers: equal to one
