@@ -32,9 +32,9 @@ cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V
 bool chunk_bwd_tok_tc_supported(int d, int chunk, bool bf16);
 size_t chunk_bwd_tok_tc_scratch_bytes(size_t tokens);
 cudaError_t launch_chunk_bwd_tok_tc(const void *K, const void *V, const float *eta, const float *dZ,
-                                    const float *W, const float *Om, int B, int H, int T, int chunk,
-                                    void *scratch, float *dQ, float *dK, float *dV, float *deta,
-                                    cudaStream_t s);
+                                    const float *W, const float *Om, float *S, size_t s_stride,
+                                    int B, int H, int T, int chunk, void *scratch, float *dQ,
+                                    float *dK, float *dV, float *deta, cudaStream_t s);
 
 namespace {
 
@@ -365,8 +365,10 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launch(s);
     if (tok_tc) {
-        if ((e = launch_chunk_bwd_tok_tc(K, V, eta, dZ, w.W, w.Om, B, H, T, C, scratch, dQ, dK, dV,
-                                         deta, s)) != cudaSuccess)
+        // each chunk's S = W_c Om_{c+1}^T + Om_{c+1} W_c^T takes the place of
+        // its A_c, which only the scans read
+        if ((e = launch_chunk_bwd_tok_tc(K, V, eta, dZ, w.W, w.Om, w.gram, 3 * (size_t)D * D, B, H,
+                                         T, C, scratch, dQ, dK, dV, deta, s)) != cudaSuccess)
             return e;
     } else {
         const size_t tsm = tok_smem_bytes(D);

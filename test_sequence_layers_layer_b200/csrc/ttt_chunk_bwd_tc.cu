@@ -249,16 +249,14 @@ bool chunk_bwd_gram_tc_supported(int d, int chunk, bool bf16) {
     return bf16 && d == kD && chunk >= kRows && chunk % kRows == 0;
 }
 
-// The token passes' operand rows in their scratch: R | P hi and lo
-// ([tokens][2d]), then dZ hi and lo ([tokens][d]), all bf16.
+// The token passes' operand rows in their scratch: dZ hi and lo
+// ([tokens][d] each), bf16.
 struct TokScratch {
-    __nv_bfloat16 *rp_hi, *rp_lo, *z_hi, *z_lo;
+    __nv_bfloat16 *z_hi, *z_lo;
 };
 TokScratch tok_scratch(void *scratch, uint64_t rows) {
     TokScratch t;
-    t.rp_hi = static_cast<__nv_bfloat16 *>(scratch);
-    t.rp_lo = t.rp_hi + rows * 2 * kD;
-    t.z_hi = t.rp_lo + rows * 2 * kD;
+    t.z_hi = static_cast<__nv_bfloat16 *>(scratch);
     t.z_lo = t.z_hi + rows * kD;
     return t;
 }
@@ -298,18 +296,24 @@ cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V
 // 128, bf16 inputs, chunk a multiple of 128), with W = W_c and Om = Om_{c+1}
 // of each token's chunk:
 //   R = K W - V,  P = K Om,  dV = diag(eta) P,  deta_t = -P_t . R_t,
-//   dK = -diag(eta) [R | P] [Om | W]^T,  dQ = dZ W^T,
+//   dK = -diag(eta) (R Om^T + P W^T) = -diag(eta) (K S - V Om^T),
+//       with S = W Om^T + Om W^T (one d x d matrix per chunk),
+//   dQ = dZ W^T,
 // as three passes of one kernel over 128-token tiles, a block per chunk:
 //   RP: D = K [W | Om] (N = 256, K = d_in): A = K (exact), B = [W | Om]^T as
-//       hi and lo terms; the epilogue forms R, dV, deta and writes R, P as
-//       bf16 hi/lo operand rows into the workspace (dZ's rows come from the
-//       Gram kernel, which splits dZ anyway);
-//   DK: D = [R | P]_{hi,lo} [Om | W]^T (K = 256);  DQ: D = dZ_{hi,lo} W^T (K = 128):
-//       B stacked as [hi rows | lo rows] (N = 256), so A_hi x B gives the hi.hi
-//       and hi.lo terms side by side and A_lo x B_hi adds lo.hi to the first half.
-// A tiles arrive by TMA one 64-wide K block at a time (3-stage ring); B is
-// built once per block in shared memory from the fp32 W and Om (K-major,
-// 128-byte swizzle); accumulators double-buffered in tensor memory.
+//       hi and lo terms; the epilogue forms R, dV and deta. Before its tiles
+//       the block also forms S from the same two B images (S[i][j] = sum over
+//       the 256 rows n of B[n][i] B[n +- 128][j]: both operands MN-major
+//       views of the images, hi.hi + hi.lo + lo.hi) and stores it in fp32;
+//   DK: D = [K | V] [S ; -Om^T] (K = 256, A exact); DQ: D = dZ_{hi,lo} W^T
+//       (K = 128): B stacked as [hi rows | lo rows] (N = 256), so A x B gives
+//       the hi and lo terms side by side (and, for DQ, A_lo x B_hi adds lo.hi
+//       to the first half).
+// So no per-token intermediate crosses HBM between the passes (dZ's bf16
+// rows come from the Gram kernel, which splits dZ anyway). A tiles arrive by
+// TMA one 64-wide K block at a time; B is built once per block in shared
+// memory from fp32 (K-major, 128-byte swizzle); accumulators double-buffered
+// in tensor memory.
 namespace {
 
 enum { kModeRP = 0, kModeDK = 1, kModeDQ = 2 };
@@ -325,7 +329,8 @@ struct TokArgs {
     const float *eta, *dZ;
     float *out;           // RP: dV; DK: dK; DQ: dQ   ([tokens][d] fp32)
     float *deta;          // RP only
-    __nv_bfloat16 *rp_hi, *rp_lo, *z_hi, *z_lo;  // RP writes them; DK and DQ read them by TMA
+    float *S;             // chunk g's S at S + g * s_stride (RP writes, DK reads)
+    size_t s_stride;
     int chunk;
     int *status;
 };
@@ -365,14 +370,14 @@ __global__ void __launch_bounds__(kTokThreads, 1)
                      TokArgs a) {
     constexpr int KD = kMode == kModeDK ? 2 * kD : kD;  // reduction length
     constexpr int NKB = KD / 64;                         // 64-wide K blocks per tile
-    constexpr bool kTwoA = kMode != kModeRP;             // A as hi and lo terms
+    constexpr bool kTwoA = kMode == kModeDQ;             // A as hi and lo terms
     // B image rows per K block: RP keeps hi and lo as two images of 256 rows
     // ([W | Om]^T); DK and DQ stack [hi rows | lo rows] of their 128 rows.
     constexpr int BR = 2 * kD;
     constexpr uint32_t kBLoOff = kMode == kModeRP ? (uint32_t)NKB * BR * 128 : 0u;
-    // A ring: one or two terms of a 64-wide K block per stage; DK's B images
-    // (128 KB) leave room for two stages beside the epilogue's staging.
-    constexpr int STAGES = kMode == kModeDK ? 2 : 3;
+    // A ring: one or two terms of a 64-wide K block per stage (DK: the K
+    // blocks of K, then of V).
+    constexpr int STAGES = kMode == kModeDK ? 4 : 3;
     constexpr int SBYTES = kTwoA ? kTokStage : kTokStage / 2;
     constexpr int BBYTES = NKB * BR * 128 * (kMode == kModeRP ? 2 : 1);  // B images
     static_assert(BBYTES + STAGES * SBYTES + 4 * kStgWarp + 1024 <= (int)kTokSmem, "smem plan");
@@ -380,7 +385,7 @@ __global__ void __launch_bounds__(kTokThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sB = smem, *sA = smem + BBYTES;
-    __shared__ uint64_t full[kTokStages], empty[kTokStages], bready, tfull[2], tempty[2], drain;
+    __shared__ uint64_t full[4], empty[4], bready, tfull[2], tempty[2], sfull, sfree, drain;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -391,11 +396,13 @@ __global__ void __launch_bounds__(kTokThreads, 1)
 
     if (threadIdx.x == 0) {
         abort_flag = 0;
-        for (int s = 0; s < kTokStages; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(&bready, 128);
+        mbar_init(&sfull, 1);
+        mbar_init(&sfree, 128);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 128);
@@ -421,7 +428,10 @@ __global__ void __launch_bounds__(kTokThreads, 1)
                 uint8_t *sb = sA + st * SBYTES;
                 const int y = (int)(row0 + (long)t * kTokTile);
                 mbar_arrive_expect_tx(&full[st], SBYTES);
-                tma_load_2d(sb, &tmA_hi, 64 * kb, y, &full[st]);
+                if (kMode == kModeDK)  // [K | V]: K blocks 0-1 of K, 2-3 of V
+                    tma_load_2d(sb, kb < 2 ? &tmA_hi : &tmA_lo, 64 * (kb & 1), y, &full[st]);
+                else
+                    tma_load_2d(sb, &tmA_hi, 64 * kb, y, &full[st]);
                 if (kTwoA) tma_load_2d(sb + kTokStage / 2, &tmA_lo, 64 * kb, y, &full[st]);
                 issued = u + 1;
             }
@@ -432,9 +442,33 @@ __global__ void __launch_bounds__(kTokThreads, 1)
         const uint32_t id128 = make_idesc_bf16(128, 128, false, false);
         const uint32_t bb = smem_u32(sB), ab = smem_u32(sA);
         if (mbar_wait(&bready, 0, &abort_flag, a.status, 102)) {
+            if (kMode == kModeRP) {
+                // S = W Om^T + Om W^T into columns 256-383 (the second
+                // accumulator, free until tile 1): row n of the image
+                // holds W[n][.] (n < 128) or Om[n - 128][.], so
+                // S[i][j] = sum_n img[n][i] img[(n + 128) % 256][j]; both
+                // operands are MN-major views (64-value blocks 32 KB apart,
+                // 8-row groups 1 KB apart), 16 rows n per instruction.
+                const uint32_t ids = make_idesc_bf16(128, 128, true, true);
+                constexpr uint32_t kBlk = (uint32_t)BR * 128;
+                for (int n0 = 0, first = 1; n0 < 2 * kD; n0 += 16) {
+                    const uint32_t ra = (uint32_t)n0 * 128, rb = (uint32_t)((n0 + kD) % (2 * kD)) * 128;
+                    const uint64_t ah = make_sdesc(bb + ra, kBlk, 1024, kSw128);
+                    const uint64_t al = make_sdesc(bb + kBLoOff + ra, kBlk, 1024, kSw128);
+                    const uint64_t bh = make_sdesc(bb + rb, kBlk, 1024, kSw128);
+                    const uint64_t bl = make_sdesc(bb + kBLoOff + rb, kBlk, 1024, kSw128);
+                    mma_bf16(tm + 256, ah, bh, ids, !first);
+                    mma_bf16(tm + 256, ah, bl, ids, true);
+                    mma_bf16(tm + 256, al, bh, ids, true);
+                    first = 0;
+                }
+                mma_commit(&sfull);
+            }
             for (int t = 0, u = 0; t < ntile; ++t) {
                 const int acc = t & 1;
                 if (t >= 2 && !mbar_wait(&tempty[acc], ((t >> 1) - 1) & 1, &abort_flag, a.status, 103))
+                    break;
+                if (kMode == kModeRP && t == 1 && !mbar_wait(&sfree, 0, &abort_flag, a.status, 106))
                     break;
                 tc_fence_after();
                 const uint32_t d = tm + 256 * acc;
@@ -457,10 +491,12 @@ __global__ void __launch_bounds__(kTokThreads, 1)
                             const uint64_t blo = make_sdesc(bb + kBLoOff + kb * BR * 128 + ko, 16, 1024, kSw128);
                             mma_bf16(d, ahi, bhi, id256, accum);
                             mma_bf16(d, ahi, blo, id256, true);
-                        } else {
+                        } else if (kTwoA) {
                             const uint64_t alo = make_sdesc(a0 + kTokStage / 2 + ko, 16, 1024, kSw128);
                             mma_bf16(d, ahi, bhi, id256, accum);  // hi.hi | hi.lo
                             mma_bf16(d, alo, bhi, id128, true);   // + lo.hi (first half)
+                        } else {
+                            mma_bf16(d, ahi, bhi, id256, accum);  // A.hi | A.lo
                         }
                     }
                     mma_commit(&empty[st]);
@@ -474,28 +510,31 @@ __global__ void __launch_bounds__(kTokThreads, 1)
         // ---- B operand images from the fp32 W and Om of the chunk
         {
             const float *Wc = a.W + (size_t)g * dd, *Oc = a.Om + (size_t)g * dd;
+            const float *Sc = a.S + (size_t)g * a.s_stride;
             // units: (row n, 8 consecutive k)
             constexpr int NROWS = kMode == kModeRP ? 2 * kD : kD;
+            constexpr bool kColRead = kMode != kModeDQ;  // consecutive threads take consecutive n
             for (int uidx = tt; uidx < NROWS * (KD / 8); uidx += 128) {
-                // RP reads W and Om transposed: consecutive threads take
-                // consecutive n (one 128-byte row segment per warp load);
-                // DK and DQ read rows: consecutive threads take consecutive k
-                const int n = kMode == kModeRP ? uidx % NROWS : uidx / (KD / 8);
-                const int k0 = kMode == kModeRP ? 8 * (uidx / NROWS) : 8 * (uidx % (KD / 8));
+                // Column reads (RP's W and Om, DK's S) go with consecutive
+                // threads on consecutive n (one 128-byte row segment per warp
+                // load); row reads with consecutive k
+                const int n = kColRead ? uidx % NROWS : uidx / (KD / 8);
+                const int k0 = kColRead ? 8 * (uidx / NROWS) : 8 * (uidx % (KD / 8));
                 float f[8];
-                if (kMode == kModeRP) {
-                    // B[n][k]: n < 128: W[k][n]; else Om[k][n - 128]  (K = d_in)
-                    const float *src = n < kD ? Wc + n : Oc + (n - kD);
+                if (kMode == kModeRP || (kMode == kModeDK && k0 < kD)) {
+                    // RP: B[n][k] = W[k][n] (n < 128) or Om[k][n - 128] (K = d_in);
+                    // DK, k < 128: B[n][k] = S[k][n]
+                    const float *src = kMode == kModeDK ? Sc + n : (n < kD ? Wc + n : Oc + (n - kD));
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[e] = src[(size_t)(k0 + e) * kD];
                 } else {
-                    // B[n][k]: DK: k < 128: Om[n][k], else W[n][k - 128]; DQ: W[n][k]
-                    const float *src = (kMode == kModeDK && k0 < kD) ? Oc + (size_t)n * kD + k0
-                                       : Wc + (size_t)n * kD + (k0 & (kD - 1));
+                    // DK, k >= 128: B[n][k] = -Om[n][k - 128]; DQ: B[n][k] = W[n][k]
+                    const float *src = (kMode == kModeDK ? Oc : Wc) + (size_t)n * kD + (k0 & (kD - 1));
+                    const float sg = kMode == kModeDK ? -1.f : 1.f;
                     const float4 u0 = *reinterpret_cast<const float4 *>(src);
                     const float4 u1 = *reinterpret_cast<const float4 *>(src + 4);
-                    f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w;
-                    f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
+                    f[0] = sg * u0.x; f[1] = sg * u0.y; f[2] = sg * u0.z; f[3] = sg * u0.w;
+                    f[4] = sg * u1.x; f[5] = sg * u1.y; f[6] = sg * u1.z; f[7] = sg * u1.w;
                 }
                 uint2 h0, l0, h1, l1;
                 split4(f[0], f[1], f[2], f[3], h0, l0);
@@ -517,7 +556,29 @@ __global__ void __launch_bounds__(kTokThreads, 1)
         // goes through the warp's staging rows (whole row segments)
         const int sp = warp & 3;
         uint8_t *stg = sA + STAGES * SBYTES + (warp - 2) * kStgWarp;
-        for (int t = 0; t < ntile; ++t) {
+        bool run = true;
+        if (kMode == kModeRP) {
+            // S: lane = row i, 128 fp32 columns from tensor memory
+            run = __all_sync(0xffffffffu, mbar_wait(&sfull, 0, &abort_flag, a.status, 107));
+            if (run) {
+                tc_fence_after();
+                uint8_t *s0 = reinterpret_cast<uint8_t *>(a.S + (size_t)g * a.s_stride + (size_t)32 * sp * kD);
+#pragma unroll 1
+                for (int q = 0; q < kD / 32; ++q) {
+                    float x[32];
+                    tmem_ld16(taddr(tm, 32 * sp, 256 + 32 * q), *reinterpret_cast<float(*)[16]>(&x[0]));
+                    tmem_ld16(taddr(tm, 32 * sp, 256 + 32 * q + 16), *reinterpret_cast<float(*)[16]>(&x[16]));
+                    tmem_ld_wait();
+                    uint4 o8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o8[e] = pack4f(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                    warp_rows_out<8>(stg, o8, s0 + 128 * q, 4 * kD, lane);
+                }
+                tc_fence_before();
+                mbar_arrive(&sfree);  // columns 256-383 are free for tile 1
+            }
+        }
+        for (int t = 0; run && t < ntile; ++t) {
             const int acc = t & 1;
             const long tokw = row0 + (long)t * kTokTile + 32 * sp;  // the warp's first token
             const long tok = tokw + lane;
@@ -566,25 +627,6 @@ __global__ void __launch_bounds__(kTokThreads, 1)
                     }
                     warp_rows_out<8>(stg, o8, reinterpret_cast<uint8_t *>(a.out + tokw * kD + 32 * q),
                                      4 * kD, lane);  // dV
-                    // R and P as bf16 hi/lo operand rows ([t][R (128) | P (128)])
-                    uint4 rh[4], rl[4], ph[4], pl[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        uint2 a0, b0, a1, b1;
-                        split4(r[8 * e], r[8 * e + 1], r[8 * e + 2], r[8 * e + 3], a0, b0);
-                        split4(r[8 * e + 4], r[8 * e + 5], r[8 * e + 6], r[8 * e + 7], a1, b1);
-                        rh[e] = make_uint4(a0.x, a0.y, a1.x, a1.y);
-                        rl[e] = make_uint4(b0.x, b0.y, b1.x, b1.y);
-                        split4(p[8 * e], p[8 * e + 1], p[8 * e + 2], p[8 * e + 3], a0, b0);
-                        split4(p[8 * e + 4], p[8 * e + 5], p[8 * e + 6], p[8 * e + 7], a1, b1);
-                        ph[e] = make_uint4(a0.x, a0.y, a1.x, a1.y);
-                        pl[e] = make_uint4(b0.x, b0.y, b1.x, b1.y);
-                    }
-                    const size_t rpo = (size_t)tokw * 2 * kD + 32 * q;
-                    warp_rows_out<4>(stg, rh, reinterpret_cast<uint8_t *>(a.rp_hi + rpo), 4 * kD, lane);
-                    warp_rows_out<4>(stg, rl, reinterpret_cast<uint8_t *>(a.rp_lo + rpo), 4 * kD, lane);
-                    warp_rows_out<4>(stg, ph, reinterpret_cast<uint8_t *>(a.rp_hi + rpo + kD), 4 * kD, lane);
-                    warp_rows_out<4>(stg, pl, reinterpret_cast<uint8_t *>(a.rp_lo + rpo + kD), 4 * kD, lane);
                 }
                 tc_fence_before();
                 mbar_arrive(&tempty[acc]);
@@ -647,32 +689,32 @@ bool chunk_bwd_tok_tc_supported(int d, int chunk, bool bf16) {
     return bf16 && d == kD && chunk >= kTokTile && chunk % kTokTile == 0;
 }
 
-// Workspace bytes of the tensor-core token passes: R | P and dZ as bf16 hi
-// and lo rows (1.5 KiB per token).
-size_t chunk_bwd_tok_tc_scratch_bytes(size_t tokens) { return tokens * (2 * 2 * kD + 2 * kD) * 2; }
+// Workspace bytes of the tensor-core token passes: dZ as bf16 hi and lo rows
+// (512 bytes per token).
+size_t chunk_bwd_tok_tc_scratch_bytes(size_t tokens) { return tokens * 2 * kD * 2; }
 
+// S of chunk g goes to S + g * s_stride floats (the caller's d x d slot per
+// chunk, free once the scans have run).
 cudaError_t launch_chunk_bwd_tok_tc(const void *K, const void *V, const float *eta, const float *dZ,
-                                    const float *W, const float *Om, int B, int H, int T, int chunk,
-                                    void *scratch, float *dQ, float *dK, float *dV, float *deta,
-                                    cudaStream_t s) {
+                                    const float *W, const float *Om, float *S, size_t s_stride,
+                                    int B, int H, int T, int chunk, void *scratch, float *dQ,
+                                    float *dK, float *dV, float *deta, cudaStream_t s) {
     const uint64_t rows = (uint64_t)B * H * T;
     const int nch = B * H * (T / chunk);
     const TokScratch ts = tok_scratch(scratch, rows);
-    __nv_bfloat16 *rp_hi = ts.rp_hi, *rp_lo = ts.rp_lo, *z_hi = ts.z_hi, *z_lo = ts.z_lo;
     int *status = device_status_word();
-    alignas(64) CUtensorMap tmK, tmRPh, tmRPl, tmZh, tmZl;
+    alignas(64) CUtensorMap tmK, tmV, tmZh, tmZl;
     if (!encode_tmap_2d(&tmK, K, false, kD, rows, 64, kTokTile) ||
-        !encode_tmap_2d(&tmRPh, rp_hi, false, 2 * kD, rows, 64, kTokTile) ||
-        !encode_tmap_2d(&tmRPl, rp_lo, false, 2 * kD, rows, 64, kTokTile) ||
-        !encode_tmap_2d(&tmZh, z_hi, false, kD, rows, 64, kTokTile) ||
-        !encode_tmap_2d(&tmZl, z_lo, false, kD, rows, 64, kTokTile))
+        !encode_tmap_2d(&tmV, V, false, kD, rows, 64, kTokTile) ||
+        !encode_tmap_2d(&tmZh, ts.z_hi, false, kD, rows, 64, kTokTile) ||
+        !encode_tmap_2d(&tmZl, ts.z_lo, false, kD, rows, 64, kTokTile))
         return cudaErrorInvalidValue;
-    TokArgs a{W, Om, static_cast<const __nv_bfloat16 *>(V), eta, dZ, dV, deta,
-              rp_hi, rp_lo, z_hi, z_lo, chunk, status};
+    TokArgs a{W, Om, static_cast<const __nv_bfloat16 *>(V), eta, dZ, dV, deta, S, s_stride,
+              chunk, status};
     cudaError_t e = launch_tok_mode<kModeRP>(tmK, tmK, a, nch, s);
     if (e != cudaSuccess) return e;
     a.out = dK;
-    if ((e = launch_tok_mode<kModeDK>(tmRPh, tmRPl, a, nch, s)) != cudaSuccess) return e;
+    if ((e = launch_tok_mode<kModeDK>(tmK, tmV, a, nch, s)) != cudaSuccess) return e;
     a.out = dQ;
     return launch_tok_mode<kModeDQ>(tmZh, tmZl, a, nch, s);
 }
