@@ -318,14 +318,15 @@ __global__ void __launch_bounds__(kT) cb_tok_kernel(const TIn *K, const TIn *V, 
 
 size_t tok_smem_bytes(int D) { return (2 * (size_t)D * (D + 1) + 5 * 32 * (size_t)D) * sizeof(float); }
 
-// out[h][e] = sum_b in[b * H + h][e], fixed order.
+// out[h][e] = sum_b in[b * H + h][e], fixed order; a thread per element
+// (grid: elements x H), so the B loads of all elements are in flight at once.
 __global__ void cb_sum_over_batch_kernel(const float *in, float *out, int B, int H, int n) {
-    const int h = blockIdx.x;
-    for (int e = threadIdx.x; e < n; e += blockDim.x) {
-        float acc = 0.f;
-        for (int bb = 0; bb < B; ++bb) acc += in[((size_t)bb * H + h) * n + e];
-        out[(size_t)h * n + e] = acc;
-    }
+    const int h = blockIdx.y;
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= n) return;
+    float acc = 0.f;
+    for (int bb = 0; bb < B; ++bb) acc += in[((size_t)bb * H + h) * n + e];
+    out[(size_t)h * n + e] = acc;
 }
 
 template <typename TIn, int D>
@@ -382,7 +383,7 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
         count_launch(s);
     }
     if (!w0_per_seq) {
-        cb_sum_over_batch_kernel<<<H, 256, 0, s>>>(w.dW0s, dW0, B, H, D * D);
+        cb_sum_over_batch_kernel<<<dim3((D * D + 255) / 256, H), 256, 0, s>>>(w.dW0s, dW0, B, H, D * D);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         count_launch(s);
     }

@@ -545,14 +545,15 @@ __global__ void __launch_bounds__(kBwdThreads) linear_bwd_kernel(BwdArgs a) {
 }
 
 // Sums per-sequence gradients of per-head parameters over the batch, in a
-// fixed order: out[h][e] = sum_b in[b * H + h][e] for e < n.
+// fixed order: out[h][e] = sum_b in[b * H + h][e] for e < n; a thread per
+// element (grid: elements x H).
 __global__ void sum_over_batch_kernel(const float *in, float *out, int B, int H, int n) {
-    const int h = blockIdx.x;
-    for (int e = threadIdx.x; e < n; e += blockDim.x) {
-        float acc = 0.f;
-        for (int bb = 0; bb < B; ++bb) acc += in[((size_t)bb * H + h) * n + e];
-        out[(size_t)h * n + e] = acc;
-    }
+    const int h = blockIdx.y;
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= n) return;
+    float acc = 0.f;
+    for (int bb = 0; bb < B; ++bb) acc += in[((size_t)bb * H + h) * n + e];
+    out[(size_t)h * n + e] = acc;
 }
 
 }  // namespace
@@ -595,15 +596,15 @@ cudaError_t launch_linear_bwd(const LinearBwdArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     count_launch(s);
     if (!a.w0_per_seq) {
-        sum_over_batch_kernel<<<a.H, 256, 0, s>>>(k.dW0s, a.dW0, a.B, a.H, (int)dd);
+        sum_over_batch_kernel<<<dim3(((int)dd + 255) / 256, a.H), 256, 0, s>>>(k.dW0s, a.dW0, a.B, a.H, (int)dd);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         count_launch(s);
     }
     if (a.ln) {
-        sum_over_batch_kernel<<<a.H, 64, 0, s>>>(k.dgs, a.dgamma, a.B, a.H, a.d);
+        sum_over_batch_kernel<<<dim3((a.d + 63) / 64, a.H), 64, 0, s>>>(k.dgs, a.dgamma, a.B, a.H, a.d);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         count_launch(s);
-        sum_over_batch_kernel<<<a.H, 64, 0, s>>>(k.dbs, a.dbeta, a.B, a.H, a.d);
+        sum_over_batch_kernel<<<dim3((a.d + 63) / 64, a.H), 64, 0, s>>>(k.dbs, a.dbeta, a.B, a.H, a.d);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         count_launch(s);
     }
