@@ -889,7 +889,9 @@ def backward_arm(args, wl):
     kern_ms = (sum(kern) if chunk else kern[0]) / args.steps
     tc_gram = chunk and wl.d == 128 and wl.dtype == "bf16" and wl.b % 32 == 0
     tc_tok = tc_gram and wl.b % 128 == 0
-    chunk_names = (["cb_gram_tc_kernel" if tc_gram else "cb_gram_kernel", "cb_scan_kernel"]
+    chunk_names = (["cb_gram_tc_kernel", "cb_scan_tc_kernel"] if tc_gram
+                   else ["cb_gram_kernel", "cb_scan_kernel"])
+    chunk_names = (chunk_names
                    + (["cb_tok_tc_kernel<RP>", "cb_tok_tc_kernel<DK>", "cb_tok_tc_kernel<DQ>"]
                       if tc_tok else ["cb_tok_kernel"]) + ["cb_sum_over_batch_kernel (dW0)"])
     knames = (chunk_names

@@ -254,7 +254,8 @@ TTT_API ttt_status ttt_linear_bwd(const void *Q, const void *K, const void *V, c
  * d = 128 the per-chunk products and (chunk % 128 == 0) the per-token
  * products run on the tensor cores, every fp32 operand as two bf16 terms,
  * dK as -diag(eta)(K_c S_c - V_c Om_{c+1}^T) with S_c = W_c Om_{c+1}^T +
- * Om_{c+1} W_c^T (the same quantity); the affine scans run on fp32 CUDA
+ * Om_{c+1} W_c^T (the same quantity); the affine scans run on the tensor
+ * cores too (A_c and the state as hi and lo terms), else on fp32 CUDA
  * cores. Deterministic.
  * Supported: d in {64, 128}, chunk % 32 == 0, T % chunk == 0; TTT_BF16 or
  * TTT_FP32. flags: only TTT_F_W0_PER_SEQ.

@@ -29,6 +29,9 @@ bool chunk_bwd_gram_tc_supported(int d, int chunk, bool bf16);
 cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V, const float *eta,
                                      const float *dZ, int B, int H, int T, int chunk, float *gram,
                                      void *tok_scratch, cudaStream_t s);
+cudaError_t launch_chunk_bwd_scan_tc(const float *W0, const float *dW_out, const float *gram,
+                                     float *Wst, float *Omst, float *dW0_out, int S, int H, int NC,
+                                     bool w0_per_seq, cudaStream_t s);
 bool chunk_bwd_tok_tc_supported(int d, int chunk, bool bf16);
 size_t chunk_bwd_tok_tc_scratch_bytes(size_t tokens);
 cudaError_t launch_chunk_bwd_tok_tc(const void *K, const void *V, const float *eta, const float *dZ,
@@ -344,27 +347,31 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
     // cores; their bf16 operand rows follow the fp32 part of the workspace
     const bool tok_tc = std::is_same<TIn, __nv_bfloat16>::value && chunk_bwd_tok_tc_supported(D, C, true);
     void *scratch = tok_tc ? reinterpret_cast<float *>(workspace) + (5 * nch + S) * (size_t)D * D : nullptr;
+    float *dW0_seq = w0_per_seq ? dW0 : w.dW0s;
     if (std::is_same<TIn, __nv_bfloat16>::value && chunk_bwd_gram_tc_supported(D, C, true)) {
         // d = 128, bf16: the Gram products on the tensor cores (also writing
-        // dZ's operand rows for the token passes)
+        // dZ's operand rows for the token passes), then the scans on the
+        // tensor cores, which read the Gram's operand layouts
         if ((e = launch_chunk_bwd_gram_tc(Q, K, V, eta, dZ, B, H, T, C, w.gram, scratch, s)) !=
             cudaSuccess)
+            return e;
+        if ((e = launch_chunk_bwd_scan_tc(W0, dW_out, w.gram, w.W, w.Om, dW0_seq, (int)S, H, NC,
+                                          w0_per_seq, s)) != cudaSuccess)
             return e;
     } else {
         cb_gram_kernel<TIn, D><<<dim3((unsigned)nch, 3, (D / 64) * (D / 64)), kT, 0, s>>>(
             q, k, v, eta, dZ, T, C, w.gram);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         count_launch(s);
+        const size_t scan_smem = ((size_t)D * D + (size_t)D * scan_cols(D)) * sizeof(float);  // A_c, M slice
+        if ((e = cudaFuncSetAttribute(cb_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)scan_smem)) != cudaSuccess)
+            return e;
+        cb_scan_kernel<D><<<dim3((unsigned)S, 2, D / scan_cols(D)), kT, scan_smem, s>>>(
+            W0, dW_out, H, NC, w0_per_seq, w, dW0_seq);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        count_launch(s);
     }
-    const size_t scan_smem = ((size_t)D * D + (size_t)D * scan_cols(D)) * sizeof(float);  // A_c, M slice
-    if ((e = cudaFuncSetAttribute(cb_scan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)scan_smem)) != cudaSuccess)
-        return e;
-    float *dW0_seq = w0_per_seq ? dW0 : w.dW0s;
-    cb_scan_kernel<D><<<dim3((unsigned)S, 2, D / scan_cols(D)), kT, scan_smem, s>>>(
-        W0, dW_out, H, NC, w0_per_seq, w, dW0_seq);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    count_launch(s);
     if (tok_tc) {
         // each chunk's S = W_c Om_{c+1}^T + Om_{c+1} W_c^T takes the place of
         // its A_c, which only the scans read

@@ -3,8 +3,9 @@
 //   A_c = K_c^T diag(eta) K_c,   B_c = K_c^T diag(eta) V_c,   D_c = Q_c^T dZ_c
 // ("Test-Time Training Done Right", abstract: the chunk's gradient step; the
 // backward's recurrences use the same A_c, and D_c carries dZ into dL/dW_c),
-// written in fp32 in the layout the backward's scan and token kernels read:
-// per chunk [A_c | B_c | D_c], each row-major [d_in][d_out].
+// written per chunk into three d x d fp32 slots [A_c | B_c | D_c] in the
+// layouts the tensor-core scan reads (A_c as bf16 hi and lo operand images,
+// B_c and D_c as fp32 column quads; see the epilogue).
 //
 // One block per chunk, 32 tokens per pipeline stage. The products run on
 // tcgen05 with M = d_in = 128 and the tokens as the reduction:
@@ -198,12 +199,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_async_smem();
             mbar_arrive(&conv[st]);
         }
-        // Epilogue: lane = d_in row i of the accumulators.
+        // Epilogue: lane = d_in row i of the accumulators. The chunk's three
+        // d x d slots take the scan's operand layouts: A_c as bf16 hi and lo
+        // images (K-major, 128-byte swizzle, 32 KB each), B_c and D_c in fp32
+        // with column quad q of row i at float4 q * 128 + i (so a 64-column
+        // slice is 32 contiguous KB).
         if (__all_sync(0xffffffffu, mbar_wait(&done, 0, &abort_flag, a.status, 94))) {
             tc_fence_after();
             const int sp = warp & 3, i = 32 * sp + lane;
             const float scale = uniform ? eta0 : 1.f;
-            float *out = a.gram + (size_t)g * 3 * kD * kD + (size_t)i * kD;
+            float *slot = a.gram + (size_t)g * 3 * kD * kD;
+            uint8_t *ahi = reinterpret_cast<uint8_t *>(slot), *alo = ahi + kD * kD * 2;
+            float4 *ob = reinterpret_cast<float4 *>(slot + kD * kD);
+            float4 *od = reinterpret_cast<float4 *>(slot + 2 * kD * kD);
 #pragma unroll 1
             for (int q = 0; q < kD / 16; ++q) {
                 float va[16], vb[16], dh[16], dl[16];
@@ -212,17 +220,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld16(taddr(tm, 32 * sp, 256 + 16 * q), dh);
                 tmem_ld16(taddr(tm, 32 * sp, 384 + 16 * q), dl);
                 tmem_ld_wait();
-                float4 *oa = reinterpret_cast<float4 *>(out + 16 * q);
-                float4 *ob = reinterpret_cast<float4 *>(out + kD * kD + 16 * q);
-                float4 *od = reinterpret_cast<float4 *>(out + 2 * kD * kD + 16 * q);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float *x = va + 8 * h;
+                    uint2 h0, l0, h1, l1;
+                    split4(scale * x[0], scale * x[1], scale * x[2], scale * x[3], h0, l0);
+                    split4(scale * x[4], scale * x[5], scale * x[6], scale * x[7], h1, l1);
+                    const uint32_t o = off_kmajor_sw128(i, 16 * q + 8 * h, kD);
+                    *reinterpret_cast<uint4 *>(ahi + o) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                    *reinterpret_cast<uint4 *>(alo + o) = make_uint4(l0.x, l0.y, l1.x, l1.y);
+                }
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    oa[e] = make_float4(scale * va[4 * e], scale * va[4 * e + 1], scale * va[4 * e + 2],
-                                        scale * va[4 * e + 3]);
-                    ob[e] = make_float4(scale * vb[4 * e], scale * vb[4 * e + 1], scale * vb[4 * e + 2],
-                                        scale * vb[4 * e + 3]);
-                    od[e] = make_float4(dh[4 * e] + dl[4 * e], dh[4 * e + 1] + dl[4 * e + 1],
-                                        dh[4 * e + 2] + dl[4 * e + 2], dh[4 * e + 3] + dl[4 * e + 3]);
+                    ob[(4 * q + e) * kD + i] = make_float4(scale * vb[4 * e], scale * vb[4 * e + 1],
+                                                           scale * vb[4 * e + 2], scale * vb[4 * e + 3]);
+                    od[(4 * q + e) * kD + i] = make_float4(dh[4 * e] + dl[4 * e], dh[4 * e + 1] + dl[4 * e + 1],
+                                                           dh[4 * e + 2] + dl[4 * e + 2],
+                                                           dh[4 * e + 3] + dl[4 * e + 3]);
                 }
             }
         }
@@ -241,6 +255,209 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tm, 512);
+}
+
+// ---------------------------------------------------------------------------
+// The backward's two affine scans on the tensor cores (d = 128, slots in the
+// layouts cb_gram_tc_kernel writes): per sequence
+//   forward:  W_{c+1} = W_c - A_c W_c + B_c from W0, storing each W_c;
+//   reverse:  Om_c = Om_{c+1} - A_c Om_{c+1} + D_c from dW_out (or 0),
+//             storing each Om_{c+1}, and at the end dW0 = Om_0.
+// A block per (sequence, direction, 64-column slice r): the columns of M
+// evolve independently. One product per chunk, D = A_c [M_hi | M_lo] (M = 128
+// rows i, N = 128: the slice's hi and lo terms side by side, K = 128), with
+// A_c's hi and lo images as two instructions per K step, so each operand
+// carries ~16 significant bits. The fp32 state is in the registers of four
+// epilogue warps (row i = tensor-memory lane, 64 columns); they store it,
+// form M - (D_hi + D_lo) + E_c and write the next slice image (K-major rows
+// n: M_hi^T then M_lo^T). A_c's images and E_c's slice arrive by bulk copy,
+// double-buffered, so a chunk's copies run while the previous product and
+// update do.
+constexpr int kScanThreads = 192;  // warp 0: copies, warp 1: MMA, warps 2-5: state
+constexpr int kScanA = 2 * kD * kD * 2;            // A_c hi | lo images: 64 KB
+constexpr int kScanE = kD * 64 * 4;                // E_c columns of the slice: 32 KB
+constexpr int kScanImg = kD * kD * 2;              // slice image [M_hi^T | M_lo^T]: 32 KB
+constexpr size_t kScanSmem = 1024 + 2 * kScanA + 2 * kScanE + kScanImg;  // 225 KB
+static_assert(kScanSmem <= 232448, "shared memory budget");
+
+struct ScanArgs {
+    const float *W0, *dW_out, *gram;
+    float *Wst, *Omst, *dW0_out;
+    int H, NC;
+    bool w0_per_seq;
+    int *status;
+};
+
+__global__ void __launch_bounds__(kScanThreads, 1) cb_scan_tc_kernel(ScanArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem, *sE = smem + 2 * kScanA, *sW = sE + 2 * kScanE;
+    __shared__ uint64_t aready[2], afree[2], eready[2], efree[2], dfull, wready, drain;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int seq = blockIdx.x, dir = blockIdx.y, j0 = 64 * blockIdx.z;
+    const int NC = a.NC;
+    const size_t dd = (size_t)kD * kD;
+    auto chunk_of = [&](int st) { return (size_t)seq * NC + (dir == 0 ? st : NC - 1 - st); };
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&aready[b], 1);
+            mbar_init(&afree[b], 1);
+            mbar_init(&eready[b], 1);
+            mbar_init(&efree[b], 4);  // one arrival per state warp
+        }
+        mbar_init(&dfull, 1);
+        mbar_init(&wready, 1);
+        mbar_init(&drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&tmem_base, 128);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_base;
+    int issued = 0;  // copy pairs issued
+
+    if (warp == 0 && lane == 0) {
+        for (int st = 0; st < NC; ++st) {
+            const int b = st & 1;
+            const float *slot = a.gram + chunk_of(st) * 3 * dd;
+            if (st >= 2 && !mbar_wait(&afree[b], ((st >> 1) - 1) & 1, &abort_flag, a.status, 111)) break;
+            mbar_arrive_expect_tx(&aready[b], kScanA);
+            bulk_load(sA + b * kScanA, slot, kScanA, &aready[b]);
+            if (st >= 2 && !mbar_wait(&efree[b], ((st >> 1) - 1) & 1, &abort_flag, a.status, 112)) {
+                issued = 2 * st + 1;
+                break;
+            }
+            mbar_arrive_expect_tx(&eready[b], kScanE);
+            bulk_load(sE + b * kScanE, slot + (dir == 0 ? 1 : 2) * dd + (size_t)j0 * kD, kScanE, &eready[b]);
+            issued = 2 * st + 2;
+        }
+    } else if (warp == 1 && lane == 0) {
+        const uint32_t idesc = make_idesc_bf16(128, 128, false, false);
+        const uint32_t wb = smem_u32(sW);
+        for (int st = 0; st < NC; ++st) {
+            const int b = st & 1;
+            if (!mbar_wait(&aready[b], (st >> 1) & 1, &abort_flag, a.status, 113)) break;
+            if (!mbar_wait(&wready, st & 1, &abort_flag, a.status, 114)) break;
+            tc_fence_after();
+            const uint32_t ab = smem_u32(sA + b * kScanA);
+#pragma unroll
+            for (int k = 0; k < kD / 16; ++k) {
+                const int k0 = 16 * k;
+                const uint32_t o = (uint32_t)((k0 >> 6) * 16384 + (k0 & 63) * 2);
+                const uint64_t bd = make_sdesc(wb + o, 16, 1024, kSw128);
+                mma_bf16(tm, make_sdesc(ab + o, 16, 1024, kSw128), bd, idesc, k != 0);
+                mma_bf16(tm, make_sdesc(ab + kScanA / 2 + o, 16, 1024, kSw128), bd, idesc, true);
+            }
+            mma_commit(&afree[b]);
+            mma_commit(&dfull);
+        }
+    } else if (warp >= 2) {
+        const int sp = warp & 3, row = 32 * sp + lane;
+        float w[64];
+        {
+            const float *src = dir == 0 ? a.W0 + (size_t)(a.w0_per_seq ? seq : seq % a.H) * dd
+                                        : (a.dW_out ? a.dW_out + (size_t)seq * dd : nullptr);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const float4 u = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * kD + j0 + 4 * q)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                w[4 * q] = u.x;
+                w[4 * q + 1] = u.y;
+                w[4 * q + 2] = u.z;
+                w[4 * q + 3] = u.w;
+            }
+        }
+        // this thread's column `row` of the slice image: K index row, rows n
+        // (M_hi^T: n = jj, M_lo^T: n = 64 + jj)
+        // (element (n, row) at off_kmajor_sw128(n, row, 128): a per-thread
+        // base plus a per-n constant plus the swizzled 16-byte chunk)
+        const uint32_t cb = (uint32_t)((row >> 6) * 16384 + (row & 7) * 2), rc = (uint32_t)((row & 63) >> 3);
+        auto emit = [&]() {
+#pragma unroll
+            for (int jj = 0; jj < 64; ++jj) {
+                __nv_bfloat16 hb, lb;
+                split_bf16(w[jj], hb, lb);
+                const uint32_t sw = (rc ^ (uint32_t)(jj & 7)) << 4;
+                *reinterpret_cast<__nv_bfloat16 *>(sW + cb + (jj >> 3) * 1024 + (jj & 7) * 128 + sw) = hb;
+                *reinterpret_cast<__nv_bfloat16 *>(sW + cb + 8192 + (jj >> 3) * 1024 + (jj & 7) * 128 + sw) = lb;
+            }
+            fence_async_smem();
+        };
+        emit();
+        bool ok = !named_bar_or(1, 128, false);
+        if (ok && warp == 2 && lane == 0) mbar_arrive(&wready);
+        for (int st = 0; ok && st < NC; ++st) {
+            const int b = st & 1;
+            const size_t g = chunk_of(st);
+            // the state entering the chunk: W_c (forward) or Om_{c+1} (reverse)
+            float *o = (dir == 0 ? a.Wst : a.Omst) + g * dd + (size_t)row * kD + j0;
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+                *reinterpret_cast<float4 *>(o + 4 * q) = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            bool got = mbar_wait(&eready[b], (st >> 1) & 1, &abort_flag, a.status, 115);
+            got = got && mbar_wait(&dfull, st & 1, &abort_flag, a.status, 116);
+            if (named_bar_or(1, 128, !__all_sync(0xffffffffu, got))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float4 *E = reinterpret_cast<const float4 *>(sE + b * kScanE);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float dh[16], dl[16];
+                tmem_ld16(taddr(tm, 32 * sp, 16 * q), dh);
+                tmem_ld16(taddr(tm, 32 * sp, 64 + 16 * q), dl);
+                float ev[16];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 f = E[(4 * q + u) * kD + row];
+                    ev[4 * u] = f.x;
+                    ev[4 * u + 1] = f.y;
+                    ev[4 * u + 2] = f.z;
+                    ev[4 * u + 3] = f.w;
+                }
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) w[16 * q + e] = w[16 * q + e] + ev[e] - (dh[e] + dl[e]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&efree[b]);  // this warp has read E_c
+            if (st + 1 < NC) emit();                // the product of this chunk is done with the image
+            if (named_bar_or(1, 128, false)) {
+                ok = false;
+                break;
+            }
+            if (st + 1 < NC && warp == 2 && lane == 0) mbar_arrive(&wready);
+        }
+        if (ok && !abort_flag && dir == 1) {
+            float *o = a.dW0_out + (size_t)seq * dd + (size_t)row * kD + j0;
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+                *reinterpret_cast<float4 *>(o + 4 * q) = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
+    }
+    // Teardown: after an abort, let this block's own copies and MMAs land
+    // before the shared memory and tensor memory are released.
+    if (abort_flag) {
+        if (warp == 0 && lane == 0 && issued > 0) {
+            const int st = (issued - 1) / 2;  // the last chunk whose copies were issued
+            mbar_drain(&aready[st & 1], (st >> 1) & 1);
+            if (issued % 2 == 0) mbar_drain(&eready[st & 1], (st >> 1) & 1);
+        }
+        if (warp == 1 && lane == 0) {
+            mma_commit(&drain);
+            mbar_drain(&drain, 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tm, 128);
 }
 
 }  // namespace
@@ -284,6 +501,23 @@ cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V
         ga.z_lo = ts.z_lo;
     }
     cb_gram_tc_kernel<<<nch, kThreads, kSmem, s>>>(tmK, tmV, tmQ, tmZ, ga);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launch(s);
+    return cudaSuccess;
+}
+
+// The two scans of the backward on the tensor cores, after
+// launch_chunk_bwd_gram_tc: W_c into Wst, Om_{c+1} into Omst (per chunk
+// [d][d] fp32, row-major), dW0 = Om_0 of each sequence into dW0_out.
+cudaError_t launch_chunk_bwd_scan_tc(const float *W0, const float *dW_out, const float *gram,
+                                     float *Wst, float *Omst, float *dW0_out, int S, int H, int NC,
+                                     bool w0_per_seq, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(cb_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kScanSmem);
+    if (e != cudaSuccess) return e;
+    ScanArgs sa{W0, dW_out, gram, Wst, Omst, dW0_out, H, NC, w0_per_seq, device_status_word()};
+    cb_scan_tc_kernel<<<dim3((unsigned)S, 2, kD / 64), kScanThreads, kScanSmem, s>>>(sa);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
