@@ -745,42 +745,54 @@ __global__ void __launch_bounds__(kTokThreads, 1)
         {
             const float *Wc = a.W + (size_t)g * dd, *Oc = a.Om + (size_t)g * dd;
             const float *Sc = a.S + (size_t)g * a.s_stride;
-            // units: (row n, 8 consecutive k)
+            // units: (row n, 8 consecutive k), NU per thread, loaded UB units
+            // at a time before any is converted (so UB x 8 loads are in flight)
             constexpr int NROWS = kMode == kModeRP ? 2 * kD : kD;
+            constexpr int NU = NROWS * (KD / 8) / 128, UB = 8;
+            static_assert(NU % UB == 0, "whole batches");
             constexpr bool kColRead = kMode != kModeDQ;  // consecutive threads take consecutive n
-            for (int uidx = tt; uidx < NROWS * (KD / 8); uidx += 128) {
-                // Column reads (RP's W and Om, DK's S) go with consecutive
-                // threads on consecutive n (one 128-byte row segment per warp
-                // load); row reads with consecutive k
-                const int n = kColRead ? uidx % NROWS : uidx / (KD / 8);
-                const int k0 = kColRead ? 8 * (uidx / NROWS) : 8 * (uidx % (KD / 8));
-                float f[8];
-                if (kMode == kModeRP || (kMode == kModeDK && k0 < kD)) {
-                    // RP: B[n][k] = W[k][n] (n < 128) or Om[k][n - 128] (K = d_in);
-                    // DK, k < 128: B[n][k] = S[k][n]
-                    const float *src = kMode == kModeDK ? Sc + n : (n < kD ? Wc + n : Oc + (n - kD));
+            // Column reads (RP's W and Om, DK's S) go with consecutive threads
+            // on consecutive n (one 128-byte row segment per warp load); row
+            // reads with consecutive k
+            auto unit_n = [&](int uidx) { return kColRead ? uidx % NROWS : uidx / (KD / 8); };
+            auto unit_k0 = [&](int uidx) { return kColRead ? 8 * (uidx / NROWS) : 8 * (uidx % (KD / 8)); };
+#pragma unroll 1
+            for (int b0 = 0; b0 < NU; b0 += UB) {
+                float f[UB][8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = src[(size_t)(k0 + e) * kD];
-                } else {
-                    // DK, k >= 128: B[n][k] = -Om[n][k - 128]; DQ: B[n][k] = W[n][k]
-                    const float *src = (kMode == kModeDK ? Oc : Wc) + (size_t)n * kD + (k0 & (kD - 1));
-                    const float sg = kMode == kModeDK ? -1.f : 1.f;
-                    const float4 u0 = *reinterpret_cast<const float4 *>(src);
-                    const float4 u1 = *reinterpret_cast<const float4 *>(src + 4);
-                    f[0] = sg * u0.x; f[1] = sg * u0.y; f[2] = sg * u0.z; f[3] = sg * u0.w;
-                    f[4] = sg * u1.x; f[5] = sg * u1.y; f[6] = sg * u1.z; f[7] = sg * u1.w;
+                for (int j = 0; j < UB; ++j) {
+                    const int uidx = tt + 128 * (b0 + j), n = unit_n(uidx), k0 = unit_k0(uidx);
+                    if (kMode == kModeRP || (kMode == kModeDK && k0 < kD)) {
+                        // RP: B[n][k] = W[k][n] (n < 128) or Om[k][n - 128] (K = d_in);
+                        // DK, k < 128: B[n][k] = S[k][n]
+                        const float *src = kMode == kModeDK ? Sc + n : (n < kD ? Wc + n : Oc + (n - kD));
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[j][e] = src[(size_t)(k0 + e) * kD];
+                    } else {
+                        // DK, k >= 128: B[n][k] = -Om[n][k - 128]; DQ: B[n][k] = W[n][k]
+                        const float *src = (kMode == kModeDK ? Oc : Wc) + (size_t)n * kD + (k0 & (kD - 1));
+                        const float sg = kMode == kModeDK ? -1.f : 1.f;
+                        const float4 u0 = *reinterpret_cast<const float4 *>(src);
+                        const float4 u1 = *reinterpret_cast<const float4 *>(src + 4);
+                        f[j][0] = sg * u0.x; f[j][1] = sg * u0.y; f[j][2] = sg * u0.z; f[j][3] = sg * u0.w;
+                        f[j][4] = sg * u1.x; f[j][5] = sg * u1.y; f[j][6] = sg * u1.z; f[j][7] = sg * u1.w;
+                    }
                 }
-                uint2 h0, l0, h1, l1;
-                split4(f[0], f[1], f[2], f[3], h0, l0);
-                split4(f[4], f[5], f[6], f[7], h1, l1);
-                if (kMode == kModeRP) {
-                    const uint32_t o = kmajor_off(n, k0, BR);
-                    *reinterpret_cast<uint4 *>(sB + o) = make_uint4(h0.x, h0.y, h1.x, h1.y);
-                    *reinterpret_cast<uint4 *>(sB + kBLoOff + o) = make_uint4(l0.x, l0.y, l1.x, l1.y);
-                } else {
-                    *reinterpret_cast<uint4 *>(sB + kmajor_off(n, k0, BR)) = make_uint4(h0.x, h0.y, h1.x, h1.y);
-                    *reinterpret_cast<uint4 *>(sB + kmajor_off(kD + n, k0, BR)) =
-                        make_uint4(l0.x, l0.y, l1.x, l1.y);
+#pragma unroll
+                for (int j = 0; j < UB; ++j) {
+                    const int uidx = tt + 128 * (b0 + j), n = unit_n(uidx), k0 = unit_k0(uidx);
+                    uint2 h0, l0, h1, l1;
+                    split4(f[j][0], f[j][1], f[j][2], f[j][3], h0, l0);
+                    split4(f[j][4], f[j][5], f[j][6], f[j][7], h1, l1);
+                    if (kMode == kModeRP) {
+                        const uint32_t o = kmajor_off(n, k0, BR);
+                        *reinterpret_cast<uint4 *>(sB + o) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                        *reinterpret_cast<uint4 *>(sB + kBLoOff + o) = make_uint4(l0.x, l0.y, l1.x, l1.y);
+                    } else {
+                        *reinterpret_cast<uint4 *>(sB + kmajor_off(n, k0, BR)) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                        *reinterpret_cast<uint4 *>(sB + kmajor_off(kD + n, k0, BR)) =
+                            make_uint4(l0.x, l0.y, l1.x, l1.y);
+                    }
                 }
             }
             fence_async_smem();
