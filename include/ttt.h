@@ -249,8 +249,7 @@ TTT_API ttt_status ttt_linear_bwd(const void *Q, const void *K, const void *V, c
  * [B][H][d][d] with TTT_F_W0_PER_SEQ), all fp32, overwritten. workspace:
  * device memory of at least ttt_chunk_bwd_workspace_bytes() bytes, 256-byte
  * aligned, owned by the caller (per chunk: A_c, B_c, Q_c^T dZ_c, W_c and
- * Om_{c+1} in fp32; with d = 128 and chunk % 128 == 0 also 512 bytes per
- * token of bf16 operand rows, dZ's hi and lo terms). With bf16 inputs and
+ * Om_{c+1} in fp32, and dW0 per sequence). With bf16 inputs and
  * d = 128 the per-chunk products and (chunk % 128 == 0) the per-token
  * products run on the tensor cores, every fp32 operand as two bf16 terms,
  * dK as -diag(eta)(K_c S_c - V_c Om_{c+1}^T) with S_c = W_c Om_{c+1}^T +

@@ -28,16 +28,15 @@ namespace ttt {
 bool chunk_bwd_gram_tc_supported(int d, int chunk, bool bf16);
 cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V, const float *eta,
                                      const float *dZ, int B, int H, int T, int chunk, float *gram,
-                                     void *tok_scratch, cudaStream_t s);
+                                     cudaStream_t s);
 cudaError_t launch_chunk_bwd_scan_tc(const float *W0, const float *dW_out, const float *gram,
                                      float *Wst, float *Omst, float *dW0_out, int S, int H, int NC,
                                      bool w0_per_seq, cudaStream_t s);
 bool chunk_bwd_tok_tc_supported(int d, int chunk, bool bf16);
-size_t chunk_bwd_tok_tc_scratch_bytes(size_t tokens);
 cudaError_t launch_chunk_bwd_tok_tc(const void *K, const void *V, const float *eta, const float *dZ,
                                     const float *W, const float *Om, float *S, size_t s_stride,
-                                    int B, int H, int T, int chunk, void *scratch, float *dQ,
-                                    float *dK, float *dV, float *deta, cudaStream_t s);
+                                    int B, int H, int T, int chunk, float *dQ, float *dK, float *dV,
+                                    float *deta, cudaStream_t s);
 
 namespace {
 
@@ -343,17 +342,13 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
     const TIn *q = static_cast<const TIn *>(Q), *k = static_cast<const TIn *>(K),
               *v = static_cast<const TIn *>(V);
     cudaError_t e;
-    // d = 128, bf16, chunk % 128 == 0: the per-token products on the tensor
-    // cores; their bf16 operand rows follow the fp32 part of the workspace
+    // d = 128, bf16, chunk % 128 == 0: the per-token products on the tensor cores
     const bool tok_tc = std::is_same<TIn, __nv_bfloat16>::value && chunk_bwd_tok_tc_supported(D, C, true);
-    void *scratch = tok_tc ? reinterpret_cast<float *>(workspace) + (5 * nch + S) * (size_t)D * D : nullptr;
     float *dW0_seq = w0_per_seq ? dW0 : w.dW0s;
     if (std::is_same<TIn, __nv_bfloat16>::value && chunk_bwd_gram_tc_supported(D, C, true)) {
-        // d = 128, bf16: the Gram products on the tensor cores (also writing
-        // dZ's operand rows for the token passes), then the scans on the
-        // tensor cores, which read the Gram's operand layouts
-        if ((e = launch_chunk_bwd_gram_tc(Q, K, V, eta, dZ, B, H, T, C, w.gram, scratch, s)) !=
-            cudaSuccess)
+        // d = 128, bf16: the Gram products on the tensor cores, then the scans
+        // on the tensor cores, which read the Gram's operand layouts
+        if ((e = launch_chunk_bwd_gram_tc(Q, K, V, eta, dZ, B, H, T, C, w.gram, s)) != cudaSuccess)
             return e;
         if ((e = launch_chunk_bwd_scan_tc(W0, dW_out, w.gram, w.W, w.Om, dW0_seq, (int)S, H, NC,
                                           w0_per_seq, s)) != cudaSuccess)
@@ -376,7 +371,7 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
         // each chunk's S = W_c Om_{c+1}^T + Om_{c+1} W_c^T takes the place of
         // its A_c, which only the scans read
         if ((e = launch_chunk_bwd_tok_tc(K, V, eta, dZ, w.W, w.Om, w.gram, 3 * (size_t)D * D, B, H,
-                                         T, C, scratch, dQ, dK, dV, deta, s)) != cudaSuccess)
+                                         T, C, dQ, dK, dV, deta, s)) != cudaSuccess)
             return e;
     } else {
         const size_t tsm = tok_smem_bytes(D);
@@ -407,11 +402,7 @@ size_t chunk_bwd_workspace_bytes(int B, int H, int T, int d, int chunk) {
     if (B <= 0 || H <= 0 || T <= 0 || chunk <= 0 || T % chunk || !chunk_bwd_supported(d, chunk))
         return 0;
     const size_t S = (size_t)B * H, nch = S * (T / chunk), dd = (size_t)d * d;
-    // d = 128, chunk % 128 == 0: the tensor-core token passes' operand rows
-    // (used with bf16 inputs; the size does not depend on the dtype)
-    const size_t tc = chunk_bwd_tok_tc_supported(d, chunk, true)
-                          ? chunk_bwd_tok_tc_scratch_bytes(S * (size_t)T) : 0;
-    return sizeof(float) * (5 * nch * dd + S * dd) + tc;
+    return sizeof(float) * (5 * nch * dd + S * dd);
 }
 
 cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const float *eta,

@@ -49,9 +49,6 @@ struct GramArgs {
     float *gram;  // [chunk][3][d][d]
     int chunk;
     int *status;
-    // optional: dZ's bf16 hi and lo rows ([tokens][d]) for the token passes,
-    // written from the terms this kernel forms anyway
-    __nv_bfloat16 *z_hi = nullptr, *z_lo = nullptr;
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -172,11 +169,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_uint4(h0.x, h0.y, h1.x, h1.y);
                 *reinterpret_cast<uint4 *>(sb + OFF_ZB + (2 + (col0 >> 6)) * kBox + off) =
                     make_uint4(l0.x, l0.y, l1.x, l1.y);
-                if (a.z_hi) {
-                    const size_t zo = (size_t)(row0 + (long)r * kRows + row) * kD + col0;
-                    *reinterpret_cast<uint4 *>(a.z_hi + zo) = make_uint4(h0.x, h0.y, h1.x, h1.y);
-                    *reinterpret_cast<uint4 *>(a.z_lo + zo) = make_uint4(l0.x, l0.y, l1.x, l1.y);
-                }
                 if (!uniform) {
                     const uint4 kq = *reinterpret_cast<const uint4 *>(sb + OFF_K + (col0 >> 6) * kBox + off);
                     const __nv_bfloat162 *kh = reinterpret_cast<const __nv_bfloat162 *>(&kq);
@@ -466,23 +458,10 @@ bool chunk_bwd_gram_tc_supported(int d, int chunk, bool bf16) {
     return bf16 && d == kD && chunk >= kRows && chunk % kRows == 0;
 }
 
-// The token passes' operand rows in their scratch: dZ hi and lo
-// ([tokens][d] each), bf16.
-struct TokScratch {
-    __nv_bfloat16 *z_hi, *z_lo;
-};
-TokScratch tok_scratch(void *scratch, uint64_t rows) {
-    TokScratch t;
-    t.z_hi = static_cast<__nv_bfloat16 *>(scratch);
-    t.z_lo = t.z_hi + rows * kD;
-    return t;
-}
-
-// gram: [B*H*(T/chunk)][3][128][128] fp32, written in full. tok_scratch:
-// the token passes' scratch (or nullptr), whose dZ rows this kernel fills.
+// gram: [B*H*(T/chunk)][3][128][128] fp32, written in full.
 cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V, const float *eta,
                                      const float *dZ, int B, int H, int T, int chunk, float *gram,
-                                     void *tok_scratch_ptr, cudaStream_t s) {
+                                     cudaStream_t s) {
     const uint64_t rows = (uint64_t)B * H * T;
     const int nch = B * H * (T / chunk);
     alignas(64) CUtensorMap tmK, tmV, tmQ, tmZ;
@@ -495,11 +474,6 @@ cudaError_t launch_chunk_bwd_gram_tc(const void *Q, const void *K, const void *V
                                          (int)kSmem);
     if (e != cudaSuccess) return e;
     GramArgs ga{eta, gram, chunk, device_status_word()};
-    if (tok_scratch_ptr) {
-        const TokScratch ts = tok_scratch(tok_scratch_ptr, rows);
-        ga.z_hi = ts.z_hi;
-        ga.z_lo = ts.z_lo;
-    }
     cb_gram_tc_kernel<<<nch, kThreads, kSmem, s>>>(tmK, tmV, tmQ, tmZ, ga);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -598,8 +572,12 @@ __device__ __forceinline__ uint4 pack4f(float a, float b, float c, float d) {
     return make_uint4(__float_as_uint(a), __float_as_uint(b), __float_as_uint(c), __float_as_uint(d));
 }
 
+// Threads of a token pass: DQ adds four warps that split dZ (fp32, by TMA)
+// into the bf16 hi and lo operand images.
+__host__ __device__ constexpr int tok_threads(int mode) { return mode == kModeDQ ? 320 : kTokThreads; }
+
 template <int kMode>
-__global__ void __launch_bounds__(kTokThreads, 1)
+__global__ void __launch_bounds__(tok_threads(kMode), 1)
     cb_tok_tc_kernel(const __grid_constant__ CUtensorMap tmA_hi, const __grid_constant__ CUtensorMap tmA_lo,
                      TokArgs a) {
     constexpr int KD = kMode == kModeDK ? 2 * kD : kD;  // reduction length
@@ -609,17 +587,20 @@ __global__ void __launch_bounds__(kTokThreads, 1)
     // ([W | Om]^T); DK and DQ stack [hi rows | lo rows] of their 128 rows.
     constexpr int BR = 2 * kD;
     constexpr uint32_t kBLoOff = kMode == kModeRP ? (uint32_t)NKB * BR * 128 : 0u;
-    // A ring: one or two terms of a 64-wide K block per stage (DK: the K
-    // blocks of K, then of V).
+    // A ring: one term of a 64-wide K block per stage (DK: the K blocks of K,
+    // then of V); DQ: dZ's fp32 K block (two 32-column boxes) per stage, and
+    // one buffer for its bf16 hi and lo images, which the converter warps
+    // fill once the product before has read them.
     constexpr int STAGES = kMode == kModeDK ? 4 : 3;
     constexpr int SBYTES = kTwoA ? kTokStage : kTokStage / 2;
+    constexpr int ABUF = kTwoA ? kTokStage : 0;  // DQ's bf16 images, after the ring
     constexpr int BBYTES = NKB * BR * 128 * (kMode == kModeRP ? 2 : 1);  // B images
-    static_assert(BBYTES + STAGES * SBYTES + 4 * kStgWarp + 1024 <= (int)kTokSmem, "smem plan");
+    static_assert(BBYTES + STAGES * SBYTES + ABUF + 4 * kStgWarp + 1024 <= (int)kTokSmem, "smem plan");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sB = smem, *sA = smem + BBYTES;
-    __shared__ uint64_t full[4], empty[4], bready, tfull[2], tempty[2], sfull, sfree, drain;
+    __shared__ uint64_t full[4], empty[4], bready, tfull[2], tempty[2], sfull, sfree, conv, aempty, drain;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -632,8 +613,10 @@ __global__ void __launch_bounds__(kTokThreads, 1)
         abort_flag = 0;
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], kMode == kModeDQ ? 128 : 1);  // DQ: the converters free a stage
         }
+        mbar_init(&conv, 128);
+        mbar_init(&aempty, 1);
         mbar_init(&bready, 128);
         mbar_init(&sfull, 1);
         mbar_init(&sfree, 128);
@@ -661,12 +644,17 @@ __global__ void __launch_bounds__(kTokThreads, 1)
                     goto producer_done;
                 uint8_t *sb = sA + st * SBYTES;
                 const int y = (int)(row0 + (long)t * kTokTile);
-                mbar_arrive_expect_tx(&full[st], SBYTES);
-                if (kMode == kModeDK)  // [K | V]: K blocks 0-1 of K, 2-3 of V
-                    tma_load_2d(sb, kb < 2 ? &tmA_hi : &tmA_lo, 64 * (kb & 1), y, &full[st]);
-                else
+                if (kMode == kModeDQ) {  // dZ fp32: two 32-column boxes
+                    mbar_arrive_expect_tx(&full[st], SBYTES);
                     tma_load_2d(sb, &tmA_hi, 64 * kb, y, &full[st]);
-                if (kTwoA) tma_load_2d(sb + kTokStage / 2, &tmA_lo, 64 * kb, y, &full[st]);
+                    tma_load_2d(sb + SBYTES / 2, &tmA_hi, 64 * kb + 32, y, &full[st]);
+                } else {
+                    mbar_arrive_expect_tx(&full[st], SBYTES);
+                    if (kMode == kModeDK)  // [K | V]: K blocks 0-1 of K, 2-3 of V
+                        tma_load_2d(sb, kb < 2 ? &tmA_hi : &tmA_lo, 64 * (kb & 1), y, &full[st]);
+                    else
+                        tma_load_2d(sb, &tmA_hi, 64 * kb, y, &full[st]);
+                }
                 issued = u + 1;
             }
         }
@@ -709,12 +697,14 @@ __global__ void __launch_bounds__(kTokThreads, 1)
                 bool ok = true;
                 for (int kb = 0; kb < NKB; ++kb, ++u) {
                     const int st = u % STAGES;
-                    if (!mbar_wait(&full[st], (u / STAGES) & 1, &abort_flag, a.status, 104)) {
+                    if (!mbar_wait(kMode == kModeDQ ? &conv : &full[st],
+                                   kMode == kModeDQ ? (u & 1) : ((u / STAGES) & 1), &abort_flag, a.status,
+                                   104)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = ab + st * SBYTES;
+                    const uint32_t a0 = kMode == kModeDQ ? ab + STAGES * SBYTES : ab + st * SBYTES;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t ko = (uint32_t)(16 * k * 2);
@@ -733,11 +723,57 @@ __global__ void __launch_bounds__(kTokThreads, 1)
                             mma_bf16(d, ahi, bhi, id256, accum);  // A.hi | A.lo
                         }
                     }
-                    mma_commit(&empty[st]);
+                    mma_commit(kMode == kModeDQ ? &aempty : &empty[st]);
                 }
                 if (!ok) break;
                 mma_commit(&tfull[acc]);
             }
+        }
+    } else if (kMode == kModeDQ && warp >= 6) {
+        // Converters: dZ (fp32 boxes of 32 columns, 128-byte swizzle) -> the
+        // K block's bf16 hi and lo images (K-major, 128-byte swizzle). A unit
+        // is 8 columns of one token row; 16-byte chunk c of row r at c ^ (r & 7).
+        const int tc = threadIdx.x - 192;  // 0..127
+        uint8_t *abuf = sA + STAGES * SBYTES;
+        for (int t = 0, u = 0; t < ntile; ++t) {
+            bool ok = true;
+            for (int kb = 0; kb < NKB; ++kb, ++u) {
+                const int st = u % STAGES;
+                bool got = mbar_wait(&full[st], (u / STAGES) & 1, &abort_flag, a.status, 108);
+                // the images of the K block before are read by its product
+                got = got && (u == 0 || mbar_wait(&aempty, (u - 1) & 1, &abort_flag, a.status, 109));
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint8_t *sb = sA + st * SBYTES;
+                uint4 hi[8], lo[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int un = tc + 128 * k, row = un >> 3, c8 = un & 7, sw = row & 7;
+                    const uint8_t *zr = sb + (c8 >> 2) * (SBYTES / 2) + row * 128;
+                    const int c32 = (c8 & 3) * 2;  // the unit's first 16-byte chunk in its box row
+                    const float4 z0 = *reinterpret_cast<const float4 *>(zr + ((c32 ^ sw) << 4));
+                    const float4 z1 = *reinterpret_cast<const float4 *>(zr + (((c32 + 1) ^ sw) << 4));
+                    uint2 h0, l0, h1, l1;
+                    split4(z0.x, z0.y, z0.z, z0.w, h0, l0);
+                    split4(z1.x, z1.y, z1.z, z1.w, h1, l1);
+                    hi[k] = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                    lo[k] = make_uint4(l0.x, l0.y, l1.x, l1.y);
+                }
+                mbar_arrive(&empty[st]);  // the fp32 stage is read: the producer may refill it
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int un = tc + 128 * k, row = un >> 3, c8 = un & 7;
+                    const int off = row * 128 + ((c8 ^ (row & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(abuf + off) = hi[k];
+                    *reinterpret_cast<uint4 *>(abuf + kTokStage / 2 + off) = lo[k];
+                }
+                fence_async_smem();
+                mbar_arrive(&conv);
+            }
+            if (!ok) break;
         }
     } else if (warp >= 2) {
         const int tt = threadIdx.x - 64;  // 0..127
@@ -801,7 +837,7 @@ __global__ void __launch_bounds__(kTokThreads, 1)
         // ---- epilogue: lane = token row of the tile; every global row access
         // goes through the warp's staging rows (whole row segments)
         const int sp = warp & 3;
-        uint8_t *stg = sA + STAGES * SBYTES + (warp - 2) * kStgWarp;
+        uint8_t *stg = sA + STAGES * SBYTES + ABUF + (warp - 2) * kStgWarp;
         bool run = true;
         if (kMode == kModeRP) {
             // S: lane = row i, 128 fp32 columns from tensor memory
@@ -922,7 +958,7 @@ cudaError_t launch_tok_mode(const CUtensorMap &hi, const CUtensorMap &lo, const 
     cudaError_t e = cudaFuncSetAttribute(cb_tok_tc_kernel<kMode>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTokSmem);
     if (e != cudaSuccess) return e;
-    cb_tok_tc_kernel<kMode><<<nch, kTokThreads, kTokSmem, s>>>(hi, lo, a);
+    cb_tok_tc_kernel<kMode><<<nch, tok_threads(kMode), kTokSmem, s>>>(hi, lo, a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launch(s);
@@ -935,25 +971,20 @@ bool chunk_bwd_tok_tc_supported(int d, int chunk, bool bf16) {
     return bf16 && d == kD && chunk >= kTokTile && chunk % kTokTile == 0;
 }
 
-// Workspace bytes of the tensor-core token passes: dZ as bf16 hi and lo rows
-// (512 bytes per token).
-size_t chunk_bwd_tok_tc_scratch_bytes(size_t tokens) { return tokens * 2 * kD * 2; }
-
 // S of chunk g goes to S + g * s_stride floats (the caller's d x d slot per
-// chunk, free once the scans have run).
+// chunk, free once the scans have run). The token passes need no other
+// workspace: DQ splits dZ into its bf16 terms on chip.
 cudaError_t launch_chunk_bwd_tok_tc(const void *K, const void *V, const float *eta, const float *dZ,
                                     const float *W, const float *Om, float *S, size_t s_stride,
-                                    int B, int H, int T, int chunk, void *scratch, float *dQ,
-                                    float *dK, float *dV, float *deta, cudaStream_t s) {
+                                    int B, int H, int T, int chunk, float *dQ, float *dK, float *dV,
+                                    float *deta, cudaStream_t s) {
     const uint64_t rows = (uint64_t)B * H * T;
     const int nch = B * H * (T / chunk);
-    const TokScratch ts = tok_scratch(scratch, rows);
     int *status = device_status_word();
-    alignas(64) CUtensorMap tmK, tmV, tmZh, tmZl;
+    alignas(64) CUtensorMap tmK, tmV, tmZ;
     if (!encode_tmap_2d(&tmK, K, false, kD, rows, 64, kTokTile) ||
         !encode_tmap_2d(&tmV, V, false, kD, rows, 64, kTokTile) ||
-        !encode_tmap_2d(&tmZh, ts.z_hi, false, kD, rows, 64, kTokTile) ||
-        !encode_tmap_2d(&tmZl, ts.z_lo, false, kD, rows, 64, kTokTile))
+        !encode_tmap_2d(&tmZ, dZ, true, kD, rows, 32, kTokTile))
         return cudaErrorInvalidValue;
     TokArgs a{W, Om, static_cast<const __nv_bfloat16 *>(V), eta, dZ, dV, deta, S, s_stride,
               chunk, status};
@@ -962,7 +993,7 @@ cudaError_t launch_chunk_bwd_tok_tc(const void *K, const void *V, const float *e
     a.out = dK;
     if ((e = launch_tok_mode<kModeDK>(tmK, tmV, a, nch, s)) != cudaSuccess) return e;
     a.out = dQ;
-    return launch_tok_mode<kModeDQ>(tmZh, tmZl, a, nch, s);
+    return launch_tok_mode<kModeDQ>(tmZ, tmZ, a, nch, s);
 }
 
 }  // namespace ttt

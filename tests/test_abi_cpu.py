@@ -111,9 +111,8 @@ def test_backward_host_validation():
               workspace_bytes=1 << 34, stream=0)
     call = lambda **kw: ttt.ttt_chunk_bwd(**{**cb, **kw}, check=False)  # noqa: E731
     need = ttt.ttt_chunk_bwd_workspace_bytes(1, 2, 4096, 128, 2048)
-    # fp32 per chunk and sequence, then 512 bytes per token of bf16 operand
-    # rows (dZ hi and lo) for the tensor-core token passes (d = 128, chunk % 128 == 0)
-    assert need == 4 * (5 * 4 * 128 * 128 + 2 * 128 * 128) + 2 * 4096 * 512
+    # fp32 per chunk (A_c, B_c, Q_c^T dZ_c, W_c, Om_{c+1}) and per sequence (dW0)
+    assert need == 4 * (5 * 4 * 128 * 128 + 2 * 128 * 128)
     assert ttt.ttt_chunk_bwd_workspace_bytes(1, 2, 4096, 128, 32) == 4 * (5 * 256 * 128 * 128
                                                                          + 2 * 128 * 128)
     assert ttt.ttt_chunk_bwd_workspace_bytes(1, 2, 4096, 64, 2048) == 4 * (5 * 4 + 2) * 64 * 64
