@@ -37,10 +37,12 @@ extern "C" int ttt_linear_bwd_host_run(const void *Q, const void *K, const void 
                          H, T, d, b, ln != 0, w0_per_seq != 0};
     if (bf16) run_kernel<__nv_bfloat16>(k, (int)S, d);
     else run_kernel<float>(k, (int)S, d);
-    if (!w0_per_seq) run_blocks(H, [&] { ttt::sum_over_batch_kernel(k.dW0s, dW0, B, H, (int)dd); });
+    // the batch sums: a thread per element, grid (elements, H), as launched
+    if (!w0_per_seq)
+        run_grid(((int)dd + 255) / 256, H, [&] { ttt::sum_over_batch_kernel(k.dW0s, dW0, B, H, (int)dd); }, 256);
     if (ln) {
-        run_blocks(H, [&] { ttt::sum_over_batch_kernel(k.dgs, dgamma, B, H, d); });
-        run_blocks(H, [&] { ttt::sum_over_batch_kernel(k.dbs, dbeta, B, H, d); });
+        run_grid((d + 63) / 64, H, [&] { ttt::sum_over_batch_kernel(k.dgs, dgamma, B, H, d); }, 64);
+        run_grid((d + 63) / 64, H, [&] { ttt::sum_over_batch_kernel(k.dbs, dbeta, B, H, d); }, 64);
     }
     return 0;
 }
