@@ -931,8 +931,8 @@ def backward_arm(args, wl):
                      "frac": ach / peaks["hbm_gbs"], "traffic": None,
                      "kernel": "all backward kernels", "peak_source": peaks_src,
                      "algorithmic_per_launch": hb, "kernel_ms": kern_ms,
-                     "note": ("Gram and per-token products on the tensor cores; bytes are the "
-                              "inputs and gradients only (not the workspace round trips)"),
+                     "note": ("Gram, scans and per-token products on the tensor cores; bytes are "
+                              "the inputs and gradients only (not the per-chunk workspace)"),
                      "tflops_algorithmic": achieved}
     else:
         line_roof = None
