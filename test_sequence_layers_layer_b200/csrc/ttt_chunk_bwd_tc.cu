@@ -1,5 +1,11 @@
-// ttt_chunk_bwd_tc.cu -- the per-chunk Gram products of the large-chunk TTT
-// backward on the tensor cores (d = 128, bf16 Q/K/V, fp32 dZ):
+// ttt_chunk_bwd_tc.cu -- the large-chunk TTT backward on the tensor cores
+// (d = 128, bf16 Q/K/V, fp32 dZ), three kernels in launch order:
+//   cb_gram_tc_kernel   the per-chunk Gram products (below);
+//   cb_scan_tc_kernel   the forward scan of W_c and the reverse scan of
+//                       Om_{c+1} (further down);
+//   cb_tok_tc_kernel<>  the per-token gradients in three passes (RP, DK, DQ).
+//
+// The per-chunk Gram products:
 //   A_c = K_c^T diag(eta) K_c,   B_c = K_c^T diag(eta) V_c,   D_c = Q_c^T dZ_c
 // ("Test-Time Training Done Right", abstract: the chunk's gradient step; the
 // backward's recurrences use the same A_c, and D_c carries dZ into dL/dW_c),
