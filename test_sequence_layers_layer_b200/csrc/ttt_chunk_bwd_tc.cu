@@ -444,9 +444,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) cb_scan_tc_kernel(ScanArgs a)
     // before the shared memory and tensor memory are released.
     if (abort_flag) {
         if (warp == 0 && lane == 0 && issued > 0) {
-            const int st = (issued - 1) / 2;  // the last chunk whose copies were issued
-            mbar_drain(&aready[st & 1], (st >> 1) & 1);
-            if (issued % 2 == 0) mbar_drain(&eready[st & 1], (st >> 1) & 1);
+            // the copies of the last two chunks may both be in flight (one
+            // per buffer): wait for each (a phase already complete returns)
+            const int last = (issued - 1) / 2;  // the last chunk whose copies were issued
+            for (int st = last > 0 ? last - 1 : 0; st <= last; ++st) {
+                mbar_drain(&aready[st & 1], (st >> 1) & 1);
+                if (st < last || issued % 2 == 0) mbar_drain(&eready[st & 1], (st >> 1) & 1);
+            }
         }
         if (warp == 1 && lane == 0) {
             mma_commit(&drain);
