@@ -145,6 +145,56 @@ def test_chunk_single_chunk_closed_form():
         assert np.abs(g[k]).max() == 0.0
 
 
+def test_chunk_recurrences_and_s_form_reproduce_the_oracle():
+    """The readings the large-chunk backward kernels compute, against the
+    autograd oracle: W_c by the forward recurrence W - A_c W + B_c, Om_{c+1}
+    by the reverse one Om - A_c Om + Q_c^T dZ_c (dW0 = Om_0), and per chunk
+    dK = -diag(eta) (K S - V Om^T) with S = W Om^T + Om W^T, which equals
+    -diag(eta) (R Om^T + P W^T) with R = K W - V, P = K Om; dV = diag(eta) P,
+    deta = -P . R, dQ = dZ W^T. Each slice of columns of W or Om also evolves
+    alone (the scans split the columns over blocks)."""
+    B, H, T, d, C = 1, 2, 24, 5, 8
+    Q, K, V, eta, W0, _, _ = _inputs(21, B, H, T, d, eta_scale=0.2)
+    r = np.random.default_rng(22)
+    dZ = r.standard_normal(Q.shape)
+    dW = r.standard_normal((B, H, d, d))
+    g = ob.chunk_grads(Q, K, V, eta, W0, dZ, dW, chunk=C)
+    for h in range(H):
+        q, k, v, e, dz = Q[0, h], K[0, h], V[0, h], eta[0, h], dZ[0, h]
+        cs = [slice(c0, c0 + C) for c0 in range(0, T, C)]
+        A = [k[c].T @ (e[c, None] * k[c]) for c in cs]
+        Bc = [k[c].T @ (e[c, None] * v[c]) for c in cs]
+        Ws, W = [], W0[h].copy()
+        for i in range(len(cs)):
+            Ws.append(W)
+            W = W - A[i] @ W + Bc[i]
+        Oms, Om = [None] * len(cs), dW[0, h].copy()
+        for i in reversed(range(len(cs))):
+            Oms[i] = Om
+            Om = Om - A[i] @ Om + q[cs[i]].T @ dz[cs[i]]
+        tol = 1e-10 * max(1.0, np.abs(g["W0"]).max())
+        assert np.abs(Om - g["W0"][h]).max() <= tol
+        # the first two columns alone follow the same recurrence
+        Om2 = dW[0, h][:, :2].copy()
+        for i in reversed(range(len(cs))):
+            Om2 = Om2 - A[i] @ Om2 + (q[cs[i]].T @ dz[cs[i]])[:, :2]
+        assert np.abs(Om2 - Om[:, :2]).max() <= tol
+        for i, c in enumerate(cs):
+            Wc, Oc = Ws[i], Oms[i]
+            R, P = k[c] @ Wc - v[c], k[c] @ Oc
+            S = Wc @ Oc.T + Oc @ Wc.T
+            dk_s = -e[c, None] * (k[c] @ S - v[c] @ Oc.T)
+            dk_rp = -e[c, None] * (R @ Oc.T + P @ Wc.T)
+            np.testing.assert_allclose(dk_s, dk_rp, rtol=0, atol=1e-12 * np.abs(dk_rp).max())
+            np.testing.assert_allclose(dk_s, g["K"][0, h, c], rtol=0, atol=1e-10 * np.abs(g["K"]).max())
+            np.testing.assert_allclose(e[c, None] * P, g["V"][0, h, c], rtol=0,
+                                       atol=1e-10 * np.abs(g["V"]).max())
+            np.testing.assert_allclose(-(P * R).sum(1), g["eta"][0, h, c], rtol=0,
+                                       atol=1e-10 * np.abs(g["eta"]).max())
+            np.testing.assert_allclose(dz[c] @ Wc.T, g["Q"][0, h, c], rtol=0,
+                                       atol=1e-10 * np.abs(g["Q"]).max())
+
+
 # ------------------------------------------------------------ TTT-MLP form
 
 def _mlp_inputs(seed, B, H, T, d, dh, eta_scale=0.1):
