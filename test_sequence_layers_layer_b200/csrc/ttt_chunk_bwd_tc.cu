@@ -599,18 +599,18 @@ __global__ void __launch_bounds__(tok_threads(kMode), 1)
     constexpr uint32_t kBLoOff = kMode == kModeRP ? (uint32_t)NKB * BR * 128 : 0u;
     // A ring: one term of a 64-wide K block per stage (DK: the K blocks of K,
     // then of V); DQ: dZ's fp32 K block (two 32-column boxes) per stage, and
-    // one buffer for its bf16 hi and lo images, which the converter warps
-    // fill once the product before has read them.
-    constexpr int STAGES = kMode == kModeDK ? 4 : 3;
+    // two buffers for the bf16 hi and lo images, which the converter warps
+    // fill once the product two K blocks before has read them.
+    constexpr int STAGES = kMode == kModeDK ? 4 : kMode == kModeDQ ? 2 : 3;
     constexpr int SBYTES = kTwoA ? kTokStage : kTokStage / 2;
-    constexpr int ABUF = kTwoA ? kTokStage : 0;  // DQ's bf16 images, after the ring
+    constexpr int ABUF = kTwoA ? 2 * kTokStage : 0;  // DQ's bf16 images, after the ring
     constexpr int BBYTES = NKB * BR * 128 * (kMode == kModeRP ? 2 : 1);  // B images
     static_assert(BBYTES + STAGES * SBYTES + ABUF + 4 * kStgWarp + 1024 <= (int)kTokSmem, "smem plan");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sB = smem, *sA = smem + BBYTES;
-    __shared__ uint64_t full[4], empty[4], bready, tfull[2], tempty[2], sfull, sfree, conv, aempty, drain;
+    __shared__ uint64_t full[4], empty[4], bready, tfull[2], tempty[2], sfull, sfree, conv[2], aempty[2], drain;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -625,8 +625,10 @@ __global__ void __launch_bounds__(tok_threads(kMode), 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kMode == kModeDQ ? 128 : 1);  // DQ: the converters free a stage
         }
-        mbar_init(&conv, 128);
-        mbar_init(&aempty, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&conv[b], 128);
+            mbar_init(&aempty[b], 1);
+        }
         mbar_init(&bready, 128);
         mbar_init(&sfull, 1);
         mbar_init(&sfree, 128);
@@ -707,14 +709,15 @@ __global__ void __launch_bounds__(tok_threads(kMode), 1)
                 bool ok = true;
                 for (int kb = 0; kb < NKB; ++kb, ++u) {
                     const int st = u % STAGES;
-                    if (!mbar_wait(kMode == kModeDQ ? &conv : &full[st],
-                                   kMode == kModeDQ ? (u & 1) : ((u / STAGES) & 1), &abort_flag, a.status,
-                                   104)) {
+                    if (!mbar_wait(kMode == kModeDQ ? &conv[u & 1] : &full[st],
+                                   kMode == kModeDQ ? ((u >> 1) & 1) : ((u / STAGES) & 1), &abort_flag,
+                                   a.status, 104)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = kMode == kModeDQ ? ab + STAGES * SBYTES : ab + st * SBYTES;
+                    const uint32_t a0 =
+                        kMode == kModeDQ ? ab + STAGES * SBYTES + (u & 1) * kTokStage : ab + st * SBYTES;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t ko = (uint32_t)(16 * k * 2);
@@ -733,7 +736,7 @@ __global__ void __launch_bounds__(tok_threads(kMode), 1)
                             mma_bf16(d, ahi, bhi, id256, accum);  // A.hi | A.lo
                         }
                     }
-                    mma_commit(kMode == kModeDQ ? &aempty : &empty[st]);
+                    mma_commit(kMode == kModeDQ ? &aempty[u & 1] : &empty[st]);
                 }
                 if (!ok) break;
                 mma_commit(&tfull[acc]);
@@ -744,14 +747,13 @@ __global__ void __launch_bounds__(tok_threads(kMode), 1)
         // K block's bf16 hi and lo images (K-major, 128-byte swizzle). A unit
         // is 8 columns of one token row; 16-byte chunk c of row r at c ^ (r & 7).
         const int tc = threadIdx.x - 192;  // 0..127
-        uint8_t *abuf = sA + STAGES * SBYTES;
         for (int t = 0, u = 0; t < ntile; ++t) {
             bool ok = true;
             for (int kb = 0; kb < NKB; ++kb, ++u) {
                 const int st = u % STAGES;
                 bool got = mbar_wait(&full[st], (u / STAGES) & 1, &abort_flag, a.status, 108);
-                // the images of the K block before are read by its product
-                got = got && (u == 0 || mbar_wait(&aempty, (u - 1) & 1, &abort_flag, a.status, 109));
+                // image buffer u & 1: read by the product of K block u - 2
+                got = got && (u < 2 || mbar_wait(&aempty[u & 1], ((u >> 1) - 1) & 1, &abort_flag, a.status, 109));
                 if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
                     break;
@@ -773,6 +775,7 @@ __global__ void __launch_bounds__(tok_threads(kMode), 1)
                     lo[k] = make_uint4(l0.x, l0.y, l1.x, l1.y);
                 }
                 mbar_arrive(&empty[st]);  // the fp32 stage is read: the producer may refill it
+                uint8_t *abuf = sA + STAGES * SBYTES + (u & 1) * kTokStage;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int un = tc + 128 * k, row = un >> 3, c8 = un & 7;
@@ -781,7 +784,7 @@ __global__ void __launch_bounds__(tok_threads(kMode), 1)
                     *reinterpret_cast<uint4 *>(abuf + kTokStage / 2 + off) = lo[k];
                 }
                 fence_async_smem();
-                mbar_arrive(&conv);
+                mbar_arrive(&conv[u & 1]);
             }
             if (!ok) break;
         }
