@@ -331,6 +331,7 @@ __global__ void cb_sum_over_batch_kernel(const float *in, float *out, int B, int
     out[(size_t)h * n + e] = acc;
 }
 
+#ifndef TTT_HOST_RUN  // launch code (a host build of the kernels for tests leaves it out)
 template <typename TIn, int D>
 cudaError_t launch_typed(const void *Q, const void *K, const void *V, const float *eta,
                          const float *W0, const float *dZ, const float *dW_out, float *dQ,
@@ -391,6 +392,7 @@ cudaError_t launch_typed(const void *Q, const void *K, const void *V, const floa
     }
     return cudaSuccess;
 }
+#endif  // TTT_HOST_RUN
 
 }  // namespace
 
@@ -405,6 +407,7 @@ size_t chunk_bwd_workspace_bytes(int B, int H, int T, int d, int chunk) {
     return sizeof(float) * (5 * nch * dd + S * dd);
 }
 
+#ifndef TTT_HOST_RUN
 cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const float *eta,
                              const float *W0, const float *dZ, const float *dW_out, float *dQ,
                              float *dK, float *dV, float *deta, float *dW0, int B, int H, int T,
@@ -422,5 +425,7 @@ cudaError_t launch_chunk_bwd(const void *Q, const void *K, const void *V, const 
                    : launch_typed<float, 128>(Q, K, V, eta, W0, dZ, dW_out, dQ, dK, dV, deta,
                                               dW0, B, H, T, chunk, w0_per_seq, workspace, s);
 }
+
+#endif  // TTT_HOST_RUN
 
 }  // namespace ttt

@@ -57,27 +57,28 @@ inline float __shfl_xor_sync(unsigned, float v, int m) {
 }
 inline float rsqrtf(float x) { return 1.f / sqrtf(x); }
 
-// Runs fn() as every thread of an nx x ny grid of blocks of nt threads (a
-// multiple of 32, at most 256), one block at a time.
+// Runs fn() as every thread of an nx x ny x nz grid of blocks of nt threads
+// (a multiple of 32, at most 256), one block at a time.
 template <class Fn>
-static void run_grid(int nx, int ny, Fn fn, int nt = emu::kMaxThreads) {
+static void run_grid(int nx, int ny, Fn fn, int nt = emu::kMaxThreads, int nz = 1) {
     emu::nthreads = nt;
     blockDim = {(unsigned)nt, 1, 1};
-    gridDim = {(unsigned)nx, (unsigned)ny, 1};
+    gridDim = {(unsigned)nx, (unsigned)ny, (unsigned)nz};
     emu::block_bar = std::make_unique<std::barrier<>>(nt);
     for (auto &w : emu::warp_bar) w = std::make_unique<std::barrier<>>(32);
-    for (int by = 0; by < ny; ++by)
-        for (int bx = 0; bx < nx; ++bx) {
-            blockIdx = {(unsigned)bx, (unsigned)by, 0};
-            std::vector<std::thread> th;
-            for (int t = 0; t < nt; ++t)
-                th.emplace_back([&, t] {
-                    emu::tid = t;
-                    threadIdx = {(unsigned)t, 0, 0};
-                    fn();
-                });
-            for (auto &x : th) x.join();
-        }
+    for (int bz = 0; bz < nz; ++bz)
+        for (int by = 0; by < ny; ++by)
+            for (int bx = 0; bx < nx; ++bx) {
+                blockIdx = {(unsigned)bx, (unsigned)by, (unsigned)bz};
+                std::vector<std::thread> th;
+                for (int t = 0; t < nt; ++t)
+                    th.emplace_back([&, t] {
+                        emu::tid = t;
+                        threadIdx = {(unsigned)t, 0, 0};
+                        fn();
+                    });
+                for (auto &x : th) x.join();
+            }
 }
 
 // Runs fn() as every thread of nblocks blocks (a one-dimensional grid).
